@@ -1,0 +1,288 @@
+// TEST INFRASTRUCTURE ONLY: a plain, slow, single-threaded CPU reference of the
+// forward pass of one Mixture-of-Experts FFN layer. It exists to check the CUDA
+// path; only the tests, the smoke check and the benchmark's CPU-baseline leg may
+// load it. It shares no code, header or table with the CUDA library.
+//
+// What it computes is the plain definition of the layer, written out step by step
+// with every accumulation in double:
+//
+//   p(x) = softmax(W_r x)                                   router
+//   y    = sum_{e in TopK(p(x), k)} p_e(x) * E_e(x)          gate-weighted experts
+//
+//   (DeepSpeed MoE and Model Compression, section "DeepSpeed-MoE: capacity growth
+//    is not per-token compute growth", the MoE formula and the pipeline listing
+//    router -> topk -> pack_by_expert(capacity) -> local_experts -> combine)
+//
+// with a per-expert capacity: tokens beyond an expert's capacity skip that
+// expert's FFN and reach the output only through the residual
+//   (Switch-vs-DeepSpeed comparison article, section "Expert Capacity Overflow":
+//    capacity = tokens_per_batch / num_experts * capacity_factor).
+//
+// Readings of points the pages leave open (each is listed in the design notes):
+//   * capacity C = ceil(k * T * cf / E), evaluated in double in that order;
+//   * overflow is first-come: slots are handed out in token order (t ascending,
+//     then the token's j-th choice), slot >= C is dropped;
+//   * gates are the unrenormalised softmax probabilities p_e;
+//   * softmax over all E experts first, then top-k; top-k is taken on the fp32
+//     logits, ordered by (logit descending, expert index ascending);
+//   * an expert is a two-layer FFN with biases and the exact erf GeLU
+//     (MoE pruning/quantisation survey notes, section 1.1.2.1 "Replacing the FFN
+//     layer": M_i(x) is a two-layer feed-forward network);
+//   * for bf16 workloads the hidden activation h is rounded to bf16 (round to
+//     nearest even) because that is the storage type of the second GEMM's operand;
+//     the expert output y and the dense-branch output are rounded to fp32;
+//   * out = [x if add_input_residual] + [DenseMLP(x) if PR-MoE] + sum_j gate_j * y_j,
+//     summed in double and rounded once to the output type
+//     (DeepSpeed-MoE notes §3.1 PR-MoE: a fixed dense MLP plus a top-1 residual
+//      expert; comparison article, "numeric example: residual correction");
+//   * load-balance statistics f_i (share of tokens whose top-1 choice is i, before
+//     the capacity drop), Q_i (mean router probability of i over all tokens) and
+//     aux = alpha * E * sum_i f_i Q_i (survey notes §1.1.4.1, Switch Transformer loss).
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <vector>
+
+extern "C" {
+
+// ---------------------------------------------------------------- number formats
+
+// bf16 bit pattern -> exact double (bf16 is the top half of an fp32 word).
+double oracle_bf16_to_double(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  std::memcpy(&f, &u, 4);
+  return (double)f;
+}
+
+// Nearest bf16 value to v, ties to even (8 significant bits), returned as bit pattern.
+// Written from the definition: scale the significand to [128, 256), round to the
+// nearest integer with ties to even, scale back. Overflow goes to +-inf.
+uint16_t oracle_round_bf16(double v) {
+  if (std::isnan(v)) return 0x7fc0;
+  if (v == 0.0 || std::isinf(v)) {
+    float f = (float)v;
+    uint32_t u;
+    std::memcpy(&u, &f, 4);
+    return (uint16_t)(u >> 16);
+  }
+  int e;
+  double m = std::frexp(v, &e);          // v = m * 2^e, 0.5 <= |m| < 1
+  int q = e - 8;                           // quantum exponent for 8 significant bits
+  if (q < -133) q = -133;                  // bf16 subnormal spacing is 2^-133
+  double r = std::nearbyint(std::ldexp(v, -q));  // default rounding mode: ties to even
+  double rv = std::ldexp(r, q);
+  float f = (float)rv;                     // exact: rv has <= 8 significant bits
+  if (std::fabs(rv) > 3.3895313892515355e38) f = v > 0 ? INFINITY : -INFINITY;
+  uint32_t u;
+  std::memcpy(&u, &f, 4);
+  return (uint16_t)(u >> 16);
+}
+
+static inline double load(const void* p, int bf16, int64_t i) {
+  return bf16 ? oracle_bf16_to_double(((const uint16_t*)p)[i]) : (double)((const float*)p)[i];
+}
+
+// GeLU, exact erf form: 0.5 * z * (1 + erf(z / sqrt(2))) = z * Phi(z).
+double oracle_gelu(double z) { return 0.5 * z * (1.0 + std::erf(z / std::sqrt(2.0))); }
+
+// ---------------------------------------------------------------- router
+
+// Router logits l[t,e] = sum_i x[t,i] * W_r[e,i] (+ b_r[e]), accumulated in double in
+// index order, rounded to fp32. W_r is stored [E, d] (row e is expert e's vector), so
+// both W_r x (blog formula) and x W_r (comparison article, "Router computation") read
+// the same numbers. b_r is the optional per-expert logit bias of the skewed workloads.
+void oracle_router_logits(const void* x, int x_bf16, int64_t T, int d, const float* w_r,
+                          const float* b_r, int E, float* logits) {
+  for (int64_t t = 0; t < T; ++t)
+    for (int e = 0; e < E; ++e) {
+      double s = 0.0;
+      for (int i = 0; i < d; ++i) s += load(x, x_bf16, t * d + i) * (double)w_r[(int64_t)e * d + i];
+      if (b_r) s += (double)b_r[e];
+      logits[t * E + e] = (float)s;
+    }
+}
+
+// Softmax over the E fp32 logits of one token, in double.
+static void softmax_row(const float* l, int E, double* p) {
+  double m = -INFINITY;
+  for (int e = 0; e < E; ++e) m = l[e] > m ? (double)l[e] : m;
+  double z = 0.0;
+  for (int e = 0; e < E; ++e) z += std::exp((double)l[e] - m);
+  for (int e = 0; e < E; ++e) p[e] = std::exp((double)l[e] - m) / z;
+}
+
+// TopK(p(x), k) and the gates p_e (unrenormalised). Softmax is monotone, so the top-k
+// of p is the top-k of the fp32 logits; ties go to the lowest expert index.
+// probs (optional) receives the full [T, E] softmax in double.
+void oracle_route(const float* logits, int64_t T, int E, int k, int32_t* ids, float* gates,
+                  double* probs) {
+  std::vector<double> p(E);
+  std::vector<char> taken(E);
+  for (int64_t t = 0; t < T; ++t) {
+    const float* l = logits + t * E;
+    softmax_row(l, E, p.data());
+    if (probs)
+      for (int e = 0; e < E; ++e) probs[t * E + e] = p[e];
+    std::fill(taken.begin(), taken.end(), 0);
+    for (int j = 0; j < k; ++j) {
+      int best = -1;
+      for (int e = 0; e < E; ++e)
+        if (!taken[e] && (best < 0 || l[e] > l[best])) best = e;
+      taken[best] = 1;
+      ids[t * k + j] = best;
+      gates[t * k + j] = (float)p[best];
+    }
+  }
+}
+
+// Switch-style load-balance statistics: f_i = (1/T) #{t : top-1 choice of t is i},
+// Q_i = (1/T) sum_t p_{t,i}, aux = alpha * E * sum_i f_i * Q_i.
+void oracle_lb_stats(const float* logits, const int32_t* ids, int64_t T, int E, int k,
+                     double alpha, double* f, double* Q, double* aux) {
+  std::vector<double> p(E);
+  for (int e = 0; e < E; ++e) f[e] = Q[e] = 0.0;
+  for (int64_t t = 0; t < T; ++t) {
+    f[ids[t * k]] += 1.0;
+    softmax_row(logits + t * E, E, p.data());
+    for (int e = 0; e < E; ++e) Q[e] += p[e];
+  }
+  double s = 0.0;
+  for (int e = 0; e < E; ++e) {
+    f[e] /= (double)T;
+    Q[e] /= (double)T;
+    s += f[e] * Q[e];
+  }
+  *aux = alpha * (double)E * s;
+}
+
+// ---------------------------------------------------------------- capacity and slots
+
+// expert_capacity = tokens_per_batch / num_experts * capacity_factor, with the k
+// choices of each token counted and rounded up: C = ceil(k * T * cf / E).
+int64_t oracle_capacity(int64_t T, int E, int k, double capacity_factor) {
+  return (int64_t)std::ceil((double)k * (double)T * capacity_factor / (double)E);
+}
+
+// First-come slot assignment: walk the (token, choice) pairs in token order and give
+// each the next free position of its expert; a position >= C is an overflow (-1).
+// counts[e] receives the demand (before the capacity drop).
+void oracle_assign_slots(const int32_t* ids, int64_t T, int k, int E, int64_t C, int32_t* slot,
+                         int32_t* counts) {
+  std::vector<int64_t> cnt(E, 0);
+  for (int64_t t = 0; t < T; ++t)
+    for (int j = 0; j < k; ++j) {
+      const int e = ids[t * k + j];
+      const int64_t s = cnt[e]++;
+      slot[t * k + j] = s < C ? (int32_t)s : -1;
+    }
+  for (int e = 0; e < E; ++e) counts[e] = (int32_t)cnt[e];
+}
+
+// ---------------------------------------------------------------- expert FFN
+
+// One expert (or the dense MLP) on one token: z = W1 x + b1, h = GeLU(z) (rounded to
+// bf16 for bf16 weights), y = W2 h + b2, rounded to fp32. W1 is [d_ff, d], W2 is
+// [d, d_ff]; b1/b2 may be NULL.
+void oracle_ffn(const void* x_row, int bf16, int d, int d_ff, const void* w1, const void* b1,
+                const void* w2, const void* b2, float* y) {
+  std::vector<double> h(d_ff);
+  for (int j = 0; j < d_ff; ++j) {
+    double z = 0.0;
+    for (int i = 0; i < d; ++i) z += load(w1, bf16, (int64_t)j * d + i) * load(x_row, bf16, i);
+    if (b1) z += load(b1, bf16, j);
+    double g = oracle_gelu(z);
+    h[j] = bf16 ? oracle_bf16_to_double(oracle_round_bf16(g)) : g;
+  }
+  for (int o = 0; o < d; ++o) {
+    double s = 0.0;
+    for (int j = 0; j < d_ff; ++j) s += load(w2, bf16, (int64_t)o * d_ff + j) * h[j];
+    if (b2) s += load(b2, bf16, o);
+    y[o] = (float)s;
+  }
+}
+
+// ---------------------------------------------------------------- combine
+
+// out[t] = [residual[t]] + [dense[t]] + sum_{j : slot[t,j] >= 0} gate[t,j] * y[t,j], in
+// double. y holds one expert output per (token, choice) pair: [T, k, d] fp32. Dropped
+// pairs (slot < 0) contribute nothing, so an overflowed token keeps only its residual.
+void oracle_combine(int64_t T, int d, int k, const void* residual, int res_bf16,
+                    const float* dense, const float* gates, const int32_t* slot, const float* y,
+                    double* out) {
+  for (int64_t t = 0; t < T; ++t)
+    for (int i = 0; i < d; ++i) {
+      double s = 0.0;
+      if (residual) s += load(residual, res_bf16, t * d + i);
+      if (dense) s += (double)dense[t * d + i];
+      for (int j = 0; j < k; ++j)
+        if (slot[t * k + j] >= 0) s += (double)gates[t * k + j] * (double)y[(t * k + j) * (int64_t)d + i];
+      out[t * d + i] = s;
+    }
+}
+
+// ---------------------------------------------------------------- whole layer
+
+// The layer, step by step: logits -> route -> statistics -> capacity -> slots -> for each
+// requested token: residual + dense MLP + gate-weighted kept experts.
+//
+// logits_in: if non-NULL these fp32 logits are used instead of computing them (routing
+//            decided from the same logits as another implementation).
+// tokens:    the tokens whose output rows are computed (NULL = all T, in order);
+//            routing, slots and statistics always cover all T tokens.
+// out_exact: [n, d] double before the final rounding; out_rounded: [n, d] in the output
+//            type (bf16 bits if out_bf16, else fp32). Either may be NULL.
+// Returns the capacity C.
+int64_t oracle_layer_forward(int64_t T, int d, int d_ff, int E, int k, double capacity_factor,
+                             int bf16, int add_input_residual, const void* x, const float* w_r,
+                             const float* b_r, const void* w1, const void* b1, const void* w2,
+                             const void* b2, const void* dense_w1, const void* dense_b1,
+                             const void* dense_w2, const void* dense_b2, double aux_alpha,
+                             const float* logits_in, const int64_t* tokens, int64_t n_tokens,
+                             float* logits_out, int32_t* ids, float* gates, int32_t* slot,
+                             int32_t* counts, double* lb_stats, double* out_exact,
+                             void* out_rounded, int out_bf16) {
+  std::vector<float> logits_own;
+  const float* logits = logits_in;
+  if (!logits) {
+    logits_own.resize((size_t)T * E);
+    oracle_router_logits(x, bf16, T, d, w_r, b_r, E, logits_own.data());
+    logits = logits_own.data();
+  }
+  if (logits_out && logits_out != logits) std::memcpy(logits_out, logits, sizeof(float) * T * E);
+  oracle_route(logits, T, E, k, ids, gates, nullptr);
+  if (lb_stats) oracle_lb_stats(logits, ids, T, E, k, aux_alpha, lb_stats, lb_stats + E, lb_stats + 2 * E);
+  const int64_t C = oracle_capacity(T, E, k, capacity_factor);
+  oracle_assign_slots(ids, T, k, E, C, slot, counts);
+
+  const int64_t n = tokens ? n_tokens : T;
+  const size_t esz = bf16 ? 2 : 4;
+  std::vector<float> y((size_t)k * d), dense((size_t)d);
+  std::vector<double> row(d);
+  for (int64_t r = 0; r < n; ++r) {
+    const int64_t t = tokens ? tokens[r] : r;
+    const char* xt = (const char*)x + (size_t)t * d * esz;
+    for (int j = 0; j < k; ++j) {
+      if (slot[t * k + j] < 0) continue;
+      const int64_t e = ids[t * k + j];
+      oracle_ffn(xt, bf16, d, d_ff, (const char*)w1 + (size_t)e * d_ff * d * esz,
+                 b1 ? (const char*)b1 + (size_t)e * d_ff * esz : nullptr,
+                 (const char*)w2 + (size_t)e * d * d_ff * esz,
+                 b2 ? (const char*)b2 + (size_t)e * d * esz : nullptr, y.data() + (size_t)j * d);
+    }
+    const bool has_dense = dense_w1 != nullptr;
+    if (has_dense) oracle_ffn(xt, bf16, d, d_ff, dense_w1, dense_b1, dense_w2, dense_b2, dense.data());
+    oracle_combine(1, d, k, add_input_residual ? xt : nullptr, bf16, has_dense ? dense.data() : nullptr,
+                   gates + t * k, slot + t * k, y.data(), row.data());
+    for (int i = 0; i < d; ++i) {
+      if (out_exact) out_exact[r * d + i] = row[i];
+      if (out_rounded) {
+        if (out_bf16) ((uint16_t*)out_rounded)[r * d + i] = oracle_round_bf16(row[i]);
+        else ((float*)out_rounded)[r * d + i] = (float)row[i];
+      }
+    }
+  }
+  return C;
+}
+
+}  // extern "C"
