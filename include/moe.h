@@ -1,0 +1,217 @@
+/*
+ * moe.h — C ABI of the single-GPU Mixture-of-Experts FFN layer forward pass (sm_100a).
+ *
+ * The layer (DeepSpeed MoE and Model Compression, section "DeepSpeed-MoE：容量增长不等于
+ * 每 token 计算增长", the MoE formula and the pipeline listing):
+ *
+ *     p(x) = softmax(W_r x)                     y = sum_{e in TopK(p(x), k)} p_e(x) E_e(x)
+ *     scores = router(hidden); expert_ids, gates = topk(scores, k);
+ *     dispatch = pack_by_expert(hidden, expert_ids, capacity); out = local_experts(dispatch);
+ *     output = combine(out, gates)
+ *
+ * Entry points, in pipeline order:
+ *     moe_router_topk   router logits, softmax, top-k, load-balance statistics
+ *     moe_dispatch      capacity-limited first-come slots and the expert-major packed copy
+ *     moe_expert_ffn    per-expert two-layer GeLU FFN on the packed rows (grouped GEMMs)
+ *     moe_combine       gate-weighted sum of the kept expert rows plus the residual terms
+ *     moe_layer_forward all of the above (plus the optional PR-MoE dense MLP branch)
+ *
+ * Conventions (every entry point):
+ *   - Tensor pointers are caller-owned DEVICE memory, row-major, 16-byte aligned. The
+ *     library never allocates or frees memory and never synchronises the device, except
+ *     moe_get_device_error / moe_workspace_reset, which say so.
+ *   - All work is enqueued asynchronously on `stream` (NULL = the legacy default stream).
+ *   - Arguments are validated on the host before anything is enqueued; on failure the
+ *     entry returns a status other than MOE_OK and enqueues nothing.
+ *   - `ws` is caller-owned device scratch of at least the size the matching
+ *     *_workspace_bytes query returns. Its first 256 bytes are the STATUS BLOCK: an int
+ *     that kernels set (first error wins) when they detect bad device-side data or give
+ *     up a bounded wait. Zero it once after allocation with moe_workspace_reset (or any
+ *     memset) and read it with moe_get_device_error. Entry points never clear it.
+ *   - Calls that share a workspace must not overlap on the GPU (same stream is enough).
+ *   - bf16 tensors are stored as 16-bit words (the top half of an IEEE fp32 word).
+ *   - Environment variable MOE_FAULT_INJECT=<entry point name> makes that entry point
+ *     return MOE_ERR_CUDA without enqueueing anything (host-side fault injection for
+ *     callers' error paths).
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_ABI_VERSION 1
+#define MOE_STATUS_BLOCK_BYTES 256
+#define MOE_MAX_EXPERTS 1024
+#define MOE_MAX_TOPK 8
+
+struct CUstream_st;
+typedef struct CUstream_st* moe_stream_t; /* the same handle as cudaStream_t */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARGUMENT = 1,    /* NULL pointer, negative size, k > E, ... */
+  MOE_ERR_UNSUPPORTED = 2,         /* valid but outside what this build implements */
+  MOE_ERR_WORKSPACE_TOO_SMALL = 3, /* ws_bytes below the *_workspace_bytes answer */
+  MOE_ERR_CUDA = 4,                /* a CUDA runtime call failed (or fault injection) */
+  MOE_ERR_DEVICE_FLAG = 5,         /* moe_get_device_error found a device-side error */
+  MOE_ERR_MISALIGNED = 6           /* a tensor pointer is not 16-byte aligned */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+/* Device-side error codes written to the status block (first error wins). */
+typedef enum {
+  MOE_DEVERR_NONE = 0,
+  MOE_DEVERR_TIMEOUT = 1,      /* a bounded wait inside a kernel gave up (about 2 s) */
+  MOE_DEVERR_BAD_EXPERT = 2,   /* an expert id outside [0, E) reached dispatch */
+  MOE_DEVERR_BAD_OFFSETS = 3,  /* expert_offsets not non-decreasing or beyond rows_max */
+  MOE_DEVERR_BAD_ROW = 4       /* combine met a (slot, offset) outside the packed rows */
+} moe_device_error;
+
+const char* moe_status_string(moe_status s);
+int moe_abi_version(void);
+
+/* ---------------------------------------------------------------- sizes
+ * Expert capacity (Switch/DeepSpeed comparison article, section "Expert Capacity Overflow":
+ * expert_capacity = tokens_per_batch / num_experts * capacity_factor), with the k choices of
+ * each token counted and rounded up: C = ceil(k * T * capacity_factor / E), evaluated in double
+ * in that order. capacity_factor must be finite and >= 0. */
+moe_status moe_capacity(int64_t T, int E, int k, double capacity_factor, int64_t* C_out);
+
+/* Rows of the expert-major packed buffers: min(T * k, E * C). Kept rows of expert e occupy
+ * [expert_offsets[e], expert_offsets[e+1]) with no padding between experts. */
+moe_status moe_packed_rows_max(int64_t T, int E, int k, int64_t C, int64_t* rows_out);
+
+/* ---------------------------------------------------------------- router
+ * logits[t,e] = sum_i x[t,i] * w_router[e,i] (+ router_bias[e])   (fp32 arithmetic)
+ * p[t,:]      = softmax(logits[t,:]) over all E experts
+ * expert_ids[t,0..k-1] = the k largest logits, descending; ties go to the lower index
+ * gates[t,j]  = p[t, expert_ids[t,j]]  (not renormalised over the k choices)
+ * lb_stats    = [f_0..f_{E-1}, Q_0..Q_{E-1}, aux]: f_i = share of tokens whose first choice is i,
+ *               Q_i = mean over tokens of p[t,i], aux = aux_alpha * E * sum_i f_i * Q_i
+ *               (MoE survey notes §1.1.4.1, Switch Transformer load-balance loss).
+ * Cites: DeepSpeed MoE blog, MoE formula; comparison article, "Router computation" and
+ * "Top-1 routing decision".
+ *
+ * x:          [T, d_model] in x_dtype.           w_router: [E, d_model] fp32 (row e = expert e).
+ * router_bias:[E] fp32 or NULL.                   logits:   [T, E] fp32 output, or NULL.
+ * expert_ids: [T, k] int32 output.                gates:    [T, k] fp32 output.
+ * lb_stats:   [2E+1] fp32 output, or NULL.
+ * Limits: 1 <= E <= 1024, 1 <= k <= min(E, 8), T >= 0 (T == 0 enqueues nothing), d_model >= 1;
+ * bf16 x needs d_model % 8 == 0. */
+moe_status moe_router_workspace_bytes(int64_t T, int E, size_t* bytes);
+moe_status moe_router_topk(const void* x, moe_dtype x_dtype, int64_t T, int d_model,
+                           const float* w_router, const float* router_bias, int E, int k,
+                           float* logits, int32_t* expert_ids, float* gates, float* lb_stats,
+                           float aux_alpha, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* ---------------------------------------------------------------- dispatch
+ * pack_by_expert with a capacity (DeepSpeed MoE blog, pipeline listing; DeepSpeed-MoE notes
+ * §4.4: top-k + prefix-sum + scatter into a dense token-to-expert mapping table, then an
+ * explicit re-order of rows by that table instead of a sparse einsum).
+ * Pairs (t, j) are taken in token order (t ascending, then j); each gets the next position of
+ * its expert: slot[t,j] = position if position < C, else -1 (overflow: the pair contributes
+ * nothing and the token keeps only its residual).
+ * expert_counts[e]   = demand of expert e (before the drop).
+ * expert_offsets[e]  = sum_{e' < e} min(expert_counts[e'], C); expert_offsets[E] = kept rows.
+ * row_token[r]       = token of packed row r for r < expert_offsets[E] (rows beyond: unspecified).
+ * x_packed[offsets[e] + slot[t,j], :] = x[t, :] for every kept pair.
+ * x, x_packed: [T, d_model] / [rows_max, d_model] in dtype; rows_max from moe_packed_rows_max.
+ * Expert ids outside [0, E) set MOE_DEVERR_BAD_EXPERT and are treated as dropped. */
+moe_status moe_dispatch_workspace_bytes(int64_t T, int E, int k, size_t* bytes);
+moe_status moe_dispatch(const void* x, moe_dtype dtype, int64_t T, int d_model,
+                        const int32_t* expert_ids, int E, int k, int64_t C, int32_t* slot,
+                        int32_t* expert_counts, int32_t* expert_offsets, int32_t* row_token,
+                        void* x_packed, int64_t rows_max, void* ws, size_t ws_bytes,
+                        moe_stream_t stream);
+
+/* ---------------------------------------------------------------- expert FFN
+ * For every expert e and every packed row r in [expert_offsets[e], expert_offsets[e+1]):
+ *     h[r,:] = GeLU(W1[e] x_packed[r,:] + b1[e])        GeLU(z) = 0.5 z (1 + erf(z / sqrt 2))
+ *     y[r,:] = W2[e] h[r,:] + b2[e]
+ * (an expert is a two-layer feed-forward network: MoE survey notes §1.1.2.1; DeepSpeed-MoE notes
+ * §4.4/§5, "Sparse GEMM -> Dense GEMM": dense per-expert GEMMs on the packed rows).
+ * w1: [E, d_ff, d_model], b1: [E, d_ff] or NULL, w2: [E, d_model, d_ff], b2: [E, d_model] or NULL,
+ * all in dtype. h_packed: [rows_max, d_ff] in dtype (intermediate, bf16 rounds h);
+ * y_packed: [rows_max, d_model] fp32. Rows outside every segment are not written.
+ * With E = 1 and expert_offsets = {0, T} this is a dense MLP (the PR-MoE fixed MLP).
+ * capacity_hint: an upper bound on the rows of any one expert (normally C); it only selects the
+ * token tile width and never affects results. bf16 needs d_model % 8 == 0 and d_ff % 8 == 0.
+ * bf16 runs on tcgen05 tensor cores (fp32 accumulate); fp32 runs on fp32 FMA (no TF32). */
+moe_status moe_expert_ffn_workspace_bytes(size_t* bytes);
+moe_status moe_expert_ffn(const void* x_packed, const int32_t* expert_offsets, int E,
+                          int64_t rows_max, int d_model, int d_ff, moe_dtype dtype, const void* w1,
+                          const void* b1, const void* w2, const void* b2, void* h_packed,
+                          float* y_packed, int64_t capacity_hint, void* ws, size_t ws_bytes,
+                          moe_stream_t stream);
+
+/* ---------------------------------------------------------------- combine
+ * out[t,:] = [residual[t,:]] + [dense[t,:]] + sum_{j : slot[t,j] >= 0} gates[t,j] *
+ *            y_packed[expert_offsets[expert_ids[t,j]] + slot[t,j], :]
+ * summed in fp32 in that order and rounded once to out_dtype (DeepSpeed MoE blog, combine(out,
+ * gates); comparison article, "Expert Capacity Overflow": a dropped token passes through the
+ * residual only; PR-MoE "residual correction" example: fixed MLP output + gate * expert).
+ * residual: [T, d_model] in res_dtype or NULL. dense: [T, d_model] fp32 or NULL.
+ * A (slot, offset) pointing outside [0, rows_max) sets MOE_DEVERR_BAD_ROW and is skipped. */
+moe_status moe_combine_workspace_bytes(size_t* bytes);
+moe_status moe_combine(const float* y_packed, const int32_t* expert_offsets,
+                       const int32_t* expert_ids, const int32_t* slot, const float* gates,
+                       int64_t T, int d_model, int E, int k, int64_t rows_max,
+                       const void* residual, moe_dtype res_dtype, const float* dense, void* out,
+                       moe_dtype out_dtype, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* ---------------------------------------------------------------- whole layer */
+typedef struct {
+  int64_t T;
+  int d_model, d_ff, E, k;
+  double capacity_factor;
+  moe_dtype dtype;      /* x, expert weights and biases, dense-branch weights */
+  moe_dtype out_dtype;  /* output */
+  const void* x;                         /* [T, d_model] */
+  const float* w_router;                 /* [E, d_model] fp32 */
+  const float* router_bias;              /* [E] fp32 or NULL */
+  const void *w1, *b1, *w2, *b2;         /* experts; biases may be NULL */
+  /* PR-MoE fixed dense MLP (DeepSpeed-MoE notes §3.1): all four NULL = no dense branch.
+   * dense_w1 [d_ff, d_model], dense_b1 [d_ff], dense_w2 [d_model, d_ff], dense_b2 [d_model]. */
+  const void *dense_w1, *dense_b1, *dense_w2, *dense_b2;
+  int add_input_residual; /* 1: out += x */
+  float aux_alpha;        /* alpha of the load-balance loss */
+} moe_layer_args;
+
+/* Optional device outputs of the intermediate results; any field may be NULL. */
+typedef struct {
+  float* logits;          /* [T, E] */
+  int32_t* expert_ids;    /* [T, k] */
+  float* gates;           /* [T, k] */
+  int32_t* slot;          /* [T, k] */
+  int32_t* expert_counts; /* [E] demand */
+  int32_t* expert_offsets;/* [E+1] */
+  float* lb_stats;        /* [2E+1] */
+} moe_layer_aux;
+
+/* out = [x if add_input_residual] + [DenseMLP(x) if dense_*] + sum_j gate_j * Expert_{e_j}(x)
+ * over the kept choices. Enqueues: router, dispatch, [dense MLP], expert FFN, combine. */
+moe_status moe_layer_workspace_bytes(const moe_layer_args* args, size_t* bytes);
+moe_status moe_layer_forward(const moe_layer_args* args, void* out, moe_layer_aux* aux, void* ws,
+                             size_t ws_bytes, moe_stream_t stream);
+
+/* ---------------------------------------------------------------- status block
+ * moe_workspace_reset: zeroes the status block (asynchronous on stream).
+ * moe_get_device_error: synchronises `stream`, copies the status word to *code_out and returns
+ * MOE_ERR_DEVICE_FLAG if it is non-zero, MOE_OK otherwise. */
+moe_status moe_workspace_reset(void* ws, size_t ws_bytes, moe_stream_t stream);
+moe_status moe_get_device_error(const void* ws, int* code_out, moe_stream_t stream);
+
+/* Number of kernel launches the last successful call of each entry point enqueued on this host
+ * thread (for launch accounting in benchmarks). */
+int moe_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H_ */

@@ -1,0 +1,438 @@
+// C ABI of the MoE-layer forward pass: argument validation, workspace layout, fault injection
+// and launch accounting around the kernels' enqueue functions. See include/moe.h.
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+
+#include "kernels.h"
+
+namespace moe {
+
+namespace {
+thread_local int g_launches = 0;
+}
+
+void count_launch() { ++g_launches; }
+
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < 64 && cache[dev]) return cache[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    n = 148;
+  if (dev >= 0 && dev < 64) cache[dev] = n;
+  return n;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+bool fault_injected(const char* entry) {
+  const char* v = std::getenv("MOE_FAULT_INJECT");
+  return v != nullptr && std::strcmp(v, entry) == 0;
+}
+
+size_t esize(moe_dtype dt) { return dt == MOE_BF16 ? 2 : 4; }
+
+bool valid_dtype(moe_dtype dt) { return dt == MOE_F32 || dt == MOE_BF16; }
+
+// Bump allocator over the caller's workspace; the first kAlign bytes are the status block.
+struct Carve {
+  uint8_t* base;
+  size_t off = kAlign;
+  template <class T>
+  T* take(size_t count) {
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += align_up(count * sizeof(T));
+    return p;
+  }
+};
+
+// ------------------------------------------------------------ workspace layouts
+
+struct RouterWs {
+  float* q_partial;
+  float* logits;
+};
+RouterWs carve_router(Carve& c, int64_t T, int E) {
+  RouterWs w;
+  w.q_partial = c.take<float>((size_t)router_num_blocks(T) * E);
+  w.logits = c.take<float>((size_t)T * E);
+  return w;
+}
+
+struct DispatchWs {
+  int32_t *local_rank, *seg_counts, *seg_base;
+};
+DispatchWs carve_dispatch(Carve& c, int64_t T, int E, int k) {
+  const int64_t nseg = dispatch_num_segments(T * k);
+  DispatchWs w;
+  w.local_rank = c.take<int32_t>((size_t)T * k);
+  w.seg_counts = c.take<int32_t>((size_t)nseg * E);
+  w.seg_base = c.take<int32_t>((size_t)nseg * E);
+  return w;
+}
+
+moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// ------------------------------------------------------------ shared validation
+
+moe_status check_router_shape(int64_t T, int d, int E, int k) {
+  if (T < 0 || d < 1 || E < 1 || k < 1) return MOE_ERR_INVALID_ARGUMENT;
+  if (k > E) return MOE_ERR_INVALID_ARGUMENT;
+  if (E > MOE_MAX_EXPERTS || k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
+  if (T * (int64_t)k >= (int64_t)INT32_MAX || T * (int64_t)E >= ((int64_t)1 << 40))
+    return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status check_ffn_shape(int E, int64_t rows_max, int d, int d_ff, moe_dtype dt) {
+  if (E < 1 || rows_max < 0 || d < 1 || d_ff < 1 || !valid_dtype(dt)) return MOE_ERR_INVALID_ARGUMENT;
+  if (E > MOE_MAX_EXPERTS || rows_max >= (int64_t)INT32_MAX) return MOE_ERR_UNSUPPORTED;
+  if ((int64_t)E * d >= (int64_t)INT32_MAX || (int64_t)E * d_ff >= (int64_t)INT32_MAX)
+    return MOE_ERR_UNSUPPORTED;
+  if (dt == MOE_BF16 && (d % 8 != 0 || d_ff % 8 != 0)) return MOE_ERR_UNSUPPORTED;
+  if (dt == MOE_F32 && (d > kFfnF32MaxDim || d_ff > kFfnF32MaxDim)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARGUMENT: return "MOE_ERR_INVALID_ARGUMENT";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_WORKSPACE_TOO_SMALL: return "MOE_ERR_WORKSPACE_TOO_SMALL";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_DEVICE_FLAG: return "MOE_ERR_DEVICE_FLAG";
+    case MOE_ERR_MISALIGNED: return "MOE_ERR_MISALIGNED";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+int moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+int moe_last_launch_count(void) { return g_launches; }
+
+moe_status moe_capacity(int64_t T, int E, int k, double capacity_factor, int64_t* C_out) {
+  if (!C_out || T < 0 || E < 1 || k < 1 || !std::isfinite(capacity_factor) || capacity_factor < 0)
+    return MOE_ERR_INVALID_ARGUMENT;
+  const double c = std::ceil((double)k * (double)T * capacity_factor / (double)E);
+  if (c > 9.0e18) return MOE_ERR_UNSUPPORTED;
+  *C_out = (int64_t)c;
+  return MOE_OK;
+}
+
+moe_status moe_packed_rows_max(int64_t T, int E, int k, int64_t C, int64_t* rows_out) {
+  if (!rows_out || T < 0 || E < 1 || k < 1 || C < 0) return MOE_ERR_INVALID_ARGUMENT;
+  const int64_t a = T * k;
+  // min(T k, E C); when C >= T k the minimum is T k (E >= 1), which also avoids overflow
+  *rows_out = C >= a ? a : ((int64_t)E * C < a ? (int64_t)E * C : a);
+  return MOE_OK;
+}
+
+// ---------------------------------------------------------------- router
+
+moe_status moe_router_workspace_bytes(int64_t T, int E, size_t* bytes) {
+  if (!bytes || T < 0 || E < 1) return MOE_ERR_INVALID_ARGUMENT;
+  Carve c{nullptr};
+  carve_router(c, T, E);
+  *bytes = c.off;
+  return MOE_OK;
+}
+
+moe_status moe_router_topk(const void* x, moe_dtype x_dtype, int64_t T, int d_model,
+                           const float* w_router, const float* router_bias, int E, int k,
+                           float* logits, int32_t* expert_ids, float* gates, float* lb_stats,
+                           float aux_alpha, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (!valid_dtype(x_dtype)) return MOE_ERR_INVALID_ARGUMENT;
+  moe_status st = check_router_shape(T, d_model, E, k);
+  if (st != MOE_OK) return st;
+  if (T > 0 && (!x || !w_router || !expert_ids || !gates)) return MOE_ERR_INVALID_ARGUMENT;
+  if (!ws) return MOE_ERR_INVALID_ARGUMENT;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(router_bias) || !aligned16(logits) ||
+      !aligned16(expert_ids) || !aligned16(gates) || !aligned16(lb_stats) ||
+      ((uintptr_t)ws % kAlign) != 0)
+    return MOE_ERR_MISALIGNED;
+  size_t need = 0;
+  moe_router_workspace_bytes(T, E, &need);
+  if (ws_bytes < need) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (fault_injected("moe_router_topk")) return MOE_ERR_CUDA;
+  g_launches = 0;
+  if (T == 0) return MOE_OK;
+  Carve c{(uint8_t*)ws};
+  RouterWs w = carve_router(c, T, E);
+  return cuda_status(enqueue_router(x, x_dtype == MOE_BF16, T, d_model, w_router, router_bias, E,
+                                    k, logits ? logits : w.logits, expert_ids, gates, lb_stats,
+                                    aux_alpha, w.q_partial, stream));
+}
+
+// ---------------------------------------------------------------- dispatch
+
+moe_status moe_dispatch_workspace_bytes(int64_t T, int E, int k, size_t* bytes) {
+  if (!bytes || T < 0 || E < 1 || k < 1) return MOE_ERR_INVALID_ARGUMENT;
+  Carve c{nullptr};
+  carve_dispatch(c, T, E, k);
+  *bytes = c.off;
+  return MOE_OK;
+}
+
+moe_status moe_dispatch(const void* x, moe_dtype dtype, int64_t T, int d_model,
+                        const int32_t* expert_ids, int E, int k, int64_t C, int32_t* slot,
+                        int32_t* expert_counts, int32_t* expert_offsets, int32_t* row_token,
+                        void* x_packed, int64_t rows_max, void* ws, size_t ws_bytes,
+                        moe_stream_t stream) {
+  if (!valid_dtype(dtype) || C < 0) return MOE_ERR_INVALID_ARGUMENT;
+  moe_status st = check_router_shape(T, d_model, E, k);
+  if (st != MOE_OK) return st;
+  int64_t need_rows = 0;
+  moe_packed_rows_max(T, E, k, C, &need_rows);
+  if (rows_max < need_rows) return MOE_ERR_INVALID_ARGUMENT;
+  if (rows_max >= (int64_t)INT32_MAX) return MOE_ERR_UNSUPPORTED;
+  if (dtype == MOE_BF16 && d_model % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  if (!expert_counts || !expert_offsets || !ws) return MOE_ERR_INVALID_ARGUMENT;
+  if (T > 0 && (!x || !expert_ids || !slot)) return MOE_ERR_INVALID_ARGUMENT;
+  if (rows_max > 0 && (!row_token || !x_packed)) return MOE_ERR_INVALID_ARGUMENT;
+  if (!aligned16(x) || !aligned16(expert_ids) || !aligned16(slot) || !aligned16(expert_counts) ||
+      !aligned16(expert_offsets) || !aligned16(row_token) || !aligned16(x_packed) ||
+      ((uintptr_t)ws % kAlign) != 0)
+    return MOE_ERR_MISALIGNED;
+  size_t need = 0;
+  moe_dispatch_workspace_bytes(T, E, k, &need);
+  if (ws_bytes < need) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (fault_injected("moe_dispatch")) return MOE_ERR_CUDA;
+  g_launches = 0;
+  Carve c{(uint8_t*)ws};
+  DispatchWs w = carve_dispatch(c, T, E, k);
+  return cuda_status(enqueue_dispatch(x, dtype == MOE_BF16, T, d_model, expert_ids, E, k, C, slot,
+                                      expert_counts, expert_offsets, row_token, x_packed, rows_max,
+                                      w.local_rank, w.seg_counts, w.seg_base, (int*)ws, stream));
+}
+
+// ---------------------------------------------------------------- expert FFN
+
+moe_status moe_expert_ffn_workspace_bytes(size_t* bytes) {
+  if (!bytes) return MOE_ERR_INVALID_ARGUMENT;
+  *bytes = kAlign;
+  return MOE_OK;
+}
+
+moe_status moe_expert_ffn(const void* x_packed, const int32_t* expert_offsets, int E,
+                          int64_t rows_max, int d_model, int d_ff, moe_dtype dtype, const void* w1,
+                          const void* b1, const void* w2, const void* b2, void* h_packed,
+                          float* y_packed, int64_t capacity_hint, void* ws, size_t ws_bytes,
+                          moe_stream_t stream) {
+  moe_status st = check_ffn_shape(E, rows_max, d_model, d_ff, dtype);
+  if (st != MOE_OK) return st;
+  if (capacity_hint < 0 || !expert_offsets || !w1 || !w2 || !ws) return MOE_ERR_INVALID_ARGUMENT;
+  if (rows_max > 0 && (!x_packed || !h_packed || !y_packed)) return MOE_ERR_INVALID_ARGUMENT;
+  if (!aligned16(x_packed) || !aligned16(expert_offsets) || !aligned16(w1) || !aligned16(b1) ||
+      !aligned16(w2) || !aligned16(b2) || !aligned16(h_packed) || !aligned16(y_packed) ||
+      ((uintptr_t)ws % kAlign) != 0)
+    return MOE_ERR_MISALIGNED;
+  if (ws_bytes < kAlign) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (fault_injected("moe_expert_ffn")) return MOE_ERR_CUDA;
+  g_launches = 0;
+  if (rows_max == 0) return MOE_OK;
+  if (dtype == MOE_BF16)
+    return cuda_status(enqueue_expert_ffn_bf16(x_packed, expert_offsets, E, rows_max, d_model, d_ff,
+                                               w1, b1, w2, b2, h_packed, y_packed, capacity_hint,
+                                               (int*)ws, stream));
+  return cuda_status(enqueue_expert_ffn_f32((const float*)x_packed, expert_offsets, E, rows_max,
+                                            d_model, d_ff, (const float*)w1, (const float*)b1,
+                                            (const float*)w2, (const float*)b2, (float*)h_packed,
+                                            y_packed, (int*)ws, stream));
+}
+
+// ---------------------------------------------------------------- combine
+
+moe_status moe_combine_workspace_bytes(size_t* bytes) {
+  if (!bytes) return MOE_ERR_INVALID_ARGUMENT;
+  *bytes = kAlign;
+  return MOE_OK;
+}
+
+moe_status moe_combine(const float* y_packed, const int32_t* expert_offsets,
+                       const int32_t* expert_ids, const int32_t* slot, const float* gates,
+                       int64_t T, int d_model, int E, int k, int64_t rows_max,
+                       const void* residual, moe_dtype res_dtype, const float* dense, void* out,
+                       moe_dtype out_dtype, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (!valid_dtype(res_dtype) || !valid_dtype(out_dtype) || rows_max < 0)
+    return MOE_ERR_INVALID_ARGUMENT;
+  moe_status st = check_router_shape(T, d_model, E, k);
+  if (st != MOE_OK) return st;
+  if (!ws || !expert_offsets) return MOE_ERR_INVALID_ARGUMENT;
+  if (T > 0 && (!expert_ids || !slot || !gates || !out)) return MOE_ERR_INVALID_ARGUMENT;
+  if (rows_max > 0 && !y_packed) return MOE_ERR_INVALID_ARGUMENT;
+  if (!aligned16(y_packed) || !aligned16(expert_offsets) || !aligned16(expert_ids) ||
+      !aligned16(slot) || !aligned16(gates) || !aligned16(residual) || !aligned16(dense) ||
+      !aligned16(out) || ((uintptr_t)ws % kAlign) != 0)
+    return MOE_ERR_MISALIGNED;
+  if (ws_bytes < kAlign) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (fault_injected("moe_combine")) return MOE_ERR_CUDA;
+  g_launches = 0;
+  return cuda_status(enqueue_combine(y_packed, expert_offsets, expert_ids, slot, gates, T, d_model,
+                                     E, k, rows_max, residual, res_dtype == MOE_BF16, dense, out,
+                                     out_dtype == MOE_BF16, (int*)ws, stream));
+}
+
+// ---------------------------------------------------------------- whole layer
+
+namespace {
+
+struct LayerWs {
+  RouterWs router;
+  DispatchWs dispatch;
+  float *logits, *gates, *lb_stats;
+  int32_t *ids, *slot, *counts, *offsets, *row_token;
+  void *x_packed, *h_packed;
+  float* y_packed;
+  void* h_dense;
+  float* r_dense;
+  int64_t C, rows_max;
+};
+
+moe_status layer_layout(const moe_layer_args* a, uint8_t* base, LayerWs* w, size_t* bytes) {
+  if (!a) return MOE_ERR_INVALID_ARGUMENT;
+  moe_status st = check_router_shape(a->T, a->d_model, a->E, a->k);
+  if (st != MOE_OK) return st;
+  if (!valid_dtype(a->dtype) || !valid_dtype(a->out_dtype)) return MOE_ERR_INVALID_ARGUMENT;
+  st = moe_capacity(a->T, a->E, a->k, a->capacity_factor, &w->C);
+  if (st != MOE_OK) return st;
+  moe_packed_rows_max(a->T, a->E, a->k, w->C, &w->rows_max);
+  st = check_ffn_shape(a->E, w->rows_max, a->d_model, a->d_ff, a->dtype);
+  if (st != MOE_OK) return st;
+  if (a->T >= (int64_t)INT32_MAX) return MOE_ERR_UNSUPPORTED;
+  const int64_t T = a->T, R = w->rows_max;
+  const int E = a->E, k = a->k, d = a->d_model, f = a->d_ff;
+  const size_t es = esize(a->dtype);
+  Carve c{base};
+  w->router = carve_router(c, T, E);
+  w->dispatch = carve_dispatch(c, T, E, k);
+  w->logits = c.take<float>((size_t)T * E);
+  w->gates = c.take<float>((size_t)T * k);
+  w->lb_stats = c.take<float>((size_t)2 * E + 1);
+  w->ids = c.take<int32_t>((size_t)T * k);
+  w->slot = c.take<int32_t>((size_t)T * k);
+  w->counts = c.take<int32_t>((size_t)E);
+  w->offsets = c.take<int32_t>((size_t)E + 1);
+  w->row_token = c.take<int32_t>((size_t)R);
+  w->x_packed = c.take<uint8_t>((size_t)R * d * es);
+  w->h_packed = c.take<uint8_t>((size_t)R * f * es);
+  w->y_packed = c.take<float>((size_t)R * d);
+  const bool dense = a->dense_w1 != nullptr;
+  w->h_dense = dense ? (void*)c.take<uint8_t>((size_t)T * f * es) : nullptr;
+  w->r_dense = dense ? c.take<float>((size_t)T * d) : nullptr;
+  *bytes = c.off;
+  return MOE_OK;
+}
+
+}  // namespace
+
+moe_status moe_layer_workspace_bytes(const moe_layer_args* args, size_t* bytes) {
+  if (!bytes) return MOE_ERR_INVALID_ARGUMENT;
+  LayerWs w;
+  return layer_layout(args, nullptr, &w, bytes);
+}
+
+moe_status moe_layer_forward(const moe_layer_args* a, void* out, moe_layer_aux* aux, void* ws,
+                             size_t ws_bytes, moe_stream_t stream) {
+  LayerWs w;
+  size_t need = 0;
+  moe_status st = layer_layout(a, (uint8_t*)ws, &w, &need);
+  if (st != MOE_OK) return st;
+  const bool dense = a->dense_w1 != nullptr;
+  if (dense && !a->dense_w2) return MOE_ERR_INVALID_ARGUMENT;
+  if (!ws) return MOE_ERR_INVALID_ARGUMENT;
+  if (a->T > 0 && (!a->x || !a->w_router || !a->w1 || !a->w2 || !out)) return MOE_ERR_INVALID_ARGUMENT;
+  if (!aligned16(a->x) || !aligned16(a->w_router) || !aligned16(a->router_bias) ||
+      !aligned16(a->w1) || !aligned16(a->b1) || !aligned16(a->w2) || !aligned16(a->b2) ||
+      !aligned16(a->dense_w1) || !aligned16(a->dense_b1) || !aligned16(a->dense_w2) ||
+      !aligned16(a->dense_b2) || !aligned16(out) || ((uintptr_t)ws % kAlign) != 0)
+    return MOE_ERR_MISALIGNED;
+  if (aux && (!aligned16(aux->logits) || !aligned16(aux->expert_ids) || !aligned16(aux->gates) ||
+              !aligned16(aux->slot) || !aligned16(aux->expert_counts) ||
+              !aligned16(aux->expert_offsets) || !aligned16(aux->lb_stats)))
+    return MOE_ERR_MISALIGNED;
+  if (ws_bytes < need) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (fault_injected("moe_layer_forward")) return MOE_ERR_CUDA;
+  g_launches = 0;
+  if (a->T == 0) return MOE_OK;
+
+  float* logits = aux && aux->logits ? aux->logits : w.logits;
+  int32_t* ids = aux && aux->expert_ids ? aux->expert_ids : w.ids;
+  float* gates = aux && aux->gates ? aux->gates : w.gates;
+  int32_t* slot = aux && aux->slot ? aux->slot : w.slot;
+  int32_t* counts = aux && aux->expert_counts ? aux->expert_counts : w.counts;
+  int32_t* offsets = aux && aux->expert_offsets ? aux->expert_offsets : w.offsets;
+  float* lb = aux ? aux->lb_stats : nullptr;
+  int* status = (int*)ws;
+  const bool bf16 = a->dtype == MOE_BF16;
+  const int64_t T = a->T;
+  const int d = a->d_model, f = a->d_ff, E = a->E, k = a->k;
+
+  cudaError_t e = enqueue_router(a->x, bf16, T, d, a->w_router, a->router_bias, E, k, logits, ids,
+                                 gates, lb, a->aux_alpha, w.router.q_partial, stream);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  e = enqueue_dispatch(a->x, bf16, T, d, ids, E, k, w.C, slot, counts, offsets, w.row_token,
+                       w.x_packed, w.rows_max, w.dispatch.local_rank, w.dispatch.seg_counts,
+                       w.dispatch.seg_base, status, stream);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  if (dense) {
+    // PR-MoE fixed MLP on every token: one "expert" whose segment is all T rows of x
+    e = bf16 ? enqueue_expert_ffn_bf16(a->x, nullptr, 1, T, d, f, a->dense_w1, a->dense_b1,
+                                       a->dense_w2, a->dense_b2, w.h_dense, w.r_dense, T, status,
+                                       stream)
+             : enqueue_expert_ffn_f32((const float*)a->x, nullptr, 1, T, d, f,
+                                      (const float*)a->dense_w1, (const float*)a->dense_b1,
+                                      (const float*)a->dense_w2, (const float*)a->dense_b2,
+                                      (float*)w.h_dense, w.r_dense, status, stream);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  if (w.rows_max > 0) {
+    e = bf16 ? enqueue_expert_ffn_bf16(w.x_packed, offsets, E, w.rows_max, d, f, a->w1, a->b1,
+                                       a->w2, a->b2, w.h_packed, w.y_packed, w.C, status, stream)
+             : enqueue_expert_ffn_f32((const float*)w.x_packed, offsets, E, w.rows_max, d, f,
+                                      (const float*)a->w1, (const float*)a->b1,
+                                      (const float*)a->w2, (const float*)a->b2,
+                                      (float*)w.h_packed, w.y_packed, status, stream);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  e = enqueue_combine(w.y_packed, offsets, ids, slot, gates, T, d, E, k, w.rows_max,
+                      a->add_input_residual ? a->x : nullptr, bf16, dense ? w.r_dense : nullptr,
+                      out, a->out_dtype == MOE_BF16, status, stream);
+  return cuda_status(e);
+}
+
+// ---------------------------------------------------------------- status block
+
+moe_status moe_workspace_reset(void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (!ws || ws_bytes < kAlign) return MOE_ERR_INVALID_ARGUMENT;
+  return cuda_status(cudaMemsetAsync(ws, 0, kAlign, stream));
+}
+
+moe_status moe_get_device_error(const void* ws, int* code_out, moe_stream_t stream) {
+  if (!ws || !code_out) return MOE_ERR_INVALID_ARGUMENT;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
+  int code = 0;
+  if (cudaMemcpy(&code, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  *code_out = code;
+  return code ? MOE_ERR_DEVICE_FLAG : MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,189 @@
+// Dispatch: capacity-limited first-come slots and the expert-major packed copy of x.
+//
+// DeepSpeed-MoE notes §4.4: the gating kernel fuses top-k, a parallel prefix sum (cumsum) and a
+// scatter into a dense token-to-expert mapping table, and the layout transformation re-orders
+// rows explicitly by that table instead of multiplying by a sparse dispatch mask; comparison
+// article, "Expert Capacity Overflow": capacity = tokens / experts * capacity_factor, tokens
+// beyond it skip the expert and keep only the residual.
+//
+// Pairs p = t * k + j are ranked per expert in pair order (token order), with no atomics, so
+// the result is unique and deterministic:
+//   dispatch_count_kernel   one warp per segment of 256 consecutive pairs: in-warp ranks from
+//                           __match_any_sync, running per-expert counts in shared memory;
+//                           writes each pair's rank inside its segment and the segment totals
+//   dispatch_scan_kernel    one block: per expert, exclusive prefix over segments (segment
+//                           bases) and the demand; kept = min(demand, C); exclusive scan over
+//                           experts of kept -> offsets
+//   dispatch_scatter_kernel one warp per pair: position = segment base + rank, slot = position
+//                           or -1 beyond C, row_token, and a 16-byte vector copy of the row
+#include <type_traits>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+namespace {
+
+constexpr int kCountWarps = 8;
+
+__global__ void __launch_bounds__(kCountWarps * 32)
+    dispatch_count_kernel(const int32_t* __restrict__ ids, int64_t pairs, int64_t nseg, int E,
+                          int32_t* __restrict__ local_rank, int32_t* __restrict__ seg_counts,
+                          int* status) {
+  extern __shared__ int cnt_all[];  // [kCountWarps][E]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int* cnt = cnt_all + warp * E;
+  const int64_t seg = (int64_t)blockIdx.x * kCountWarps + warp;
+  if (seg >= nseg) return;
+  for (int e = lane; e < E; e += 32) cnt[e] = 0;
+  __syncwarp();
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int c = 0; c < kDispatchSeg / 32; ++c) {
+    const int64_t p = seg * kDispatchSeg + c * 32 + lane;
+    int e = -1;
+    if (p < pairs) {
+      e = ids[p];
+      if (e < 0 || e >= E) {
+        set_device_error(status, MOE_DEVERR_BAD_EXPERT);
+        e = -1;
+      }
+    }
+    const unsigned same = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(same & lt_mask);
+    const int base = e >= 0 ? cnt[e] : 0;
+    __syncwarp();
+    if (e >= 0 && rank == 0) cnt[e] = base + __popc(same);
+    __syncwarp();
+    if (p < pairs) local_rank[p] = e >= 0 ? base + rank : -1;
+  }
+  for (int e = lane; e < E; e += 32) seg_counts[seg * E + e] = cnt[e];
+}
+
+__global__ void __launch_bounds__(1024)
+    dispatch_scan_kernel(const int32_t* __restrict__ seg_counts, int64_t nseg, int E, int64_t C,
+                         int32_t* __restrict__ seg_base, int32_t* __restrict__ counts,
+                         int32_t* __restrict__ offsets) {
+  __shared__ int kept[MOE_MAX_EXPERTS];
+  __shared__ int warp_sums[32];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = 0;
+    int64_t s = 0;
+    for (; s + 8 <= nseg; s += 8) {
+      int v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = seg_counts[(s + u) * E + e];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        seg_base[(s + u) * E + e] = run;
+        run += v[u];
+      }
+    }
+    for (; s < nseg; ++s) {
+      const int v = seg_counts[s * E + e];
+      seg_base[s * E + e] = run;
+      run += v;
+    }
+    counts[e] = run;
+    kept[e] = (int)min((int64_t)run, C);
+  }
+  __syncthreads();
+  // exclusive scan of kept over experts (E <= 1024), one element per thread
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int v = tid < E ? kept[tid] : 0;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += u;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int ws = warp_sums[lane];
+    int wincl = ws;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, wincl, o);
+      if (lane >= o) wincl += u;
+    }
+    warp_sums[lane] = wincl - ws;  // exclusive prefix of warp totals
+  }
+  __syncthreads();
+  const int excl = incl - v + warp_sums[warp];
+  if (tid < E) offsets[tid] = excl;
+  if (tid == E - 1) offsets[E] = excl + v;
+}
+
+template <int VEC_BYTES>
+__global__ void __launch_bounds__(256)
+    dispatch_scatter_kernel(const uint8_t* __restrict__ x, int64_t row_bytes, int64_t pairs, int k,
+                            int E, int64_t C, const int32_t* __restrict__ ids,
+                            const int32_t* __restrict__ local_rank,
+                            const int32_t* __restrict__ seg_base,
+                            const int32_t* __restrict__ offsets, int32_t* __restrict__ slot,
+                            int32_t* __restrict__ row_token, uint8_t* __restrict__ x_packed,
+                            int64_t rows_max) {
+  const int lane = threadIdx.x & 31;
+  const int64_t p = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (p >= pairs) return;
+  const int e = ids[p];
+  const int r = local_rank[p];
+  int s = -1;
+  if (e >= 0 && e < E && r >= 0) {
+    const int pos = seg_base[(p / kDispatchSeg) * E + e] + r;
+    if (pos < C) s = pos;
+  }
+  if (lane == 0) slot[p] = s;
+  if (s < 0) return;
+  const int64_t row = (int64_t)offsets[e] + s;
+  if (row >= rows_max) return;  // cannot happen with rows_max >= min(T k, E C)
+  const int64_t t = p / k;
+  if (lane == 0) row_token[row] = (int32_t)t;
+  using V = typename std::conditional<VEC_BYTES == 16, uint4,
+            typename std::conditional<VEC_BYTES == 8, uint2, uint32_t>::type>::type;
+  const V* src = reinterpret_cast<const V*>(x + t * row_bytes);
+  V* dst = reinterpret_cast<V*>(x_packed + row * row_bytes);
+  const int64_t n = row_bytes / VEC_BYTES;
+  for (int64_t i = lane; i < n; i += 32) dst[i] = src[i];
+}
+
+}  // namespace
+
+cudaError_t enqueue_dispatch(const void* x, bool bf16, int64_t T, int d, const int32_t* ids, int E,
+                             int k, int64_t C, int32_t* slot, int32_t* counts, int32_t* offsets,
+                             int32_t* row_token, void* x_packed, int64_t rows_max,
+                             int32_t* local_rank, int32_t* seg_counts, int32_t* seg_base,
+                             int* status, cudaStream_t stream) {
+  const int64_t pairs = T * k;
+  const int64_t nseg = dispatch_num_segments(pairs);
+  if (pairs > 0) {
+    const unsigned blocks = (unsigned)((nseg + kCountWarps - 1) / kCountWarps);
+    dispatch_count_kernel<<<blocks, kCountWarps * 32, kCountWarps * E * sizeof(int), stream>>>(
+        ids, pairs, nseg, E, local_rank, seg_counts, status);
+    count_launch();
+  }
+  dispatch_scan_kernel<<<1, 1024, 0, stream>>>(seg_counts, nseg, E, C, seg_base, counts, offsets);
+  count_launch();
+  if (pairs > 0) {
+    const int64_t row_bytes = (int64_t)d * (bf16 ? 2 : 4);
+    const unsigned blocks = (unsigned)((pairs * 32 + 255) / 256);
+    const uint8_t* xs = (const uint8_t*)x;
+    uint8_t* xp = (uint8_t*)x_packed;
+    if (row_bytes % 16 == 0)
+      dispatch_scatter_kernel<16><<<blocks, 256, 0, stream>>>(xs, row_bytes, pairs, k, E, C, ids,
+                                                              local_rank, seg_base, offsets, slot,
+                                                              row_token, xp, rows_max);
+    else if (row_bytes % 8 == 0)
+      dispatch_scatter_kernel<8><<<blocks, 256, 0, stream>>>(xs, row_bytes, pairs, k, E, C, ids,
+                                                             local_rank, seg_base, offsets, slot,
+                                                             row_token, xp, rows_max);
+    else
+      dispatch_scatter_kernel<4><<<blocks, 256, 0, stream>>>(xs, row_bytes, pairs, k, E, C, ids,
+                                                             local_rank, seg_base, offsets, slot,
+                                                             row_token, xp, rows_max);
+    count_launch();
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace moe

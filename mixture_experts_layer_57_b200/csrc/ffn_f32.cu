@@ -1,0 +1,81 @@
+// Expert FFN for fp32 tensors on fp32 FMA units (no TF32): one block per (packed row, 128
+// output features); the row is staged in shared memory and each thread accumulates one output
+// feature over K in index order. Used for fp32 layers, whose tolerance (1e-5) TF32 or bf16
+// tensor-core inputs cannot meet; bf16 layers use the tcgen05 grouped GEMM.
+//     h[r, :] = GeLU(W1[e] x[r, :] + b1[e]),   y[r, :] = W2[e] h[r, :] + b2[e]
+// (MoE survey notes §1.1.2.1: an expert is a two-layer feed-forward network.)
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+namespace {
+
+constexpr int kFeat = 128;
+
+template <bool GELU>
+__global__ void __launch_bounds__(kFeat)
+    ffn_f32_kernel(const float* __restrict__ X, const int32_t* __restrict__ offsets, int E,
+                   int n_out, int K, int64_t rows_max, const float* __restrict__ W,
+                   const float* __restrict__ bias, float* __restrict__ out, int* status) {
+  extern __shared__ float xs[];
+  // offsets == nullptr: one segment covering all rows_max rows (dense MLP, E == 1)
+  const int64_t start = offsets ? offsets[0] : 0, total = offsets ? offsets[E] : rows_max;
+  if (start < 0 || total < start || total > rows_max) {
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
+      set_device_error(status, MOE_DEVERR_BAD_OFFSETS);
+    return;
+  }
+  const int f = blockIdx.y * kFeat + threadIdx.x;
+  for (int64_t r = start + blockIdx.x; r < total; r += gridDim.x) {
+    // expert owning row r: largest e with offsets[e] <= r
+    int lo = 0, hi = E;
+    while (offsets && hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (offsets[mid] <= r) lo = mid;
+      else hi = mid;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < K; i += kFeat) xs[i] = X[r * K + i];
+    __syncthreads();
+    if (f < n_out) {
+      const float* w = W + ((int64_t)lo * n_out + f) * K;
+      float acc = 0.0f;
+      for (int i = 0; i < K; ++i) acc = fmaf(xs[i], w[i], acc);
+      float v = acc + (bias ? bias[(int64_t)lo * n_out + f] : 0.0f);
+      if (GELU) v = gelu_erf(v);
+      out[r * n_out + f] = v;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t enqueue_expert_ffn_f32(const float* x_packed, const int32_t* offsets, int E,
+                                   int64_t rows_max, int d, int d_ff, const float* w1,
+                                   const float* b1, const float* w2, const float* b2,
+                                   float* h_packed, float* y_packed, int* status,
+                                   cudaStream_t stream) {
+  if (rows_max == 0) return cudaSuccess;
+  const unsigned gx = (unsigned)(rows_max < 65536 ? rows_max : 65536);
+  const size_t smem1 = (size_t)d * sizeof(float), smem2 = (size_t)d_ff * sizeof(float);
+  const size_t smem_max = smem1 > smem2 ? smem1 : smem2;
+  static size_t attr_done = 0;
+  if (smem_max > 48 * 1024 && attr_done < smem_max) {
+    cudaError_t e1 = cudaFuncSetAttribute(ffn_f32_kernel<true>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max);
+    cudaError_t e2 = cudaFuncSetAttribute(ffn_f32_kernel<false>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max);
+    if (e1 != cudaSuccess) return e1;
+    if (e2 != cudaSuccess) return e2;
+    attr_done = smem_max;
+  }
+  ffn_f32_kernel<true><<<dim3(gx, (d_ff + kFeat - 1) / kFeat), kFeat, smem1, stream>>>(
+      x_packed, offsets, E, d_ff, d, rows_max, w1, b1, h_packed, status);
+  count_launch();
+  ffn_f32_kernel<false><<<dim3(gx, (d + kFeat - 1) / kFeat), kFeat, smem2, stream>>>(
+      h_packed, offsets, E, d, d_ff, rows_max, w2, b2, y_packed, status);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,417 @@
+// Grouped expert GEMM on sm_100a tensor cores (tcgen05 + TMEM + TMA), with the bias(+GeLU)
+// epilogue fused.
+//
+// Computes, for every expert e and every packed row r of its segment
+// [offsets[e], offsets[e+1]):
+//     out[r, f] = act( sum_k W[e*N + f, k] * X[r, k] + bias[e, f] ),   f < N
+// which is one layer of the expert FFN ("Sparse GEMM -> Dense GEMM": dense per-expert GEMMs on
+// the rows the layout transform packed together, DeepSpeed-MoE notes §4.4 / §5).
+//
+// Orientation: the weights are the MMA's A operand (M = 128 output features per tile) and the
+// packed token rows are the B operand (N = BN tokens per tile, 16..256). The accumulator tile
+// is therefore [features x tokens] in TMEM (lane = feature, column = token). A tile of an
+// expert with few rows (decode: one row) issues an MMA with N = 16 instead of padding tokens
+// to M = 128, so ragged and tiny experts cost no extra tensor work; the weight tiles stream
+// from HBM once per token tile.
+//
+// Schedule: persistent CTAs (one per SM) walk tiles t = blockIdx.x, blockIdx.x + gridDim.x, ...
+// of a list ordered (expert, feature tile, token tile), built in shared memory from the device
+// offsets, so no host synchronisation is needed for the ragged sizes. Roles per CTA:
+//     warp 0      TMA producer: K-major 128x64 weight tile and BNx64 token tile per stage,
+//                 128-byte swizzle, STAGES-deep mbarrier ring
+//     warp 1      allocates TMEM, one thread issues tcgen05.mma (K = 16 per instruction) into
+//                 one of two accumulators, commits stage release and accumulator-full barriers
+//     warps 2..5  epilogue: tcgen05.ld of the accumulator, + bias, GeLU (erf form) and bf16
+//                 rounding for the first layer, or fp32 for the second, masked to the valid
+//                 rows/features, stored to global; then release the accumulator
+// Every wait is bounded (about 2 s): on expiry the kernel records MOE_DEVERR_TIMEOUT in the
+// status word, the other roles stop, in-flight TMA copies and MMAs are drained, TMEM is freed.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+namespace {
+
+constexpr int kBM = 128;         // output features per tile (MMA M)
+constexpr int kBK = 64;          // K per stage: one 128-byte swizzle row of bf16
+constexpr int kUmmaK = 16;       // K per tcgen05.mma (kind::f16)
+constexpr int kThreads = 192;    // 6 warps
+
+template <int BN>
+struct Cfg {
+  static constexpr int kABytes = kBM * kBK * 2;
+  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStagesFit = (200 * 1024) / kStageBytes;
+  static constexpr int kStages = kStagesFit > 12 ? 12 : kStagesFit;
+  static constexpr int kTmemCols = (2 * BN) < 32 ? 32 : (2 * BN);
+  // barriers: full[S], empty[S], tmem_full[2], tmem_empty[2], drain  (8 bytes each, <= 64 of them)
+  static constexpr int kBarBytes = 8 * 64;
+  static constexpr int kAuxBytes = kBarBytes + 16 + 2 * 4 * (MOE_MAX_EXPERTS + 1);
+  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kAuxBytes;
+  static_assert(kStageBytes % 1024 == 0, "stage tiles must stay 1024-byte aligned");
+  static_assert(2 * kStages + 5 <= 64, "barrier area too small");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+};
+
+struct Params {
+  const int32_t* offsets;  // [E+1]
+  int E;
+  int n_out;               // output features per expert
+  int K;
+  int64_t rows_max;
+  const uint16_t* bias;    // [E, n_out] bf16, or nullptr
+  void* out;               // [rows_max, n_out]: bf16 (GeLU layer) or fp32
+  int* status;
+};
+
+struct Tile {
+  int e, f0, row0, n_valid;
+};
+
+template <int BN>
+__device__ __forceinline__ Tile decode_tile(int t, const int* prefix, const int* seg, int E,
+                                            int n_ftiles) {
+  int lo = 0, hi = E;  // prefix[lo] <= t < prefix[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (prefix[mid] <= t) lo = mid;
+    else hi = mid;
+  }
+  const int rows = seg[lo + 1] - seg[lo];
+  const int ntt = (rows + BN - 1) / BN;
+  const int local = t - prefix[lo];
+  const int ft = local / ntt;
+  const int jt = local - ft * ntt;
+  Tile tl;
+  tl.e = lo;
+  tl.f0 = ft * kBM;
+  tl.row0 = seg[lo] + jt * BN;
+  tl.n_valid = min(BN, rows - jt * BN);
+  return tl;
+}
+
+// Wait bounded by time only (used to drain in-flight copies/MMAs while unwinding).
+__device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity, int* status) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      set_device_error(status, MOE_DEVERR_TIMEOUT);
+      return;
+    }
+  }
+}
+
+template <int BN, bool GELU_BF16_OUT>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmW,
+                        const __grid_constant__ CUtensorMap tmX, const Params p) {
+  using C = Cfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t base_addr = (raw_addr + 1023u) & ~1023u;
+  uint8_t* base = smem_raw + (base_addr - raw_addr);
+
+  uint8_t* aux = base + C::kStages * C::kStageBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(aux);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(aux + C::kBarBytes);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(aux + C::kBarBytes + 4);
+  int* prefix = reinterpret_cast<int*>(aux + C::kBarBytes + 16);
+  int* seg = prefix + (MOE_MAX_EXPERTS + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int S = C::kStages;
+  auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
+  auto empty_bar = [&](int s) { return smem_u32(&bars[S + s]); };
+  auto tfull_bar = [&](int a) { return smem_u32(&bars[2 * S + a]); };
+  auto tempty_bar = [&](int a) { return smem_u32(&bars[2 * S + 2 + a]); };
+  const uint32_t drain_bar = smem_u32(&bars[2 * S + 4]);
+
+  // ------------------------------------------------------------ prologue
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 128);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(&tmX);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), C::kTmemCols);
+    tmem_relinquish();
+  }
+  const int n_ftiles = (p.n_out + kBM - 1) / kBM;
+  if (warp == 2) {
+    // Tile list: prefix[e] = first tile of expert e; validates the device offsets.
+    const int E = p.E;
+    const int chunk = (E + 31) / 32;
+    const int e0 = min(E, lane * chunk), e1 = min(E, e0 + chunk);
+    bool bad = false;
+    int local = 0;
+    // offsets == nullptr: one segment covering all rows_max rows (dense MLP, E == 1)
+    auto off = [&](int e) -> int {
+      return p.offsets ? p.offsets[e] : (e == 0 ? 0 : (int)p.rows_max);
+    };
+    for (int e = e0; e < e1; ++e) {
+      const int a = off(e), b = off(e + 1);
+      seg[e] = a;
+      if (a < 0 || b < a || (int64_t)b > p.rows_max) bad = true;
+      else local += n_ftiles * ((b - a + BN - 1) / BN);
+    }
+    if (lane == 0) seg[E] = off(E);
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int run = incl - local;
+    for (int e = e0; e < e1; ++e) {
+      prefix[e] = run;
+      const int a = seg[e], b = off(e + 1);
+      if (!(a < 0 || b < a || (int64_t)b > p.rows_max)) run += n_ftiles * ((b - a + BN - 1) / BN);
+    }
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    bad = __any_sync(0xffffffffu, bad);
+    __syncwarp();
+    if (lane == 0) {
+      prefix[E] = bad ? 0 : total;
+      if (bad && blockIdx.x == 0) set_device_error(p.status, MOE_DEVERR_BAD_OFFSETS);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const int total_tiles = prefix[p.E];
+  const int n_kb = (p.K + kBK - 1) / kBK;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+        const Tile tl = decode_tile<BN>(t, prefix, seg, p.E, n_ftiles);
+        const int w_row = tl.e * p.n_out + tl.f0;
+        bool ok = true;
+        for (int kb = 0; kb < n_kb; ++kb) {
+          if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sa = base_addr + stage * C::kStageBytes;
+          mbar_arrive_expect_tx(full_bar(stage), C::kStageBytes);
+          tma_load_2d(sa, &tmW, kb * kBK, w_row, full_bar(stage));
+          tma_load_2d(sa + C::kABytes, &tmX, kb * kBK, tl.row0, full_bar(stage));
+          ++issued;
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+      }
+      // drain: the last min(issued, S) loads may still be landing
+      for (int i = max(0, issued - S); i < issued; ++i)
+        mbar_wait_drain(full_bar(i % S), (uint32_t)((i / S) & 1), p.status);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+        const Tile tl = decode_tile<BN>(t, prefix, seg, p.E, n_ftiles);
+        if (!mbar_wait_bounded(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        const int n_mma = max(16, (tl.n_valid + 15) & ~15);
+        const uint32_t idesc = idesc_bf16_f32(kBM, n_mma);
+        for (int kb = 0; kb < n_kb; ++kb) {
+          if (!mbar_wait_bounded(full_bar(stage), phase, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = base_addr + stage * C::kStageBytes;
+          const uint64_t adesc = smem_desc_sw128(sa);
+          const uint64_t bdesc = smem_desc_sw128(sa + C::kABytes);
+#pragma unroll
+          for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
+            // +32 bytes along K inside the swizzled 128-byte row = +2 in the 16-byte address field
+            tc_mma_bf16(d_tmem, adesc + (uint64_t)(2 * kk), bdesc + (uint64_t)(2 * kk), idesc,
+                        (kb | kk) != 0 ? 1u : 0u);
+          }
+          tc_commit(empty_bar(stage));
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(tfull_bar(acc));
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      // drain every MMA this thread issued before TMEM is released
+      tc_commit(drain_bar);
+      mbar_wait_drain(drain_bar, 0, p.status);
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue (warps 2..5)
+    const int quarter = warp & 3;  // TMEM lanes this warp may access: [32*quarter, 32*quarter+32)
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+      const Tile tl = decode_tile<BN>(t, prefix, seg, p.E, n_ftiles);
+      if (!mbar_wait_bounded_warp(tfull_bar(acc), acc_phase, abort_flag, p.status)) break;
+      tc_fence_after();
+      const int f = tl.f0 + quarter * 32 + lane;
+      const bool f_ok = f < p.n_out;
+      const float bv = (p.bias != nullptr && f_ok)
+                           ? bf16_to_f32(p.bias[(int64_t)tl.e * p.n_out + f])
+                           : 0.0f;
+      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
+      for (int c0 = 0; c0 < tl.n_valid; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld_32x32b_x16(taddr + (uint32_t)c0, r);
+        tmem_ld_wait();
+        if (f_ok) {
+          const int nc = min(16, tl.n_valid - c0);
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            if (c < nc) {
+              const int64_t o = (int64_t)(tl.row0 + c0 + c) * p.n_out + f;
+              const float v = __uint_as_float(r[c]) + bv;
+              if constexpr (GELU_BF16_OUT) {
+                reinterpret_cast<uint16_t*>(p.out)[o] = f32_to_bf16_rn(gelu_erf(v));
+              } else {
+                reinterpret_cast<float*>(p.out)[o] = v;
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(tempty_bar(acc));
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(f);
+  }();
+  return fn;
+}
+
+// K-major bf16 matrix [rows, K] (row stride K elements) read in boxes of box_rows x 64.
+bool make_kmajor_map(CUtensorMap* m, const void* ptr, int64_t rows, int K, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t gstride[1] = {(cuuint64_t)K * 2};
+  cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)box_rows};
+  cuuint32_t estride[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), gdim, gstride, box,
+            estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, bool GELU>
+cudaError_t launch_one(const CUtensorMap& tmW, const CUtensorMap& tmX, const Params& p,
+                       cudaStream_t stream) {
+  auto kern = grouped_gemm_kernel<BN, GELU>;
+  static bool attr_set = false;  // per instantiation
+  if (!attr_set) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<BN>::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  kern<<<num_sms(), kThreads, Cfg<BN>::kSmemBytes, stream>>>(tmW, tmX, p);
+  count_launch();
+  return cudaGetLastError();
+}
+
+template <int BN>
+cudaError_t launch_pair(const CUtensorMap& tmW1, const CUtensorMap& tmX, const CUtensorMap& tmW2,
+                        const CUtensorMap& tmH, const Params& p1, const Params& p2,
+                        cudaStream_t stream) {
+  cudaError_t e = launch_one<BN, true>(tmW1, tmX, p1, stream);
+  if (e != cudaSuccess) return e;
+  return launch_one<BN, false>(tmW2, tmH, p2, stream);
+}
+
+}  // namespace
+
+cudaError_t enqueue_expert_ffn_bf16(const void* x_packed, const int32_t* offsets, int E,
+                                    int64_t rows_max, int d, int d_ff, const void* w1,
+                                    const void* b1, const void* w2, const void* b2, void* h_packed,
+                                    float* y_packed, int64_t capacity_hint, int* status,
+                                    cudaStream_t stream) {
+  int BN = 256;
+  if (capacity_hint <= 16) BN = 16;
+  else if (capacity_hint <= 32) BN = 32;
+  else if (capacity_hint <= 64) BN = 64;
+  else if (capacity_hint <= 128) BN = 128;
+
+  CUtensorMap tmW1, tmX, tmW2, tmH;
+  if (!make_kmajor_map(&tmW1, w1, (int64_t)E * d_ff, d, kBM) ||
+      !make_kmajor_map(&tmX, x_packed, rows_max, d, BN) ||
+      !make_kmajor_map(&tmW2, w2, (int64_t)E * d, d_ff, kBM) ||
+      !make_kmajor_map(&tmH, h_packed, rows_max, d_ff, BN))
+    return cudaErrorInvalidValue;
+
+  Params p1{offsets, E, d_ff, d, rows_max, (const uint16_t*)b1, h_packed, status};
+  Params p2{offsets, E, d, d_ff, rows_max, (const uint16_t*)b2, y_packed, status};
+  switch (BN) {
+    case 16: return launch_pair<16>(tmW1, tmX, tmW2, tmH, p1, p2, stream);
+    case 32: return launch_pair<32>(tmW1, tmX, tmW2, tmH, p1, p2, stream);
+    case 64: return launch_pair<64>(tmW1, tmX, tmW2, tmH, p1, p2, stream);
+    case 128: return launch_pair<128>(tmW1, tmX, tmW2, tmH, p1, p2, stream);
+    default: return launch_pair<256>(tmW1, tmX, tmW2, tmH, p1, p2, stream);
+  }
+}
+
+}  // namespace moe

@@ -1,0 +1,60 @@
+// Internal enqueue functions of the MoE-layer kernels (host side). Not part of the C ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+// Incremented once per kernel launch on the calling host thread (reset by every entry point).
+void count_launch();
+
+// Number of SMs of the current device (cached per device).
+int num_sms();
+
+// ---------------------------------------------------------------- router
+constexpr int kRouterTokensPerBlock = 64;
+inline int64_t router_num_blocks(int64_t T) {
+  return (T + kRouterTokensPerBlock - 1) / kRouterTokensPerBlock;
+}
+cudaError_t enqueue_router(const void* x, bool x_bf16, int64_t T, int d, const float* w_router,
+                           const float* router_bias, int E, int k, float* logits, int32_t* ids,
+                           float* gates, float* lb_stats, float aux_alpha, float* q_partial,
+                           cudaStream_t stream);
+
+// ---------------------------------------------------------------- dispatch
+constexpr int kDispatchSeg = 256;  // (token, choice) pairs per counting segment (one warp)
+inline int64_t dispatch_num_segments(int64_t pairs) {
+  return (pairs + kDispatchSeg - 1) / kDispatchSeg;
+}
+cudaError_t enqueue_dispatch(const void* x, bool bf16, int64_t T, int d, const int32_t* ids, int E,
+                             int k, int64_t C, int32_t* slot, int32_t* counts, int32_t* offsets,
+                             int32_t* row_token, void* x_packed, int64_t rows_max,
+                             int32_t* local_rank, int32_t* seg_counts, int32_t* seg_base,
+                             int* status, cudaStream_t stream);
+
+// ---------------------------------------------------------------- expert FFN
+cudaError_t enqueue_expert_ffn_bf16(const void* x_packed, const int32_t* offsets, int E,
+                                    int64_t rows_max, int d, int d_ff, const void* w1,
+                                    const void* b1, const void* w2, const void* b2, void* h_packed,
+                                    float* y_packed, int64_t capacity_hint, int* status,
+                                    cudaStream_t stream);
+cudaError_t enqueue_expert_ffn_f32(const float* x_packed, const int32_t* offsets, int E,
+                                   int64_t rows_max, int d, int d_ff, const float* w1,
+                                   const float* b1, const float* w2, const float* b2,
+                                   float* h_packed, float* y_packed, int* status,
+                                   cudaStream_t stream);
+// Largest d_model / d_ff the fp32 FFN accepts (one activation row is staged in shared memory).
+constexpr int kFfnF32MaxDim = 16384;
+
+// ---------------------------------------------------------------- combine
+cudaError_t enqueue_combine(const float* y_packed, const int32_t* offsets, const int32_t* ids,
+                            const int32_t* slot, const float* gates, int64_t T, int d, int E,
+                            int k, int64_t rows_max, const void* residual, bool res_bf16,
+                            const float* dense, void* out, bool out_bf16, int* status,
+                            cudaStream_t stream);
+
+}  // namespace moe

@@ -1,0 +1,231 @@
+// Router: logits = x W_r^T (+ b_r) in fp32, softmax over all E experts, top-k, and the Switch
+// load-balance statistics (f_i, Q_i, aux).
+//
+// DeepSpeed MoE blog, MoE formula p(x) = softmax(W_r x) and the listing's
+// `expert_ids, gates = topk(scores, k)`; comparison article, "Router computation"
+// (logits = x W_r, p = softmax(logits)) and "Top-1 routing decision"; MoE survey notes
+// §1.1.4.1 (f_i, Q_i, loss = alpha * N * sum f_i Q_i).
+//
+// Kernels:
+//   router_logits_kernel  tiled fp32 GEMM, 64 tokens x 64 experts per block, fixed K order
+//   router_topk_kernel    one warp per token: max, sum of exp, p = exp(l - max) / sum,
+//                         k rounds of warp argmax on the logits (ties -> lower index);
+//                         per-block partial sums of p per expert in a fixed order
+//   router_stats_kernel   one block: f from the first choices, Q from the partials in block
+//                         order, aux = alpha * E * sum f Q (sequential)
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+namespace {
+
+constexpr int kLBM = 64, kLBN = 64, kLBK = 32;
+
+template <bool XBF16>
+__global__ void __launch_bounds__(256) router_logits_kernel(const void* __restrict__ x,
+                                                            const float* __restrict__ w,
+                                                            const float* __restrict__ bias,
+                                                            int64_t T, int d, int E,
+                                                            float* __restrict__ logits) {
+  __shared__ float xs[kLBK][kLBM + 4];
+  __shared__ float ws[kLBK][kLBN + 4];
+  const int tx = threadIdx.x & 15;   // expert lane
+  const int ty = threadIdx.x >> 4;   // token lane
+  const int64_t t0 = (int64_t)blockIdx.x * kLBM;
+  const int e0 = blockIdx.y * kLBN;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < d; k0 += kLBK) {
+    // stage x[t0 .. t0+64, k0 .. k0+32] and w[e0 .. e0+64, k0 .. k0+32] (transposed in smem)
+    for (int i = threadIdx.x; i < kLBM * kLBK; i += 256) {
+      const int r = i / kLBK, c = i % kLBK;
+      const int64_t t = t0 + r;
+      const int kk = k0 + c;
+      xs[c][r] = (t < T && kk < d) ? load_elem<XBF16>(x, t * d + kk) : 0.0f;
+      const int e = e0 + r;
+      ws[c][r] = (e < E && kk < d) ? w[(int64_t)e * d + kk] : 0.0f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int c = 0; c < kLBK; ++c) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = xs[c][ty + 16 * i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b[j] = ws[c][tx + 16 * j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t t = t0 + ty + 16 * i;
+    if (t >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = e0 + tx + 16 * j;
+      if (e < E) logits[t * E + e] = acc[i][j] + (bias ? bias[e] : 0.0f);
+    }
+  }
+}
+
+// EPL = experts per lane (E <= 32 * EPL); expert e lives in lane e % 32, slot e / 32.
+template <int EPL>
+__global__ void __launch_bounds__(256) router_topk_kernel(const float* __restrict__ logits,
+                                                          int64_t T, int E, int k,
+                                                          int32_t* __restrict__ ids,
+                                                          float* __restrict__ gates,
+                                                          float* __restrict__ q_partial) {
+  __shared__ float qs[8][MOE_MAX_EXPERTS];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float q[EPL];
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) q[i] = 0.0f;
+  const int64_t tb = (int64_t)blockIdx.x * kRouterTokensPerBlock;
+  for (int r = warp; r < kRouterTokensPerBlock; r += 8) {
+    const int64_t t = tb + r;
+    if (t >= T) break;
+    float l[EPL];
+    float m = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      l[i] = e < E ? logits[t * E + e] : -INFINITY;
+      m = fmaxf(m, l[i]);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float ex[EPL];
+    float s = 0.0f;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      ex[i] = (lane + 32 * i) < E ? expf(l[i] - m) : 0.0f;
+      s += ex[i];
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    float p[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      p[i] = ex[i] / s;
+      q[i] += p[i];
+    }
+    // top-k on the logits: k rounds of (value desc, index asc) warp argmax
+    uint32_t taken = 0;
+    for (int j = 0; j < k; ++j) {
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E && !(taken >> i & 1u) && (l[i] > bv || bi == 0x7fffffff)) {
+          bv = l[i];
+          bi = e;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ov > bv || (ov == bv && oi < bi)) {
+          bv = ov;
+          bi = oi;
+        }
+      }
+      const int owner = bi & 31, slot_i = bi >> 5;
+      float pv = 0.0f;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i)
+        if (i == slot_i) pv = p[i];
+      pv = __shfl_sync(0xffffffffu, pv, owner);
+      if (lane == owner) taken |= 1u << slot_i;
+      if (lane == 0) {
+        ids[t * k + j] = bi;
+        gates[t * k + j] = pv;
+      }
+    }
+  }
+  // fixed-order reduction of the per-warp partial sums of p
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    const int e = lane + 32 * i;
+    if (e < E) qs[warp][e] = q[i];
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += 256) {
+    float s = 0.0f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) s += qs[w][e];
+    q_partial[(int64_t)blockIdx.x * E + e] = s;
+  }
+}
+
+__global__ void __launch_bounds__(1024) router_stats_kernel(const int32_t* __restrict__ ids,
+                                                            int64_t T, int E, int k,
+                                                            const float* __restrict__ q_partial,
+                                                            int64_t nblk, float alpha,
+                                                            float* __restrict__ lb) {
+  __shared__ int hist[MOE_MAX_EXPERTS];
+  __shared__ float prod[MOE_MAX_EXPERTS];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  for (int64_t t = threadIdx.x; t < T; t += blockDim.x) {
+    const int e = ids[t * k];
+    if (e >= 0 && e < E) atomicAdd(&hist[e], 1);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    float s = 0.0f;
+    for (int64_t b = 0; b < nblk; ++b) s += q_partial[b * E + e];
+    const float Q = s / (float)T;
+    const float f = (float)hist[e] / (float)T;
+    lb[e] = f;
+    lb[E + e] = Q;
+    prod[e] = f * Q;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float s = 0.0f;
+    for (int e = 0; e < E; ++e) s += prod[e];
+    lb[2 * E] = alpha * (float)E * s;
+  }
+}
+
+template <int EPL>
+void launch_topk(const float* logits, int64_t T, int E, int k, int32_t* ids, float* gates,
+                 float* q_partial, cudaStream_t stream) {
+  router_topk_kernel<EPL><<<(unsigned)router_num_blocks(T), 256, 0, stream>>>(logits, T, E, k, ids,
+                                                                              gates, q_partial);
+}
+
+}  // namespace
+
+cudaError_t enqueue_router(const void* x, bool x_bf16, int64_t T, int d, const float* w_router,
+                           const float* router_bias, int E, int k, float* logits, int32_t* ids,
+                           float* gates, float* lb_stats, float aux_alpha, float* q_partial,
+                           cudaStream_t stream) {
+  if (T == 0) return cudaSuccess;
+  dim3 grid((unsigned)((T + kLBM - 1) / kLBM), (E + kLBN - 1) / kLBN);
+  if (x_bf16)
+    router_logits_kernel<true><<<grid, 256, 0, stream>>>(x, w_router, router_bias, T, d, E, logits);
+  else
+    router_logits_kernel<false><<<grid, 256, 0, stream>>>(x, w_router, router_bias, T, d, E, logits);
+  count_launch();
+  if (E <= 32) launch_topk<1>(logits, T, E, k, ids, gates, q_partial, stream);
+  else if (E <= 64) launch_topk<2>(logits, T, E, k, ids, gates, q_partial, stream);
+  else if (E <= 128) launch_topk<4>(logits, T, E, k, ids, gates, q_partial, stream);
+  else if (E <= 256) launch_topk<8>(logits, T, E, k, ids, gates, q_partial, stream);
+  else if (E <= 512) launch_topk<16>(logits, T, E, k, ids, gates, q_partial, stream);
+  else launch_topk<32>(logits, T, E, k, ids, gates, q_partial, stream);
+  count_launch();
+  if (lb_stats) {
+    router_stats_kernel<<<1, 1024, 0, stream>>>(ids, T, E, k, q_partial, router_num_blocks(T),
+                                                aux_alpha, lb_stats);
+    count_launch();
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace moe

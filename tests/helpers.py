@@ -1,0 +1,106 @@
+"""Shared helpers of the GPU parity tests: device copies of the synthetic inputs, one call of the
+layer through the C ABI, and the output tolerances.
+
+Tolerances (floating-point outputs; integer routing/dispatch results are compared bit-exactly):
+  * fp32 layers: max |out - oracle| <= 1e-5 (absolute, outputs are O(1)).
+  * bf16 layers, parity run with fp32 output: max-abs <= 2e-2 and relative L2 <= 1e-2.
+  * bf16 layers, bf16 output: |out - oracle| <= 2e-2 + half a bf16 ulp of |oracle| per element,
+    and relative L2 <= 1e-2 (rounding the output to bf16 alone costs up to half an ulp, which
+    exceeds 2e-2 once |out| >= 4).
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import synth
+from mixture_experts_layer_57_b200 import moe
+
+FP32_ATOL = 1e-5
+BF16_ATOL = 2e-2
+BF16_REL_L2 = 1e-2
+
+
+def to_dev(a: np.ndarray, device="cuda") -> torch.Tensor:
+    """Host array (bf16 as uint16 bits, or f32/int32) -> device tensor of the same values."""
+    if a is None:
+        return None
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).to(device).view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+
+def to_host(t: torch.Tensor) -> np.ndarray:
+    """Device tensor -> host array (bf16 as uint16 bits)."""
+    t = t.detach().cpu()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view(np.uint16).copy()
+    return t.numpy().copy()
+
+
+def as_f64(a: np.ndarray) -> np.ndarray:
+    return synth.bf16_bits_to_f32(a).astype(np.float64) if a.dtype == np.uint16 else a.astype(np.float64)
+
+
+def dev_inputs(inp: dict, device="cuda") -> dict:
+    return {k: (to_dev(v, device) if isinstance(v, np.ndarray) else v) for k, v in inp.items()}
+
+
+def run_layer(w: synth.Workload, d_inp: dict, out_dtype=None, add_input_residual=None,
+              ws: torch.Tensor = None) -> dict:
+    """One moe_layer_forward on device inputs; returns host copies of every output."""
+    T, E, k = w.T, w.E, w.k
+    x = d_inp["x"]
+    dense = None
+    if w.dense:
+        dense = (d_inp["dense_w1"], d_inp["dense_b1"], d_inp["dense_w2"], d_inp["dense_b2"])
+    res = w.add_input_residual if add_input_residual is None else add_input_residual
+    args = moe.layer_args(x, d_inp["w_router"], d_inp["w1"], d_inp["b1"], d_inp["w2"], d_inp["b2"],
+                          k=k, capacity_factor=w.capacity_factor, router_bias=d_inp.get("router_bias"),
+                          dense=dense, add_input_residual=res, aux_alpha=w.aux_alpha,
+                          out_dtype=out_dtype)
+    dev = x.device
+    aux = dict(logits=torch.empty(T, E, dtype=torch.float32, device=dev),
+               expert_ids=torch.empty(T, k, dtype=torch.int32, device=dev),
+               gates=torch.empty(T, k, dtype=torch.float32, device=dev),
+               slot=torch.empty(T, k, dtype=torch.int32, device=dev),
+               expert_counts=torch.empty(E, dtype=torch.int32, device=dev),
+               expert_offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+               lb_stats=torch.empty(2 * E + 1, dtype=torch.float32, device=dev))
+    odt = x.dtype if out_dtype is None else out_dtype
+    out = torch.empty(T, w.d_model, dtype=odt, device=dev)
+    if ws is None:
+        ws = moe.workspace(moe.moe_layer_workspace_bytes(args), dev)
+    moe.moe_layer_forward(args, out, aux=aux, ws=ws)
+    err = moe.moe_get_device_error(ws)
+    r = {name: to_host(t) for name, t in aux.items()}
+    r["out"] = to_host(out)
+    r["device_error"] = err
+    r["launches"] = moe.moe_last_launch_count()
+    return r
+
+
+def bf16_half_ulp(v: np.ndarray) -> np.ndarray:
+    """Half the spacing of bf16 values around |v| (8 significant bits)."""
+    a = np.abs(v)
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -126)))
+    return 2.0 ** (e - 8)
+
+
+def check_out(got: np.ndarray, ref: np.ndarray, layer_bf16: bool, out_bf16: bool, what=""):
+    """Assert the output tolerances; returns (max_abs, rel_l2)."""
+    g = as_f64(got)
+    diff = np.abs(g - ref)
+    max_abs = float(diff.max()) if diff.size else 0.0
+    rel = float(np.linalg.norm(g - ref) / max(np.linalg.norm(ref), 1e-30)) if diff.size else 0.0
+    if not layer_bf16:
+        assert max_abs <= FP32_ATOL, f"{what}: fp32 max-abs {max_abs}"
+    elif not out_bf16:
+        assert max_abs <= BF16_ATOL, f"{what}: max-abs {max_abs}"
+        assert rel <= BF16_REL_L2, f"{what}: rel-L2 {rel}"
+    else:
+        tol = BF16_ATOL + bf16_half_ulp(ref)
+        bad = diff > tol
+        assert not bad.any(), f"{what}: {bad.sum()} elements beyond 2e-2 + half ulp (max {max_abs})"
+        assert rel <= BF16_REL_L2, f"{what}: rel-L2 {rel}"
+    return max_abs, rel
