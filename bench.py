@@ -1,0 +1,524 @@
+"""Benchmark of the MoE-layer forward pass on B200: tokens/s, roofline fraction, oracle baseline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 2] [--impl ours|reference]
+
+A step is one moe_layer_forward (router, dispatch, expert GEMMs, combine) over the workload's T
+tokens of seeded synthetic input already resident in HBM. L2 is flushed (256 MiB write) between
+timed steps; each step is timed with CUDA events on the launching stream; the K-step region is
+bracketed by a barrier and device synchronisation on both sides; the max over ranks is taken.
+N > 1 (under torchrun) runs N independent replicas, one per GPU: the layer has no exchange step
+on one GPU's worth of tokens, so `value` is N * T / (max-over-ranks time per step).
+
+Also measured: each kernel's share (decomposed entry points timed with events), the roofline of
+the dominant kernel (algorithmic bytes or FLOPs per launch / its event-timed duration, against
+MEASURED_PEAKS.json), the end-to-end throughput through the public API with pinned host buffers
+(H2D of x and D2H of the output inside the timed region), SM clocks and throttle reasons sampled
+through NVML during the timed region, and the CPU oracle's throughput on a bounded sample.
+
+--impl reference times the CPU oracle (the only reference implementation of this method) on a
+bounded sample per step and prints the same JSON line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "MoE-layer forward tokens/sec on 1 B200; % of bf16 tensor peak / % of HBM BW"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ---------------------------------------------------------------- distributed plumbing
+
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = False
+
+    def init(self, device):
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            dist.init_process_group("nccl", device_id=device, timeout=datetime.timedelta(seconds=300))
+            self.pg = True
+
+    def barrier(self):
+        if self.pg:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max(self, v: float, device) -> float:
+        if not self.pg:
+            return v
+        import torch.distributed as dist
+        t = torch.tensor([v], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------- clocks (NVML, read-only)
+
+class ClockSampler:
+    """Samples SM clock, max SM clock, power and clock-event reasons every ~2 ms in a thread."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.h = None
+            try:  # the CUDA device's UUID names the same GPU in NVML whatever the visibility mask
+                u = str(torch.cuda.get_device_properties(device_index).uuid)
+                u = u if u.startswith("GPU-") else "GPU-" + u
+                self.h = pynvml.nvmlDeviceGetHandleByUUID(u.encode())
+            except Exception:
+                self.h = None
+            if self.h is None:
+                vis = [v for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
+                ent = vis[device_index].strip() if device_index < len(vis) else str(device_index)
+                self.h = (pynvml.nvmlDeviceGetHandleByUUID(ent.encode()) if ent.startswith("GPU-")
+                          else pynvml.nvmlDeviceGetHandleByIndex(int(ent)))
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # NVML unavailable: report no clocks rather than guess
+            self.err = str(e)
+        self._stop = threading.Event()
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                try:
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except Exception:
+                    rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                self.samples.append((time.time(), sm, rs))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self) -> dict:
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "note": getattr(self, "err", "no samples")}
+        sms = [s[1] for s in self.samples]
+        mask = 0
+        for s in self.samples:
+            mask |= s[2]
+        reasons = [n for b, n in self.REASONS.items() if mask & b and n != "gpu_idle"]
+        return {"sm_mhz": float(statistics.median(sms)), "sm_max_mhz": float(self.max_mhz),
+                "reasons": reasons, "samples": len(sms), "source": "NVML during the timed region"}
+
+
+# ---------------------------------------------------------------- helpers
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def to_dev(a: np.ndarray, device):
+    if a is None:
+        return None
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).to(device).view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("grouped_gemm.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "mixture_experts_layer_57_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str, kernel: str):
+    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, if the kernel's source
+    is unchanged since it was taken (the summary records the source hash)."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.md")
+    if not os.path.exists(path):
+        return None, None
+    src = kernel_source_hash()
+    for line in open(path):
+        # | workload | kernel | source hash | dram bytes per launch | ...
+        cells = [c.strip() for c in line.strip().strip("|").split("|")]
+        if len(cells) >= 4 and cells[0] == workload and cells[1] == kernel and cells[2] == src:
+            try:
+                return float(cells[3]), path
+            except ValueError:
+                return None, None
+    return None, None
+
+
+# ---------------------------------------------------------------- CPU oracle timing
+
+def oracle_sample_rate(w: synth.Workload, inp: dict, n_tokens: int, full_logits=None):
+    """Oracle tokens/s on a sample: router logits of n tokens + routing/slots of all T tokens
+    (from given logits) + expert FFN and combine of the same n tokens. Single-threaded."""
+    import oracle
+    if full_logits is None:
+        full_logits = np.zeros((w.T, w.E), dtype=np.float32)
+    tok = np.arange(n_tokens, dtype=np.int64)
+    t0 = time.perf_counter()
+    oracle.router_logits(inp["x"][:n_tokens], inp["w_router"], inp.get("router_bias"))
+    oracle.layer_forward(inp, w.T, w.d_model, w.d_ff, w.E, w.k, w.capacity_factor,
+                         add_input_residual=w.add_input_residual, aux_alpha=w.aux_alpha,
+                         logits_in=full_logits, tokens=tok)
+    dt = time.perf_counter() - t0
+    return n_tokens / dt, dt
+
+
+def run_reference(args, dist: Dist):
+    """The reference arm: the CPU oracle, as it stands, on a bounded sample per step."""
+    if dist.rank != 0:
+        return 0
+    w = synth.WORKLOADS[args.workload]
+    if args.tokens:
+        w = w.with_(T=args.tokens, name=f"{w.name}-T{args.tokens}")
+    inp = synth.make_inputs(w)
+    # the GPU path's routing is not used here: the logits of all T tokens come from the oracle,
+    # computed once (outside the steps); each step then pays the router for its own tokens
+    import oracle
+    full_logits = oracle.router_logits(inp["x"], inp["w_router"], inp.get("router_bias"))
+    budget_s = 150.0 / max(1, args.steps + args.warmup)
+    per_token = oracle_sample_rate(w, inp, 2, full_logits)[1] / 2
+    n = int(max(2, min(256, budget_s / per_token)))
+    times = []
+    for i in range(args.warmup + args.steps):
+        _, dt = oracle_sample_rate(w, inp, n, full_logits)
+        if i >= args.warmup:
+            times.append(dt)
+    ms = 1e3 * float(np.mean(times))
+    value = n / (ms / 1e3)
+    sample = (f"{n} tokens per step (router logits, routing and slots of all {w.T} tokens from "
+              f"their logits, expert FFN and combine of the {n}), single-threaded C++ oracle")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step_sample": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(w, args.gpus),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w: synth.Workload, n_gpus: int) -> dict:
+    return {"workload": f"{w.name}: {w.description}", "T": w.T, "d_model": w.d_model,
+            "d_ff": w.d_ff, "E": w.E, "k": w.k, "capacity_factor": w.capacity_factor,
+            "dense_branch": w.dense, "global_batch_tokens": w.T * n_gpus,
+            "parallelism": f"replicas x{n_gpus}" if n_gpus > 1 else "single GPU",
+            "l2": "flushed between timed steps (256 MiB write)", "seed": w.seed}
+
+
+# ---------------------------------------------------------------- the GPU arm
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", type=int, default=2, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="run the workload with T tokens instead of its own (profiling captures)")
+    args = ap.parse_args()
+    dist = Dist()
+    if args.gpus != dist.world and dist.world > 1:
+        print(f"--gpus {args.gpus} but WORLD_SIZE {dist.world}", file=sys.stderr)
+    if args.gpus > 1 and dist.world == 1:
+        print("N > 1 runs one process per GPU: launch with torchrun", file=sys.stderr)
+        return 2
+    if args.impl == "reference":
+        return run_reference(args, dist)
+
+    from mixture_experts_layer_57_b200 import moe
+
+    device = torch.device("cuda", dist.local_rank)
+    torch.cuda.set_device(device)
+    dist.init(device)
+    w = synth.WORKLOADS[args.workload]
+    if args.tokens:
+        w = w.with_(T=args.tokens, name=f"{w.name}-T{args.tokens}")
+    inp = synth.make_inputs(w)
+    d = {k: to_dev(v, device) for k, v in inp.items()}
+    T, E, k, dm, df = w.T, w.E, w.k, w.d_model, w.d_ff
+    bf16 = w.dtype == "bf16"
+    dense = (d["dense_w1"], d["dense_b1"], d["dense_w2"], d["dense_b2"]) if w.dense else None
+    args_c = moe.layer_args(d["x"], d["w_router"], d["w1"], d["b1"], d["w2"], d["b2"], k=k,
+                            capacity_factor=w.capacity_factor, router_bias=d.get("router_bias"),
+                            dense=dense, add_input_residual=w.add_input_residual,
+                            aux_alpha=w.aux_alpha)
+    ws = moe.workspace(moe.moe_layer_workspace_bytes(args_c), device)
+    out = torch.empty(T, dm, dtype=d["x"].dtype, device=device)
+    aux = dict(expert_offsets=torch.empty(E + 1, dtype=torch.int32, device=device),
+               expert_counts=torch.empty(E, dtype=torch.int32, device=device),
+               lb_stats=torch.empty(2 * E + 1, dtype=torch.float32, device=device))
+    flush_buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        moe.moe_layer_forward(args_c, out, aux=aux, ws=ws, stream=stream)
+
+    # ---------------------------------------------------------- timed region
+    for _ in range(args.warmup):
+        flush_buf.zero_()
+        step()
+    torch.cuda.synchronize()
+    launches_per_step = moe.moe_last_launch_count()
+    clocks = ClockSampler(dist.local_rank)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    for i in range(args.steps):
+        flush_buf.zero_()
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    ms_local = float(np.mean(step_ms))
+    ms = dist.max(ms_local, device)
+    assert moe.moe_get_device_error(ws) == 0, "device error during the timed steps"
+    value = args.gpus * T / (ms / 1e3)
+
+    # ---------------------------------------------------------- routing statistics
+    off = aux["expert_offsets"].cpu().numpy()
+    counts = aux["expert_counts"].cpu().numpy()
+    kept = off[1:] - off[:-1]
+    R = int(off[-1])
+    E_t = int((kept > 0).sum())
+    lb = aux["lb_stats"].cpu().numpy()
+    routing = {"kept_rows": R, "pairs": T * k, "drop_rate": 1.0 - R / (T * k),
+               "experts_touched": E_t, "max_expert_demand": int(counts.max()),
+               "capacity": moe.moe_capacity(T, E, k, w.capacity_factor), "aux_loss": float(lb[-1])}
+
+    # ---------------------------------------------------------- per-kernel breakdown
+    bd = breakdown(moe, w, d, ws, stream, flush_buf, reps=max(3, min(20, args.steps)))
+    es = 2 if bf16 else 4
+    gemm_bytes = {
+        "gemm1": E_t * df * dm * es + E_t * df * es + R * dm * es + R * df * es,
+        "gemm2": E_t * dm * df * es + E_t * dm * es + R * df * es + R * dm * 4,
+    }
+    gemm_flops = {"gemm1": 2.0 * R * dm * df, "gemm2": 2.0 * R * dm * df}
+    if w.dense:
+        gemm_bytes["dense_gemm1"] = df * dm * es + df * es + T * dm * es + T * df * es
+        gemm_bytes["dense_gemm2"] = dm * df * es + dm * es + T * df * es + T * dm * 4
+        gemm_flops["dense_gemm1"] = gemm_flops["dense_gemm2"] = 2.0 * T * dm * df
+    peaks, peak_src = load_peaks()
+    dom = max((n for n in bd if n in gemm_bytes), key=lambda n: bd[n])
+    t_dom = bd[dom] / 1e3
+    ai = gemm_flops[dom] / gemm_bytes[dom]
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    kernel_name = {"gemm1": "grouped_gemm (layer 1, bias+GeLU epilogue)",
+                   "gemm2": "grouped_gemm (layer 2, bias epilogue)",
+                   "dense_gemm1": "dense MLP layer 1", "dense_gemm2": "dense MLP layer 2"}[dom]
+    traffic, _ = profiled_traffic(w.name, dom)
+    if ai < ridge:
+        roof = {"kernel": kernel_name, "bound": "hbm", "achieved": gemm_bytes[dom] / t_dom / 1e9,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    else:
+        roof = {"kernel": kernel_name, "bound": "tensor", "achieved": gemm_flops[dom] / t_dom / 1e12,
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = traffic
+    roof["algorithmic_bytes"] = gemm_bytes[dom]
+    roof["algorithmic_flops"] = gemm_flops[dom]
+    roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
+    roof["tensor_frac"] = gemm_flops[dom] / t_dom / 1e12 / peaks["bf16_tflops"]
+    roof["hbm_frac"] = gemm_bytes[dom] / t_dom / 1e9 / peaks["hbm_gbs"]
+
+    # ---------------------------------------------------------- end to end through the API
+    e2e = None
+    if not args.skip_e2e:
+        e2e = end_to_end(moe, args_c, d, w, ws, stream, args, dist, device)
+
+    # ---------------------------------------------------------- CPU oracle baseline
+    cpu = None
+    if dist.rank == 0 and dist.world == 1 and not args.skip_cpu_baseline:
+        logits = torch.empty(T, E, dtype=torch.float32, device=device)
+        moe.moe_router_topk(d["x"], d["w_router"], k, router_bias=d.get("router_bias"), logits=logits)
+        full_logits = logits.cpu().numpy()
+        per_tok = oracle_sample_rate(w, inp, 2, full_logits)[1] / 2
+        n = int(max(8, min(2048, 12.0 / per_tok)))
+        rate, dt = oracle_sample_rate(w, inp, n, full_logits)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+               "sample": f"{n} tokens ({dt:.1f} s): their router logits, routing and slots of all "
+                         f"{T} tokens from given logits, expert FFN and combine of the {n}; "
+                         "single-threaded C++ oracle in double"}
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if bf16 else "f32",
+            "data": "synthetic (seeded splitmix64 + Box-Muller, shapes and distributions of the workload)",
+            "config": workload_config(w, args.gpus), "roofline": roof, "cpu_baseline": cpu,
+            "clocks": clocks.summary(), "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps,
+            "breakdown_ms": bd, "routing": routing,
+            "step_ms": {"min": float(min(step_ms)), "median": float(np.median(step_ms)),
+                        "max": float(max(step_ms))}}
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.close()
+    return 0
+
+
+def breakdown(moe, w, d, ws_layer, stream, flush_buf, reps: int) -> dict:
+    """Median event time (ms) of each entry point of the pipeline, run one by one as the layer
+    forward runs them (same kernels, same order)."""
+    dev = d["x"].device
+    T, E, k, dm, df = w.T, w.E, w.k, w.d_model, w.d_ff
+    C = moe.moe_capacity(T, E, k, w.capacity_factor)
+    R = moe.moe_packed_rows_max(T, E, k, C)
+    logits = torch.empty(T, E, dtype=torch.float32, device=dev)
+    ids = torch.empty(T, k, dtype=torch.int32, device=dev)
+    gates = torch.empty(T, k, dtype=torch.float32, device=dev)
+    lb = torch.empty(2 * E + 1, dtype=torch.float32, device=dev)
+    ws_r = moe.workspace(moe.moe_router_workspace_bytes(T, E), dev)
+    ws_d = moe.workspace(moe.moe_dispatch_workspace_bytes(T, E, k), dev)
+    ws_s = moe.workspace(256, dev)
+    slot = torch.empty(T, k, dtype=torch.int32, device=dev)
+    cnt = torch.empty(E, dtype=torch.int32, device=dev)
+    off = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    rt = torch.empty(max(R, 1), dtype=torch.int32, device=dev)
+    xp = torch.empty(max(R, 1), dm, dtype=d["x"].dtype, device=dev)
+    hp = torch.empty(max(R, 1), df, dtype=d["x"].dtype, device=dev)
+    yp = torch.empty(max(R, 1), dm, dtype=torch.float32, device=dev)
+    out = torch.empty(T, dm, dtype=d["x"].dtype, device=dev)
+    dense_on = w.dense
+    if dense_on:
+        hd = torch.empty(T, df, dtype=d["x"].dtype, device=dev)
+        rd = torch.empty(T, dm, dtype=torch.float32, device=dev)
+        one_seg = torch.tensor([0, T], dtype=torch.int32, device=dev)
+
+    stages = [
+        ("router", lambda: moe.moe_router_topk(d["x"], d["w_router"], k, router_bias=d.get("router_bias"),
+                                               logits=logits, expert_ids=ids, gates=gates, lb_stats=lb,
+                                               aux_alpha=w.aux_alpha, ws=ws_r, stream=stream)),
+        ("dispatch", lambda: moe.moe_dispatch(d["x"], ids, E, C, rows_max=R, slot=slot, expert_counts=cnt,
+                                              expert_offsets=off, row_token=rt, x_packed=xp, ws=ws_d,
+                                              stream=stream)),
+    ]
+    if dense_on:
+        stages += [
+            ("dense_gemm1", lambda: moe.moe_grouped_gemm(d["x"], one_seg, d["dense_w1"][None], d["dense_b1"][None],
+                                                         gelu=True, rows_max=T, capacity_hint=T, out=hd,
+                                                         ws=ws_s, stream=stream)),
+            ("dense_gemm2", lambda: moe.moe_grouped_gemm(hd, one_seg, d["dense_w2"][None], d["dense_b2"][None],
+                                                         gelu=False, rows_max=T, capacity_hint=T, out=rd,
+                                                         ws=ws_s, stream=stream)),
+        ]
+    stages += [
+        ("gemm1", lambda: moe.moe_grouped_gemm(xp, off, d["w1"], d["b1"], gelu=True, rows_max=R,
+                                               capacity_hint=C, out=hp, ws=ws_s, stream=stream)),
+        ("gemm2", lambda: moe.moe_grouped_gemm(hp, off, d["w2"], d["b2"], gelu=False, rows_max=R,
+                                               capacity_hint=C, out=yp, ws=ws_s, stream=stream)),
+        ("combine", lambda: moe.moe_combine(yp, off, ids, slot, gates,
+                                            residual=d["x"] if w.add_input_residual else None,
+                                            dense=rd if dense_on else None, out=out, rows_max=R,
+                                            ws=ws_s, stream=stream)),
+    ]
+    times = {n: [] for n, _ in stages}
+    for _ in range(reps):
+        flush_buf.zero_()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)]
+        ev[0].record(stream)
+        for i, (_, fn) in enumerate(stages):
+            fn()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+        for i, (n, _) in enumerate(stages):
+            times[n].append(ev[i].elapsed_time(ev[i + 1]))
+    assert moe.moe_get_device_error(ws_s) == 0
+    return {n: float(np.median(v)) for n, v in times.items()}
+
+
+def end_to_end(moe, args_c, d, w, ws, stream, args, dist, device) -> dict:
+    """Same metric through the public call with host buffers: per step H2D of x from pinned
+    memory, moe_layer_forward, D2H of the output into pinned memory, all inside the events."""
+    T, dm = w.T, w.d_model
+    x_dev = d["x"]
+    x_pin = torch.empty(x_dev.shape, dtype=x_dev.dtype, pin_memory=True)
+    x_pin.copy_(x_dev.cpu())
+    out_dev = torch.empty(T, dm, dtype=x_dev.dtype, device=device)
+    out_pin = torch.empty(T, dm, dtype=x_dev.dtype, pin_memory=True)
+
+    def step():
+        x_dev.copy_(x_pin, non_blocking=True)
+        moe.moe_layer_forward(args_c, out_dev, ws=ws, stream=stream)
+        out_pin.copy_(out_dev, non_blocking=True)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    n = max(3, min(args.steps, 50))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(n):
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    ms = dist.max(float(np.mean([a.elapsed_time(b) for a, b in evs])), device)
+    es = x_dev.element_size()
+    return {"value": args.gpus * T / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms, "steps": n,
+            "h2d_bytes_per_step": T * dm * es, "d2h_bytes_per_step": T * dm * out_pin.element_size()}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -150,6 +150,18 @@ moe_status moe_expert_ffn(const void* x_packed, const int32_t* expert_offsets, i
                           float* y_packed, int64_t capacity_hint, void* ws, size_t ws_bytes,
                           moe_stream_t stream);
 
+/* One layer of the grouped expert GEMM (a single kernel launch):
+ *     out[r, :] = act(W[e] x_packed[r, :] + bias[e])   for r in [expert_offsets[e], expert_offsets[e+1])
+ * w: [E, N, K] in dtype, bias: [E, N] in dtype or NULL, x_packed: [rows_max, K] in dtype.
+ * MOE_EPILOGUE_BIAS_GELU writes out [rows_max, N] in dtype (bf16 rounds GeLU(z));
+ * MOE_EPILOGUE_BIAS writes out [rows_max, N] in fp32. moe_expert_ffn is this entry twice
+ * (K=d_model, N=d_ff with GeLU; then K=d_ff, N=d_model). Same limits as moe_expert_ffn. */
+typedef enum { MOE_EPILOGUE_BIAS_GELU = 0, MOE_EPILOGUE_BIAS = 1 } moe_epilogue;
+moe_status moe_grouped_gemm(const void* x_packed, const int32_t* expert_offsets, int E,
+                            int64_t rows_max, int K, int N, moe_dtype dtype, const void* w,
+                            const void* bias, moe_epilogue epilogue, void* out,
+                            int64_t capacity_hint, void* ws, size_t ws_bytes, moe_stream_t stream);
+
 /* ---------------------------------------------------------------- combine
  * out[t,:] = [residual[t,:]] + [dense[t,:]] + sum_{j : slot[t,j] >= 0} gates[t,j] *
  *            y_packed[expert_offsets[expert_ids[t,j]] + slot[t,j], :]

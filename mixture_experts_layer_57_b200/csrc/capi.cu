@@ -259,6 +259,31 @@ moe_status moe_expert_ffn(const void* x_packed, const int32_t* expert_offsets, i
                                             y_packed, (int*)ws, stream));
 }
 
+moe_status moe_grouped_gemm(const void* x_packed, const int32_t* expert_offsets, int E,
+                            int64_t rows_max, int K, int N, moe_dtype dtype, const void* w,
+                            const void* bias, moe_epilogue epilogue, void* out,
+                            int64_t capacity_hint, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = check_ffn_shape(E, rows_max, K, N, dtype);
+  if (st != MOE_OK) return st;
+  if (epilogue != MOE_EPILOGUE_BIAS_GELU && epilogue != MOE_EPILOGUE_BIAS)
+    return MOE_ERR_INVALID_ARGUMENT;
+  if (capacity_hint < 0 || !expert_offsets || !w || !ws) return MOE_ERR_INVALID_ARGUMENT;
+  if (rows_max > 0 && (!x_packed || !out)) return MOE_ERR_INVALID_ARGUMENT;
+  if (!aligned16(x_packed) || !aligned16(expert_offsets) || !aligned16(w) || !aligned16(bias) ||
+      !aligned16(out) || ((uintptr_t)ws % kAlign) != 0)
+    return MOE_ERR_MISALIGNED;
+  if (ws_bytes < kAlign) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (fault_injected("moe_grouped_gemm")) return MOE_ERR_CUDA;
+  g_launches = 0;
+  const bool gelu = epilogue == MOE_EPILOGUE_BIAS_GELU;
+  if (dtype == MOE_BF16)
+    return cuda_status(enqueue_grouped_gemm_bf16(x_packed, expert_offsets, E, rows_max, K, N, w,
+                                                 bias, gelu, out, capacity_hint, (int*)ws, stream));
+  return cuda_status(enqueue_grouped_gemm_f32((const float*)x_packed, expert_offsets, E, rows_max,
+                                              K, N, (const float*)w, (const float*)bias, gelu,
+                                              (float*)out, (int*)ws, stream));
+}
+
 // ---------------------------------------------------------------- combine
 
 moe_status moe_combine_workspace_bytes(size_t* bytes) {

@@ -50,32 +50,41 @@ __global__ void __launch_bounds__(kFeat)
 
 }  // namespace
 
+cudaError_t enqueue_grouped_gemm_f32(const float* x, const int32_t* offsets, int E,
+                                     int64_t rows_max, int K, int N, const float* w,
+                                     const float* bias, bool gelu, float* out, int* status,
+                                     cudaStream_t stream) {
+  if (rows_max == 0) return cudaSuccess;
+  const unsigned gx = (unsigned)(rows_max < 65536 ? rows_max : 65536);
+  const size_t smem = (size_t)K * sizeof(float);
+  static size_t attr_done[2] = {48 * 1024, 48 * 1024};
+  if (smem > attr_done[gelu]) {
+    cudaError_t e = cudaFuncSetAttribute(gelu ? ffn_f32_kernel<true> : ffn_f32_kernel<false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr_done[gelu] = smem;
+  }
+  const dim3 grid(gx, (N + kFeat - 1) / kFeat);
+  if (gelu)
+    ffn_f32_kernel<true><<<grid, kFeat, smem, stream>>>(x, offsets, E, N, K, rows_max, w, bias, out,
+                                                        status);
+  else
+    ffn_f32_kernel<false><<<grid, kFeat, smem, stream>>>(x, offsets, E, N, K, rows_max, w, bias, out,
+                                                         status);
+  count_launch();
+  return cudaGetLastError();
+}
+
 cudaError_t enqueue_expert_ffn_f32(const float* x_packed, const int32_t* offsets, int E,
                                    int64_t rows_max, int d, int d_ff, const float* w1,
                                    const float* b1, const float* w2, const float* b2,
                                    float* h_packed, float* y_packed, int* status,
                                    cudaStream_t stream) {
-  if (rows_max == 0) return cudaSuccess;
-  const unsigned gx = (unsigned)(rows_max < 65536 ? rows_max : 65536);
-  const size_t smem1 = (size_t)d * sizeof(float), smem2 = (size_t)d_ff * sizeof(float);
-  const size_t smem_max = smem1 > smem2 ? smem1 : smem2;
-  static size_t attr_done = 0;
-  if (smem_max > 48 * 1024 && attr_done < smem_max) {
-    cudaError_t e1 = cudaFuncSetAttribute(ffn_f32_kernel<true>,
-                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max);
-    cudaError_t e2 = cudaFuncSetAttribute(ffn_f32_kernel<false>,
-                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max);
-    if (e1 != cudaSuccess) return e1;
-    if (e2 != cudaSuccess) return e2;
-    attr_done = smem_max;
-  }
-  ffn_f32_kernel<true><<<dim3(gx, (d_ff + kFeat - 1) / kFeat), kFeat, smem1, stream>>>(
-      x_packed, offsets, E, d_ff, d, rows_max, w1, b1, h_packed, status);
-  count_launch();
-  ffn_f32_kernel<false><<<dim3(gx, (d + kFeat - 1) / kFeat), kFeat, smem2, stream>>>(
-      h_packed, offsets, E, d, d_ff, rows_max, w2, b2, y_packed, status);
-  count_launch();
-  return cudaGetLastError();
+  cudaError_t e = enqueue_grouped_gemm_f32(x_packed, offsets, E, rows_max, d, d_ff, w1, b1, true,
+                                           h_packed, status, stream);
+  if (e != cudaSuccess) return e;
+  return enqueue_grouped_gemm_f32(h_packed, offsets, E, rows_max, d_ff, d, w2, b2, false, y_packed,
+                                  status, stream);
 }
 
 }  // namespace moe

@@ -374,44 +374,52 @@ cudaError_t launch_one(const CUtensorMap& tmW, const CUtensorMap& tmX, const Par
   return cudaGetLastError();
 }
 
-template <int BN>
-cudaError_t launch_pair(const CUtensorMap& tmW1, const CUtensorMap& tmX, const CUtensorMap& tmW2,
-                        const CUtensorMap& tmH, const Params& p1, const Params& p2,
-                        cudaStream_t stream) {
-  cudaError_t e = launch_one<BN, true>(tmW1, tmX, p1, stream);
-  if (e != cudaSuccess) return e;
-  return launch_one<BN, false>(tmW2, tmH, p2, stream);
+}  // namespace
+
+static int pick_token_tile(int64_t capacity_hint) {
+  if (capacity_hint <= 16) return 16;
+  if (capacity_hint <= 32) return 32;
+  if (capacity_hint <= 64) return 64;
+  if (capacity_hint <= 128) return 128;
+  return 256;
 }
 
-}  // namespace
+cudaError_t enqueue_grouped_gemm_bf16(const void* x, const int32_t* offsets, int E,
+                                      int64_t rows_max, int K, int N, const void* w,
+                                      const void* bias, bool gelu, void* out,
+                                      int64_t capacity_hint, int* status, cudaStream_t stream) {
+  if (rows_max == 0) return cudaSuccess;
+  const int BN = pick_token_tile(capacity_hint);
+  CUtensorMap tmW, tmX;
+  if (!make_kmajor_map(&tmW, w, (int64_t)E * N, K, kBM) || !make_kmajor_map(&tmX, x, rows_max, K, BN))
+    return cudaErrorInvalidValue;
+  const Params p{offsets, E, N, K, rows_max, (const uint16_t*)bias, out, status};
+#define MOE_GG_CASE(BNV)                                                          \
+  case BNV:                                                                      \
+    return gelu ? launch_one<BNV, true>(tmW, tmX, p, stream)                      \
+                : launch_one<BNV, false>(tmW, tmX, p, stream);
+  switch (BN) {
+    MOE_GG_CASE(16)
+    MOE_GG_CASE(32)
+    MOE_GG_CASE(64)
+    MOE_GG_CASE(128)
+    default:
+      return gelu ? launch_one<256, true>(tmW, tmX, p, stream)
+                  : launch_one<256, false>(tmW, tmX, p, stream);
+  }
+#undef MOE_GG_CASE
+}
 
 cudaError_t enqueue_expert_ffn_bf16(const void* x_packed, const int32_t* offsets, int E,
                                     int64_t rows_max, int d, int d_ff, const void* w1,
                                     const void* b1, const void* w2, const void* b2, void* h_packed,
                                     float* y_packed, int64_t capacity_hint, int* status,
                                     cudaStream_t stream) {
-  int BN = 256;
-  if (capacity_hint <= 16) BN = 16;
-  else if (capacity_hint <= 32) BN = 32;
-  else if (capacity_hint <= 64) BN = 64;
-  else if (capacity_hint <= 128) BN = 128;
-
-  CUtensorMap tmW1, tmX, tmW2, tmH;
-  if (!make_kmajor_map(&tmW1, w1, (int64_t)E * d_ff, d, kBM) ||
-      !make_kmajor_map(&tmX, x_packed, rows_max, d, BN) ||
-      !make_kmajor_map(&tmW2, w2, (int64_t)E * d, d_ff, kBM) ||
-      !make_kmajor_map(&tmH, h_packed, rows_max, d_ff, BN))
-    return cudaErrorInvalidValue;
-
-  Params p1{offsets, E, d_ff, d, rows_max, (const uint16_t*)b1, h_packed, status};
-  Params p2{offsets, E, d, d_ff, rows_max, (const uint16_t*)b2, y_packed, status};
-  switch (BN) {
-    case 16: return launch_pair<16>(tmW1, tmX, tmW2, tmH, p1, p2, stream);
-    case 32: return launch_pair<32>(tmW1, tmX, tmW2, tmH, p1, p2, stream);
-    case 64: return launch_pair<64>(tmW1, tmX, tmW2, tmH, p1, p2, stream);
-    case 128: return launch_pair<128>(tmW1, tmX, tmW2, tmH, p1, p2, stream);
-    default: return launch_pair<256>(tmW1, tmX, tmW2, tmH, p1, p2, stream);
-  }
+  cudaError_t e = enqueue_grouped_gemm_bf16(x_packed, offsets, E, rows_max, d, d_ff, w1, b1, true,
+                                            h_packed, capacity_hint, status, stream);
+  if (e != cudaSuccess) return e;
+  return enqueue_grouped_gemm_bf16(h_packed, offsets, E, rows_max, d_ff, d, w2, b2, false, y_packed,
+                                   capacity_hint, status, stream);
 }
 
 }  // namespace moe

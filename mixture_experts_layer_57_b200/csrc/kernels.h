@@ -37,6 +37,17 @@ cudaError_t enqueue_dispatch(const void* x, bool bf16, int64_t T, int d, const i
                              int* status, cudaStream_t stream);
 
 // ---------------------------------------------------------------- expert FFN
+// One grouped GEMM layer: out = act(W[e] x + bias[e]) over every expert segment. offsets ==
+// nullptr means one segment [0, rows_max) (E must be 1). gelu: GeLU epilogue with output in the
+// input type; otherwise bias only with fp32 output.
+cudaError_t enqueue_grouped_gemm_bf16(const void* x, const int32_t* offsets, int E,
+                                      int64_t rows_max, int K, int N, const void* w,
+                                      const void* bias, bool gelu, void* out,
+                                      int64_t capacity_hint, int* status, cudaStream_t stream);
+cudaError_t enqueue_grouped_gemm_f32(const float* x, const int32_t* offsets, int E,
+                                     int64_t rows_max, int K, int N, const float* w,
+                                     const float* bias, bool gelu, float* out, int* status,
+                                     cudaStream_t stream);
 cudaError_t enqueue_expert_ffn_bf16(const void* x_packed, const int32_t* offsets, int E,
                                     int64_t rows_max, int d, int d_ff, const void* w1,
                                     const void* b1, const void* w2, const void* b2, void* h_packed,

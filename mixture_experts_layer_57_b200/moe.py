@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_PKG, "libmoe.so")
 HEADER = os.path.join(os.path.dirname(_PKG), "include", "moe.h")
 
 MOE_F32, MOE_BF16 = 0, 1
+MOE_EPILOGUE_BIAS_GELU, MOE_EPILOGUE_BIAS = 0, 1
 STATUS_BLOCK_BYTES = 256
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARGUMENT", 2: "MOE_ERR_UNSUPPORTED",
                 3: "MOE_ERR_WORKSPACE_TOO_SMALL", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_FLAG",
@@ -78,6 +79,7 @@ def lib() -> ctypes.CDLL:
             "moe_dispatch": ([vp, i32, i64, i32, vp, i32, i32, i64, vp, vp, vp, vp, vp, i64, vp, sz, vp], i32),
             "moe_expert_ffn_workspace_bytes": ([P(sz)], i32),
             "moe_expert_ffn": ([vp, vp, i32, i64, i32, i32, i32, vp, vp, vp, vp, vp, vp, i64, vp, sz, vp], i32),
+            "moe_grouped_gemm": ([vp, vp, i32, i64, i32, i32, i32, vp, vp, i32, vp, i64, vp, sz, vp], i32),
             "moe_combine_workspace_bytes": ([P(sz)], i32),
             "moe_combine": ([vp, vp, vp, vp, vp, i64, i32, i32, i32, i64, vp, i32, vp, vp, i32, vp, sz, vp], i32),
             "moe_layer_workspace_bytes": ([P(LayerArgs), P(sz)], i32),
@@ -245,6 +247,28 @@ def moe_expert_ffn(x_packed: torch.Tensor, expert_offsets: torch.Tensor, w1, b1,
         _ptr(w2), _ptr(b2), _ptr(h_packed), _ptr(y_packed), capacity_hint, _ptr(ws), ws.numel(),
         _stream(stream)))
     return dict(h_packed=h_packed, y_packed=y_packed, ws=ws)
+
+
+def moe_grouped_gemm(x_packed: torch.Tensor, expert_offsets: torch.Tensor, w: torch.Tensor, bias=None,
+                     gelu: bool = True, rows_max=None, capacity_hint=None, out=None, ws=None,
+                     stream=None) -> dict:
+    """One grouped GEMM layer: out = GeLU(W[e] x + b[e]) (input dtype) or W[e] x + b[e] (fp32)."""
+    E, N, K = w.shape
+    dev = x_packed.device
+    if rows_max is None:
+        rows_max = x_packed.shape[0]
+    if capacity_hint is None:
+        capacity_hint = rows_max
+    if out is None:
+        out = torch.empty(max(rows_max, 1), N, dtype=x_packed.dtype if gelu else torch.float32,
+                          device=dev)
+    if ws is None:
+        ws = workspace(moe_expert_ffn_workspace_bytes(), dev)
+    _check("moe_grouped_gemm", lib().moe_grouped_gemm(
+        _ptr(x_packed), _ptr(expert_offsets), E, rows_max, K, N, _dt(x_packed), _ptr(w), _ptr(bias),
+        MOE_EPILOGUE_BIAS_GELU if gelu else MOE_EPILOGUE_BIAS, _ptr(out), capacity_hint, _ptr(ws),
+        ws.numel(), _stream(stream)))
+    return dict(out=out, ws=ws)
 
 
 def moe_combine(y_packed: torch.Tensor, expert_offsets, expert_ids, slot, gates, residual=None,
