@@ -130,6 +130,27 @@ moe_status moe_dispatch(const void* x, moe_dtype dtype, int64_t T, int d_model,
                         void* x_packed, int64_t rows_max, void* ws, size_t ws_bytes,
                         moe_stream_t stream);
 
+/* Allocation-free variant of moe_dispatch (no counterpart on the pages: it exists for callers).
+ * Some callers cannot allocate device memory at all: a plug-in running inside a host application
+ * that owns every device buffer and offers no allocation hook, or a latency-critical serving loop
+ * that must never call cudaMalloc/cudaFree because they can block and synchronise the device.
+ * Such a caller passes only its inputs and outputs; the dispatch scratch (per-pair ranks and
+ * per-segment counts and bases: align256(4*T*k) + 2*align256(4*ceil(T*k/256)*E) bytes) comes
+ * from one static device array of MOE_NOALLOC_SCRATCH_BYTES (4 MiB) that every GPU loading the
+ * library holds until the process exits. Larger problems return MOE_ERR_WORKSPACE_TOO_SMALL
+ * (use moe_dispatch with a workspace instead). Arguments, outputs and results are those of
+ * moe_dispatch, except that no status block exists: ids outside [0, E) become dropped pairs
+ * without a device error code. The first call on each device (with that device current) looks
+ * up the array's device address; make that first call before any stream capture begins.
+ * Nothing in the array needs to start at zero (every element read is written first in the same
+ * call), but all calls share it: calls that overlap on the GPU race and must be serialised. */
+#define MOE_NOALLOC_SCRATCH_BYTES (4u << 20)
+moe_status moe_dispatch_noalloc(const void* x, moe_dtype dtype, int64_t T, int d_model,
+                                const int32_t* expert_ids, int E, int k, int64_t C, int32_t* slot,
+                                int32_t* expert_counts, int32_t* expert_offsets,
+                                int32_t* row_token, void* x_packed, int64_t rows_max,
+                                moe_stream_t stream);
+
 /* ---------------------------------------------------------------- expert FFN
  * For every expert e and every packed row r in [expert_offsets[e], expert_offsets[e+1]):
  *     h[r,:] = GeLU(W1[e] x_packed[r,:] + b1[e])        GeLU(z) = 0.5 z (1 + erf(z / sqrt 2))

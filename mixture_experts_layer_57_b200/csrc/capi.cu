@@ -14,6 +14,7 @@ thread_local int g_launches = 0;
 }
 
 void count_launch() { ++g_launches; }
+void reset_launch_count() { g_launches = 0; }
 
 int num_sms() {
   static int cache[64] = {0};

@@ -11,6 +11,7 @@ namespace moe {
 
 // Incremented once per kernel launch on the calling host thread (reset by every entry point).
 void count_launch();
+void reset_launch_count();
 
 // Number of SMs of the current device (cached per device).
 int num_sms();

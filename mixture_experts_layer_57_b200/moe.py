@@ -77,6 +77,7 @@ def lib() -> ctypes.CDLL:
             "moe_router_topk": ([vp, i32, i64, i32, vp, vp, i32, i32, vp, vp, vp, vp, f32, vp, sz, vp], i32),
             "moe_dispatch_workspace_bytes": ([i64, i32, i32, P(sz)], i32),
             "moe_dispatch": ([vp, i32, i64, i32, vp, i32, i32, i64, vp, vp, vp, vp, vp, i64, vp, sz, vp], i32),
+            "moe_dispatch_noalloc": ([vp, i32, i64, i32, vp, i32, i32, i64, vp, vp, vp, vp, vp, i64, vp], i32),
             "moe_expert_ffn_workspace_bytes": ([P(sz)], i32),
             "moe_expert_ffn": ([vp, vp, i32, i64, i32, i32, i32, vp, vp, vp, vp, vp, vp, i64, vp, sz, vp], i32),
             "moe_grouped_gemm": ([vp, vp, i32, i64, i32, i32, i32, vp, vp, i32, vp, i64, vp, sz, vp], i32),
@@ -225,6 +226,33 @@ def moe_dispatch(x: torch.Tensor, expert_ids: torch.Tensor, E: int, C: int, rows
         _stream(stream)))
     return dict(slot=slot, expert_counts=expert_counts, expert_offsets=expert_offsets,
                 row_token=row_token, x_packed=x_packed, rows_max=rows_max, ws=ws)
+
+
+def moe_dispatch_noalloc(x: torch.Tensor, expert_ids: torch.Tensor, E: int, C: int, rows_max=None,
+                         slot=None, expert_counts=None, expert_offsets=None, row_token=None,
+                         x_packed=None, stream=None) -> dict:
+    """moe_dispatch without a workspace: the library's built-in static scratch is used (for
+    callers that cannot allocate; the outputs here are still allocated by torch when omitted)."""
+    T, d = x.shape
+    k = expert_ids.shape[1]
+    dev = x.device
+    if rows_max is None:
+        rows_max = moe_packed_rows_max(T, E, k, C)
+    if slot is None:
+        slot = torch.empty(T, k, dtype=torch.int32, device=dev)
+    if expert_counts is None:
+        expert_counts = torch.empty(E, dtype=torch.int32, device=dev)
+    if expert_offsets is None:
+        expert_offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    if row_token is None:
+        row_token = torch.empty(max(rows_max, 1), dtype=torch.int32, device=dev)
+    if x_packed is None:
+        x_packed = torch.empty(max(rows_max, 1), d, dtype=x.dtype, device=dev)
+    _check("moe_dispatch_noalloc", lib().moe_dispatch_noalloc(
+        _ptr(x), _dt(x), T, d, _ptr(expert_ids), E, k, C, _ptr(slot), _ptr(expert_counts),
+        _ptr(expert_offsets), _ptr(row_token), _ptr(x_packed), rows_max, _stream(stream)))
+    return dict(slot=slot, expert_counts=expert_counts, expert_offsets=expert_offsets,
+                row_token=row_token, x_packed=x_packed, rows_max=rows_max)
 
 
 def moe_expert_ffn(x_packed: torch.Tensor, expert_offsets: torch.Tensor, w1, b1, w2, b2,
