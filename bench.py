@@ -51,13 +51,16 @@ class Dist:
         self.rank = int(os.environ.get("RANK", "0"))
         self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
         self.pg = False
+        self.backend = None
 
-    def init(self, device):
+    def init(self, device=None, backend: str = "nccl"):
         if self.world > 1:
             import datetime
             import torch.distributed as dist
-            dist.init_process_group("nccl", device_id=device, timeout=datetime.timedelta(seconds=300))
+            kw = {"device_id": device} if backend == "nccl" else {}
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300), **kw)
             self.pg = True
+            self.backend = backend
 
     def barrier(self):
         if self.pg:
@@ -68,7 +71,7 @@ class Dist:
         if not self.pg:
             return v
         import torch.distributed as dist
-        t = torch.tensor([v], dtype=torch.float64, device=device)
+        t = torch.tensor([v], dtype=torch.float64, device=device if self.backend == "nccl" else "cpu")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
