@@ -430,7 +430,7 @@ def breakdown(moe, w, d, ws_layer, stream, flush_buf, reps: int) -> dict:
     ids = torch.empty(T, k, dtype=torch.int32, device=dev)
     gates = torch.empty(T, k, dtype=torch.float32, device=dev)
     lb = torch.empty(2 * E + 1, dtype=torch.float32, device=dev)
-    ws_r = moe.workspace(moe.moe_router_workspace_bytes(T, E), dev)
+    ws_r = moe.workspace(moe.moe_router_workspace_bytes(T, E, dm), dev)
     ws_d = moe.workspace(moe.moe_dispatch_workspace_bytes(T, E, k), dev)
     ws_s = moe.workspace(256, dev)
     slot = torch.empty(T, k, dtype=torch.int32, device=dev)

@@ -104,7 +104,7 @@ moe_status moe_packed_rows_max(int64_t T, int E, int k, int64_t C, int64_t* rows
  * lb_stats:   [2E+1] fp32 output, or NULL.
  * Limits: 1 <= E <= 1024, 1 <= k <= min(E, 8), T >= 0 (T == 0 enqueues nothing), d_model >= 1;
  * bf16 x needs d_model % 8 == 0. */
-moe_status moe_router_workspace_bytes(int64_t T, int E, size_t* bytes);
+moe_status moe_router_workspace_bytes(int64_t T, int E, int d_model, size_t* bytes);
 moe_status moe_router_topk(const void* x, moe_dtype x_dtype, int64_t T, int d_model,
                            const float* w_router, const float* router_bias, int E, int k,
                            float* logits, int32_t* expert_ids, float* gates, float* lb_stats,

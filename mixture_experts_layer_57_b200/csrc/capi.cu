@@ -64,12 +64,14 @@ struct Carve {
 // ------------------------------------------------------------ workspace layouts
 
 struct RouterWs {
-  float* q_partial;
+  RouterScratch scr;
   float* logits;
 };
-RouterWs carve_router(Carve& c, int64_t T, int E) {
+RouterWs carve_router(Carve& c, int64_t T, int E, int d) {
   RouterWs w;
-  w.q_partial = c.take<float>((size_t)router_num_blocks(T) * E);
+  w.scr.q_partial = c.take<float>((size_t)router_num_blocks(T) * E);
+  w.scr.c_partial = c.take<int32_t>((size_t)router_num_blocks(T) * E);
+  w.scr.w_split = c.take<uint16_t>((size_t)E * 3 * router_split_dpad(d));
   w.logits = c.take<float>((size_t)T * E);
   return w;
 }
@@ -149,10 +151,10 @@ moe_status moe_packed_rows_max(int64_t T, int E, int k, int64_t C, int64_t* rows
 
 // ---------------------------------------------------------------- router
 
-moe_status moe_router_workspace_bytes(int64_t T, int E, size_t* bytes) {
-  if (!bytes || T < 0 || E < 1) return MOE_ERR_INVALID_ARGUMENT;
+moe_status moe_router_workspace_bytes(int64_t T, int E, int d_model, size_t* bytes) {
+  if (!bytes || T < 0 || E < 1 || d_model < 1) return MOE_ERR_INVALID_ARGUMENT;
   Carve c{nullptr};
-  carve_router(c, T, E);
+  carve_router(c, T, E, d_model);
   *bytes = c.off;
   return MOE_OK;
 }
@@ -171,16 +173,16 @@ moe_status moe_router_topk(const void* x, moe_dtype x_dtype, int64_t T, int d_mo
       ((uintptr_t)ws % kAlign) != 0)
     return MOE_ERR_MISALIGNED;
   size_t need = 0;
-  moe_router_workspace_bytes(T, E, &need);
+  moe_router_workspace_bytes(T, E, d_model, &need);
   if (ws_bytes < need) return MOE_ERR_WORKSPACE_TOO_SMALL;
   if (fault_injected("moe_router_topk")) return MOE_ERR_CUDA;
   g_launches = 0;
   if (T == 0) return MOE_OK;
   Carve c{(uint8_t*)ws};
-  RouterWs w = carve_router(c, T, E);
+  RouterWs w = carve_router(c, T, E, d_model);
   return cuda_status(enqueue_router(x, x_dtype == MOE_BF16, T, d_model, w_router, router_bias, E,
                                     k, logits ? logits : w.logits, expert_ids, gates, lb_stats,
-                                    aux_alpha, w.q_partial, stream));
+                                    aux_alpha, w.scr, (int*)ws, stream));
 }
 
 // ---------------------------------------------------------------- dispatch
@@ -348,7 +350,7 @@ moe_status layer_layout(const moe_layer_args* a, uint8_t* base, LayerWs* w, size
   const int E = a->E, k = a->k, d = a->d_model, f = a->d_ff;
   const size_t es = esize(a->dtype);
   Carve c{base};
-  w->router = carve_router(c, T, E);
+  w->router = carve_router(c, T, E, d);
   w->dispatch = carve_dispatch(c, T, E, k);
   w->logits = c.take<float>((size_t)T * E);
   w->gates = c.take<float>((size_t)T * k);
@@ -413,7 +415,7 @@ moe_status moe_layer_forward(const moe_layer_args* a, void* out, moe_layer_aux* 
   const int d = a->d_model, f = a->d_ff, E = a->E, k = a->k;
 
   cudaError_t e = enqueue_router(a->x, bf16, T, d, a->w_router, a->router_bias, E, k, logits, ids,
-                                 gates, lb, a->aux_alpha, w.router.q_partial, stream);
+                                 gates, lb, a->aux_alpha, w.router.scr, status, stream);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   e = enqueue_dispatch(a->x, bf16, T, d, ids, E, k, w.C, slot, counts, offsets, w.row_token,
                        w.x_packed, w.rows_max, w.dispatch.local_rank, w.dispatch.seg_counts,

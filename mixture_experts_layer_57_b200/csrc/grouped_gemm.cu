@@ -21,9 +21,11 @@
 //                 128-byte swizzle, STAGES-deep mbarrier ring
 //     warp 1      allocates TMEM, one thread issues tcgen05.mma (K = 16 per instruction) into
 //                 one of two accumulators, commits stage release and accumulator-full barriers
-//     warps 2..5  epilogue: tcgen05.ld of the accumulator, + bias, GeLU (erf form) and bf16
-//                 rounding for the first layer, or fp32 for the second, masked to the valid
-//                 rows/features, stored to global; then release the accumulator
+//     warps 2..9  epilogue, two warps per TMEM lane quarter taking alternate 16-column chunks:
+//                 tcgen05.ld of the accumulator, + bias, GeLU (erf form) and bf16 rounding for
+//                 the first layer or fp32 for the second, transposed through a per-warp shared
+//                 staging tile into 16-byte stores of whole token rows, masked to the valid
+//                 rows/features; then release the accumulator
 // Every wait is bounded (about 2 s): on expiry the kernel records MOE_DEVERR_TIMEOUT in the
 // status word, the other roles stop, in-flight TMA copies and MMAs are drained, TMEM is freed.
 #include "common.cuh"
@@ -35,7 +37,14 @@ namespace {
 constexpr int kBM = 128;         // output features per tile (MMA M)
 constexpr int kBK = 64;          // K per stage: one 128-byte swizzle row of bf16
 constexpr int kUmmaK = 16;       // K per tcgen05.mma (kind::f16)
-constexpr int kThreads = 192;    // 6 warps
+constexpr int kThreads = 320;    // 10 warps: TMA, MMA, 8 epilogue
+constexpr int kEpiWarps = 8;
+constexpr int kStageTileBytes = 16 * 32 * 4;  // per epilogue warp: 16 tokens x 32 features, fp32
+
+// Epilogue kinds.
+constexpr int kEpiGeluBf16 = 0;  // out = bf16(GeLU(acc + bias)), bias bf16   (expert layer 1)
+constexpr int kEpiF32 = 1;       // out = acc + bias (fp32), bias bf16          (expert layer 2)
+constexpr int kEpiRouter = 2;    // out = acc + bias (fp32), bias fp32          (router logits)
 
 template <int BN>
 struct Cfg {
@@ -48,21 +57,23 @@ struct Cfg {
   // barriers: full[S], empty[S], tmem_full[2], tmem_empty[2], drain  (8 bytes each, <= 64 of them)
   static constexpr int kBarBytes = 8 * 64;
   static constexpr int kAuxBytes = kBarBytes + 16 + 2 * 4 * (MOE_MAX_EXPERTS + 1);
-  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kAuxBytes;
+  static constexpr int kSmemBytes =
+      1024 + kStages * kStageBytes + kEpiWarps * kStageTileBytes + kAuxBytes;
   static_assert(kStageBytes % 1024 == 0, "stage tiles must stay 1024-byte aligned");
   static_assert(2 * kStages + 5 <= 64, "barrier area too small");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 
 struct Params {
-  const int32_t* offsets;  // [E+1]
+  const int32_t* offsets;  // [E+1], or nullptr: one segment [0, rows_max) (E == 1)
   int E;
   int n_out;               // output features per expert
-  int K;
+  int K;                   // reduction length of the weight operand
   int64_t rows_max;
-  const uint16_t* bias;    // [E, n_out] bf16, or nullptr
+  const void* bias;        // [E, n_out], bf16 (layers) or fp32 (router), or nullptr
   void* out;               // [rows_max, n_out]: bf16 (GeLU layer) or fp32
   int* status;
+  int x_kb_period;         // 0, or: the token operand's K block = (weight K block) mod this
 };
 
 struct Tile {
@@ -102,7 +113,7 @@ __device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity, i
   }
 }
 
-template <int BN, bool GELU_BF16_OUT>
+template <int BN, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmW,
                         const __grid_constant__ CUtensorMap tmX, const Params p) {
@@ -112,7 +123,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t base_addr = (raw_addr + 1023u) & ~1023u;
   uint8_t* base = smem_raw + (base_addr - raw_addr);
 
-  uint8_t* aux = base + C::kStages * C::kStageBytes;
+  uint8_t* stage_tiles = base + C::kStages * C::kStageBytes;
+  uint8_t* aux = stage_tiles + kEpiWarps * kStageTileBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(aux);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(aux + C::kBarBytes);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(aux + C::kBarBytes + 4);
@@ -136,7 +148,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), 128);
+      mbar_init(tempty_bar(a), kEpiWarps * 32);
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -212,7 +224,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t sa = base_addr + stage * C::kStageBytes;
           mbar_arrive_expect_tx(full_bar(stage), C::kStageBytes);
           tma_load_2d(sa, &tmW, kb * kBK, w_row, full_bar(stage));
-          tma_load_2d(sa + C::kABytes, &tmX, kb * kBK, tl.row0, full_bar(stage));
+          const int xkb = p.x_kb_period ? kb % p.x_kb_period : kb;
+          tma_load_2d(sa + C::kABytes, &tmX, xkb * kBK, tl.row0, full_bar(stage));
           ++issued;
           if (++stage == S) {
             stage = 0;
@@ -273,38 +286,73 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait_drain(drain_bar, 0, p.status);
     }
   } else {
-    // ---------------------------------------------------------- epilogue (warps 2..5)
-    const int quarter = warp & 3;  // TMEM lanes this warp may access: [32*quarter, 32*quarter+32)
+    // ---------------------------------------------------------- epilogue (warps 2..9)
+    const int ew = warp - 2;         // 0..7
+    const int quarter = warp & 3;    // TMEM lanes this warp may access: [32*quarter, 32*quarter+32)
+    const int half = ew >> 2;        // this warp takes 16-column chunks half, half+2, half+4, ...
+    uint8_t* st = stage_tiles + ew * kStageTileBytes;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
       const Tile tl = decode_tile<BN>(t, prefix, seg, p.E, n_ftiles);
       if (!mbar_wait_bounded_warp(tfull_bar(acc), acc_phase, abort_flag, p.status)) break;
       tc_fence_after();
-      const int f = tl.f0 + quarter * 32 + lane;
+      const int fw = tl.f0 + quarter * 32;  // first feature of this warp
+      const int f = fw + lane;
       const bool f_ok = f < p.n_out;
-      const float bv = (p.bias != nullptr && f_ok)
-                           ? bf16_to_f32(p.bias[(int64_t)tl.e * p.n_out + f])
-                           : 0.0f;
+      float bv = 0.0f;
+      if (p.bias != nullptr && f_ok) {
+        const int64_t bi = (int64_t)tl.e * p.n_out + f;
+        bv = EPI == kEpiRouter ? reinterpret_cast<const float*>(p.bias)[bi]
+                               : bf16_to_f32(reinterpret_cast<const uint16_t*>(p.bias)[bi]);
+      }
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
-      for (int c0 = 0; c0 < tl.n_valid; c0 += 16) {
+      for (int c0 = half * 16; c0 < tl.n_valid; c0 += 32) {
         uint32_t r[16];
         tmem_ld_32x32b_x16(taddr + (uint32_t)c0, r);
         tmem_ld_wait();
-        if (f_ok) {
-          const int nc = min(16, tl.n_valid - c0);
+        const int nc = min(16, tl.n_valid - c0);
+        if constexpr (EPI == kEpiRouter) {
+          // fp32 logits, E need not be a multiple of 4: coalesced scalar stores per token row
+          if (f_ok) {
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            if (c < nc) {
-              const int64_t o = (int64_t)(tl.row0 + c0 + c) * p.n_out + f;
-              const float v = __uint_as_float(r[c]) + bv;
-              if constexpr (GELU_BF16_OUT) {
-                reinterpret_cast<uint16_t*>(p.out)[o] = f32_to_bf16_rn(gelu_erf(v));
-              } else {
-                reinterpret_cast<float*>(p.out)[o] = v;
-              }
-            }
+            for (int c = 0; c < 16; ++c)
+              if (c < nc)
+                reinterpret_cast<float*>(p.out)[(int64_t)(tl.row0 + c0 + c) * p.n_out + f] =
+                    __uint_as_float(r[c]) + bv;
           }
+        } else if constexpr (EPI == kEpiGeluBf16) {
+          // stage [16 tokens][32 features] bf16, then 16-byte stores of 8 features of one token
+          uint16_t* s16 = reinterpret_cast<uint16_t*>(st);
+#pragma unroll
+          for (int c = 0; c < 16; ++c) s16[c * 32 + lane] = f32_to_bf16_rn(gelu_erf(__uint_as_float(r[c]) + bv));
+          __syncwarp();
+#pragma unroll
+          for (int id = lane; id < 64; id += 32) {
+            const int row = id >> 2, q = id & 3;
+            const int ff = fw + 8 * q;
+            if (row < nc && ff < p.n_out)
+              *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.out) +
+                                        (int64_t)(tl.row0 + c0 + row) * p.n_out + ff) =
+                  *reinterpret_cast<const uint4*>(st + row * 64 + q * 16);
+          }
+          __syncwarp();
+        } else {
+          // stage [16 tokens][32 features] fp32, then 16-byte stores of 4 features of one token
+          float* s32 = reinterpret_cast<float*>(st);
+#pragma unroll
+          for (int c = 0; c < 16; ++c) s32[c * 32 + lane] = __uint_as_float(r[c]) + bv;
+          __syncwarp();
+#pragma unroll
+          for (int id = lane; id < 128; id += 32) {
+            const int row = id >> 3, q = id & 7;
+            const int ff = fw + 4 * q;
+            if (row < nc && ff < p.n_out)
+              *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) +
+                                         (int64_t)(tl.row0 + c0 + row) * p.n_out + ff) =
+                  *reinterpret_cast<const float4*>(st + row * 128 + q * 16);
+          }
+          __syncwarp();
         }
       }
       tc_fence_before();
@@ -358,10 +406,10 @@ bool make_kmajor_map(CUtensorMap* m, const void* ptr, int64_t rows, int K, int b
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, bool GELU>
+template <int BN, int EPI>
 cudaError_t launch_one(const CUtensorMap& tmW, const CUtensorMap& tmX, const Params& p,
                        cudaStream_t stream) {
-  auto kern = grouped_gemm_kernel<BN, GELU>;
+  auto kern = grouped_gemm_kernel<BN, EPI>;
   static bool attr_set = false;  // per instantiation
   if (!attr_set) {
     cudaError_t e =
@@ -384,6 +432,18 @@ static int pick_token_tile(int64_t capacity_hint) {
   return 256;
 }
 
+template <int EPI>
+cudaError_t launch_bn(int BN, const CUtensorMap& tmW, const CUtensorMap& tmX, const Params& p,
+                      cudaStream_t stream) {
+  switch (BN) {
+    case 16: return launch_one<16, EPI>(tmW, tmX, p, stream);
+    case 32: return launch_one<32, EPI>(tmW, tmX, p, stream);
+    case 64: return launch_one<64, EPI>(tmW, tmX, p, stream);
+    case 128: return launch_one<128, EPI>(tmW, tmX, p, stream);
+    default: return launch_one<256, EPI>(tmW, tmX, p, stream);
+  }
+}
+
 cudaError_t enqueue_grouped_gemm_bf16(const void* x, const int32_t* offsets, int E,
                                       int64_t rows_max, int K, int N, const void* w,
                                       const void* bias, bool gelu, void* out,
@@ -393,21 +453,24 @@ cudaError_t enqueue_grouped_gemm_bf16(const void* x, const int32_t* offsets, int
   CUtensorMap tmW, tmX;
   if (!make_kmajor_map(&tmW, w, (int64_t)E * N, K, kBM) || !make_kmajor_map(&tmX, x, rows_max, K, BN))
     return cudaErrorInvalidValue;
-  const Params p{offsets, E, N, K, rows_max, (const uint16_t*)bias, out, status};
-#define MOE_GG_CASE(BNV)                                                          \
-  case BNV:                                                                      \
-    return gelu ? launch_one<BNV, true>(tmW, tmX, p, stream)                      \
-                : launch_one<BNV, false>(tmW, tmX, p, stream);
-  switch (BN) {
-    MOE_GG_CASE(16)
-    MOE_GG_CASE(32)
-    MOE_GG_CASE(64)
-    MOE_GG_CASE(128)
-    default:
-      return gelu ? launch_one<256, true>(tmW, tmX, p, stream)
-                  : launch_one<256, false>(tmW, tmX, p, stream);
-  }
-#undef MOE_GG_CASE
+  const Params p{offsets, E, N, K, rows_max, bias, out, status, 0};
+  return gelu ? launch_bn<kEpiGeluBf16>(BN, tmW, tmX, p, stream)
+              : launch_bn<kEpiF32>(BN, tmW, tmX, p, stream);
+}
+
+cudaError_t enqueue_router_logits_tc(const void* x, int64_t T, int d, const uint16_t* w_split,
+                                     int dpad, const float* router_bias, int E, float* logits,
+                                     int* status, cudaStream_t stream) {
+  if (T == 0) return cudaSuccess;
+  // token tile: the widest that still gives every SM at least one tile
+  const int n_ftiles = (E + kBM - 1) / kBM;
+  int BN = 256;
+  while (BN > 16 && (int64_t)n_ftiles * ((T + BN - 1) / BN) < num_sms()) BN >>= 1;
+  CUtensorMap tmW, tmX;
+  if (!make_kmajor_map(&tmW, w_split, E, 3 * dpad, kBM) || !make_kmajor_map(&tmX, x, T, d, BN))
+    return cudaErrorInvalidValue;
+  const Params p{nullptr, 1, E, 3 * dpad, T, router_bias, logits, status, dpad / kBK};
+  return launch_bn<kEpiRouter>(BN, tmW, tmX, p, stream);
 }
 
 cudaError_t enqueue_expert_ffn_bf16(const void* x_packed, const int32_t* offsets, int E,

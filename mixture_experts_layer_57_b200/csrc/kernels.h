@@ -21,10 +21,23 @@ constexpr int kRouterTokensPerBlock = 64;
 inline int64_t router_num_blocks(int64_t T) {
   return (T + kRouterTokensPerBlock - 1) / kRouterTokensPerBlock;
 }
+// K of each bf16 part of the split router weight, padded to the 64-element TMA block.
+inline int router_split_dpad(int d) { return (d + 63) / 64 * 64; }
+// The tensor-core router needs bf16 x whose rows are whole 16-byte units.
+inline bool router_uses_tensor_cores(bool x_bf16, int d) { return x_bf16 && d % 8 == 0; }
+struct RouterScratch {
+  float* q_partial;   // [router_num_blocks(T), E] per-block sums of p
+  int32_t* c_partial; // [router_num_blocks(T), E] per-block counts of first choices
+  uint16_t* w_split;  // [E, 3 * router_split_dpad(d)] bf16: hi | mid | lo parts of W_r
+};
 cudaError_t enqueue_router(const void* x, bool x_bf16, int64_t T, int d, const float* w_router,
                            const float* router_bias, int E, int k, float* logits, int32_t* ids,
-                           float* gates, float* lb_stats, float aux_alpha, float* q_partial,
-                           cudaStream_t stream);
+                           float* gates, float* lb_stats, float aux_alpha,
+                           const RouterScratch& scratch, int* status, cudaStream_t stream);
+// logits = x W_r^T + b_r on tcgen05 from the exact split W_r = hi + mid + lo (bf16 each).
+cudaError_t enqueue_router_logits_tc(const void* x, int64_t T, int d, const uint16_t* w_split,
+                                     int dpad, const float* router_bias, int E, float* logits,
+                                     int* status, cudaStream_t stream);
 
 // ---------------------------------------------------------------- dispatch
 constexpr int kDispatchSeg = 256;  // (token, choice) pairs per counting segment (one warp)

@@ -7,12 +7,16 @@
 // §1.1.4.1 (f_i, Q_i, loss = alpha * N * sum f_i Q_i).
 //
 // Kernels:
-//   router_logits_kernel  tiled fp32 GEMM, 64 tokens x 64 experts per block, fixed K order
+//   router_split_kernel   W_r (fp32) -> three bf16 parts hi + mid + lo that sum to W_r exactly
+//                         (each part takes the next 8 significant bits), for the tensor-core
+//                         logits: x is bf16, so x * W_r = x*hi + x*mid + x*lo with exact
+//                         products, accumulated in fp32 by tcgen05 (grouped_gemm.cu)
+//   router_logits_kernel  tiled fp32-FMA GEMM for fp32 x, 64 tokens x 64 experts per block
 //   router_topk_kernel    one warp per token: max, sum of exp, p = exp(l - max) / sum,
 //                         k rounds of warp argmax on the logits (ties -> lower index);
-//                         per-block partial sums of p per expert in a fixed order
-//   router_stats_kernel   one block: f from the first choices, Q from the partials in block
-//                         order, aux = alpha * E * sum f Q (sequential)
+//                         per-block sums of p and counts of first choices per expert
+//   router_stats_kernel   one block: fixed-order reduction of the per-block partials into
+//                         f, Q and aux = alpha * E * sum f Q
 #include "common.cuh"
 #include "kernels.h"
 
@@ -71,15 +75,39 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const void* __restri
   }
 }
 
+__global__ void __launch_bounds__(256) router_split_kernel(const float* __restrict__ w, int E,
+                                                           int d, int dpad,
+                                                           uint16_t* __restrict__ out) {
+  const int64_t n = (int64_t)E * dpad;
+  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < n;
+       idx += (int64_t)gridDim.x * blockDim.x) {
+    const int e = (int)(idx / dpad), i = (int)(idx % dpad);
+    const float v = i < d ? w[(int64_t)e * d + i] : 0.0f;
+    const uint16_t hi = f32_to_bf16_rn(v);
+    const float r1 = v - bf16_to_f32(hi);     // exact: hi is v rounded to 8 significant bits
+    const uint16_t mid = f32_to_bf16_rn(r1);
+    const float r2 = r1 - bf16_to_f32(mid);   // exact, at most 8 significant bits left
+    const uint16_t lo = f32_to_bf16_rn(r2);   // == r2
+    uint16_t* row = out + (int64_t)e * 3 * dpad;
+    row[i] = hi;
+    row[dpad + i] = mid;
+    row[2 * dpad + i] = lo;
+  }
+}
+
 // EPL = experts per lane (E <= 32 * EPL); expert e lives in lane e % 32, slot e / 32.
 template <int EPL>
 __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restrict__ logits,
                                                           int64_t T, int E, int k,
                                                           int32_t* __restrict__ ids,
                                                           float* __restrict__ gates,
-                                                          float* __restrict__ q_partial) {
+                                                          float* __restrict__ q_partial,
+                                                          int32_t* __restrict__ c_partial) {
   __shared__ float qs[8][MOE_MAX_EXPERTS];
+  __shared__ int cs[MOE_MAX_EXPERTS];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int e = threadIdx.x; e < E; e += 256) cs[e] = 0;
+  __syncthreads();
   float q[EPL];
 #pragma unroll
   for (int i = 0; i < EPL; ++i) q[i] = 0.0f;
@@ -144,6 +172,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
       if (lane == 0) {
         ids[t * k + j] = bi;
         gates[t * k + j] = pv;
+        if (j == 0) atomicAdd(&cs[bi], 1);  // integer counts: order-independent
       }
     }
   }
@@ -159,34 +188,48 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
 #pragma unroll
     for (int w = 0; w < 8; ++w) s += qs[w][e];
     q_partial[(int64_t)blockIdx.x * E + e] = s;
+    c_partial[(int64_t)blockIdx.x * E + e] = cs[e];
   }
 }
 
-__global__ void __launch_bounds__(1024) router_stats_kernel(const int32_t* __restrict__ ids,
-                                                            int64_t T, int E, int k,
-                                                            const float* __restrict__ q_partial,
-                                                            int64_t nblk, float alpha,
-                                                            float* __restrict__ lb) {
-  __shared__ int hist[MOE_MAX_EXPERTS];
+// Thread (g, e) sums the partials of blocks g, g + G, g + 2G, ... of expert e; the G group sums
+// are then added in group order. G = 1024 / E groups; fixed assignment and order.
+__global__ void __launch_bounds__(1024) router_stats_kernel(const float* __restrict__ q_partial,
+                                                            const int32_t* __restrict__ c_partial,
+                                                            int64_t nblk, int64_t T, int E,
+                                                            float alpha, float* __restrict__ lb) {
+  __shared__ float sq[1024];
+  __shared__ int sc[1024];
   __shared__ float prod[MOE_MAX_EXPERTS];
-  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
-  __syncthreads();
-  for (int64_t t = threadIdx.x; t < T; t += blockDim.x) {
-    const int e = ids[t * k];
-    if (e >= 0 && e < E) atomicAdd(&hist[e], 1);
+  const int G = 1024 / E;
+  const int tid = threadIdx.x;
+  if (tid < G * E) {
+    const int g = tid / E, e = tid % E;
+    float q = 0.0f;
+    int c = 0;
+    for (int64_t b = g; b < nblk; b += G) {
+      q += q_partial[b * E + e];
+      c += c_partial[b * E + e];
+    }
+    sq[tid] = q;
+    sc[tid] = c;
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    float s = 0.0f;
-    for (int64_t b = 0; b < nblk; ++b) s += q_partial[b * E + e];
-    const float Q = s / (float)T;
-    const float f = (float)hist[e] / (float)T;
-    lb[e] = f;
-    lb[E + e] = Q;
-    prod[e] = f * Q;
+  if (tid < E) {
+    float q = 0.0f;
+    int c = 0;
+    for (int g = 0; g < G; ++g) {
+      q += sq[g * E + tid];
+      c += sc[g * E + tid];
+    }
+    const float Q = q / (float)T;
+    const float f = (float)c / (float)T;
+    lb[tid] = f;
+    lb[E + tid] = Q;
+    prod[tid] = f * Q;
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (tid == 0) {
     float s = 0.0f;
     for (int e = 0; e < E; ++e) s += prod[e];
     lb[2 * E] = alpha * (float)E * s;
@@ -195,34 +238,47 @@ __global__ void __launch_bounds__(1024) router_stats_kernel(const int32_t* __res
 
 template <int EPL>
 void launch_topk(const float* logits, int64_t T, int E, int k, int32_t* ids, float* gates,
-                 float* q_partial, cudaStream_t stream) {
-  router_topk_kernel<EPL><<<(unsigned)router_num_blocks(T), 256, 0, stream>>>(logits, T, E, k, ids,
-                                                                              gates, q_partial);
+                 float* q_partial, int32_t* c_partial, cudaStream_t stream) {
+  router_topk_kernel<EPL><<<(unsigned)router_num_blocks(T), 256, 0, stream>>>(
+      logits, T, E, k, ids, gates, q_partial, c_partial);
 }
 
 }  // namespace
 
 cudaError_t enqueue_router(const void* x, bool x_bf16, int64_t T, int d, const float* w_router,
                            const float* router_bias, int E, int k, float* logits, int32_t* ids,
-                           float* gates, float* lb_stats, float aux_alpha, float* q_partial,
-                           cudaStream_t stream) {
+                           float* gates, float* lb_stats, float aux_alpha,
+                           const RouterScratch& scr, int* status, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
-  dim3 grid((unsigned)((T + kLBM - 1) / kLBM), (E + kLBN - 1) / kLBN);
-  if (x_bf16)
-    router_logits_kernel<true><<<grid, 256, 0, stream>>>(x, w_router, router_bias, T, d, E, logits);
-  else
-    router_logits_kernel<false><<<grid, 256, 0, stream>>>(x, w_router, router_bias, T, d, E, logits);
-  count_launch();
-  if (E <= 32) launch_topk<1>(logits, T, E, k, ids, gates, q_partial, stream);
-  else if (E <= 64) launch_topk<2>(logits, T, E, k, ids, gates, q_partial, stream);
-  else if (E <= 128) launch_topk<4>(logits, T, E, k, ids, gates, q_partial, stream);
-  else if (E <= 256) launch_topk<8>(logits, T, E, k, ids, gates, q_partial, stream);
-  else if (E <= 512) launch_topk<16>(logits, T, E, k, ids, gates, q_partial, stream);
-  else launch_topk<32>(logits, T, E, k, ids, gates, q_partial, stream);
+  if (router_uses_tensor_cores(x_bf16, d)) {
+    const int dpad = router_split_dpad(d);
+    const int64_t n = (int64_t)E * dpad;
+    const unsigned blocks = (unsigned)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+    router_split_kernel<<<blocks, 256, 0, stream>>>(w_router, E, d, dpad, scr.w_split);
+    count_launch();
+    cudaError_t e = enqueue_router_logits_tc(x, T, d, scr.w_split, dpad, router_bias, E, logits,
+                                             status, stream);
+    if (e != cudaSuccess) return e;
+  } else {
+    dim3 grid((unsigned)((T + kLBM - 1) / kLBM), (E + kLBN - 1) / kLBN);
+    if (x_bf16)
+      router_logits_kernel<true><<<grid, 256, 0, stream>>>(x, w_router, router_bias, T, d, E, logits);
+    else
+      router_logits_kernel<false><<<grid, 256, 0, stream>>>(x, w_router, router_bias, T, d, E, logits);
+    count_launch();
+  }
+  float* qp = scr.q_partial;
+  int32_t* cp = scr.c_partial;
+  if (E <= 32) launch_topk<1>(logits, T, E, k, ids, gates, qp, cp, stream);
+  else if (E <= 64) launch_topk<2>(logits, T, E, k, ids, gates, qp, cp, stream);
+  else if (E <= 128) launch_topk<4>(logits, T, E, k, ids, gates, qp, cp, stream);
+  else if (E <= 256) launch_topk<8>(logits, T, E, k, ids, gates, qp, cp, stream);
+  else if (E <= 512) launch_topk<16>(logits, T, E, k, ids, gates, qp, cp, stream);
+  else launch_topk<32>(logits, T, E, k, ids, gates, qp, cp, stream);
   count_launch();
   if (lb_stats) {
-    router_stats_kernel<<<1, 1024, 0, stream>>>(ids, T, E, k, q_partial, router_num_blocks(T),
-                                                aux_alpha, lb_stats);
+    router_stats_kernel<<<1, 1024, 0, stream>>>(qp, cp, router_num_blocks(T), T, E, aux_alpha,
+                                                lb_stats);
     count_launch();
   }
   return cudaGetLastError();

@@ -73,7 +73,7 @@ def lib() -> ctypes.CDLL:
             "moe_last_launch_count": ([], i32),
             "moe_capacity": ([i64, i32, i32, f64, P(i64)], i32),
             "moe_packed_rows_max": ([i64, i32, i32, i64, P(i64)], i32),
-            "moe_router_workspace_bytes": ([i64, i32, P(sz)], i32),
+            "moe_router_workspace_bytes": ([i64, i32, i32, P(sz)], i32),
             "moe_router_topk": ([vp, i32, i64, i32, vp, vp, i32, i32, vp, vp, vp, vp, f32, vp, sz, vp], i32),
             "moe_dispatch_workspace_bytes": ([i64, i32, i32, P(sz)], i32),
             "moe_dispatch": ([vp, i32, i64, i32, vp, i32, i32, i64, vp, vp, vp, vp, vp, i64, vp, sz, vp], i32),
@@ -159,8 +159,8 @@ def _ws_bytes(fn: str, *args) -> int:
     return out.value
 
 
-def moe_router_workspace_bytes(T, E):
-    return _ws_bytes("moe_router_workspace_bytes", T, E)
+def moe_router_workspace_bytes(T, E, d_model):
+    return _ws_bytes("moe_router_workspace_bytes", T, E, d_model)
 
 
 def moe_dispatch_workspace_bytes(T, E, k):
@@ -193,7 +193,7 @@ def moe_router_topk(x: torch.Tensor, w_router: torch.Tensor, k: int,
     if lb_stats is None and want_stats:
         lb_stats = torch.empty(2 * E + 1, dtype=torch.float32, device=dev)
     if ws is None:
-        ws = workspace(moe_router_workspace_bytes(T, E), dev)
+        ws = workspace(moe_router_workspace_bytes(T, E, d), dev)
     _check("moe_router_topk", lib().moe_router_topk(
         _ptr(x), _dt(x), T, d, _ptr(w_router), _ptr(router_bias), E, k, _ptr(logits),
         _ptr(expert_ids), _ptr(gates), _ptr(lb_stats), aux_alpha, _ptr(ws), ws.numel(), _stream(stream)))
