@@ -69,10 +69,12 @@ struct RouterWs {
 };
 RouterWs carve_router(Carve& c, int64_t T, int E, int d) {
   RouterWs w;
-  w.scr.q_partial = c.take<float>((size_t)router_num_blocks(T) * E);
-  w.scr.c_partial = c.take<int32_t>((size_t)router_num_blocks(T) * E);
+  w.scr.acc.q = c.take<unsigned long long>((size_t)E);
+  w.scr.acc.c = c.take<unsigned>((size_t)E);
+  w.scr.acc.ticket = c.take<unsigned>(1);
   w.scr.w_split = c.take<uint16_t>((size_t)E * 3 * router_split_dpad(d));
   w.logits = c.take<float>((size_t)T * E);
+  w.scr.logits_scratch = w.logits;
   return w;
 }
 
@@ -181,8 +183,8 @@ moe_status moe_router_topk(const void* x, moe_dtype x_dtype, int64_t T, int d_mo
   Carve c{(uint8_t*)ws};
   RouterWs w = carve_router(c, T, E, d_model);
   return cuda_status(enqueue_router(x, x_dtype == MOE_BF16, T, d_model, w_router, router_bias, E,
-                                    k, logits ? logits : w.logits, expert_ids, gates, lb_stats,
-                                    aux_alpha, w.scr, (int*)ws, stream));
+                                    k, logits, expert_ids, gates, lb_stats, aux_alpha, w.scr,
+                                    (int*)ws, stream));
 }
 
 // ---------------------------------------------------------------- dispatch
@@ -326,7 +328,7 @@ namespace {
 struct LayerWs {
   RouterWs router;
   DispatchWs dispatch;
-  float *logits, *gates, *lb_stats;
+  float *gates, *lb_stats;
   int32_t *ids, *slot, *counts, *offsets, *row_token;
   void *x_packed, *h_packed;
   float* y_packed;
@@ -352,7 +354,6 @@ moe_status layer_layout(const moe_layer_args* a, uint8_t* base, LayerWs* w, size
   Carve c{base};
   w->router = carve_router(c, T, E, d);
   w->dispatch = carve_dispatch(c, T, E, k);
-  w->logits = c.take<float>((size_t)T * E);
   w->gates = c.take<float>((size_t)T * k);
   w->lb_stats = c.take<float>((size_t)2 * E + 1);
   w->ids = c.take<int32_t>((size_t)T * k);
@@ -402,7 +403,7 @@ moe_status moe_layer_forward(const moe_layer_args* a, void* out, moe_layer_aux* 
   g_launches = 0;
   if (a->T == 0) return MOE_OK;
 
-  float* logits = aux && aux->logits ? aux->logits : w.logits;
+  float* logits = aux ? aux->logits : nullptr;  // the router keeps its own scratch if needed
   int32_t* ids = aux && aux->expert_ids ? aux->expert_ids : w.ids;
   float* gates = aux && aux->gates ? aux->gates : w.gates;
   int32_t* slot = aux && aux->slot ? aux->slot : w.slot;

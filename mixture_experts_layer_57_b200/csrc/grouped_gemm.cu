@@ -44,7 +44,6 @@ constexpr int kStageTileBytes = 16 * 32 * 4;  // per epilogue warp: 16 tokens x 
 // Epilogue kinds.
 constexpr int kEpiGeluBf16 = 0;  // out = bf16(GeLU(acc + bias)), bias bf16   (expert layer 1)
 constexpr int kEpiF32 = 1;       // out = acc + bias (fp32), bias bf16          (expert layer 2)
-constexpr int kEpiRouter = 2;    // out = acc + bias (fp32), bias fp32          (router logits)
 
 template <int BN>
 struct Cfg {
@@ -70,10 +69,9 @@ struct Params {
   int n_out;               // output features per expert
   int K;                   // reduction length of the weight operand
   int64_t rows_max;
-  const void* bias;        // [E, n_out], bf16 (layers) or fp32 (router), or nullptr
+  const void* bias;        // [E, n_out] bf16, or nullptr
   void* out;               // [rows_max, n_out]: bf16 (GeLU layer) or fp32
   int* status;
-  int x_kb_period;         // 0, or: the token operand's K block = (weight K block) mod this
 };
 
 struct Tile {
@@ -224,8 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t sa = base_addr + stage * C::kStageBytes;
           mbar_arrive_expect_tx(full_bar(stage), C::kStageBytes);
           tma_load_2d(sa, &tmW, kb * kBK, w_row, full_bar(stage));
-          const int xkb = p.x_kb_period ? kb % p.x_kb_period : kb;
-          tma_load_2d(sa + C::kABytes, &tmX, xkb * kBK, tl.row0, full_bar(stage));
+          tma_load_2d(sa + C::kABytes, &tmX, kb * kBK, tl.row0, full_bar(stage));
           ++issued;
           if (++stage == S) {
             stage = 0;
@@ -300,28 +297,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int fw = tl.f0 + quarter * 32;  // first feature of this warp
       const int f = fw + lane;
       const bool f_ok = f < p.n_out;
-      float bv = 0.0f;
-      if (p.bias != nullptr && f_ok) {
-        const int64_t bi = (int64_t)tl.e * p.n_out + f;
-        bv = EPI == kEpiRouter ? reinterpret_cast<const float*>(p.bias)[bi]
-                               : bf16_to_f32(reinterpret_cast<const uint16_t*>(p.bias)[bi]);
-      }
+      const float bv = (p.bias != nullptr && f_ok)
+                           ? bf16_to_f32(reinterpret_cast<const uint16_t*>(p.bias)[(int64_t)tl.e * p.n_out + f])
+                           : 0.0f;
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
       for (int c0 = half * 16; c0 < tl.n_valid; c0 += 32) {
         uint32_t r[16];
         tmem_ld_32x32b_x16(taddr + (uint32_t)c0, r);
         tmem_ld_wait();
         const int nc = min(16, tl.n_valid - c0);
-        if constexpr (EPI == kEpiRouter) {
-          // fp32 logits, E need not be a multiple of 4: coalesced scalar stores per token row
-          if (f_ok) {
-#pragma unroll
-            for (int c = 0; c < 16; ++c)
-              if (c < nc)
-                reinterpret_cast<float*>(p.out)[(int64_t)(tl.row0 + c0 + c) * p.n_out + f] =
-                    __uint_as_float(r[c]) + bv;
-          }
-        } else if constexpr (EPI == kEpiGeluBf16) {
+        if constexpr (EPI == kEpiGeluBf16) {
           // stage [16 tokens][32 features] bf16, then 16-byte stores of 8 features of one token
           uint16_t* s16 = reinterpret_cast<uint16_t*>(st);
 #pragma unroll
@@ -453,24 +438,9 @@ cudaError_t enqueue_grouped_gemm_bf16(const void* x, const int32_t* offsets, int
   CUtensorMap tmW, tmX;
   if (!make_kmajor_map(&tmW, w, (int64_t)E * N, K, kBM) || !make_kmajor_map(&tmX, x, rows_max, K, BN))
     return cudaErrorInvalidValue;
-  const Params p{offsets, E, N, K, rows_max, bias, out, status, 0};
+  const Params p{offsets, E, N, K, rows_max, bias, out, status};
   return gelu ? launch_bn<kEpiGeluBf16>(BN, tmW, tmX, p, stream)
               : launch_bn<kEpiF32>(BN, tmW, tmX, p, stream);
-}
-
-cudaError_t enqueue_router_logits_tc(const void* x, int64_t T, int d, const uint16_t* w_split,
-                                     int dpad, const float* router_bias, int E, float* logits,
-                                     int* status, cudaStream_t stream) {
-  if (T == 0) return cudaSuccess;
-  // token tile: the widest that still gives every SM at least one tile
-  const int n_ftiles = (E + kBM - 1) / kBM;
-  int BN = 256;
-  while (BN > 16 && (int64_t)n_ftiles * ((T + BN - 1) / BN) < num_sms()) BN >>= 1;
-  CUtensorMap tmW, tmX;
-  if (!make_kmajor_map(&tmW, w_split, E, 3 * dpad, kBM) || !make_kmajor_map(&tmX, x, T, d, BN))
-    return cudaErrorInvalidValue;
-  const Params p{nullptr, 1, E, 3 * dpad, T, router_bias, logits, status, dpad / kBK};
-  return launch_bn<kEpiRouter>(BN, tmW, tmX, p, stream);
 }
 
 cudaError_t enqueue_expert_ffn_bf16(const void* x_packed, const int32_t* offsets, int E,

@@ -25,11 +25,18 @@ inline int64_t router_num_blocks(int64_t T) {
 inline int router_split_dpad(int d) { return (d + 63) / 64 * 64; }
 // The tensor-core router needs bf16 x whose rows are whole 16-byte units.
 inline bool router_uses_tensor_cores(bool x_bf16, int d) { return x_bf16 && d % 8 == 0; }
-struct RouterScratch {
-  float* q_partial;   // [router_num_blocks(T), E] per-block sums of p
-  int32_t* c_partial; // [router_num_blocks(T), E] per-block counts of first choices
-  uint16_t* w_split;  // [E, 3 * router_split_dpad(d)] bf16: hi | mid | lo parts of W_r
+// Load-balance statistics accumulators (zeroed by the router's first kernel each call).
+struct RouterAccum {
+  unsigned long long* q;  // [E] sums of p in 2^-32 fixed point
+  unsigned* c;            // [E] counts of first choices
+  unsigned* ticket;       // blocks finished
 };
+struct RouterScratch {
+  RouterAccum acc;
+  uint16_t* w_split;      // [E, 3 * router_split_dpad(d)] bf16: hi | mid | lo parts of W_r
+  float* logits_scratch;  // [T, E], used when the caller does not ask for the logits
+};
+// logits may be nullptr (not returned).
 cudaError_t enqueue_router(const void* x, bool x_bf16, int64_t T, int d, const float* w_router,
                            const float* router_bias, int E, int k, float* logits, int32_t* ids,
                            float* gates, float* lb_stats, float aux_alpha,

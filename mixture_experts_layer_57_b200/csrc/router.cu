@@ -4,25 +4,29 @@
 // DeepSpeed MoE blog, MoE formula p(x) = softmax(W_r x) and the listing's
 // `expert_ids, gates = topk(scores, k)`; comparison article, "Router computation"
 // (logits = x W_r, p = softmax(logits)) and "Top-1 routing decision"; MoE survey notes
-// §1.1.4.1 (f_i, Q_i, loss = alpha * N * sum f_i Q_i).
+// §1.1.4.1 (f_i = share of tokens whose first choice is i, Q_i = mean p_i,
+// loss = alpha * N * sum_i f_i Q_i).
 //
-// Kernels:
-//   router_split_kernel   W_r (fp32) -> three bf16 parts hi + mid + lo that sum to W_r exactly
-//                         (each part takes the next 8 significant bits), for the tensor-core
-//                         logits: x is bf16, so x * W_r = x*hi + x*mid + x*lo with exact
-//                         products, accumulated in fp32 by tcgen05 (grouped_gemm.cu)
-//   router_logits_kernel  tiled fp32-FMA GEMM for fp32 x, 64 tokens x 64 experts per block
+// Kernels, in launch order:
+//   router_prep_kernel    zeroes the statistics accumulators; for bf16 x also splits W_r (fp32)
+//                         into three bf16 parts hi + mid + lo that sum to W_r exactly (each takes
+//                         the next 8 significant bits), for the tensor-core logits
+//   logits                router_logits_tc_kernel (router_fused.cu, tcgen05: x * W_r =
+//                         x*hi + x*mid + x*lo from exact products, fp32 accumulation) for bf16 x,
+//                         or router_logits_kernel below (fp32 FMA) for fp32 x
 //   router_topk_kernel    one warp per token: max, sum of exp, p = exp(l - max) / sum,
-//                         k rounds of warp argmax on the logits (ties -> lower index);
-//                         per-block sums of p and counts of first choices per expert
-//   router_stats_kernel   one block: fixed-order reduction of the per-block partials into
-//                         f, Q and aux = alpha * E * sum f Q
+//                         k rounds of warp argmax on the logits (ties -> lower index), gates;
+//                         per-block sums of p (fixed order) and first-choice counts are added to
+//                         global accumulators as integers (p sums in 2^-32 fixed point), so the
+//                         totals do not depend on the order of the blocks; the last block to
+//                         finish turns them into f, Q and aux
 #include "common.cuh"
 #include "kernels.h"
 
 namespace moe {
 namespace {
 
+// fp32-FMA logits for fp32 x: 64 tokens x 64 experts per block, K in index order.
 constexpr int kLBM = 64, kLBN = 64, kLBK = 32;
 
 template <bool XBF16>
@@ -75,9 +79,17 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const void* __restri
   }
 }
 
-__global__ void __launch_bounds__(256) router_split_kernel(const float* __restrict__ w, int E,
-                                                           int d, int dpad,
-                                                           uint16_t* __restrict__ out) {
+__global__ void __launch_bounds__(256) router_prep_kernel(const float* __restrict__ w, int E,
+                                                          int d, int dpad, uint16_t* __restrict__ out,
+                                                          RouterAccum acc) {
+  if (blockIdx.x == 0) {
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+      acc.q[e] = 0ull;
+      acc.c[e] = 0u;
+    }
+    if (threadIdx.x == 0) *acc.ticket = 0u;
+  }
+  if (out == nullptr) return;
   const int64_t n = (int64_t)E * dpad;
   for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < n;
        idx += (int64_t)gridDim.x * blockDim.x) {
@@ -95,16 +107,20 @@ __global__ void __launch_bounds__(256) router_split_kernel(const float* __restri
   }
 }
 
+constexpr double kQScale = 4294967296.0;  // 2^32: fixed-point scale of the p sums
+
 // EPL = experts per lane (E <= 32 * EPL); expert e lives in lane e % 32, slot e / 32.
 template <int EPL>
 __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restrict__ logits,
                                                           int64_t T, int E, int k,
                                                           int32_t* __restrict__ ids,
                                                           float* __restrict__ gates,
-                                                          float* __restrict__ q_partial,
-                                                          int32_t* __restrict__ c_partial) {
+                                                          RouterAccum acc, float alpha,
+                                                          float* __restrict__ lb) {
   __shared__ float qs[8][MOE_MAX_EXPERTS];
   __shared__ int cs[MOE_MAX_EXPERTS];
+  __shared__ float prod[MOE_MAX_EXPERTS];
+  __shared__ int is_last;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int e = threadIdx.x; e < E; e += 256) cs[e] = 0;
   __syncthreads();
@@ -176,7 +192,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
       }
     }
   }
-  // fixed-order reduction of the per-warp partial sums of p
+  // block sums of p in a fixed order (warps ascending), then integer accumulation
 #pragma unroll
   for (int i = 0; i < EPL; ++i) {
     const int e = lane + 32 * i;
@@ -184,52 +200,32 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
   }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += 256) {
-    float s = 0.0f;
+    float sum = 0.0f;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) s += qs[w][e];
-    q_partial[(int64_t)blockIdx.x * E + e] = s;
-    c_partial[(int64_t)blockIdx.x * E + e] = cs[e];
+    for (int w = 0; w < 8; ++w) sum += qs[w][e];
+    const unsigned long long fx = (unsigned long long)llrint((double)sum * kQScale);
+    if (fx) atomicAdd(&acc.q[e], fx);
+    if (cs[e]) atomicAdd(&acc.c[e], (unsigned)cs[e]);
   }
-}
-
-// Thread (g, e) sums the partials of blocks g, g + G, g + 2G, ... of expert e; the G group sums
-// are then added in group order. G = 1024 / E groups; fixed assignment and order.
-__global__ void __launch_bounds__(1024) router_stats_kernel(const float* __restrict__ q_partial,
-                                                            const int32_t* __restrict__ c_partial,
-                                                            int64_t nblk, int64_t T, int E,
-                                                            float alpha, float* __restrict__ lb) {
-  __shared__ float sq[1024];
-  __shared__ int sc[1024];
-  __shared__ float prod[MOE_MAX_EXPERTS];
-  const int G = 1024 / E;
-  const int tid = threadIdx.x;
-  if (tid < G * E) {
-    const int g = tid / E, e = tid % E;
-    float q = 0.0f;
-    int c = 0;
-    for (int64_t b = g; b < nblk; b += G) {
-      q += q_partial[b * E + e];
-      c += c_partial[b * E + e];
-    }
-    sq[tid] = q;
-    sc[tid] = c;
+  if (lb == nullptr) return;
+  // the last block to finish turns the totals into f, Q, aux
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) is_last = atomicAdd(acc.ticket, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  for (int e = threadIdx.x; e < E; e += 256) {
+    const unsigned long long qf = atomicAdd(&acc.q[e], 0ull);
+    const unsigned cf = atomicAdd(&acc.c[e], 0u);
+    const float Q = (float)((double)qf / kQScale / (double)T);
+    const float f = (float)cf / (float)T;
+    lb[e] = f;
+    lb[E + e] = Q;
+    prod[e] = f * Q;
   }
   __syncthreads();
-  if (tid < E) {
-    float q = 0.0f;
-    int c = 0;
-    for (int g = 0; g < G; ++g) {
-      q += sq[g * E + tid];
-      c += sc[g * E + tid];
-    }
-    const float Q = q / (float)T;
-    const float f = (float)c / (float)T;
-    lb[tid] = f;
-    lb[E + tid] = Q;
-    prod[tid] = f * Q;
-  }
-  __syncthreads();
-  if (tid == 0) {
+  if (threadIdx.x == 0) {
     float s = 0.0f;
     for (int e = 0; e < E; ++e) s += prod[e];
     lb[2 * E] = alpha * (float)E * s;
@@ -238,9 +234,9 @@ __global__ void __launch_bounds__(1024) router_stats_kernel(const float* __restr
 
 template <int EPL>
 void launch_topk(const float* logits, int64_t T, int E, int k, int32_t* ids, float* gates,
-                 float* q_partial, int32_t* c_partial, cudaStream_t stream) {
+                 const RouterAccum& acc, float alpha, float* lb, cudaStream_t stream) {
   router_topk_kernel<EPL><<<(unsigned)router_num_blocks(T), 256, 0, stream>>>(
-      logits, T, E, k, ids, gates, q_partial, c_partial);
+      logits, T, E, k, ids, gates, acc, alpha, lb);
 }
 
 }  // namespace
@@ -250,12 +246,15 @@ cudaError_t enqueue_router(const void* x, bool x_bf16, int64_t T, int d, const f
                            float* gates, float* lb_stats, float aux_alpha,
                            const RouterScratch& scr, int* status, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
-  if (router_uses_tensor_cores(x_bf16, d)) {
-    const int dpad = router_split_dpad(d);
-    const int64_t n = (int64_t)E * dpad;
-    const unsigned blocks = (unsigned)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
-    router_split_kernel<<<blocks, 256, 0, stream>>>(w_router, E, d, dpad, scr.w_split);
-    count_launch();
+  if (!logits) logits = scr.logits_scratch;
+  const bool tc = router_uses_tensor_cores(x_bf16, d);
+  const int dpad = router_split_dpad(d);
+  const int64_t n = tc ? (int64_t)E * dpad : 0;
+  const unsigned blocks = (unsigned)(n == 0 ? 1 : ((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096));
+  router_prep_kernel<<<blocks, 256, 0, stream>>>(w_router, E, d, dpad, tc ? scr.w_split : nullptr,
+                                                 scr.acc);
+  count_launch();
+  if (tc) {
     cudaError_t e = enqueue_router_logits_tc(x, T, d, scr.w_split, dpad, router_bias, E, logits,
                                              status, stream);
     if (e != cudaSuccess) return e;
@@ -267,20 +266,14 @@ cudaError_t enqueue_router(const void* x, bool x_bf16, int64_t T, int d, const f
       router_logits_kernel<false><<<grid, 256, 0, stream>>>(x, w_router, router_bias, T, d, E, logits);
     count_launch();
   }
-  float* qp = scr.q_partial;
-  int32_t* cp = scr.c_partial;
-  if (E <= 32) launch_topk<1>(logits, T, E, k, ids, gates, qp, cp, stream);
-  else if (E <= 64) launch_topk<2>(logits, T, E, k, ids, gates, qp, cp, stream);
-  else if (E <= 128) launch_topk<4>(logits, T, E, k, ids, gates, qp, cp, stream);
-  else if (E <= 256) launch_topk<8>(logits, T, E, k, ids, gates, qp, cp, stream);
-  else if (E <= 512) launch_topk<16>(logits, T, E, k, ids, gates, qp, cp, stream);
-  else launch_topk<32>(logits, T, E, k, ids, gates, qp, cp, stream);
+  const RouterAccum& a = scr.acc;
+  if (E <= 32) launch_topk<1>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, stream);
+  else if (E <= 64) launch_topk<2>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, stream);
+  else if (E <= 128) launch_topk<4>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, stream);
+  else if (E <= 256) launch_topk<8>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, stream);
+  else if (E <= 512) launch_topk<16>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, stream);
+  else launch_topk<32>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, stream);
   count_launch();
-  if (lb_stats) {
-    router_stats_kernel<<<1, 1024, 0, stream>>>(qp, cp, router_num_blocks(T), T, E, aux_alpha,
-                                                lb_stats);
-    count_launch();
-  }
   return cudaGetLastError();
 }
 

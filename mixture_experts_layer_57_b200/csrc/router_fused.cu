@@ -1,0 +1,303 @@
+// Router logits on sm_100a tensor cores, token-major: logits[t, e] = x[t, :] . W_r[e, :] + b_r[e].
+//
+// DeepSpeed MoE blog, MoE formula p(x) = softmax(W_r x); comparison article, "Router computation"
+// (logits = x W_r).
+//
+// Arithmetic: x is bf16 and W_r (fp32) arrives split exactly into bf16 parts hi + mid + lo (each
+// holds the next 8 significant bits; router.cu), so x * W_r = x*hi + x*mid + x*lo is formed from
+// exact products and accumulated in fp32 by tcgen05.mma; b_r is added in fp32.
+//
+// Tile = 128 tokens x NE experts (one 128-expert slice of E, NE = the slice rounded up to a
+// power of two >= 16): the x tile is the MMA's A operand (M = 128, TMEM lane = token) and the three
+// weight parts are three B operands over the same A tile, so each x tile is read once per slice.
+// Roles per CTA (persistent over tiles, two TMEM accumulators):
+//     warp 0      TMA: x [128 x 64] and the three W parts [NE x 64] per stage, 128-byte swizzle
+//     warp 1      TMEM allocation; one thread issues 3 x 4 MMAs per stage
+//     warps 2..5  tcgen05.ld of 16-expert chunks, + bias, staged in shared memory and stored as
+//                 64-byte runs of a token's logits row (two tokens per warp store)
+// Bounded waits as in the grouped GEMM (MOE_DEVERR_TIMEOUT, drain, free TMEM).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+namespace {
+
+constexpr int kTM = 128;       // tokens per tile
+constexpr int kBK = 64;        // K per stage
+constexpr int kSlice = 128;    // experts per tile (at most)
+constexpr int kThreads = 192;  // 6 warps
+
+template <int NE>
+struct RCfg {
+  static constexpr int kABytes = kTM * kBK * 2;           // 16 KB
+  static constexpr int kBPartBytes = NE * kBK * 2;        // per weight part
+  static constexpr int kStageBytes = kABytes + 3 * kBPartBytes;
+  static constexpr int kStagesFit = (188 * 1024) / kStageBytes;
+  static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
+  static constexpr int kTmemCols = (2 * NE) < 32 ? 32 : (2 * NE);
+  static constexpr int kBarBytes = 8 * 32;
+  static constexpr int kStageTile = 32 * 16 * 4;          // per epilogue warp: 32 tokens x 16 fp32
+  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 4 * kStageTile + kBarBytes + 16;
+  static_assert(kStageBytes % 1024 == 0, "stage alignment");
+  static_assert(kStages >= 2, "pipeline depth");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+};
+
+struct RParams {
+  int64_t T;
+  int E, dpad, n_slices;
+  const float* bias;  // [E] fp32 or nullptr
+  float* logits;      // [T, E]
+  int* status;
+};
+
+__device__ __forceinline__ void mbar_wait_drain_r(uint32_t bar, uint32_t parity, int* status) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      set_device_error(status, MOE_DEVERR_TIMEOUT);
+      return;
+    }
+  }
+}
+
+template <int NE>
+__global__ void __launch_bounds__(kThreads, 1)
+    router_logits_tc_kernel(const __grid_constant__ CUtensorMap tmX,
+                            const __grid_constant__ CUtensorMap tmW, const RParams p) {
+  using C = RCfg<NE>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t base_addr = (raw_addr + 1023u) & ~1023u;
+  uint8_t* base = smem_raw + (base_addr - raw_addr);
+  uint8_t* stage_tiles = base + C::kStages * C::kStageBytes;
+  uint8_t* aux = stage_tiles + 4 * C::kStageTile;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(aux);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(aux + C::kBarBytes);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(aux + C::kBarBytes + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = C::kStages;
+  auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
+  auto empty_bar = [&](int s) { return smem_u32(&bars[S + s]); };
+  auto tfull_bar = [&](int a) { return smem_u32(&bars[2 * S + a]); };
+  auto tempty_bar = [&](int a) { return smem_u32(&bars[2 * S + 2 + a]); };
+  const uint32_t drain_bar = smem_u32(&bars[2 * S + 4]);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 128);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmW);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const int ntiles = (int)((p.T + kTM - 1) / kTM) * p.n_slices;
+  const int n_kb = p.dpad / kBK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0, issued = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        const int tok_tile = t / p.n_slices, slice = t % p.n_slices;
+        for (int kb = 0; kb < n_kb; ++kb) {
+          if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sa = base_addr + stage * C::kStageBytes;
+          mbar_arrive_expect_tx(full_bar(stage), C::kStageBytes);
+          tma_load_2d(sa, &tmX, kb * kBK, tok_tile * kTM, full_bar(stage));
+#pragma unroll
+          for (int part = 0; part < 3; ++part)
+            tma_load_2d(sa + C::kABytes + part * C::kBPartBytes, &tmW, part * p.dpad + kb * kBK,
+                        slice * kSlice, full_bar(stage));
+          ++issued;
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      for (int i = max(0, issued - S); i < issued; ++i)
+        mbar_wait_drain_r(full_bar(i % S), (uint32_t)((i / S) & 1), p.status);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      constexpr uint32_t idesc = idesc_bf16_f32(kTM, NE);
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        if (!mbar_wait_bounded(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * NE);
+        for (int kb = 0; kb < n_kb; ++kb) {
+          if (!mbar_wait_bounded(full_bar(stage), phase, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = base_addr + stage * C::kStageBytes;
+          const uint64_t adesc = smem_desc_sw128(sa);
+#pragma unroll
+          for (int part = 0; part < 3; ++part) {
+            const uint64_t bdesc = smem_desc_sw128(sa + C::kABytes + part * C::kBPartBytes);
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk)
+              tc_mma_bf16(d_tmem, adesc + (uint64_t)(2 * kk), bdesc + (uint64_t)(2 * kk), idesc,
+                          (kb | part | kk) != 0 ? 1u : 0u);
+          }
+          tc_commit(empty_bar(stage));
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(tfull_bar(acc));
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      tc_commit(drain_bar);
+      mbar_wait_drain_r(drain_bar, 0, p.status);
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue: logits rows
+    const int quarter = warp & 3;  // TMEM lanes (tokens) [32*quarter, 32*quarter + 32)
+    float* st = reinterpret_cast<float*>(stage_tiles + (warp - 2) * C::kStageTile);  // [32][16]
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+      const int tok_tile = t / p.n_slices, slice = t % p.n_slices;
+      if (!mbar_wait_bounded_warp(tfull_bar(acc), acc_phase, abort_flag, p.status)) break;
+      tc_fence_after();
+      const int64_t tok0 = (int64_t)tok_tile * kTM + quarter * 32;  // this warp's first token
+      const int e_base = slice * kSlice;
+      const int ne = min(NE, p.E - e_base);
+      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * NE);
+      for (int c0 = 0; c0 < ne; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld_32x32b_x16(taddr + (uint32_t)c0, r);
+        tmem_ld_wait();
+        // row = this lane's token, 16 experts; columns rotated by the row to spread banks
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const int e = e_base + c0 + c;
+          const float b = (p.bias && e < p.E) ? p.bias[e] : 0.0f;
+          st[lane * 16 + ((c + lane) & 15)] = __uint_as_float(r[c]) + b;
+        }
+        __syncwarp();
+        const int nc = min(16, ne - c0);
+        const int j = lane & 15;  // expert within the chunk
+#pragma unroll 4
+        for (int i = 0; i < 16; ++i) {
+          const int row = 2 * i + (lane >> 4);  // two tokens per store instruction
+          const int64_t tok = tok0 + row;
+          if (j < nc && tok < p.T)
+            p.logits[tok * p.E + e_base + c0 + j] = st[row * 16 + ((j + row) & 15)];
+        }
+        __syncwarp();
+      }
+      tc_fence_before();
+      mbar_arrive(tempty_bar(acc));
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+bool make_map(CUtensorMap* m, const void* ptr, int64_t rows, int K, int box_rows) {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(f);
+  }();
+  if (!fn) return false;
+  cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t gstride[1] = {(cuuint64_t)K * 2};
+  cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)box_rows};
+  cuuint32_t estride[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), gdim, gstride, box,
+            estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int NE>
+cudaError_t launch_tc(const CUtensorMap& tmX, const CUtensorMap& tmW, const RParams& p,
+                      int ntiles, cudaStream_t stream) {
+  auto kern = router_logits_tc_kernel<NE>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         RCfg<NE>::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int grid = ntiles < num_sms() ? ntiles : num_sms();
+  kern<<<grid, kThreads, RCfg<NE>::kSmemBytes, stream>>>(tmX, tmW, p);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t enqueue_router_logits_tc(const void* x, int64_t T, int d, const uint16_t* w_split,
+                                     int dpad, const float* router_bias, int E, float* logits,
+                                     int* status, cudaStream_t stream) {
+  if (T == 0) return cudaSuccess;
+  const int slice = E < kSlice ? E : kSlice;
+  int NE = 16;
+  while (NE < slice) NE <<= 1;  // instantiated N tiles: 16, 32, 64, 128
+  const int n_slices = (E + kSlice - 1) / kSlice;
+  CUtensorMap tmX, tmW;
+  if (!make_map(&tmX, x, T, d, kTM) || !make_map(&tmW, w_split, E, 3 * dpad, NE))
+    return cudaErrorInvalidValue;
+  const RParams p{T, E, dpad, n_slices, router_bias, logits, status};
+  const int ntiles = (int)((T + kTM - 1) / kTM) * n_slices;
+  switch (NE) {
+    case 16: return launch_tc<16>(tmX, tmW, p, ntiles, stream);
+    case 32: return launch_tc<32>(tmX, tmW, p, ntiles, stream);
+    case 64: return launch_tc<64>(tmX, tmW, p, ntiles, stream);
+    default: return launch_tc<128>(tmX, tmW, p, ntiles, stream);
+  }
+}
+
+}  // namespace moe

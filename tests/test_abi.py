@@ -56,7 +56,8 @@ def test_capacity_matches_oracle_formula(L):
 
 
 def test_workspace_queries(L):
-    assert moe.moe_router_workspace_bytes(16384, 128, 1024) >= 256 + 256 * 128 * 8 + 128 * 3 * 1024 * 2 + 16384 * 128 * 4
+    # status block + statistics accumulators + split weight (3 bf16 parts) + logits scratch
+    assert moe.moe_router_workspace_bytes(16384, 128, 1024) >= 256 + 128 * 12 + 128 * 3 * 1024 * 2 + 16384 * 128 * 4
     assert moe.moe_dispatch_workspace_bytes(16384, 128, 1) > 256
     assert moe.moe_expert_ffn_workspace_bytes() == 256
     assert moe.moe_combine_workspace_bytes() == 256

@@ -139,6 +139,6 @@ def test_determinism_bitwise(cuda_ok):
 def test_launch_count(cuda_ok):
     w = synth.WORKLOADS[3].with_(T=256, d_model=128, d_ff=256)
     got = run_layer(w, dev_inputs(synth.make_inputs(w)))
-    # router 4 (weight split, tensor-core logits, top-k, statistics), dispatch 3, dense MLP 2,
-    # experts 2, combine 1
-    assert got["launches"] == 12
+    # router 3 (prep: weight split + zeroed accumulators, tensor-core logits, top-k with the
+    # statistics), dispatch 3, dense MLP 2, experts 2, combine 1
+    assert got["launches"] == 11
