@@ -366,7 +366,8 @@ moe_status layer_layout(const moe_layer_args* a, uint8_t* base, LayerWs* w, size
   w->y_packed = c.take<float>((size_t)R * d);
   const bool dense = a->dense_w1 != nullptr;
   w->h_dense = dense ? (void*)c.take<uint8_t>((size_t)T * f * es) : nullptr;
-  w->r_dense = dense ? c.take<float>((size_t)T * d) : nullptr;
+  // the fp32 layers' dense output; bf16 layers fuse it into the combine epilogue
+  w->r_dense = (dense && a->dtype != MOE_BF16) ? c.take<float>((size_t)T * d) : nullptr;
   *bytes = c.off;
   return MOE_OK;
 }
@@ -418,19 +419,71 @@ moe_status moe_layer_forward(const moe_layer_args* a, void* out, moe_layer_aux* 
   cudaError_t e = enqueue_router(a->x, bf16, T, d, a->w_router, a->router_bias, E, k, logits, ids,
                                  gates, lb, a->aux_alpha, w.router.scr, status, stream);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
+
+  // bf16 layers fuse the combine into a layer-2 epilogue: the PR-MoE dense MLP's (any k, experts
+  // run first) or, without the dense branch, the top-1 experts' (dropped tokens are then written
+  // by dispatch). Other layers use the gather combine kernel.
+  const bool fuse_dense = bf16 && dense;
+  const bool fuse_expert = bf16 && !dense && k == 1;
+  const bool out_bf16 = a->out_dtype == MOE_BF16;
+  const void* residual = a->add_input_residual ? a->x : nullptr;
+  DroppedRows dropped;
+  if (fuse_expert) {
+    dropped.out = out;
+    dropped.out_bf16 = out_bf16;
+    dropped.add_x = a->add_input_residual != 0;
+  }
   e = enqueue_dispatch(a->x, bf16, T, d, ids, E, k, w.C, slot, counts, offsets, w.row_token,
                        w.x_packed, w.rows_max, w.dispatch.local_rank, w.dispatch.seg_counts,
-                       w.dispatch.seg_base, status, stream);
+                       w.dispatch.seg_base, status, stream, dropped);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
+
+  FusedCombine fc{};
+  fc.row_token = w.row_token;
+  fc.slot = slot;
+  fc.ids = ids;
+  fc.offsets = offsets;
+  fc.gates = gates;
+  fc.y = w.y_packed;
+  fc.rows_y = w.rows_max;
+  fc.residual = residual;
+  fc.out = out;
+  fc.out_bf16 = out_bf16;
+  fc.k = k;
+  fc.E_experts = E;
+
+  if (fuse_dense) {
+    if (w.rows_max > 0) {
+      e = enqueue_expert_ffn_bf16(w.x_packed, offsets, E, w.rows_max, d, f, a->w1, a->b1, a->w2,
+                                  a->b2, w.h_packed, w.y_packed, w.C, status, stream);
+      if (e != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    e = enqueue_grouped_gemm_bf16(a->x, nullptr, 1, T, d, f, a->dense_w1, a->dense_b1, true,
+                                  w.h_dense, T, status, stream);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    fc.dense = true;
+    e = enqueue_gemm2_combine(w.h_dense, nullptr, 1, T, f, d, a->dense_w2, a->dense_b2, fc, T,
+                              status, stream);
+    return cuda_status(e);
+  }
+  if (fuse_expert) {
+    if (w.rows_max > 0) {
+      e = enqueue_grouped_gemm_bf16(w.x_packed, offsets, E, w.rows_max, d, f, a->w1, a->b1, true,
+                                    w.h_packed, w.C, status, stream);
+      if (e != cudaSuccess) return MOE_ERR_CUDA;
+      fc.dense = false;
+      e = enqueue_gemm2_combine(w.h_packed, offsets, E, w.rows_max, f, d, a->w2, a->b2, fc, w.C,
+                                status, stream);
+      if (e != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    return MOE_OK;
+  }
   if (dense) {
-    // PR-MoE fixed MLP on every token: one "expert" whose segment is all T rows of x
-    e = bf16 ? enqueue_expert_ffn_bf16(a->x, nullptr, 1, T, d, f, a->dense_w1, a->dense_b1,
-                                       a->dense_w2, a->dense_b2, w.h_dense, w.r_dense, T, status,
-                                       stream)
-             : enqueue_expert_ffn_f32((const float*)a->x, nullptr, 1, T, d, f,
-                                      (const float*)a->dense_w1, (const float*)a->dense_b1,
-                                      (const float*)a->dense_w2, (const float*)a->dense_b2,
-                                      (float*)w.h_dense, w.r_dense, status, stream);
+    // fp32 PR-MoE: dense MLP on every token as one segment of all T rows of x
+    e = enqueue_expert_ffn_f32((const float*)a->x, nullptr, 1, T, d, f, (const float*)a->dense_w1,
+                               (const float*)a->dense_b1, (const float*)a->dense_w2,
+                               (const float*)a->dense_b2, (float*)w.h_dense, w.r_dense, status,
+                               stream);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
   }
   if (w.rows_max > 0) {
@@ -442,9 +495,8 @@ moe_status moe_layer_forward(const moe_layer_args* a, void* out, moe_layer_aux* 
                                       (float*)w.h_packed, w.y_packed, status, stream);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
   }
-  e = enqueue_combine(w.y_packed, offsets, ids, slot, gates, T, d, E, k, w.rows_max,
-                      a->add_input_residual ? a->x : nullptr, bf16, dense ? w.r_dense : nullptr,
-                      out, a->out_dtype == MOE_BF16, status, stream);
+  e = enqueue_combine(w.y_packed, offsets, ids, slot, gates, T, d, E, k, w.rows_max, residual, bf16,
+                      dense ? w.r_dense : nullptr, out, out_bf16, status, stream);
   return cuda_status(e);
 }
 

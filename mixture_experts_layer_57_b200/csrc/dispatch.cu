@@ -122,7 +122,7 @@ __global__ void __launch_bounds__(256)
                             const int32_t* __restrict__ seg_base,
                             const int32_t* __restrict__ offsets, int32_t* __restrict__ slot,
                             int32_t* __restrict__ row_token, uint8_t* __restrict__ x_packed,
-                            int64_t rows_max) {
+                            int64_t rows_max, DroppedRows dropped, int d) {
   const int lane = threadIdx.x & 31;
   const int64_t p = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (p >= pairs) return;
@@ -134,7 +134,21 @@ __global__ void __launch_bounds__(256)
     if (pos < C) s = pos;
   }
   if (lane == 0) slot[p] = s;
-  if (s < 0) return;
+  if (s < 0) {
+    if (dropped.out != nullptr) {
+      // top-1 with the combine fused into layer 2: this token's output is its residual alone
+      const int64_t t = p / k;
+      for (int64_t i = lane; i < d; i += 32) {
+        float v = 0.0f;
+        if (dropped.add_x)
+          v = row_bytes == (int64_t)d * 2 ? bf16_to_f32(reinterpret_cast<const uint16_t*>(x)[t * d + i])
+                                          : reinterpret_cast<const float*>(x)[t * d + i];
+        if (dropped.out_bf16) reinterpret_cast<uint16_t*>(dropped.out)[t * d + i] = f32_to_bf16_rn(v);
+        else reinterpret_cast<float*>(dropped.out)[t * d + i] = v;
+      }
+    }
+    return;
+  }
   const int64_t row = (int64_t)offsets[e] + s;
   if (row >= rows_max) return;  // cannot happen with rows_max >= min(T k, E C)
   const int64_t t = p / k;
@@ -153,7 +167,7 @@ cudaError_t enqueue_dispatch(const void* x, bool bf16, int64_t T, int d, const i
                              int k, int64_t C, int32_t* slot, int32_t* counts, int32_t* offsets,
                              int32_t* row_token, void* x_packed, int64_t rows_max,
                              int32_t* local_rank, int32_t* seg_counts, int32_t* seg_base,
-                             int* status, cudaStream_t stream) {
+                             int* status, cudaStream_t stream, DroppedRows dropped) {
   const int64_t pairs = T * k;
   const int64_t nseg = dispatch_num_segments(pairs);
   if (pairs > 0) {
@@ -172,15 +186,15 @@ cudaError_t enqueue_dispatch(const void* x, bool bf16, int64_t T, int d, const i
     if (row_bytes % 16 == 0)
       dispatch_scatter_kernel<16><<<blocks, 256, 0, stream>>>(xs, row_bytes, pairs, k, E, C, ids,
                                                               local_rank, seg_base, offsets, slot,
-                                                              row_token, xp, rows_max);
+                                                              row_token, xp, rows_max, dropped, d);
     else if (row_bytes % 8 == 0)
       dispatch_scatter_kernel<8><<<blocks, 256, 0, stream>>>(xs, row_bytes, pairs, k, E, C, ids,
                                                              local_rank, seg_base, offsets, slot,
-                                                             row_token, xp, rows_max);
+                                                             row_token, xp, rows_max, dropped, d);
     else
       dispatch_scatter_kernel<4><<<blocks, 256, 0, stream>>>(xs, row_bytes, pairs, k, E, C, ids,
                                                              local_rank, seg_base, offsets, slot,
-                                                             row_token, xp, rows_max);
+                                                             row_token, xp, rows_max, dropped, d);
     count_launch();
   }
   return cudaGetLastError();

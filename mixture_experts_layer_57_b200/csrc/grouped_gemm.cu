@@ -44,6 +44,11 @@ constexpr int kStageTileBytes = 16 * 32 * 4;  // per epilogue warp: 16 tokens x 
 // Epilogue kinds.
 constexpr int kEpiGeluBf16 = 0;  // out = bf16(GeLU(acc + bias)), bias bf16   (expert layer 1)
 constexpr int kEpiF32 = 1;       // out = acc + bias (fp32), bias bf16          (expert layer 2)
+// Layer 2 with the combine fused (see CombineArgs): y = acc + bias stays in registers and the
+// epilogue writes the layer output row of the token instead of y.
+constexpr int kEpiCombineExpert = 2;  // top-1: out[token(r)] = [x] + gate * y[r]
+constexpr int kEpiCombineDense = 3;   // PR-MoE dense MLP, row = token t:
+                                      // out[t] = [x] + y_dense[t] + sum_j gate_j * y_expert[row_j]
 
 template <int BN>
 struct Cfg {
@@ -63,6 +68,21 @@ struct Cfg {
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 
+// Operands of the fused combine epilogues. The arithmetic is the combine kernel's, in its order:
+// acc = [x] + [y_dense]; acc = fma(gate_j, y_j, acc) for the kept choices j ascending; one rounding.
+struct CombineArgs {
+  const int32_t* row_token;  // [rows] token of each packed row (expert mode)
+  const int32_t* slot;       // [T, k] (dense mode)
+  const int32_t* ids;        // [T, k] (dense mode)
+  const int32_t* offsets;    // [E_experts + 1] (dense mode)
+  const float* gates;        // [T, k]
+  const float* y;            // [rows_y, n_out] fp32 expert outputs (dense mode)
+  const uint16_t* residual;  // [T, n_out] bf16 x, or nullptr
+  void* out;                 // [T, n_out] bf16 or fp32
+  int out_bf16, k, E_experts;
+  int64_t rows_y;            // rows of y (bounds check)
+};
+
 struct Params {
   const int32_t* offsets;  // [E+1], or nullptr: one segment [0, rows_max) (E == 1)
   int E;
@@ -72,6 +92,7 @@ struct Params {
   const void* bias;        // [E, n_out] bf16, or nullptr
   void* out;               // [rows_max, n_out]: bf16 (GeLU layer) or fp32
   int* status;
+  CombineArgs cmb;         // used by the combine epilogues only
 };
 
 struct Tile {
@@ -322,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   *reinterpret_cast<const uint4*>(st + row * 64 + q * 16);
           }
           __syncwarp();
-        } else {
+        } else if constexpr (EPI == kEpiF32) {
           // stage [16 tokens][32 features] fp32, then 16-byte stores of 4 features of one token
           float* s32 = reinterpret_cast<float*>(st);
 #pragma unroll
@@ -336,6 +357,76 @@ __global__ void __launch_bounds__(kThreads, 1)
               *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) +
                                          (int64_t)(tl.row0 + c0 + row) * p.n_out + ff) =
                   *reinterpret_cast<const float4*>(st + row * 128 + q * 16);
+          }
+          __syncwarp();
+        } else {
+          // fused combine: y (or the dense MLP output) = acc + bias staged as fp32 [16][32]; each
+          // lane then finishes 4 features of one token row of the layer output
+          const CombineArgs& cb = p.cmb;
+          float* s32 = reinterpret_cast<float*>(st);
+#pragma unroll
+          for (int c = 0; c < 16; ++c) s32[c * 32 + lane] = __uint_as_float(r[c]) + bv;
+          __syncwarp();
+#pragma unroll
+          for (int id = lane; id < 128; id += 32) {
+            const int row = id >> 3, q = id & 7;
+            const int ff = fw + 4 * q;
+            if (row < nc && ff < p.n_out) {
+              const int64_t pr = (int64_t)(tl.row0 + c0 + row);  // packed row (dense: token)
+              const float4 v = *reinterpret_cast<const float4*>(st + row * 128 + q * 16);
+              int64_t t;
+              float a[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+              if constexpr (EPI == kEpiCombineExpert) {
+                t = cb.row_token[pr];
+              } else {
+                t = pr;
+              }
+              if (cb.residual) {
+                const uint2 rb = *reinterpret_cast<const uint2*>(cb.residual + t * p.n_out + ff);
+                a[0] = __uint_as_float(rb.x << 16);
+                a[1] = __uint_as_float(rb.x & 0xffff0000u);
+                a[2] = __uint_as_float(rb.y << 16);
+                a[3] = __uint_as_float(rb.y & 0xffff0000u);
+              }
+              if constexpr (EPI == kEpiCombineExpert) {
+                const float g = cb.gates[t];
+                a[0] = fmaf(g, v.x, a[0]);
+                a[1] = fmaf(g, v.y, a[1]);
+                a[2] = fmaf(g, v.z, a[2]);
+                a[3] = fmaf(g, v.w, a[3]);
+              } else {
+                a[0] += v.x;
+                a[1] += v.y;
+                a[2] += v.z;
+                a[3] += v.w;
+                for (int j = 0; j < cb.k; ++j) {
+                  const int sl = cb.slot[t * cb.k + j];
+                  if (sl < 0) continue;
+                  const int e = cb.ids[t * cb.k + j];
+                  if (e < 0 || e >= cb.E_experts) continue;
+                  const int64_t yr = (int64_t)cb.offsets[e] + sl;
+                  if (yr >= cb.rows_y) {
+                    set_device_error(p.status, MOE_DEVERR_BAD_ROW);
+                    continue;
+                  }
+                  const float g = cb.gates[t * cb.k + j];
+                  const float4 y = *reinterpret_cast<const float4*>(cb.y + yr * p.n_out + ff);
+                  a[0] = fmaf(g, y.x, a[0]);
+                  a[1] = fmaf(g, y.y, a[1]);
+                  a[2] = fmaf(g, y.z, a[2]);
+                  a[3] = fmaf(g, y.w, a[3]);
+                }
+              }
+              if (cb.out_bf16) {
+                uint2 o;
+                o.x = (uint32_t)f32_to_bf16_rn(a[0]) | ((uint32_t)f32_to_bf16_rn(a[1]) << 16);
+                o.y = (uint32_t)f32_to_bf16_rn(a[2]) | ((uint32_t)f32_to_bf16_rn(a[3]) << 16);
+                *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(cb.out) + t * p.n_out + ff) = o;
+              } else {
+                *reinterpret_cast<float4*>(reinterpret_cast<float*>(cb.out) + t * p.n_out + ff) =
+                    make_float4(a[0], a[1], a[2], a[3]);
+              }
+            }
           }
           __syncwarp();
         }
@@ -438,9 +529,26 @@ cudaError_t enqueue_grouped_gemm_bf16(const void* x, const int32_t* offsets, int
   CUtensorMap tmW, tmX;
   if (!make_kmajor_map(&tmW, w, (int64_t)E * N, K, kBM) || !make_kmajor_map(&tmX, x, rows_max, K, BN))
     return cudaErrorInvalidValue;
-  const Params p{offsets, E, N, K, rows_max, bias, out, status};
+  Params p{offsets, E, N, K, rows_max, bias, out, status, CombineArgs{}};
   return gelu ? launch_bn<kEpiGeluBf16>(BN, tmW, tmX, p, stream)
               : launch_bn<kEpiF32>(BN, tmW, tmX, p, stream);
+}
+
+cudaError_t enqueue_gemm2_combine(const void* h, const int32_t* offsets, int E, int64_t rows_max,
+                                  int K, int N, const void* w, const void* bias,
+                                  const FusedCombine& fc, int64_t capacity_hint, int* status,
+                                  cudaStream_t stream) {
+  if (rows_max == 0) return cudaSuccess;
+  const int BN = pick_token_tile(capacity_hint);
+  CUtensorMap tmW, tmX;
+  if (!make_kmajor_map(&tmW, w, (int64_t)E * N, K, kBM) || !make_kmajor_map(&tmX, h, rows_max, K, BN))
+    return cudaErrorInvalidValue;
+  CombineArgs c{fc.row_token, fc.slot, fc.ids, fc.offsets, fc.gates, fc.y,
+                (const uint16_t*)fc.residual, fc.out, fc.out_bf16 ? 1 : 0, fc.k, fc.E_experts,
+                fc.rows_y};
+  Params p{offsets, E, N, K, rows_max, bias, nullptr, status, c};
+  return fc.dense ? launch_bn<kEpiCombineDense>(BN, tmW, tmX, p, stream)
+                  : launch_bn<kEpiCombineExpert>(BN, tmW, tmX, p, stream);
 }
 
 cudaError_t enqueue_expert_ffn_bf16(const void* x_packed, const int32_t* offsets, int E,

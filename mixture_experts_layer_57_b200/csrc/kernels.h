@@ -51,11 +51,18 @@ constexpr int kDispatchSeg = 256;  // (token, choice) pairs per counting segment
 inline int64_t dispatch_num_segments(int64_t pairs) {
   return (pairs + kDispatchSeg - 1) / kDispatchSeg;
 }
+// dropped_out (optional, top-1 layers whose combine is fused into layer 2): for every token whose
+// only choice overflowed, writes out[t] = x[t] (dropped_add_x) or 0, in the output type.
+struct DroppedRows {
+  void* out = nullptr;
+  bool out_bf16 = true;
+  bool add_x = true;
+};
 cudaError_t enqueue_dispatch(const void* x, bool bf16, int64_t T, int d, const int32_t* ids, int E,
                              int k, int64_t C, int32_t* slot, int32_t* counts, int32_t* offsets,
                              int32_t* row_token, void* x_packed, int64_t rows_max,
                              int32_t* local_rank, int32_t* seg_counts, int32_t* seg_base,
-                             int* status, cudaStream_t stream);
+                             int* status, cudaStream_t stream, DroppedRows dropped = DroppedRows{});
 
 // ---------------------------------------------------------------- expert FFN
 // One grouped GEMM layer: out = act(W[e] x + bias[e]) over every expert segment. offsets ==
@@ -69,6 +76,29 @@ cudaError_t enqueue_grouped_gemm_f32(const float* x, const int32_t* offsets, int
                                      int64_t rows_max, int K, int N, const float* w,
                                      const float* bias, bool gelu, float* out, int* status,
                                      cudaStream_t stream);
+// Layer 2 with the combine fused into its epilogue (bf16 layers):
+//   dense == false: top-1 experts; row r of the packed buffer belongs to token row_token[r]:
+//                   out[t] = [residual[t]] + gates[t] * (W2[e] h[r] + b2[e])
+//   dense == true:  the PR-MoE dense MLP's layer 2 over all T tokens (offsets == nullptr, E == 1):
+//                   out[t] = [residual[t]] + (W2d h[t] + b2d) + sum_{j kept} gates[t,j] * y[row_j]
+struct FusedCombine {
+  bool dense;
+  const int32_t* row_token;
+  const int32_t* slot;
+  const int32_t* ids;
+  const int32_t* offsets;   // expert offsets (dense mode)
+  const float* gates;
+  const float* y;           // expert outputs [rows_y, d] (dense mode)
+  int64_t rows_y;
+  const void* residual;     // bf16 x or nullptr
+  void* out;
+  bool out_bf16;
+  int k, E_experts;
+};
+cudaError_t enqueue_gemm2_combine(const void* h, const int32_t* offsets, int E, int64_t rows_max,
+                                  int K, int N, const void* w, const void* bias,
+                                  const FusedCombine& fc, int64_t capacity_hint, int* status,
+                                  cudaStream_t stream);
 cudaError_t enqueue_expert_ffn_bf16(const void* x_packed, const int32_t* offsets, int E,
                                     int64_t rows_max, int d, int d_ff, const void* w1,
                                     const void* b1, const void* w2, const void* b2, void* h_packed,

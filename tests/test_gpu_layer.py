@@ -101,6 +101,8 @@ def test_prmoe_both_residual_conventions(cuda_ok):
     ("C>=Tk", dict(capacity_factor=1000.0)),
     ("ragged T", dict(T=1001)),
     ("E=1", dict(E=1, k=1)),
+    ("top1 C=0", dict(k=1, capacity_factor=0.0)),
+    ("top1 ragged T", dict(k=1, T=777, capacity_factor=0.7)),
 ])
 def test_edge_cases(cuda_ok, name, kw):
     base = dict(T=200, d_model=128, d_ff=256, E=8, k=2, capacity_factor=1.0, dtype="bf16",
@@ -108,8 +110,20 @@ def test_edge_cases(cuda_ok, name, kw):
     base.update(kw)
     w = synth.Workload("edge", **base)
     r = layer_parity(w)
-    if name == "C=0":
+    if name in ("C=0", "top1 C=0"):
         assert np.array_equal(r["got"]["out"], synth.make_inputs(w)["x"])
+
+
+@pytest.mark.parametrize("k,res,out32", [(1, False, False), (1, False, True), (1, True, True),
+                                         (2, False, False)])
+def test_residual_and_output_type_variants(cuda_ok, k, res, out32):
+    w = synth.Workload("variants", T=333, d_model=128, d_ff=256, E=8, k=k, capacity_factor=0.8,
+                       dtype="bf16", w_router_std=0.1, w_std=0.05, b_std=0.05, seed=79)
+    r = layer_parity(w, add_input_residual=res, out_dtype=torch.float32 if out32 else None)
+    dropped = (r["got"]["slot"] < 0).all(1)
+    assert dropped.any()
+    if not res:   # a token dropped by every choice has no residual: its output is zero
+        assert np.all(r["got"]["out"][dropped] == 0)
 
 
 def test_all_tokens_to_one_expert(cuda_ok):
@@ -140,5 +154,11 @@ def test_launch_count(cuda_ok):
     w = synth.WORKLOADS[3].with_(T=256, d_model=128, d_ff=256)
     got = run_layer(w, dev_inputs(synth.make_inputs(w)))
     # router 3 (prep: weight split + zeroed accumulators, tensor-core logits, top-k with the
-    # statistics), dispatch 3, dense MLP 2, experts 2, combine 1
-    assert got["launches"] == 11
+    # statistics), dispatch 3, experts 2, dense MLP 2 (its layer 2 carries the combine)
+    assert got["launches"] == 10
+    w1 = synth.WORKLOADS[2].with_(T=256, d_model=128, d_ff=256)
+    got = run_layer(w1, dev_inputs(synth.make_inputs(w1)))
+    assert got["launches"] == 8      # top-1: the combine is fused into the experts' layer 2
+    w2 = synth.WORKLOADS[4].with_(T=256, d_model=128, d_ff=256)
+    got = run_layer(w2, dev_inputs(synth.make_inputs(w2)))
+    assert got["launches"] == 9      # top-2: gather combine kernel
