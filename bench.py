@@ -348,40 +348,51 @@ def main():
                "experts_touched": E_t, "max_expert_demand": int(counts.max()),
                "capacity": moe.moe_capacity(T, E, k, w.capacity_factor), "aux_loss": float(lb[-1])}
 
-    # ---------------------------------------------------------- per-kernel breakdown
-    bd = breakdown(moe, w, d, ws, stream, flush_buf, reps=max(3, min(20, args.steps)))
+    # ---------------------------------------------------------- per-stage breakdown
+    bd = stage_breakdown(moe, args_c, out, aux, ws, stream, flush_buf, reps=max(3, min(20, args.steps)))
     es = 2 if bf16 else 4
-    gemm_bytes = {
-        "gemm1": E_t * df * dm * es + E_t * df * es + R * dm * es + R * df * es,
-        "gemm2": E_t * dm * df * es + E_t * dm * es + R * df * es + R * dm * 4,
+    res_b = es if w.add_input_residual else 0
+    out_b = es
+    stage_bytes = {
+        "expert_gemm1": E_t * df * dm * es + E_t * df * es + R * dm * es + R * df * es,
+        "expert_gemm2": E_t * dm * df * es + E_t * dm * es + R * df * es + R * dm * 4,
+        "expert_gemm2_combine": (E_t * dm * df * es + E_t * dm * es + R * df * es + R * 8
+                                 + R * dm * (res_b + out_b)),
+        "dense_gemm1": df * dm * es + df * es + T * dm * es + T * df * es,
+        "dense_gemm2_combine": (dm * df * es + dm * es + T * df * es + T * k * 12 + R * dm * 4
+                                + T * dm * (res_b + out_b)),
     }
-    gemm_flops = {"gemm1": 2.0 * R * dm * df, "gemm2": 2.0 * R * dm * df}
-    if w.dense:
-        gemm_bytes["dense_gemm1"] = df * dm * es + df * es + T * dm * es + T * df * es
-        gemm_bytes["dense_gemm2"] = dm * df * es + dm * es + T * df * es + T * dm * 4
-        gemm_flops["dense_gemm1"] = gemm_flops["dense_gemm2"] = 2.0 * T * dm * df
+    stage_flops = {n: 2.0 * (T if n.startswith("dense") else R) * dm * df for n in stage_bytes}
     peaks, peak_src = load_peaks()
-    dom = max((n for n in bd if n in gemm_bytes), key=lambda n: bd[n])
+    gemm_stages = [n for n in bd if n in stage_bytes]
+    dom = max(gemm_stages, key=lambda n: bd[n])
     t_dom = bd[dom] / 1e3
-    ai = gemm_flops[dom] / gemm_bytes[dom]
+    ai = stage_flops[dom] / stage_bytes[dom]
     ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
-    kernel_name = {"gemm1": "grouped_gemm (layer 1, bias+GeLU epilogue)",
-                   "gemm2": "grouped_gemm (layer 2, bias epilogue)",
-                   "dense_gemm1": "dense MLP layer 1", "dense_gemm2": "dense MLP layer 2"}[dom]
+    kernel_name = {"expert_gemm1": "grouped_gemm (expert layer 1, bias+GeLU epilogue)",
+                   "expert_gemm2": "grouped_gemm (expert layer 2, bias epilogue)",
+                   "expert_gemm2_combine": "grouped_gemm (expert layer 2, bias + fused combine epilogue)",
+                   "dense_gemm1": "grouped_gemm (dense MLP layer 1, bias+GeLU epilogue)",
+                   "dense_gemm2_combine": "grouped_gemm (dense MLP layer 2, bias + fused combine epilogue)"}[dom]
     traffic, _ = profiled_traffic(w.name, dom)
     if ai < ridge:
-        roof = {"kernel": kernel_name, "bound": "hbm", "achieved": gemm_bytes[dom] / t_dom / 1e9,
+        roof = {"kernel": kernel_name, "bound": "hbm", "achieved": stage_bytes[dom] / t_dom / 1e9,
                 "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     else:
-        roof = {"kernel": kernel_name, "bound": "tensor", "achieved": gemm_flops[dom] / t_dom / 1e12,
-                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+        roof = {"kernel": kernel_name, "bound": "tensor",
+                "achieved": stage_flops[dom] / t_dom / 1e12, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = traffic
-    roof["algorithmic_bytes"] = gemm_bytes[dom]
-    roof["algorithmic_flops"] = gemm_flops[dom]
-    roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
-    roof["tensor_frac"] = gemm_flops[dom] / t_dom / 1e12 / peaks["bf16_tflops"]
-    roof["hbm_frac"] = gemm_bytes[dom] / t_dom / 1e9 / peaks["hbm_gbs"]
+    roof["algorithmic_bytes"] = stage_bytes[dom]
+    roof["algorithmic_flops"] = stage_flops[dom]
+    roof["launch_ms"] = bd[dom]
+    roof["peak_source"] = "measured (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
+    roof["tensor_frac"] = stage_flops[dom] / t_dom / 1e12 / peaks["bf16_tflops"]
+    roof["hbm_frac"] = stage_bytes[dom] / t_dom / 1e9 / peaks["hbm_gbs"]
+    roof["per_stage"] = {n: {"ms": bd[n], "GB/s": stage_bytes[n] / (bd[n] / 1e3) / 1e9,
+                             "TFLOP/s": stage_flops[n] / (bd[n] / 1e3) / 1e12}
+                         for n in gemm_stages}
 
     # ---------------------------------------------------------- end to end through the API
     e2e = None
@@ -419,73 +430,18 @@ def main():
     return 0
 
 
-def breakdown(moe, w, d, ws_layer, stream, flush_buf, reps: int) -> dict:
-    """Median event time (ms) of each entry point of the pipeline, run one by one as the layer
-    forward runs them (same kernels, same order)."""
-    dev = d["x"].device
-    T, E, k, dm, df = w.T, w.E, w.k, w.d_model, w.d_ff
-    C = moe.moe_capacity(T, E, k, w.capacity_factor)
-    R = moe.moe_packed_rows_max(T, E, k, C)
-    logits = torch.empty(T, E, dtype=torch.float32, device=dev)
-    ids = torch.empty(T, k, dtype=torch.int32, device=dev)
-    gates = torch.empty(T, k, dtype=torch.float32, device=dev)
-    lb = torch.empty(2 * E + 1, dtype=torch.float32, device=dev)
-    ws_r = moe.workspace(moe.moe_router_workspace_bytes(T, E, dm), dev)
-    ws_d = moe.workspace(moe.moe_dispatch_workspace_bytes(T, E, k), dev)
-    ws_s = moe.workspace(256, dev)
-    slot = torch.empty(T, k, dtype=torch.int32, device=dev)
-    cnt = torch.empty(E, dtype=torch.int32, device=dev)
-    off = torch.empty(E + 1, dtype=torch.int32, device=dev)
-    rt = torch.empty(max(R, 1), dtype=torch.int32, device=dev)
-    xp = torch.empty(max(R, 1), dm, dtype=d["x"].dtype, device=dev)
-    hp = torch.empty(max(R, 1), df, dtype=d["x"].dtype, device=dev)
-    yp = torch.empty(max(R, 1), dm, dtype=torch.float32, device=dev)
-    out = torch.empty(T, dm, dtype=d["x"].dtype, device=dev)
-    dense_on = w.dense
-    if dense_on:
-        hd = torch.empty(T, df, dtype=d["x"].dtype, device=dev)
-        rd = torch.empty(T, dm, dtype=torch.float32, device=dev)
-        one_seg = torch.tensor([0, T], dtype=torch.int32, device=dev)
-
-    stages = [
-        ("router", lambda: moe.moe_router_topk(d["x"], d["w_router"], k, router_bias=d.get("router_bias"),
-                                               logits=logits, expert_ids=ids, gates=gates, lb_stats=lb,
-                                               aux_alpha=w.aux_alpha, ws=ws_r, stream=stream)),
-        ("dispatch", lambda: moe.moe_dispatch(d["x"], ids, E, C, rows_max=R, slot=slot, expert_counts=cnt,
-                                              expert_offsets=off, row_token=rt, x_packed=xp, ws=ws_d,
-                                              stream=stream)),
-    ]
-    if dense_on:
-        stages += [
-            ("dense_gemm1", lambda: moe.moe_grouped_gemm(d["x"], one_seg, d["dense_w1"][None], d["dense_b1"][None],
-                                                         gelu=True, rows_max=T, capacity_hint=T, out=hd,
-                                                         ws=ws_s, stream=stream)),
-            ("dense_gemm2", lambda: moe.moe_grouped_gemm(hd, one_seg, d["dense_w2"][None], d["dense_b2"][None],
-                                                         gelu=False, rows_max=T, capacity_hint=T, out=rd,
-                                                         ws=ws_s, stream=stream)),
-        ]
-    stages += [
-        ("gemm1", lambda: moe.moe_grouped_gemm(xp, off, d["w1"], d["b1"], gelu=True, rows_max=R,
-                                               capacity_hint=C, out=hp, ws=ws_s, stream=stream)),
-        ("gemm2", lambda: moe.moe_grouped_gemm(hp, off, d["w2"], d["b2"], gelu=False, rows_max=R,
-                                               capacity_hint=C, out=yp, ws=ws_s, stream=stream)),
-        ("combine", lambda: moe.moe_combine(yp, off, ids, slot, gates,
-                                            residual=d["x"] if w.add_input_residual else None,
-                                            dense=rd if dense_on else None, out=out, rows_max=R,
-                                            ws=ws_s, stream=stream)),
-    ]
-    times = {n: [] for n, _ in stages}
+def stage_breakdown(moe, args_c, out, aux, ws, stream, flush_buf, reps: int) -> dict:
+    """Median time (ms) of each stage of moe_layer_forward, from CUDA events the library records
+    at its stage boundaries (moe_layer_forward_profiled), L2 flushed before each repetition."""
+    times = {}
     for _ in range(reps):
         flush_buf.zero_()
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)]
-        ev[0].record(stream)
-        for i, (_, fn) in enumerate(stages):
-            fn()
-            ev[i + 1].record(stream)
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(12)]
+        names = moe.moe_layer_forward_profiled(args_c, out, evs, aux=aux, ws=ws, stream=stream)
         torch.cuda.synchronize()
-        for i, (n, _) in enumerate(stages):
-            times[n].append(ev[i].elapsed_time(ev[i + 1]))
-    assert moe.moe_get_device_error(ws_s) == 0
+        for i in range(1, len(names)):
+            times.setdefault(names[i], []).append(evs[i - 1].elapsed_time(evs[i]))
+    assert moe.moe_get_device_error(ws) == 0
     return {n: float(np.median(v)) for n, v in times.items()}
 
 

@@ -233,6 +233,17 @@ moe_status moe_layer_workspace_bytes(const moe_layer_args* args, size_t* bytes);
 moe_status moe_layer_forward(const moe_layer_args* args, void* out, moe_layer_aux* aux, void* ws,
                              size_t ws_bytes, moe_stream_t stream);
 
+/* moe_layer_forward that also records caller-created CUDA events (cudaEvent_t handles passed as
+ * void*) on `stream` at stage boundaries: events[0] before the first kernel, then one after each
+ * stage ("router", "dispatch", "expert_gemm1", "expert_gemm2" or "expert_gemm2_combine",
+ * "dense_gemm1", "dense_gemm2_combine", "dense_ffn", "combine", as the layer's path has them).
+ * *n_events receives the number recorded (at most max_events); `names` (may be NULL) receives the
+ * comma-separated labels, starting with "start". Results are identical to moe_layer_forward. */
+moe_status moe_layer_forward_profiled(const moe_layer_args* args, void* out, moe_layer_aux* aux,
+                                      void* ws, size_t ws_bytes, moe_stream_t stream,
+                                      void* const* events, int max_events, int* n_events,
+                                      char* names, size_t names_len);
+
 /* ---------------------------------------------------------------- status block
  * moe_workspace_reset: zeroes the status block (asynchronous on stream).
  * moe_get_device_error: synchronises `stream`, copies the status word to *code_out and returns

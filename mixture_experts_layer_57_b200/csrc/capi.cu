@@ -16,6 +16,14 @@ thread_local int g_launches = 0;
 void count_launch() { ++g_launches; }
 void reset_launch_count() { g_launches = 0; }
 
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* v = std::getenv("MOE_PDL");
+    return !(v != nullptr && v[0] == '0');
+  }();
+  return on;
+}
+
 int num_sms() {
   static int cache[64] = {0};
   int dev = 0;
@@ -380,8 +388,37 @@ moe_status moe_layer_workspace_bytes(const moe_layer_args* args, size_t* bytes) 
   return layer_layout(args, nullptr, &w, bytes);
 }
 
-moe_status moe_layer_forward(const moe_layer_args* a, void* out, moe_layer_aux* aux, void* ws,
-                             size_t ws_bytes, moe_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Records caller-created CUDA events at stage boundaries (moe_layer_forward_profiled).
+struct StageRecorder {
+  void* const* events = nullptr;
+  int max_events = 0;
+  int n = 0;
+  char* names = nullptr;
+  size_t names_len = 0;
+  size_t used = 0;
+  cudaStream_t stream = nullptr;
+  void mark(const char* name) {
+    if (events == nullptr || n >= max_events) return;
+    cudaEventRecord((cudaEvent_t)events[n], stream);
+    ++n;
+    if (names != nullptr && names_len > 0) {
+      const size_t len = std::strlen(name);
+      if (used + len + 2 <= names_len) {
+        if (used > 0) names[used++] = ',';
+        std::memcpy(names + used, name, len);
+        used += len;
+        names[used] = '\0';
+      }
+    }
+  }
+};
+
+moe_status layer_forward_impl(const moe_layer_args* a, void* out, moe_layer_aux* aux, void* ws,
+                              size_t ws_bytes, moe_stream_t stream, StageRecorder& rec) {
   LayerWs w;
   size_t need = 0;
   moe_status st = layer_layout(a, (uint8_t*)ws, &w, &need);
@@ -416,9 +453,12 @@ moe_status moe_layer_forward(const moe_layer_args* a, void* out, moe_layer_aux* 
   const int64_t T = a->T;
   const int d = a->d_model, f = a->d_ff, E = a->E, k = a->k;
 
+  rec.stream = stream;
+  rec.mark("start");
   cudaError_t e = enqueue_router(a->x, bf16, T, d, a->w_router, a->router_bias, E, k, logits, ids,
                                  gates, lb, a->aux_alpha, w.router.scr, status, stream);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
+  rec.mark("router");
 
   // bf16 layers fuse the combine into a layer-2 epilogue: the PR-MoE dense MLP's (any k, experts
   // run first) or, without the dense branch, the top-1 experts' (dropped tokens are then written
@@ -437,6 +477,7 @@ moe_status moe_layer_forward(const moe_layer_args* a, void* out, moe_layer_aux* 
                        w.x_packed, w.rows_max, w.dispatch.local_rank, w.dispatch.seg_counts,
                        w.dispatch.seg_base, status, stream, dropped);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
+  rec.mark("dispatch");
 
   FusedCombine fc{};
   fc.row_token = w.row_token;
@@ -454,27 +495,37 @@ moe_status moe_layer_forward(const moe_layer_args* a, void* out, moe_layer_aux* 
 
   if (fuse_dense) {
     if (w.rows_max > 0) {
-      e = enqueue_expert_ffn_bf16(w.x_packed, offsets, E, w.rows_max, d, f, a->w1, a->b1, a->w2,
-                                  a->b2, w.h_packed, w.y_packed, w.C, status, stream);
+      e = enqueue_grouped_gemm_bf16(w.x_packed, offsets, E, w.rows_max, d, f, a->w1, a->b1, true,
+                                    w.h_packed, w.C, status, stream);
       if (e != cudaSuccess) return MOE_ERR_CUDA;
+      rec.mark("expert_gemm1");
+      e = enqueue_grouped_gemm_bf16(w.h_packed, offsets, E, w.rows_max, f, d, a->w2, a->b2, false,
+                                    w.y_packed, w.C, status, stream);
+      if (e != cudaSuccess) return MOE_ERR_CUDA;
+      rec.mark("expert_gemm2");
     }
     e = enqueue_grouped_gemm_bf16(a->x, nullptr, 1, T, d, f, a->dense_w1, a->dense_b1, true,
                                   w.h_dense, T, status, stream);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
+    rec.mark("dense_gemm1");
     fc.dense = true;
     e = enqueue_gemm2_combine(w.h_dense, nullptr, 1, T, f, d, a->dense_w2, a->dense_b2, fc, T,
                               status, stream);
-    return cuda_status(e);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    rec.mark("dense_gemm2_combine");
+    return MOE_OK;
   }
   if (fuse_expert) {
     if (w.rows_max > 0) {
       e = enqueue_grouped_gemm_bf16(w.x_packed, offsets, E, w.rows_max, d, f, a->w1, a->b1, true,
                                     w.h_packed, w.C, status, stream);
       if (e != cudaSuccess) return MOE_ERR_CUDA;
+      rec.mark("expert_gemm1");
       fc.dense = false;
       e = enqueue_gemm2_combine(w.h_packed, offsets, E, w.rows_max, f, d, a->w2, a->b2, fc, w.C,
                                 status, stream);
       if (e != cudaSuccess) return MOE_ERR_CUDA;
+      rec.mark("expert_gemm2_combine");
     }
     return MOE_OK;
   }
@@ -485,19 +536,62 @@ moe_status moe_layer_forward(const moe_layer_args* a, void* out, moe_layer_aux* 
                                (const float*)a->dense_b2, (float*)w.h_dense, w.r_dense, status,
                                stream);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
+    rec.mark("dense_ffn");
   }
   if (w.rows_max > 0) {
-    e = bf16 ? enqueue_expert_ffn_bf16(w.x_packed, offsets, E, w.rows_max, d, f, a->w1, a->b1,
-                                       a->w2, a->b2, w.h_packed, w.y_packed, w.C, status, stream)
-             : enqueue_expert_ffn_f32((const float*)w.x_packed, offsets, E, w.rows_max, d, f,
-                                      (const float*)a->w1, (const float*)a->b1,
-                                      (const float*)a->w2, (const float*)a->b2,
-                                      (float*)w.h_packed, w.y_packed, status, stream);
+    if (bf16) {
+      e = enqueue_grouped_gemm_bf16(w.x_packed, offsets, E, w.rows_max, d, f, a->w1, a->b1, true,
+                                    w.h_packed, w.C, status, stream);
+      if (e != cudaSuccess) return MOE_ERR_CUDA;
+      rec.mark("expert_gemm1");
+      e = enqueue_grouped_gemm_bf16(w.h_packed, offsets, E, w.rows_max, f, d, a->w2, a->b2, false,
+                                    w.y_packed, w.C, status, stream);
+    } else {
+      e = enqueue_grouped_gemm_f32((const float*)w.x_packed, offsets, E, w.rows_max, d, f,
+                                   (const float*)a->w1, (const float*)a->b1, true,
+                                   (float*)w.h_packed, status, stream);
+      if (e != cudaSuccess) return MOE_ERR_CUDA;
+      rec.mark("expert_gemm1");
+      e = enqueue_grouped_gemm_f32((const float*)w.h_packed, offsets, E, w.rows_max, f, d,
+                                   (const float*)a->w2, (const float*)a->b2, false, w.y_packed,
+                                   status, stream);
+    }
     if (e != cudaSuccess) return MOE_ERR_CUDA;
+    rec.mark("expert_gemm2");
   }
   e = enqueue_combine(w.y_packed, offsets, ids, slot, gates, T, d, E, k, w.rows_max, residual, bf16,
                       dense ? w.r_dense : nullptr, out, out_bf16, status, stream);
-  return cuda_status(e);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  rec.mark("combine");
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_layer_forward(const moe_layer_args* a, void* out, moe_layer_aux* aux, void* ws,
+                             size_t ws_bytes, moe_stream_t stream) {
+  StageRecorder rec;
+  return layer_forward_impl(a, out, aux, ws, ws_bytes, stream, rec);
+}
+
+moe_status moe_layer_forward_profiled(const moe_layer_args* a, void* out, moe_layer_aux* aux,
+                                      void* ws, size_t ws_bytes, moe_stream_t stream,
+                                      void* const* events, int max_events, int* n_events,
+                                      char* names, size_t names_len) {
+  if (!events || max_events < 1 || !n_events) return MOE_ERR_INVALID_ARGUMENT;
+  for (int i = 0; i < max_events; ++i)
+    if (!events[i]) return MOE_ERR_INVALID_ARGUMENT;
+  StageRecorder rec;
+  rec.events = events;
+  rec.max_events = max_events;
+  rec.names = names;
+  rec.names_len = names_len;
+  if (names && names_len > 0) names[0] = '\0';
+  const moe_status st = layer_forward_impl(a, out, aux, ws, ws_bytes, stream, rec);
+  *n_events = rec.n;
+  return st;
 }
 
 // ---------------------------------------------------------------- status block

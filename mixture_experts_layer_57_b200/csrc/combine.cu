@@ -21,6 +21,7 @@ __global__ void __launch_bounds__(256)
                    const float* __restrict__ gates, int64_t T, int d, int E, int k,
                    int64_t rows_max, const void* __restrict__ residual,
                    const float* __restrict__ dense, void* __restrict__ out, int* status) {
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (t >= T) return;
@@ -76,6 +77,7 @@ __global__ void __launch_bounds__(256)
       for (int v = 0; v < VEC; ++v) o[v] = acc[v];
     }
   }
+  pdl_trigger();
 }
 
 template <int VEC>
@@ -84,17 +86,16 @@ cudaError_t launch(const float* y, const int32_t* offsets, const int32_t* ids, c
                    const void* residual, bool res_bf16, const float* dense, void* out,
                    bool out_bf16, int* status, cudaStream_t stream) {
   const unsigned blocks = (unsigned)((T * 32 + 255) / 256);
-#define MOE_COMBINE_LAUNCH(RB, OB)                                                          \
-  combine_kernel<VEC, RB, OB><<<blocks, 256, 0, stream>>>(y, offsets, ids, slot, gates, T, d, E, \
-                                                          k, rows_max, residual, dense, out,     \
-                                                          status)
-  if (res_bf16 && out_bf16) MOE_COMBINE_LAUNCH(true, true);
-  else if (res_bf16) MOE_COMBINE_LAUNCH(true, false);
-  else if (out_bf16) MOE_COMBINE_LAUNCH(false, true);
-  else MOE_COMBINE_LAUNCH(false, false);
+#define MOE_COMBINE_LAUNCH(RB, OB)                                                              \
+  launch_kernel(combine_kernel<VEC, RB, OB>, dim3(blocks), dim3(256), 0, stream, y, offsets, ids, \
+                slot, gates, T, d, E, k, rows_max, residual, dense, out, status)
+  cudaError_t e;
+  if (res_bf16 && out_bf16) e = MOE_COMBINE_LAUNCH(true, true);
+  else if (res_bf16) e = MOE_COMBINE_LAUNCH(true, false);
+  else if (out_bf16) e = MOE_COMBINE_LAUNCH(false, true);
+  else e = MOE_COMBINE_LAUNCH(false, false);
 #undef MOE_COMBINE_LAUNCH
-  count_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace

@@ -216,6 +216,18 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          ((uint32_t)(M >> 4) << 24);
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// Every kernel of the library is launched as a programmatic dependent of the work before it on
+// the stream. pdl_wait() blocks until those grids have completed and their memory is visible: each
+// kernel calls it before its first global memory access (and before allocating TMEM), so only
+// shared-memory set-up overlaps the predecessor. pdl_trigger() (at the end of a kernel's work)
+// lets the next kernel launch once every CTA has triggered or exited. Both are no-ops when the
+// kernel was launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- warp helpers
 
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }

@@ -31,6 +31,7 @@ __global__ void __launch_bounds__(kCountWarps * 32)
                           int32_t* __restrict__ local_rank, int32_t* __restrict__ seg_counts,
                           int* status) {
   extern __shared__ int cnt_all[];  // [kCountWarps][E]
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int* cnt = cnt_all + warp * E;
   const int64_t seg = (int64_t)blockIdx.x * kCountWarps + warp;
@@ -57,6 +58,7 @@ __global__ void __launch_bounds__(kCountWarps * 32)
     if (p < pairs) local_rank[p] = e >= 0 ? base + rank : -1;
   }
   for (int e = lane; e < E; e += 32) seg_counts[seg * E + e] = cnt[e];
+  pdl_trigger();
 }
 
 __global__ void __launch_bounds__(1024)
@@ -65,6 +67,7 @@ __global__ void __launch_bounds__(1024)
                          int32_t* __restrict__ offsets) {
   __shared__ int kept[MOE_MAX_EXPERTS];
   __shared__ int warp_sums[32];
+  pdl_wait();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int run = 0;
     int64_t s = 0;
@@ -112,6 +115,7 @@ __global__ void __launch_bounds__(1024)
   const int excl = incl - v + warp_sums[warp];
   if (tid < E) offsets[tid] = excl;
   if (tid == E - 1) offsets[E] = excl + v;
+  pdl_trigger();
 }
 
 template <int VEC_BYTES>
@@ -123,6 +127,7 @@ __global__ void __launch_bounds__(256)
                             const int32_t* __restrict__ offsets, int32_t* __restrict__ slot,
                             int32_t* __restrict__ row_token, uint8_t* __restrict__ x_packed,
                             int64_t rows_max, DroppedRows dropped, int d) {
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t p = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (p >= pairs) return;
@@ -159,6 +164,7 @@ __global__ void __launch_bounds__(256)
   V* dst = reinterpret_cast<V*>(x_packed + row * row_bytes);
   const int64_t n = row_bytes / VEC_BYTES;
   for (int64_t i = lane; i < n; i += 32) dst[i] = src[i];
+  pdl_trigger();
 }
 
 }  // namespace
@@ -172,30 +178,30 @@ cudaError_t enqueue_dispatch(const void* x, bool bf16, int64_t T, int d, const i
   const int64_t nseg = dispatch_num_segments(pairs);
   if (pairs > 0) {
     const unsigned blocks = (unsigned)((nseg + kCountWarps - 1) / kCountWarps);
-    dispatch_count_kernel<<<blocks, kCountWarps * 32, kCountWarps * E * sizeof(int), stream>>>(
-        ids, pairs, nseg, E, local_rank, seg_counts, status);
-    count_launch();
+    cudaError_t e = launch_kernel(dispatch_count_kernel, dim3(blocks), dim3(kCountWarps * 32),
+                                  kCountWarps * E * sizeof(int), stream, ids, pairs, nseg, E,
+                                  local_rank, seg_counts, status);
+    if (e != cudaSuccess) return e;
   }
-  dispatch_scan_kernel<<<1, 1024, 0, stream>>>(seg_counts, nseg, E, C, seg_base, counts, offsets);
-  count_launch();
+  {
+    cudaError_t e = launch_kernel(dispatch_scan_kernel, dim3(1), dim3(1024), 0, stream,
+                                  (const int32_t*)seg_counts, nseg, E, C, seg_base, counts, offsets);
+    if (e != cudaSuccess) return e;
+  }
   if (pairs > 0) {
     const int64_t row_bytes = (int64_t)d * (bf16 ? 2 : 4);
     const unsigned blocks = (unsigned)((pairs * 32 + 255) / 256);
     const uint8_t* xs = (const uint8_t*)x;
     uint8_t* xp = (uint8_t*)x_packed;
-    if (row_bytes % 16 == 0)
-      dispatch_scatter_kernel<16><<<blocks, 256, 0, stream>>>(xs, row_bytes, pairs, k, E, C, ids,
-                                                              local_rank, seg_base, offsets, slot,
-                                                              row_token, xp, rows_max, dropped, d);
-    else if (row_bytes % 8 == 0)
-      dispatch_scatter_kernel<8><<<blocks, 256, 0, stream>>>(xs, row_bytes, pairs, k, E, C, ids,
-                                                             local_rank, seg_base, offsets, slot,
-                                                             row_token, xp, rows_max, dropped, d);
-    else
-      dispatch_scatter_kernel<4><<<blocks, 256, 0, stream>>>(xs, row_bytes, pairs, k, E, C, ids,
-                                                             local_rank, seg_base, offsets, slot,
-                                                             row_token, xp, rows_max, dropped, d);
-    count_launch();
+    auto launch = [&](auto kern) {
+      return launch_kernel(kern, dim3(blocks), dim3(256), 0, stream, xs, row_bytes, pairs, k, E, C,
+                           ids, (const int32_t*)local_rank, (const int32_t*)seg_base,
+                           (const int32_t*)offsets, slot, row_token, xp, rows_max, dropped, d);
+    };
+    cudaError_t e = row_bytes % 16 == 0  ? launch(dispatch_scatter_kernel<16>)
+                    : row_bytes % 8 == 0 ? launch(dispatch_scatter_kernel<8>)
+                                         : launch(dispatch_scatter_kernel<4>);
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }

@@ -18,6 +18,7 @@ __global__ void __launch_bounds__(kFeat)
                    int n_out, int K, int64_t rows_max, const float* __restrict__ W,
                    const float* __restrict__ bias, float* __restrict__ out, int* status) {
   extern __shared__ float xs[];
+  pdl_wait();
   // offsets == nullptr: one segment covering all rows_max rows (dense MLP, E == 1)
   const int64_t start = offsets ? offsets[0] : 0, total = offsets ? offsets[E] : rows_max;
   if (start < 0 || total < start || total > rows_max) {
@@ -46,6 +47,7 @@ __global__ void __launch_bounds__(kFeat)
       out[r * n_out + f] = v;
     }
   }
+  pdl_trigger();
 }
 
 }  // namespace
@@ -65,14 +67,8 @@ cudaError_t enqueue_grouped_gemm_f32(const float* x, const int32_t* offsets, int
     attr_done[gelu] = smem;
   }
   const dim3 grid(gx, (N + kFeat - 1) / kFeat);
-  if (gelu)
-    ffn_f32_kernel<true><<<grid, kFeat, smem, stream>>>(x, offsets, E, N, K, rows_max, w, bias, out,
-                                                        status);
-  else
-    ffn_f32_kernel<false><<<grid, kFeat, smem, stream>>>(x, offsets, E, N, K, rows_max, w, bias, out,
-                                                         status);
-  count_launch();
-  return cudaGetLastError();
+  return launch_kernel(gelu ? ffn_f32_kernel<true> : ffn_f32_kernel<false>, grid, dim3(kFeat), smem,
+                       stream, x, offsets, E, N, K, rows_max, w, bias, out, status);
 }
 
 cudaError_t enqueue_expert_ffn_f32(const float* x_packed, const int32_t* offsets, int E,

@@ -172,6 +172,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
+  }
+  // everything above touches shared memory only; wait for the preceding kernels before any global
+  // access or TMEM allocation
+  pdl_wait();
+  if (threadIdx.x == 0) {
     tma_prefetch_desc(&tmW);
     tma_prefetch_desc(&tmX);
   }
@@ -443,6 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ------------------------------------------------------------ teardown
   tc_fence_before();
   __syncthreads();
+  pdl_trigger();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::kTmemCols);
@@ -493,9 +499,7 @@ cudaError_t launch_one(const CUtensorMap& tmW, const CUtensorMap& tmX, const Par
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  kern<<<num_sms(), kThreads, Cfg<BN>::kSmemBytes, stream>>>(tmW, tmX, p);
-  count_launch();
-  return cudaGetLastError();
+  return launch_kernel(kern, dim3(num_sms()), dim3(kThreads), Cfg<BN>::kSmemBytes, stream, tmW, tmX, p);
 }
 
 }  // namespace

@@ -16,11 +16,36 @@ void reset_launch_count();
 // Number of SMs of the current device (cached per device).
 int num_sms();
 
+// Whether launches carry the programmatic-dependent-launch attribute (MOE_PDL=0 disables it).
+bool pdl_enabled();
+
+// Launches kern<<<grid, block, smem, stream>>>(args...) as a programmatic dependent launch and
+// counts it.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
+  count_launch();
+  return e;
+}
+
 // ---------------------------------------------------------------- router
 constexpr int kRouterTokensPerBlock = 64;
 inline int64_t router_num_blocks(int64_t T) {
   return (T + kRouterTokensPerBlock - 1) / kRouterTokensPerBlock;
 }
+// Batches up to this many tokens use the GEMV router (one block per expert).
+constexpr int64_t kRouterGemvMaxT = 64;
 // K of each bf16 part of the split router weight, padded to the 64-element TMA block.
 inline int router_split_dpad(int d) { return (d + 63) / 64 * 64; }
 // The tensor-core router needs bf16 x whose rows are whole 16-byte units.

@@ -37,6 +37,7 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const void* __restri
                                                             float* __restrict__ logits) {
   __shared__ float xs[kLBK][kLBM + 4];
   __shared__ float ws[kLBK][kLBN + 4];
+  pdl_wait();
   const int tx = threadIdx.x & 15;   // expert lane
   const int ty = threadIdx.x >> 4;   // token lane
   const int64_t t0 = (int64_t)blockIdx.x * kLBM;
@@ -77,11 +78,77 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const void* __restri
       if (e < E) logits[t * E + e] = acc[i][j] + (bias ? bias[e] : 0.0f);
     }
   }
+  pdl_trigger();
+}
+
+// Decode-sized batches (T <= kRouterGemvMaxT): one block per expert, warp per token, lanes over
+// K with 16-byte loads, fp32 FMA, fixed-order warp reduction; block 0 also zeroes the statistics
+// accumulators (this kernel then replaces the prep kernel).
+template <bool XBF16>
+__global__ void __launch_bounds__(256) router_gemv_kernel(const void* __restrict__ x,
+                                                          const float* __restrict__ w,
+                                                          const float* __restrict__ bias,
+                                                          int64_t T, int d, int E,
+                                                          float* __restrict__ logits,
+                                                          RouterAccum acc) {
+  pdl_wait();
+  const int e = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (e == 0) {
+    for (int i = threadIdx.x; i < E; i += blockDim.x) {
+      acc.q[i] = 0ull;
+      acc.c[i] = 0u;
+    }
+    if (threadIdx.x == 0) *acc.ticket = 0u;
+  }
+  const float* wr = w + (int64_t)e * d;
+  for (int64_t t = warp; t < T; t += 8) {
+    float s = 0.0f;
+    if constexpr (XBF16) {
+      const uint16_t* xr = reinterpret_cast<const uint16_t*>(x) + t * d;
+      if ((d & 7) == 0) {
+        for (int i = lane * 8; i < d; i += 256) {
+          const uint4 xv = *reinterpret_cast<const uint4*>(xr + i);
+          const float4 w0 = *reinterpret_cast<const float4*>(wr + i);
+          const float4 w1 = *reinterpret_cast<const float4*>(wr + i + 4);
+          s = fmaf(__uint_as_float(xv.x << 16), w0.x, s);
+          s = fmaf(__uint_as_float(xv.x & 0xffff0000u), w0.y, s);
+          s = fmaf(__uint_as_float(xv.y << 16), w0.z, s);
+          s = fmaf(__uint_as_float(xv.y & 0xffff0000u), w0.w, s);
+          s = fmaf(__uint_as_float(xv.z << 16), w1.x, s);
+          s = fmaf(__uint_as_float(xv.z & 0xffff0000u), w1.y, s);
+          s = fmaf(__uint_as_float(xv.w << 16), w1.z, s);
+          s = fmaf(__uint_as_float(xv.w & 0xffff0000u), w1.w, s);
+        }
+      } else {
+        for (int i = lane; i < d; i += 32) s = fmaf(bf16_to_f32(xr[i]), wr[i], s);
+      }
+    } else {
+      const float* xr = reinterpret_cast<const float*>(x) + t * d;
+      if ((d & 3) == 0) {
+        for (int i = lane * 4; i < d; i += 128) {
+          const float4 xv = *reinterpret_cast<const float4*>(xr + i);
+          const float4 wv = *reinterpret_cast<const float4*>(wr + i);
+          s = fmaf(xv.x, wv.x, s);
+          s = fmaf(xv.y, wv.y, s);
+          s = fmaf(xv.z, wv.z, s);
+          s = fmaf(xv.w, wv.w, s);
+        }
+      } else {
+        for (int i = lane; i < d; i += 32) s = fmaf(xr[i], wr[i], s);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) logits[t * E + e] = s + (bias ? bias[e] : 0.0f);
+  }
+  pdl_trigger();
 }
 
 __global__ void __launch_bounds__(256) router_prep_kernel(const float* __restrict__ w, int E,
                                                           int d, int dpad, uint16_t* __restrict__ out,
                                                           RouterAccum acc) {
+  pdl_wait();
   if (blockIdx.x == 0) {
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
       acc.q[e] = 0ull;
@@ -89,7 +156,10 @@ __global__ void __launch_bounds__(256) router_prep_kernel(const float* __restric
     }
     if (threadIdx.x == 0) *acc.ticket = 0u;
   }
-  if (out == nullptr) return;
+  if (out == nullptr) {
+    pdl_trigger();
+    return;
+  }
   const int64_t n = (int64_t)E * dpad;
   for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < n;
        idx += (int64_t)gridDim.x * blockDim.x) {
@@ -105,6 +175,7 @@ __global__ void __launch_bounds__(256) router_prep_kernel(const float* __restric
     row[dpad + i] = mid;
     row[2 * dpad + i] = lo;
   }
+  pdl_trigger();
 }
 
 constexpr double kQScale = 4294967296.0;  // 2^32: fixed-point scale of the p sums
@@ -121,6 +192,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
   __shared__ int cs[MOE_MAX_EXPERTS];
   __shared__ float prod[MOE_MAX_EXPERTS];
   __shared__ int is_last;
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int e = threadIdx.x; e < E; e += 256) cs[e] = 0;
   __syncthreads();
@@ -207,6 +279,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
     if (fx) atomicAdd(&acc.q[e], fx);
     if (cs[e]) atomicAdd(&acc.c[e], (unsigned)cs[e]);
   }
+  pdl_trigger();
   if (lb == nullptr) return;
   // the last block to finish turns the totals into f, Q, aux
   __threadfence();
@@ -233,10 +306,10 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
 }
 
 template <int EPL>
-void launch_topk(const float* logits, int64_t T, int E, int k, int32_t* ids, float* gates,
-                 const RouterAccum& acc, float alpha, float* lb, cudaStream_t stream) {
-  router_topk_kernel<EPL><<<(unsigned)router_num_blocks(T), 256, 0, stream>>>(
-      logits, T, E, k, ids, gates, acc, alpha, lb);
+cudaError_t launch_topk(const float* logits, int64_t T, int E, int k, int32_t* ids, float* gates,
+                        const RouterAccum& acc, float alpha, float* lb, cudaStream_t stream) {
+  return launch_kernel(router_topk_kernel<EPL>, dim3((unsigned)router_num_blocks(T)), dim3(256), 0, stream,
+                (const float*)logits, T, E, k, ids, gates, acc, alpha, lb);
 }
 
 }  // namespace
@@ -247,34 +320,37 @@ cudaError_t enqueue_router(const void* x, bool x_bf16, int64_t T, int d, const f
                            const RouterScratch& scr, int* status, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
   if (!logits) logits = scr.logits_scratch;
-  const bool tc = router_uses_tensor_cores(x_bf16, d);
+  const bool gemv = T <= kRouterGemvMaxT;
+  const bool tc = !gemv && router_uses_tensor_cores(x_bf16, d);
   const int dpad = router_split_dpad(d);
   const int64_t n = tc ? (int64_t)E * dpad : 0;
   const unsigned blocks = (unsigned)(n == 0 ? 1 : ((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096));
-  router_prep_kernel<<<blocks, 256, 0, stream>>>(w_router, E, d, dpad, tc ? scr.w_split : nullptr,
-                                                 scr.acc);
-  count_launch();
+  cudaError_t err;
+  if (gemv) {
+    err = launch_kernel(x_bf16 ? router_gemv_kernel<true> : router_gemv_kernel<false>, dim3(E),
+                        dim3(256), 0, stream, x, w_router, router_bias, T, d, E, logits, scr.acc);
+  } else {
+    err = launch_kernel(router_prep_kernel, dim3(blocks), dim3(256), 0, stream, w_router, E, d, dpad,
+                        tc ? scr.w_split : nullptr, scr.acc);
+  }
+  if (err != cudaSuccess) return err;
   if (tc) {
     cudaError_t e = enqueue_router_logits_tc(x, T, d, scr.w_split, dpad, router_bias, E, logits,
                                              status, stream);
     if (e != cudaSuccess) return e;
-  } else {
+  } else if (!gemv) {
     dim3 grid((unsigned)((T + kLBM - 1) / kLBM), (E + kLBN - 1) / kLBN);
-    if (x_bf16)
-      router_logits_kernel<true><<<grid, 256, 0, stream>>>(x, w_router, router_bias, T, d, E, logits);
-    else
-      router_logits_kernel<false><<<grid, 256, 0, stream>>>(x, w_router, router_bias, T, d, E, logits);
-    count_launch();
+    err = launch_kernel(x_bf16 ? router_logits_kernel<true> : router_logits_kernel<false>, grid,
+                        dim3(256), 0, stream, x, w_router, router_bias, T, d, E, logits);
+    if (err != cudaSuccess) return err;
   }
   const RouterAccum& a = scr.acc;
-  if (E <= 32) launch_topk<1>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, stream);
-  else if (E <= 64) launch_topk<2>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, stream);
-  else if (E <= 128) launch_topk<4>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, stream);
-  else if (E <= 256) launch_topk<8>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, stream);
-  else if (E <= 512) launch_topk<16>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, stream);
-  else launch_topk<32>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, stream);
-  count_launch();
-  return cudaGetLastError();
+  if (E <= 32) return launch_topk<1>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, stream);
+  if (E <= 64) return launch_topk<2>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, stream);
+  if (E <= 128) return launch_topk<4>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, stream);
+  if (E <= 256) return launch_topk<8>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, stream);
+  if (E <= 512) return launch_topk<16>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, stream);
+  return launch_topk<32>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, stream);
 }
 
 }  // namespace moe

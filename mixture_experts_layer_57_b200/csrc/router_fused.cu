@@ -96,6 +96,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
+  }
+  pdl_wait();  // global memory and TMEM only after the preceding kernels have completed
+  if (threadIdx.x == 0) {
     tma_prefetch_desc(&tmX);
     tma_prefetch_desc(&tmW);
   }
@@ -229,6 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  pdl_trigger();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::kTmemCols);
@@ -272,9 +276,7 @@ cudaError_t launch_tc(const CUtensorMap& tmX, const CUtensorMap& tmW, const RPar
     attr_set = true;
   }
   const int grid = ntiles < num_sms() ? ntiles : num_sms();
-  kern<<<grid, kThreads, RCfg<NE>::kSmemBytes, stream>>>(tmX, tmW, p);
-  count_launch();
-  return cudaGetLastError();
+  return launch_kernel(kern, dim3(grid), dim3(kThreads), RCfg<NE>::kSmemBytes, stream, tmX, tmW, p);
 }
 
 }  // namespace

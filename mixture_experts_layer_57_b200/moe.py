@@ -85,6 +85,8 @@ def lib() -> ctypes.CDLL:
             "moe_combine": ([vp, vp, vp, vp, vp, i64, i32, i32, i32, i64, vp, i32, vp, vp, i32, vp, sz, vp], i32),
             "moe_layer_workspace_bytes": ([P(LayerArgs), P(sz)], i32),
             "moe_layer_forward": ([P(LayerArgs), vp, P(LayerAux), vp, sz, vp], i32),
+            "moe_layer_forward_profiled": ([P(LayerArgs), vp, P(LayerAux), vp, sz, vp,
+                                            P(vp), i32, P(i32), ctypes.c_char_p, sz], i32),
             "moe_workspace_reset": ([vp, sz, vp], i32),
             "moe_get_device_error": ([vp, P(i32), vp], i32),
         }
@@ -355,6 +357,28 @@ def moe_layer_forward(args: LayerArgs, out: torch.Tensor, aux: Optional[dict] = 
     _check("moe_layer_forward", lib().moe_layer_forward(
         ctypes.byref(args), _ptr(out), ctypes.byref(a), _ptr(ws), ws.numel(), _stream(stream)))
     return out
+
+
+def moe_layer_forward_profiled(args: LayerArgs, out: torch.Tensor, events: list, aux=None, ws=None,
+                               stream=None):
+    """moe_layer_forward recording ``events`` (torch.cuda.Event(enable_timing=True)) at stage
+    boundaries; returns the list of stage labels, starting with "start"."""
+    if ws is None:
+        ws = workspace(moe_layer_workspace_bytes(args), out.device)
+    for ev in events:
+        if ev.cuda_event == 0:
+            ev.record()   # create the underlying CUDA event
+    a = LayerAux()
+    if aux:
+        for name, t in aux.items():
+            setattr(a, name, _ptr(t))
+    handles = (ctypes.c_void_p * len(events))(*[ev.cuda_event for ev in events])
+    n = ctypes.c_int()
+    names = ctypes.create_string_buffer(512)
+    _check("moe_layer_forward_profiled", lib().moe_layer_forward_profiled(
+        ctypes.byref(args), _ptr(out), ctypes.byref(a), _ptr(ws), ws.numel(), _stream(stream),
+        handles, len(events), ctypes.byref(n), names, 512))
+    return names.value.decode().split(",")[: n.value]
 
 
 def moe_workspace_reset(ws: torch.Tensor, stream=None):

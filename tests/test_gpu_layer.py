@@ -162,3 +162,28 @@ def test_launch_count(cuda_ok):
     w2 = synth.WORKLOADS[4].with_(T=256, d_model=128, d_ff=256)
     got = run_layer(w2, dev_inputs(synth.make_inputs(w2)))
     assert got["launches"] == 9      # top-2: gather combine kernel
+
+
+@pytest.mark.parametrize("cfg", [2, 3, 4])
+def test_profiled_forward_matches_and_labels_stages(cuda_ok, cfg):
+    from mixture_experts_layer_57_b200 import moe
+    w = synth.WORKLOADS[cfg].with_(T=256, d_model=128, d_ff=256)
+    d_inp = dev_inputs(synth.make_inputs(w))
+    ref = run_layer(w, d_inp)
+    dense = (d_inp["dense_w1"], d_inp["dense_b1"], d_inp["dense_w2"], d_inp["dense_b2"]) if w.dense else None
+    args = moe.layer_args(d_inp["x"], d_inp["w_router"], d_inp["w1"], d_inp["b1"], d_inp["w2"],
+                          d_inp["b2"], k=w.k, capacity_factor=w.capacity_factor,
+                          router_bias=d_inp.get("router_bias"), dense=dense,
+                          add_input_residual=w.add_input_residual, aux_alpha=w.aux_alpha)
+    out = torch.empty(w.T, w.d_model, dtype=torch.bfloat16, device="cuda")
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(12)]
+    names = moe.moe_layer_forward_profiled(args, out, evs)
+    torch.cuda.synchronize()
+    want = {2: ["start", "router", "dispatch", "expert_gemm1", "expert_gemm2_combine"],
+            3: ["start", "router", "dispatch", "expert_gemm1", "expert_gemm2", "dense_gemm1",
+                "dense_gemm2_combine"],
+            4: ["start", "router", "dispatch", "expert_gemm1", "expert_gemm2", "combine"]}[cfg]
+    assert names == want
+    assert all(evs[i].elapsed_time(evs[i + 1]) >= 0 for i in range(len(names) - 1))
+    from tests.helpers import to_host
+    assert np.array_equal(to_host(out), ref["out"])
