@@ -90,7 +90,10 @@ struct DispatchWs {
   int32_t *local_rank, *seg_counts, *seg_base;
 };
 DispatchWs carve_dispatch(Carve& c, int64_t T, int E, int k) {
-  const int64_t nseg = dispatch_num_segments(T * k);
+  // segments of 256 pairs (counting kernel) or of one 64-token router block (layer forward)
+  const int64_t nseg = dispatch_num_segments(T * k) > router_num_blocks(T)
+                           ? dispatch_num_segments(T * k)
+                           : router_num_blocks(T);
   DispatchWs w;
   w.local_rank = c.take<int32_t>((size_t)T * k);
   w.seg_counts = c.take<int32_t>((size_t)nseg * E);
@@ -455,8 +458,12 @@ moe_status layer_forward_impl(const moe_layer_args* a, void* out, moe_layer_aux*
 
   rec.stream = stream;
   rec.mark("start");
+  // the router's top-k kernel also ranks each 64-token segment's pairs for dispatch
+  RouterDispatchCount dcount;
+  dcount.local_rank = w.dispatch.local_rank;
+  dcount.seg_counts = w.dispatch.seg_counts;
   cudaError_t e = enqueue_router(a->x, bf16, T, d, a->w_router, a->router_bias, E, k, logits, ids,
-                                 gates, lb, a->aux_alpha, w.router.scr, status, stream);
+                                 gates, lb, a->aux_alpha, w.router.scr, status, stream, dcount);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   rec.mark("router");
 
@@ -475,7 +482,8 @@ moe_status layer_forward_impl(const moe_layer_args* a, void* out, moe_layer_aux*
   }
   e = enqueue_dispatch(a->x, bf16, T, d, ids, E, k, w.C, slot, counts, offsets, w.row_token,
                        w.x_packed, w.rows_max, w.dispatch.local_rank, w.dispatch.seg_counts,
-                       w.dispatch.seg_base, status, stream, dropped);
+                       w.dispatch.seg_base, status, stream, dropped,
+                       (int)kRouterTokensPerBlock * k);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   rec.mark("dispatch");
 

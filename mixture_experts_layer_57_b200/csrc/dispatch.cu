@@ -11,9 +11,11 @@
 //   dispatch_count_kernel   one warp per segment of 256 consecutive pairs: in-warp ranks from
 //                           __match_any_sync, running per-expert counts in shared memory;
 //                           writes each pair's rank inside its segment and the segment totals
+//                           (inside the layer forward the router's top-k kernel does this for its
+//                           own 64-token segments and this kernel is skipped)
 //   dispatch_scan_kernel    one block: per expert, exclusive prefix over segments (segment
-//                           bases) and the demand; kept = min(demand, C); exclusive scan over
-//                           experts of kept -> offsets
+//                           bases, runs of segments in parallel) and the demand;
+//                           kept = min(demand, C); exclusive scan over experts -> offsets
 //   dispatch_scatter_kernel one warp per pair: position = segment base + rank, slot = position
 //                           or -1 beyond C, row_token, and a 16-byte vector copy of the row
 #include <type_traits>
@@ -61,37 +63,48 @@ __global__ void __launch_bounds__(kCountWarps * 32)
   pdl_trigger();
 }
 
+// Thread (g, e) owns a contiguous run of segments of expert e (G = 1024 / E runs per expert): it
+// sums them, takes the sum of the earlier runs from shared memory as its base, then writes the
+// exclusive prefix of its run (the segment bases). The last run's end is the demand.
 __global__ void __launch_bounds__(1024)
     dispatch_scan_kernel(const int32_t* __restrict__ seg_counts, int64_t nseg, int E, int64_t C,
                          int32_t* __restrict__ seg_base, int32_t* __restrict__ counts,
                          int32_t* __restrict__ offsets) {
+  __shared__ int run_sum[1024];
   __shared__ int kept[MOE_MAX_EXPERTS];
   __shared__ int warp_sums[32];
   pdl_wait();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+  const int tid = threadIdx.x;
+  int G = 1024 / E;
+  if ((int64_t)G > nseg) G = nseg > 0 ? (int)nseg : 1;
+  const int64_t chunk = (nseg + G - 1) / G;
+  const bool active = tid < G * E;
+  const int e = active ? tid % E : 0, g = active ? tid / E : 0;
+  const int64_t s0 = (int64_t)g * chunk, s1 = min(nseg, s0 + chunk);
+  int sum = 0;
+  if (active) {
+#pragma unroll 8
+    for (int64_t s = s0; s < s1; ++s) sum += seg_counts[s * E + e];
+    run_sum[tid] = sum;
+  }
+  __syncthreads();
+  if (active) {
     int run = 0;
-    int64_t s = 0;
-    for (; s + 8 <= nseg; s += 8) {
-      int v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = seg_counts[(s + u) * E + e];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        seg_base[(s + u) * E + e] = run;
-        run += v[u];
-      }
-    }
-    for (; s < nseg; ++s) {
+    for (int gg = 0; gg < g; ++gg) run += run_sum[gg * E + e];
+#pragma unroll 8
+    for (int64_t s = s0; s < s1; ++s) {
       const int v = seg_counts[s * E + e];
       seg_base[s * E + e] = run;
       run += v;
     }
-    counts[e] = run;
-    kept[e] = (int)min((int64_t)run, C);
+    if (g == G - 1) {
+      counts[e] = run;
+      kept[e] = (int)min((int64_t)run, C);
+    }
   }
   __syncthreads();
   // exclusive scan of kept over experts (E <= 1024), one element per thread
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int lane = tid & 31, warp = tid >> 5;
   const int v = tid < E ? kept[tid] : 0;
   int incl = v;
 #pragma unroll
@@ -126,7 +139,7 @@ __global__ void __launch_bounds__(256)
                             const int32_t* __restrict__ seg_base,
                             const int32_t* __restrict__ offsets, int32_t* __restrict__ slot,
                             int32_t* __restrict__ row_token, uint8_t* __restrict__ x_packed,
-                            int64_t rows_max, DroppedRows dropped, int d) {
+                            int64_t rows_max, DroppedRows dropped, int d, int seg_len) {
   pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t p = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -135,7 +148,7 @@ __global__ void __launch_bounds__(256)
   const int r = local_rank[p];
   int s = -1;
   if (e >= 0 && e < E && r >= 0) {
-    const int pos = seg_base[(p / kDispatchSeg) * E + e] + r;
+    const int pos = seg_base[(p / seg_len) * E + e] + r;
     if (pos < C) s = pos;
   }
   if (lane == 0) slot[p] = s;
@@ -173,10 +186,12 @@ cudaError_t enqueue_dispatch(const void* x, bool bf16, int64_t T, int d, const i
                              int k, int64_t C, int32_t* slot, int32_t* counts, int32_t* offsets,
                              int32_t* row_token, void* x_packed, int64_t rows_max,
                              int32_t* local_rank, int32_t* seg_counts, int32_t* seg_base,
-                             int* status, cudaStream_t stream, DroppedRows dropped) {
+                             int* status, cudaStream_t stream, DroppedRows dropped,
+                             int counted_seg_len) {
   const int64_t pairs = T * k;
-  const int64_t nseg = dispatch_num_segments(pairs);
-  if (pairs > 0) {
+  const int seg_len = counted_seg_len > 0 ? counted_seg_len : kDispatchSeg;
+  const int64_t nseg = (pairs + seg_len - 1) / seg_len;
+  if (pairs > 0 && counted_seg_len <= 0) {
     const unsigned blocks = (unsigned)((nseg + kCountWarps - 1) / kCountWarps);
     cudaError_t e = launch_kernel(dispatch_count_kernel, dim3(blocks), dim3(kCountWarps * 32),
                                   kCountWarps * E * sizeof(int), stream, ids, pairs, nseg, E,
@@ -196,7 +211,8 @@ cudaError_t enqueue_dispatch(const void* x, bool bf16, int64_t T, int d, const i
     auto launch = [&](auto kern) {
       return launch_kernel(kern, dim3(blocks), dim3(256), 0, stream, xs, row_bytes, pairs, k, E, C,
                            ids, (const int32_t*)local_rank, (const int32_t*)seg_base,
-                           (const int32_t*)offsets, slot, row_token, xp, rows_max, dropped, d);
+                           (const int32_t*)offsets, slot, row_token, xp, rows_max, dropped, d,
+                           seg_len);
     };
     cudaError_t e = row_bytes % 16 == 0  ? launch(dispatch_scatter_kernel<16>)
                     : row_bytes % 8 == 0 ? launch(dispatch_scatter_kernel<8>)

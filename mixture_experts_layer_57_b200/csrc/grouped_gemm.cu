@@ -34,6 +34,10 @@
 namespace moe {
 namespace {
 
+#ifndef MOE_GG_MAX_STAGES
+#define MOE_GG_MAX_STAGES 12
+#endif
+
 constexpr int kBM = 128;         // output features per tile (MMA M)
 constexpr int kBK = 64;          // K per stage: one 128-byte swizzle row of bf16
 constexpr int kUmmaK = 16;       // K per tcgen05.mma (kind::f16)
@@ -56,7 +60,7 @@ struct Cfg {
   static constexpr int kBBytes = BN * kBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kStagesFit = (200 * 1024) / kStageBytes;
-  static constexpr int kStages = kStagesFit > 12 ? 12 : kStagesFit;
+  static constexpr int kStages = kStagesFit > MOE_GG_MAX_STAGES ? MOE_GG_MAX_STAGES : kStagesFit;
   static constexpr int kTmemCols = (2 * BN) < 32 ? 32 : (2 * BN);
   // barriers: full[S], empty[S], tmem_full[2], tmem_empty[2], drain  (8 bytes each, <= 64 of them)
   static constexpr int kBarBytes = 8 * 64;

@@ -61,11 +61,18 @@ struct RouterScratch {
   uint16_t* w_split;      // [E, 3 * router_split_dpad(d)] bf16: hi | mid | lo parts of W_r
   float* logits_scratch;  // [T, E], used when the caller does not ask for the logits
 };
+// Optional: let the top-k kernel also rank each 64-token segment's (token, choice) pairs per
+// expert for dispatch (segments of kRouterTokensPerBlock * k pairs).
+struct RouterDispatchCount {
+  int32_t* local_rank = nullptr;  // [T * k]
+  int32_t* seg_counts = nullptr;  // [router_num_blocks(T), E]
+};
 // logits may be nullptr (not returned).
 cudaError_t enqueue_router(const void* x, bool x_bf16, int64_t T, int d, const float* w_router,
                            const float* router_bias, int E, int k, float* logits, int32_t* ids,
                            float* gates, float* lb_stats, float aux_alpha,
-                           const RouterScratch& scratch, int* status, cudaStream_t stream);
+                           const RouterScratch& scratch, int* status, cudaStream_t stream,
+                           RouterDispatchCount dcount = RouterDispatchCount{});
 // logits = x W_r^T + b_r on tcgen05 from the exact split W_r = hi + mid + lo (bf16 each).
 cudaError_t enqueue_router_logits_tc(const void* x, int64_t T, int d, const uint16_t* w_split,
                                      int dpad, const float* router_bias, int E, float* logits,
@@ -87,7 +94,10 @@ cudaError_t enqueue_dispatch(const void* x, bool bf16, int64_t T, int d, const i
                              int k, int64_t C, int32_t* slot, int32_t* counts, int32_t* offsets,
                              int32_t* row_token, void* x_packed, int64_t rows_max,
                              int32_t* local_rank, int32_t* seg_counts, int32_t* seg_base,
-                             int* status, cudaStream_t stream, DroppedRows dropped = DroppedRows{});
+                             int* status, cudaStream_t stream, DroppedRows dropped = DroppedRows{},
+                             int counted_seg_len = 0);
+// counted_seg_len > 0: local_rank and seg_counts were already written (segments of that many
+// pairs) by the router's top-k kernel; the counting kernel is skipped.
 
 // ---------------------------------------------------------------- expert FFN
 // One grouped GEMM layer: out = act(W[e] x + bias[e]) over every expert segment. offsets ==

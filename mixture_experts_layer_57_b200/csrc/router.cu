@@ -181,17 +181,20 @@ __global__ void __launch_bounds__(256) router_prep_kernel(const float* __restric
 constexpr double kQScale = 4294967296.0;  // 2^32: fixed-point scale of the p sums
 
 // EPL = experts per lane (E <= 32 * EPL); expert e lives in lane e % 32, slot e / 32.
-template <int EPL>
+// COUNT: also rank this block's (token, choice) pairs per expert in pair order for dispatch.
+template <int EPL, bool COUNT>
 __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restrict__ logits,
                                                           int64_t T, int E, int k,
                                                           int32_t* __restrict__ ids,
                                                           float* __restrict__ gates,
                                                           RouterAccum acc, float alpha,
-                                                          float* __restrict__ lb) {
+                                                          float* __restrict__ lb,
+                                                          RouterDispatchCount dc) {
   __shared__ float qs[8][MOE_MAX_EXPERTS];
   __shared__ int cs[MOE_MAX_EXPERTS];
   __shared__ float prod[MOE_MAX_EXPERTS];
   __shared__ int is_last;
+  __shared__ int blk_ids[COUNT ? kRouterTokensPerBlock * MOE_MAX_TOPK : 1];
   pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int e = threadIdx.x; e < E; e += 256) cs[e] = 0;
@@ -228,26 +231,35 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
       p[i] = ex[i] / s;
       q[i] += p[i];
     }
-    // top-k on the logits: k rounds of (value desc, index asc) warp argmax
+    // first choice: the lowest expert index holding the maximum logit (ballot per slot)
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int i = EPL - 1; i >= 0; --i) {
+      const unsigned b = __ballot_sync(0xffffffffu, (lane + 32 * i) < E && l[i] == m);
+      if (b) bi = 32 * i + __ffs(b) - 1;
+    }
     uint32_t taken = 0;
     for (int j = 0; j < k; ++j) {
-      float bv = -INFINITY;
-      int bi = 0x7fffffff;
+      if (j > 0) {
+        // later choices: (value desc, index asc) warp argmax over the experts not yet taken
+        float bv = -INFINITY;
+        bi = 0x7fffffff;
 #pragma unroll
-      for (int i = 0; i < EPL; ++i) {
-        const int e = lane + 32 * i;
-        if (e < E && !(taken >> i & 1u) && (l[i] > bv || bi == 0x7fffffff)) {
-          bv = l[i];
-          bi = e;
+        for (int i = 0; i < EPL; ++i) {
+          const int e = lane + 32 * i;
+          if (e < E && !(taken >> i & 1u) && (l[i] > bv || bi == 0x7fffffff)) {
+            bv = l[i];
+            bi = e;
+          }
         }
-      }
 #pragma unroll
-      for (int o = 16; o; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (ov > bv || (ov == bv && oi < bi)) {
-          bv = ov;
-          bi = oi;
+        for (int o = 16; o; o >>= 1) {
+          const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+          const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+          if (ov > bv || (ov == bv && oi < bi)) {
+            bv = ov;
+            bi = oi;
+          }
         }
       }
       const int owner = bi & 31, slot_i = bi >> 5;
@@ -261,8 +273,35 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
         ids[t * k + j] = bi;
         gates[t * k + j] = pv;
         if (j == 0) atomicAdd(&cs[bi], 1);  // integer counts: order-independent
+        if constexpr (COUNT) blk_ids[r * k + j] = bi;
       }
     }
+  }
+  if constexpr (COUNT) {
+    // rank the block's pairs per expert in pair order (warp 0), write ranks and segment counts
+    __syncthreads();
+    int* run = reinterpret_cast<int*>(prod);  // reused as running counts until the finalize
+    for (int e = threadIdx.x; e < E; e += 256) run[e] = 0;
+    __syncthreads();
+    const int64_t ntok = min((int64_t)kRouterTokensPerBlock, T - tb);
+    const int npairs = (int)ntok * k;
+    if (warp == 0) {
+      const unsigned lt = (1u << lane) - 1u;
+      for (int c = 0; c < npairs; c += 32) {
+        const int pl = c + lane;
+        const int e = pl < npairs ? blk_ids[pl] : -1;
+        const unsigned same = __match_any_sync(0xffffffffu, e);
+        const int rank = __popc(same & lt);
+        const int base = e >= 0 ? run[e] : 0;
+        __syncwarp();
+        if (e >= 0 && rank == 0) run[e] = base + __popc(same);
+        __syncwarp();
+        if (pl < npairs) dc.local_rank[tb * k + pl] = base + rank;
+      }
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += 256) dc.seg_counts[(int64_t)blockIdx.x * E + e] = run[e];
+    __syncthreads();
   }
   // block sums of p in a fixed order (warps ascending), then integer accumulation
 #pragma unroll
@@ -307,9 +346,14 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
 
 template <int EPL>
 cudaError_t launch_topk(const float* logits, int64_t T, int E, int k, int32_t* ids, float* gates,
-                        const RouterAccum& acc, float alpha, float* lb, cudaStream_t stream) {
-  return launch_kernel(router_topk_kernel<EPL>, dim3((unsigned)router_num_blocks(T)), dim3(256), 0, stream,
-                (const float*)logits, T, E, k, ids, gates, acc, alpha, lb);
+                        const RouterAccum& acc, float alpha, float* lb, RouterDispatchCount dc,
+                        cudaStream_t stream) {
+  const dim3 grid((unsigned)router_num_blocks(T));
+  if (dc.local_rank != nullptr)
+    return launch_kernel(router_topk_kernel<EPL, true>, grid, dim3(256), 0, stream,
+                         (const float*)logits, T, E, k, ids, gates, acc, alpha, lb, dc);
+  return launch_kernel(router_topk_kernel<EPL, false>, grid, dim3(256), 0, stream,
+                       (const float*)logits, T, E, k, ids, gates, acc, alpha, lb, dc);
 }
 
 }  // namespace
@@ -317,7 +361,8 @@ cudaError_t launch_topk(const float* logits, int64_t T, int E, int k, int32_t* i
 cudaError_t enqueue_router(const void* x, bool x_bf16, int64_t T, int d, const float* w_router,
                            const float* router_bias, int E, int k, float* logits, int32_t* ids,
                            float* gates, float* lb_stats, float aux_alpha,
-                           const RouterScratch& scr, int* status, cudaStream_t stream) {
+                           const RouterScratch& scr, int* status, cudaStream_t stream,
+                           RouterDispatchCount dc) {
   if (T == 0) return cudaSuccess;
   if (!logits) logits = scr.logits_scratch;
   const bool gemv = T <= kRouterGemvMaxT;
@@ -345,12 +390,12 @@ cudaError_t enqueue_router(const void* x, bool x_bf16, int64_t T, int d, const f
     if (err != cudaSuccess) return err;
   }
   const RouterAccum& a = scr.acc;
-  if (E <= 32) return launch_topk<1>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, stream);
-  if (E <= 64) return launch_topk<2>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, stream);
-  if (E <= 128) return launch_topk<4>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, stream);
-  if (E <= 256) return launch_topk<8>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, stream);
-  if (E <= 512) return launch_topk<16>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, stream);
-  return launch_topk<32>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, stream);
+  if (E <= 32) return launch_topk<1>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, stream);
+  if (E <= 64) return launch_topk<2>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, stream);
+  if (E <= 128) return launch_topk<4>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, stream);
+  if (E <= 256) return launch_topk<8>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, stream);
+  if (E <= 512) return launch_topk<16>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, stream);
+  return launch_topk<32>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, stream);
 }
 
 }  // namespace moe

@@ -154,14 +154,15 @@ def test_launch_count(cuda_ok):
     w = synth.WORKLOADS[3].with_(T=256, d_model=128, d_ff=256)
     got = run_layer(w, dev_inputs(synth.make_inputs(w)))
     # router 3 (prep: weight split + zeroed accumulators, tensor-core logits, top-k with the
-    # statistics), dispatch 3, experts 2, dense MLP 2 (its layer 2 carries the combine)
-    assert got["launches"] == 10
+    # statistics and the dispatch ranks), dispatch 2 (scan, scatter), experts 2, dense MLP 2 (its
+    # layer 2 carries the combine)
+    assert got["launches"] == 9
     w1 = synth.WORKLOADS[2].with_(T=256, d_model=128, d_ff=256)
     got = run_layer(w1, dev_inputs(synth.make_inputs(w1)))
-    assert got["launches"] == 8      # top-1: the combine is fused into the experts' layer 2
+    assert got["launches"] == 7      # top-1: the combine is fused into the experts' layer 2
     w2 = synth.WORKLOADS[4].with_(T=256, d_model=128, d_ff=256)
     got = run_layer(w2, dev_inputs(synth.make_inputs(w2)))
-    assert got["launches"] == 9      # top-2: gather combine kernel
+    assert got["launches"] == 8      # top-2: gather combine kernel
 
 
 @pytest.mark.parametrize("cfg", [2, 3, 4])
