@@ -17,7 +17,7 @@
 //                           bases, runs of segments in parallel) and the demand;
 //                           kept = min(demand, C); exclusive scan over experts -> offsets
 //   dispatch_scatter_kernel one warp per pair: position = segment base + rank, slot = position
-//                           or -1 beyond C, row_token, and a 16-byte vector copy of the row
+//                           or -1 beyond C, row_token, and 16-byte vector copies of the row
 #include <type_traits>
 
 #include "common.cuh"
@@ -81,21 +81,40 @@ __global__ void __launch_bounds__(1024)
   const bool active = tid < G * E;
   const int e = active ? tid % E : 0, g = active ? tid / E : 0;
   const int64_t s0 = (int64_t)g * chunk, s1 = min(nseg, s0 + chunk);
+  // runs of up to kBatch segments are held in registers: one sweep of independent loads
+  constexpr int kBatch = 32;
+  int vals[kBatch];
+  const bool in_regs = chunk <= kBatch;
   int sum = 0;
   if (active) {
+    if (in_regs) {
+#pragma unroll
+      for (int b = 0; b < kBatch; ++b) vals[b] = (s0 + b < s1) ? seg_counts[(s0 + b) * E + e] : 0;
+#pragma unroll
+      for (int b = 0; b < kBatch; ++b) sum += vals[b];
+    } else {
 #pragma unroll 8
-    for (int64_t s = s0; s < s1; ++s) sum += seg_counts[s * E + e];
+      for (int64_t s = s0; s < s1; ++s) sum += seg_counts[s * E + e];
+    }
     run_sum[tid] = sum;
   }
   __syncthreads();
   if (active) {
     int run = 0;
     for (int gg = 0; gg < g; ++gg) run += run_sum[gg * E + e];
+    if (in_regs) {
+#pragma unroll
+      for (int b = 0; b < kBatch; ++b) {
+        if (s0 + b < s1) seg_base[(s0 + b) * E + e] = run;
+        run += vals[b];
+      }
+    } else {
 #pragma unroll 8
-    for (int64_t s = s0; s < s1; ++s) {
-      const int v = seg_counts[s * E + e];
-      seg_base[s * E + e] = run;
-      run += v;
+      for (int64_t s = s0; s < s1; ++s) {
+        const int v = seg_counts[s * E + e];
+        seg_base[s * E + e] = run;
+        run += v;
+      }
     }
     if (g == G - 1) {
       counts[e] = run;
@@ -131,6 +150,11 @@ __global__ void __launch_bounds__(1024)
   pdl_trigger();
 }
 
+constexpr int kScatterPairsPerWarp = 1;  // measured: more pairs per warp is slower
+
+// One warp per kScatterPairsPerWarp consecutive pairs: the first lanes resolve the pairs' slots and
+// packed rows, then the warp copies the kept rows, each lane issuing its loads before its stores
+// (16-byte vectors when the row allows).
 template <int VEC_BYTES>
 __global__ void __launch_bounds__(256)
     dispatch_scatter_kernel(const uint8_t* __restrict__ x, int64_t row_bytes, int64_t pairs, int k,
@@ -140,22 +164,43 @@ __global__ void __launch_bounds__(256)
                             const int32_t* __restrict__ offsets, int32_t* __restrict__ slot,
                             int32_t* __restrict__ row_token, uint8_t* __restrict__ x_packed,
                             int64_t rows_max, DroppedRows dropped, int d, int seg_len) {
+  constexpr int P = kScatterPairsPerWarp;
   pdl_wait();
   const int lane = threadIdx.x & 31;
-  const int64_t p = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (p >= pairs) return;
-  const int e = ids[p];
-  const int r = local_rank[p];
-  int s = -1;
-  if (e >= 0 && e < E && r >= 0) {
-    const int pos = seg_base[(p / seg_len) * E + e] + r;
-    if (pos < C) s = pos;
+  const int64_t p0 = (((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5) * P;
+  if (p0 >= pairs) return;
+  int my_s = -1;
+  int64_t my_row = -1;
+  if (lane < P && p0 + lane < pairs) {
+    const int64_t p = p0 + lane;
+    const int e = ids[p];
+    const int r = local_rank[p];
+    if (e >= 0 && e < E && r >= 0) {
+      const int pos = seg_base[(p / seg_len) * E + e] + r;
+      if (pos < C) my_s = pos;
+    }
+    slot[p] = my_s;
+    if (my_s >= 0) {
+      my_row = (int64_t)offsets[e] + my_s;
+      if (my_row < rows_max) row_token[my_row] = (int32_t)(p / k);
+      else my_row = -1;  // cannot happen with rows_max >= min(T k, E C)
+    }
   }
-  if (lane == 0) slot[p] = s;
-  if (s < 0) {
-    if (dropped.out != nullptr) {
-      // top-1 with the combine fused into layer 2: this token's output is its residual alone
-      const int64_t t = p / k;
+  int64_t rows[P], toks[P];
+  int ss[P];
+#pragma unroll
+  for (int q = 0; q < P; ++q) {
+    ss[q] = __shfl_sync(0xffffffffu, my_s, q);
+    rows[q] = __shfl_sync(0xffffffffu, my_row, q);
+    toks[q] = (p0 + q) / k;
+    if (p0 + q >= pairs) ss[q] = -2;  // no such pair
+  }
+  if (dropped.out != nullptr) {
+    // top-1 with the combine fused into layer 2: a dropped token's output is its residual alone
+#pragma unroll
+    for (int q = 0; q < P; ++q) {
+      if (ss[q] != -1) continue;
+      const int64_t t = toks[q];
       for (int64_t i = lane; i < d; i += 32) {
         float v = 0.0f;
         if (dropped.add_x)
@@ -165,18 +210,29 @@ __global__ void __launch_bounds__(256)
         else reinterpret_cast<float*>(dropped.out)[t * d + i] = v;
       }
     }
-    return;
   }
-  const int64_t row = (int64_t)offsets[e] + s;
-  if (row >= rows_max) return;  // cannot happen with rows_max >= min(T k, E C)
-  const int64_t t = p / k;
-  if (lane == 0) row_token[row] = (int32_t)t;
   using V = typename std::conditional<VEC_BYTES == 16, uint4,
             typename std::conditional<VEC_BYTES == 8, uint2, uint32_t>::type>::type;
-  const V* src = reinterpret_cast<const V*>(x + t * row_bytes);
-  V* dst = reinterpret_cast<V*>(x_packed + row * row_bytes);
   const int64_t n = row_bytes / VEC_BYTES;
-  for (int64_t i = lane; i < n; i += 32) dst[i] = src[i];
+  for (int64_t i0 = lane; i0 < n; i0 += 4 * 32) {
+    V v[P][4];
+#pragma unroll
+    for (int q = 0; q < P; ++q) {
+      if (rows[q] < 0) continue;
+      const V* src = reinterpret_cast<const V*>(x + toks[q] * row_bytes);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (i0 + 32 * u < n) v[q][u] = src[i0 + 32 * u];
+    }
+#pragma unroll
+    for (int q = 0; q < P; ++q) {
+      if (rows[q] < 0) continue;
+      V* dst = reinterpret_cast<V*>(x_packed + rows[q] * row_bytes);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (i0 + 32 * u < n) dst[i0 + 32 * u] = v[q][u];
+    }
+  }
   pdl_trigger();
 }
 
@@ -205,7 +261,8 @@ cudaError_t enqueue_dispatch(const void* x, bool bf16, int64_t T, int d, const i
   }
   if (pairs > 0) {
     const int64_t row_bytes = (int64_t)d * (bf16 ? 2 : 4);
-    const unsigned blocks = (unsigned)((pairs * 32 + 255) / 256);
+    const int64_t warps = (pairs + kScatterPairsPerWarp - 1) / kScatterPairsPerWarp;
+    const unsigned blocks = (unsigned)((warps * 32 + 255) / 256);
     const uint8_t* xs = (const uint8_t*)x;
     uint8_t* xp = (uint8_t*)x_packed;
     auto launch = [&](auto kern) {

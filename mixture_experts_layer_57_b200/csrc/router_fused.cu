@@ -32,7 +32,7 @@ struct RCfg {
   static constexpr int kABytes = kTM * kBK * 2;           // 16 KB
   static constexpr int kBPartBytes = NE * kBK * 2;        // per weight part
   static constexpr int kStageBytes = kABytes + 3 * kBPartBytes;
-  static constexpr int kStagesFit = (188 * 1024) / kStageBytes;
+  static constexpr int kStagesFit = (200 * 1024) / kStageBytes;  // 3 stages at NE = 128
   static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
   static constexpr int kTmemCols = (2 * NE) < 32 ? 32 : (2 * NE);
   static constexpr int kBarBytes = 8 * 32;
