@@ -66,8 +66,15 @@ def lib():
         L.oracle_ffn.restype = None
         L.oracle_combine.argtypes = [i64, i32, i32, vp, i32, vp, vp, vp, vp, vp]
         L.oracle_combine.restype = None
+        L.oracle_assign_slots_priority.argtypes = [vp, vp, i64, i32, i32, i64, vp, vp]
+        L.oracle_assign_slots_priority.restype = None
+        L.oracle_renormalize_gates.argtypes = [vp, i64, i32]
+        L.oracle_renormalize_gates.restype = None
+        L.oracle_router_losses.argtypes = [vp, vp, vp, i64, i32, i32, vp, vp, vp]
+        L.oracle_router_losses.restype = None
         L.oracle_layer_forward.argtypes = (
-            [i64, i32, i32, i32, i32, dbl, i32, i32] + [vp] * 11 + [dbl, vp, vp, i64] + [vp] * 8 + [i32])
+            [i64, i32, i32, i32, i32, dbl, i32, i32] + [vp] * 11 + [dbl, vp, vp, i64] + [vp] * 8
+            + [i32, i32, i32, vp, vp])
         L.oracle_layer_forward.restype = i64
         _lib = L
     return _lib
@@ -152,6 +159,37 @@ def assign_slots(ids: np.ndarray, E: int, C: int):
     return slot, counts
 
 
+def assign_slots_priority(ids: np.ndarray, gates: np.ndarray, E: int, C: int):
+    """Priority overflow: (slot [T,k], counts [E]); ranks by gate desc, then pair index."""
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    gates = np.ascontiguousarray(gates, dtype=np.float32)
+    T, k = ids.shape
+    slot = np.empty((T, k), dtype=np.int32)
+    counts = np.empty(E, dtype=np.int32)
+    lib().oracle_assign_slots_priority(_p(ids), _p(gates), T, k, E, C, _p(slot), _p(counts))
+    return slot, counts
+
+
+def renormalize_gates(gates: np.ndarray) -> np.ndarray:
+    g = np.array(gates, dtype=np.float32, copy=True, order="C")
+    T, k = g.shape
+    lib().oracle_renormalize_gates(_p(g), T, k)
+    return g
+
+
+def router_losses(logits: np.ndarray, ids: np.ndarray, gates: np.ndarray):
+    """(z_loss, cov2_importance, cov2_load) in double."""
+    logits = np.ascontiguousarray(logits, dtype=np.float32)
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    gates = np.ascontiguousarray(gates, dtype=np.float32)
+    T, E = logits.shape
+    k = ids.shape[1]
+    out = np.empty(3)
+    lib().oracle_router_losses(_p(logits), _p(ids), _p(gates), T, E, k, _p(out[0:1]), _p(out[1:2]),
+                               _p(out[2:3]))
+    return float(out[0]), float(out[1]), float(out[2])
+
+
 def ffn(x_row: np.ndarray, w1, b1, w2, b2) -> np.ndarray:
     """One two-layer GeLU FFN on one token row; returns y [d] fp32."""
     d = x_row.shape[-1]
@@ -179,7 +217,8 @@ def combine(gates, slot, y, residual=None, dense=None) -> np.ndarray:
 def layer_forward(inp: dict, T: int, d_model: int, d_ff: int, E: int, k: int,
                   capacity_factor: float, add_input_residual: bool = True, aux_alpha: float = 0.01,
                   logits_in: Optional[np.ndarray] = None, tokens: Optional[np.ndarray] = None,
-                  out_bf16: Optional[bool] = None) -> dict:
+                  out_bf16: Optional[bool] = None, overflow_priority: bool = False,
+                  renormalize: bool = False, gates_in: Optional[np.ndarray] = None) -> dict:
     """The whole layer on host arrays (``synth.make_inputs`` layout).
 
     Returns dict: logits, ids, gates, slot, counts, C, f, Q, aux, out_exact [n,d] f64,
@@ -200,7 +239,9 @@ def layer_forward(inp: dict, T: int, d_model: int, d_ff: int, E: int, k: int,
     stats = np.empty(2 * E + 1, dtype=np.float64)
     out_exact = np.empty((n, d_model), dtype=np.float64)
     out = np.empty((n, d_model), dtype=np.uint16 if out_bf16 else np.float32)
+    losses = np.empty(3, dtype=np.float64)
     li = None if logits_in is None else np.ascontiguousarray(logits_in, dtype=np.float32)
+    gi = None if gates_in is None else np.ascontiguousarray(gates_in, dtype=np.float32)
     g = inp.get
     C = L.oracle_layer_forward(
         T, d_model, d_ff, E, k, capacity_factor, bf16, int(bool(add_input_residual)),
@@ -209,7 +250,8 @@ def layer_forward(inp: dict, T: int, d_model: int, d_ff: int, E: int, k: int,
         _p(g("dense_w1")), _p(g("dense_b1")), _p(g("dense_w2")), _p(g("dense_b2")),
         aux_alpha, _p(li), _p(tok), n,
         _p(logits), _p(ids), _p(gates), _p(slot), _p(counts), _p(stats), _p(out_exact), _p(out),
-        int(bool(out_bf16)))
+        int(bool(out_bf16)), int(bool(overflow_priority)), int(bool(renormalize)), _p(gi), _p(losses))
     return dict(logits=logits, ids=ids, gates=gates, slot=slot, counts=counts, C=int(C),
                 f=stats[:E], Q=stats[E:2 * E], aux=float(stats[2 * E]), out_exact=out_exact,
-                out=out, tokens=tok)
+                out=out, tokens=tok, z_loss=float(losses[0]), cov2_importance=float(losses[1]),
+                cov2_load=float(losses[2]))

@@ -40,6 +40,7 @@
 //     aux = alpha * E * sum_i f_i Q_i (survey notes §1.1.4.1, Switch Transformer loss).
 #include <cmath>
 #include <cstdint>
+#include <algorithm>
 #include <cstring>
 #include <vector>
 
@@ -179,6 +180,77 @@ void oracle_assign_slots(const int32_t* ids, int64_t T, int k, int E, int64_t C,
   for (int e = 0; e < E; ++e) counts[e] = (int32_t)cnt[e];
 }
 
+// Priority overflow (a routing variant): inside each expert, the pairs are ranked by router
+// probability, highest first (equal probabilities: lower pair index first), and the first C
+// ranks are kept. The comparison article's capacity example ranks E0's tokens by probability
+// (t3 0.859 > t0 0.817 > t1 0.669) and keeps t3, t0, dropping t1. gates are the fp32 gate
+// values the ranking is decided on.
+void oracle_assign_slots_priority(const int32_t* ids, const float* gates, int64_t T, int k, int E,
+                                  int64_t C, int32_t* slot, int32_t* counts) {
+  std::vector<std::vector<int64_t>> members(E);
+  for (int64_t p = 0; p < T * k; ++p) members[ids[p]].push_back(p);
+  for (int e = 0; e < E; ++e) {
+    std::vector<int64_t>& m = members[e];
+    std::sort(m.begin(), m.end(), [&](int64_t a, int64_t b) {
+      if (gates[a] != gates[b]) return gates[a] > gates[b];
+      return a < b;
+    });
+    for (size_t r = 0; r < m.size(); ++r) slot[m[r]] = (int64_t)r < C ? (int32_t)r : -1;
+    counts[e] = (int32_t)m.size();
+  }
+}
+
+// Renormalised gates (a routing variant): the k chosen probabilities divided by their sum (the
+// survey notes §1.1.1.1: taking top-k after the softmax leaves values that need an extra
+// normalisation). Computed in double from the given fp32 gates, rounded to fp32.
+void oracle_renormalize_gates(float* gates, int64_t T, int k) {
+  for (int64_t t = 0; t < T; ++t) {
+    double s = 0.0;
+    for (int j = 0; j < k; ++j) s += (double)gates[t * k + j];
+    for (int j = 0; j < k; ++j) gates[t * k + j] = (float)((double)gates[t * k + j] / s);
+  }
+}
+
+// Extra router statistics:
+//   z-loss L_z = (1/T) sum_t (log sum_e exp(l_te))^2 (comparison article, "Router Z-loss");
+//   CoV^2 of Importance_i = sum over choices routed to i of their gate, and of Load_i = number of
+//   choices routed to i (survey notes §1.1.4.1, Importance and Load losses; without noise the
+//   probability that expert i is selected is the indicator of the selection). CoV = std / mean
+//   with the population variance; 0 when the mean is 0.
+static double cov2(const std::vector<double>& v) {
+  double mean = 0.0;
+  for (double a : v) mean += a;
+  mean /= (double)v.size();
+  if (mean == 0.0) return 0.0;
+  double var = 0.0;
+  for (double a : v) var += (a - mean) * (a - mean);
+  var /= (double)v.size();
+  return var / (mean * mean);
+}
+
+void oracle_router_losses(const float* logits, const int32_t* ids, const float* gates, int64_t T,
+                          int E, int k, double* z_loss, double* cov2_importance,
+                          double* cov2_load) {
+  double z = 0.0;
+  for (int64_t t = 0; t < T; ++t) {
+    const float* l = logits + t * E;
+    double m = -INFINITY;
+    for (int e = 0; e < E; ++e) m = (double)l[e] > m ? (double)l[e] : m;
+    double s = 0.0;
+    for (int e = 0; e < E; ++e) s += std::exp((double)l[e] - m);
+    const double lz = m + std::log(s);
+    z += lz * lz;
+  }
+  *z_loss = T > 0 ? z / (double)T : 0.0;
+  std::vector<double> imp(E, 0.0), load(E, 0.0);
+  for (int64_t p = 0; p < T * k; ++p) {
+    imp[ids[p]] += (double)gates[p];
+    load[ids[p]] += 1.0;
+  }
+  *cov2_importance = cov2(imp);
+  *cov2_load = cov2(load);
+}
+
 // ---------------------------------------------------------------- expert FFN
 
 // One expert (or the dense MLP) on one token: z = W1 x + b1, h = GeLU(z) (rounded to
@@ -241,7 +313,8 @@ int64_t oracle_layer_forward(int64_t T, int d, int d_ff, int E, int k, double ca
                              const float* logits_in, const int64_t* tokens, int64_t n_tokens,
                              float* logits_out, int32_t* ids, float* gates, int32_t* slot,
                              int32_t* counts, double* lb_stats, double* out_exact,
-                             void* out_rounded, int out_bf16) {
+                             void* out_rounded, int out_bf16, int overflow_priority,
+                             int renormalize, const float* gates_in, double* losses) {
   std::vector<float> logits_own;
   const float* logits = logits_in;
   if (!logits) {
@@ -251,9 +324,15 @@ int64_t oracle_layer_forward(int64_t T, int d, int d_ff, int E, int k, double ca
   }
   if (logits_out && logits_out != logits) std::memcpy(logits_out, logits, sizeof(float) * T * E);
   oracle_route(logits, T, E, k, ids, gates, nullptr);
+  if (renormalize) oracle_renormalize_gates(gates, T, k);
+  // gates_in: the gate values another implementation decided on (a priority ranking between two
+  // nearly equal probabilities is decided in that implementation's precision); NULL = own gates
+  if (gates_in && gates_in != gates) std::memcpy(gates, gates_in, sizeof(float) * T * k);
   if (lb_stats) oracle_lb_stats(logits, ids, T, E, k, aux_alpha, lb_stats, lb_stats + E, lb_stats + 2 * E);
+  if (losses) oracle_router_losses(logits, ids, gates, T, E, k, losses, losses + 1, losses + 2);
   const int64_t C = oracle_capacity(T, E, k, capacity_factor);
-  oracle_assign_slots(ids, T, k, E, C, slot, counts);
+  if (overflow_priority) oracle_assign_slots_priority(ids, gates, T, k, E, C, slot, counts);
+  else oracle_assign_slots(ids, T, k, E, C, slot, counts);
 
   const int64_t n = tokens ? n_tokens : T;
   const size_t esz = bf16 ? 2 : 4;
