@@ -44,7 +44,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 1
+#define MOE_ABI_VERSION 2
 #define MOE_STATUS_BLOCK_BYTES 256
 #define MOE_MAX_EXPERTS 1024
 #define MOE_MAX_TOPK 8
@@ -110,6 +110,22 @@ moe_status moe_router_topk(const void* x, moe_dtype x_dtype, int64_t T, int d_mo
                            float* logits, int32_t* expert_ids, float* gates, float* lb_stats,
                            float aux_alpha, void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* moe_router_topk with two routing variants (same workspace):
+ * renormalize != 0: gates[t,j] = p[t,e_j] / sum_{j'} p[t,e_j'] (the k chosen probabilities
+ *               renormalised to sum to 1: MoE survey notes §1.1.1.1, top-k after the softmax).
+ * router_losses (NULL or [3] fp32 output):
+ *   [0] z-loss = (1/T) sum_t (log sum_e exp(logits[t,e]))^2 (comparison article, "Router
+ *       Z-loss"; without the coefficient);
+ *   [1] CoV^2 of Importance_i = sum of the gates routed to expert i (after renormalisation);
+ *   [2] CoV^2 of Load_i = number of choices routed to expert i
+ *   (MoE survey notes §1.1.4.1; CoV = standard deviation / mean with the population variance,
+ *   0 when the mean is 0; without the coefficients). lb_stats still uses the softmax p. */
+moe_status moe_router_topk_ex(const void* x, moe_dtype x_dtype, int64_t T, int d_model,
+                              const float* w_router, const float* router_bias, int E, int k,
+                              float* logits, int32_t* expert_ids, float* gates, float* lb_stats,
+                              float aux_alpha, int renormalize, float* router_losses, void* ws,
+                              size_t ws_bytes, moe_stream_t stream);
+
 /* ---------------------------------------------------------------- dispatch
  * pack_by_expert with a capacity (DeepSpeed MoE blog, pipeline listing; DeepSpeed-MoE notes
  * §4.4: top-k + prefix-sum + scatter into a dense token-to-expert mapping table, then an
@@ -129,6 +145,19 @@ moe_status moe_dispatch(const void* x, moe_dtype dtype, int64_t T, int d_model,
                         int32_t* expert_counts, int32_t* expert_offsets, int32_t* row_token,
                         void* x_packed, int64_t rows_max, void* ws, size_t ws_bytes,
                         moe_stream_t stream);
+
+/* moe_dispatch with overflow by priority (comparison article, "Expert Capacity Overflow": the
+ * tokens of highest router probability keep the capacity): the pairs of each expert are ranked
+ * by gate, largest first, ties to the lower pair index p = t * k + j; slot[t,j] = rank if
+ * rank < C, else -1, and kept rows are packed in rank order. gates: [T, k] fp32 (the router's,
+ * renormalised or not). Counts, offsets, row_token and x_packed follow moe_dispatch. Same
+ * workspace as moe_dispatch. */
+moe_status moe_dispatch_priority(const void* x, moe_dtype dtype, int64_t T, int d_model,
+                                 const int32_t* expert_ids, const float* gates, int E, int k,
+                                 int64_t C, int32_t* slot, int32_t* expert_counts,
+                                 int32_t* expert_offsets, int32_t* row_token, void* x_packed,
+                                 int64_t rows_max, void* ws, size_t ws_bytes,
+                                 moe_stream_t stream);
 
 /* Allocation-free variant of moe_dispatch (no counterpart on the pages: it exists for callers).
  * Some callers cannot allocate device memory at all: a plug-in running inside a host application
@@ -214,7 +243,13 @@ typedef struct {
   const void *dense_w1, *dense_b1, *dense_w2, *dense_b2;
   int add_input_residual; /* 1: out += x */
   float aux_alpha;        /* alpha of the load-balance loss */
+  int overflow_policy;    /* moe_overflow_policy */
+  int renormalize_gates;  /* 1: gates renormalised over the k choices (moe_router_topk_ex) */
 } moe_layer_args;
+
+/* Which pairs an expert keeps when its demand exceeds C: the first in token order (moe_dispatch),
+ * or those of largest gate (moe_dispatch_priority). */
+typedef enum { MOE_OVERFLOW_FIRST_COME = 0, MOE_OVERFLOW_PRIORITY = 1 } moe_overflow_policy;
 
 /* Optional device outputs of the intermediate results; any field may be NULL. */
 typedef struct {
@@ -225,6 +260,7 @@ typedef struct {
   int32_t* expert_counts; /* [E] demand */
   int32_t* expert_offsets;/* [E+1] */
   float* lb_stats;        /* [2E+1] */
+  float* router_losses;   /* [3]: z-loss, CoV^2 Importance, CoV^2 Load (moe_router_topk_ex) */
 } moe_layer_aux;
 
 /* out = [x if add_input_residual] + [DenseMLP(x) if dense_*] + sum_j gate_j * Expert_{e_j}(x)

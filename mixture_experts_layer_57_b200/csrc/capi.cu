@@ -79,6 +79,9 @@ RouterWs carve_router(Carve& c, int64_t T, int E, int d) {
   RouterWs w;
   w.scr.acc.q = c.take<unsigned long long>((size_t)E);
   w.scr.acc.c = c.take<unsigned>((size_t)E);
+  w.scr.acc.imp = c.take<unsigned long long>((size_t)E);
+  w.scr.acc.load = c.take<unsigned>((size_t)E);
+  w.scr.acc.z = c.take<unsigned long long>(1);
   w.scr.acc.ticket = c.take<unsigned>(1);
   w.scr.w_split = c.take<uint16_t>((size_t)E * 3 * router_split_dpad(d));
   w.logits = c.take<float>((size_t)T * E);
@@ -88,6 +91,7 @@ RouterWs carve_router(Carve& c, int64_t T, int E, int d) {
 
 struct DispatchWs {
   int32_t *local_rank, *seg_counts, *seg_base;
+  int32_t *prio_list, *demand_offsets;  // overflow by priority
 };
 DispatchWs carve_dispatch(Carve& c, int64_t T, int E, int k) {
   // segments of 256 pairs (counting kernel) or of one 64-token router block (layer forward)
@@ -98,6 +102,8 @@ DispatchWs carve_dispatch(Carve& c, int64_t T, int E, int k) {
   w.local_rank = c.take<int32_t>((size_t)T * k);
   w.seg_counts = c.take<int32_t>((size_t)nseg * E);
   w.seg_base = c.take<int32_t>((size_t)nseg * E);
+  w.prio_list = c.take<int32_t>((size_t)T * k);
+  w.demand_offsets = c.take<int32_t>((size_t)E + 1);
   return w;
 }
 
@@ -172,10 +178,12 @@ moe_status moe_router_workspace_bytes(int64_t T, int E, int d_model, size_t* byt
   return MOE_OK;
 }
 
-moe_status moe_router_topk(const void* x, moe_dtype x_dtype, int64_t T, int d_model,
-                           const float* w_router, const float* router_bias, int E, int k,
-                           float* logits, int32_t* expert_ids, float* gates, float* lb_stats,
-                           float aux_alpha, void* ws, size_t ws_bytes, moe_stream_t stream) {
+namespace {
+moe_status router_topk_impl(const char* entry, const void* x, moe_dtype x_dtype, int64_t T,
+                            int d_model, const float* w_router, const float* router_bias, int E,
+                            int k, float* logits, int32_t* expert_ids, float* gates,
+                            float* lb_stats, float aux_alpha, int renormalize,
+                            float* router_losses, void* ws, size_t ws_bytes, moe_stream_t stream) {
   if (!valid_dtype(x_dtype)) return MOE_ERR_INVALID_ARGUMENT;
   moe_status st = check_router_shape(T, d_model, E, k);
   if (st != MOE_OK) return st;
@@ -183,19 +191,40 @@ moe_status moe_router_topk(const void* x, moe_dtype x_dtype, int64_t T, int d_mo
   if (!ws) return MOE_ERR_INVALID_ARGUMENT;
   if (!aligned16(x) || !aligned16(w_router) || !aligned16(router_bias) || !aligned16(logits) ||
       !aligned16(expert_ids) || !aligned16(gates) || !aligned16(lb_stats) ||
-      ((uintptr_t)ws % kAlign) != 0)
+      !aligned16(router_losses) || ((uintptr_t)ws % kAlign) != 0)
     return MOE_ERR_MISALIGNED;
   size_t need = 0;
   moe_router_workspace_bytes(T, E, d_model, &need);
   if (ws_bytes < need) return MOE_ERR_WORKSPACE_TOO_SMALL;
-  if (fault_injected("moe_router_topk")) return MOE_ERR_CUDA;
+  if (fault_injected(entry)) return MOE_ERR_CUDA;
   g_launches = 0;
   if (T == 0) return MOE_OK;
   Carve c{(uint8_t*)ws};
   RouterWs w = carve_router(c, T, E, d_model);
   return cuda_status(enqueue_router(x, x_dtype == MOE_BF16, T, d_model, w_router, router_bias, E,
                                     k, logits, expert_ids, gates, lb_stats, aux_alpha, w.scr,
-                                    (int*)ws, stream));
+                                    (int*)ws, stream, RouterDispatchCount{}, renormalize != 0,
+                                    router_losses));
+}
+}  // namespace
+
+moe_status moe_router_topk(const void* x, moe_dtype x_dtype, int64_t T, int d_model,
+                           const float* w_router, const float* router_bias, int E, int k,
+                           float* logits, int32_t* expert_ids, float* gates, float* lb_stats,
+                           float aux_alpha, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  return router_topk_impl("moe_router_topk", x, x_dtype, T, d_model, w_router, router_bias, E, k,
+                          logits, expert_ids, gates, lb_stats, aux_alpha, 0, nullptr, ws,
+                          ws_bytes, stream);
+}
+
+moe_status moe_router_topk_ex(const void* x, moe_dtype x_dtype, int64_t T, int d_model,
+                              const float* w_router, const float* router_bias, int E, int k,
+                              float* logits, int32_t* expert_ids, float* gates, float* lb_stats,
+                              float aux_alpha, int renormalize, float* router_losses, void* ws,
+                              size_t ws_bytes, moe_stream_t stream) {
+  return router_topk_impl("moe_router_topk_ex", x, x_dtype, T, d_model, w_router, router_bias, E,
+                          k, logits, expert_ids, gates, lb_stats, aux_alpha, renormalize,
+                          router_losses, ws, ws_bytes, stream);
 }
 
 // ---------------------------------------------------------------- dispatch
@@ -208,11 +237,12 @@ moe_status moe_dispatch_workspace_bytes(int64_t T, int E, int k, size_t* bytes) 
   return MOE_OK;
 }
 
-moe_status moe_dispatch(const void* x, moe_dtype dtype, int64_t T, int d_model,
-                        const int32_t* expert_ids, int E, int k, int64_t C, int32_t* slot,
-                        int32_t* expert_counts, int32_t* expert_offsets, int32_t* row_token,
-                        void* x_packed, int64_t rows_max, void* ws, size_t ws_bytes,
-                        moe_stream_t stream) {
+namespace {
+moe_status dispatch_impl(const char* entry, const void* x, moe_dtype dtype, int64_t T,
+                         int d_model, const int32_t* expert_ids, const float* prio_gates, int E,
+                         int k, int64_t C, int32_t* slot, int32_t* expert_counts,
+                         int32_t* expert_offsets, int32_t* row_token, void* x_packed,
+                         int64_t rows_max, void* ws, size_t ws_bytes, moe_stream_t stream) {
   if (!valid_dtype(dtype) || C < 0) return MOE_ERR_INVALID_ARGUMENT;
   moe_status st = check_router_shape(T, d_model, E, k);
   if (st != MOE_OK) return st;
@@ -226,18 +256,46 @@ moe_status moe_dispatch(const void* x, moe_dtype dtype, int64_t T, int d_model,
   if (rows_max > 0 && (!row_token || !x_packed)) return MOE_ERR_INVALID_ARGUMENT;
   if (!aligned16(x) || !aligned16(expert_ids) || !aligned16(slot) || !aligned16(expert_counts) ||
       !aligned16(expert_offsets) || !aligned16(row_token) || !aligned16(x_packed) ||
-      ((uintptr_t)ws % kAlign) != 0)
+      !aligned16(prio_gates) || ((uintptr_t)ws % kAlign) != 0)
     return MOE_ERR_MISALIGNED;
   size_t need = 0;
   moe_dispatch_workspace_bytes(T, E, k, &need);
   if (ws_bytes < need) return MOE_ERR_WORKSPACE_TOO_SMALL;
-  if (fault_injected("moe_dispatch")) return MOE_ERR_CUDA;
+  if (fault_injected(entry)) return MOE_ERR_CUDA;
   g_launches = 0;
   Carve c{(uint8_t*)ws};
   DispatchWs w = carve_dispatch(c, T, E, k);
+  PriorityDispatch prio;
+  prio.gates = prio_gates;
+  prio.list = w.prio_list;
+  prio.demand_offsets = w.demand_offsets;
   return cuda_status(enqueue_dispatch(x, dtype == MOE_BF16, T, d_model, expert_ids, E, k, C, slot,
                                       expert_counts, expert_offsets, row_token, x_packed, rows_max,
-                                      w.local_rank, w.seg_counts, w.seg_base, (int*)ws, stream));
+                                      w.local_rank, w.seg_counts, w.seg_base, (int*)ws, stream,
+                                      DroppedRows{}, 0, prio));
+}
+}  // namespace
+
+moe_status moe_dispatch(const void* x, moe_dtype dtype, int64_t T, int d_model,
+                        const int32_t* expert_ids, int E, int k, int64_t C, int32_t* slot,
+                        int32_t* expert_counts, int32_t* expert_offsets, int32_t* row_token,
+                        void* x_packed, int64_t rows_max, void* ws, size_t ws_bytes,
+                        moe_stream_t stream) {
+  return dispatch_impl("moe_dispatch", x, dtype, T, d_model, expert_ids, nullptr, E, k, C, slot,
+                       expert_counts, expert_offsets, row_token, x_packed, rows_max, ws, ws_bytes,
+                       stream);
+}
+
+moe_status moe_dispatch_priority(const void* x, moe_dtype dtype, int64_t T, int d_model,
+                                 const int32_t* expert_ids, const float* gates, int E, int k,
+                                 int64_t C, int32_t* slot, int32_t* expert_counts,
+                                 int32_t* expert_offsets, int32_t* row_token, void* x_packed,
+                                 int64_t rows_max, void* ws, size_t ws_bytes,
+                                 moe_stream_t stream) {
+  if (T > 0 && !gates) return MOE_ERR_INVALID_ARGUMENT;
+  return dispatch_impl("moe_dispatch_priority", x, dtype, T, d_model, expert_ids,
+                       T > 0 ? gates : nullptr, E, k, C, slot, expert_counts, expert_offsets,
+                       row_token, x_packed, rows_max, ws, ws_bytes, stream);
 }
 
 // ---------------------------------------------------------------- expert FFN
@@ -353,6 +411,8 @@ moe_status layer_layout(const moe_layer_args* a, uint8_t* base, LayerWs* w, size
   moe_status st = check_router_shape(a->T, a->d_model, a->E, a->k);
   if (st != MOE_OK) return st;
   if (!valid_dtype(a->dtype) || !valid_dtype(a->out_dtype)) return MOE_ERR_INVALID_ARGUMENT;
+  if (a->overflow_policy != MOE_OVERFLOW_FIRST_COME && a->overflow_policy != MOE_OVERFLOW_PRIORITY)
+    return MOE_ERR_INVALID_ARGUMENT;
   st = moe_capacity(a->T, a->E, a->k, a->capacity_factor, &w->C);
   if (st != MOE_OK) return st;
   moe_packed_rows_max(a->T, a->E, a->k, w->C, &w->rows_max);
@@ -437,7 +497,8 @@ moe_status layer_forward_impl(const moe_layer_args* a, void* out, moe_layer_aux*
     return MOE_ERR_MISALIGNED;
   if (aux && (!aligned16(aux->logits) || !aligned16(aux->expert_ids) || !aligned16(aux->gates) ||
               !aligned16(aux->slot) || !aligned16(aux->expert_counts) ||
-              !aligned16(aux->expert_offsets) || !aligned16(aux->lb_stats)))
+              !aligned16(aux->expert_offsets) || !aligned16(aux->lb_stats) ||
+              !aligned16(aux->router_losses)))
     return MOE_ERR_MISALIGNED;
   if (ws_bytes < need) return MOE_ERR_WORKSPACE_TOO_SMALL;
   if (fault_injected("moe_layer_forward")) return MOE_ERR_CUDA;
@@ -451,6 +512,7 @@ moe_status layer_forward_impl(const moe_layer_args* a, void* out, moe_layer_aux*
   int32_t* counts = aux && aux->expert_counts ? aux->expert_counts : w.counts;
   int32_t* offsets = aux && aux->expert_offsets ? aux->expert_offsets : w.offsets;
   float* lb = aux ? aux->lb_stats : nullptr;
+  float* losses = aux ? aux->router_losses : nullptr;
   int* status = (int*)ws;
   const bool bf16 = a->dtype == MOE_BF16;
   const int64_t T = a->T;
@@ -463,7 +525,8 @@ moe_status layer_forward_impl(const moe_layer_args* a, void* out, moe_layer_aux*
   dcount.local_rank = w.dispatch.local_rank;
   dcount.seg_counts = w.dispatch.seg_counts;
   cudaError_t e = enqueue_router(a->x, bf16, T, d, a->w_router, a->router_bias, E, k, logits, ids,
-                                 gates, lb, a->aux_alpha, w.router.scr, status, stream, dcount);
+                                 gates, lb, a->aux_alpha, w.router.scr, status, stream, dcount,
+                                 a->renormalize_gates != 0, losses);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   rec.mark("router");
 
@@ -480,10 +543,16 @@ moe_status layer_forward_impl(const moe_layer_args* a, void* out, moe_layer_aux*
     dropped.out_bf16 = out_bf16;
     dropped.add_x = a->add_input_residual != 0;
   }
+  PriorityDispatch prio;
+  if (a->overflow_policy == MOE_OVERFLOW_PRIORITY) {
+    prio.gates = gates;
+    prio.list = w.dispatch.prio_list;
+    prio.demand_offsets = w.dispatch.demand_offsets;
+  }
   e = enqueue_dispatch(a->x, bf16, T, d, ids, E, k, w.C, slot, counts, offsets, w.row_token,
                        w.x_packed, w.rows_max, w.dispatch.local_rank, w.dispatch.seg_counts,
                        w.dispatch.seg_base, status, stream, dropped,
-                       (int)kRouterTokensPerBlock * k);
+                       (int)kRouterTokensPerBlock * k, prio);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   rec.mark("dispatch");
 

@@ -18,6 +18,17 @@
 //                           kept = min(demand, C); exclusive scan over experts -> offsets
 //   dispatch_scatter_kernel one warp per pair: position = segment base + rank, slot = position
 //                           or -1 beyond C, row_token, and 16-byte vector copies of the row
+//
+// Overflow by priority (comparison article, "Expert Capacity Overflow": the capacity goes to the
+// tokens of highest router probability; Switch-style priority routing): the scan also writes the
+// demand offsets (exclusive prefix of the demands), then
+//   dispatch_list_kernel    one thread per pair: list[demand_offset[e] + position] = pair, i.e.
+//                           each expert's pairs in token order
+//   dispatch_priority_rank_kernel  one block per (expert, 256 of its pairs): a pair's rank is the
+//                           number of the expert's pairs with a larger gate, or an equal gate and
+//                           a lower pair index (shared-memory tiles of the expert's pairs);
+//                           slot = rank, or -1 from C on
+// and the scatter takes those slots instead of the first-come positions.
 #include <type_traits>
 
 #include "common.cuh"
@@ -66,12 +77,42 @@ __global__ void __launch_bounds__(kCountWarps * 32)
 // Thread (g, e) owns a contiguous run of segments of expert e (G = 1024 / E runs per expert): it
 // sums them, takes the sum of the earlier runs from shared memory as its base, then writes the
 // exclusive prefix of its run (the segment bases). The last run's end is the demand.
+// Exclusive prefix over experts of v (one element per thread of a 1024-thread block); thread
+// E - 1 also writes the total to out[E].
+__device__ void block_exclusive_scan_experts(int v, int E, int* warp_sums, int32_t* out) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += u;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int ws = warp_sums[lane];
+    int wincl = ws;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, wincl, o);
+      if (lane >= o) wincl += u;
+    }
+    warp_sums[lane] = wincl - ws;  // exclusive prefix of warp totals
+  }
+  __syncthreads();
+  const int excl = incl - v + warp_sums[warp];
+  if (tid < E) out[tid] = excl;
+  if (tid == E - 1) out[E] = excl + v;
+  __syncthreads();  // warp_sums may be reused
+}
+
 __global__ void __launch_bounds__(1024)
     dispatch_scan_kernel(const int32_t* __restrict__ seg_counts, int64_t nseg, int E, int64_t C,
                          int32_t* __restrict__ seg_base, int32_t* __restrict__ counts,
-                         int32_t* __restrict__ offsets) {
+                         int32_t* __restrict__ offsets, int32_t* __restrict__ demand_offsets) {
   __shared__ int run_sum[1024];
   __shared__ int kept[MOE_MAX_EXPERTS];
+  __shared__ int demand[MOE_MAX_EXPERTS];
   __shared__ int warp_sums[32];
   pdl_wait();
   const int tid = threadIdx.x;
@@ -119,34 +160,78 @@ __global__ void __launch_bounds__(1024)
     if (g == G - 1) {
       counts[e] = run;
       kept[e] = (int)min((int64_t)run, C);
+      demand[e] = run;
     }
   }
   __syncthreads();
-  // exclusive scan of kept over experts (E <= 1024), one element per thread
-  const int lane = tid & 31, warp = tid >> 5;
-  const int v = tid < E ? kept[tid] : 0;
-  int incl = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int u = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += u;
+  // exclusive scans over experts (E <= 1024), one element per thread
+  block_exclusive_scan_experts(tid < E ? kept[tid] : 0, E, warp_sums, offsets);
+  if (demand_offsets != nullptr)
+    block_exclusive_scan_experts(tid < E ? demand[tid] : 0, E, warp_sums, demand_offsets);
+  pdl_trigger();
+}
+
+__global__ void __launch_bounds__(256)
+    dispatch_list_kernel(const int32_t* __restrict__ ids, int64_t pairs, int E,
+                         const int32_t* __restrict__ local_rank,
+                         const int32_t* __restrict__ seg_base, int seg_len,
+                         const int32_t* __restrict__ demand_offsets, int32_t* __restrict__ list) {
+  pdl_wait();
+  const int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (p < pairs) {
+    const int e = ids[p];
+    const int r = local_rank[p];
+    if (e >= 0 && e < E && r >= 0)
+      list[demand_offsets[e] + seg_base[(p / seg_len) * E + e] + r] = (int32_t)p;
   }
-  if (lane == 31) warp_sums[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    int ws = warp_sums[lane];
-    int wincl = ws;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int u = __shfl_up_sync(0xffffffffu, wincl, o);
-      if (lane >= o) wincl += u;
+  pdl_trigger();
+}
+
+constexpr int kRankThreads = 256;
+constexpr int kRankTile = 1024;
+
+// Block (c, e): pairs [256 c, 256 c + 256) of expert e's list. The expert's demand is at most T
+// (a token chooses an expert once), so gridDim.x = ceil(T / 256) covers every list.
+__global__ void __launch_bounds__(kRankThreads)
+    dispatch_priority_rank_kernel(const int32_t* __restrict__ list,
+                                  const int32_t* __restrict__ demand_offsets,
+                                  const int32_t* __restrict__ counts,
+                                  const float* __restrict__ gates, int64_t C,
+                                  int32_t* __restrict__ slot) {
+  __shared__ float tile_g[kRankTile];
+  __shared__ int tile_p[kRankTile];
+  pdl_wait();
+  const int e = blockIdx.y;
+  const int n = counts[e];
+  const int i0 = blockIdx.x * kRankThreads;
+  if (i0 < n) {  // block-uniform
+    const int32_t* mine = list + demand_offsets[e];
+    const int i = i0 + threadIdx.x;
+    int p = -1;
+    float g = 0.0f;
+    if (i < n) {
+      p = mine[i];
+      g = gates[p];
     }
-    warp_sums[lane] = wincl - ws;  // exclusive prefix of warp totals
+    int rank = 0;
+    for (int t0 = 0; t0 < n; t0 += kRankTile) {
+      const int m = min(kRankTile, n - t0);
+      __syncthreads();
+      for (int u = threadIdx.x; u < m; u += kRankThreads) {
+        const int q = mine[t0 + u];
+        tile_p[u] = q;
+        tile_g[u] = gates[q];
+      }
+      __syncthreads();
+      if (i < n) {
+        for (int u = 0; u < m; ++u) {
+          const float gq = tile_g[u];
+          rank += (gq > g || (gq == g && tile_p[u] < p)) ? 1 : 0;
+        }
+      }
+    }
+    if (i < n) slot[p] = rank < C ? rank : -1;
   }
-  __syncthreads();
-  const int excl = incl - v + warp_sums[warp];
-  if (tid < E) offsets[tid] = excl;
-  if (tid == E - 1) offsets[E] = excl + v;
   pdl_trigger();
 }
 
@@ -163,7 +248,8 @@ __global__ void __launch_bounds__(256)
                             const int32_t* __restrict__ seg_base,
                             const int32_t* __restrict__ offsets, int32_t* __restrict__ slot,
                             int32_t* __restrict__ row_token, uint8_t* __restrict__ x_packed,
-                            int64_t rows_max, DroppedRows dropped, int d, int seg_len) {
+                            int64_t rows_max, DroppedRows dropped, int d, int seg_len,
+                            int prio) {
   constexpr int P = kScatterPairsPerWarp;
   pdl_wait();
   const int lane = threadIdx.x & 31;
@@ -176,8 +262,12 @@ __global__ void __launch_bounds__(256)
     const int e = ids[p];
     const int r = local_rank[p];
     if (e >= 0 && e < E && r >= 0) {
-      const int pos = seg_base[(p / seg_len) * E + e] + r;
-      if (pos < C) my_s = pos;
+      if (prio) {
+        my_s = slot[p];  // the priority rank kernel's slot
+      } else {
+        const int pos = seg_base[(p / seg_len) * E + e] + r;
+        if (pos < C) my_s = pos;
+      }
     }
     slot[p] = my_s;
     if (my_s >= 0) {
@@ -243,7 +333,7 @@ cudaError_t enqueue_dispatch(const void* x, bool bf16, int64_t T, int d, const i
                              int32_t* row_token, void* x_packed, int64_t rows_max,
                              int32_t* local_rank, int32_t* seg_counts, int32_t* seg_base,
                              int* status, cudaStream_t stream, DroppedRows dropped,
-                             int counted_seg_len) {
+                             int counted_seg_len, PriorityDispatch prio) {
   const int64_t pairs = T * k;
   const int seg_len = counted_seg_len > 0 ? counted_seg_len : kDispatchSeg;
   const int64_t nseg = (pairs + seg_len - 1) / seg_len;
@@ -256,7 +346,21 @@ cudaError_t enqueue_dispatch(const void* x, bool bf16, int64_t T, int d, const i
   }
   {
     cudaError_t e = launch_kernel(dispatch_scan_kernel, dim3(1), dim3(1024), 0, stream,
-                                  (const int32_t*)seg_counts, nseg, E, C, seg_base, counts, offsets);
+                                  (const int32_t*)seg_counts, nseg, E, C, seg_base, counts, offsets,
+                                  prio.gates != nullptr ? prio.demand_offsets : nullptr);
+    if (e != cudaSuccess) return e;
+  }
+  const int use_prio = prio.gates != nullptr && pairs > 0 ? 1 : 0;
+  if (use_prio) {
+    cudaError_t e = launch_kernel(dispatch_list_kernel, dim3((unsigned)((pairs + 255) / 256)),
+                                  dim3(256), 0, stream, ids, pairs, E,
+                                  (const int32_t*)local_rank, (const int32_t*)seg_base, seg_len,
+                                  (const int32_t*)prio.demand_offsets, prio.list);
+    if (e != cudaSuccess) return e;
+    const dim3 grid((unsigned)((T + kRankThreads - 1) / kRankThreads), (unsigned)E);
+    e = launch_kernel(dispatch_priority_rank_kernel, grid, dim3(kRankThreads), 0, stream,
+                      (const int32_t*)prio.list, (const int32_t*)prio.demand_offsets,
+                      (const int32_t*)counts, prio.gates, C, slot);
     if (e != cudaSuccess) return e;
   }
   if (pairs > 0) {
@@ -269,7 +373,7 @@ cudaError_t enqueue_dispatch(const void* x, bool bf16, int64_t T, int d, const i
       return launch_kernel(kern, dim3(blocks), dim3(256), 0, stream, xs, row_bytes, pairs, k, E, C,
                            ids, (const int32_t*)local_rank, (const int32_t*)seg_base,
                            (const int32_t*)offsets, slot, row_token, xp, rows_max, dropped, d,
-                           seg_len);
+                           seg_len, use_prio);
     };
     cudaError_t e = row_bytes % 16 == 0  ? launch(dispatch_scatter_kernel<16>)
                     : row_bytes % 8 == 0 ? launch(dispatch_scatter_kernel<8>)

@@ -52,9 +52,12 @@ inline int router_split_dpad(int d) { return (d + 63) / 64 * 64; }
 inline bool router_uses_tensor_cores(bool x_bf16, int d) { return x_bf16 && d % 8 == 0; }
 // Load-balance statistics accumulators (zeroed by the router's first kernel each call).
 struct RouterAccum {
-  unsigned long long* q;  // [E] sums of p in 2^-32 fixed point
-  unsigned* c;            // [E] counts of first choices
-  unsigned* ticket;       // blocks finished
+  unsigned long long* q;    // [E] sums of p in 2^-32 fixed point
+  unsigned* c;              // [E] counts of first choices
+  unsigned long long* imp;  // [E] sums of the gates routed to each expert, 2^-24 fixed point
+  unsigned* load;           // [E] counts of all choices routed to each expert
+  unsigned long long* z;    // [1] sum over tokens of (log sum exp logits)^2, 2^-24 fixed point
+  unsigned* ticket;         // blocks finished
 };
 struct RouterScratch {
   RouterAccum acc;
@@ -68,11 +71,14 @@ struct RouterDispatchCount {
   int32_t* seg_counts = nullptr;  // [router_num_blocks(T), E]
 };
 // logits may be nullptr (not returned).
+// renormalize: gates of the k choices divided by their sum. losses (optional): [z-loss,
+// CoV^2 of Importance, CoV^2 of Load].
 cudaError_t enqueue_router(const void* x, bool x_bf16, int64_t T, int d, const float* w_router,
                            const float* router_bias, int E, int k, float* logits, int32_t* ids,
                            float* gates, float* lb_stats, float aux_alpha,
                            const RouterScratch& scratch, int* status, cudaStream_t stream,
-                           RouterDispatchCount dcount = RouterDispatchCount{});
+                           RouterDispatchCount dcount = RouterDispatchCount{},
+                           bool renormalize = false, float* losses = nullptr);
 // logits = x W_r^T + b_r on tcgen05 from the exact split W_r = hi + mid + lo (bf16 each).
 cudaError_t enqueue_router_logits_tc(const void* x, int64_t T, int d, const uint16_t* w_split,
                                      int dpad, const float* router_bias, int E, float* logits,
@@ -90,12 +96,19 @@ struct DroppedRows {
   bool out_bf16 = true;
   bool add_x = true;
 };
+// Overflow by priority (optional): each expert keeps its C pairs of largest gate (ties -> lower
+// pair index) and packs them in that order. prio_list [T k] and demand_offsets [E + 1] are scratch.
+struct PriorityDispatch {
+  const float* gates = nullptr;  // [T, k]; nullptr = first-come
+  int32_t* list = nullptr;
+  int32_t* demand_offsets = nullptr;
+};
 cudaError_t enqueue_dispatch(const void* x, bool bf16, int64_t T, int d, const int32_t* ids, int E,
                              int k, int64_t C, int32_t* slot, int32_t* counts, int32_t* offsets,
                              int32_t* row_token, void* x_packed, int64_t rows_max,
                              int32_t* local_rank, int32_t* seg_counts, int32_t* seg_base,
                              int* status, cudaStream_t stream, DroppedRows dropped = DroppedRows{},
-                             int counted_seg_len = 0);
+                             int counted_seg_len = 0, PriorityDispatch prio = PriorityDispatch{});
 // counted_seg_len > 0: local_rank and seg_counts were already written (segments of that many
 // pairs) by the router's top-k kernel; the counting kernel is skipped.
 

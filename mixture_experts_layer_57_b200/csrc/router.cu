@@ -15,11 +15,14 @@
 //                         x*hi + x*mid + x*lo from exact products, fp32 accumulation) for bf16 x,
 //                         or router_logits_kernel below (fp32 FMA) for fp32 x
 //   router_topk_kernel    one warp per token: max, sum of exp, p = exp(l - max) / sum,
-//                         k rounds of warp argmax on the logits (ties -> lower index), gates;
-//                         per-block sums of p (fixed order) and first-choice counts are added to
-//                         global accumulators as integers (p sums in 2^-32 fixed point), so the
-//                         totals do not depend on the order of the blocks; the last block to
-//                         finish turns them into f, Q and aux
+//                         k rounds of warp argmax on the logits (ties -> lower index), gates
+//                         (optionally renormalised over the k choices: survey notes §1.1.1.1);
+//                         per-block sums of p (fixed order), first-choice counts, gate sums
+//                         (Importance), choice counts (Load) and (log Z)^2 (comparison article,
+//                         "Router Z-loss") are added to global accumulators as integers (fixed
+//                         point), so the totals do not depend on the order of the blocks; the last
+//                         block to finish turns them into f, Q, aux, z-loss and the CoV^2 of
+//                         Importance and Load (survey notes §1.1.4.1)
 #include "common.cuh"
 #include "kernels.h"
 
@@ -98,8 +101,13 @@ __global__ void __launch_bounds__(256) router_gemv_kernel(const void* __restrict
     for (int i = threadIdx.x; i < E; i += blockDim.x) {
       acc.q[i] = 0ull;
       acc.c[i] = 0u;
+      acc.imp[i] = 0ull;
+      acc.load[i] = 0u;
     }
-    if (threadIdx.x == 0) *acc.ticket = 0u;
+    if (threadIdx.x == 0) {
+      *acc.z = 0ull;
+      *acc.ticket = 0u;
+    }
   }
   const float* wr = w + (int64_t)e * d;
   for (int64_t t = warp; t < T; t += 8) {
@@ -153,8 +161,13 @@ __global__ void __launch_bounds__(256) router_prep_kernel(const float* __restric
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
       acc.q[e] = 0ull;
       acc.c[e] = 0u;
+      acc.imp[e] = 0ull;
+      acc.load[e] = 0u;
     }
-    if (threadIdx.x == 0) *acc.ticket = 0u;
+    if (threadIdx.x == 0) {
+      *acc.z = 0ull;
+      *acc.ticket = 0u;
+    }
   }
   if (out == nullptr) {
     pdl_trigger();
@@ -179,6 +192,8 @@ __global__ void __launch_bounds__(256) router_prep_kernel(const float* __restric
 }
 
 constexpr double kQScale = 4294967296.0;  // 2^32: fixed-point scale of the p sums
+constexpr double kZScale = 16777216.0;    // 2^24: fixed-point scale of the (log Z)^2 sums
+constexpr double kIScale = 16777216.0;    // 2^24: fixed-point scale of the gate sums
 
 // EPL = experts per lane (E <= 32 * EPL); expert e lives in lane e % 32, slot e / 32.
 // COUNT: also rank this block's (token, choice) pairs per expert in pair order for dispatch.
@@ -189,16 +204,24 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
                                                           float* __restrict__ gates,
                                                           RouterAccum acc, float alpha,
                                                           float* __restrict__ lb,
-                                                          RouterDispatchCount dc) {
+                                                          RouterDispatchCount dc, int renorm,
+                                                          float* __restrict__ losses) {
   __shared__ float qs[8][MOE_MAX_EXPERTS];
-  __shared__ int cs[MOE_MAX_EXPERTS];
+  // per expert: first-choice count << 16 | choice count (each at most kRouterTokensPerBlock)
+  __shared__ unsigned cs[MOE_MAX_EXPERTS];
+  __shared__ unsigned imp_s[MOE_MAX_EXPERTS];  // gate sums, 2^-24 fixed point (< 2^31 per block)
+  __shared__ float zs[8];
   __shared__ float prod[MOE_MAX_EXPERTS];
   __shared__ int is_last;
   __shared__ int blk_ids[COUNT ? kRouterTokensPerBlock * MOE_MAX_TOPK : 1];
   pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int e = threadIdx.x; e < E; e += 256) cs[e] = 0;
+  for (int e = threadIdx.x; e < E; e += 256) {
+    cs[e] = 0u;
+    imp_s[e] = 0u;
+  }
   __syncthreads();
+  float zw = 0.0f;  // this warp's sum of (log Z)^2 over its tokens, in token order
   float q[EPL];
 #pragma unroll
   for (int i = 0; i < EPL; ++i) q[i] = 0.0f;
@@ -225,6 +248,10 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (losses != nullptr) {
+      const float lz = m + logf(s);  // log sum_e exp(l_e)
+      zw += lz * lz;
+    }
     float p[EPL];
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
@@ -239,6 +266,9 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
       if (b) bi = 32 * i + __ffs(b) - 1;
     }
     uint32_t taken = 0;
+    float gv[MOE_MAX_TOPK];
+    int gi[MOE_MAX_TOPK];
+    float gsum = 0.0f;
     for (int j = 0; j < k; ++j) {
       if (j > 0) {
         // later choices: (value desc, index asc) warp argmax over the experts not yet taken
@@ -269,14 +299,33 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
         if (i == slot_i) pv = p[i];
       pv = __shfl_sync(0xffffffffu, pv, owner);
       if (lane == owner) taken |= 1u << slot_i;
-      if (lane == 0) {
-        ids[t * k + j] = bi;
-        gates[t * k + j] = pv;
-        if (j == 0) atomicAdd(&cs[bi], 1);  // integer counts: order-independent
-        if constexpr (COUNT) blk_ids[r * k + j] = bi;
+#pragma unroll
+      for (int jj = 0; jj < MOE_MAX_TOPK; ++jj)
+        if (jj == j) {
+          gv[jj] = pv;
+          gi[jj] = bi;
+        }
+      gsum += pv;
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int j = 0; j < MOE_MAX_TOPK; ++j) {
+        if (j >= k) break;
+        const float g = renorm ? gv[j] / gsum : gv[j];
+        ids[t * k + j] = gi[j];
+        gates[t * k + j] = g;
+        // integers: order-independent
+        if (losses != nullptr) {
+          atomicAdd(&cs[gi[j]], j == 0 ? 0x10001u : 1u);
+          atomicAdd(&imp_s[gi[j]], __float2uint_rn(g * (float)kIScale));
+        } else if (j == 0) {
+          atomicAdd(&cs[gi[j]], 0x10000u);
+        }
+        if constexpr (COUNT) blk_ids[r * k + j] = gi[j];
       }
     }
   }
+  if (lane == 0) zs[warp] = zw;
   if constexpr (COUNT) {
     // rank the block's pairs per expert in pair order (warp 0), write ranks and segment counts
     __syncthreads();
@@ -316,10 +365,18 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
     for (int w = 0; w < 8; ++w) sum += qs[w][e];
     const unsigned long long fx = (unsigned long long)llrint((double)sum * kQScale);
     if (fx) atomicAdd(&acc.q[e], fx);
-    if (cs[e]) atomicAdd(&acc.c[e], (unsigned)cs[e]);
+    if (cs[e] >> 16) atomicAdd(&acc.c[e], cs[e] >> 16);
+    if (cs[e] & 0xffffu) atomicAdd(&acc.load[e], cs[e] & 0xffffu);
+    if (imp_s[e]) atomicAdd(&acc.imp[e], (unsigned long long)imp_s[e]);
+  }
+  if (losses != nullptr && threadIdx.x == 0) {
+    float zb = 0.0f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) zb += zs[w];
+    atomicAdd(acc.z, (unsigned long long)llrint((double)zb * kZScale));
   }
   pdl_trigger();
-  if (lb == nullptr) return;
+  if (lb == nullptr && losses == nullptr) return;
   // the last block to finish turns the totals into f, Q, aux
   __threadfence();
   __syncthreads();
@@ -327,33 +384,59 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
   __syncthreads();
   if (!is_last) return;
   __threadfence();
-  for (int e = threadIdx.x; e < E; e += 256) {
-    const unsigned long long qf = atomicAdd(&acc.q[e], 0ull);
-    const unsigned cf = atomicAdd(&acc.c[e], 0u);
-    const float Q = (float)((double)qf / kQScale / (double)T);
-    const float f = (float)cf / (float)T;
-    lb[e] = f;
-    lb[E + e] = Q;
-    prod[e] = f * Q;
+  if (lb != nullptr) {
+    for (int e = threadIdx.x; e < E; e += 256) {
+      const unsigned long long qf = atomicAdd(&acc.q[e], 0ull);
+      const unsigned cf = atomicAdd(&acc.c[e], 0u);
+      const float Q = (float)((double)qf / kQScale / (double)T);
+      const float f = (float)cf / (float)T;
+      lb[e] = f;
+      lb[E + e] = Q;
+      prod[e] = f * Q;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float s = 0.0f;
+      for (int e = 0; e < E; ++e) s += prod[e];
+      lb[2 * E] = alpha * (float)E * s;
+    }
   }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float s = 0.0f;
-    for (int e = 0; e < E; ++e) s += prod[e];
-    lb[2 * E] = alpha * (float)E * s;
+  if (losses != nullptr && threadIdx.x == 0) {
+    // z-loss = mean over tokens of (log Z)^2; CoV^2 = population variance / mean^2 over experts
+    losses[0] = (float)((double)atomicAdd(acc.z, 0ull) / kZScale / (double)T);
+    double mi = 0.0, ml = 0.0;
+    for (int e = 0; e < E; ++e) {
+      mi += (double)atomicAdd(&acc.imp[e], 0ull) / kIScale;
+      ml += (double)atomicAdd(&acc.load[e], 0u);
+    }
+    mi /= E;
+    ml /= E;
+    double vi = 0.0, vl = 0.0;
+    for (int e = 0; e < E; ++e) {
+      const double a = (double)atomicAdd(&acc.imp[e], 0ull) / kIScale - mi;
+      const double b = (double)atomicAdd(&acc.load[e], 0u) - ml;
+      vi += a * a;
+      vl += b * b;
+    }
+    vi /= E;
+    vl /= E;
+    losses[1] = mi > 0.0 ? (float)(vi / (mi * mi)) : 0.0f;
+    losses[2] = ml > 0.0 ? (float)(vl / (ml * ml)) : 0.0f;
   }
 }
 
 template <int EPL>
 cudaError_t launch_topk(const float* logits, int64_t T, int E, int k, int32_t* ids, float* gates,
                         const RouterAccum& acc, float alpha, float* lb, RouterDispatchCount dc,
-                        cudaStream_t stream) {
+                        int renorm, float* losses, cudaStream_t stream) {
   const dim3 grid((unsigned)router_num_blocks(T));
   if (dc.local_rank != nullptr)
     return launch_kernel(router_topk_kernel<EPL, true>, grid, dim3(256), 0, stream,
-                         (const float*)logits, T, E, k, ids, gates, acc, alpha, lb, dc);
+                         (const float*)logits, T, E, k, ids, gates, acc, alpha, lb, dc, renorm,
+                         losses);
   return launch_kernel(router_topk_kernel<EPL, false>, grid, dim3(256), 0, stream,
-                       (const float*)logits, T, E, k, ids, gates, acc, alpha, lb, dc);
+                       (const float*)logits, T, E, k, ids, gates, acc, alpha, lb, dc, renorm,
+                       losses);
 }
 
 }  // namespace
@@ -362,7 +445,7 @@ cudaError_t enqueue_router(const void* x, bool x_bf16, int64_t T, int d, const f
                            const float* router_bias, int E, int k, float* logits, int32_t* ids,
                            float* gates, float* lb_stats, float aux_alpha,
                            const RouterScratch& scr, int* status, cudaStream_t stream,
-                           RouterDispatchCount dc) {
+                           RouterDispatchCount dc, bool renormalize, float* losses) {
   if (T == 0) return cudaSuccess;
   if (!logits) logits = scr.logits_scratch;
   const bool gemv = T <= kRouterGemvMaxT;
@@ -390,12 +473,24 @@ cudaError_t enqueue_router(const void* x, bool x_bf16, int64_t T, int d, const f
     if (err != cudaSuccess) return err;
   }
   const RouterAccum& a = scr.acc;
-  if (E <= 32) return launch_topk<1>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, stream);
-  if (E <= 64) return launch_topk<2>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, stream);
-  if (E <= 128) return launch_topk<4>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, stream);
-  if (E <= 256) return launch_topk<8>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, stream);
-  if (E <= 512) return launch_topk<16>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, stream);
-  return launch_topk<32>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, stream);
+  const int rn = renormalize ? 1 : 0;
+  if (E <= 32)
+    return launch_topk<1>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, rn, losses,
+                          stream);
+  if (E <= 64)
+    return launch_topk<2>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, rn, losses,
+                          stream);
+  if (E <= 128)
+    return launch_topk<4>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, rn, losses,
+                          stream);
+  if (E <= 256)
+    return launch_topk<8>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, rn, losses,
+                          stream);
+  if (E <= 512)
+    return launch_topk<16>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, rn, losses,
+                          stream);
+  return launch_topk<32>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, rn, losses,
+                         stream);
 }
 
 }  // namespace moe

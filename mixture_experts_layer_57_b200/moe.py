@@ -20,6 +20,7 @@ HEADER = os.path.join(os.path.dirname(_PKG), "include", "moe.h")
 
 MOE_F32, MOE_BF16 = 0, 1
 MOE_EPILOGUE_BIAS_GELU, MOE_EPILOGUE_BIAS = 0, 1
+MOE_OVERFLOW_FIRST_COME, MOE_OVERFLOW_PRIORITY = 0, 1
 STATUS_BLOCK_BYTES = 256
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARGUMENT", 2: "MOE_ERR_UNSUPPORTED",
                 3: "MOE_ERR_WORKSPACE_TOO_SMALL", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_FLAG",
@@ -43,14 +44,15 @@ class LayerArgs(ctypes.Structure):
                 ("w2", ctypes.c_void_p), ("b2", ctypes.c_void_p), ("dense_w1", ctypes.c_void_p),
                 ("dense_b1", ctypes.c_void_p), ("dense_w2", ctypes.c_void_p),
                 ("dense_b2", ctypes.c_void_p), ("add_input_residual", ctypes.c_int),
-                ("aux_alpha", ctypes.c_float)]
+                ("aux_alpha", ctypes.c_float), ("overflow_policy", ctypes.c_int),
+                ("renormalize_gates", ctypes.c_int)]
 
 
 class LayerAux(ctypes.Structure):
     _fields_ = [("logits", ctypes.c_void_p), ("expert_ids", ctypes.c_void_p),
                 ("gates", ctypes.c_void_p), ("slot", ctypes.c_void_p),
                 ("expert_counts", ctypes.c_void_p), ("expert_offsets", ctypes.c_void_p),
-                ("lb_stats", ctypes.c_void_p)]
+                ("lb_stats", ctypes.c_void_p), ("router_losses", ctypes.c_void_p)]
 
 
 _lib = None
@@ -75,8 +77,12 @@ def lib() -> ctypes.CDLL:
             "moe_packed_rows_max": ([i64, i32, i32, i64, P(i64)], i32),
             "moe_router_workspace_bytes": ([i64, i32, i32, P(sz)], i32),
             "moe_router_topk": ([vp, i32, i64, i32, vp, vp, i32, i32, vp, vp, vp, vp, f32, vp, sz, vp], i32),
+            "moe_router_topk_ex": ([vp, i32, i64, i32, vp, vp, i32, i32, vp, vp, vp, vp, f32, i32, vp,
+                                    vp, sz, vp], i32),
             "moe_dispatch_workspace_bytes": ([i64, i32, i32, P(sz)], i32),
             "moe_dispatch": ([vp, i32, i64, i32, vp, i32, i32, i64, vp, vp, vp, vp, vp, i64, vp, sz, vp], i32),
+            "moe_dispatch_priority": ([vp, i32, i64, i32, vp, vp, i32, i32, i64, vp, vp, vp, vp, vp, i64,
+                                       vp, sz, vp], i32),
             "moe_dispatch_noalloc": ([vp, i32, i64, i32, vp, i32, i32, i64, vp, vp, vp, vp, vp, i64, vp], i32),
             "moe_expert_ffn_workspace_bytes": ([P(sz)], i32),
             "moe_expert_ffn": ([vp, vp, i32, i64, i32, i32, i32, vp, vp, vp, vp, vp, vp, i64, vp, sz, vp], i32),
@@ -182,7 +188,10 @@ def moe_combine_workspace_bytes():
 def moe_router_topk(x: torch.Tensor, w_router: torch.Tensor, k: int,
                     router_bias: Optional[torch.Tensor] = None, logits=None, expert_ids=None,
                     gates=None, lb_stats=None, aux_alpha: float = 0.01, want_stats: bool = True,
-                    ws: Optional[torch.Tensor] = None, stream=None) -> dict:
+                    ws: Optional[torch.Tensor] = None, stream=None, renormalize: bool = False,
+                    router_losses=None) -> dict:
+    """moe_router_topk, or moe_router_topk_ex when ``renormalize`` is set or ``router_losses``
+    (a [3] fp32 tensor, or True to allocate one) is given."""
     T, d = x.shape
     E = w_router.shape[0]
     dev = x.device
@@ -196,15 +205,26 @@ def moe_router_topk(x: torch.Tensor, w_router: torch.Tensor, k: int,
         lb_stats = torch.empty(2 * E + 1, dtype=torch.float32, device=dev)
     if ws is None:
         ws = workspace(moe_router_workspace_bytes(T, E, d), dev)
-    _check("moe_router_topk", lib().moe_router_topk(
-        _ptr(x), _dt(x), T, d, _ptr(w_router), _ptr(router_bias), E, k, _ptr(logits),
-        _ptr(expert_ids), _ptr(gates), _ptr(lb_stats), aux_alpha, _ptr(ws), ws.numel(), _stream(stream)))
-    return dict(logits=logits, expert_ids=expert_ids, gates=gates, lb_stats=lb_stats, ws=ws)
+    if router_losses is True:
+        router_losses = torch.empty(3, dtype=torch.float32, device=dev)
+    if renormalize or router_losses is not None:
+        _check("moe_router_topk_ex", lib().moe_router_topk_ex(
+            _ptr(x), _dt(x), T, d, _ptr(w_router), _ptr(router_bias), E, k, _ptr(logits),
+            _ptr(expert_ids), _ptr(gates), _ptr(lb_stats), aux_alpha, int(bool(renormalize)),
+            _ptr(router_losses), _ptr(ws), ws.numel(), _stream(stream)))
+    else:
+        _check("moe_router_topk", lib().moe_router_topk(
+            _ptr(x), _dt(x), T, d, _ptr(w_router), _ptr(router_bias), E, k, _ptr(logits),
+            _ptr(expert_ids), _ptr(gates), _ptr(lb_stats), aux_alpha, _ptr(ws), ws.numel(),
+            _stream(stream)))
+    return dict(logits=logits, expert_ids=expert_ids, gates=gates, lb_stats=lb_stats, ws=ws,
+                router_losses=router_losses)
 
 
 def moe_dispatch(x: torch.Tensor, expert_ids: torch.Tensor, E: int, C: int, rows_max=None,
                  slot=None, expert_counts=None, expert_offsets=None, row_token=None, x_packed=None,
-                 ws=None, stream=None) -> dict:
+                 ws=None, stream=None, priority_gates: Optional[torch.Tensor] = None) -> dict:
+    """moe_dispatch, or moe_dispatch_priority when ``priority_gates`` ([T, k] fp32) is given."""
     T, d = x.shape
     k = expert_ids.shape[1]
     dev = x.device
@@ -222,10 +242,16 @@ def moe_dispatch(x: torch.Tensor, expert_ids: torch.Tensor, E: int, C: int, rows
         x_packed = torch.empty(max(rows_max, 1), d, dtype=x.dtype, device=dev)
     if ws is None:
         ws = workspace(moe_dispatch_workspace_bytes(T, E, k), dev)
-    _check("moe_dispatch", lib().moe_dispatch(
-        _ptr(x), _dt(x), T, d, _ptr(expert_ids), E, k, C, _ptr(slot), _ptr(expert_counts),
-        _ptr(expert_offsets), _ptr(row_token), _ptr(x_packed), rows_max, _ptr(ws), ws.numel(),
-        _stream(stream)))
+    if priority_gates is not None:
+        _check("moe_dispatch_priority", lib().moe_dispatch_priority(
+            _ptr(x), _dt(x), T, d, _ptr(expert_ids), _ptr(priority_gates), E, k, C, _ptr(slot),
+            _ptr(expert_counts), _ptr(expert_offsets), _ptr(row_token), _ptr(x_packed), rows_max,
+            _ptr(ws), ws.numel(), _stream(stream)))
+    else:
+        _check("moe_dispatch", lib().moe_dispatch(
+            _ptr(x), _dt(x), T, d, _ptr(expert_ids), E, k, C, _ptr(slot), _ptr(expert_counts),
+            _ptr(expert_offsets), _ptr(row_token), _ptr(x_packed), rows_max, _ptr(ws), ws.numel(),
+            _stream(stream)))
     return dict(slot=slot, expert_counts=expert_counts, expert_offsets=expert_offsets,
                 row_token=row_token, x_packed=x_packed, rows_max=rows_max, ws=ws)
 
@@ -324,7 +350,8 @@ def moe_combine(y_packed: torch.Tensor, expert_offsets, expert_ids, slot, gates,
 
 def layer_args(x, w_router, w1, b1, w2, b2, k: int, capacity_factor: float, router_bias=None,
                dense=None, add_input_residual: bool = True, aux_alpha: float = 0.01,
-               out_dtype=None) -> LayerArgs:
+               out_dtype=None, overflow_priority: bool = False,
+               renormalize_gates: bool = False) -> LayerArgs:
     """Fill a ``moe_layer_args`` struct from tensors (dense = (w1, b1, w2, b2) or None)."""
     T, d = x.shape
     E, d_ff, _ = w1.shape
@@ -336,7 +363,10 @@ def layer_args(x, w_router, w1, b1, w2, b2, k: int, capacity_factor: float, rout
                      w1=_ptr(w1), b1=_ptr(b1), w2=_ptr(w2), b2=_ptr(b2),
                      dense_w1=_ptr(dw[0]), dense_b1=_ptr(dw[1]), dense_w2=_ptr(dw[2]),
                      dense_b2=_ptr(dw[3]), add_input_residual=int(bool(add_input_residual)),
-                     aux_alpha=aux_alpha)
+                     aux_alpha=aux_alpha,
+                     overflow_policy=MOE_OVERFLOW_PRIORITY if overflow_priority else
+                     MOE_OVERFLOW_FIRST_COME,
+                     renormalize_gates=int(bool(renormalize_gates)))
 
 
 def moe_layer_workspace_bytes(args: LayerArgs) -> int:

@@ -47,7 +47,8 @@ def dev_inputs(inp: dict, device="cuda") -> dict:
 
 
 def run_layer(w: synth.Workload, d_inp: dict, out_dtype=None, add_input_residual=None,
-              ws: torch.Tensor = None) -> dict:
+              ws: torch.Tensor = None, overflow_priority: bool = False, renormalize: bool = False,
+              want_losses: bool = False) -> dict:
     """One moe_layer_forward on device inputs; returns host copies of every output."""
     T, E, k = w.T, w.E, w.k
     x = d_inp["x"]
@@ -58,7 +59,8 @@ def run_layer(w: synth.Workload, d_inp: dict, out_dtype=None, add_input_residual
     args = moe.layer_args(x, d_inp["w_router"], d_inp["w1"], d_inp["b1"], d_inp["w2"], d_inp["b2"],
                           k=k, capacity_factor=w.capacity_factor, router_bias=d_inp.get("router_bias"),
                           dense=dense, add_input_residual=res, aux_alpha=w.aux_alpha,
-                          out_dtype=out_dtype)
+                          out_dtype=out_dtype, overflow_priority=overflow_priority,
+                          renormalize_gates=renormalize)
     dev = x.device
     aux = dict(logits=torch.empty(T, E, dtype=torch.float32, device=dev),
                expert_ids=torch.empty(T, k, dtype=torch.int32, device=dev),
@@ -67,6 +69,8 @@ def run_layer(w: synth.Workload, d_inp: dict, out_dtype=None, add_input_residual
                expert_counts=torch.empty(E, dtype=torch.int32, device=dev),
                expert_offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
                lb_stats=torch.empty(2 * E + 1, dtype=torch.float32, device=dev))
+    if want_losses:
+        aux["router_losses"] = torch.empty(3, dtype=torch.float32, device=dev)
     odt = x.dtype if out_dtype is None else out_dtype
     out = torch.empty(T, w.d_model, dtype=odt, device=dev)
     if ws is None:

@@ -28,7 +28,7 @@ def test_exports_every_declared_symbol(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.moe_abi_version() == 1
+    assert L.moe_abi_version() == 2
     for code, name in moe.STATUS_NAMES.items():
         assert L.moe_status_string(code).decode() == name
 
@@ -89,6 +89,37 @@ def test_router_validation(L):
     assert _router(L, wsb=100) == 3             # workspace too small
 
 
+def test_router_ex_validation(L, monkeypatch):
+    def call(**kw):
+        a = dict(x=FAKE, xdt=1, T=16, d=64, w=FAKE, b=None, E=8, k=2, logits=None, ids=FAKE,
+                 gates=FAKE, lb=None, alpha=0.01, rn=1, losses=FAKE, ws=FAKE, wsb=1 << 30)
+        a.update(kw)
+        return L.moe_router_topk_ex(a["x"], a["xdt"], a["T"], a["d"], a["w"], a["b"], a["E"],
+                                    a["k"], a["logits"], a["ids"], a["gates"], a["lb"], a["alpha"],
+                                    a["rn"], a["losses"], a["ws"], a["wsb"], None)
+    assert call(k=3, E=2) == 1
+    assert call(losses=FAKE + 4) == 6           # misaligned router_losses
+    assert call(wsb=100) == 3
+    monkeypatch.setenv("MOE_FAULT_INJECT", "moe_router_topk_ex")
+    assert call() == 4
+    assert _router(L, wsb=100) == 3             # the plain entry is a different name
+
+
+def test_dispatch_priority_validation(L):
+    def call(**kw):
+        a = dict(x=FAKE, dt=1, T=16, d=64, ids=FAKE, g=FAKE, E=4, k=1, C=4, slot=FAKE, cnt=FAKE,
+                 off=FAKE, rt=FAKE, xp=FAKE, rows=16, ws=FAKE, wsb=1 << 30)
+        a.update(kw)
+        return L.moe_dispatch_priority(a["x"], a["dt"], a["T"], a["d"], a["ids"], a["g"], a["E"],
+                                       a["k"], a["C"], a["slot"], a["cnt"], a["off"], a["rt"],
+                                       a["xp"], a["rows"], a["ws"], a["wsb"], None)
+    assert call(g=None) == 1                    # gates are required
+    assert call(g=FAKE + 4) == 6
+    assert call(C=-1) == 1
+    assert call(rows=15) == 1
+    assert call(wsb=10) == 3
+
+
 def test_dispatch_validation(L):
     def call(**kw):
         a = dict(x=FAKE, dt=1, T=16, d=64, ids=FAKE, E=4, k=1, C=4, slot=FAKE, cnt=FAKE, off=FAKE,
@@ -147,6 +178,13 @@ def test_layer_validation_and_workspace(L):
     args.k = 1
     args.d_ff = 4100
     assert L.moe_layer_forward(ctypes.byref(args), FAKE, ctypes.byref(aux), FAKE, nbytes, None) == 2
+    args.d_ff = 4096
+    args.overflow_policy = 2                    # neither first-come nor priority
+    assert L.moe_layer_forward(ctypes.byref(args), FAKE, ctypes.byref(aux), FAKE, nbytes, None) == 1
+    args.overflow_policy = moe.MOE_OVERFLOW_PRIORITY
+    assert moe.moe_layer_workspace_bytes(args) == nbytes
+    aux.router_losses = FAKE + 4
+    assert L.moe_layer_forward(ctypes.byref(args), FAKE, ctypes.byref(aux), FAKE, nbytes, None) == 6
 
 
 def test_fault_injection_is_host_side(L, monkeypatch):
