@@ -264,7 +264,8 @@ typedef struct {
 } moe_layer_aux;
 
 /* out = [x if add_input_residual] + [DenseMLP(x) if dense_*] + sum_j gate_j * Expert_{e_j}(x)
- * over the kept choices. Enqueues: router, dispatch, [dense MLP], expert FFN, combine. */
+ * over the kept choices. Enqueues: router, dispatch, [dense MLP], expert FFN, combine.
+ * T == 0 launches no kernel; it only zeroes aux expert_counts / expert_offsets when given. */
 moe_status moe_layer_workspace_bytes(const moe_layer_args* args, size_t* bytes);
 moe_status moe_layer_forward(const moe_layer_args* args, void* out, moe_layer_aux* aux, void* ws,
                              size_t ws_bytes, moe_stream_t stream);
@@ -279,6 +280,40 @@ moe_status moe_layer_forward_profiled(const moe_layer_args* args, void* out, moe
                                       void* ws, size_t ws_bytes, moe_stream_t stream,
                                       void* const* events, int max_events, int* n_events,
                                       char* names, size_t names_len);
+
+/* ---------------------------------------------------------------- token shards
+ * The layer split over G GPUs by tokens, every weight replicated (data parallelism as the
+ * DeepSpeed-MoE notes §4.2 use it: parameters copied, tokens divided). Shard r holds tokens [T_0 + ... + T_{r-1}, ... + T_r) of the batch of
+ * T_global tokens, args->T = T_r. The capacity is the whole batch's, C = ceil(k T_global cf / E),
+ * and the overflow rule is the single-GPU one: pairs in global token order, first come first
+ * kept. One exchange step sits between the two halves:
+ *   1. moe_layer_forward_shard_begin: router and top-k of the shard's tokens; writes the shard's
+ *      demand per expert (demand [E] int32) and its integer router statistics
+ *      (stat_partials [moe_router_partials_count(E)] int64: fixed-point sums of p, first-choice
+ *      counts, gate sums, choice counts, (log Z)^2).
+ *   2. the caller gathers every shard's demand into demand_all [G, E] (shard order) and sums
+ *      the partials over shards into stat_totals (e.g. NCCL all-gather and all-reduce).
+ *   3. moe_layer_forward_shard_end: the shard's global slot base per expert (sum of the earlier
+ *      shards' demand), expert e keeps its first clamp(C - base_e, 0, demand_e) pairs; then
+ *      dispatch, expert FFN and combine of the shard's tokens into out [T_r, d_model], and
+ *      lb_stats / router_losses of the whole batch from stat_totals.
+ * Results equal the single-GPU layer over the whole batch: ids, gates, slots and outputs of each
+ * token bit for bit; lb_stats and router losses too when every shard but the last holds a
+ * multiple of 64 tokens (the router's statistics blocks), else within fixed-point rounding.
+ * Both calls take the same args, aux pointers and workspace (the workspace carries the shard's
+ * routing from begin to end and must not be used in between). overflow_policy must be
+ * MOE_OVERFLOW_FIRST_COME (MOE_ERR_UNSUPPORTED otherwise). begin's `out` is not used. */
+moe_status moe_layer_shard_workspace_bytes(const moe_layer_args* args, int64_t T_global,
+                                           size_t* bytes);
+int64_t moe_router_partials_count(int E); /* 4 E + 1 */
+moe_status moe_layer_forward_shard_begin(const moe_layer_args* args, int64_t T_global,
+                                         moe_layer_aux* aux, int32_t* demand,
+                                         int64_t* stat_partials, void* ws, size_t ws_bytes,
+                                         moe_stream_t stream);
+moe_status moe_layer_forward_shard_end(const moe_layer_args* args, int64_t T_global, int G,
+                                       int rank, const int32_t* demand_all,
+                                       const int64_t* stat_totals, void* out, moe_layer_aux* aux,
+                                       void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* ---------------------------------------------------------------- status block
  * moe_workspace_reset: zeroes the status block (asynchronous on stream).

@@ -403,17 +403,22 @@ struct LayerWs {
   float* y_packed;
   void* h_dense;
   float* r_dense;
+  int32_t* cap_local;
   int64_t C, rows_max;
 };
 
-moe_status layer_layout(const moe_layer_args* a, uint8_t* base, LayerWs* w, size_t* bytes) {
+// T_cap: the batch the capacity is computed from (T, or the whole batch of a token shard).
+moe_status layer_layout(const moe_layer_args* a, uint8_t* base, LayerWs* w, size_t* bytes,
+                        int64_t T_cap = -1) {
   if (!a) return MOE_ERR_INVALID_ARGUMENT;
+  if (T_cap < 0) T_cap = a->T;
+  if (T_cap < a->T) return MOE_ERR_INVALID_ARGUMENT;
   moe_status st = check_router_shape(a->T, a->d_model, a->E, a->k);
   if (st != MOE_OK) return st;
   if (!valid_dtype(a->dtype) || !valid_dtype(a->out_dtype)) return MOE_ERR_INVALID_ARGUMENT;
   if (a->overflow_policy != MOE_OVERFLOW_FIRST_COME && a->overflow_policy != MOE_OVERFLOW_PRIORITY)
     return MOE_ERR_INVALID_ARGUMENT;
-  st = moe_capacity(a->T, a->E, a->k, a->capacity_factor, &w->C);
+  st = moe_capacity(T_cap, a->E, a->k, a->capacity_factor, &w->C);
   if (st != MOE_OK) return st;
   moe_packed_rows_max(a->T, a->E, a->k, w->C, &w->rows_max);
   st = check_ffn_shape(a->E, w->rows_max, a->d_model, a->d_ff, a->dtype);
@@ -431,6 +436,7 @@ moe_status layer_layout(const moe_layer_args* a, uint8_t* base, LayerWs* w, size
   w->slot = c.take<int32_t>((size_t)T * k);
   w->counts = c.take<int32_t>((size_t)E);
   w->offsets = c.take<int32_t>((size_t)E + 1);
+  w->cap_local = c.take<int32_t>((size_t)E);
   w->row_token = c.take<int32_t>((size_t)R);
   w->x_packed = c.take<uint8_t>((size_t)R * d * es);
   w->h_packed = c.take<uint8_t>((size_t)R * f * es);
@@ -480,16 +486,32 @@ struct StageRecorder {
   }
 };
 
+// A token shard's half of the layer (moe_layer_forward_shard_begin / _end), or the whole layer.
+enum ShardMode { kWhole = 0, kShardBegin = 1, kShardEnd = 2 };
+struct ShardCall {
+  ShardMode mode = kWhole;
+  int64_t T_global = -1;
+  int32_t* demand_out = nullptr;    // begin
+  int64_t* partials_out = nullptr;  // begin
+  const int32_t* demand_all = nullptr;  // end
+  const int64_t* totals = nullptr;      // end
+  int G = 1, rank = 0;                  // end
+};
+
 moe_status layer_forward_impl(const moe_layer_args* a, void* out, moe_layer_aux* aux, void* ws,
-                              size_t ws_bytes, moe_stream_t stream, StageRecorder& rec) {
+                              size_t ws_bytes, moe_stream_t stream, StageRecorder& rec,
+                              const ShardCall& sh = ShardCall{}) {
   LayerWs w;
   size_t need = 0;
-  moe_status st = layer_layout(a, (uint8_t*)ws, &w, &need);
+  moe_status st = layer_layout(a, (uint8_t*)ws, &w, &need, sh.T_global);
   if (st != MOE_OK) return st;
+  if (sh.mode != kWhole && a->overflow_policy != MOE_OVERFLOW_FIRST_COME)
+    return MOE_ERR_UNSUPPORTED;  // a global priority order would need every shard's gates
   const bool dense = a->dense_w1 != nullptr;
   if (dense && !a->dense_w2) return MOE_ERR_INVALID_ARGUMENT;
   if (!ws) return MOE_ERR_INVALID_ARGUMENT;
-  if (a->T > 0 && (!a->x || !a->w_router || !a->w1 || !a->w2 || !out)) return MOE_ERR_INVALID_ARGUMENT;
+  if (a->T > 0 && (!a->x || !a->w_router || !a->w1 || !a->w2 || (!out && sh.mode != kShardBegin)))
+    return MOE_ERR_INVALID_ARGUMENT;
   if (!aligned16(a->x) || !aligned16(a->w_router) || !aligned16(a->router_bias) ||
       !aligned16(a->w1) || !aligned16(a->b1) || !aligned16(a->w2) || !aligned16(a->b2) ||
       !aligned16(a->dense_w1) || !aligned16(a->dense_b1) || !aligned16(a->dense_w2) ||
@@ -501,9 +523,33 @@ moe_status layer_forward_impl(const moe_layer_args* a, void* out, moe_layer_aux*
               !aligned16(aux->router_losses)))
     return MOE_ERR_MISALIGNED;
   if (ws_bytes < need) return MOE_ERR_WORKSPACE_TOO_SMALL;
-  if (fault_injected("moe_layer_forward")) return MOE_ERR_CUDA;
+  const char* entry = sh.mode == kShardBegin ? "moe_layer_forward_shard_begin"
+                      : sh.mode == kShardEnd ? "moe_layer_forward_shard_end"
+                                             : "moe_layer_forward";
+  if (fault_injected(entry)) return MOE_ERR_CUDA;
   g_launches = 0;
-  if (a->T == 0) return MOE_OK;
+  if (a->T == 0) {
+    if (sh.mode == kShardBegin) {  // an empty shard demands nothing and adds nothing
+      if (cudaMemsetAsync(sh.demand_out, 0, sizeof(int32_t) * a->E, stream) != cudaSuccess ||
+          cudaMemsetAsync(sh.partials_out, 0, sizeof(int64_t) * router_partials_count(a->E),
+                          stream) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    }
+    if (sh.mode == kShardEnd && aux &&
+        enqueue_router_finalize(sh.totals, sh.T_global, a->E, a->aux_alpha, aux->lb_stats,
+                                aux->router_losses, stream) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (sh.mode != kShardBegin && aux) {  // no demand and no packed rows
+      if (aux->expert_counts &&
+          cudaMemsetAsync(aux->expert_counts, 0, sizeof(int32_t) * a->E, stream) != cudaSuccess)
+        return MOE_ERR_CUDA;
+      if (aux->expert_offsets &&
+          cudaMemsetAsync(aux->expert_offsets, 0, sizeof(int32_t) * (a->E + 1), stream) !=
+              cudaSuccess)
+        return MOE_ERR_CUDA;
+    }
+    return MOE_OK;
+  }
 
   float* logits = aux ? aux->logits : nullptr;  // the router keeps its own scratch if needed
   int32_t* ids = aux && aux->expert_ids ? aux->expert_ids : w.ids;
@@ -520,15 +566,41 @@ moe_status layer_forward_impl(const moe_layer_args* a, void* out, moe_layer_aux*
 
   rec.stream = stream;
   rec.mark("start");
-  // the router's top-k kernel also ranks each 64-token segment's pairs for dispatch
-  RouterDispatchCount dcount;
-  dcount.local_rank = w.dispatch.local_rank;
-  dcount.seg_counts = w.dispatch.seg_counts;
-  cudaError_t e = enqueue_router(a->x, bf16, T, d, a->w_router, a->router_bias, E, k, logits, ids,
-                                 gates, lb, a->aux_alpha, w.router.scr, status, stream, dcount,
-                                 a->renormalize_gates != 0, losses);
-  if (e != cudaSuccess) return MOE_ERR_CUDA;
-  rec.mark("router");
+  cudaError_t e = cudaSuccess;
+  if (sh.mode != kShardEnd) {
+    // the router's top-k kernel also ranks each 64-token segment's pairs for dispatch; a shard
+    // exports its integer statistics instead of finalising them
+    RouterDispatchCount dcount;
+    dcount.local_rank = w.dispatch.local_rank;
+    dcount.seg_counts = w.dispatch.seg_counts;
+    const bool begin = sh.mode == kShardBegin;
+    e = enqueue_router(a->x, bf16, T, d, a->w_router, a->router_bias, E, k, logits, ids, gates,
+                       begin ? nullptr : lb, a->aux_alpha, w.router.scr, status, stream, dcount,
+                       a->renormalize_gates != 0, begin ? nullptr : losses,
+                       begin ? sh.partials_out : nullptr, sh.T_global);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    rec.mark("router");
+  }
+  if (sh.mode == kShardBegin) {
+    // the shard's demand per expert (what the other shards need for their global slot base)
+    e = enqueue_dispatch(a->x, bf16, T, d, ids, E, k, w.C, slot, sh.demand_out, offsets,
+                         w.row_token, w.x_packed, w.rows_max, w.dispatch.local_rank,
+                         w.dispatch.seg_counts, w.dispatch.seg_base, status, stream,
+                         DroppedRows{}, (int)kRouterTokensPerBlock * k, PriorityDispatch{},
+                         ShardBase{}, true);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    rec.mark("demand");
+    return MOE_OK;
+  }
+  ShardBase shard;
+  if (sh.mode == kShardEnd) {
+    e = enqueue_router_finalize(sh.totals, sh.T_global, E, a->aux_alpha, lb, losses, stream);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    shard.demand_all = sh.demand_all;
+    shard.G = sh.G;
+    shard.rank = sh.rank;
+    shard.cap_local = w.cap_local;
+  }
 
   // bf16 layers fuse the combine into a layer-2 epilogue: the PR-MoE dense MLP's (any k, experts
   // run first) or, without the dense branch, the top-1 experts' (dropped tokens are then written
@@ -552,7 +624,7 @@ moe_status layer_forward_impl(const moe_layer_args* a, void* out, moe_layer_aux*
   e = enqueue_dispatch(a->x, bf16, T, d, ids, E, k, w.C, slot, counts, offsets, w.row_token,
                        w.x_packed, w.rows_max, w.dispatch.local_rank, w.dispatch.seg_counts,
                        w.dispatch.seg_base, status, stream, dropped,
-                       (int)kRouterTokensPerBlock * k, prio);
+                       (int)kRouterTokensPerBlock * k, prio, shard);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   rec.mark("dispatch");
 
@@ -581,13 +653,15 @@ moe_status layer_forward_impl(const moe_layer_args* a, void* out, moe_layer_aux*
       if (e != cudaSuccess) return MOE_ERR_CUDA;
       rec.mark("expert_gemm2");
     }
+    // the tile width follows the whole batch, so a shard's rows get the whole batch's arithmetic
+    const int64_t dense_hint = sh.T_global > T ? sh.T_global : T;
     e = enqueue_grouped_gemm_bf16(a->x, nullptr, 1, T, d, f, a->dense_w1, a->dense_b1, true,
-                                  w.h_dense, T, status, stream);
+                                  w.h_dense, dense_hint, status, stream);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     rec.mark("dense_gemm1");
     fc.dense = true;
-    e = enqueue_gemm2_combine(w.h_dense, nullptr, 1, T, f, d, a->dense_w2, a->dense_b2, fc, T,
-                              status, stream);
+    e = enqueue_gemm2_combine(w.h_dense, nullptr, 1, T, f, d, a->dense_w2, a->dense_b2, fc,
+                              dense_hint, status, stream);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     rec.mark("dense_gemm2_combine");
     return MOE_OK;
@@ -669,6 +743,49 @@ moe_status moe_layer_forward_profiled(const moe_layer_args* a, void* out, moe_la
   const moe_status st = layer_forward_impl(a, out, aux, ws, ws_bytes, stream, rec);
   *n_events = rec.n;
   return st;
+}
+
+moe_status moe_layer_shard_workspace_bytes(const moe_layer_args* args, int64_t T_global,
+                                           size_t* bytes) {
+  if (!bytes || !args || T_global < args->T) return MOE_ERR_INVALID_ARGUMENT;
+  LayerWs w;
+  return layer_layout(args, nullptr, &w, bytes, T_global);
+}
+
+int64_t moe_router_partials_count(int E) { return E < 1 ? 0 : router_partials_count(E); }
+
+moe_status moe_layer_forward_shard_begin(const moe_layer_args* args, int64_t T_global,
+                                         moe_layer_aux* aux, int32_t* demand,
+                                         int64_t* stat_partials, void* ws, size_t ws_bytes,
+                                         moe_stream_t stream) {
+  if (!args || T_global < args->T || !demand || !stat_partials) return MOE_ERR_INVALID_ARGUMENT;
+  if (!aligned16(demand) || !aligned16(stat_partials)) return MOE_ERR_MISALIGNED;
+  ShardCall sh;
+  sh.mode = kShardBegin;
+  sh.T_global = T_global;
+  sh.demand_out = demand;
+  sh.partials_out = stat_partials;
+  StageRecorder rec;
+  return layer_forward_impl(args, nullptr, aux, ws, ws_bytes, stream, rec, sh);
+}
+
+moe_status moe_layer_forward_shard_end(const moe_layer_args* args, int64_t T_global, int G,
+                                       int rank, const int32_t* demand_all,
+                                       const int64_t* stat_totals, void* out, moe_layer_aux* aux,
+                                       void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (!args || T_global < args->T || G < 1 || rank < 0 || rank >= G || !demand_all ||
+      !stat_totals)
+    return MOE_ERR_INVALID_ARGUMENT;
+  if (!aligned16(demand_all) || !aligned16(stat_totals)) return MOE_ERR_MISALIGNED;
+  ShardCall sh;
+  sh.mode = kShardEnd;
+  sh.T_global = T_global;
+  sh.demand_all = demand_all;
+  sh.totals = stat_totals;
+  sh.G = G;
+  sh.rank = rank;
+  StageRecorder rec;
+  return layer_forward_impl(args, out, aux, ws, ws_bytes, stream, rec, sh);
 }
 
 // ---------------------------------------------------------------- status block

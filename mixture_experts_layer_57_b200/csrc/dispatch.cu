@@ -109,7 +109,8 @@ __device__ void block_exclusive_scan_experts(int v, int E, int* warp_sums, int32
 __global__ void __launch_bounds__(1024)
     dispatch_scan_kernel(const int32_t* __restrict__ seg_counts, int64_t nseg, int E, int64_t C,
                          int32_t* __restrict__ seg_base, int32_t* __restrict__ counts,
-                         int32_t* __restrict__ offsets, int32_t* __restrict__ demand_offsets) {
+                         int32_t* __restrict__ offsets, int32_t* __restrict__ demand_offsets,
+                         ShardBase shard) {
   __shared__ int run_sum[1024];
   __shared__ int kept[MOE_MAX_EXPERTS];
   __shared__ int demand[MOE_MAX_EXPERTS];
@@ -159,7 +160,17 @@ __global__ void __launch_bounds__(1024)
     }
     if (g == G - 1) {
       counts[e] = run;
-      kept[e] = (int)min((int64_t)run, C);
+      int64_t cap = C;
+      if (shard.demand_all != nullptr) {
+        // global first-come: the earlier shards' pairs of expert e come first
+        int64_t base = 0;
+        for (int r = 0; r < shard.rank; ++r) base += shard.demand_all[(int64_t)r * E + e];
+        cap = C - base;
+        if (cap < 0) cap = 0;
+        if (cap > run) cap = run;
+        shard.cap_local[e] = (int32_t)cap;
+      }
+      kept[e] = (int)min((int64_t)run, cap);
       demand[e] = run;
     }
   }
@@ -249,7 +260,7 @@ __global__ void __launch_bounds__(256)
                             const int32_t* __restrict__ offsets, int32_t* __restrict__ slot,
                             int32_t* __restrict__ row_token, uint8_t* __restrict__ x_packed,
                             int64_t rows_max, DroppedRows dropped, int d, int seg_len,
-                            int prio) {
+                            int prio, const int32_t* __restrict__ cap_local) {
   constexpr int P = kScatterPairsPerWarp;
   pdl_wait();
   const int lane = threadIdx.x & 31;
@@ -266,7 +277,7 @@ __global__ void __launch_bounds__(256)
         my_s = slot[p];  // the priority rank kernel's slot
       } else {
         const int pos = seg_base[(p / seg_len) * E + e] + r;
-        if (pos < C) my_s = pos;
+        if (pos < (cap_local != nullptr ? (int64_t)cap_local[e] : C)) my_s = pos;
       }
     }
     slot[p] = my_s;
@@ -333,7 +344,8 @@ cudaError_t enqueue_dispatch(const void* x, bool bf16, int64_t T, int d, const i
                              int32_t* row_token, void* x_packed, int64_t rows_max,
                              int32_t* local_rank, int32_t* seg_counts, int32_t* seg_base,
                              int* status, cudaStream_t stream, DroppedRows dropped,
-                             int counted_seg_len, PriorityDispatch prio) {
+                             int counted_seg_len, PriorityDispatch prio, ShardBase shard,
+                             bool scan_only) {
   const int64_t pairs = T * k;
   const int seg_len = counted_seg_len > 0 ? counted_seg_len : kDispatchSeg;
   const int64_t nseg = (pairs + seg_len - 1) / seg_len;
@@ -347,9 +359,10 @@ cudaError_t enqueue_dispatch(const void* x, bool bf16, int64_t T, int d, const i
   {
     cudaError_t e = launch_kernel(dispatch_scan_kernel, dim3(1), dim3(1024), 0, stream,
                                   (const int32_t*)seg_counts, nseg, E, C, seg_base, counts, offsets,
-                                  prio.gates != nullptr ? prio.demand_offsets : nullptr);
+                                  prio.gates != nullptr ? prio.demand_offsets : nullptr, shard);
     if (e != cudaSuccess) return e;
   }
+  if (scan_only) return cudaGetLastError();
   const int use_prio = prio.gates != nullptr && pairs > 0 ? 1 : 0;
   if (use_prio) {
     cudaError_t e = launch_kernel(dispatch_list_kernel, dim3((unsigned)((pairs + 255) / 256)),
@@ -373,7 +386,7 @@ cudaError_t enqueue_dispatch(const void* x, bool bf16, int64_t T, int d, const i
       return launch_kernel(kern, dim3(blocks), dim3(256), 0, stream, xs, row_bytes, pairs, k, E, C,
                            ids, (const int32_t*)local_rank, (const int32_t*)seg_base,
                            (const int32_t*)offsets, slot, row_token, xp, rows_max, dropped, d,
-                           seg_len, use_prio);
+                           seg_len, use_prio, (const int32_t*)shard.cap_local);
     };
     cudaError_t e = row_bytes % 16 == 0  ? launch(dispatch_scatter_kernel<16>)
                     : row_bytes % 8 == 0 ? launch(dispatch_scatter_kernel<8>)

@@ -70,15 +70,26 @@ struct RouterDispatchCount {
   int32_t* local_rank = nullptr;  // [T * k]
   int32_t* seg_counts = nullptr;  // [router_num_blocks(T), E]
 };
+// Integer statistics partials of one token shard: [q (E), c (E), imp (E), load (E), z (1)] as
+// int64 (the accumulators' fixed-point values); sums over shards give the whole batch's.
+inline int64_t router_partials_count(int E) { return 4 * (int64_t)E + 1; }
 // logits may be nullptr (not returned).
 // renormalize: gates of the k choices divided by their sum. losses (optional): [z-loss,
-// CoV^2 of Importance, CoV^2 of Load].
+// CoV^2 of Importance, CoV^2 of Load]. export_partials (optional): instead of finalising, the
+// last block writes the integer partials there (lb_stats and losses must then be nullptr).
 cudaError_t enqueue_router(const void* x, bool x_bf16, int64_t T, int d, const float* w_router,
                            const float* router_bias, int E, int k, float* logits, int32_t* ids,
                            float* gates, float* lb_stats, float aux_alpha,
                            const RouterScratch& scratch, int* status, cudaStream_t stream,
                            RouterDispatchCount dcount = RouterDispatchCount{},
-                           bool renormalize = false, float* losses = nullptr);
+                           bool renormalize = false, float* losses = nullptr,
+                           int64_t* export_partials = nullptr, int64_t T_kernel_choice = -1);
+// T_kernel_choice (>= T): the batch size that selects the logits kernel (a token shard takes the
+// whole batch's, so every token's logits come from the same arithmetic).
+// f, Q, aux (lb_stats, optional) and the router losses (optional) from summed partials of T
+// tokens, with the same arithmetic as the top-k kernel's own finalisation (one block).
+cudaError_t enqueue_router_finalize(const int64_t* totals, int64_t T, int E, float aux_alpha,
+                                    float* lb_stats, float* losses, cudaStream_t stream);
 // logits = x W_r^T + b_r on tcgen05 from the exact split W_r = hi + mid + lo (bf16 each).
 cudaError_t enqueue_router_logits_tc(const void* x, int64_t T, int d, const uint16_t* w_split,
                                      int dpad, const float* router_bias, int E, float* logits,
@@ -103,12 +114,23 @@ struct PriorityDispatch {
   int32_t* list = nullptr;
   int32_t* demand_offsets = nullptr;
 };
+// Token shards (optional): this shard is `rank` of G consecutive token blocks; demand_all [G, E]
+// holds every shard's demand. Expert e keeps the pairs whose global first-come position
+// (sum of the earlier shards' demand + local position) is below C: cap_local[e] (scratch [E])
+// = clamp(C - base_e, 0, demand_e) of them.
+struct ShardBase {
+  const int32_t* demand_all = nullptr;  // nullptr = one shard
+  int G = 1;
+  int rank = 0;
+  int32_t* cap_local = nullptr;
+};
 cudaError_t enqueue_dispatch(const void* x, bool bf16, int64_t T, int d, const int32_t* ids, int E,
                              int k, int64_t C, int32_t* slot, int32_t* counts, int32_t* offsets,
                              int32_t* row_token, void* x_packed, int64_t rows_max,
                              int32_t* local_rank, int32_t* seg_counts, int32_t* seg_base,
                              int* status, cudaStream_t stream, DroppedRows dropped = DroppedRows{},
-                             int counted_seg_len = 0, PriorityDispatch prio = PriorityDispatch{});
+                             int counted_seg_len = 0, PriorityDispatch prio = PriorityDispatch{},
+                             ShardBase shard = ShardBase{}, bool scan_only = false);
 // counted_seg_len > 0: local_rank and seg_counts were already written (segments of that many
 // pairs) by the router's top-k kernel; the counting kernel is skipped.
 

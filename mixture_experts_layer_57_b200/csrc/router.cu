@@ -195,6 +195,66 @@ constexpr double kQScale = 4294967296.0;  // 2^32: fixed-point scale of the p su
 constexpr double kZScale = 16777216.0;    // 2^24: fixed-point scale of the (log Z)^2 sums
 constexpr double kIScale = 16777216.0;    // 2^24: fixed-point scale of the gate sums
 
+// f, Q, aux and the router losses from the integer totals of T tokens; called by every thread
+// of one 256-thread block (prod: E floats of shared memory). Totals are read through accessors so
+// that the top-k kernel's last block and the shard finalisation run the same arithmetic.
+template <class Q, class Cn, class I, class L>
+__device__ void router_finalize_block(int E, int64_t T, float alpha, Q q_at, Cn c_at, I imp_at,
+                                      L load_at, unsigned long long zsum, float* lb, float* losses,
+                                      float* prod) {
+  if (lb != nullptr) {
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+      const float Qe = (float)((double)q_at(e) / kQScale / (double)T);
+      const float f = (float)c_at(e) / (float)T;
+      lb[e] = f;
+      lb[E + e] = Qe;
+      prod[e] = f * Qe;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float s = 0.0f;
+      for (int e = 0; e < E; ++e) s += prod[e];
+      lb[2 * E] = alpha * (float)E * s;
+    }
+  }
+  if (losses != nullptr && threadIdx.x == 0) {
+    // z-loss = mean over tokens of (log Z)^2; CoV^2 = population variance / mean^2 over experts
+    losses[0] = (float)((double)zsum / kZScale / (double)T);
+    double mi = 0.0, ml = 0.0;
+    for (int e = 0; e < E; ++e) {
+      mi += (double)imp_at(e) / kIScale;
+      ml += (double)load_at(e);
+    }
+    mi /= E;
+    ml /= E;
+    double vi = 0.0, vl = 0.0;
+    for (int e = 0; e < E; ++e) {
+      const double a = (double)imp_at(e) / kIScale - mi;
+      const double b = (double)load_at(e) - ml;
+      vi += a * a;
+      vl += b * b;
+    }
+    vi /= E;
+    vl /= E;
+    losses[1] = mi > 0.0 ? (float)(vi / (mi * mi)) : 0.0f;
+    losses[2] = ml > 0.0 ? (float)(vl / (ml * ml)) : 0.0f;
+  }
+}
+
+__global__ void __launch_bounds__(256)
+    router_finalize_kernel(const int64_t* __restrict__ tot, int64_t T, int E, float alpha,
+                           float* __restrict__ lb, float* __restrict__ losses) {
+  __shared__ float prod[MOE_MAX_EXPERTS];
+  pdl_wait();
+  router_finalize_block(
+      E, T, alpha, [&](int e) { return (unsigned long long)tot[e]; },
+      [&](int e) { return (unsigned long long)tot[E + e]; },
+      [&](int e) { return (unsigned long long)tot[2 * E + e]; },
+      [&](int e) { return (unsigned long long)tot[3 * E + e]; }, (unsigned long long)tot[4 * E],
+      lb, losses, prod);
+  pdl_trigger();
+}
+
 // EPL = experts per lane (E <= 32 * EPL); expert e lives in lane e % 32, slot e / 32.
 // COUNT: also rank this block's (token, choice) pairs per expert in pair order for dispatch.
 template <int EPL, bool COUNT>
@@ -205,7 +265,8 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
                                                           RouterAccum acc, float alpha,
                                                           float* __restrict__ lb,
                                                           RouterDispatchCount dc, int renorm,
-                                                          float* __restrict__ losses) {
+                                                          float* __restrict__ losses, int extra,
+                                                          int64_t* __restrict__ exported) {
   __shared__ float qs[8][MOE_MAX_EXPERTS];
   // per expert: first-choice count << 16 | choice count (each at most kRouterTokensPerBlock)
   __shared__ unsigned cs[MOE_MAX_EXPERTS];
@@ -248,7 +309,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (losses != nullptr) {
+    if (extra) {
       const float lz = m + logf(s);  // log sum_e exp(l_e)
       zw += lz * lz;
     }
@@ -265,6 +326,16 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
       const unsigned b = __ballot_sync(0xffffffffu, (lane + 32 * i) < E && l[i] == m);
       if (b) bi = 32 * i + __ffs(b) - 1;
     }
+    // per-block integer counts (order-independent): first choices, and with the extra
+    // statistics every choice and its gate
+    auto count_choice = [&](int e, int j, float g) {
+      if (extra) {
+        atomicAdd(&cs[e], j == 0 ? 0x10001u : 1u);
+        atomicAdd(&imp_s[e], __float2uint_rn(g * (float)kIScale));
+      } else if (j == 0) {
+        atomicAdd(&cs[e], 0x10000u);
+      }
+    };
     uint32_t taken = 0;
     float gv[MOE_MAX_TOPK];
     int gi[MOE_MAX_TOPK];
@@ -299,29 +370,31 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
         if (i == slot_i) pv = p[i];
       pv = __shfl_sync(0xffffffffu, pv, owner);
       if (lane == owner) taken |= 1u << slot_i;
-#pragma unroll
-      for (int jj = 0; jj < MOE_MAX_TOPK; ++jj)
-        if (jj == j) {
-          gv[jj] = pv;
-          gi[jj] = bi;
+      if (lane == 0) {
+        ids[t * k + j] = bi;
+        if (!renorm) {
+          gates[t * k + j] = pv;
+          count_choice(bi, j, pv);
         }
-      gsum += pv;
+        if constexpr (COUNT) blk_ids[r * k + j] = bi;
+      }
+      if (renorm) {
+#pragma unroll
+        for (int jj = 0; jj < MOE_MAX_TOPK; ++jj)
+          if (jj == j) {
+            gv[jj] = pv;
+            gi[jj] = bi;
+          }
+        gsum += pv;
+      }
     }
-    if (lane == 0) {
+    if (renorm && lane == 0) {
 #pragma unroll
       for (int j = 0; j < MOE_MAX_TOPK; ++j) {
         if (j >= k) break;
-        const float g = renorm ? gv[j] / gsum : gv[j];
-        ids[t * k + j] = gi[j];
+        const float g = gv[j] / gsum;
         gates[t * k + j] = g;
-        // integers: order-independent
-        if (losses != nullptr) {
-          atomicAdd(&cs[gi[j]], j == 0 ? 0x10001u : 1u);
-          atomicAdd(&imp_s[gi[j]], __float2uint_rn(g * (float)kIScale));
-        } else if (j == 0) {
-          atomicAdd(&cs[gi[j]], 0x10000u);
-        }
-        if constexpr (COUNT) blk_ids[r * k + j] = gi[j];
+        count_choice(gi[j], j, g);
       }
     }
   }
@@ -369,74 +442,52 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
     if (cs[e] & 0xffffu) atomicAdd(&acc.load[e], cs[e] & 0xffffu);
     if (imp_s[e]) atomicAdd(&acc.imp[e], (unsigned long long)imp_s[e]);
   }
-  if (losses != nullptr && threadIdx.x == 0) {
+  if (extra && threadIdx.x == 0) {
     float zb = 0.0f;
 #pragma unroll
     for (int w = 0; w < 8; ++w) zb += zs[w];
     atomicAdd(acc.z, (unsigned long long)llrint((double)zb * kZScale));
   }
   pdl_trigger();
-  if (lb == nullptr && losses == nullptr) return;
-  // the last block to finish turns the totals into f, Q, aux
+  if (lb == nullptr && losses == nullptr && exported == nullptr) return;
+  // the last block to finish turns the totals into f, Q, aux (and the losses), or exports them
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) is_last = atomicAdd(acc.ticket, 1u) == gridDim.x - 1;
   __syncthreads();
   if (!is_last) return;
   __threadfence();
-  if (lb != nullptr) {
+  if (exported != nullptr) {
     for (int e = threadIdx.x; e < E; e += 256) {
-      const unsigned long long qf = atomicAdd(&acc.q[e], 0ull);
-      const unsigned cf = atomicAdd(&acc.c[e], 0u);
-      const float Q = (float)((double)qf / kQScale / (double)T);
-      const float f = (float)cf / (float)T;
-      lb[e] = f;
-      lb[E + e] = Q;
-      prod[e] = f * Q;
+      exported[e] = (int64_t)atomicAdd(&acc.q[e], 0ull);
+      exported[E + e] = (int64_t)atomicAdd(&acc.c[e], 0u);
+      exported[2 * E + e] = (int64_t)atomicAdd(&acc.imp[e], 0ull);
+      exported[3 * E + e] = (int64_t)atomicAdd(&acc.load[e], 0u);
     }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      float s = 0.0f;
-      for (int e = 0; e < E; ++e) s += prod[e];
-      lb[2 * E] = alpha * (float)E * s;
-    }
+    if (threadIdx.x == 0) exported[4 * E] = (int64_t)atomicAdd(acc.z, 0ull);
+    return;
   }
-  if (losses != nullptr && threadIdx.x == 0) {
-    // z-loss = mean over tokens of (log Z)^2; CoV^2 = population variance / mean^2 over experts
-    losses[0] = (float)((double)atomicAdd(acc.z, 0ull) / kZScale / (double)T);
-    double mi = 0.0, ml = 0.0;
-    for (int e = 0; e < E; ++e) {
-      mi += (double)atomicAdd(&acc.imp[e], 0ull) / kIScale;
-      ml += (double)atomicAdd(&acc.load[e], 0u);
-    }
-    mi /= E;
-    ml /= E;
-    double vi = 0.0, vl = 0.0;
-    for (int e = 0; e < E; ++e) {
-      const double a = (double)atomicAdd(&acc.imp[e], 0ull) / kIScale - mi;
-      const double b = (double)atomicAdd(&acc.load[e], 0u) - ml;
-      vi += a * a;
-      vl += b * b;
-    }
-    vi /= E;
-    vl /= E;
-    losses[1] = mi > 0.0 ? (float)(vi / (mi * mi)) : 0.0f;
-    losses[2] = ml > 0.0 ? (float)(vl / (ml * ml)) : 0.0f;
-  }
+  router_finalize_block(
+      E, T, alpha, [&](int e) { return atomicAdd(&acc.q[e], 0ull); },
+      [&](int e) { return (unsigned long long)atomicAdd(&acc.c[e], 0u); },
+      [&](int e) { return atomicAdd(&acc.imp[e], 0ull); },
+      [&](int e) { return (unsigned long long)atomicAdd(&acc.load[e], 0u); },
+      atomicAdd(acc.z, 0ull), lb, losses, prod);
 }
 
 template <int EPL>
 cudaError_t launch_topk(const float* logits, int64_t T, int E, int k, int32_t* ids, float* gates,
                         const RouterAccum& acc, float alpha, float* lb, RouterDispatchCount dc,
-                        int renorm, float* losses, cudaStream_t stream) {
+                        int renorm, float* losses, int64_t* exported, cudaStream_t stream) {
   const dim3 grid((unsigned)router_num_blocks(T));
+  const int extra = (losses != nullptr || exported != nullptr) ? 1 : 0;
   if (dc.local_rank != nullptr)
     return launch_kernel(router_topk_kernel<EPL, true>, grid, dim3(256), 0, stream,
                          (const float*)logits, T, E, k, ids, gates, acc, alpha, lb, dc, renorm,
-                         losses);
+                         losses, extra, exported);
   return launch_kernel(router_topk_kernel<EPL, false>, grid, dim3(256), 0, stream,
                        (const float*)logits, T, E, k, ids, gates, acc, alpha, lb, dc, renorm,
-                       losses);
+                       losses, extra, exported);
 }
 
 }  // namespace
@@ -445,10 +496,11 @@ cudaError_t enqueue_router(const void* x, bool x_bf16, int64_t T, int d, const f
                            const float* router_bias, int E, int k, float* logits, int32_t* ids,
                            float* gates, float* lb_stats, float aux_alpha,
                            const RouterScratch& scr, int* status, cudaStream_t stream,
-                           RouterDispatchCount dc, bool renormalize, float* losses) {
+                           RouterDispatchCount dc, bool renormalize, float* losses,
+                           int64_t* exported, int64_t T_kernel_choice) {
   if (T == 0) return cudaSuccess;
   if (!logits) logits = scr.logits_scratch;
-  const bool gemv = T <= kRouterGemvMaxT;
+  const bool gemv = (T_kernel_choice > T ? T_kernel_choice : T) <= kRouterGemvMaxT;
   const bool tc = !gemv && router_uses_tensor_cores(x_bf16, d);
   const int dpad = router_split_dpad(d);
   const int64_t n = tc ? (int64_t)E * dpad : 0;
@@ -475,22 +527,29 @@ cudaError_t enqueue_router(const void* x, bool x_bf16, int64_t T, int d, const f
   const RouterAccum& a = scr.acc;
   const int rn = renormalize ? 1 : 0;
   if (E <= 32)
-    return launch_topk<1>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, rn, losses,
-                          stream);
+    return launch_topk<1>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, rn,
+                          losses, exported, stream);
   if (E <= 64)
-    return launch_topk<2>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, rn, losses,
-                          stream);
+    return launch_topk<2>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, rn,
+                          losses, exported, stream);
   if (E <= 128)
-    return launch_topk<4>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, rn, losses,
-                          stream);
+    return launch_topk<4>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, rn,
+                          losses, exported, stream);
   if (E <= 256)
-    return launch_topk<8>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, rn, losses,
-                          stream);
+    return launch_topk<8>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, rn,
+                          losses, exported, stream);
   if (E <= 512)
-    return launch_topk<16>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, rn, losses,
-                          stream);
-  return launch_topk<32>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, rn, losses,
-                         stream);
+    return launch_topk<16>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, rn,
+                           losses, exported, stream);
+  return launch_topk<32>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, rn,
+                         losses, exported, stream);
+}
+
+cudaError_t enqueue_router_finalize(const int64_t* totals, int64_t T, int E, float aux_alpha,
+                                    float* lb_stats, float* losses, cudaStream_t stream) {
+  if (lb_stats == nullptr && losses == nullptr) return cudaSuccess;
+  return launch_kernel(router_finalize_kernel, dim3(1), dim3(256), 0, stream, totals, T, E,
+                       aux_alpha, lb_stats, losses);
 }
 
 }  // namespace moe

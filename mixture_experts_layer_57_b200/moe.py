@@ -93,6 +93,11 @@ def lib() -> ctypes.CDLL:
             "moe_layer_forward": ([P(LayerArgs), vp, P(LayerAux), vp, sz, vp], i32),
             "moe_layer_forward_profiled": ([P(LayerArgs), vp, P(LayerAux), vp, sz, vp,
                                             P(vp), i32, P(i32), ctypes.c_char_p, sz], i32),
+            "moe_layer_shard_workspace_bytes": ([P(LayerArgs), i64, P(sz)], i32),
+            "moe_router_partials_count": ([i32], i64),
+            "moe_layer_forward_shard_begin": ([P(LayerArgs), i64, P(LayerAux), vp, vp, vp, sz, vp], i32),
+            "moe_layer_forward_shard_end": ([P(LayerArgs), i64, i32, i32, vp, vp, vp, P(LayerAux), vp,
+                                             sz, vp], i32),
             "moe_workspace_reset": ([vp, sz, vp], i32),
             "moe_get_device_error": ([vp, P(i32), vp], i32),
         }
@@ -108,7 +113,7 @@ def header_symbols() -> list:
     """Names of the functions ``include/moe.h`` declares."""
     import re
     text = open(HEADER).read()
-    return sorted(set(re.findall(r"^\s*(?:const\s+char\s*\*|int|moe_status)\s+(moe_\w+)\s*\(", text, re.M)))
+    return sorted(set(re.findall(r"^\s*(?:const\s+char\s*\*|int64_t|int|moe_status)\s+(moe_\w+)\s*\(", text, re.M)))
 
 
 def _check(fn: str, status: int):
@@ -409,6 +414,84 @@ def moe_layer_forward_profiled(args: LayerArgs, out: torch.Tensor, events: list,
         ctypes.byref(args), _ptr(out), ctypes.byref(a), _ptr(ws), ws.numel(), _stream(stream),
         handles, len(events), ctypes.byref(n), names, 512))
     return names.value.decode().split(",")[: n.value]
+
+
+def _aux_struct(aux: Optional[dict]) -> LayerAux:
+    a = LayerAux()
+    if aux:
+        for name, t in aux.items():
+            setattr(a, name, _ptr(t))
+    return a
+
+
+def moe_layer_shard_workspace_bytes(args: LayerArgs, T_global: int) -> int:
+    out = ctypes.c_size_t()
+    _check("moe_layer_shard_workspace_bytes",
+           lib().moe_layer_shard_workspace_bytes(ctypes.byref(args), T_global, ctypes.byref(out)))
+    return out.value
+
+
+def moe_router_partials_count(E: int) -> int:
+    return int(lib().moe_router_partials_count(E))
+
+
+def moe_layer_forward_shard_begin(args: LayerArgs, T_global: int, demand: torch.Tensor,
+                                  stat_partials: torch.Tensor, aux: Optional[dict] = None,
+                                  ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """First half of a token shard's layer: writes ``demand`` [E] int32 and ``stat_partials``
+    [4E+1] int64; returns the workspace, which the second half must get unchanged."""
+    if ws is None:
+        ws = workspace(moe_layer_shard_workspace_bytes(args, T_global), demand.device)
+    _check("moe_layer_forward_shard_begin", lib().moe_layer_forward_shard_begin(
+        ctypes.byref(args), T_global, ctypes.byref(_aux_struct(aux)), _ptr(demand),
+        _ptr(stat_partials), _ptr(ws), ws.numel(), _stream(stream)))
+    return ws
+
+
+def moe_layer_forward_shard_end(args: LayerArgs, T_global: int, G: int, rank: int,
+                                demand_all: torch.Tensor, stat_totals: torch.Tensor,
+                                out: torch.Tensor, ws: torch.Tensor, aux: Optional[dict] = None,
+                                stream=None) -> torch.Tensor:
+    """Second half: dispatch with the global slot base, expert FFN and combine into ``out``."""
+    _check("moe_layer_forward_shard_end", lib().moe_layer_forward_shard_end(
+        ctypes.byref(args), T_global, G, rank, _ptr(demand_all), _ptr(stat_totals), _ptr(out),
+        ctypes.byref(_aux_struct(aux)), _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def exchange_shard_routing(demand: torch.Tensor, stat_partials: torch.Tensor, group=None):
+    """The one exchange step of the token-sharded layer: every shard's demand gathered in rank
+    order ([G, E] int32) and the statistics partials summed over shards (int64, exact)."""
+    import torch.distributed as dist
+    G = dist.get_world_size(group)
+    demand_all = torch.empty(G, demand.numel(), dtype=demand.dtype, device=demand.device)
+    if dist.get_backend(group) == "nccl":
+        dist.all_gather_into_tensor(demand_all, demand, group=group)
+    else:
+        dist.all_gather(list(demand_all.unbind(0)), demand, group=group)
+    totals = stat_partials.clone()
+    dist.all_reduce(totals, op=dist.ReduceOp.SUM, group=group)
+    return demand_all, totals
+
+
+def moe_layer_forward_sharded(args: LayerArgs, T_global: int, out: torch.Tensor, group=None,
+                              aux: Optional[dict] = None, ws: Optional[torch.Tensor] = None,
+                              stream=None) -> torch.Tensor:
+    """The token-sharded layer on this rank (tokens of the ranks in rank order make the batch of
+    ``T_global``): begin, the exchange over ``group``, end."""
+    import torch.distributed as dist
+    E = args.E
+    dev = out.device
+    demand = torch.empty(E, dtype=torch.int32, device=dev)
+    partials = torch.empty(moe_router_partials_count(E), dtype=torch.int64, device=dev)
+    s = torch.cuda.current_stream(dev) if stream is None else stream
+    with torch.cuda.stream(s):  # the collectives run on the same stream as the kernels
+        ws = moe_layer_forward_shard_begin(args, T_global, demand, partials, aux=aux, ws=ws,
+                                           stream=s)
+        demand_all, totals = exchange_shard_routing(demand, partials, group)
+        return moe_layer_forward_shard_end(args, T_global, dist.get_world_size(group),
+                                           dist.get_rank(group), demand_all, totals, out, ws,
+                                           aux=aux, stream=s)
 
 
 def moe_workspace_reset(ws: torch.Tensor, stream=None):

@@ -187,6 +187,32 @@ def test_layer_validation_and_workspace(L):
     assert L.moe_layer_forward(ctypes.byref(args), FAKE, ctypes.byref(aux), FAKE, nbytes, None) == 6
 
 
+def test_shard_entry_validation(L):
+    args = moe.LayerArgs(T=4096, d_model=1024, d_ff=4096, E=128, k=1, capacity_factor=1.0,
+                         dtype=1, out_dtype=1, x=FAKE, w_router=FAKE, w1=FAKE, w2=FAKE,
+                         add_input_residual=1, aux_alpha=0.01)
+    assert moe.moe_router_partials_count(128) == 513
+    nb = moe.moe_layer_shard_workspace_bytes(args, 16384)
+    # the capacity (and so nothing else in the layout) follows the whole batch
+    assert nb >= moe.moe_layer_workspace_bytes(args)
+    sz = ctypes.c_size_t()
+    assert L.moe_layer_shard_workspace_bytes(ctypes.byref(args), 4095, ctypes.byref(sz)) == 1
+    aux = moe.LayerAux()
+    beg = lambda T_global=16384, dem=FAKE, par=FAKE, wsb=nb: L.moe_layer_forward_shard_begin(
+        ctypes.byref(args), T_global, ctypes.byref(aux), dem, par, FAKE, wsb, None)
+    end = lambda T_global=16384, G=4, r=1, da=FAKE, tot=FAKE, wsb=nb: L.moe_layer_forward_shard_end(
+        ctypes.byref(args), T_global, G, r, da, tot, FAKE, ctypes.byref(aux), FAKE, wsb, None)
+    assert beg(T_global=100) == 1               # the shard is part of the batch
+    assert beg(dem=None) == 1 and beg(par=None) == 1
+    assert beg(par=FAKE + 8) == 6
+    assert beg(wsb=nb - 1) == 3
+    assert end(G=0) == 1 and end(r=4) == 1 and end(r=-1) == 1
+    assert end(da=None) == 1 and end(tot=None) == 1
+    assert end(tot=FAKE + 4) == 6
+    args.overflow_policy = moe.MOE_OVERFLOW_PRIORITY
+    assert beg() == 2 and end() == 2            # a global priority order is not sharded
+
+
 def test_fault_injection_is_host_side(L, monkeypatch):
     # the injected failure is returned after validation and before any enqueue
     monkeypatch.setenv("MOE_FAULT_INJECT", "moe_router_topk")
