@@ -103,7 +103,6 @@ __device__ void block_exclusive_scan_experts(int v, int E, int* warp_sums, int32
   const int excl = incl - v + warp_sums[warp];
   if (tid < E) out[tid] = excl;
   if (tid == E - 1) out[E] = excl + v;
-  __syncthreads();  // warp_sums may be reused
 }
 
 __global__ void __launch_bounds__(1024)
@@ -113,7 +112,6 @@ __global__ void __launch_bounds__(1024)
                          ShardBase shard) {
   __shared__ int run_sum[1024];
   __shared__ int kept[MOE_MAX_EXPERTS];
-  __shared__ int demand[MOE_MAX_EXPERTS];
   __shared__ int warp_sums[32];
   pdl_wait();
   const int tid = threadIdx.x;
@@ -171,14 +169,15 @@ __global__ void __launch_bounds__(1024)
         shard.cap_local[e] = (int32_t)cap;
       }
       kept[e] = (int)min((int64_t)run, cap);
-      demand[e] = run;
     }
   }
   __syncthreads();
   // exclusive scans over experts (E <= 1024), one element per thread
   block_exclusive_scan_experts(tid < E ? kept[tid] : 0, E, warp_sums, offsets);
-  if (demand_offsets != nullptr)
-    block_exclusive_scan_experts(tid < E ? demand[tid] : 0, E, warp_sums, demand_offsets);
+  if (demand_offsets != nullptr) {
+    __syncthreads();  // warp_sums is reused; counts (global) were written before the first sync
+    block_exclusive_scan_experts(tid < E ? counts[tid] : 0, E, warp_sums, demand_offsets);
+  }
   pdl_trigger();
 }
 

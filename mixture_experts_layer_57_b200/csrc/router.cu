@@ -257,7 +257,7 @@ __global__ void __launch_bounds__(256)
 
 // EPL = experts per lane (E <= 32 * EPL); expert e lives in lane e % 32, slot e / 32.
 // COUNT: also rank this block's (token, choice) pairs per expert in pair order for dispatch.
-template <int EPL, bool COUNT>
+template <int EPL, bool COUNT, bool EXTRA>
 __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restrict__ logits,
                                                           int64_t T, int E, int k,
                                                           int32_t* __restrict__ ids,
@@ -265,12 +265,13 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
                                                           RouterAccum acc, float alpha,
                                                           float* __restrict__ lb,
                                                           RouterDispatchCount dc, int renorm,
-                                                          float* __restrict__ losses, int extra,
+                                                          float* __restrict__ losses,
                                                           int64_t* __restrict__ exported) {
   __shared__ float qs[8][MOE_MAX_EXPERTS];
   // per expert: first-choice count << 16 | choice count (each at most kRouterTokensPerBlock)
   __shared__ unsigned cs[MOE_MAX_EXPERTS];
-  __shared__ unsigned imp_s[MOE_MAX_EXPERTS];  // gate sums, 2^-24 fixed point (< 2^31 per block)
+  // gate sums, 2^-24 fixed point (< 2^31 per block); only with the extra statistics
+  __shared__ unsigned imp_s[EXTRA ? MOE_MAX_EXPERTS : 1];
   __shared__ float zs[8];
   __shared__ float prod[MOE_MAX_EXPERTS];
   __shared__ int is_last;
@@ -279,7 +280,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int e = threadIdx.x; e < E; e += 256) {
     cs[e] = 0u;
-    imp_s[e] = 0u;
+    if constexpr (EXTRA) imp_s[e] = 0u;
   }
   __syncthreads();
   float zw = 0.0f;  // this warp's sum of (log Z)^2 over its tokens, in token order
@@ -309,7 +310,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (extra) {
+    if constexpr (EXTRA) {
       const float lz = m + logf(s);  // log sum_e exp(l_e)
       zw += lz * lz;
     }
@@ -329,7 +330,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
     // per-block integer counts (order-independent): first choices, and with the extra
     // statistics every choice and its gate
     auto count_choice = [&](int e, int j, float g) {
-      if (extra) {
+      if constexpr (EXTRA) {
         atomicAdd(&cs[e], j == 0 ? 0x10001u : 1u);
         atomicAdd(&imp_s[e], __float2uint_rn(g * (float)kIScale));
       } else if (j == 0) {
@@ -439,10 +440,12 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
     const unsigned long long fx = (unsigned long long)llrint((double)sum * kQScale);
     if (fx) atomicAdd(&acc.q[e], fx);
     if (cs[e] >> 16) atomicAdd(&acc.c[e], cs[e] >> 16);
-    if (cs[e] & 0xffffu) atomicAdd(&acc.load[e], cs[e] & 0xffffu);
-    if (imp_s[e]) atomicAdd(&acc.imp[e], (unsigned long long)imp_s[e]);
+    if constexpr (EXTRA) {
+      if (cs[e] & 0xffffu) atomicAdd(&acc.load[e], cs[e] & 0xffffu);
+      if (imp_s[e]) atomicAdd(&acc.imp[e], (unsigned long long)imp_s[e]);
+    }
   }
-  if (extra && threadIdx.x == 0) {
+  if (EXTRA && threadIdx.x == 0) {
     float zb = 0.0f;
 #pragma unroll
     for (int w = 0; w < 8; ++w) zb += zs[w];
@@ -480,14 +483,16 @@ cudaError_t launch_topk(const float* logits, int64_t T, int E, int k, int32_t* i
                         const RouterAccum& acc, float alpha, float* lb, RouterDispatchCount dc,
                         int renorm, float* losses, int64_t* exported, cudaStream_t stream) {
   const dim3 grid((unsigned)router_num_blocks(T));
-  const int extra = (losses != nullptr || exported != nullptr) ? 1 : 0;
+  const bool extra = losses != nullptr || exported != nullptr;
+  auto go = [&](auto kern) {
+    return launch_kernel(kern, grid, dim3(256), 0, stream, (const float*)logits, T, E, k, ids,
+                         gates, acc, alpha, lb, dc, renorm, losses, exported);
+  };
   if (dc.local_rank != nullptr)
-    return launch_kernel(router_topk_kernel<EPL, true>, grid, dim3(256), 0, stream,
-                         (const float*)logits, T, E, k, ids, gates, acc, alpha, lb, dc, renorm,
-                         losses, extra, exported);
-  return launch_kernel(router_topk_kernel<EPL, false>, grid, dim3(256), 0, stream,
-                       (const float*)logits, T, E, k, ids, gates, acc, alpha, lb, dc, renorm,
-                       losses, extra, exported);
+    return extra ? go(router_topk_kernel<EPL, true, true>)
+                 : go(router_topk_kernel<EPL, true, false>);
+  return extra ? go(router_topk_kernel<EPL, false, true>)
+               : go(router_topk_kernel<EPL, false, false>);
 }
 
 }  // namespace
