@@ -76,6 +76,12 @@ def lib():
             [i64, i32, i32, i32, i32, dbl, i32, i32] + [vp] * 11 + [dbl, vp, vp, i64] + [vp] * 8
             + [i32, i32, i32, vp, vp])
         L.oracle_layer_forward.restype = i64
+        L.oracle_gelu_grad.argtypes = [dbl]
+        L.oracle_gelu_grad.restype = dbl
+        L.oracle_layer_backward.argtypes = (
+            [i64, i32, i32, i32, i32, dbl, i32, i32] + [vp] * 11 + [dbl, i32, i32, vp, vp, vp, dbl, dbl]
+            + [vp] * 13)
+        L.oracle_layer_backward.restype = None
         _lib = L
     return _lib
 
@@ -255,3 +261,59 @@ def layer_forward(inp: dict, T: int, d_model: int, d_ff: int, E: int, k: int,
                 f=stats[:E], Q=stats[E:2 * E], aux=float(stats[2 * E]), out_exact=out_exact,
                 out=out, tokens=tok, z_loss=float(losses[0]), cov2_importance=float(losses[1]),
                 cov2_load=float(losses[2]))
+
+
+def gelu_grad(z: float) -> float:
+    return lib().oracle_gelu_grad(float(z))
+
+
+def layer_backward(inp: dict, T: int, d_model: int, d_ff: int, E: int, k: int,
+                   capacity_factor: float, dout: np.ndarray, add_input_residual: bool = True,
+                   aux_alpha: float = 0.01, aux_weight: float = 0.0, z_weight: float = 0.0,
+                   logits_in: Optional[np.ndarray] = None, gates_in: Optional[np.ndarray] = None,
+                   overflow_priority: bool = False, renormalize: bool = False) -> dict:
+    """Gradients (float64) of L = sum(dout * out) + aux_weight * aux + z_weight * z_loss.
+
+    Returns dict: dx, dw_router, db_router, dw1, db1, dw2, db2, dense_dw1, dense_db1,
+    dense_dw2, dense_db2 (dense ones None without the dense MLP), dgates [T,k], dlogits [T,E].
+    """
+    L = lib()
+    x = inp["x"]
+    bf16 = _is_bf16(x)
+    d, f = d_model, d_ff
+    g = inp.get
+    dense = g("dense_w1") is not None
+    out = dict(dx=np.empty((T, d)), dw_router=np.empty((E, d)), db_router=np.empty(E),
+               dw1=np.empty((E, f, d)), db1=np.empty((E, f)), dw2=np.empty((E, d, f)),
+               db2=np.empty((E, d)), dgates=np.empty((T, k)), dlogits=np.empty((T, E)))
+    out.update(dense_dw1=np.empty((f, d)) if dense else None,
+               dense_db1=np.empty(f) if dense else None,
+               dense_dw2=np.empty((d, f)) if dense else None,
+               dense_db2=np.empty(d) if dense else None)
+    li = None if logits_in is None else np.ascontiguousarray(logits_in, dtype=np.float32)
+    gi = None if gates_in is None else np.ascontiguousarray(gates_in, dtype=np.float32)
+    go = np.ascontiguousarray(dout, dtype=np.float64)
+    L.oracle_layer_backward(
+        T, d, f, E, k, capacity_factor, bf16, int(bool(add_input_residual)),
+        _p(x), _p(np.ascontiguousarray(inp["w_router"], dtype=np.float32)), _p(g("router_bias")),
+        _p(inp["w1"]), _p(g("b1")), _p(inp["w2"]), _p(g("b2")),
+        _p(g("dense_w1")), _p(g("dense_b1")), _p(g("dense_w2")), _p(g("dense_b2")),
+        aux_alpha, int(bool(overflow_priority)), int(bool(renormalize)), _p(li), _p(gi), _p(go),
+        aux_weight, z_weight,
+        _p(out["dx"]), _p(out["dw_router"]), _p(out["db_router"]), _p(out["dw1"]), _p(out["db1"]),
+        _p(out["dw2"]), _p(out["db2"]), _p(out["dense_dw1"]), _p(out["dense_db1"]),
+        _p(out["dense_dw2"]), _p(out["dense_db2"]), _p(out["dgates"]), _p(out["dlogits"]))
+    return out
+
+
+def layer_loss(inp: dict, T: int, d_model: int, d_ff: int, E: int, k: int, capacity_factor: float,
+               dout: np.ndarray, add_input_residual: bool = True, aux_alpha: float = 0.01,
+               aux_weight: float = 0.0, z_weight: float = 0.0, overflow_priority: bool = False,
+               renormalize: bool = False) -> float:
+    """L = sum(dout * out) + aux_weight * aux + z_weight * z_loss from the forward oracle (the
+    objective layer_backward differentiates)."""
+    r = layer_forward(inp, T, d_model, d_ff, E, k, capacity_factor,
+                      add_input_residual=add_input_residual, aux_alpha=aux_alpha,
+                      overflow_priority=overflow_priority, renormalize=renormalize)
+    return (float(np.sum(np.asarray(dout, dtype=np.float64) * r["out_exact"]))
+            + aux_weight * r["aux"] + z_weight * r["z_loss"])

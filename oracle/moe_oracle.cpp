@@ -364,4 +364,185 @@ int64_t oracle_layer_forward(int64_t T, int d, int d_ff, int E, int k, double ca
   return C;
 }
 
+// ---------------------------------------------------------------- backward (training)
+//
+// The gradient of the training objective
+//     L = sum_{t,i} dout[t,i] * out[t,i] + aux_weight * aux + z_weight * z_loss
+// with respect to x, W_r, b_r, every expert's W1, b1, W2, b2 and the dense MLP's weights, by the
+// chain rule through the forward pass above (the pages' headline numbers are training
+// throughput; DeepSpeed-MoE notes on training cost; survey notes §1.1.4.1 and the comparison
+// article's "Router Z-loss" give the two extra loss terms). Readings:
+//   * the routing decisions (top-k ids, slots, the counts f_i) are piecewise constant and carry
+//     no gradient; the gates carry it through the softmax (and the renormalisation);
+//   * a dropped pair contributes nothing forward, so nothing backward (comparison article,
+//     "Expert Capacity Overflow": no gradient for that expert);
+//   * the roundings of the forward pass (fp32 logits, bf16 h) are passed straight through, and
+//     every gradient uses the forward's own values (y rounded to fp32, h to bf16).
+
+// dGeLU/dz for GeLU(z) = z * Phi(z): Phi(z) + z * phi(z).
+double oracle_gelu_grad(double z) {
+  const double Phi = 0.5 * (1.0 + std::erf(z / std::sqrt(2.0)));
+  const double phi = std::exp(-0.5 * z * z) / std::sqrt(2.0 * M_PI);
+  return Phi + z * phi;
+}
+
+// One FFN (an expert or the dense MLP) on one token, forward then backward for an output
+// gradient dy (d doubles). Accumulates dW1 [d_ff, d], db1 [d_ff], dW2 [d, d_ff], db2 [d] and
+// dx_row [d]; y_out (optional) receives the forward output rounded to fp32.
+static void ffn_backward(const void* x_row, int bf16, int d, int d_ff, const void* w1,
+                         const void* b1, const void* w2, const void* b2, const double* dy,
+                         double* dw1, double* db1, double* dw2, double* db2, double* dx_row) {
+  std::vector<double> z(d_ff), h(d_ff), dz(d_ff);
+  for (int j = 0; j < d_ff; ++j) {
+    double a = 0.0;
+    for (int i = 0; i < d; ++i) a += load(w1, bf16, (int64_t)j * d + i) * load(x_row, bf16, i);
+    if (b1) a += load(b1, bf16, j);
+    z[j] = a;
+    const double g = oracle_gelu(a);
+    h[j] = bf16 ? oracle_bf16_to_double(oracle_round_bf16(g)) : g;
+  }
+  // y = W2 h + b2: dW2 += dy h^T, db2 += dy, dh = W2^T dy
+  for (int o = 0; o < d; ++o) {
+    if (db2) db2[o] += dy[o];
+    for (int j = 0; j < d_ff; ++j) dw2[(int64_t)o * d_ff + j] += dy[o] * h[j];
+  }
+  for (int j = 0; j < d_ff; ++j) {
+    double dh = 0.0;
+    for (int o = 0; o < d; ++o) dh += load(w2, bf16, (int64_t)o * d_ff + j) * dy[o];
+    dz[j] = dh * oracle_gelu_grad(z[j]);
+  }
+  // z = W1 x + b1: dW1 += dz x^T, db1 += dz, dx += W1^T dz
+  for (int j = 0; j < d_ff; ++j) {
+    if (db1) db1[j] += dz[j];
+    for (int i = 0; i < d; ++i) dw1[(int64_t)j * d + i] += dz[j] * load(x_row, bf16, i);
+  }
+  for (int i = 0; i < d; ++i) {
+    double s = 0.0;
+    for (int j = 0; j < d_ff; ++j) s += load(w1, bf16, (int64_t)j * d + i) * dz[j];
+    dx_row[i] += s;
+  }
+}
+
+// Gradients of the whole layer. Inputs are those of oracle_layer_forward (logits_in / gates_in
+// as there: routing decided on another implementation's fp32 values), plus dout [T, d] and the
+// weights of the two extra loss terms. Outputs (double, zeroed here, any may be NULL):
+// dx [T, d], dw_r [E, d], db_r [E], dw1 [E, d_ff, d], db1 [E, d_ff], dw2 [E, d, d_ff],
+// db2 [E, d], and the dense MLP's ddw1 [d_ff, d], ddb1 [d_ff], ddw2 [d, d_ff], ddb2 [d].
+// dgates (optional, [T, k]) receives dL/dgate of each choice; dlogits (optional, [T, E]) dL/dl.
+void oracle_layer_backward(int64_t T, int d, int d_ff, int E, int k, double capacity_factor,
+                           int bf16, int add_input_residual, const void* x, const float* w_r,
+                           const float* b_r, const void* w1, const void* b1, const void* w2,
+                           const void* b2, const void* dense_w1, const void* dense_b1,
+                           const void* dense_w2, const void* dense_b2, double aux_alpha,
+                           int overflow_priority, int renormalize, const float* logits_in,
+                           const float* gates_in, const double* dout, double aux_weight,
+                           double z_weight, double* dx, double* dw_r, double* db_r, double* dw1,
+                           double* db1, double* dw2, double* db2, double* ddw1, double* ddb1,
+                           double* ddw2, double* ddb2, double* dgates, double* dlogits) {
+  // ---- forward decisions
+  std::vector<float> logits((size_t)T * E);
+  if (logits_in) std::memcpy(logits.data(), logits_in, sizeof(float) * T * E);
+  else oracle_router_logits(x, bf16, T, d, w_r, b_r, E, logits.data());
+  std::vector<int32_t> ids((size_t)T * k), slot((size_t)T * k), counts(E);
+  std::vector<float> gates((size_t)T * k);
+  std::vector<double> probs((size_t)T * E);
+  oracle_route(logits.data(), T, E, k, ids.data(), gates.data(), probs.data());
+  std::vector<float> raw = gates;  // the chosen p before any renormalisation
+  if (renormalize) oracle_renormalize_gates(gates.data(), T, k);
+  if (gates_in) std::memcpy(gates.data(), gates_in, sizeof(float) * T * k);
+  std::vector<double> f(E), Q(E);
+  double aux = 0.0;
+  oracle_lb_stats(logits.data(), ids.data(), T, E, k, aux_alpha, f.data(), Q.data(), &aux);
+  const int64_t C = oracle_capacity(T, E, k, capacity_factor);
+  if (overflow_priority) oracle_assign_slots_priority(ids.data(), gates.data(), T, k, E, C, slot.data(), counts.data());
+  else oracle_assign_slots(ids.data(), T, k, E, C, slot.data(), counts.data());
+
+  auto zero = [](double* a, size_t n) { if (a) std::fill(a, a + n, 0.0); };
+  zero(dx, (size_t)T * d);
+  zero(dw_r, (size_t)E * d);
+  zero(db_r, E);
+  zero(dw1, (size_t)E * d_ff * d);
+  zero(db1, (size_t)E * d_ff);
+  zero(dw2, (size_t)E * d * d_ff);
+  zero(db2, (size_t)E * d);
+  zero(ddw1, (size_t)d_ff * d);
+  zero(ddb1, d_ff);
+  zero(ddw2, (size_t)d * d_ff);
+  zero(ddb2, d);
+  const size_t es = bf16 ? 2 : 4;
+  std::vector<double> dx_row(d), dy(d), dl(E), dp(E);
+  std::vector<float> y(d);
+  for (int64_t t = 0; t < T; ++t) {
+    const char* xt = (const char*)x + (size_t)t * d * es;
+    const double* go = dout + (size_t)t * d;
+    std::fill(dx_row.begin(), dx_row.end(), 0.0);
+    // residual: out += x
+    if (add_input_residual)
+      for (int i = 0; i < d; ++i) dx_row[i] += go[i];
+    // dense MLP: out += DenseMLP(x)
+    if (dense_w1) ffn_backward(xt, bf16, d, d_ff, dense_w1, dense_b1, dense_w2, dense_b2, go, ddw1,
+                               dense_b1 ? ddb1 : nullptr, ddw2, dense_b2 ? ddb2 : nullptr,
+                               dx_row.data());
+    // experts: out += gate_j * y_j over the kept choices
+    std::vector<double> dg(k, 0.0);
+    for (int j = 0; j < k; ++j) {
+      if (slot[t * k + j] < 0) continue;
+      const int e = ids[t * k + j];
+      const size_t w1o = (size_t)e * d_ff * d * es, w2o = (size_t)e * d * d_ff * es;
+      const void* we1 = (const char*)w1 + w1o;
+      const void* we2 = (const char*)w2 + w2o;
+      const void* be1 = b1 ? (const void*)((const char*)b1 + (size_t)e * d_ff * es) : nullptr;
+      const void* be2 = b2 ? (const void*)((const char*)b2 + (size_t)e * d * es) : nullptr;
+      oracle_ffn(xt, bf16, d, d_ff, we1, be1, we2, be2, y.data());
+      double s = 0.0;
+      for (int i = 0; i < d; ++i) s += go[i] * (double)y[i];
+      dg[j] = s;  // dL/dgate
+      const double g = gates[t * k + j];
+      for (int i = 0; i < d; ++i) dy[i] = g * go[i];
+      ffn_backward(xt, bf16, d, d_ff, we1, be1, we2, be2, dy.data(), dw1 + (size_t)e * d_ff * d,
+                   b1 ? db1 + (size_t)e * d_ff : nullptr, dw2 + (size_t)e * d * d_ff,
+                   b2 ? db2 + (size_t)e * d : nullptr, dx_row.data());
+    }
+    if (dgates)
+      for (int j = 0; j < k; ++j) dgates[t * k + j] = dg[j];
+    // gates -> p: gate_j = p_{e_j} (or p_{e_j} / S with S = sum of the chosen p)
+    const double* pt = probs.data() + (size_t)t * E;
+    std::fill(dp.begin(), dp.end(), 0.0);
+    if (renormalize) {
+      double S = 0.0, gdg = 0.0;
+      for (int j = 0; j < k; ++j) S += (double)raw[t * k + j];
+      for (int j = 0; j < k; ++j) gdg += dg[j] * ((double)raw[t * k + j] / S);
+      for (int j = 0; j < k; ++j) dp[ids[t * k + j]] += (dg[j] - gdg) / S;
+    } else {
+      for (int j = 0; j < k; ++j) dp[ids[t * k + j]] += dg[j];
+    }
+    // aux = alpha * E * sum_e f_e * Q_e, Q_e = (1/T) sum_t p_te, f constant
+    for (int e = 0; e < E; ++e) dp[e] += aux_weight * aux_alpha * E * f[e] / (double)T;
+    // p = softmax(l): dl_e = p_e (dp_e - sum_e' p_e' dp_e')
+    double pdp = 0.0;
+    for (int e = 0; e < E; ++e) pdp += pt[e] * dp[e];
+    for (int e = 0; e < E; ++e) dl[e] = pt[e] * (dp[e] - pdp);
+    // z-loss = (1/T) sum_t (log sum_e exp l_te)^2: dl_e += 2 log Z p_e / T
+    if (z_weight != 0.0) {
+      double m = -INFINITY;
+      for (int e = 0; e < E; ++e) m = std::max(m, (double)logits[(size_t)t * E + e]);
+      double zs = 0.0;
+      for (int e = 0; e < E; ++e) zs += std::exp((double)logits[(size_t)t * E + e] - m);
+      const double lz = m + std::log(zs);
+      for (int e = 0; e < E; ++e) dl[e] += z_weight * 2.0 * lz * pt[e] / (double)T;
+    }
+    if (dlogits)
+      for (int e = 0; e < E; ++e) dlogits[(size_t)t * E + e] = dl[e];
+    // l = W_r x + b_r
+    for (int e = 0; e < E; ++e) {
+      if (db_r) db_r[e] += dl[e];
+      if (dw_r)
+        for (int i = 0; i < d; ++i) dw_r[(size_t)e * d + i] += dl[e] * load(xt, bf16, i);
+      for (int i = 0; i < d; ++i) dx_row[i] += (double)w_r[(size_t)e * d + i] * dl[e];
+    }
+    if (dx)
+      for (int i = 0; i < d; ++i) dx[(size_t)t * d + i] = dx_row[i];
+  }
+}
+
 }  // extern "C"
