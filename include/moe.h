@@ -315,6 +315,48 @@ moe_status moe_layer_forward_shard_end(const moe_layer_args* args, int64_t T_glo
                                        const int64_t* stat_totals, void* out, moe_layer_aux* aux,
                                        void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* ---------------------------------------------------------------- training
+ * The backward pass of the layer: gradients of the objective
+ *     L = sum_{t,i} d_out[t,i] * out[t,i] + aux_weight * aux + z_weight * z_loss
+ * (aux = lb_stats[2E], the load-balance loss; z_loss the router z-loss of moe_router_topk_ex),
+ * by the chain rule through the forward pass. The routing decisions (top-k ids, slots, the
+ * counts f_i) are held fixed; the gates carry the gradient to the router through the softmax
+ * (and the renormalisation when enabled); a dropped choice contributes nothing (comparison
+ * article, "Expert Capacity Overflow": no gradient for that expert).
+ *
+ * moe_layer_forward_train is moe_layer_forward that also keeps, in the workspace, what the
+ * backward pass reads: logits, routing, the packed rows, h and GeLU'(z) of every expert row and
+ * of the dense MLP, and the expert outputs y. moe_layer_backward then takes the same args and
+ * workspace (unchanged in between) and the output gradient d_out [T, d_model] in args.dtype.
+ * Results are identical to moe_layer_forward (the combine runs as its own kernel here).
+ *
+ * Gradients (fp32, overwritten; shapes those of the parameters): dw_router, db_router, dw1, db1,
+ * dw2, db2 and the dense MLP's; dx [T, d_model] in args.dtype. A bias gradient pointer may be
+ * NULL (not computed). dgates [T, k] (dL/dgate) and dlogits [T, E] (dL/dlogits) are optional.
+ * bf16 layers run the expert and dense GEMMs on tcgen05 (bf16 operands: dY, dZ rounded to bf16;
+ * fp32 accumulation); the router's GEMMs and fp32 layers run on fp32 FMA. */
+typedef struct {
+  void* dx;                /* [T, d_model], args.dtype */
+  float* dw_router;        /* [E, d_model] */
+  float* db_router;        /* [E] or NULL */
+  float* dw1;              /* [E, d_ff, d_model] */
+  float* db1;              /* [E, d_ff] or NULL */
+  float* dw2;              /* [E, d_model, d_ff] */
+  float* db2;              /* [E, d_model] or NULL */
+  float* dense_dw1;        /* [d_ff, d_model] (dense MLP only) */
+  float* dense_db1;        /* [d_ff] or NULL */
+  float* dense_dw2;        /* [d_model, d_ff] */
+  float* dense_db2;        /* [d_model] or NULL */
+  float* dgates;           /* [T, k] or NULL */
+  float* dlogits;          /* [T, E] or NULL */
+} moe_layer_grads;
+moe_status moe_layer_train_workspace_bytes(const moe_layer_args* args, size_t* bytes);
+moe_status moe_layer_forward_train(const moe_layer_args* args, void* out, moe_layer_aux* aux,
+                                   void* ws, size_t ws_bytes, moe_stream_t stream);
+moe_status moe_layer_backward(const moe_layer_args* args, const void* d_out, float aux_weight,
+                              float z_weight, moe_layer_grads* grads, void* ws, size_t ws_bytes,
+                              moe_stream_t stream);
+
 /* ---------------------------------------------------------------- status block
  * moe_workspace_reset: zeroes the status block (asynchronous on stream).
  * moe_get_device_error: synchronises `stream`, copies the status word to *code_out and returns

@@ -790,6 +790,381 @@ moe_status moe_layer_forward_shard_end(const moe_layer_args* args, int64_t T_glo
 
 // ---------------------------------------------------------------- status block
 
+// ---------------------------------------------------------------- training
+
+}  // extern "C"
+
+namespace {
+
+// Training workspace: the forward layout, then what the backward pass needs beyond it.
+struct TrainWs {
+  LayerWs L;
+  void* g_packed;      // [R, d_ff] GeLU'(z) of the experts' layer 1 (dtype)
+  void* g_dense;       // [T, d_ff] the dense MLP's (dtype)
+  float* r_dense;      // [T, d] dense MLP output (fp32)
+  float* dgate;        // [T, k]
+  float* dl;           // [T, E]
+  void* dy;            // [R, d] (dtype)
+  void* dz;            // [R, d_ff] (dtype)
+  float* dxp;          // [R, d]
+  float* dx_router;    // [T, d]
+  void* dzd;           // [T, d_ff] (dtype)
+  float* dxd;          // [T, d]
+  float* part_colsum;
+  float* part_router;
+  int S_e, S_d, splits_r;
+};
+
+int router_wgrad_splits(int64_t T) {
+  const int64_t s = (T + 1023) / 1024;
+  return (int)(s < 1 ? 1 : (s > 64 ? 64 : s));
+}
+
+moe_status train_layout(const moe_layer_args* a, uint8_t* base, TrainWs* w, size_t* bytes) {
+  size_t fwd = 0;
+  moe_status st = layer_layout(a, base, &w->L, &fwd);
+  if (st != MOE_OK) return st;
+  const int64_t T = a->T, R = w->L.rows_max;
+  const int E = a->E, k = a->k, d = a->d_model, f = a->d_ff;
+  const size_t es = esize(a->dtype);
+  const bool dense = a->dense_w1 != nullptr;
+  Carve c{base};
+  c.off = fwd;
+  w->g_packed = c.take<uint8_t>((size_t)R * f * es);
+  w->g_dense = dense ? (void*)c.take<uint8_t>((size_t)T * f * es) : nullptr;
+  w->r_dense = dense ? (w->L.r_dense ? w->L.r_dense : c.take<float>((size_t)T * d)) : nullptr;
+  w->dgate = c.take<float>((size_t)T * k);
+  w->dl = c.take<float>((size_t)T * E);
+  w->dy = c.take<uint8_t>((size_t)R * d * es);
+  w->dz = c.take<uint8_t>((size_t)R * f * es);
+  w->dxp = c.take<float>((size_t)R * d);
+  w->dx_router = c.take<float>((size_t)T * d);
+  w->dzd = dense ? (void*)c.take<uint8_t>((size_t)T * f * es) : nullptr;
+  w->dxd = dense ? c.take<float>((size_t)T * d) : nullptr;
+  const int64_t seg = w->L.C < T ? w->L.C : T;
+  w->S_e = colsum_splits(seg);
+  w->S_d = colsum_splits(T);
+  const int64_t wide = d > f ? d : f;
+  int64_t pc = (int64_t)E * w->S_e * wide;
+  if ((int64_t)w->S_d * wide > pc) pc = (int64_t)w->S_d * wide;
+  if ((int64_t)w->S_d * E > pc) pc = (int64_t)w->S_d * E;
+  w->part_colsum = c.take<float>((size_t)pc);
+  w->splits_r = router_wgrad_splits(T);
+  w->part_router = c.take<float>((size_t)w->splits_r * E * d);
+  *bytes = c.off;
+  return MOE_OK;
+}
+
+moe_status copy_out(void* dst, const void* src, size_t n, cudaStream_t stream) {
+  if (dst == nullptr || n == 0) return MOE_OK;
+  return cudaMemcpyAsync(dst, src, n, cudaMemcpyDeviceToDevice, stream) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
+}
+
+moe_status check_layer_pointers(const moe_layer_args* a, const void* out, const void* ws) {
+  const bool dense = a->dense_w1 != nullptr;
+  if (dense && !a->dense_w2) return MOE_ERR_INVALID_ARGUMENT;
+  if (!ws) return MOE_ERR_INVALID_ARGUMENT;
+  if (a->T > 0 && (!a->x || !a->w_router || !a->w1 || !a->w2 || !out))
+    return MOE_ERR_INVALID_ARGUMENT;
+  if (!aligned16(a->x) || !aligned16(a->w_router) || !aligned16(a->router_bias) ||
+      !aligned16(a->w1) || !aligned16(a->b1) || !aligned16(a->w2) || !aligned16(a->b2) ||
+      !aligned16(a->dense_w1) || !aligned16(a->dense_b1) || !aligned16(a->dense_w2) ||
+      !aligned16(a->dense_b2) || !aligned16(out) || ((uintptr_t)ws % kAlign) != 0)
+    return MOE_ERR_MISALIGNED;
+  return MOE_OK;
+}
+
+moe_status forward_train_impl(const moe_layer_args* a, void* out, moe_layer_aux* aux, void* ws,
+                              size_t ws_bytes, cudaStream_t stream) {
+  TrainWs w;
+  size_t need = 0;
+  moe_status st = train_layout(a, (uint8_t*)ws, &w, &need);
+  if (st != MOE_OK) return st;
+  st = check_layer_pointers(a, out, ws);
+  if (st != MOE_OK) return st;
+  if (aux && (!aligned16(aux->logits) || !aligned16(aux->expert_ids) || !aligned16(aux->gates) ||
+              !aligned16(aux->slot) || !aligned16(aux->expert_counts) ||
+              !aligned16(aux->expert_offsets) || !aligned16(aux->lb_stats) ||
+              !aligned16(aux->router_losses)))
+    return MOE_ERR_MISALIGNED;
+  if (ws_bytes < need) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (fault_injected("moe_layer_forward_train")) return MOE_ERR_CUDA;
+  g_launches = 0;
+  if (a->T == 0) return MOE_OK;
+  const LayerWs& L = w.L;
+  int* status = (int*)ws;
+  const bool bf16 = a->dtype == MOE_BF16;
+  const bool dense = a->dense_w1 != nullptr;
+  const int64_t T = a->T;
+  const int d = a->d_model, f = a->d_ff, E = a->E, k = a->k;
+  // routing state stays in the workspace for the backward pass; aux receives copies
+  RouterDispatchCount dcount;
+  dcount.local_rank = L.dispatch.local_rank;
+  dcount.seg_counts = L.dispatch.seg_counts;
+  cudaError_t e = enqueue_router(a->x, bf16, T, d, a->w_router, a->router_bias, E, k,
+                                 L.router.logits, L.ids, L.gates, L.lb_stats, a->aux_alpha,
+                                 L.router.scr, status, stream, dcount, a->renormalize_gates != 0,
+                                 aux ? aux->router_losses : nullptr);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  PriorityDispatch prio;
+  if (a->overflow_policy == MOE_OVERFLOW_PRIORITY) {
+    prio.gates = L.gates;
+    prio.list = L.dispatch.prio_list;
+    prio.demand_offsets = L.dispatch.demand_offsets;
+  }
+  e = enqueue_dispatch(a->x, bf16, T, d, L.ids, E, k, L.C, L.slot, L.counts, L.offsets,
+                       L.row_token, L.x_packed, L.rows_max, L.dispatch.local_rank,
+                       L.dispatch.seg_counts, L.dispatch.seg_base, status, stream, DroppedRows{},
+                       (int)kRouterTokensPerBlock * k, prio);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  if (bf16) {
+    if (L.rows_max > 0) {
+      e = enqueue_grouped_gemm_bf16_train(L.x_packed, L.offsets, E, L.rows_max, d, f, a->w1, a->b1,
+                                          L.h_packed, w.g_packed, L.C, status, stream);
+      if (e == cudaSuccess)
+        e = enqueue_grouped_gemm_bf16(L.h_packed, L.offsets, E, L.rows_max, f, d, a->w2, a->b2,
+                                      false, L.y_packed, L.C, status, stream);
+      if (e != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    if (dense) {
+      e = enqueue_grouped_gemm_bf16_train(a->x, nullptr, 1, T, d, f, a->dense_w1, a->dense_b1,
+                                          L.h_dense, w.g_dense, T, status, stream);
+      if (e == cudaSuccess)
+        e = enqueue_grouped_gemm_bf16(L.h_dense, nullptr, 1, T, f, d, a->dense_w2, a->dense_b2,
+                                      false, w.r_dense, T, status, stream);
+      if (e != cudaSuccess) return MOE_ERR_CUDA;
+    }
+  } else {
+    if (L.rows_max > 0) {
+      e = enqueue_grouped_gemm_f32((const float*)L.x_packed, L.offsets, E, L.rows_max, d, f,
+                                   (const float*)a->w1, (const float*)a->b1, true,
+                                   (float*)L.h_packed, status, stream, (float*)w.g_packed);
+      if (e == cudaSuccess)
+        e = enqueue_grouped_gemm_f32((const float*)L.h_packed, L.offsets, E, L.rows_max, f, d,
+                                     (const float*)a->w2, (const float*)a->b2, false, L.y_packed,
+                                     status, stream);
+      if (e != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    if (dense) {
+      e = enqueue_grouped_gemm_f32((const float*)a->x, nullptr, 1, T, d, f,
+                                   (const float*)a->dense_w1, (const float*)a->dense_b1, true,
+                                   (float*)L.h_dense, status, stream, (float*)w.g_dense);
+      if (e == cudaSuccess)
+        e = enqueue_grouped_gemm_f32((const float*)L.h_dense, nullptr, 1, T, f, d,
+                                     (const float*)a->dense_w2, (const float*)a->dense_b2, false,
+                                     w.r_dense, status, stream);
+      if (e != cudaSuccess) return MOE_ERR_CUDA;
+    }
+  }
+  e = enqueue_combine(L.y_packed, L.offsets, L.ids, L.slot, L.gates, T, d, E, k, L.rows_max,
+                      a->add_input_residual ? a->x : nullptr, bf16, dense ? w.r_dense : nullptr,
+                      out, a->out_dtype == MOE_BF16, status, stream);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  if (aux) {
+    if ((st = copy_out(aux->logits, L.router.logits, sizeof(float) * T * E, stream)) != MOE_OK ||
+        (st = copy_out(aux->expert_ids, L.ids, sizeof(int32_t) * T * k, stream)) != MOE_OK ||
+        (st = copy_out(aux->gates, L.gates, sizeof(float) * T * k, stream)) != MOE_OK ||
+        (st = copy_out(aux->slot, L.slot, sizeof(int32_t) * T * k, stream)) != MOE_OK ||
+        (st = copy_out(aux->expert_counts, L.counts, sizeof(int32_t) * E, stream)) != MOE_OK ||
+        (st = copy_out(aux->expert_offsets, L.offsets, sizeof(int32_t) * (E + 1), stream)) !=
+            MOE_OK ||
+        (st = copy_out(aux->lb_stats, L.lb_stats, sizeof(float) * (2 * E + 1), stream)) != MOE_OK)
+      return st;
+  }
+  return MOE_OK;
+}
+
+moe_status backward_impl(const moe_layer_args* a, const void* dout, float aux_weight,
+                         float z_weight, moe_layer_grads* g, void* ws, size_t ws_bytes,
+                         cudaStream_t stream) {
+  if (!g) return MOE_ERR_INVALID_ARGUMENT;
+  TrainWs w;
+  size_t need = 0;
+  moe_status st = train_layout(a, (uint8_t*)ws, &w, &need);
+  if (st != MOE_OK) return st;
+  st = check_layer_pointers(a, dout, ws);
+  if (st != MOE_OK) return st;
+  const bool dense = a->dense_w1 != nullptr;
+  if (a->T > 0 && (!g->dx || !g->dw_router || !g->dw1 || !g->dw2)) return MOE_ERR_INVALID_ARGUMENT;
+  if (a->T > 0 && dense && (!g->dense_dw1 || !g->dense_dw2)) return MOE_ERR_INVALID_ARGUMENT;
+  if (!std::isfinite(aux_weight) || !std::isfinite(z_weight)) return MOE_ERR_INVALID_ARGUMENT;
+  if (!aligned16(g->dx) || !aligned16(g->dw_router) || !aligned16(g->db_router) ||
+      !aligned16(g->dw1) || !aligned16(g->db1) || !aligned16(g->dw2) || !aligned16(g->db2) ||
+      !aligned16(g->dense_dw1) || !aligned16(g->dense_db1) || !aligned16(g->dense_dw2) ||
+      !aligned16(g->dense_db2) || !aligned16(g->dgates) || !aligned16(g->dlogits))
+    return MOE_ERR_MISALIGNED;
+  if (ws_bytes < need) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (fault_injected("moe_layer_backward")) return MOE_ERR_CUDA;
+  g_launches = 0;
+  const int64_t T = a->T;
+  const int d = a->d_model, f = a->d_ff, E = a->E, k = a->k;
+  const LayerWs& L = w.L;
+  if (T == 0) return MOE_OK;
+  int* status = (int*)ws;
+  const bool bf16 = a->dtype == MOE_BF16;
+  const int64_t R = L.rows_max;
+  cudaError_t e;
+  auto fail = [&](cudaError_t err) { return err != cudaSuccess; };
+
+  // ---- combine: dgate, dY
+  e = enqueue_combine_backward(dout, bf16, L.y_packed, L.offsets, L.ids, L.slot, L.gates, T, d, E,
+                               k, R, w.dgate, w.dy, status, stream);
+  if (fail(e)) return MOE_ERR_CUDA;
+  if (g->dgates && copy_out(g->dgates, w.dgate, sizeof(float) * T * k, stream) != MOE_OK)
+    return MOE_ERR_CUDA;
+  // ---- router: dl, then dW_r = dl^T x, db_r = column sums of dl, dx_r = dl W_r
+  e = enqueue_router_backward(L.router.logits, L.ids, w.dgate, L.router.scr.acc.c, T, E, k,
+                              a->aux_alpha, aux_weight, z_weight, a->renormalize_gates != 0, w.dl,
+                              stream);
+  if (fail(e)) return MOE_ERR_CUDA;
+  if (g->dlogits && copy_out(g->dlogits, w.dl, sizeof(float) * T * E, stream) != MOE_OK)
+    return MOE_ERR_CUDA;
+  {
+    SimtGemm p;
+    p.M = E; p.N = d; p.K = T;
+    p.a = w.dl; p.a_m = 1; p.a_k = E;
+    p.b = a->x; p.b_bf16 = bf16; p.b_k = d; p.b_n = 1;
+    p.c = w.part_router; p.c_m = d; p.c_n = 1;
+    p.splits = w.splits_r; p.split_stride = (int64_t)E * d;
+    e = enqueue_simt_gemm(p, E, stream);
+    if (fail(e) || fail(enqueue_split_reduce(w.part_router, 1, w.splits_r, (int64_t)E * d,
+                                             g->dw_router, stream)))
+      return MOE_ERR_CUDA;
+    if (g->db_router &&
+        fail(enqueue_colsum(w.dl, false, nullptr, 1, T, E, w.S_d, w.part_colsum, g->db_router, stream)))
+      return MOE_ERR_CUDA;
+    SimtGemm q;
+    q.M = T; q.N = d; q.K = E;
+    q.a = w.dl; q.a_m = E; q.a_k = 1;
+    q.b = a->w_router; q.b_k = d; q.b_n = 1;
+    q.c = w.dx_router; q.c_m = d; q.c_n = 1;
+    if (fail(enqueue_simt_gemm(q, T, stream))) return MOE_ERR_CUDA;
+  }
+  // ---- experts
+  const int64_t m_ext = L.C < T ? L.C : T;  // rows of one expert at most
+  if (R > 0) {
+    if (bf16) {
+      e = enqueue_grouped_gemm_dgrad_bf16(w.dy, L.offsets, E, R, d, f, a->w2, w.g_packed, w.dz,
+                                          L.C, status, stream);
+      if (!fail(e))
+        e = enqueue_grouped_gemm_dgrad_bf16(w.dz, L.offsets, E, R, f, d, a->w1, nullptr, w.dxp,
+                                            L.C, status, stream);
+      if (!fail(e)) e = enqueue_wgrad_bf16(w.dy, L.h_packed, L.offsets, E, R, d, f, g->dw2, status, stream);
+      if (!fail(e)) e = enqueue_wgrad_bf16(w.dz, L.x_packed, L.offsets, E, R, f, d, g->dw1, status, stream);
+      if (fail(e)) return MOE_ERR_CUDA;
+    } else {
+      SimtGemm p;  // dZ = (dY W2[e]) * GeLU'(z)
+      p.M = 0; p.N = f; p.K = d; p.ragged = 1; p.offsets = L.offsets; p.E = E; p.rows_max = R;
+      p.a = w.dy; p.a_m = d; p.a_k = 1;
+      p.b = a->w2; p.b_e = (int64_t)d * f; p.b_k = f; p.b_n = 1;
+      p.c = (float*)w.dz; p.c_m = f; p.c_n = 1;
+      p.mul = w.g_packed;
+      if (fail(enqueue_simt_gemm(p, m_ext, stream))) return MOE_ERR_CUDA;
+      SimtGemm q;  // dX_packed = dZ W1[e]
+      q.N = d; q.K = f; q.ragged = 1; q.offsets = L.offsets; q.E = E; q.rows_max = R;
+      q.a = w.dz; q.a_m = f; q.a_k = 1;
+      q.b = a->w1; q.b_e = (int64_t)f * d; q.b_k = d; q.b_n = 1;
+      q.c = w.dxp; q.c_m = d; q.c_n = 1;
+      if (fail(enqueue_simt_gemm(q, m_ext, stream))) return MOE_ERR_CUDA;
+      SimtGemm r;  // dW2[e] = dY^T h
+      r.M = d; r.N = f; r.ragged = 2; r.offsets = L.offsets; r.E = E; r.rows_max = R;
+      r.a = w.dy; r.a_m = 1; r.a_k = d;
+      r.b = L.h_packed; r.b_k = f; r.b_n = 1;
+      r.c = g->dw2; r.c_e = (int64_t)d * f; r.c_m = f; r.c_n = 1;
+      if (fail(enqueue_simt_gemm(r, d, stream))) return MOE_ERR_CUDA;
+      SimtGemm u;  // dW1[e] = dZ^T x
+      u.M = f; u.N = d; u.ragged = 2; u.offsets = L.offsets; u.E = E; u.rows_max = R;
+      u.a = w.dz; u.a_m = 1; u.a_k = f;
+      u.b = L.x_packed; u.b_k = d; u.b_n = 1;
+      u.c = g->dw1; u.c_e = (int64_t)f * d; u.c_m = d; u.c_n = 1;
+      if (fail(enqueue_simt_gemm(u, f, stream))) return MOE_ERR_CUDA;
+    }
+  } else {
+    if (cudaMemsetAsync(g->dw1, 0, sizeof(float) * E * f * d, stream) != cudaSuccess ||
+        cudaMemsetAsync(g->dw2, 0, sizeof(float) * E * d * f, stream) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+  if (g->db2 && fail(enqueue_colsum(w.dy, bf16, L.offsets, E, R, d, w.S_e, w.part_colsum, g->db2, stream)))
+    return MOE_ERR_CUDA;
+  if (g->db1 && fail(enqueue_colsum(w.dz, bf16, L.offsets, E, R, f, w.S_e, w.part_colsum, g->db1, stream)))
+    return MOE_ERR_CUDA;
+  // ---- dense MLP (one segment of all T rows; its output gradient is dout itself)
+  if (dense) {
+    if (bf16) {
+      e = enqueue_grouped_gemm_dgrad_bf16(dout, nullptr, 1, T, d, f, a->dense_w2, w.g_dense, w.dzd,
+                                          T, status, stream);
+      if (!fail(e))
+        e = enqueue_grouped_gemm_dgrad_bf16(w.dzd, nullptr, 1, T, f, d, a->dense_w1, nullptr, w.dxd,
+                                            T, status, stream);
+      if (!fail(e)) e = enqueue_wgrad_bf16(dout, L.h_dense, nullptr, 1, T, d, f, g->dense_dw2, status, stream);
+      if (!fail(e)) e = enqueue_wgrad_bf16(w.dzd, a->x, nullptr, 1, T, f, d, g->dense_dw1, status, stream);
+      if (fail(e)) return MOE_ERR_CUDA;
+    } else {
+      SimtGemm p;
+      p.N = f; p.K = d; p.ragged = 1; p.E = 1; p.rows_max = T;
+      p.a = dout; p.a_m = d; p.a_k = 1;
+      p.b = a->dense_w2; p.b_k = f; p.b_n = 1;
+      p.c = (float*)w.dzd; p.c_m = f; p.c_n = 1;
+      p.mul = w.g_dense;
+      if (fail(enqueue_simt_gemm(p, T, stream))) return MOE_ERR_CUDA;
+      SimtGemm q;
+      q.N = d; q.K = f; q.ragged = 1; q.E = 1; q.rows_max = T;
+      q.a = w.dzd; q.a_m = f; q.a_k = 1;
+      q.b = a->dense_w1; q.b_k = d; q.b_n = 1;
+      q.c = w.dxd; q.c_m = d; q.c_n = 1;
+      if (fail(enqueue_simt_gemm(q, T, stream))) return MOE_ERR_CUDA;
+      SimtGemm r;
+      r.M = d; r.N = f; r.ragged = 2; r.E = 1; r.rows_max = T;
+      r.a = dout; r.a_m = 1; r.a_k = d;
+      r.b = L.h_dense; r.b_k = f; r.b_n = 1;
+      r.c = g->dense_dw2; r.c_m = f; r.c_n = 1;
+      r.splits = 1;
+      if (fail(enqueue_simt_gemm(r, d, stream))) return MOE_ERR_CUDA;
+      SimtGemm u;
+      u.M = f; u.N = d; u.ragged = 2; u.E = 1; u.rows_max = T;
+      u.a = w.dzd; u.a_m = 1; u.a_k = f;
+      u.b = a->x; u.b_k = d; u.b_n = 1;
+      u.c = g->dense_dw1; u.c_m = d; u.c_n = 1;
+      if (fail(enqueue_simt_gemm(u, f, stream))) return MOE_ERR_CUDA;
+    }
+    if (g->dense_db2 &&
+        fail(enqueue_colsum(dout, bf16, nullptr, 1, T, d, w.S_d, w.part_colsum, g->dense_db2, stream)))
+      return MOE_ERR_CUDA;
+    if (g->dense_db1 &&
+        fail(enqueue_colsum(w.dzd, bf16, nullptr, 1, T, f, w.S_d, w.part_colsum, g->dense_db1, stream)))
+      return MOE_ERR_CUDA;
+  }
+  // ---- dx = [dout] + [dense dx] + packed expert dx rows + router dx
+  e = enqueue_dx_gather(dout, bf16, a->add_input_residual != 0, dense ? w.dxd : nullptr, w.dxp,
+                        L.offsets, L.ids, L.slot, T, d, E, k, R, w.dx_router, g->dx, stream);
+  return fail(e) ? MOE_ERR_CUDA : MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_layer_train_workspace_bytes(const moe_layer_args* args, size_t* bytes) {
+  if (!bytes) return MOE_ERR_INVALID_ARGUMENT;
+  TrainWs w;
+  return train_layout(args, nullptr, &w, bytes);
+}
+
+moe_status moe_layer_forward_train(const moe_layer_args* args, void* out, moe_layer_aux* aux,
+                                   void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (!args) return MOE_ERR_INVALID_ARGUMENT;
+  return forward_train_impl(args, out, aux, ws, ws_bytes, stream);
+}
+
+moe_status moe_layer_backward(const moe_layer_args* args, const void* d_out, float aux_weight,
+                              float z_weight, moe_layer_grads* grads, void* ws, size_t ws_bytes,
+                              moe_stream_t stream) {
+  if (!args) return MOE_ERR_INVALID_ARGUMENT;
+  return backward_impl(args, d_out, aux_weight, z_weight, grads, ws, ws_bytes, stream);
+}
+
 moe_status moe_workspace_reset(void* ws, size_t ws_bytes, moe_stream_t stream) {
   if (!ws || ws_bytes < kAlign) return MOE_ERR_INVALID_ARGUMENT;
   return cuda_status(cudaMemsetAsync(ws, 0, kAlign, stream));

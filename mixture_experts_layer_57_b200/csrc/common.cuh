@@ -35,6 +35,11 @@ __device__ __forceinline__ float gelu_erf(float z) {
   // exact (erf) form of GeLU: z * Phi(z)
   return 0.5f * z * (1.0f + erff(z * 0.70710678118654752440f));
 }
+// d GeLU / dz = Phi(z) + z * phi(z), phi the standard normal density (1 / sqrt(2 pi) e^{-z^2/2})
+__device__ __forceinline__ float gelu_erf_grad(float z) {
+  return 0.5f * (1.0f + erff(z * 0.70710678118654752440f)) +
+         z * 0.39894228040143267794f * expf(-0.5f * z * z);
+}
 
 // ---------------------------------------------------------------- timers
 
@@ -210,10 +215,29 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
   return d;
 }
 
+// Shared-memory matrix descriptor for an MN-major tile written by TMA with 128-byte swizzle in
+// boxes of 64 (MN, contiguous) x 64 (K rows): each K row is 128 bytes of 64 MN-consecutive
+// elements, 8-row groups are 1024 bytes apart (stride byte offset) and the next 64 MN elements
+// start one box (8 KB, leading byte offset) further. One MMA (K = 16) reads two 8-row groups.
+__device__ __forceinline__ uint64_t smem_desc_sw128_mn(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);  // start address, 16-byte units
+  d |= (uint64_t)(8192 >> 4) << 16;           // leading byte offset: next 64 MN elements
+  d |= (uint64_t)(1024 >> 4) << 32;           // stride byte offset: next 8 K rows
+  d |= (uint64_t)1 << 46;                     // descriptor version
+  d |= (uint64_t)2 << 61;                     // layout: 128-byte swizzle
+  return d;
+}
+constexpr uint32_t kMnKStepBytes = 2048;  // K = 16 rows of an MN-major tile
+
 // Instruction descriptor of kind::f16 with bf16 A/B, fp32 D, both operands K-major.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
          ((uint32_t)(M >> 4) << 24);
+}
+// The same with each operand's major-ness: bit 15 = A MN-major, bit 16 = B MN-major.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_major(int M, int N, bool a_mn, bool b_mn) {
+  return idesc_bf16_f32(M, N) | (a_mn ? (1u << 15) : 0u) | (b_mn ? (1u << 16) : 0u);
 }
 
 // ---------------------------------------------------------------- programmatic dependent launch

@@ -16,7 +16,8 @@ template <bool GELU>
 __global__ void __launch_bounds__(kFeat)
     ffn_f32_kernel(const float* __restrict__ X, const int32_t* __restrict__ offsets, int E,
                    int n_out, int K, int64_t rows_max, const float* __restrict__ W,
-                   const float* __restrict__ bias, float* __restrict__ out, int* status) {
+                   const float* __restrict__ bias, float* __restrict__ out, int* status,
+                   float* __restrict__ gout) {
   extern __shared__ float xs[];
   pdl_wait();
   // offsets == nullptr: one segment covering all rows_max rows (dense MLP, E == 1)
@@ -43,7 +44,10 @@ __global__ void __launch_bounds__(kFeat)
       float acc = 0.0f;
       for (int i = 0; i < K; ++i) acc = fmaf(xs[i], w[i], acc);
       float v = acc + (bias ? bias[(int64_t)lo * n_out + f] : 0.0f);
-      if (GELU) v = gelu_erf(v);
+      if (GELU) {
+        if (gout != nullptr) gout[r * n_out + f] = gelu_erf_grad(v);  // saved for the backward
+        v = gelu_erf(v);
+      }
       out[r * n_out + f] = v;
     }
   }
@@ -55,7 +59,7 @@ __global__ void __launch_bounds__(kFeat)
 cudaError_t enqueue_grouped_gemm_f32(const float* x, const int32_t* offsets, int E,
                                      int64_t rows_max, int K, int N, const float* w,
                                      const float* bias, bool gelu, float* out, int* status,
-                                     cudaStream_t stream) {
+                                     cudaStream_t stream, float* gelu_grad_out) {
   if (rows_max == 0) return cudaSuccess;
   const unsigned gx = (unsigned)(rows_max < 65536 ? rows_max : 65536);
   const size_t smem = (size_t)K * sizeof(float);
@@ -68,7 +72,8 @@ cudaError_t enqueue_grouped_gemm_f32(const float* x, const int32_t* offsets, int
   }
   const dim3 grid(gx, (N + kFeat - 1) / kFeat);
   return launch_kernel(gelu ? ffn_f32_kernel<true> : ffn_f32_kernel<false>, grid, dim3(kFeat), smem,
-                       stream, x, offsets, E, N, K, rows_max, w, bias, out, status);
+                       stream, x, offsets, E, N, K, rows_max, w, bias, out, status,
+                       gelu ? gelu_grad_out : nullptr);
 }
 
 cudaError_t enqueue_expert_ffn_f32(const float* x_packed, const int32_t* offsets, int E,

@@ -53,6 +53,10 @@ constexpr int kEpiF32 = 1;       // out = acc + bias (fp32), bias bf16          
 constexpr int kEpiCombineExpert = 2;  // top-1: out[token(r)] = [x] + gate * y[r]
 constexpr int kEpiCombineDense = 3;   // PR-MoE dense MLP, row = token t:
                                       // out[t] = [x] + y_dense[t] + sum_j gate_j * y_expert[row_j]
+// Training.
+constexpr int kEpiGeluGradBf16 = 4;   // out = bf16(acc * g[r, f]), g = GeLU'(z) saved by the
+                                      // forward (backward through layer 2 into layer 1's input)
+constexpr int kEpiGeluBf16Train = 5;  // layer 1 forward that also saves g = bf16(GeLU'(z))
 
 template <int BN>
 struct Cfg {
@@ -97,6 +101,8 @@ struct Params {
   void* out;               // [rows_max, n_out]: bf16 (GeLU layer) or fp32
   int* status;
   CombineArgs cmb;         // used by the combine epilogues only
+  const uint16_t* g_in;    // [rows_max, n_out] bf16 GeLU'(z) (kEpiGeluGradBf16)
+  uint16_t* g_out;         // [rows_max, n_out] bf16 GeLU'(z) (kEpiGeluBf16Train)
 };
 
 struct Tile {
@@ -136,7 +142,9 @@ __device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity, i
   }
 }
 
-template <int BN, int EPI>
+// A_MN: the weight operand is stored [E][K][n_out] (the transpose of the forward layout, as the
+// backward pass reads W1 and W2) and loaded MN-major: two 64-feature x 64-K boxes per stage.
+template <int BN, int EPI, bool A_MN = false>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmW,
                         const __grid_constant__ CUtensorMap tmX, const Params p) {
@@ -251,7 +259,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint32_t sa = base_addr + stage * C::kStageBytes;
           mbar_arrive_expect_tx(full_bar(stage), C::kStageBytes);
-          tma_load_2d(sa, &tmW, kb * kBK, w_row, full_bar(stage));
+          if constexpr (A_MN) {
+            const int k_row = tl.e * p.K + kb * kBK;
+            tma_load_2d(sa, &tmW, tl.f0, k_row, full_bar(stage));
+            tma_load_2d(sa + C::kABytes / 2, &tmW, tl.f0 + 64, k_row, full_bar(stage));
+          } else {
+            tma_load_2d(sa, &tmW, kb * kBK, w_row, full_bar(stage));
+          }
           tma_load_2d(sa + C::kABytes, &tmX, kb * kBK, tl.row0, full_bar(stage));
           ++issued;
           if (++stage == S) {
@@ -279,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
         const int n_mma = max(16, (tl.n_valid + 15) & ~15);
-        const uint32_t idesc = idesc_bf16_f32(kBM, n_mma);
+        const uint32_t idesc = idesc_bf16_f32_major(kBM, n_mma, A_MN, false);
         for (int kb = 0; kb < n_kb; ++kb) {
           if (!mbar_wait_bounded(full_bar(stage), phase, abort_flag, p.status)) {
             ok = false;
@@ -287,12 +301,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const uint32_t sa = base_addr + stage * C::kStageBytes;
-          const uint64_t adesc = smem_desc_sw128(sa);
+          const uint64_t adesc = A_MN ? smem_desc_sw128_mn(sa) : smem_desc_sw128(sa);
           const uint64_t bdesc = smem_desc_sw128(sa + C::kABytes);
+          // K step: +32 bytes inside a K-major 128-byte row (+2 in the 16-byte address field),
+          // or two 8-row groups of an MN-major tile
+          constexpr uint64_t a_step = A_MN ? (kMnKStepBytes >> 4) : 2;
 #pragma unroll
           for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
-            // +32 bytes along K inside the swizzled 128-byte row = +2 in the 16-byte address field
-            tc_mma_bf16(d_tmem, adesc + (uint64_t)(2 * kk), bdesc + (uint64_t)(2 * kk), idesc,
+            tc_mma_bf16(d_tmem, adesc + a_step * (uint64_t)kk, bdesc + (uint64_t)(2 * kk), idesc,
                         (kb | kk) != 0 ? 1u : 0u);
           }
           tc_commit(empty_bar(stage));
@@ -336,11 +352,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_32x32b_x16(taddr + (uint32_t)c0, r);
         tmem_ld_wait();
         const int nc = min(16, tl.n_valid - c0);
-        if constexpr (EPI == kEpiGeluBf16) {
+        if constexpr (EPI == kEpiGeluBf16 || EPI == kEpiGeluBf16Train || EPI == kEpiGeluGradBf16) {
           // stage [16 tokens][32 features] bf16, then 16-byte stores of 8 features of one token
           uint16_t* s16 = reinterpret_cast<uint16_t*>(st);
+          if constexpr (EPI == kEpiGeluGradBf16) {
+            // dZ = dH * GeLU'(z) of the same (row, feature)
 #pragma unroll
-          for (int c = 0; c < 16; ++c) s16[c * 32 + lane] = f32_to_bf16_rn(gelu_erf(__uint_as_float(r[c]) + bv));
+            for (int c = 0; c < 16; ++c) {
+              const float g = (c < nc && f_ok)
+                                  ? bf16_to_f32(p.g_in[(int64_t)(tl.row0 + c0 + c) * p.n_out + f])
+                                  : 0.0f;
+              s16[c * 32 + lane] = f32_to_bf16_rn(__uint_as_float(r[c]) * g);
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const float z = __uint_as_float(r[c]) + bv;
+              s16[c * 32 + lane] = f32_to_bf16_rn(gelu_erf(z));
+              if constexpr (EPI == kEpiGeluBf16Train) {
+                if (c < nc && f_ok)
+                  p.g_out[(int64_t)(tl.row0 + c0 + c) * p.n_out + f] = f32_to_bf16_rn(gelu_erf_grad(z));
+              }
+            }
+          }
           __syncwarp();
 #pragma unroll
           for (int id = lane; id < 64; id += 32) {
@@ -492,10 +526,23 @@ bool make_kmajor_map(CUtensorMap* m, const void* ptr, int64_t rows, int K, int b
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, int EPI>
+// MN-major bf16 matrix [rows, cols] (row stride cols elements) read in boxes of 64 x 64.
+bool make_mn_map(CUtensorMap* m, const void* ptr, int64_t rows, int cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t gstride[1] = {(cuuint64_t)cols * 2};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t estride[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), gdim, gstride, box,
+            estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, int EPI, bool A_MN = false>
 cudaError_t launch_one(const CUtensorMap& tmW, const CUtensorMap& tmX, const Params& p,
                        cudaStream_t stream) {
-  auto kern = grouped_gemm_kernel<BN, EPI>;
+  auto kern = grouped_gemm_kernel<BN, EPI, A_MN>;
   static bool attr_set = false;  // per instantiation
   if (!attr_set) {
     cudaError_t e =
@@ -508,6 +555,19 @@ cudaError_t launch_one(const CUtensorMap& tmW, const CUtensorMap& tmX, const Par
 
 }  // namespace
 
+bool make_bf16_map_2d(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols, int box_cols,
+                      int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t gstride[1] = {(cuuint64_t)cols * 2};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+  cuuint32_t estride[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), gdim, gstride, box,
+            estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 static int pick_token_tile(int64_t capacity_hint) {
   if (capacity_hint <= 16) return 16;
   if (capacity_hint <= 32) return 32;
@@ -516,15 +576,15 @@ static int pick_token_tile(int64_t capacity_hint) {
   return 256;
 }
 
-template <int EPI>
+template <int EPI, bool A_MN = false>
 cudaError_t launch_bn(int BN, const CUtensorMap& tmW, const CUtensorMap& tmX, const Params& p,
                       cudaStream_t stream) {
   switch (BN) {
-    case 16: return launch_one<16, EPI>(tmW, tmX, p, stream);
-    case 32: return launch_one<32, EPI>(tmW, tmX, p, stream);
-    case 64: return launch_one<64, EPI>(tmW, tmX, p, stream);
-    case 128: return launch_one<128, EPI>(tmW, tmX, p, stream);
-    default: return launch_one<256, EPI>(tmW, tmX, p, stream);
+    case 16: return launch_one<16, EPI, A_MN>(tmW, tmX, p, stream);
+    case 32: return launch_one<32, EPI, A_MN>(tmW, tmX, p, stream);
+    case 64: return launch_one<64, EPI, A_MN>(tmW, tmX, p, stream);
+    case 128: return launch_one<128, EPI, A_MN>(tmW, tmX, p, stream);
+    default: return launch_one<256, EPI, A_MN>(tmW, tmX, p, stream);
   }
 }
 
@@ -537,9 +597,39 @@ cudaError_t enqueue_grouped_gemm_bf16(const void* x, const int32_t* offsets, int
   CUtensorMap tmW, tmX;
   if (!make_kmajor_map(&tmW, w, (int64_t)E * N, K, kBM) || !make_kmajor_map(&tmX, x, rows_max, K, BN))
     return cudaErrorInvalidValue;
-  Params p{offsets, E, N, K, rows_max, bias, out, status, CombineArgs{}};
+  Params p{offsets, E, N, K, rows_max, bias, out, status, CombineArgs{}, nullptr, nullptr};
   return gelu ? launch_bn<kEpiGeluBf16>(BN, tmW, tmX, p, stream)
               : launch_bn<kEpiF32>(BN, tmW, tmX, p, stream);
+}
+
+cudaError_t enqueue_grouped_gemm_bf16_train(const void* x, const int32_t* offsets, int E,
+                                            int64_t rows_max, int K, int N, const void* w,
+                                            const void* bias, void* h_out, void* g_out,
+                                            int64_t capacity_hint, int* status,
+                                            cudaStream_t stream) {
+  if (rows_max == 0) return cudaSuccess;
+  const int BN = pick_token_tile(capacity_hint);
+  CUtensorMap tmW, tmX;
+  if (!make_kmajor_map(&tmW, w, (int64_t)E * N, K, kBM) || !make_kmajor_map(&tmX, x, rows_max, K, BN))
+    return cudaErrorInvalidValue;
+  Params p{offsets, E, N, K, rows_max, bias, h_out, status, CombineArgs{}, nullptr,
+           (uint16_t*)g_out};
+  return launch_bn<kEpiGeluBf16Train>(BN, tmW, tmX, p, stream);
+}
+
+cudaError_t enqueue_grouped_gemm_dgrad_bf16(const void* dy, const int32_t* offsets, int E,
+                                            int64_t rows_max, int K, int N, const void* w_t,
+                                            const void* g_in, void* out, int64_t capacity_hint,
+                                            int* status, cudaStream_t stream) {
+  if (rows_max == 0) return cudaSuccess;
+  const int BN = pick_token_tile(capacity_hint);
+  CUtensorMap tmW, tmX;
+  if (!make_mn_map(&tmW, w_t, (int64_t)E * K, N) || !make_kmajor_map(&tmX, dy, rows_max, K, BN))
+    return cudaErrorInvalidValue;
+  Params p{offsets, E, N, K, rows_max, nullptr, out, status, CombineArgs{},
+           (const uint16_t*)g_in, nullptr};
+  return g_in != nullptr ? launch_bn<kEpiGeluGradBf16, true>(BN, tmW, tmX, p, stream)
+                         : launch_bn<kEpiF32, true>(BN, tmW, tmX, p, stream);
 }
 
 cudaError_t enqueue_gemm2_combine(const void* h, const int32_t* offsets, int E, int64_t rows_max,
@@ -554,7 +644,7 @@ cudaError_t enqueue_gemm2_combine(const void* h, const int32_t* offsets, int E, 
   CombineArgs c{fc.row_token, fc.slot, fc.ids, fc.offsets, fc.gates, fc.y,
                 (const uint16_t*)fc.residual, fc.out, fc.out_bf16 ? 1 : 0, fc.k, fc.E_experts,
                 fc.rows_y};
-  Params p{offsets, E, N, K, rows_max, bias, nullptr, status, c};
+  Params p{offsets, E, N, K, rows_max, bias, nullptr, status, c, nullptr, nullptr};
   return fc.dense ? launch_bn<kEpiCombineDense>(BN, tmW, tmX, p, stream)
                   : launch_bn<kEpiCombineExpert>(BN, tmW, tmX, p, stream);
 }

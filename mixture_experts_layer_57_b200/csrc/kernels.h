@@ -138,14 +138,39 @@ cudaError_t enqueue_dispatch(const void* x, bool bf16, int64_t T, int d, const i
 // One grouped GEMM layer: out = act(W[e] x + bias[e]) over every expert segment. offsets ==
 // nullptr means one segment [0, rows_max) (E must be 1). gelu: GeLU epilogue with output in the
 // input type; otherwise bias only with fp32 output.
+// A bf16 tensor map over a row-major [rows, cols] matrix, boxes of box_cols x box_rows,
+// 128-byte swizzle, out-of-range elements read as zero.
+bool make_bf16_map_2d(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols, int box_cols,
+                      int box_rows);
+// Weight-gradient GEMM (tcgen05): for every expert e,
+//     out[e][m][n] = sum over the rows r of segment e of a[r][m] * b[r][n]    (fp32, overwritten)
+// a [rows_max, M] and b [rows_max, N] bf16, token-major; offsets == nullptr: one segment
+// [0, rows_max) (E == 1). Experts without rows get zeros.
+cudaError_t enqueue_wgrad_bf16(const void* a, const void* b, const int32_t* offsets, int E,
+                               int64_t rows_max, int M, int N, float* out, int* status,
+                               cudaStream_t stream);
+// Layer 1 for training: h = bf16(GeLU(W x + b)) and g = bf16(GeLU'(W x + b)), both [rows, N].
+cudaError_t enqueue_grouped_gemm_bf16_train(const void* x, const int32_t* offsets, int E,
+                                            int64_t rows_max, int K, int N, const void* w,
+                                            const void* bias, void* h_out, void* g_out,
+                                            int64_t capacity_hint, int* status,
+                                            cudaStream_t stream);
+// Backward data GEMM: out[r, n] = sum_k w_t[e][k][n] * dy[r, k] for the rows of expert e, with
+// w_t the weight stored [E][K][N] (W1 [E][d_ff][d] gives dx = dz W1; W2 [E][d][d_ff] gives
+// dh = dy W2). g_in (bf16 [rows, N]) given: out = bf16(result * g_in), else out fp32.
+cudaError_t enqueue_grouped_gemm_dgrad_bf16(const void* dy, const int32_t* offsets, int E,
+                                            int64_t rows_max, int K, int N, const void* w_t,
+                                            const void* g_in, void* out, int64_t capacity_hint,
+                                            int* status, cudaStream_t stream);
 cudaError_t enqueue_grouped_gemm_bf16(const void* x, const int32_t* offsets, int E,
                                       int64_t rows_max, int K, int N, const void* w,
                                       const void* bias, bool gelu, void* out,
                                       int64_t capacity_hint, int* status, cudaStream_t stream);
+// gelu_grad_out (optional, GeLU layer): also writes GeLU'(z) for the backward pass.
 cudaError_t enqueue_grouped_gemm_f32(const float* x, const int32_t* offsets, int E,
                                      int64_t rows_max, int K, int N, const float* w,
                                      const float* bias, bool gelu, float* out, int* status,
-                                     cudaStream_t stream);
+                                     cudaStream_t stream, float* gelu_grad_out = nullptr);
 // Layer 2 with the combine fused into its epilogue (bf16 layers):
 //   dense == false: top-1 experts; row r of the packed buffer belongs to token row_token[r]:
 //                   out[t] = [residual[t]] + gates[t] * (W2[e] h[r] + b2[e])
@@ -188,5 +213,58 @@ cudaError_t enqueue_combine(const float* y_packed, const int32_t* offsets, const
                             int k, int64_t rows_max, const void* residual, bool res_bf16,
                             const float* dense, void* out, bool out_bf16, int* status,
                             cudaStream_t stream);
+
+// ---------------------------------------------------------------- backward
+cudaError_t enqueue_combine_backward(const void* dout, bool bf16, const float* y_packed,
+                                     const int32_t* offsets, const int32_t* ids,
+                                     const int32_t* slot, const float* gates, int64_t T, int d,
+                                     int E, int k, int64_t rows_max, float* dgate, void* dy,
+                                     int* status, cudaStream_t stream);
+// first_counts: the forward's first-choice counts per expert (f_e * T).
+cudaError_t enqueue_router_backward(const float* logits, const int32_t* ids, const float* dgate,
+                                    const unsigned* first_counts, int64_t T, int E, int k,
+                                    float alpha, float aux_weight, float z_weight,
+                                    bool renormalize, float* dl, cudaStream_t stream);
+// Row splits for a column sum over segments of at most longest_segment rows.
+int colsum_splits(int64_t longest_segment);
+// out[e][n] = sum of X[r][n] over segment e (offsets == nullptr: one segment of rows_max rows);
+// S > 1 needs partial [E * S * N].
+cudaError_t enqueue_colsum(const void* X, bool bf16, const int32_t* offsets, int E,
+                           int64_t rows_max, int N, int S, float* partial, float* out,
+                           cudaStream_t stream);
+cudaError_t enqueue_split_reduce(const float* part, int64_t groups, int S, int64_t N, float* out,
+                                 cudaStream_t stream);
+cudaError_t enqueue_dx_gather(const void* dout, bool bf16, bool add_dout, const float* dense_dx,
+                              const float* dxp, const int32_t* offsets, const int32_t* ids,
+                              const int32_t* slot, int64_t T, int d, int E, int k,
+                              int64_t rows_max, const float* dx_router, void* dx,
+                              cudaStream_t stream);
+// fp32 FMA GEMM C(m, n) = sum_k A(m, k) B(k, n) per expert e (blockIdx.z = e * splits + s):
+// A(m, k) at a[e * a_e + m * a_m + k * a_k] (bf16 or fp32), B(k, n) at b[e * b_e + k * b_k +
+// n * b_n], C at c (fp32) or c16 (bf16) [e * c_e + s * split_stride + m * c_m + n * c_n], times
+// mul at the same index when given. ragged = 1: M is the rows of segment e and the m index of A
+// and C is offset by the segment start; ragged = 2: the same for K and the k index of A and B.
+struct SimtGemm {
+  int64_t M = 0, N = 0, K = 0;
+  int ragged = 0;
+  const int32_t* offsets = nullptr;
+  int E = 1;
+  int64_t rows_max = 0;
+  const void* a = nullptr;
+  int a_bf16 = 0;
+  int64_t a_e = 0, a_m = 0, a_k = 0;
+  const void* b = nullptr;
+  int b_bf16 = 0;
+  int64_t b_e = 0, b_k = 0, b_n = 0;
+  float* c = nullptr;
+  uint16_t* c16 = nullptr;
+  int64_t c_e = 0, c_m = 0, c_n = 0;
+  const void* mul = nullptr;
+  int mul_bf16 = 0;
+  int splits = 1;
+  int64_t split_stride = 0;
+};
+// m_extent: the largest M over the experts (grid rows).
+cudaError_t enqueue_simt_gemm(const SimtGemm& p, int64_t m_extent, cudaStream_t stream);
 
 }  // namespace moe

@@ -55,6 +55,12 @@ class LayerAux(ctypes.Structure):
                 ("lb_stats", ctypes.c_void_p), ("router_losses", ctypes.c_void_p)]
 
 
+class LayerGrads(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "dx", "dw_router", "db_router", "dw1", "db1", "dw2", "db2", "dense_dw1", "dense_db1",
+        "dense_dw2", "dense_db2", "dgates", "dlogits")]
+
+
 _lib = None
 
 
@@ -98,6 +104,9 @@ def lib() -> ctypes.CDLL:
             "moe_layer_forward_shard_begin": ([P(LayerArgs), i64, P(LayerAux), vp, vp, vp, sz, vp], i32),
             "moe_layer_forward_shard_end": ([P(LayerArgs), i64, i32, i32, vp, vp, vp, P(LayerAux), vp,
                                              sz, vp], i32),
+            "moe_layer_train_workspace_bytes": ([P(LayerArgs), P(sz)], i32),
+            "moe_layer_forward_train": ([P(LayerArgs), vp, P(LayerAux), vp, sz, vp], i32),
+            "moe_layer_backward": ([P(LayerArgs), vp, f32, f32, P(LayerGrads), vp, sz, vp], i32),
             "moe_workspace_reset": ([vp, sz, vp], i32),
             "moe_get_device_error": ([vp, P(i32), vp], i32),
         }
@@ -492,6 +501,37 @@ def moe_layer_forward_sharded(args: LayerArgs, T_global: int, out: torch.Tensor,
         return moe_layer_forward_shard_end(args, T_global, dist.get_world_size(group),
                                            dist.get_rank(group), demand_all, totals, out, ws,
                                            aux=aux, stream=s)
+
+
+def moe_layer_train_workspace_bytes(args: LayerArgs) -> int:
+    out = ctypes.c_size_t()
+    _check("moe_layer_train_workspace_bytes",
+           lib().moe_layer_train_workspace_bytes(ctypes.byref(args), ctypes.byref(out)))
+    return out.value
+
+
+def moe_layer_forward_train(args: LayerArgs, out: torch.Tensor, aux: Optional[dict] = None,
+                            ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Forward pass that keeps the backward pass's state in the returned workspace."""
+    if ws is None:
+        ws = workspace(moe_layer_train_workspace_bytes(args), out.device)
+    _check("moe_layer_forward_train", lib().moe_layer_forward_train(
+        ctypes.byref(args), _ptr(out), ctypes.byref(_aux_struct(aux)), _ptr(ws), ws.numel(),
+        _stream(stream)))
+    return ws
+
+
+def moe_layer_backward(args: LayerArgs, d_out: torch.Tensor, grads: dict, ws: torch.Tensor,
+                       aux_weight: float = 0.0, z_weight: float = 0.0, stream=None) -> dict:
+    """Backward pass after moe_layer_forward_train with the same args and workspace. ``grads``
+    maps moe_layer_grads field names to output tensors."""
+    g = LayerGrads()
+    for name, t in grads.items():
+        setattr(g, name, _ptr(t))
+    _check("moe_layer_backward", lib().moe_layer_backward(
+        ctypes.byref(args), _ptr(d_out), aux_weight, z_weight, ctypes.byref(g), _ptr(ws),
+        ws.numel(), _stream(stream)))
+    return grads
 
 
 def moe_workspace_reset(ws: torch.Tensor, stream=None):
