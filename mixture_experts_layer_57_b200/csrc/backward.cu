@@ -180,22 +180,83 @@ __global__ void __launch_bounds__(256)
   pdl_trigger();
 }
 
-// out[g * N + n] = sum_{s < S} part[(g * S + s) * N + n], s ascending.
+// out[g * N + n] = sum_{s < S} part[(g * S + s) * N_stride + n], s ascending (N <= N_stride).
 __global__ void __launch_bounds__(256)
     split_reduce_kernel(const float* __restrict__ part, int64_t groups, int S, int64_t N,
-                        float* __restrict__ out) {
+                        int64_t N_stride, float* __restrict__ out) {
   pdl_wait();
   const int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x;
   if (i < groups * N) {
     const int64_t g = i / N, n = i - g * N;
     float acc = 0.0f;
-    for (int s = 0; s < S; ++s) acc += part[(g * S + s) * N + n];
+    for (int s = 0; s < S; ++s) acc += part[(g * S + s) * N_stride + n];
     out[i] = acc;
   }
   pdl_trigger();
 }
 
-template <bool BF16>
+// Exact three-way bf16 split v = hi + mid + lo (each part the next 8 significant bits).
+__device__ __forceinline__ void split3(float v, uint16_t* hi, uint16_t* mid, uint16_t* lo) {
+  *hi = f32_to_bf16_rn(v);
+  const float r1 = v - bf16_to_f32(*hi);
+  *mid = f32_to_bf16_rn(r1);
+  *lo = f32_to_bf16_rn(r1 - bf16_to_f32(*mid));
+}
+
+// The router's backward GEMMs on tensor cores from bf16 parts of fp32 operands:
+//   dl3 [3 Tpad, Epad]: rows p * Tpad + t hold part p (hi, mid, lo) of dl[t, :]; padding zero
+//     (dW_r = sum_p part_p^T x: x is bf16, so the three products are exact and the sum is fp32-
+//     accurate);
+//   dlx [T, Kx]: columns [dl_hi | dl_mid | dl_hi | 0], wx [Kx, d]: rows [W_hi; W_hi; W_mid; 0]
+//     (dx_r = dl W_r as W_hi dl_hi + W_hi dl_mid + W_mid dl_hi: 16 significant bits of each
+//     operand, for a dx that is returned in bf16).
+__global__ void __launch_bounds__(256)
+    router_bwd_split_kernel(const float* __restrict__ dl, int64_t T, int64_t Tpad, int E,
+                            int Epad, int Kx, uint16_t* __restrict__ dl3,
+                            uint16_t* __restrict__ dlx) {
+  pdl_wait();
+  const int64_t n = Tpad * Epad;
+  for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < n; i += (int64_t)gridDim.x * 256) {
+    const int64_t t = i / Epad;
+    const int e = (int)(i - t * Epad);
+    const float v = (t < T && e < E) ? dl[t * E + e] : 0.0f;
+    uint16_t hi, mid, lo;
+    split3(v, &hi, &mid, &lo);
+    dl3[t * Epad + e] = hi;
+    dl3[(Tpad + t) * Epad + e] = mid;
+    dl3[(2 * Tpad + t) * Epad + e] = lo;
+    if (t < T) {
+      if (e < E) {
+        dlx[t * Kx + e] = hi;
+        dlx[t * Kx + E + e] = mid;
+        dlx[t * Kx + 2 * E + e] = hi;
+      }
+      for (int c = 3 * E + e; c < Kx; c += Epad) dlx[t * Kx + c] = 0;  // padding columns
+    }
+  }
+  pdl_trigger();
+}
+
+__global__ void __launch_bounds__(256)
+    router_w_split_kernel(const float* __restrict__ w, int E, int d, int Kx,
+                          uint16_t* __restrict__ wx) {
+  pdl_wait();
+  const int64_t n = (int64_t)Kx * d;
+  for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < n; i += (int64_t)gridDim.x * 256) {
+    const int r = (int)(i / d), c = (int)(i - (int64_t)r * d);
+    const int part = r / E, e = r - part * E;
+    uint16_t v = 0;
+    if (part < 3) {
+      uint16_t hi, mid, lo;
+      split3(w[(int64_t)e * d + c], &hi, &mid, &lo);
+      v = part == 2 ? mid : hi;
+    }
+    wx[i] = v;
+  }
+  pdl_trigger();
+}
+
+template <bool BF16, int VEC>
 __global__ void __launch_bounds__(256)
     dx_gather_kernel(const void* __restrict__ dout, int add_dout, const float* __restrict__ dense_dx,
                      const float* __restrict__ dxp, const int32_t* __restrict__ offsets,
@@ -215,12 +276,28 @@ __global__ void __launch_bounds__(256)
       const int64_t r = (int64_t)offsets[e] + s;
       if (r < rows_max) rows[nk++] = r;
     }
-    for (int c = lane; c < d; c += 32) {
-      float acc = add_dout ? ld_any<BF16>(dout, t * d + c) : 0.0f;
-      if (dense_dx) acc += dense_dx[t * d + c];
-      for (int j = 0; j < nk; ++j) acc += dxp[rows[j] * d + c];
-      if (dx_router) acc += dx_router[t * d + c];
-      st_any<BF16>(dx, t * d + c, acc);
+    for (int c = lane * VEC; c < d; c += 32 * VEC) {
+      float acc[VEC];
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) acc[v] = 0.0f;
+      auto add4 = [&](const float* src) {
+        if constexpr (VEC == 4) {
+          const float4 q = *reinterpret_cast<const float4*>(src);
+          acc[0] += q.x; acc[1] += q.y; acc[2] += q.z; acc[3] += q.w;
+        } else {
+#pragma unroll
+          for (int v = 0; v < VEC; ++v) acc[v] += src[v];
+        }
+      };
+      if (add_dout) {
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) acc[v] = ld_any<BF16>(dout, t * d + c + v);
+      }
+      if (dense_dx) add4(dense_dx + t * d + c);
+      for (int j = 0; j < nk; ++j) add4(dxp + rows[j] * d + c);
+      if (dx_router) add4(dx_router + t * d + c);
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) st_any<BF16>(dx, t * d + c + v, acc[v]);
     }
   }
   pdl_trigger();
@@ -357,11 +434,25 @@ cudaError_t enqueue_colsum(const void* X, bool bf16, const int32_t* offsets, int
 }
 
 cudaError_t enqueue_split_reduce(const float* part, int64_t groups, int S, int64_t N, float* out,
-                                 cudaStream_t stream) {
+                                 cudaStream_t stream, int64_t N_stride) {
   const int64_t n = groups * N;
   if (n == 0) return cudaSuccess;
   return launch_kernel(split_reduce_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0,
-                       stream, part, groups, S, N, out);
+                       stream, part, groups, S, N, N_stride > 0 ? N_stride : N, out);
+}
+
+cudaError_t enqueue_router_bwd_split(const float* dl, int64_t T, int64_t Tpad, int E, int Epad,
+                                     int Kx, uint16_t* dl3, uint16_t* dlx, const float* w_router,
+                                     int d, uint16_t* wx, cudaStream_t stream) {
+  const int64_t n = Tpad * Epad;
+  const unsigned blocks = (unsigned)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+  cudaError_t e = launch_kernel(router_bwd_split_kernel, dim3(blocks), dim3(256), 0, stream, dl,
+                                T, Tpad, E, Epad, Kx, dl3, dlx);
+  if (e != cudaSuccess) return e;
+  const int64_t nw = (int64_t)Kx * d;
+  const unsigned bw = (unsigned)((nw + 255) / 256 < 4096 ? (nw + 255) / 256 : 4096);
+  return launch_kernel(router_w_split_kernel, dim3(bw), dim3(256), 0, stream, w_router, E, d, Kx,
+                       wx);
 }
 
 cudaError_t enqueue_dx_gather(const void* dout, bool bf16, bool add_dout, const float* dense_dx,
@@ -372,11 +463,12 @@ cudaError_t enqueue_dx_gather(const void* dout, bool bf16, bool add_dout, const 
   if (T == 0) return cudaSuccess;
   const dim3 grid((unsigned)((T * 32 + 255) / 256));
   const int ad = add_dout ? 1 : 0;
-  return bf16 ? launch_kernel(dx_gather_kernel<true>, grid, dim3(256), 0, stream, dout, ad,
-                              dense_dx, dxp, offsets, ids, slot, T, d, E, k, rows_max, dx_router, dx)
-              : launch_kernel(dx_gather_kernel<false>, grid, dim3(256), 0, stream, dout, ad,
-                              dense_dx, dxp, offsets, ids, slot, T, d, E, k, rows_max, dx_router,
-                              dx);
+  auto go = [&](auto kern) {
+    return launch_kernel(kern, grid, dim3(256), 0, stream, dout, ad, dense_dx, dxp, offsets, ids,
+                         slot, T, d, E, k, rows_max, dx_router, dx);
+  };
+  if (d % 4 == 0) return bf16 ? go(dx_gather_kernel<true, 4>) : go(dx_gather_kernel<false, 4>);
+  return bf16 ? go(dx_gather_kernel<true, 1>) : go(dx_gather_kernel<false, 1>);
 }
 
 cudaError_t enqueue_simt_gemm(const SimtGemm& p, int64_t m_extent, cudaStream_t stream) {

@@ -1,5 +1,6 @@
 // C ABI of the MoE-layer forward pass: argument validation, workspace layout, fault injection
 // and launch accounting around the kernels' enqueue functions. See include/moe.h.
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
@@ -812,7 +813,11 @@ struct TrainWs {
   float* dxd;          // [T, d]
   float* part_colsum;
   float* part_router;
-  int S_e, S_d, splits_r;
+  int S_e, S_d, S_rb, splits_r;
+  // bf16 layers: the router's backward GEMMs on tensor cores
+  int64_t Tpad;
+  int Epad, Kx, S_rt;
+  uint16_t *dl3, *dlx, *wx;
 };
 
 int router_wgrad_splits(int64_t T) {
@@ -844,13 +849,33 @@ moe_status train_layout(const moe_layer_args* a, uint8_t* base, TrainWs* w, size
   const int64_t seg = w->L.C < T ? w->L.C : T;
   w->S_e = colsum_splits(seg);
   w->S_d = colsum_splits(T);
+  w->S_rb = (int)std::min<int64_t>(256, std::max<int64_t>(1, (T + 127) / 128));
   const int64_t wide = d > f ? d : f;
   int64_t pc = (int64_t)E * w->S_e * wide;
   if ((int64_t)w->S_d * wide > pc) pc = (int64_t)w->S_d * wide;
-  if ((int64_t)w->S_d * E > pc) pc = (int64_t)w->S_d * E;
+  if ((int64_t)w->S_rb * E > pc) pc = (int64_t)w->S_rb * E;
   w->part_colsum = c.take<float>((size_t)pc);
   w->splits_r = router_wgrad_splits(T);
-  w->part_router = c.take<float>((size_t)w->splits_r * E * d);
+  w->Tpad = (T + 63) / 64 * 64;
+  w->Epad = (E + 7) / 8 * 8;
+  w->Kx = (3 * E + 7) / 8 * 8;
+  {
+    // split-K of dW_r = dl^T x over the three stacked parts: about one tile per SM
+    const int bn = d <= 64 ? 64 : (d <= 128 ? 128 : 256);
+    const int64_t tiles = (int64_t)((w->Epad + 127) / 128) * ((d + bn - 1) / bn);
+    const int64_t n_kb = 3 * w->Tpad / 64;
+    int64_t s = (148 + tiles - 1) / tiles;
+    if (s > 64) s = 64;
+    if (s > n_kb) s = n_kb;
+    w->S_rt = (int)(s < 1 ? 1 : s);
+  }
+  const bool bf16 = a->dtype == MOE_BF16;
+  int64_t pr = (int64_t)w->splits_r * E * d;
+  if (bf16 && (int64_t)w->S_rt * w->Epad * d > pr) pr = (int64_t)w->S_rt * w->Epad * d;
+  w->part_router = c.take<float>((size_t)pr);
+  w->dl3 = bf16 ? c.take<uint16_t>((size_t)3 * w->Tpad * w->Epad) : nullptr;
+  w->dlx = bf16 ? c.take<uint16_t>((size_t)T * w->Kx) : nullptr;
+  w->wx = bf16 ? c.take<uint16_t>((size_t)w->Kx * d) : nullptr;
   *bytes = c.off;
   return MOE_OK;
 }
@@ -1021,19 +1046,34 @@ moe_status backward_impl(const moe_layer_args* a, const void* dout, float aux_we
   if (fail(e)) return MOE_ERR_CUDA;
   if (g->dlogits && copy_out(g->dlogits, w.dl, sizeof(float) * T * E, stream) != MOE_OK)
     return MOE_ERR_CUDA;
-  {
+  if (g->db_router &&
+      fail(enqueue_colsum(w.dl, false, nullptr, 1, T, E, w.S_rb, w.part_colsum, g->db_router, stream)))
+    return MOE_ERR_CUDA;
+  if (bf16) {
+    // tensor cores on bf16 parts: dW_r = sum of the three stacked parts^T x (split-K),
+    // dx_r = [dl_hi | dl_mid | dl_hi] [W_hi; W_hi; W_mid]
+    e = enqueue_router_bwd_split(w.dl, T, w.Tpad, E, w.Epad, w.Kx, w.dl3, w.dlx, a->w_router, d,
+                                 w.wx, stream);
+    if (!fail(e))
+      e = enqueue_wgrad_bf16(w.dl3, a->x, nullptr, 1, 3 * w.Tpad, w.Epad, d, w.part_router, status,
+                             stream, w.S_rt, w.Tpad, T);
+    if (!fail(e))
+      e = enqueue_split_reduce(w.part_router, 1, w.S_rt, (int64_t)E * d, g->dw_router, stream,
+                               (int64_t)w.Epad * d);
+    if (!fail(e))
+      e = enqueue_grouped_gemm_dgrad_bf16(w.dlx, nullptr, 1, T, w.Kx, d, w.wx, nullptr,
+                                          w.dx_router, T, status, stream);
+    if (fail(e)) return MOE_ERR_CUDA;
+  } else {
     SimtGemm p;
     p.M = E; p.N = d; p.K = T;
     p.a = w.dl; p.a_m = 1; p.a_k = E;
-    p.b = a->x; p.b_bf16 = bf16; p.b_k = d; p.b_n = 1;
+    p.b = a->x; p.b_k = d; p.b_n = 1;
     p.c = w.part_router; p.c_m = d; p.c_n = 1;
     p.splits = w.splits_r; p.split_stride = (int64_t)E * d;
     e = enqueue_simt_gemm(p, E, stream);
     if (fail(e) || fail(enqueue_split_reduce(w.part_router, 1, w.splits_r, (int64_t)E * d,
                                              g->dw_router, stream)))
-      return MOE_ERR_CUDA;
-    if (g->db_router &&
-        fail(enqueue_colsum(w.dl, false, nullptr, 1, T, E, w.S_d, w.part_colsum, g->db_router, stream)))
       return MOE_ERR_CUDA;
     SimtGemm q;
     q.M = T; q.N = d; q.K = E;

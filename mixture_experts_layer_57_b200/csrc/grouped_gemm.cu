@@ -352,30 +352,57 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_32x32b_x16(taddr + (uint32_t)c0, r);
         tmem_ld_wait();
         const int nc = min(16, tl.n_valid - c0);
-        if constexpr (EPI == kEpiGeluBf16 || EPI == kEpiGeluBf16Train || EPI == kEpiGeluGradBf16) {
-          // stage [16 tokens][32 features] bf16, then 16-byte stores of 8 features of one token
-          uint16_t* s16 = reinterpret_cast<uint16_t*>(st);
-          if constexpr (EPI == kEpiGeluGradBf16) {
-            // dZ = dH * GeLU'(z) of the same (row, feature)
+        if constexpr (EPI == kEpiGeluGradBf16) {
+          // dZ = dH * GeLU'(z): stage dH [16 tokens][32 features] fp32, then each lane takes 8
+          // features of one token: 16-byte loads of GeLU'(z) and 16-byte stores of dZ
+          float* s32 = reinterpret_cast<float*>(st);
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              const float g = (c < nc && f_ok)
-                                  ? bf16_to_f32(p.g_in[(int64_t)(tl.row0 + c0 + c) * p.n_out + f])
-                                  : 0.0f;
-              s16[c * 32 + lane] = f32_to_bf16_rn(__uint_as_float(r[c]) * g);
-            }
-          } else {
+          for (int c = 0; c < 16; ++c) s32[c * 32 + lane] = __uint_as_float(r[c]);
+          __syncwarp();
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              const float z = __uint_as_float(r[c]) + bv;
-              s16[c * 32 + lane] = f32_to_bf16_rn(gelu_erf(z));
-              if constexpr (EPI == kEpiGeluBf16Train) {
-                if (c < nc && f_ok)
-                  p.g_out[(int64_t)(tl.row0 + c0 + c) * p.n_out + f] = f32_to_bf16_rn(gelu_erf_grad(z));
-              }
+          for (int id = lane; id < 64; id += 32) {
+            const int row = id >> 2, q = id & 3;
+            const int ff = fw + 8 * q;
+            if (row < nc && ff < p.n_out) {
+              const int64_t o = (int64_t)(tl.row0 + c0 + row) * p.n_out + ff;
+              const uint4 gv = *reinterpret_cast<const uint4*>(p.g_in + o);
+              const float4 h0 = *reinterpret_cast<const float4*>(s32 + row * 32 + 8 * q);
+              const float4 h1 = *reinterpret_cast<const float4*>(s32 + row * 32 + 8 * q + 4);
+              uint4 ov;
+              ov.x = (uint32_t)f32_to_bf16_rn(h0.x * __uint_as_float(gv.x << 16)) |
+                     ((uint32_t)f32_to_bf16_rn(h0.y * __uint_as_float(gv.x & 0xffff0000u)) << 16);
+              ov.y = (uint32_t)f32_to_bf16_rn(h0.z * __uint_as_float(gv.y << 16)) |
+                     ((uint32_t)f32_to_bf16_rn(h0.w * __uint_as_float(gv.y & 0xffff0000u)) << 16);
+              ov.z = (uint32_t)f32_to_bf16_rn(h1.x * __uint_as_float(gv.z << 16)) |
+                     ((uint32_t)f32_to_bf16_rn(h1.y * __uint_as_float(gv.z & 0xffff0000u)) << 16);
+              ov.w = (uint32_t)f32_to_bf16_rn(h1.z * __uint_as_float(gv.w << 16)) |
+                     ((uint32_t)f32_to_bf16_rn(h1.w * __uint_as_float(gv.w & 0xffff0000u)) << 16);
+              *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.out) + o) = ov;
             }
           }
           __syncwarp();
+        } else if constexpr (EPI == kEpiGeluBf16 || EPI == kEpiGeluBf16Train) {
+          // stage [16 tokens][32 features] bf16, then 16-byte stores of 8 features of one token
+          // (the training variant stages GeLU'(z) the same way, after GeLU(z))
+          uint16_t* s16 = reinterpret_cast<uint16_t*>(st);
+#pragma unroll
+          for (int c = 0; c < 16; ++c) s16[c * 32 + lane] = f32_to_bf16_rn(gelu_erf(__uint_as_float(r[c]) + bv));
+          __syncwarp();
+          if constexpr (EPI == kEpiGeluBf16Train) {
+            uint16_t* g16 = s16 + 16 * 32;
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+              g16[c * 32 + lane] = f32_to_bf16_rn(gelu_erf_grad(__uint_as_float(r[c]) + bv));
+            __syncwarp();
+#pragma unroll
+            for (int id = lane; id < 64; id += 32) {
+              const int row = id >> 2, q = id & 3;
+              const int ff = fw + 8 * q;
+              if (row < nc && ff < p.n_out)
+                *reinterpret_cast<uint4*>(p.g_out + (int64_t)(tl.row0 + c0 + row) * p.n_out + ff) =
+                    *reinterpret_cast<const uint4*>(st + 1024 + row * 64 + q * 16);
+            }
+          }
 #pragma unroll
           for (int id = lane; id < 64; id += 32) {
             const int row = id >> 2, q = id & 3;

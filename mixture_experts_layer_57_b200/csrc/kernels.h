@@ -146,9 +146,14 @@ bool make_bf16_map_2d(CUtensorMap* m, const void* ptr, int64_t rows, int64_t col
 //     out[e][m][n] = sum over the rows r of segment e of a[r][m] * b[r][n]    (fp32, overwritten)
 // a [rows_max, M] and b [rows_max, N] bf16, token-major; offsets == nullptr: one segment
 // [0, rows_max) (E == 1). Experts without rows get zeros.
+// splits > 1: split-K, out holds [splits][E][M][N] partial sums (add them in split order).
+// b_period > 0 (a multiple of 64): row r of a pairs with row r % b_period of b, which has
+// b_rows <= b_period rows (the rest read as zero); the router's weight gradient stacks three
+// bf16 parts of dL/dlogits against x this way.
 cudaError_t enqueue_wgrad_bf16(const void* a, const void* b, const int32_t* offsets, int E,
                                int64_t rows_max, int M, int N, float* out, int* status,
-                               cudaStream_t stream);
+                               cudaStream_t stream, int splits = 1, int64_t b_period = 0,
+                               int64_t b_rows = 0);
 // Layer 1 for training: h = bf16(GeLU(W x + b)) and g = bf16(GeLU'(W x + b)), both [rows, N].
 cudaError_t enqueue_grouped_gemm_bf16_train(const void* x, const int32_t* offsets, int E,
                                             int64_t rows_max, int K, int N, const void* w,
@@ -232,8 +237,15 @@ int colsum_splits(int64_t longest_segment);
 cudaError_t enqueue_colsum(const void* X, bool bf16, const int32_t* offsets, int E,
                            int64_t rows_max, int N, int S, float* partial, float* out,
                            cudaStream_t stream);
+// out[g][n] = sum_s part[g][s][n] for n < N, rows of part N_stride apart (0: N).
 cudaError_t enqueue_split_reduce(const float* part, int64_t groups, int S, int64_t N, float* out,
-                                 cudaStream_t stream);
+                                 cudaStream_t stream, int64_t N_stride = 0);
+// bf16 parts of dL/dlogits and W_r for the router's backward GEMMs on tensor cores:
+// dl3 [3 Tpad, Epad] (hi; mid; lo stacked by rows), dlx [T, Kx] ([hi | mid | hi | 0]),
+// wx [Kx, d] ([W_hi; W_hi; W_mid; 0]); Tpad % 64 == 0, Epad % 8 == 0, Kx = roundup(3E, 8).
+cudaError_t enqueue_router_bwd_split(const float* dl, int64_t T, int64_t Tpad, int E, int Epad,
+                                     int Kx, uint16_t* dl3, uint16_t* dlx, const float* w_router,
+                                     int d, uint16_t* wx, cudaStream_t stream);
 cudaError_t enqueue_dx_gather(const void* dout, bool bf16, bool add_dout, const float* dense_dx,
                               const float* dxp, const int32_t* offsets, const int32_t* ids,
                               const int32_t* slot, int64_t T, int d, int E, int k,

@@ -213,6 +213,37 @@ def test_shard_entry_validation(L):
     assert beg() == 2 and end() == 2            # a global priority order is not sharded
 
 
+def test_training_entry_validation(L, monkeypatch):
+    args = moe.LayerArgs(T=4096, d_model=1024, d_ff=4096, E=128, k=1, capacity_factor=1.0,
+                         dtype=1, out_dtype=1, x=FAKE, w_router=FAKE, w1=FAKE, w2=FAKE,
+                         add_input_residual=1, aux_alpha=0.01)
+    nb = moe.moe_layer_train_workspace_bytes(args)
+    # the training workspace holds the forward's plus h, GeLU'(z), dY, dZ, dX rows and more
+    assert nb > moe.moe_layer_workspace_bytes(args) + 4096 * 4096 * 2 * 2
+    aux = moe.LayerAux()
+    fwd = lambda wsb=nb, out=FAKE: L.moe_layer_forward_train(ctypes.byref(args), out, ctypes.byref(aux),
+                                                             FAKE, wsb, None)
+    assert fwd(wsb=nb - 1) == 3
+    assert fwd(out=None) == 1
+    assert fwd(out=FAKE + 2) == 6
+    g = moe.LayerGrads(dx=FAKE, dw_router=FAKE, dw1=FAKE, dw2=FAKE)
+    bwd = lambda dout=FAKE, aw=0.0, zw=0.0, wsb=nb, grads=g: L.moe_layer_backward(
+        ctypes.byref(args), dout, aw, zw, ctypes.byref(grads) if grads is not None else None,
+        FAKE, wsb, None)
+    assert bwd(grads=None) == 1
+    assert bwd(dout=None) == 1
+    assert bwd(aw=float("nan")) == 1
+    assert bwd(wsb=nb - 1) == 3
+    g2 = moe.LayerGrads(dx=FAKE, dw_router=FAKE, dw1=None, dw2=FAKE)
+    assert bwd(grads=g2) == 1                   # expert weight gradients are required
+    g3 = moe.LayerGrads(dx=FAKE, dw_router=FAKE, dw1=FAKE, dw2=FAKE, db1=FAKE + 4)
+    assert bwd(grads=g3) == 6
+    monkeypatch.setenv("MOE_FAULT_INJECT", "moe_layer_backward")
+    assert bwd() == 4
+    monkeypatch.setenv("MOE_FAULT_INJECT", "moe_layer_forward_train")
+    assert fwd() == 4
+
+
 def test_fault_injection_is_host_side(L, monkeypatch):
     # the injected failure is returned after validation and before any enqueue
     monkeypatch.setenv("MOE_FAULT_INJECT", "moe_router_topk")
