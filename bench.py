@@ -14,6 +14,9 @@ the dominant kernel (algorithmic bytes or FLOPs per launch / its event-timed dur
 MEASURED_PEAKS.json), the end-to-end throughput through the public API with pinned host buffers
 (H2D of x and D2H of the output inside the timed region), SM clocks and throttle reasons sampled
 through NVML during the timed region, and the CPU oracle's throughput on a bounded sample.
+`train_step` times one training step of the same layer (moe_layer_forward_train keeping the
+backward's state, then moe_layer_backward for a fixed output gradient with the load-balance and
+z-loss terms) with events, and the backward's algorithmic bytes against the HBM peak.
 
 --impl reference times the CPU oracle (the only reference implementation of this method) on a
 bounded sample per step and prints the same JSON line with "impl": "reference".
@@ -271,6 +274,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--skip-train", action="store_true",
+                    help="skip the training-step measurement (forward keeping state + backward)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="run the workload with T tokens instead of its own (profiling captures)")
     args = ap.parse_args()
@@ -399,6 +404,11 @@ def main():
     if not args.skip_e2e:
         e2e = end_to_end(moe, args_c, d, w, ws, stream, args, dist, device)
 
+    # ---------------------------------------------------------- training step
+    train = None
+    if not args.skip_train:
+        train = train_step(moe, args_c, d, w, stream, flush_buf, args, dist, device, E_t, R)
+
     # ---------------------------------------------------------- CPU oracle baseline
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.skip_cpu_baseline:
@@ -421,7 +431,7 @@ def main():
             "config": workload_config(w, args.gpus), "roofline": roof, "cpu_baseline": cpu,
             "clocks": clocks.summary(), "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps,
-            "breakdown_ms": bd, "routing": routing,
+            "breakdown_ms": bd, "routing": routing, "train_step": train,
             "step_ms": {"min": float(min(step_ms)), "median": float(np.median(step_ms)),
                         "max": float(max(step_ms))}}
     if dist.rank == 0:
@@ -443,6 +453,76 @@ def stage_breakdown(moe, args_c, out, aux, ws, stream, flush_buf, reps: int) -> 
             times.setdefault(names[i], []).append(evs[i - 1].elapsed_time(evs[i]))
     assert moe.moe_get_device_error(ws) == 0
     return {n: float(np.median(v)) for n, v in times.items()}
+
+
+def train_step(moe, args_c, d, w, stream, flush_buf, args, dist, device, E_t, R) -> dict:
+    """One training step of the layer: moe_layer_forward_train, then moe_layer_backward for a
+    fixed output gradient (with the load-balance and z-loss terms), L2 flushed before each step,
+    timed with CUDA events around both calls and around each."""
+    T, E, k, dm, df = w.T, w.E, w.k, w.d_model, w.d_ff
+    dt = d["x"].dtype
+    f32 = dict(dtype=torch.float32, device=device)
+    ws_t = moe.workspace(moe.moe_layer_train_workspace_bytes(args_c), device)
+    out = torch.empty(T, dm, dtype=dt, device=device)
+    g = dict(dx=torch.empty(T, dm, dtype=dt, device=device), dw_router=torch.empty(E, dm, **f32),
+             db_router=torch.empty(E, **f32), dw1=torch.empty(E, df, dm, **f32),
+             db1=torch.empty(E, df, **f32), dw2=torch.empty(E, dm, df, **f32),
+             db2=torch.empty(E, dm, **f32))
+    if w.dense:
+        g.update(dense_dw1=torch.empty(df, dm, **f32), dense_db1=torch.empty(df, **f32),
+                 dense_dw2=torch.empty(dm, df, **f32), dense_db2=torch.empty(dm, **f32))
+    gen = torch.Generator(device=device).manual_seed(57)
+    dout = torch.randn(T, dm, generator=gen, device=device).to(dt)
+
+    def fwd():
+        moe.moe_layer_forward_train(args_c, out, ws=ws_t, stream=stream)
+
+    def bwd():
+        moe.moe_layer_backward(args_c, dout, g, ws_t, aux_weight=0.01, z_weight=0.001, stream=stream)
+
+    for _ in range(max(3, min(args.warmup, 5))):
+        flush_buf.zero_()
+        fwd()
+        bwd()
+    torch.cuda.synchronize()
+    launches = moe.moe_last_launch_count()
+    n = max(3, min(args.steps, 20))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
+    dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(n):
+        flush_buf.zero_()
+        evs[i][0].record(stream)
+        fwd()
+        evs[i][1].record(stream)
+        bwd()
+        evs[i][2].record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    assert moe.moe_get_device_error(ws_t) == 0, "device error during the training steps"
+    f_ms = float(np.median([e[0].elapsed_time(e[1]) for e in evs]))
+    b_ms = float(np.median([e[1].elapsed_time(e[2]) for e in evs]))
+    ms = dist.max(float(np.mean([e[0].elapsed_time(e[2]) for e in evs])), device)
+    es = d["x"].element_size()
+    # algorithmic bytes of the backward: the weights read by the two data-gradient GEMMs, fp32
+    # weight and bias gradients written (every expert's), and the activations it reads/writes
+    wbytes = 2 * E_t * dm * df * es + 2 * E * dm * df * 4 + E * (dm + df) * 4
+    act = (T * dm * es + R * dm * 4 + R * dm * es          # combine backward
+           + R * df * es * 3 + R * dm * es                  # dZ GEMM: g' and dZ, dY in
+           + R * df * es + R * dm * 4                       # dX GEMM
+           + R * dm * es + R * df * es * 2 + R * dm * es    # weight gradients' operands
+           + T * E * 4 * 4 + T * dm * es + T * dm * 4       # router backward
+           + T * dm * es + R * dm * 4 + T * dm * 4 + T * dm * es)  # dx gather
+    if w.dense:
+        wbytes += 2 * dm * df * es + 2 * dm * df * 4
+        act += 6 * T * df * es + 4 * T * dm * es + T * dm * 4
+    peaks, _ = load_peaks()
+    bw_frac = (wbytes + act) / (b_ms / 1e3) / (peaks["hbm_gbs"] * 1e9)
+    return {"ms_per_step": ms, "tokens_per_s": args.gpus * T / (ms / 1e3), "fwd_ms": f_ms,
+            "bwd_ms": b_ms, "steps": n, "gpu_launches_bwd": launches,
+            "bwd_algorithmic_bytes": wbytes + act, "bwd_hbm_frac": bw_frac,
+            "objective": "sum(dout * out) + 0.01 aux + 0.001 z_loss, dout ~ N(0, 1)",
+            "grads": "dx (bf16) and fp32 dW_r, db_r, dW1, db1, dW2, db2 (+ dense MLP)"}
 
 
 def end_to_end(moe, args_c, d, w, ws, stream, args, dist, device) -> dict:
