@@ -28,6 +28,8 @@
 //                 rows/features; then release the accumulator
 // Every wait is bounded (about 2 s): on expiry the kernel records MOE_DEVERR_TIMEOUT in the
 // status word, the other roles stop, in-flight TMA copies and MMAs are drained, TMEM is freed.
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -58,14 +60,17 @@ constexpr int kEpiGeluGradBf16 = 4;   // out = bf16(acc * g[r, f]), g = GeLU'(z)
                                       // forward (backward through layer 2 into layer 1's input)
 constexpr int kEpiGeluBf16Train = 5;  // layer 1 forward that also saves g = bf16(GeLU'(z))
 
-template <int BN>
+// FT: 128-feature tiles per CTA tile. With FT = 2 both feature tiles multiply the same token
+// tile, so each token tile is read from L2 half as often (two accumulators per buffer).
+template <int BN, int FT = 1>
 struct Cfg {
-  static constexpr int kABytes = kBM * kBK * 2;
+  static constexpr int kABytes = FT * kBM * kBK * 2;
   static constexpr int kBBytes = BN * kBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kStagesFit = (200 * 1024) / kStageBytes;
   static constexpr int kStages = kStagesFit > MOE_GG_MAX_STAGES ? MOE_GG_MAX_STAGES : kStagesFit;
-  static constexpr int kTmemCols = (2 * BN) < 32 ? 32 : (2 * BN);
+  static constexpr int kTmemCols = (2 * FT * BN) < 32 ? 32 : (2 * FT * BN);
+  static_assert(2 * FT * BN <= 512, "two buffers of FT accumulators must fit TMEM");
   // barriers: full[S], empty[S], tmem_full[2], tmem_empty[2], drain  (8 bytes each, <= 64 of them)
   static constexpr int kBarBytes = 8 * 64;
   static constexpr int kAuxBytes = kBarBytes + 16 + 2 * 4 * (MOE_MAX_EXPERTS + 1);
@@ -109,7 +114,7 @@ struct Tile {
   int e, f0, row0, n_valid;
 };
 
-template <int BN>
+template <int BN, int FT>
 __device__ __forceinline__ Tile decode_tile(int t, const int* prefix, const int* seg, int E,
                                             int n_ftiles) {
   int lo = 0, hi = E;  // prefix[lo] <= t < prefix[hi]
@@ -125,7 +130,7 @@ __device__ __forceinline__ Tile decode_tile(int t, const int* prefix, const int*
   const int jt = local - ft * ntt;
   Tile tl;
   tl.e = lo;
-  tl.f0 = ft * kBM;
+  tl.f0 = ft * kBM * FT;
   tl.row0 = seg[lo] + jt * BN;
   tl.n_valid = min(BN, rows - jt * BN);
   return tl;
@@ -144,11 +149,11 @@ __device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity, i
 
 // A_MN: the weight operand is stored [E][K][n_out] (the transpose of the forward layout, as the
 // backward pass reads W1 and W2) and loaded MN-major: two 64-feature x 64-K boxes per stage.
-template <int BN, int EPI, bool A_MN = false>
+template <int BN, int EPI, bool A_MN = false, int FT = 1>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmW,
                         const __grid_constant__ CUtensorMap tmX, const Params p) {
-  using C = Cfg<BN>;
+  using C = Cfg<BN, FT>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t base_addr = (raw_addr + 1023u) & ~1023u;
@@ -196,7 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(smem_u32(tmem_holder), C::kTmemCols);
     tmem_relinquish();
   }
-  const int n_ftiles = (p.n_out + kBM - 1) / kBM;
+  const int n_ftiles = (p.n_out + kBM * FT - 1) / (kBM * FT);
   if (warp == 2) {
     // Tile list: prefix[e] = first tile of expert e; validates the device offsets.
     const int E = p.E;
@@ -249,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       int issued = 0;
       for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
-        const Tile tl = decode_tile<BN>(t, prefix, seg, p.E, n_ftiles);
+        const Tile tl = decode_tile<BN, FT>(t, prefix, seg, p.E, n_ftiles);
         const int w_row = tl.e * p.n_out + tl.f0;
         bool ok = true;
         for (int kb = 0; kb < n_kb; ++kb) {
@@ -259,12 +264,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint32_t sa = base_addr + stage * C::kStageBytes;
           mbar_arrive_expect_tx(full_bar(stage), C::kStageBytes);
-          if constexpr (A_MN) {
-            const int k_row = tl.e * p.K + kb * kBK;
-            tma_load_2d(sa, &tmW, tl.f0, k_row, full_bar(stage));
-            tma_load_2d(sa + C::kABytes / 2, &tmW, tl.f0 + 64, k_row, full_bar(stage));
-          } else {
-            tma_load_2d(sa, &tmW, kb * kBK, w_row, full_bar(stage));
+#pragma unroll
+          for (int i = 0; i < FT; ++i) {
+            const uint32_t sai = sa + i * (kBM * kBK * 2);
+            if constexpr (A_MN) {
+              const int k_row = tl.e * p.K + kb * kBK;
+              tma_load_2d(sai, &tmW, tl.f0 + i * kBM, k_row, full_bar(stage));
+              tma_load_2d(sai + kBM * kBK, &tmW, tl.f0 + i * kBM + 64, k_row, full_bar(stage));
+            } else {
+              // rows past this expert's n_out (odd tile count) belong to the next expert or are
+              // out of range; the epilogue masks those features
+              tma_load_2d(sai, &tmW, kb * kBK, w_row + i * kBM, full_bar(stage));
+            }
           }
           tma_load_2d(sa + C::kABytes, &tmX, kb * kBK, tl.row0, full_bar(stage));
           ++issued;
@@ -288,10 +299,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-        const Tile tl = decode_tile<BN>(t, prefix, seg, p.E, n_ftiles);
+        const Tile tl = decode_tile<BN, FT>(t, prefix, seg, p.E, n_ftiles);
         if (!mbar_wait_bounded(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.status)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * FT * BN);
         const int n_mma = max(16, (tl.n_valid + 15) & ~15);
         const uint32_t idesc = idesc_bf16_f32_major(kBM, n_mma, A_MN, false);
         for (int kb = 0; kb < n_kb; ++kb) {
@@ -301,15 +312,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const uint32_t sa = base_addr + stage * C::kStageBytes;
-          const uint64_t adesc = A_MN ? smem_desc_sw128_mn(sa) : smem_desc_sw128(sa);
           const uint64_t bdesc = smem_desc_sw128(sa + C::kABytes);
           // K step: +32 bytes inside a K-major 128-byte row (+2 in the 16-byte address field),
           // or two 8-row groups of an MN-major tile
           constexpr uint64_t a_step = A_MN ? (kMnKStepBytes >> 4) : 2;
 #pragma unroll
-          for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
-            tc_mma_bf16(d_tmem, adesc + a_step * (uint64_t)kk, bdesc + (uint64_t)(2 * kk), idesc,
-                        (kb | kk) != 0 ? 1u : 0u);
+          for (int i = 0; i < FT; ++i) {
+            const uint32_t sai = sa + i * (kBM * kBK * 2);
+            const uint64_t adesc = A_MN ? smem_desc_sw128_mn(sai) : smem_desc_sw128(sai);
+#pragma unroll
+            for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
+              tc_mma_bf16(d_tmem + (uint32_t)(i * BN), adesc + a_step * (uint64_t)kk,
+                          bdesc + (uint64_t)(2 * kk), idesc, (kb | kk) != 0 ? 1u : 0u);
+            }
           }
           tc_commit(empty_bar(stage));
           if (++stage == S) {
@@ -337,16 +352,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
-      const Tile tl = decode_tile<BN>(t, prefix, seg, p.E, n_ftiles);
+      const Tile tl = decode_tile<BN, FT>(t, prefix, seg, p.E, n_ftiles);
       if (!mbar_wait_bounded_warp(tfull_bar(acc), acc_phase, abort_flag, p.status)) break;
       tc_fence_after();
-      const int fw = tl.f0 + quarter * 32;  // first feature of this warp
+#pragma unroll 1
+      for (int fi = 0; fi < FT; ++fi) {
+      const int fw = tl.f0 + fi * kBM + quarter * 32;  // first feature of this warp
       const int f = fw + lane;
       const bool f_ok = f < p.n_out;
       const float bv = (p.bias != nullptr && f_ok)
                            ? bf16_to_f32(reinterpret_cast<const uint16_t*>(p.bias)[(int64_t)tl.e * p.n_out + f])
                            : 0.0f;
-      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
+      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) +
+                             (uint32_t)(acc * FT * BN + fi * BN);
       for (int c0 = half * 16; c0 < tl.n_valid; c0 += 32) {
         uint32_t r[16];
         tmem_ld_32x32b_x16(taddr + (uint32_t)c0, r);
@@ -501,6 +519,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
         }
       }
+      }  // feature tiles
       tc_fence_before();
       mbar_arrive(tempty_bar(acc));
       if (++acc == 2) {
@@ -566,18 +585,18 @@ bool make_mn_map(CUtensorMap* m, const void* ptr, int64_t rows, int cols) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, int EPI, bool A_MN = false>
+template <int BN, int EPI, bool A_MN = false, int FT = 1>
 cudaError_t launch_one(const CUtensorMap& tmW, const CUtensorMap& tmX, const Params& p,
                        cudaStream_t stream) {
-  auto kern = grouped_gemm_kernel<BN, EPI, A_MN>;
+  auto kern = grouped_gemm_kernel<BN, EPI, A_MN, FT>;
+  constexpr int smem = Cfg<BN, FT>::kSmemBytes;
   static bool attr_set = false;  // per instantiation
   if (!attr_set) {
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<BN>::kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  return launch_kernel(kern, dim3(num_sms()), dim3(kThreads), Cfg<BN>::kSmemBytes, stream, tmW, tmX, p);
+  return launch_kernel(kern, dim3(num_sms()), dim3(kThreads), smem, stream, tmW, tmX, p);
 }
 
 }  // namespace
@@ -603,15 +622,41 @@ static int pick_token_tile(int64_t capacity_hint) {
   return 256;
 }
 
+#ifndef MOE_GG_FT
+#define MOE_GG_FT 2
+#endif
+
+// Fraction of the last wave's CTA slots that hold a tile (tiles over persistent CTAs).
+static double wave_efficiency(int64_t tiles) {
+  const int64_t s = num_sms();
+  if (tiles <= 0) return 1.0;
+  return (double)tiles / (double)(((tiles + s - 1) / s) * s);
+}
+
+// Two feature tiles per CTA tile (each token tile read from L2 half as often) when the layer has
+// more than one feature tile, TMEM holds them, and halving the tile count does not leave the
+// last wave of the persistent grid emptier (estimated from E and the capacity hint).
 template <int EPI, bool A_MN = false>
 cudaError_t launch_bn(int BN, const CUtensorMap& tmW, const CUtensorMap& tmX, const Params& p,
-                      cudaStream_t stream) {
+                      cudaStream_t stream, int64_t capacity_hint) {
+  bool two = MOE_GG_FT == 2 && p.n_out > kBM && BN <= 128;
+  if (two) {
+    const int64_t rows = std::min<int64_t>(std::max<int64_t>(capacity_hint, 1), p.rows_max);
+    const int64_t tok_tiles = (int64_t)p.E * ((rows + BN - 1) / BN);
+    const int64_t t1 = tok_tiles * ((p.n_out + kBM - 1) / kBM);
+    const int64_t t2 = tok_tiles * ((p.n_out + 2 * kBM - 1) / (2 * kBM));
+    two = wave_efficiency(t2) >= wave_efficiency(t1) - 0.02;
+  }
   switch (BN) {
-    case 16: return launch_one<16, EPI, A_MN>(tmW, tmX, p, stream);
-    case 32: return launch_one<32, EPI, A_MN>(tmW, tmX, p, stream);
-    case 64: return launch_one<64, EPI, A_MN>(tmW, tmX, p, stream);
-    case 128: return launch_one<128, EPI, A_MN>(tmW, tmX, p, stream);
-    default: return launch_one<256, EPI, A_MN>(tmW, tmX, p, stream);
+    case 16: return two ? launch_one<16, EPI, A_MN, 2>(tmW, tmX, p, stream)
+                        : launch_one<16, EPI, A_MN, 1>(tmW, tmX, p, stream);
+    case 32: return two ? launch_one<32, EPI, A_MN, 2>(tmW, tmX, p, stream)
+                        : launch_one<32, EPI, A_MN, 1>(tmW, tmX, p, stream);
+    case 64: return two ? launch_one<64, EPI, A_MN, 2>(tmW, tmX, p, stream)
+                        : launch_one<64, EPI, A_MN, 1>(tmW, tmX, p, stream);
+    case 128: return two ? launch_one<128, EPI, A_MN, 2>(tmW, tmX, p, stream)
+                         : launch_one<128, EPI, A_MN, 1>(tmW, tmX, p, stream);
+    default: return launch_one<256, EPI, A_MN, 1>(tmW, tmX, p, stream);
   }
 }
 
@@ -625,8 +670,8 @@ cudaError_t enqueue_grouped_gemm_bf16(const void* x, const int32_t* offsets, int
   if (!make_kmajor_map(&tmW, w, (int64_t)E * N, K, kBM) || !make_kmajor_map(&tmX, x, rows_max, K, BN))
     return cudaErrorInvalidValue;
   Params p{offsets, E, N, K, rows_max, bias, out, status, CombineArgs{}, nullptr, nullptr};
-  return gelu ? launch_bn<kEpiGeluBf16>(BN, tmW, tmX, p, stream)
-              : launch_bn<kEpiF32>(BN, tmW, tmX, p, stream);
+  return gelu ? launch_bn<kEpiGeluBf16>(BN, tmW, tmX, p, stream, capacity_hint)
+              : launch_bn<kEpiF32>(BN, tmW, tmX, p, stream, capacity_hint);
 }
 
 cudaError_t enqueue_grouped_gemm_bf16_train(const void* x, const int32_t* offsets, int E,
@@ -641,7 +686,7 @@ cudaError_t enqueue_grouped_gemm_bf16_train(const void* x, const int32_t* offset
     return cudaErrorInvalidValue;
   Params p{offsets, E, N, K, rows_max, bias, h_out, status, CombineArgs{}, nullptr,
            (uint16_t*)g_out};
-  return launch_bn<kEpiGeluBf16Train>(BN, tmW, tmX, p, stream);
+  return launch_bn<kEpiGeluBf16Train>(BN, tmW, tmX, p, stream, capacity_hint);
 }
 
 cudaError_t enqueue_grouped_gemm_dgrad_bf16(const void* dy, const int32_t* offsets, int E,
@@ -655,8 +700,8 @@ cudaError_t enqueue_grouped_gemm_dgrad_bf16(const void* dy, const int32_t* offse
     return cudaErrorInvalidValue;
   Params p{offsets, E, N, K, rows_max, nullptr, out, status, CombineArgs{},
            (const uint16_t*)g_in, nullptr};
-  return g_in != nullptr ? launch_bn<kEpiGeluGradBf16, true>(BN, tmW, tmX, p, stream)
-                         : launch_bn<kEpiF32, true>(BN, tmW, tmX, p, stream);
+  return g_in != nullptr ? launch_bn<kEpiGeluGradBf16, true>(BN, tmW, tmX, p, stream, capacity_hint)
+                         : launch_bn<kEpiF32, true>(BN, tmW, tmX, p, stream, capacity_hint);
 }
 
 cudaError_t enqueue_gemm2_combine(const void* h, const int32_t* offsets, int E, int64_t rows_max,
@@ -672,8 +717,8 @@ cudaError_t enqueue_gemm2_combine(const void* h, const int32_t* offsets, int E, 
                 (const uint16_t*)fc.residual, fc.out, fc.out_bf16 ? 1 : 0, fc.k, fc.E_experts,
                 fc.rows_y};
   Params p{offsets, E, N, K, rows_max, bias, nullptr, status, c, nullptr, nullptr};
-  return fc.dense ? launch_bn<kEpiCombineDense>(BN, tmW, tmX, p, stream)
-                  : launch_bn<kEpiCombineExpert>(BN, tmW, tmX, p, stream);
+  return fc.dense ? launch_bn<kEpiCombineDense>(BN, tmW, tmX, p, stream, capacity_hint)
+                  : launch_bn<kEpiCombineExpert>(BN, tmW, tmX, p, stream, capacity_hint);
 }
 
 cudaError_t enqueue_expert_ffn_bf16(const void* x_packed, const int32_t* offsets, int E,
