@@ -1,4 +1,5 @@
-"""CPU oracle of the MoE-layer forward pass — TEST INFRASTRUCTURE ONLY.
+"""CPU oracle of the MoE layer (forward pass, routing variants, backward pass) — TEST
+INFRASTRUCTURE ONLY.
 
 A plain, slow, single-threaded C++ reference (``moe_oracle.cpp``) with every
 accumulation in double, plus this thin ctypes wrapper. Only ``tests/``,
@@ -9,7 +10,8 @@ Every function follows a passage of the pages (cited in ``moe_oracle.cpp``):
 the MoE formula p(x)=softmax(W_r x), y=sum_{e in TopK} p_e E_e(x) of the
 DeepSpeed MoE blog; the expert-capacity rule of the Switch/DeepSpeed comparison
 article; the PR-MoE residual form of the DeepSpeed-MoE notes; the Switch
-load-balance loss of the MoE survey notes.
+load-balance loss of the MoE survey notes; the comparison article's router z-loss
+and capacity-by-probability example; the chain rule through all of them.
 """
 from __future__ import annotations
 

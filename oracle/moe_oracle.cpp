@@ -1,7 +1,8 @@
 // TEST INFRASTRUCTURE ONLY: a plain, slow, single-threaded CPU reference of the
-// forward pass of one Mixture-of-Experts FFN layer. It exists to check the CUDA
-// path; only the tests, the smoke check and the benchmark's CPU-baseline leg may
-// load it. It shares no code, header or table with the CUDA library.
+// forward pass of one Mixture-of-Experts FFN layer (and, at the end of this file,
+// of its backward pass). It exists to check the CUDA path; only the tests, the
+// smoke check and the benchmark's CPU-baseline leg may load it. It shares no
+// code, header or table with the CUDA library.
 //
 // What it computes is the plain definition of the layer, written out step by step
 // with every accumulation in double:
