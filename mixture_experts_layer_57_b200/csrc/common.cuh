@@ -134,7 +134,7 @@ __device__ __forceinline__ bool mbar_wait_bounded_warp(uint32_t bar, uint32_t pa
   }
 }
 
-// ---------------------------------------------------------------- TMA (no multicast)
+// ---------------------------------------------------------------- TMA (loads into this CTA only)
 
 __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
