@@ -398,6 +398,16 @@ def main():
     roof["per_stage"] = {n: {"ms": bd[n], "GB/s": stage_bytes[n] / (bd[n] / 1e3) / 1e9,
                              "TFLOP/s": stage_flops[n] / (bd[n] / 1e3) / 1e12}
                          for n in gemm_stages}
+    # the routing stages against their own bounds: the router's logits are 2 T d E FLOP over
+    # x (read once), W_r and the logits/ids/gates; dispatch moves the kept rows (read + write)
+    other = {
+        "router": (T * dm * es + E * dm * 4 + 2 * T * E * 4 + T * k * 8, 2.0 * T * dm * E),
+        "dispatch": (2 * R * dm * es + T * k * 12 + 2 * (E + 1) * 4, 0.0),
+    }
+    for n, (b_n, f_n) in other.items():
+        if n in bd and bd[n] > 0:
+            roof["per_stage"][n] = {"ms": bd[n], "GB/s": b_n / (bd[n] / 1e3) / 1e9,
+                                    "TFLOP/s": f_n / (bd[n] / 1e3) / 1e12}
 
     # ---------------------------------------------------------- end to end through the API
     e2e = None
@@ -419,6 +429,7 @@ def main():
         n = int(max(8, min(2048, 12.0 / per_tok)))
         rate, dt = oracle_sample_rate(w, inp, n, full_logits)
         cpu = {"value": rate, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+               "host": host_cpu(),
                "sample": f"{n} tokens ({dt:.1f} s): their router logits, routing and slots of all "
                          f"{T} tokens from given logits, expert FFN and combine of the {n}; "
                          "single-threaded C++ oracle in double"}
@@ -432,12 +443,27 @@ def main():
             "clocks": clocks.summary(), "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps,
             "breakdown_ms": bd, "routing": routing, "train_step": train,
-            "step_ms": {"min": float(min(step_ms)), "median": float(np.median(step_ms)),
-                        "max": float(max(step_ms))}}
+            "step_ms": {"min": float(min(step_ms)), "p10": float(np.percentile(step_ms, 10)),
+                        "median": float(np.median(step_ms)),
+                        "p90": float(np.percentile(step_ms, 90)), "max": float(max(step_ms))}}
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
     dist.close()
     return 0
+
+
+def host_cpu() -> dict:
+    """The host the CPU baseline ran on: logical CPUs and the CPU model."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count(), "cpu_model": model}
 
 
 def stage_breakdown(moe, args_c, out, aux, ws, stream, flush_buf, reps: int) -> dict:
