@@ -175,10 +175,15 @@ def to_dev(a: np.ndarray, device):
 
 
 def kernel_source_hash() -> str:
+    """Hash of the expert GEMM's code (grouped_gemm.cu + common.cuh), `//` comments and blank
+    lines left out, so an edit of the comments keeps the committed traffic figures."""
     h = hashlib.sha256()
     for name in ("grouped_gemm.cu", "common.cuh"):
-        with open(os.path.join(ROOT, "mixture_experts_layer_57_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "mixture_experts_layer_57_b200", "csrc", name)) as f:
+            for line in f:
+                code = line.split("//", 1)[0].rstrip()
+                if code:
+                    h.update(code.encode() + b"\n")
     return h.hexdigest()[:16]
 
 

@@ -16,8 +16,14 @@
 //
 // Schedule: persistent CTAs (one per SM) walk tiles t = blockIdx.x, blockIdx.x + gridDim.x, ...
 // of a list ordered (expert, feature tile, token tile), built in shared memory from the device
-// offsets, so no host synchronisation is needed for the ragged sizes. Roles per CTA:
-//     warp 0      TMA producer: K-major 128x64 weight tile and BNx64 token tile per stage,
+// offsets, so no host synchronisation is needed for the ragged sizes. A tile may hold FT = 2
+// feature tiles of 128 that multiply the same token tile (two accumulators per buffer), so each
+// token tile is read from L2 half as often; the host picks FT = 2 when the layer has more than
+// one feature tile and the halved tile count still fills the persistent grid's waves.
+// A_MN (backward pass): the weights arrive stored [E][K][N] and are read MN-major (two 64-feature
+// boxes per feature tile, MN-major shared-memory descriptors), for dH = dY W2 and dX = dZ W1.
+// Roles per CTA:
+//     warp 0      TMA producer: FT 128x64 weight tiles and a BNx64 token tile per stage,
 //                 128-byte swizzle, STAGES-deep mbarrier ring
 //     warp 1      allocates TMEM, one thread issues tcgen05.mma (K = 16 per instruction) into
 //                 one of two accumulators, commits stage release and accumulator-full barriers
