@@ -332,7 +332,7 @@ moe_status moe_layer_forward_shard_end(const moe_layer_args* args, int64_t T_glo
  *
  * Gradients (fp32, overwritten; shapes those of the parameters): dw_router, db_router, dw1, db1,
  * dw2, db2 and the dense MLP's; dx [T, d_model] in args.dtype. A bias gradient pointer may be
- * NULL (not computed). dgates [T, k] (dL/dgate) and dlogits [T, E] (dL/dlogits) are optional.
+ * NULL (not computed). T == 0 zeroes the parameter gradients. dgates [T, k] (dL/dgate) and dlogits [T, E] (dL/dlogits) are optional.
  * bf16 layers run the expert and dense GEMMs on tcgen05 (bf16 operands: dY, dZ rounded to bf16;
  * fp32 accumulation); the router's GEMMs and fp32 layers run on fp32 FMA. */
 typedef struct {

@@ -5,6 +5,7 @@
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
+#include <utility>
 
 #include "kernels.h"
 
@@ -1026,7 +1027,19 @@ moe_status backward_impl(const moe_layer_args* a, const void* dout, float aux_we
   const int64_t T = a->T;
   const int d = a->d_model, f = a->d_ff, E = a->E, k = a->k;
   const LayerWs& L = w.L;
-  if (T == 0) return MOE_OK;
+  if (T == 0) {
+    // no tokens: every parameter gradient is zero (dx has no rows)
+    const size_t ef = (size_t)E * f, ed = (size_t)E * d, fd = (size_t)f * d;
+    const std::pair<float*, size_t> zero[] = {
+        {g->dw_router, ed}, {g->db_router, (size_t)E}, {g->dw1, ef * d}, {g->db1, ef},
+        {g->dw2, ed * f},   {g->db2, ed},              {g->dense_dw1, fd}, {g->dense_db1, (size_t)f},
+        {g->dense_dw2, fd}, {g->dense_db2, (size_t)d}};
+    for (const auto& z : zero)
+      if (z.first != nullptr && z.second > 0 &&
+          cudaMemsetAsync(z.first, 0, sizeof(float) * z.second, stream) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
   int* status = (int*)ws;
   const bool bf16 = a->dtype == MOE_BF16;
   const int64_t R = L.rows_max;

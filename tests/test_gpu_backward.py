@@ -162,3 +162,27 @@ def test_backward_deterministic(cuda_ok):
     b = run_train(w, d_inp, dout, 0.2, 0.1)
     for n in a:
         assert np.array_equal(a[n], b[n]), n
+
+
+def test_backward_no_tokens_zeroes_gradients(cuda_ok):
+    w = synth.WORKLOADS[2].with_(T=0, d_model=128, d_ff=256)
+    d_inp = dev_inputs(synth.make_inputs(w.with_(T=4)))
+    d_inp["x"] = d_inp["x"][:0]
+    args = moe.layer_args(d_inp["x"], d_inp["w_router"], d_inp["w1"], d_inp["b1"], d_inp["w2"],
+                          d_inp["b2"], k=1, capacity_factor=1.0)
+    out = torch.empty(0, w.d_model, dtype=torch.bfloat16, device="cuda")
+    ws = moe.moe_layer_forward_train(args, out)
+    f32 = dict(dtype=torch.float32, device="cuda")
+    g = dict(dx=torch.empty(0, w.d_model, dtype=torch.bfloat16, device="cuda"),
+             dw_router=torch.full((w.E, w.d_model), 7.0, **f32),
+             db_router=torch.full((w.E,), 7.0, **f32),
+             dw1=torch.full((w.E, w.d_ff, w.d_model), 7.0, **f32),
+             db1=torch.full((w.E, w.d_ff), 7.0, **f32),
+             dw2=torch.full((w.E, w.d_model, w.d_ff), 7.0, **f32),
+             db2=torch.full((w.E, w.d_model), 7.0, **f32))
+    moe.moe_layer_backward(args, torch.empty(0, w.d_model, dtype=torch.bfloat16, device="cuda"),
+                           g, ws)
+    torch.cuda.synchronize()
+    for n, t in g.items():
+        if n != "dx":
+            assert float(t.abs().max()) == 0.0, n
