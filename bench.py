@@ -249,11 +249,12 @@ def run_reference(args, dist: Dist):
               f"their logits, expert FFN and combine of the {n}), single-threaded C++ oracle")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step_sample": ms, "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": ms, "ms_per_step_sample": ms, "tokens_per_step_sample": n,
+            "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(w, args.gpus),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                             "sample": sample},
+                             "sample": sample, "host": host_cpu()},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
