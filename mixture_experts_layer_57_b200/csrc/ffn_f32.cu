@@ -63,12 +63,11 @@ cudaError_t enqueue_grouped_gemm_f32(const float* x, const int32_t* offsets, int
   if (rows_max == 0) return cudaSuccess;
   const unsigned gx = (unsigned)(rows_max < 65536 ? rows_max : 65536);
   const size_t smem = (size_t)K * sizeof(float);
-  static size_t attr_done[2] = {48 * 1024, 48 * 1024};
-  if (smem > attr_done[gelu]) {
-    cudaError_t e = cudaFuncSetAttribute(gelu ? ffn_f32_kernel<true> : ffn_f32_kernel<false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (smem > 48 * 1024) {  // above the default limit: raise it once per device
+    static int attr_done[2][64] = {{0}};
+    cudaError_t e = ensure_dynamic_smem(gelu ? ffn_f32_kernel<true> : ffn_f32_kernel<false>,
+                                        (int)smem, attr_done[gelu ? 1 : 0]);
     if (e != cudaSuccess) return e;
-    attr_done[gelu] = smem;
   }
   const dim3 grid(gx, (N + kFeat - 1) / kFeat);
   return launch_kernel(gelu ? ffn_f32_kernel<true> : ffn_f32_kernel<false>, grid, dim3(kFeat), smem,

@@ -596,12 +596,9 @@ cudaError_t launch_one(const CUtensorMap& tmW, const CUtensorMap& tmX, const Par
                        cudaStream_t stream) {
   auto kern = grouped_gemm_kernel<BN, EPI, A_MN, FT>;
   constexpr int smem = Cfg<BN, FT>::kSmemBytes;
-  static bool attr_set = false;  // per instantiation
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static int attr_done[64] = {0};  // per instantiation and device
+  cudaError_t e = ensure_dynamic_smem(kern, smem, attr_done);
+  if (e != cudaSuccess) return e;
   return launch_kernel(kern, dim3(num_sms()), dim3(kThreads), smem, stream, tmW, tmX, p);
 }
 

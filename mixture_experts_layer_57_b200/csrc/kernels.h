@@ -95,6 +95,20 @@ cudaError_t enqueue_router_logits_tc(const void* x, int64_t T, int d, const uint
                                      int dpad, const float* router_bias, int E, float* logits,
                                      int* status, cudaStream_t stream);
 
+// Raises a kernel's dynamic shared-memory limit to `bytes` on the current device, once per
+// device (done_per_device: a zero-initialised [64] array owned by the launching function).
+template <class Kern>
+cudaError_t ensure_dynamic_smem(Kern kern, int bytes, int* done_per_device) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const bool cached = dev >= 0 && dev < 64;
+  if (cached && done_per_device[dev] >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && cached) done_per_device[dev] = bytes;
+  return e;
+}
+
 // ---------------------------------------------------------------- dispatch
 constexpr int kDispatchSeg = 256;  // (token, choice) pairs per counting segment (one warp)
 inline int64_t dispatch_num_segments(int64_t pairs) {

@@ -268,13 +268,9 @@ template <int NE>
 cudaError_t launch_tc(const CUtensorMap& tmX, const CUtensorMap& tmW, const RParams& p,
                       int ntiles, cudaStream_t stream) {
   auto kern = router_logits_tc_kernel<NE>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         RCfg<NE>::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static int attr_done[64] = {0};  // per device
+  cudaError_t e = ensure_dynamic_smem(kern, RCfg<NE>::kSmemBytes, attr_done);
+  if (e != cudaSuccess) return e;
   const int grid = ntiles < num_sms() ? ntiles : num_sms();
   return launch_kernel(kern, dim3(grid), dim3(kThreads), RCfg<NE>::kSmemBytes, stream, tmX, tmW, p);
 }

@@ -322,13 +322,9 @@ template <int BN>
 cudaError_t launch_w(const CUtensorMap& tmA, const CUtensorMap& tmB, const WParams& p,
                      cudaStream_t stream) {
   auto kern = wgrad_kernel<BN>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, WCfg<BN>::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static int attr_done[64] = {0};  // per device
+  cudaError_t e = ensure_dynamic_smem(kern, WCfg<BN>::kSmemBytes, attr_done);
+  if (e != cudaSuccess) return e;
   return launch_kernel(kern, dim3(num_sms()), dim3(kThreads), WCfg<BN>::kSmemBytes, stream, tmA,
                        tmB, p);
 }
