@@ -5,9 +5,11 @@
  * 每 token 计算增长", the MoE formula and the pipeline listing):
  *
  *     p(x) = softmax(W_r x)                     y = sum_{e in TopK(p(x), k)} p_e(x) E_e(x)
- *     scores = router(hidden); expert_ids, gates = topk(scores, k);
- *     dispatch = pack_by_expert(hidden, expert_ids, capacity); out = local_experts(dispatch);
- *     output = combine(out, gates)
+ *
+ * i.e. score every expert for every token, keep each token's k best experts and their
+ * probabilities as gates, pack the tokens expert by expert within a per-expert capacity, run
+ * each expert's FFN on its packed rows, and sum each token's expert outputs weighted by its
+ * gates.
  *
  * Entry points, in pipeline order:
  *     moe_router_topk   router logits, softmax, top-k, load-balance statistics
@@ -78,7 +80,7 @@ int moe_abi_version(void);
 
 /* ---------------------------------------------------------------- sizes
  * Expert capacity (Switch/DeepSpeed comparison article, section "Expert Capacity Overflow":
- * expert_capacity = tokens_per_batch / num_experts * capacity_factor), with the k choices of
+ * capacity = (tokens in the batch / experts) x capacity factor), with the k choices of
  * each token counted and rounded up: C = ceil(k * T * capacity_factor / E), evaluated in double
  * in that order. capacity_factor must be finite and >= 0. */
 moe_status moe_capacity(int64_t T, int E, int k, double capacity_factor, int64_t* C_out);
@@ -215,9 +217,10 @@ moe_status moe_grouped_gemm(const void* x_packed, const int32_t* expert_offsets,
 /* ---------------------------------------------------------------- combine
  * out[t,:] = [residual[t,:]] + [dense[t,:]] + sum_{j : slot[t,j] >= 0} gates[t,j] *
  *            y_packed[expert_offsets[expert_ids[t,j]] + slot[t,j], :]
- * summed in fp32 in that order and rounded once to out_dtype (DeepSpeed MoE blog, combine(out,
- * gates); comparison article, "Expert Capacity Overflow": a dropped token passes through the
- * residual only; PR-MoE "residual correction" example: fixed MLP output + gate * expert).
+ * summed in fp32 in that order and rounded once to out_dtype (DeepSpeed MoE blog, the combine
+ * step of the pipeline listing; comparison article, "Expert Capacity Overflow": a dropped token
+ * passes through the residual only; PR-MoE "residual correction" example: fixed MLP output +
+ * gate * expert).
  * residual: [T, d_model] in res_dtype or NULL. dense: [T, d_model] fp32 or NULL.
  * A (slot, offset) pointing outside [0, rows_max) sets MOE_DEVERR_BAD_ROW and is skipped. */
 moe_status moe_combine_workspace_bytes(size_t* bytes);

@@ -2,7 +2,7 @@
 //     out[t] = [residual[t]] + [dense[t]] + sum_{j : slot[t,j] >= 0} gate[t,j] * y[row(t,j)]
 //     row(t,j) = offsets[expert_ids[t,j]] + slot[t,j]
 // in fp32, in that order, rounded once to the output type.
-// DeepSpeed MoE blog, `output = combine(returned, gates)` with gates p_e(x); comparison article,
+// DeepSpeed MoE blog, the combine step of its pipeline listing, gates p_e(x); comparison article,
 // "Expert Capacity Overflow" (a dropped token passes through the residual only) and the PR-MoE
 // "residual correction" example (fixed MLP output + gate * expert output).
 //

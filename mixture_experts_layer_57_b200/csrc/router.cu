@@ -1,8 +1,8 @@
 // Router: logits = x W_r^T (+ b_r) in fp32, softmax over all E experts, top-k, and the Switch
 // load-balance statistics (f_i, Q_i, aux).
 //
-// DeepSpeed MoE blog, MoE formula p(x) = softmax(W_r x) and the listing's
-// `expert_ids, gates = topk(scores, k)`; comparison article, "Router computation"
+// DeepSpeed MoE blog, MoE formula p(x) = softmax(W_r x) and the top-k step of its pipeline
+// listing (expert ids and gates per token); comparison article, "Router computation"
 // (logits = x W_r, p = softmax(logits)) and "Top-1 routing decision"; MoE survey notes
 // §1.1.4.1 (f_i = share of tokens whose first choice is i, Q_i = mean p_i,
 // loss = alpha * N * sum_i f_i Q_i).

@@ -11,13 +11,14 @@
 //   y    = sum_{e in TopK(p(x), k)} p_e(x) * E_e(x)          gate-weighted experts
 //
 //   (DeepSpeed MoE and Model Compression, section "DeepSpeed-MoE: capacity growth
-//    is not per-token compute growth", the MoE formula and the pipeline listing
-//    router -> topk -> pack_by_expert(capacity) -> local_experts -> combine)
+//    is not per-token compute growth", the MoE formula and the pipeline listing:
+//    route, keep the top k, pack by expert within a capacity, run the experts,
+//    combine)
 //
 // with a per-expert capacity: tokens beyond an expert's capacity skip that
 // expert's FFN and reach the output only through the residual
 //   (Switch-vs-DeepSpeed comparison article, section "Expert Capacity Overflow":
-//    capacity = tokens_per_batch / num_experts * capacity_factor).
+//    capacity = (tokens in the batch / experts) x capacity factor).
 //
 // Readings of points the pages leave open (each is listed in the design notes):
 //   * capacity C = ceil(k * T * cf / E), evaluated in double in that order;
@@ -160,8 +161,9 @@ void oracle_lb_stats(const float* logits, const int32_t* ids, int64_t T, int E, 
 
 // ---------------------------------------------------------------- capacity and slots
 
-// expert_capacity = tokens_per_batch / num_experts * capacity_factor, with the k
-// choices of each token counted and rounded up: C = ceil(k * T * cf / E).
+// Capacity = (tokens in the batch / experts) x capacity factor (comparison article,
+// "Expert Capacity Overflow"), with the k choices of each token counted and rounded up:
+// C = ceil(k * T * cf / E).
 int64_t oracle_capacity(int64_t T, int E, int k, double capacity_factor) {
   return (int64_t)std::ceil((double)k * (double)T * capacity_factor / (double)E);
 }
