@@ -167,14 +167,15 @@ def assign_slots(ids: np.ndarray, E: int, C: int):
     return slot, counts
 
 
-def assign_slots_priority(ids: np.ndarray, gates: np.ndarray, E: int, C: int):
-    """Priority overflow: (slot [T,k], counts [E]); ranks by gate desc, then pair index."""
+def assign_slots_priority(ids: np.ndarray, probs: np.ndarray, E: int, C: int):
+    """Priority overflow: (slot [T,k], counts [E]); ranks each expert's pairs by router
+    probability (before any renormalisation) descending, then by pair index."""
     ids = np.ascontiguousarray(ids, dtype=np.int32)
-    gates = np.ascontiguousarray(gates, dtype=np.float32)
+    probs = np.ascontiguousarray(probs, dtype=np.float32)
     T, k = ids.shape
     slot = np.empty((T, k), dtype=np.int32)
     counts = np.empty(E, dtype=np.int32)
-    lib().oracle_assign_slots_priority(_p(ids), _p(gates), T, k, E, C, _p(slot), _p(counts))
+    lib().oracle_assign_slots_priority(_p(ids), _p(probs), T, k, E, C, _p(slot), _p(counts))
     return slot, counts
 
 
@@ -226,8 +227,12 @@ def layer_forward(inp: dict, T: int, d_model: int, d_ff: int, E: int, k: int,
                   capacity_factor: float, add_input_residual: bool = True, aux_alpha: float = 0.01,
                   logits_in: Optional[np.ndarray] = None, tokens: Optional[np.ndarray] = None,
                   out_bf16: Optional[bool] = None, overflow_priority: bool = False,
-                  renormalize: bool = False, gates_in: Optional[np.ndarray] = None) -> dict:
+                  renormalize: bool = False, probs_in: Optional[np.ndarray] = None) -> dict:
     """The whole layer on host arrays (``synth.make_inputs`` layout).
+
+    logits_in: [T,E] fp32 logits to route on instead of the oracle's own; probs_in: [T,k] fp32
+    softmax probabilities of the chosen experts (before any renormalisation) to rank and gate
+    with instead of the oracle's own.
 
     Returns dict: logits, ids, gates, slot, counts, C, f, Q, aux, out_exact [n,d] f64,
     out (rounded to the output type: uint16 bf16 bits or f32), tokens.
@@ -249,7 +254,7 @@ def layer_forward(inp: dict, T: int, d_model: int, d_ff: int, E: int, k: int,
     out = np.empty((n, d_model), dtype=np.uint16 if out_bf16 else np.float32)
     losses = np.empty(3, dtype=np.float64)
     li = None if logits_in is None else np.ascontiguousarray(logits_in, dtype=np.float32)
-    gi = None if gates_in is None else np.ascontiguousarray(gates_in, dtype=np.float32)
+    gi = None if probs_in is None else np.ascontiguousarray(probs_in, dtype=np.float32)
     g = inp.get
     C = L.oracle_layer_forward(
         T, d_model, d_ff, E, k, capacity_factor, bf16, int(bool(add_input_residual)),
@@ -272,7 +277,7 @@ def gelu_grad(z: float) -> float:
 def layer_backward(inp: dict, T: int, d_model: int, d_ff: int, E: int, k: int,
                    capacity_factor: float, dout: np.ndarray, add_input_residual: bool = True,
                    aux_alpha: float = 0.01, aux_weight: float = 0.0, z_weight: float = 0.0,
-                   logits_in: Optional[np.ndarray] = None, gates_in: Optional[np.ndarray] = None,
+                   logits_in: Optional[np.ndarray] = None, probs_in: Optional[np.ndarray] = None,
                    overflow_priority: bool = False, renormalize: bool = False) -> dict:
     """Gradients (float64) of L = sum(dout * out) + aux_weight * aux + z_weight * z_loss.
 
@@ -293,7 +298,7 @@ def layer_backward(inp: dict, T: int, d_model: int, d_ff: int, E: int, k: int,
                dense_dw2=np.empty((d, f)) if dense else None,
                dense_db2=np.empty(d) if dense else None)
     li = None if logits_in is None else np.ascontiguousarray(logits_in, dtype=np.float32)
-    gi = None if gates_in is None else np.ascontiguousarray(gates_in, dtype=np.float32)
+    gi = None if probs_in is None else np.ascontiguousarray(probs_in, dtype=np.float32)
     go = np.ascontiguousarray(dout, dtype=np.float64)
     L.oracle_layer_backward(
         T, d, f, E, k, capacity_factor, bf16, int(bool(add_input_residual)),

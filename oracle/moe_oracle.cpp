@@ -20,8 +20,10 @@
 //   (Switch-vs-DeepSpeed comparison article, section "Expert Capacity Overflow":
 //    capacity = (tokens in the batch / experts) x capacity factor).
 //
-// Readings of points the pages leave open (each is listed in the design notes):
-//   * capacity C = ceil(k * T * cf / E), evaluated in double in that order;
+// Readings of points the pages leave open:
+//   * capacity C = ceil(k * T / E * cf): the article's tokens-over-experts times the
+//     capacity factor, with the k choices counted; a product within rounding error above an
+//     integer is that integer (the capacity of the decimal factor);
 //   * overflow is first-come: slots are handed out in token order (t ascending,
 //     then the token's j-th choice), slot >= C is dropped;
 //   * gates are the unrenormalised softmax probabilities p_e;
@@ -163,9 +165,17 @@ void oracle_lb_stats(const float* logits, const int32_t* ids, int64_t T, int E, 
 
 // Capacity = (tokens in the batch / experts) x capacity factor (comparison article,
 // "Expert Capacity Overflow"), with the k choices of each token counted and rounded up:
-// C = ceil(k * T * cf / E).
+// C = ceil(k * T / E * cf). The factor is a decimal number held in binary (1.1 is stored a
+// little above 1.1), and the two operations round, so a product that lands within a few units
+// in the last place above an integer is that integer: the capacity the decimal factor means
+// (k = 1, T = 100, E = 10, cf = 1.1 gives 11, not 12).
 int64_t oracle_capacity(int64_t T, int E, int k, double capacity_factor) {
-  return (int64_t)std::ceil((double)k * (double)T * capacity_factor / (double)E);
+  const double share = (double)k * (double)T / (double)E;
+  const double v = share * capacity_factor;
+  const double below = std::floor(v);
+  const double ulp = std::nextafter(v, INFINITY) - v;
+  if (v - below <= 8.0 * ulp) return (int64_t)below;
+  return (int64_t)std::ceil(v);
 }
 
 // First-come slot assignment: walk the (token, choice) pairs in token order and give
@@ -185,17 +195,20 @@ void oracle_assign_slots(const int32_t* ids, int64_t T, int k, int E, int64_t C,
 
 // Priority overflow (a routing variant): inside each expert, the pairs are ranked by router
 // probability, highest first (equal probabilities: lower pair index first), and the first C
-// ranks are kept. The comparison article's capacity example ranks E0's tokens by probability
-// (t3 0.859 > t0 0.817 > t1 0.669) and keeps t3, t0, dropping t1. gates are the fp32 gate
-// values the ranking is decided on.
-void oracle_assign_slots_priority(const int32_t* ids, const float* gates, int64_t T, int k, int E,
+// ranks are kept. The comparison article's capacity example ranks E0's tokens by their router
+// probability (t3 0.859 > t0 0.817 > t1 0.669) and keeps t3, t0, dropping t1. probs are the
+// softmax probabilities p of each chosen expert, [T, k] fp32, before any renormalisation of the
+// gates: renormalising over a token's k choices changes what multiplies the expert output, not
+// how strongly the router prefers that token for the expert (at k = 1 every renormalised gate
+// is 1 and would carry no preference at all).
+void oracle_assign_slots_priority(const int32_t* ids, const float* probs, int64_t T, int k, int E,
                                   int64_t C, int32_t* slot, int32_t* counts) {
   std::vector<std::vector<int64_t>> members(E);
   for (int64_t p = 0; p < T * k; ++p) members[ids[p]].push_back(p);
   for (int e = 0; e < E; ++e) {
     std::vector<int64_t>& m = members[e];
     std::sort(m.begin(), m.end(), [&](int64_t a, int64_t b) {
-      if (gates[a] != gates[b]) return gates[a] > gates[b];
+      if (probs[a] != probs[b]) return probs[a] > probs[b];
       return a < b;
     });
     for (size_t r = 0; r < m.size(); ++r) slot[m[r]] = (int64_t)r < C ? (int32_t)r : -1;
@@ -303,6 +316,9 @@ void oracle_combine(int64_t T, int d, int k, const void* residual, int res_bf16,
 //
 // logits_in: if non-NULL these fp32 logits are used instead of computing them (routing
 //            decided from the same logits as another implementation).
+// probs_in:  if non-NULL, [T, k] fp32 softmax probabilities of the chosen experts (before any
+//            renormalisation) used instead of the oracle's own: the priority ranking key and,
+//            renormalised when asked, the gates.
 // tokens:    the tokens whose output rows are computed (NULL = all T, in order);
 //            routing, slots and statistics always cover all T tokens.
 // out_exact: [n, d] double before the final rounding; out_rounded: [n, d] in the output
@@ -317,7 +333,7 @@ int64_t oracle_layer_forward(int64_t T, int d, int d_ff, int E, int k, double ca
                              float* logits_out, int32_t* ids, float* gates, int32_t* slot,
                              int32_t* counts, double* lb_stats, double* out_exact,
                              void* out_rounded, int out_bf16, int overflow_priority,
-                             int renormalize, const float* gates_in, double* losses) {
+                             int renormalize, const float* probs_in, double* losses) {
   std::vector<float> logits_own;
   const float* logits = logits_in;
   if (!logits) {
@@ -327,14 +343,16 @@ int64_t oracle_layer_forward(int64_t T, int d, int d_ff, int E, int k, double ca
   }
   if (logits_out && logits_out != logits) std::memcpy(logits_out, logits, sizeof(float) * T * E);
   oracle_route(logits, T, E, k, ids, gates, nullptr);
+  // probs_in: the fp32 probabilities of the chosen experts another implementation computed (a
+  // priority ranking between two nearly equal probabilities is decided in that implementation's
+  // precision); NULL = the oracle's own
+  if (probs_in && probs_in != gates) std::memcpy(gates, probs_in, sizeof(float) * T * k);
+  const std::vector<float> probs(gates, gates + T * k);  // before any renormalisation
   if (renormalize) oracle_renormalize_gates(gates, T, k);
-  // gates_in: the gate values another implementation decided on (a priority ranking between two
-  // nearly equal probabilities is decided in that implementation's precision); NULL = own gates
-  if (gates_in && gates_in != gates) std::memcpy(gates, gates_in, sizeof(float) * T * k);
   if (lb_stats) oracle_lb_stats(logits, ids, T, E, k, aux_alpha, lb_stats, lb_stats + E, lb_stats + 2 * E);
   if (losses) oracle_router_losses(logits, ids, gates, T, E, k, losses, losses + 1, losses + 2);
   const int64_t C = oracle_capacity(T, E, k, capacity_factor);
-  if (overflow_priority) oracle_assign_slots_priority(ids, gates, T, k, E, C, slot, counts);
+  if (overflow_priority) oracle_assign_slots_priority(ids, probs.data(), T, k, E, C, slot, counts);
   else oracle_assign_slots(ids, T, k, E, C, slot, counts);
 
   const int64_t n = tokens ? n_tokens : T;
@@ -426,7 +444,7 @@ static void ffn_backward(const void* x_row, int bf16, int d, int d_ff, const voi
   }
 }
 
-// Gradients of the whole layer. Inputs are those of oracle_layer_forward (logits_in / gates_in
+// Gradients of the whole layer. Inputs are those of oracle_layer_forward (logits_in / probs_in
 // as there: routing decided on another implementation's fp32 values), plus dout [T, d] and the
 // weights of the two extra loss terms. Outputs (double, zeroed here, any may be NULL):
 // dx [T, d], dw_r [E, d], db_r [E], dw1 [E, d_ff, d], db1 [E, d_ff], dw2 [E, d, d_ff],
@@ -438,7 +456,7 @@ void oracle_layer_backward(int64_t T, int d, int d_ff, int E, int k, double capa
                            const void* b2, const void* dense_w1, const void* dense_b1,
                            const void* dense_w2, const void* dense_b2, double aux_alpha,
                            int overflow_priority, int renormalize, const float* logits_in,
-                           const float* gates_in, const double* dout, double aux_weight,
+                           const float* probs_in, const double* dout, double aux_weight,
                            double z_weight, double* dx, double* dw_r, double* db_r, double* dw1,
                            double* db1, double* dw2, double* db2, double* ddw1, double* ddb1,
                            double* ddw2, double* ddb2, double* dgates, double* dlogits) {
@@ -450,14 +468,14 @@ void oracle_layer_backward(int64_t T, int d, int d_ff, int E, int k, double capa
   std::vector<float> gates((size_t)T * k);
   std::vector<double> probs((size_t)T * E);
   oracle_route(logits.data(), T, E, k, ids.data(), gates.data(), probs.data());
+  if (probs_in) std::memcpy(gates.data(), probs_in, sizeof(float) * T * k);
   std::vector<float> raw = gates;  // the chosen p before any renormalisation
   if (renormalize) oracle_renormalize_gates(gates.data(), T, k);
-  if (gates_in) std::memcpy(gates.data(), gates_in, sizeof(float) * T * k);
   std::vector<double> f(E), Q(E);
   double aux = 0.0;
   oracle_lb_stats(logits.data(), ids.data(), T, E, k, aux_alpha, f.data(), Q.data(), &aux);
   const int64_t C = oracle_capacity(T, E, k, capacity_factor);
-  if (overflow_priority) oracle_assign_slots_priority(ids.data(), gates.data(), T, k, E, C, slot.data(), counts.data());
+  if (overflow_priority) oracle_assign_slots_priority(ids.data(), raw.data(), T, k, E, C, slot.data(), counts.data());
   else oracle_assign_slots(ids.data(), T, k, E, C, slot.data(), counts.data());
 
   auto zero = [](double* a, size_t n) { if (a) std::fill(a, a + n, 0.0); };

@@ -123,8 +123,34 @@ def test_capacity_page_example():
     (5, 2, 2, 1e9, 5000000000),
 ])
 def test_capacity_formula(T, E, k, cf, C):
-    # ceil(k * T * cf / E), values worked by hand
+    # ceil(k * T / E * cf), values worked by hand
     assert oracle.capacity(T, E, k, cf) == C
+
+
+@pytest.mark.parametrize("T,E,k,cf,C", [
+    (100, 10, 1, 1.1, 11), (1000, 100, 1, 1.1, 11), (30, 10, 1, 1.1, 4), (20, 10, 1, 1.15, 3),
+    (700, 10, 1, 0.7, 49), (300, 100, 1, 0.7, 3), (60, 20, 1, 1.1, 4), (8, 8, 1, 1.001, 2),
+])
+def test_capacity_decimal_factor(T, E, k, cf, C):
+    # a decimal factor held in binary (1.1 is stored slightly above 1.1) still gives the capacity
+    # of the decimal number: 100 tokens / 10 experts x 1.1 = 11 exactly, so C = 11, not 12
+    assert oracle.capacity(T, E, k, cf) == C
+
+
+def test_capacity_matches_exact_decimal_arithmetic():
+    # ceil(k T / E x cf) in exact rational arithmetic on the decimal factor, over a grid of shapes
+    from fractions import Fraction
+    rng = np.random.default_rng(11)
+    factors = ["1.0", "1.1", "1.2", "1.25", "1.5", "2.0", "0.5", "0.7", "1.3", "0.9", "1.05", "0.3",
+               "0.01", "3.3", "1.001", "1.123456"]
+    cases = [(T, E, k) for T in range(1, 130, 3) for E in (1, 2, 3, 7, 8, 10, 16, 64, 128)
+             for k in (1, 2)]
+    cases += [(int(rng.integers(1, 2 ** 30)), int(rng.integers(1, 1025)), int(rng.integers(1, 9)))
+              for _ in range(300)]
+    for T, E, k in cases:
+        for cf in factors:
+            exact = -((-Fraction(k * T, E) * Fraction(cf)).__floor__())
+            assert oracle.capacity(T, E, k, float(cf)) == exact, (T, E, k, cf)
 
 
 # ---------------------------------------------------------------- number formats

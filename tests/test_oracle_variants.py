@@ -60,6 +60,48 @@ def test_priority_overflow_page_example():
     assert counts.tolist() == g["demand"]
 
 
+def test_priority_overflow_page_example_with_renormalised_gates():
+    # the article ranks E0's tokens by router probability; renormalising a top-1 gate makes it
+    # 1.0 for every token, but the ranking still follows the probability: keep t3 and t0, drop t1
+    import synth
+    g = golden("capacity_overflow.json")
+    t = golden("top1_four_tokens.json")
+    logits = np.array(t["logits"], dtype=np.float32)
+    w = synth.Workload("page", T=4, d_model=8, d_ff=8, E=2, k=1, capacity_factor=1.0, dtype="f32",
+                       w_router_std=1.0, w_std=0.3, b_std=0.1, seed=3)
+    inp = synth.make_inputs(w)
+    for renorm in (False, True):
+        r = oracle.layer_forward(inp, 4, 8, 8, 2, 1, 1.0, logits_in=logits, overflow_priority=True,
+                                 renormalize=renorm)
+        assert [tk for tk in (3, 0, 1) if r["slot"][tk, 0] >= 0] == g["page_priority_order_kept_E0"]
+        assert [tk for tk in range(4) if r["slot"][tk, 0] < 0] == g["page_priority_order_dropped"]
+        assert r["slot"][3, 0] == 0 and r["slot"][0, 0] == 1 and r["slot"][2, 0] == 0
+        if renorm:
+            assert r["gates"].ravel().tolist() == [1.0, 1.0, 1.0, 1.0]
+
+
+def test_priority_ranks_by_probability_not_renormalised_gate():
+    # token 0 picks E0 (p 0.5) then E1 (p 0.4): renormalised E1 gate 0.4/0.9 = 0.444;
+    # token 1 picks E1 (p 0.35) then E2 (p 0.30): renormalised E1 gate 0.35/0.65 = 0.538.
+    # E1 has one place: by router probability token 0 (0.4 > 0.35) keeps it, although token 1's
+    # renormalised gate is the larger one.
+    import synth
+    p = np.array([[0.5, 0.4, 0.05, 0.05], [0.29, 0.35, 0.30, 0.06]])
+    logits = np.log(p).astype(np.float32)
+    w = synth.Workload("rank", T=2, d_model=8, d_ff=8, E=4, k=2, capacity_factor=0.5, dtype="f32",
+                       w_router_std=1.0, w_std=0.3, b_std=0.1, seed=4)
+    inp = synth.make_inputs(w)
+    r = oracle.layer_forward(inp, 2, 8, 8, 4, 2, 0.5, logits_in=logits, overflow_priority=True,
+                             renormalize=True)
+    assert r["C"] == 1
+    assert r["ids"].tolist() == [[0, 1], [1, 2]]
+    assert r["gates"][1, 0] > r["gates"][0, 1]          # renormalised: token 1's E1 gate is larger
+    assert r["slot"][0, 1] == 0 and r["slot"][1, 0] == -1  # but token 0 keeps E1's place
+    raw_ids, raw = oracle.route(logits, 2)
+    s2, _ = oracle.assign_slots_priority(raw_ids, raw, 4, 1)
+    assert np.array_equal(r["slot"], s2)
+
+
 def priority_brute(ids, gates, E, C):
     T, k = ids.shape
     slot = np.full((T, k), -1, dtype=np.int32)
@@ -111,10 +153,10 @@ def test_layer_with_variants_matches_composition():
     inp = synth.make_inputs(w)
     r = oracle.layer_forward(inp, w.T, w.d_model, w.d_ff, w.E, w.k, w.capacity_factor,
                              overflow_priority=True, renormalize=True)
-    ids, gates = oracle.route(r["logits"], 2)
-    gates = oracle.renormalize_gates(gates)
+    ids, probs = oracle.route(r["logits"], 2)
+    gates = oracle.renormalize_gates(probs)
     assert np.array_equal(r["gates"], gates)
-    slot, _ = oracle.assign_slots_priority(ids, gates, 4, r["C"])
+    slot, _ = oracle.assign_slots_priority(ids, probs, 4, r["C"])
     assert np.array_equal(r["slot"], slot)
     z, ci, cl = oracle.router_losses(r["logits"], ids, gates)
     assert (r["z_loss"], r["cov2_importance"], r["cov2_load"]) == (z, ci, cl)
