@@ -46,7 +46,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 2
+#define MOE_ABI_VERSION 3
 #define MOE_STATUS_BLOCK_BYTES 256
 #define MOE_MAX_EXPERTS 1024
 #define MOE_MAX_TOPK 8
@@ -81,8 +81,11 @@ int moe_abi_version(void);
 /* ---------------------------------------------------------------- sizes
  * Expert capacity (Switch/DeepSpeed comparison article, section "Expert Capacity Overflow":
  * capacity = (tokens in the batch / experts) x capacity factor), with the k choices of
- * each token counted and rounded up: C = ceil(k * T * capacity_factor / E), evaluated in double
- * in that order. capacity_factor must be finite and >= 0. */
+ * each token counted and rounded up: C = ceil(k * T / E * capacity_factor). The product is
+ * formed in double in that order; one that lies within 8 units in the last place above an
+ * integer counts as that integer, so a decimal factor gives the capacity the decimal number
+ * means (T = 100, E = 10, k = 1, capacity_factor = 1.1 gives 11, although 1.1 is stored a
+ * little above 1.1). capacity_factor must be finite and >= 0. */
 moe_status moe_capacity(int64_t T, int E, int k, double capacity_factor, int64_t* C_out);
 
 /* Rows of the expert-major packed buffers: min(T * k, E * C). Kept rows of expert e occupy
@@ -107,6 +110,20 @@ moe_status moe_packed_rows_max(int64_t T, int E, int k, int64_t C, int64_t* rows
  * Limits: 1 <= E <= 1024, 1 <= k <= min(E, 8), T >= 0 (T == 0 enqueues nothing), d_model >= 1;
  * bf16 x needs d_model % 8 == 0. */
 moe_status moe_router_workspace_bytes(int64_t T, int E, int d_model, size_t* bytes);
+
+/* The router weight prepared for the tensor-core logits kernel: W_r (fp32) split exactly into
+ * three bf16 parts hi + mid + lo = W_r (each holds the next 8 significant bits), stored
+ * [E, 3 * ceil64(d_model)]. The router entry points split W_r on every call; a caller that keeps
+ * W_r fixed between calls (inference, or between optimizer steps) prepares it once per weight
+ * version with moe_router_prepare and passes it as moe_layer_args.w_router_prepared, which
+ * saves one launch per layer call. The prepared buffer is caller-owned device memory of
+ * moe_router_prepare_bytes bytes; it must be prepared again whenever W_r changes (the library
+ * cannot see a change). Prepared weights only serve bf16 x with d_model % 8 == 0 and T > 64
+ * (the tensor-core path); elsewhere they are ignored and W_r is used directly. */
+moe_status moe_router_prepare_bytes(int E, int d_model, size_t* bytes);
+moe_status moe_router_prepare(const float* w_router, int E, int d_model, void* w_prepared,
+                              size_t bytes, moe_stream_t stream);
+
 moe_status moe_router_topk(const void* x, moe_dtype x_dtype, int64_t T, int d_model,
                            const float* w_router, const float* router_bias, int E, int k,
                            float* logits, int32_t* expert_ids, float* gates, float* lb_stats,
@@ -115,6 +132,9 @@ moe_status moe_router_topk(const void* x, moe_dtype x_dtype, int64_t T, int d_mo
 /* moe_router_topk with two routing variants (same workspace):
  * renormalize != 0: gates[t,j] = p[t,e_j] / sum_{j'} p[t,e_j'] (the k chosen probabilities
  *               renormalised to sum to 1: MoE survey notes §1.1.1.1, top-k after the softmax).
+ * probs (NULL or [T, k] fp32 output): p[t, expert_ids[t,j]], the softmax probability of each
+ *               choice before any renormalisation (equal to gates when renormalize == 0); the
+ *               ranking key of moe_dispatch_priority.
  * router_losses (NULL or [3] fp32 output):
  *   [0] z-loss = (1/T) sum_t (log sum_e exp(logits[t,e]))^2 (comparison article, "Router
  *       Z-loss"; without the coefficient);
@@ -125,8 +145,8 @@ moe_status moe_router_topk(const void* x, moe_dtype x_dtype, int64_t T, int d_mo
 moe_status moe_router_topk_ex(const void* x, moe_dtype x_dtype, int64_t T, int d_model,
                               const float* w_router, const float* router_bias, int E, int k,
                               float* logits, int32_t* expert_ids, float* gates, float* lb_stats,
-                              float aux_alpha, int renormalize, float* router_losses, void* ws,
-                              size_t ws_bytes, moe_stream_t stream);
+                              float aux_alpha, int renormalize, float* router_losses,
+                              float* probs, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* ---------------------------------------------------------------- dispatch
  * pack_by_expert with a capacity (DeepSpeed MoE blog, pipeline listing; DeepSpeed-MoE notes
@@ -149,13 +169,16 @@ moe_status moe_dispatch(const void* x, moe_dtype dtype, int64_t T, int d_model,
                         moe_stream_t stream);
 
 /* moe_dispatch with overflow by priority (comparison article, "Expert Capacity Overflow": the
- * tokens of highest router probability keep the capacity): the pairs of each expert are ranked
- * by gate, largest first, ties to the lower pair index p = t * k + j; slot[t,j] = rank if
- * rank < C, else -1, and kept rows are packed in rank order. gates: [T, k] fp32 (the router's,
- * renormalised or not). Counts, offsets, row_token and x_packed follow moe_dispatch. Same
- * workspace as moe_dispatch. */
+ * example ranks an expert's tokens by router probability and keeps the most probable): the
+ * pairs of each expert are ranked by probs, largest first, ties to the lower pair index
+ * p = t * k + j; slot[t,j] = rank if rank < C, else -1, and kept rows are packed in rank order.
+ * probs: [T, k] fp32, the softmax probability of each choice BEFORE any renormalisation
+ * (moe_router_topk's gates, or moe_router_topk_ex's probs output): renormalised top-1 gates are
+ * all 1 and carry no preference. Finite values; the order is that of the fp32 numbers.
+ * Counts, offsets, row_token and x_packed follow moe_dispatch. Same workspace as moe_dispatch.
+ * Cost: O(n log^2 n) per expert of demand n (chunk ranks, then merge passes). */
 moe_status moe_dispatch_priority(const void* x, moe_dtype dtype, int64_t T, int d_model,
-                                 const int32_t* expert_ids, const float* gates, int E, int k,
+                                 const int32_t* expert_ids, const float* probs, int E, int k,
                                  int64_t C, int32_t* slot, int32_t* expert_counts,
                                  int32_t* expert_offsets, int32_t* row_token, void* x_packed,
                                  int64_t rows_max, void* ws, size_t ws_bytes,
@@ -171,8 +194,10 @@ moe_status moe_dispatch_priority(const void* x, moe_dtype dtype, int64_t T, int 
  * library holds until the process exits. Larger problems return MOE_ERR_WORKSPACE_TOO_SMALL
  * (use moe_dispatch with a workspace instead). Arguments, outputs and results are those of
  * moe_dispatch, except that no status block exists: ids outside [0, E) become dropped pairs
- * without a device error code. The first call on each device (with that device current) looks
- * up the array's device address; make that first call before any stream capture begins.
+ * without a device error code. Each call looks up the array's device address on the current
+ * device, except a call whose stream is being captured, which reuses the address an earlier call
+ * on that device found: make the first call on each device before any stream capture begins
+ * (after a device reset, too, the first call must come before a capture).
  * Nothing in the array needs to start at zero (every element read is written first in the same
  * call), but all calls share it: calls that overlap on the GPU race and must be serialised. */
 #define MOE_NOALLOC_SCRATCH_BYTES (4u << 20)
@@ -248,10 +273,13 @@ typedef struct {
   float aux_alpha;        /* alpha of the load-balance loss */
   int overflow_policy;    /* moe_overflow_policy */
   int renormalize_gates;  /* 1: gates renormalised over the k choices (moe_router_topk_ex) */
+  /* w_router split by moe_router_prepare (NULL: split on every call inside the workspace) */
+  const void* w_router_prepared;
 } moe_layer_args;
 
 /* Which pairs an expert keeps when its demand exceeds C: the first in token order (moe_dispatch),
- * or those of largest gate (moe_dispatch_priority). */
+ * or those of largest router probability (moe_dispatch_priority; the probability before any
+ * renormalisation of the gates). */
 typedef enum { MOE_OVERFLOW_FIRST_COME = 0, MOE_OVERFLOW_PRIORITY = 1 } moe_overflow_policy;
 
 /* Optional device outputs of the intermediate results; any field may be NULL. */
@@ -264,6 +292,7 @@ typedef struct {
   int32_t* expert_offsets;/* [E+1] */
   float* lb_stats;        /* [2E+1] */
   float* router_losses;   /* [3]: z-loss, CoV^2 Importance, CoV^2 Load (moe_router_topk_ex) */
+  float* topk_probs;      /* [T, k]: softmax probability of each choice before renormalisation */
 } moe_layer_aux;
 
 /* out = [x if add_input_residual] + [DenseMLP(x) if dense_*] + sum_j gate_j * Expert_{e_j}(x)
@@ -370,6 +399,19 @@ moe_status moe_get_device_error(const void* ws, int* code_out, moe_stream_t stre
 /* Number of kernel launches the last successful call of each entry point enqueued on this host
  * thread (for launch accounting in benchmarks). */
 int moe_last_launch_count(void);
+
+/* ---------------------------------------------------------------- failure-detection self-test
+ * Checks, on the caller's GPU, that a kernel whose wait can never complete gives up instead of
+ * hanging (no counterpart on the pages: it tests the library's own failure detection). Launches
+ * the grouped expert GEMM once on a one-tile problem whose TMA role is told to issue no copy, so
+ * the MMA role waits on a barrier that nobody arrives at. Every wait of that launch gives up after
+ * wait_limit_ns (1000 <= wait_limit_ns <= 10^10), MOE_DEVERR_TIMEOUT is recorded in the status
+ * block of ws, the roles stop, TMEM is freed and the kernel returns; nothing else in ws is read
+ * or written, and the context stays usable. Read the result with moe_get_device_error.
+ * ws: >= MOE_SELFTEST_WS_BYTES bytes, 256-byte aligned, status block zeroed by the caller. */
+#define MOE_SELFTEST_WS_BYTES (256u + 32768u)
+moe_status moe_selftest_bounded_wait(void* ws, size_t ws_bytes, uint64_t wait_limit_ns,
+                                     moe_stream_t stream);
 
 #ifdef __cplusplus
 }

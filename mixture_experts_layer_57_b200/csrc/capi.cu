@@ -26,6 +26,14 @@ bool pdl_enabled() {
   return on;
 }
 
+// Whether bf16 PR-MoE layers co-schedule each expert GEMM layer with the dense MLP's layer in one
+// launch (MOE_COSCHEDULE=0 runs them one after another, the dense layer 2 with the combine fused;
+// both give the same bits). Read at every call.
+bool coschedule_enabled() {
+  const char* v = std::getenv("MOE_COSCHEDULE");
+  return !(v != nullptr && v[0] == '0');
+}
+
 int num_sms() {
   static int cache[64] = {0};
   int dev = 0;
@@ -93,7 +101,8 @@ RouterWs carve_router(Carve& c, int64_t T, int E, int d) {
 
 struct DispatchWs {
   int32_t *local_rank, *seg_counts, *seg_base;
-  int32_t *prio_list, *demand_offsets;  // overflow by priority
+  uint64_t* prio_keys;       // overflow by priority: [2 T k] ping-pong sort keys
+  int32_t* demand_offsets;   // overflow by priority: [E + 1]
 };
 DispatchWs carve_dispatch(Carve& c, int64_t T, int E, int k) {
   // segments of 256 pairs (counting kernel) or of one 64-token router block (layer forward)
@@ -104,7 +113,7 @@ DispatchWs carve_dispatch(Carve& c, int64_t T, int E, int k) {
   w.local_rank = c.take<int32_t>((size_t)T * k);
   w.seg_counts = c.take<int32_t>((size_t)nseg * E);
   w.seg_base = c.take<int32_t>((size_t)nseg * E);
-  w.prio_list = c.take<int32_t>((size_t)T * k);
+  w.prio_keys = c.take<uint64_t>((size_t)2 * T * k);
   w.demand_offsets = c.take<int32_t>((size_t)E + 1);
   return w;
 }
@@ -153,10 +162,24 @@ int moe_abi_version(void) { return MOE_ABI_VERSION; }
 
 int moe_last_launch_count(void) { return g_launches; }
 
+moe_status moe_selftest_bounded_wait(void* ws, size_t ws_bytes, uint64_t wait_limit_ns,
+                                     moe_stream_t stream) {
+  if (!ws || wait_limit_ns < 1000 || wait_limit_ns > 10000000000ull) return MOE_ERR_INVALID_ARGUMENT;
+  if (((uintptr_t)ws % kAlign) != 0) return MOE_ERR_MISALIGNED;
+  if (ws_bytes < MOE_SELFTEST_WS_BYTES) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  g_launches = 0;
+  return cuda_status(enqueue_selftest_bounded_wait((uint8_t*)ws + kAlign, wait_limit_ns, (int*)ws,
+                                                   stream));
+}
+
 moe_status moe_capacity(int64_t T, int E, int k, double capacity_factor, int64_t* C_out) {
   if (!C_out || T < 0 || E < 1 || k < 1 || !std::isfinite(capacity_factor) || capacity_factor < 0)
     return MOE_ERR_INVALID_ARGUMENT;
-  const double c = std::ceil((double)k * (double)T * capacity_factor / (double)E);
+  // k T / E first, then the factor; a product within 8 ulps above an integer is that integer
+  // (the factor is a decimal number held in binary, e.g. 1.1 is stored slightly above 1.1)
+  const double v = ((double)k * (double)T / (double)E) * capacity_factor;
+  const double fl = std::floor(v);
+  const double c = (v - fl <= 8.0 * (std::nextafter(v, INFINITY) - v)) ? fl : std::ceil(v);
   if (c > 9.0e18) return MOE_ERR_UNSUPPORTED;
   *C_out = (int64_t)c;
   return MOE_OK;
@@ -185,7 +208,8 @@ moe_status router_topk_impl(const char* entry, const void* x, moe_dtype x_dtype,
                             int d_model, const float* w_router, const float* router_bias, int E,
                             int k, float* logits, int32_t* expert_ids, float* gates,
                             float* lb_stats, float aux_alpha, int renormalize,
-                            float* router_losses, void* ws, size_t ws_bytes, moe_stream_t stream) {
+                            float* router_losses, float* probs, void* ws, size_t ws_bytes,
+                            moe_stream_t stream) {
   if (!valid_dtype(x_dtype)) return MOE_ERR_INVALID_ARGUMENT;
   moe_status st = check_router_shape(T, d_model, E, k);
   if (st != MOE_OK) return st;
@@ -193,7 +217,7 @@ moe_status router_topk_impl(const char* entry, const void* x, moe_dtype x_dtype,
   if (!ws) return MOE_ERR_INVALID_ARGUMENT;
   if (!aligned16(x) || !aligned16(w_router) || !aligned16(router_bias) || !aligned16(logits) ||
       !aligned16(expert_ids) || !aligned16(gates) || !aligned16(lb_stats) ||
-      !aligned16(router_losses) || ((uintptr_t)ws % kAlign) != 0)
+      !aligned16(router_losses) || !aligned16(probs) || ((uintptr_t)ws % kAlign) != 0)
     return MOE_ERR_MISALIGNED;
   size_t need = 0;
   moe_router_workspace_bytes(T, E, d_model, &need);
@@ -206,27 +230,47 @@ moe_status router_topk_impl(const char* entry, const void* x, moe_dtype x_dtype,
   return cuda_status(enqueue_router(x, x_dtype == MOE_BF16, T, d_model, w_router, router_bias, E,
                                     k, logits, expert_ids, gates, lb_stats, aux_alpha, w.scr,
                                     (int*)ws, stream, RouterDispatchCount{}, renormalize != 0,
-                                    router_losses));
+                                    router_losses, nullptr, -1, probs));
 }
 }  // namespace
+
+moe_status moe_router_prepare_bytes(int E, int d_model, size_t* bytes) {
+  if (!bytes || E < 1 || d_model < 1) return MOE_ERR_INVALID_ARGUMENT;
+  if (E > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+  *bytes = (size_t)E * 3 * router_split_dpad(d_model) * sizeof(uint16_t);
+  return MOE_OK;
+}
+
+moe_status moe_router_prepare(const float* w_router, int E, int d_model, void* w_prepared,
+                              size_t bytes, moe_stream_t stream) {
+  size_t need = 0;
+  moe_status st = moe_router_prepare_bytes(E, d_model, &need);
+  if (st != MOE_OK) return st;
+  if (!w_router || !w_prepared) return MOE_ERR_INVALID_ARGUMENT;
+  if (!aligned16(w_router) || !aligned16(w_prepared)) return MOE_ERR_MISALIGNED;
+  if (bytes < need) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (fault_injected("moe_router_prepare")) return MOE_ERR_CUDA;
+  g_launches = 0;
+  return cuda_status(enqueue_router_prepare(w_router, E, d_model, (uint16_t*)w_prepared, stream));
+}
 
 moe_status moe_router_topk(const void* x, moe_dtype x_dtype, int64_t T, int d_model,
                            const float* w_router, const float* router_bias, int E, int k,
                            float* logits, int32_t* expert_ids, float* gates, float* lb_stats,
                            float aux_alpha, void* ws, size_t ws_bytes, moe_stream_t stream) {
   return router_topk_impl("moe_router_topk", x, x_dtype, T, d_model, w_router, router_bias, E, k,
-                          logits, expert_ids, gates, lb_stats, aux_alpha, 0, nullptr, ws,
+                          logits, expert_ids, gates, lb_stats, aux_alpha, 0, nullptr, nullptr, ws,
                           ws_bytes, stream);
 }
 
 moe_status moe_router_topk_ex(const void* x, moe_dtype x_dtype, int64_t T, int d_model,
                               const float* w_router, const float* router_bias, int E, int k,
                               float* logits, int32_t* expert_ids, float* gates, float* lb_stats,
-                              float aux_alpha, int renormalize, float* router_losses, void* ws,
-                              size_t ws_bytes, moe_stream_t stream) {
+                              float aux_alpha, int renormalize, float* router_losses,
+                              float* probs, void* ws, size_t ws_bytes, moe_stream_t stream) {
   return router_topk_impl("moe_router_topk_ex", x, x_dtype, T, d_model, w_router, router_bias, E,
                           k, logits, expert_ids, gates, lb_stats, aux_alpha, renormalize,
-                          router_losses, ws, ws_bytes, stream);
+                          router_losses, probs, ws, ws_bytes, stream);
 }
 
 // ---------------------------------------------------------------- dispatch
@@ -241,7 +285,7 @@ moe_status moe_dispatch_workspace_bytes(int64_t T, int E, int k, size_t* bytes) 
 
 namespace {
 moe_status dispatch_impl(const char* entry, const void* x, moe_dtype dtype, int64_t T,
-                         int d_model, const int32_t* expert_ids, const float* prio_gates, int E,
+                         int d_model, const int32_t* expert_ids, const float* prio_probs, int E,
                          int k, int64_t C, int32_t* slot, int32_t* expert_counts,
                          int32_t* expert_offsets, int32_t* row_token, void* x_packed,
                          int64_t rows_max, void* ws, size_t ws_bytes, moe_stream_t stream) {
@@ -258,7 +302,7 @@ moe_status dispatch_impl(const char* entry, const void* x, moe_dtype dtype, int6
   if (rows_max > 0 && (!row_token || !x_packed)) return MOE_ERR_INVALID_ARGUMENT;
   if (!aligned16(x) || !aligned16(expert_ids) || !aligned16(slot) || !aligned16(expert_counts) ||
       !aligned16(expert_offsets) || !aligned16(row_token) || !aligned16(x_packed) ||
-      !aligned16(prio_gates) || ((uintptr_t)ws % kAlign) != 0)
+      !aligned16(prio_probs) || ((uintptr_t)ws % kAlign) != 0)
     return MOE_ERR_MISALIGNED;
   size_t need = 0;
   moe_dispatch_workspace_bytes(T, E, k, &need);
@@ -268,8 +312,8 @@ moe_status dispatch_impl(const char* entry, const void* x, moe_dtype dtype, int6
   Carve c{(uint8_t*)ws};
   DispatchWs w = carve_dispatch(c, T, E, k);
   PriorityDispatch prio;
-  prio.gates = prio_gates;
-  prio.list = w.prio_list;
+  prio.probs = prio_probs;
+  prio.keys = w.prio_keys;
   prio.demand_offsets = w.demand_offsets;
   return cuda_status(enqueue_dispatch(x, dtype == MOE_BF16, T, d_model, expert_ids, E, k, C, slot,
                                       expert_counts, expert_offsets, row_token, x_packed, rows_max,
@@ -289,14 +333,14 @@ moe_status moe_dispatch(const void* x, moe_dtype dtype, int64_t T, int d_model,
 }
 
 moe_status moe_dispatch_priority(const void* x, moe_dtype dtype, int64_t T, int d_model,
-                                 const int32_t* expert_ids, const float* gates, int E, int k,
+                                 const int32_t* expert_ids, const float* probs, int E, int k,
                                  int64_t C, int32_t* slot, int32_t* expert_counts,
                                  int32_t* expert_offsets, int32_t* row_token, void* x_packed,
                                  int64_t rows_max, void* ws, size_t ws_bytes,
                                  moe_stream_t stream) {
-  if (T > 0 && !gates) return MOE_ERR_INVALID_ARGUMENT;
+  if (T > 0 && !probs) return MOE_ERR_INVALID_ARGUMENT;
   return dispatch_impl("moe_dispatch_priority", x, dtype, T, d_model, expert_ids,
-                       T > 0 ? gates : nullptr, E, k, C, slot, expert_counts, expert_offsets,
+                       T > 0 ? probs : nullptr, E, k, C, slot, expert_counts, expert_offsets,
                        row_token, x_packed, rows_max, ws, ws_bytes, stream);
 }
 
@@ -399,7 +443,7 @@ namespace {
 struct LayerWs {
   RouterWs router;
   DispatchWs dispatch;
-  float *gates, *lb_stats;
+  float *gates, *probs, *lb_stats;
   int32_t *ids, *slot, *counts, *offsets, *row_token;
   void *x_packed, *h_packed;
   float* y_packed;
@@ -433,6 +477,7 @@ moe_status layer_layout(const moe_layer_args* a, uint8_t* base, LayerWs* w, size
   w->router = carve_router(c, T, E, d);
   w->dispatch = carve_dispatch(c, T, E, k);
   w->gates = c.take<float>((size_t)T * k);
+  w->probs = c.take<float>((size_t)T * k);
   w->lb_stats = c.take<float>((size_t)2 * E + 1);
   w->ids = c.take<int32_t>((size_t)T * k);
   w->slot = c.take<int32_t>((size_t)T * k);
@@ -445,8 +490,10 @@ moe_status layer_layout(const moe_layer_args* a, uint8_t* base, LayerWs* w, size
   w->y_packed = c.take<float>((size_t)R * d);
   const bool dense = a->dense_w1 != nullptr;
   w->h_dense = dense ? (void*)c.take<uint8_t>((size_t)T * f * es) : nullptr;
-  // the fp32 layers' dense output; bf16 layers fuse it into the combine epilogue
-  w->r_dense = (dense && a->dtype != MOE_BF16) ? c.take<float>((size_t)T * d) : nullptr;
+  // the dense MLP's fp32 output, read by the combine kernel (fp32 layers, and bf16 layers whose
+  // dense layers are co-scheduled with the experts'; otherwise the combine is fused into the
+  // dense layer 2 epilogue)
+  w->r_dense = dense ? c.take<float>((size_t)T * d) : nullptr;
   *bytes = c.off;
   return MOE_OK;
 }
@@ -517,12 +564,13 @@ moe_status layer_forward_impl(const moe_layer_args* a, void* out, moe_layer_aux*
   if (!aligned16(a->x) || !aligned16(a->w_router) || !aligned16(a->router_bias) ||
       !aligned16(a->w1) || !aligned16(a->b1) || !aligned16(a->w2) || !aligned16(a->b2) ||
       !aligned16(a->dense_w1) || !aligned16(a->dense_b1) || !aligned16(a->dense_w2) ||
-      !aligned16(a->dense_b2) || !aligned16(out) || ((uintptr_t)ws % kAlign) != 0)
+      !aligned16(a->dense_b2) || !aligned16(out) || !aligned16(a->w_router_prepared) ||
+      ((uintptr_t)ws % kAlign) != 0)
     return MOE_ERR_MISALIGNED;
   if (aux && (!aligned16(aux->logits) || !aligned16(aux->expert_ids) || !aligned16(aux->gates) ||
               !aligned16(aux->slot) || !aligned16(aux->expert_counts) ||
               !aligned16(aux->expert_offsets) || !aligned16(aux->lb_stats) ||
-              !aligned16(aux->router_losses)))
+              !aligned16(aux->router_losses) || !aligned16(aux->topk_probs)))
     return MOE_ERR_MISALIGNED;
   if (ws_bytes < need) return MOE_ERR_WORKSPACE_TOO_SMALL;
   const char* entry = sh.mode == kShardBegin ? "moe_layer_forward_shard_begin"
@@ -561,6 +609,13 @@ moe_status layer_forward_impl(const moe_layer_args* a, void* out, moe_layer_aux*
   int32_t* offsets = aux && aux->expert_offsets ? aux->expert_offsets : w.offsets;
   float* lb = aux ? aux->lb_stats : nullptr;
   float* losses = aux ? aux->router_losses : nullptr;
+  // the priority ranking key: the probabilities before renormalisation (the gates themselves
+  // when they are not renormalised)
+  const bool prio_on = a->overflow_policy == MOE_OVERFLOW_PRIORITY;
+  float* probs = aux && aux->topk_probs ? aux->topk_probs
+                 : (prio_on && a->renormalize_gates) ? w.probs
+                                                     : nullptr;
+  const float* prio_key = a->renormalize_gates ? probs : gates;
   int* status = (int*)ws;
   const bool bf16 = a->dtype == MOE_BF16;
   const int64_t T = a->T;
@@ -579,7 +634,8 @@ moe_status layer_forward_impl(const moe_layer_args* a, void* out, moe_layer_aux*
     e = enqueue_router(a->x, bf16, T, d, a->w_router, a->router_bias, E, k, logits, ids, gates,
                        begin ? nullptr : lb, a->aux_alpha, w.router.scr, status, stream, dcount,
                        a->renormalize_gates != 0, begin ? nullptr : losses,
-                       begin ? sh.partials_out : nullptr, sh.T_global);
+                       begin ? sh.partials_out : nullptr, sh.T_global, probs,
+                       (const uint16_t*)a->w_router_prepared);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     rec.mark("router");
   }
@@ -618,9 +674,9 @@ moe_status layer_forward_impl(const moe_layer_args* a, void* out, moe_layer_aux*
     dropped.add_x = a->add_input_residual != 0;
   }
   PriorityDispatch prio;
-  if (a->overflow_policy == MOE_OVERFLOW_PRIORITY) {
-    prio.gates = gates;
-    prio.list = w.dispatch.prio_list;
+  if (prio_on) {
+    prio.probs = prio_key;
+    prio.keys = w.dispatch.prio_keys;
     prio.demand_offsets = w.dispatch.demand_offsets;
   }
   e = enqueue_dispatch(a->x, bf16, T, d, ids, E, k, w.C, slot, counts, offsets, w.row_token,
@@ -644,6 +700,27 @@ moe_status layer_forward_impl(const moe_layer_args* a, void* out, moe_layer_aux*
   fc.k = k;
   fc.E_experts = E;
 
+  // the tile width follows the whole batch, so a shard's rows get the whole batch's arithmetic
+  const int64_t dense_hint = sh.T_global > T ? sh.T_global : T;
+  if (fuse_dense && coschedule_enabled() && co_gemm_supported(w.C) && dense_hint >= 256) {
+    // each expert layer co-scheduled with the dense MLP's layer (one launch per layer), then the
+    // gather combine: out = [x] + dense + sum_j gate_j y_j, the fused epilogue's arithmetic
+    e = enqueue_co_gemm_bf16(w.x_packed, offsets, E, w.rows_max, a->w1, a->b1, w.h_packed, w.C,
+                             a->x, T, a->dense_w1, a->dense_b1, w.h_dense, d, f, true, status,
+                             stream);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    rec.mark("experts_dense_gemm1");
+    e = enqueue_co_gemm_bf16(w.h_packed, offsets, E, w.rows_max, a->w2, a->b2, w.y_packed, w.C,
+                             w.h_dense, T, a->dense_w2, a->dense_b2, w.r_dense, f, d, false, status,
+                             stream);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    rec.mark("experts_dense_gemm2");
+    e = enqueue_combine(w.y_packed, offsets, ids, slot, gates, T, d, E, k, w.rows_max, residual,
+                        bf16, w.r_dense, out, out_bf16, status, stream);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    rec.mark("combine");
+    return MOE_OK;
+  }
   if (fuse_dense) {
     if (w.rows_max > 0) {
       e = enqueue_grouped_gemm_bf16(w.x_packed, offsets, E, w.rows_max, d, f, a->w1, a->b1, true,
@@ -655,8 +732,6 @@ moe_status layer_forward_impl(const moe_layer_args* a, void* out, moe_layer_aux*
       if (e != cudaSuccess) return MOE_ERR_CUDA;
       rec.mark("expert_gemm2");
     }
-    // the tile width follows the whole batch, so a shard's rows get the whole batch's arithmetic
-    const int64_t dense_hint = sh.T_global > T ? sh.T_global : T;
     e = enqueue_grouped_gemm_bf16(a->x, nullptr, 1, T, d, f, a->dense_w1, a->dense_b1, true,
                                   w.h_dense, dense_hint, status, stream);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
@@ -897,7 +972,8 @@ moe_status check_layer_pointers(const moe_layer_args* a, const void* out, const 
   if (!aligned16(a->x) || !aligned16(a->w_router) || !aligned16(a->router_bias) ||
       !aligned16(a->w1) || !aligned16(a->b1) || !aligned16(a->w2) || !aligned16(a->b2) ||
       !aligned16(a->dense_w1) || !aligned16(a->dense_b1) || !aligned16(a->dense_w2) ||
-      !aligned16(a->dense_b2) || !aligned16(out) || ((uintptr_t)ws % kAlign) != 0)
+      !aligned16(a->dense_b2) || !aligned16(out) || !aligned16(a->w_router_prepared) ||
+      ((uintptr_t)ws % kAlign) != 0)
     return MOE_ERR_MISALIGNED;
   return MOE_OK;
 }
@@ -913,7 +989,7 @@ moe_status forward_train_impl(const moe_layer_args* a, void* out, moe_layer_aux*
   if (aux && (!aligned16(aux->logits) || !aligned16(aux->expert_ids) || !aligned16(aux->gates) ||
               !aligned16(aux->slot) || !aligned16(aux->expert_counts) ||
               !aligned16(aux->expert_offsets) || !aligned16(aux->lb_stats) ||
-              !aligned16(aux->router_losses)))
+              !aligned16(aux->router_losses) || !aligned16(aux->topk_probs)))
     return MOE_ERR_MISALIGNED;
   if (ws_bytes < need) return MOE_ERR_WORKSPACE_TOO_SMALL;
   if (fault_injected("moe_layer_forward_train")) return MOE_ERR_CUDA;
@@ -932,12 +1008,13 @@ moe_status forward_train_impl(const moe_layer_args* a, void* out, moe_layer_aux*
   cudaError_t e = enqueue_router(a->x, bf16, T, d, a->w_router, a->router_bias, E, k,
                                  L.router.logits, L.ids, L.gates, L.lb_stats, a->aux_alpha,
                                  L.router.scr, status, stream, dcount, a->renormalize_gates != 0,
-                                 aux ? aux->router_losses : nullptr);
+                                 aux ? aux->router_losses : nullptr, nullptr, -1, L.probs,
+                                 (const uint16_t*)a->w_router_prepared);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   PriorityDispatch prio;
   if (a->overflow_policy == MOE_OVERFLOW_PRIORITY) {
-    prio.gates = L.gates;
-    prio.list = L.dispatch.prio_list;
+    prio.probs = L.probs;  // before renormalisation
+    prio.keys = L.dispatch.prio_keys;
     prio.demand_offsets = L.dispatch.demand_offsets;
   }
   e = enqueue_dispatch(a->x, bf16, T, d, L.ids, E, k, L.C, L.slot, L.counts, L.offsets,
@@ -996,7 +1073,8 @@ moe_status forward_train_impl(const moe_layer_args* a, void* out, moe_layer_aux*
         (st = copy_out(aux->expert_counts, L.counts, sizeof(int32_t) * E, stream)) != MOE_OK ||
         (st = copy_out(aux->expert_offsets, L.offsets, sizeof(int32_t) * (E + 1), stream)) !=
             MOE_OK ||
-        (st = copy_out(aux->lb_stats, L.lb_stats, sizeof(float) * (2 * E + 1), stream)) != MOE_OK)
+        (st = copy_out(aux->lb_stats, L.lb_stats, sizeof(float) * (2 * E + 1), stream)) != MOE_OK ||
+        (st = copy_out(aux->topk_probs, L.probs, sizeof(float) * T * k, stream)) != MOE_OK)
       return st;
   }
   return MOE_OK;

@@ -89,11 +89,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete. Gives up after kWaitLimitNs or as soon
-// as *abort is set by another role of the same CTA; on giving up it records
-// MOE_DEVERR_TIMEOUT (first time only), raises *abort and returns false.
+// Wait for the phase with the given parity to complete. Gives up after `limit_ns` (default
+// kWaitLimitNs) or as soon as *abort is set by another role of the same CTA; on giving up it
+// records MOE_DEVERR_TIMEOUT (first time only), raises *abort and returns false.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
-                                                  volatile int* abort, int* status) {
+                                                  volatile int* abort, int* status,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
 #pragma unroll 1
   for (int i = 0; i < 256; ++i)
     if (mbar_try_wait(bar, parity)) return true;
@@ -102,7 +103,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+    if (global_timer_ns() - t0 > limit_ns) {
       set_device_error(status, MOE_DEVERR_TIMEOUT);
       *abort = 1;
       return false;
@@ -115,14 +116,15 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
 // phase stays completed until this warp itself lets the next phase start, so readiness is
 // monotone and __all_sync converges.
 __device__ __forceinline__ bool mbar_wait_bounded_warp(uint32_t bar, uint32_t parity,
-                                                       volatile int* abort, int* status) {
+                                                       volatile int* abort, int* status,
+                                                       uint64_t limit_ns = kWaitLimitNs) {
   const uint64_t t0 = global_timer_ns();
 #pragma unroll 1
   for (int it = 0;; ++it) {
     if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
     int give_up = 0;
     if ((threadIdx.x & 31) == 0 && it >= 256)
-      give_up = (*abort != 0) || (global_timer_ns() - t0 > kWaitLimitNs);
+      give_up = (*abort != 0) || (global_timer_ns() - t0 > limit_ns);
     give_up = __shfl_sync(0xffffffffu, give_up, 0);
     if (give_up) {
       if ((threadIdx.x & 31) == 0 && *abort == 0) {

@@ -19,16 +19,19 @@
 //   dispatch_scatter_kernel one warp per pair: position = segment base + rank, slot = position
 //                           or -1 beyond C, row_token, and 16-byte vector copies of the row
 //
-// Overflow by priority (comparison article, "Expert Capacity Overflow": the capacity goes to the
-// tokens of highest router probability; Switch-style priority routing): the scan also writes the
-// demand offsets (exclusive prefix of the demands), then
-//   dispatch_list_kernel    one thread per pair: list[demand_offset[e] + position] = pair, i.e.
-//                           each expert's pairs in token order
-//   dispatch_priority_rank_kernel  one block per (expert, 256 of its pairs): a pair's rank is the
-//                           number of the expert's pairs with a larger gate, or an equal gate and
-//                           a lower pair index (shared-memory tiles of the expert's pairs);
-//                           slot = rank, or -1 from C on
-// and the scatter takes those slots instead of the first-come positions.
+// Overflow by priority (comparison article, "Expert Capacity Overflow": the example ranks an
+// expert's tokens by router probability and keeps the most probable): the scan also writes the
+// demand offsets (exclusive prefix of the demands), then each expert's pairs are sorted by the
+// 64-bit key (probability descending, pair index ascending; the probability is the softmax value
+// before any renormalisation of the gates):
+//   dispatch_prio_keys_kernel   one thread per pair: its key at its first-come place in its
+//                               expert's list (every expert's pairs in token order)
+//   dispatch_prio_chunk_kernel  one block per (expert, 1024 list entries): sorts the chunk in
+//                               shared memory (rank = number of smaller keys)
+//   dispatch_prio_merge_kernel  log2(T / 1024) passes, one thread per entry: runs of L merge
+//                               pairwise, each entry placed by a binary search in its partner run
+// the last launch writes slot = sorted position, or -1 from C on, and the scatter takes those
+// slots instead of the first-come positions. Work is O(n log^2 n) for an expert of demand n.
 #include <type_traits>
 
 #include "common.cuh"
@@ -181,66 +184,105 @@ __global__ void __launch_bounds__(1024)
   pdl_trigger();
 }
 
+// Sort key of a pair for the priority order: ascending keys = probability descending, then pair
+// index ascending. The fp32 probability is mapped to an unsigned integer of the same order
+// (negative zero folded onto zero, so equal probabilities tie), inverted, and followed by the pair.
+__device__ __forceinline__ uint64_t priority_key(float prob, int64_t pair) {
+  uint32_t u = __float_as_uint(prob == 0.0f ? 0.0f : prob);
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);  // float order -> unsigned order
+  return ((uint64_t)(~u) << 32) | (uint64_t)(uint32_t)pair;
+}
+
+// One thread per pair: the pair's key at its first-come place in its expert's list
+// (keys[demand_offset[e] + position]), i.e. every expert's pairs in token order.
 __global__ void __launch_bounds__(256)
-    dispatch_list_kernel(const int32_t* __restrict__ ids, int64_t pairs, int E,
-                         const int32_t* __restrict__ local_rank,
-                         const int32_t* __restrict__ seg_base, int seg_len,
-                         const int32_t* __restrict__ demand_offsets, int32_t* __restrict__ list) {
+    dispatch_prio_keys_kernel(const int32_t* __restrict__ ids, const float* __restrict__ probs,
+                              int64_t pairs, int E, const int32_t* __restrict__ local_rank,
+                              const int32_t* __restrict__ seg_base, int seg_len,
+                              const int32_t* __restrict__ demand_offsets,
+                              uint64_t* __restrict__ keys) {
   pdl_wait();
   const int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (p < pairs) {
     const int e = ids[p];
     const int r = local_rank[p];
     if (e >= 0 && e < E && r >= 0)
-      list[demand_offsets[e] + seg_base[(p / seg_len) * E + e] + r] = (int32_t)p;
+      keys[demand_offsets[e] + seg_base[(p / seg_len) * E + e] + r] = priority_key(probs[p], p);
   }
   pdl_trigger();
 }
 
-constexpr int kRankThreads = 256;
-constexpr int kRankTile = 1024;
+constexpr int kPrioChunk = 1024;  // list entries ranked together in shared memory
 
-// Block (c, e): pairs [256 c, 256 c + 256) of expert e's list. The expert's demand is at most T
-// (a token chooses an expert once), so gridDim.x = ceil(T / 256) covers every list.
-__global__ void __launch_bounds__(kRankThreads)
-    dispatch_priority_rank_kernel(const int32_t* __restrict__ list,
-                                  const int32_t* __restrict__ demand_offsets,
-                                  const int32_t* __restrict__ counts,
-                                  const float* __restrict__ gates, int64_t C,
-                                  int32_t* __restrict__ slot) {
-  __shared__ float tile_g[kRankTile];
-  __shared__ int tile_p[kRankTile];
+// Block (c, e): entries [1024 c, 1024 c + 1024) of expert e's list are sorted in shared memory
+// (each key's rank is the number of smaller keys in the chunk; keys are unique). The expert's
+// demand is at most T (a token chooses an expert once), so gridDim.x = ceil(T / 1024) covers
+// every list. final: no merge pass follows, so the rank is the slot (-1 from C on).
+__global__ void __launch_bounds__(kPrioChunk)
+    dispatch_prio_chunk_kernel(const uint64_t* __restrict__ in, uint64_t* __restrict__ out,
+                               const int32_t* __restrict__ demand_offsets, int64_t C, int final,
+                               int32_t* __restrict__ slot) {
+  __shared__ uint64_t tile[kPrioChunk];
   pdl_wait();
   const int e = blockIdx.y;
-  const int n = counts[e];
-  const int i0 = blockIdx.x * kRankThreads;
-  if (i0 < n) {  // block-uniform
-    const int32_t* mine = list + demand_offsets[e];
-    const int i = i0 + threadIdx.x;
-    int p = -1;
-    float g = 0.0f;
-    if (i < n) {
-      p = mine[i];
-      g = gates[p];
+  const int start = demand_offsets[e];
+  const int n = demand_offsets[e + 1] - start;
+  const int c0 = blockIdx.x * kPrioChunk;
+  if (c0 < n) {  // block-uniform
+    const int m = min(kPrioChunk, n - c0);
+    const int i = threadIdx.x;
+    uint64_t key = 0;
+    if (i < m) {
+      key = in[start + c0 + i];
+      tile[i] = key;
     }
-    int rank = 0;
-    for (int t0 = 0; t0 < n; t0 += kRankTile) {
-      const int m = min(kRankTile, n - t0);
-      __syncthreads();
-      for (int u = threadIdx.x; u < m; u += kRankThreads) {
-        const int q = mine[t0 + u];
-        tile_p[u] = q;
-        tile_g[u] = gates[q];
-      }
-      __syncthreads();
-      if (i < n) {
-        for (int u = 0; u < m; ++u) {
-          const float gq = tile_g[u];
-          rank += (gq > g || (gq == g && tile_p[u] < p)) ? 1 : 0;
-        }
-      }
+    __syncthreads();
+    if (i < m) {
+      int rank = 0;
+      for (int u = 0; u < m; ++u) rank += tile[u] < key ? 1 : 0;
+      const int pos = c0 + rank;
+      out[start + pos] = key;
+      if (final) slot[(uint32_t)key] = pos < C ? pos : -1;
     }
-    if (i < n) slot[p] = rank < C ? rank : -1;
+  }
+  pdl_trigger();
+}
+
+// One merge pass: every expert's list is a sequence of sorted runs of L entries; runs 2q and
+// 2q + 1 merge into one. Entry i of run r finds how many entries of the partner run r ^ 1 are
+// smaller (binary search; keys are unique) and moves to its place in the merged run.
+// final: the last pass, which also writes slot = position (-1 from C on).
+__global__ void __launch_bounds__(256)
+    dispatch_prio_merge_kernel(const uint64_t* __restrict__ in, uint64_t* __restrict__ out,
+                               const int32_t* __restrict__ ids,
+                               const int32_t* __restrict__ demand_offsets, int E, int L,
+                               int64_t C, int final, int32_t* __restrict__ slot) {
+  pdl_wait();
+  const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (j < demand_offsets[E]) {
+    const uint64_t key = in[j];
+    const int64_t pair = (uint32_t)key;
+    const int e = ids[pair];
+    const int start = demand_offsets[e];
+    const int n = demand_offsets[e + 1] - start;
+    const int i = (int)(j - start);
+    const int r = i / L;
+    const int partner = r ^ 1;
+    const int64_t ps = (int64_t)partner * L;
+    int pos = i;
+    if (ps < n) {
+      const int plen = (int)min((int64_t)L, n - ps);
+      const uint64_t* run = in + start + ps;
+      int lo = 0, hi = plen;  // first partner entry not smaller than key
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (run[mid] < key) lo = mid + 1;
+        else hi = mid;
+      }
+      pos = min(r, partner) * L + (i - r * L) + lo;
+    }
+    out[start + pos] = key;
+    if (final) slot[pair] = pos < C ? pos : -1;
   }
   pdl_trigger();
 }
@@ -358,22 +400,37 @@ cudaError_t enqueue_dispatch(const void* x, bool bf16, int64_t T, int d, const i
   {
     cudaError_t e = launch_kernel(dispatch_scan_kernel, dim3(1), dim3(1024), 0, stream,
                                   (const int32_t*)seg_counts, nseg, E, C, seg_base, counts, offsets,
-                                  prio.gates != nullptr ? prio.demand_offsets : nullptr, shard);
+                                  prio.probs != nullptr ? prio.demand_offsets : nullptr, shard);
     if (e != cudaSuccess) return e;
   }
   if (scan_only) return cudaGetLastError();
-  const int use_prio = prio.gates != nullptr && pairs > 0 ? 1 : 0;
+  const int use_prio = prio.probs != nullptr && pairs > 0 ? 1 : 0;
   if (use_prio) {
-    cudaError_t e = launch_kernel(dispatch_list_kernel, dim3((unsigned)((pairs + 255) / 256)),
-                                  dim3(256), 0, stream, ids, pairs, E,
+    // keys in first-come order per expert, sorted chunks of 1024, then merge passes until a run
+    // covers the largest possible list (T entries)
+    uint64_t* buf[2] = {prio.keys, prio.keys + pairs};
+    cudaError_t e = launch_kernel(dispatch_prio_keys_kernel, dim3((unsigned)((pairs + 255) / 256)),
+                                  dim3(256), 0, stream, ids, prio.probs, pairs, E,
                                   (const int32_t*)local_rank, (const int32_t*)seg_base, seg_len,
-                                  (const int32_t*)prio.demand_offsets, prio.list);
+                                  (const int32_t*)prio.demand_offsets, buf[0]);
     if (e != cudaSuccess) return e;
-    const dim3 grid((unsigned)((T + kRankThreads - 1) / kRankThreads), (unsigned)E);
-    e = launch_kernel(dispatch_priority_rank_kernel, grid, dim3(kRankThreads), 0, stream,
-                      (const int32_t*)prio.list, (const int32_t*)prio.demand_offsets,
-                      (const int32_t*)counts, prio.gates, C, slot);
+    int passes = 0;
+    for (int64_t L = kPrioChunk; L < T; L *= 2) ++passes;
+    const dim3 grid((unsigned)((T + kPrioChunk - 1) / kPrioChunk), (unsigned)E);
+    e = launch_kernel(dispatch_prio_chunk_kernel, grid, dim3(kPrioChunk), 0, stream,
+                      (const uint64_t*)buf[0], buf[1], (const int32_t*)prio.demand_offsets, C,
+                      passes == 0 ? 1 : 0, slot);
     if (e != cudaSuccess) return e;
+    int cur = 1;
+    int64_t L = kPrioChunk;
+    for (int q = 0; q < passes; ++q, L *= 2) {
+      e = launch_kernel(dispatch_prio_merge_kernel, dim3((unsigned)((pairs + 255) / 256)),
+                        dim3(256), 0, stream, (const uint64_t*)buf[cur], buf[cur ^ 1], ids,
+                        (const int32_t*)prio.demand_offsets, E, (int)L, C,
+                        q == passes - 1 ? 1 : 0, slot);
+      if (e != cudaSuccess) return e;
+      cur ^= 1;
+    }
   }
   if (pairs > 0) {
     const int64_t row_bytes = (int64_t)d * (bf16 ? 2 : 4);

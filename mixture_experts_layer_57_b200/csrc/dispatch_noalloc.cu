@@ -9,8 +9,11 @@
 // file-scope array below, which every GPU that loads the library holds until the process exits.
 //
 // Host code cannot use the array's name as a device address (on the host it names a stand-in
-// object), so the first call on each device, with that device current, looks the address up with
-// cudaGetSymbolAddress and caches it; later calls on that device reuse it.
+// object), so each call looks the address up with cudaGetSymbolAddress on the current device and
+// keeps it per device. A call made while its stream is being captured into a CUDA graph reuses the
+// kept address instead (the first call on a device must therefore come before any capture); every
+// other call looks it up again, so a device reset, which unloads the module and with it the
+// array, cannot leave a stale address behind.
 //
 // The kernels write every scratch element they later read (counts and bases for all segments and
 // experts, a rank for every pair), so nothing has to start at zero and the contents left by the
@@ -36,14 +39,19 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mutex;
 void* g_scratch_addr[kMaxDevices] = {};
 
-// Device address of g_dispatch_scratch on the current device (looked up once per device).
-cudaError_t scratch_address(void** out) {
+// Device address of g_dispatch_scratch on the current device: looked up again unless `stream` is
+// capturing (then the address kept from an earlier call on this device is used).
+cudaError_t scratch_address(cudaStream_t stream, void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  bool capturing = true;
+  if (cudaStreamIsCapturing(stream, &cs) == cudaSuccess) capturing = cs != cudaStreamCaptureStatusNone;
+  else (void)cudaGetLastError();  // the query failed: keep the kept address, clear the error
   std::lock_guard<std::mutex> lock(g_mutex);
-  if (g_scratch_addr[dev] == nullptr) {
+  if (!capturing || g_scratch_addr[dev] == nullptr) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_dispatch_scratch);
     if (e != cudaSuccess) return e;
@@ -85,7 +93,7 @@ extern "C" moe_status moe_dispatch_noalloc(const void* x, moe_dtype dtype, int64
   const char* inj = std::getenv("MOE_FAULT_INJECT");
   if (inj && std::strcmp(inj, "moe_dispatch_noalloc") == 0) return MOE_ERR_CUDA;
   void* base = nullptr;
-  if (scratch_address(&base) != cudaSuccess) return MOE_ERR_CUDA;
+  if (scratch_address(stream, &base) != cudaSuccess) return MOE_ERR_CUDA;
   moe::reset_launch_count();
   unsigned char* b = static_cast<unsigned char*>(base);
   int32_t* local_rank = reinterpret_cast<int32_t*>(b);

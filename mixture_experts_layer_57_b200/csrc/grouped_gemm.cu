@@ -35,6 +35,7 @@
 // Every wait is bounded (about 2 s): on expiry the kernel records MOE_DEVERR_TIMEOUT in the
 // status word, the other roles stop, in-flight TMA copies and MMAs are drained, TMEM is freed.
 #include <algorithm>
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -114,6 +115,11 @@ struct Params {
   CombineArgs cmb;         // used by the combine epilogues only
   const uint16_t* g_in;    // [rows_max, n_out] bf16 GeLU'(z) (kEpiGeluGradBf16)
   uint16_t* g_out;         // [rows_max, n_out] bf16 GeLU'(z) (kEpiGeluBf16Train)
+  // Failure-detection self-test only (moe_selftest_bounded_wait): the TMA role issues no copy, so
+  // the MMA role's first wait can never complete, and every bounded wait gives up after
+  // wait_limit_ns. Normal launches: selftest_no_copies = 0, wait_limit_ns = kWaitLimitNs.
+  int selftest_no_copies = 0;
+  uint64_t wait_limit_ns = kWaitLimitNs;
 };
 
 struct Tile {
@@ -142,6 +148,29 @@ __device__ __forceinline__ Tile decode_tile(int t, const int* prefix, const int*
   return tl;
 }
 
+// Tile order of a one-segment problem (the dense MLP: rows = tokens): groups of kDenseGroup token
+// tiles; inside a group, every token tile of the group for feature tile 0, then for feature tile
+// 1, and so on. The tiles in flight at one time then share a few weight tiles and a few token
+// tiles (a working set that stays in L2), where a feature-tile-major order would sweep all the
+// tokens once per feature tile.
+constexpr int kDenseGroup = 16;
+template <int BN, int FT>
+__device__ __forceinline__ Tile decode_dense_tile(int u, int64_t rows, int n_ftiles) {
+  const int n_tt = (int)((rows + BN - 1) / BN);
+  const int per_group = n_ftiles * kDenseGroup;
+  const int g = u / per_group;
+  const int in = u - g * per_group;
+  const int gt = min(kDenseGroup, n_tt - g * kDenseGroup);
+  const int ft = in / gt;
+  const int jt = g * kDenseGroup + (in - ft * gt);
+  Tile tl;
+  tl.e = 0;
+  tl.f0 = ft * kBM * FT;
+  tl.row0 = jt * BN;
+  tl.n_valid = (int)min((int64_t)BN, rows - (int64_t)jt * BN);
+  return tl;
+}
+
 // Wait bounded by time only (used to drain in-flight copies/MMAs while unwinding).
 __device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity, int* status) {
   const uint64_t t0 = global_timer_ns();
@@ -150,6 +179,315 @@ __device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity, i
       set_device_error(status, MOE_DEVERR_TIMEOUT);
       return;
     }
+  }
+}
+
+// The mbarriers of one CTA: S stage-full, S stage-empty, 2 accumulator-full, 2 accumulator-empty
+// and one drain barrier, 8 bytes each from `base`.
+struct Bars {
+  uint32_t base;
+  int S;
+  __device__ __forceinline__ uint32_t full(int s) const { return base + 8u * s; }
+  __device__ __forceinline__ uint32_t empty(int s) const { return base + 8u * (S + s); }
+  __device__ __forceinline__ uint32_t tfull(int a) const { return base + 8u * (2 * S + a); }
+  __device__ __forceinline__ uint32_t tempty(int a) const { return base + 8u * (2 * S + 2 + a); }
+  __device__ __forceinline__ uint32_t drain() const { return base + 8u * (2 * S + 4); }
+};
+
+// Position in the stage ring (shared by the TMA and MMA roles' loops).
+struct Ring {
+  int stage = 0;
+  uint32_t phase = 0;
+  __device__ __forceinline__ void next(int S) {
+    if (++stage == S) {
+      stage = 0;
+      phase ^= 1u;
+    }
+  }
+};
+
+// TMA role, one tile: per 64-wide K block, FT weight boxes of 128 rows (A) and one token box of BN
+// rows (B) into the next stage (A at the stage start, B at +a_bytes). Returns false if a wait
+// gave up.
+template <int BN, int FT, bool A_MN>
+__device__ __forceinline__ bool produce_tile(const Tile& tl, const CUtensorMap* tmW,
+                                             const CUtensorMap* tmX, const Params& p, int n_kb,
+                                             uint32_t base_addr, uint32_t stage_stride,
+                                             uint32_t a_bytes, const Bars& B, Ring& ring,
+                                             int& issued, volatile int* abort_flag) {
+  constexpr uint32_t kTx = FT * kBM * kBK * 2 + BN * kBK * 2;
+  const int w_row = tl.e * p.n_out + tl.f0;
+  for (int kb = 0; kb < n_kb; ++kb) {
+    if (!mbar_wait_bounded(B.empty(ring.stage), ring.phase ^ 1u, abort_flag, p.status,
+                           p.wait_limit_ns))
+      return false;
+    const uint32_t sa = base_addr + ring.stage * stage_stride;
+    mbar_arrive_expect_tx(B.full(ring.stage), kTx);
+#pragma unroll
+    for (int i = 0; i < FT; ++i) {
+      const uint32_t sai = sa + i * (kBM * kBK * 2);
+      if constexpr (A_MN) {
+        const int k_row = tl.e * p.K + kb * kBK;
+        tma_load_2d(sai, tmW, tl.f0 + i * kBM, k_row, B.full(ring.stage));
+        tma_load_2d(sai + kBM * kBK, tmW, tl.f0 + i * kBM + 64, k_row, B.full(ring.stage));
+      } else {
+        // rows past this expert's n_out (odd tile count) belong to the next expert or are out
+        // of range; the epilogue masks those features
+        tma_load_2d(sai, tmW, kb * kBK, w_row + i * kBM, B.full(ring.stage));
+      }
+    }
+    tma_load_2d(sa + a_bytes, tmX, kb * kBK, tl.row0, B.full(ring.stage));
+    ++issued;
+    ring.next(B.S);
+  }
+  return true;
+}
+
+// MMA role, one tile: K blocks of FT MMAs (M = 128 features, N = the tile's tokens rounded up to
+// 16, K = 16 each) into FT accumulators of BN columns at d_tmem. Returns false if a wait gave up.
+template <int BN, int FT, bool A_MN>
+__device__ __forceinline__ bool mma_tile(const Tile& tl, uint32_t d_tmem, const Params& p,
+                                         int n_kb, uint32_t base_addr, uint32_t stage_stride,
+                                         uint32_t a_bytes, const Bars& B, Ring& ring,
+                                         volatile int* abort_flag) {
+  const int n_mma = max(16, (tl.n_valid + 15) & ~15);
+  const uint32_t idesc = idesc_bf16_f32_major(kBM, n_mma, A_MN, false);
+  for (int kb = 0; kb < n_kb; ++kb) {
+    if (!mbar_wait_bounded(B.full(ring.stage), ring.phase, abort_flag, p.status, p.wait_limit_ns))
+      return false;
+    tc_fence_after();
+    const uint32_t sa = base_addr + ring.stage * stage_stride;
+    const uint64_t bdesc = smem_desc_sw128(sa + a_bytes);
+    // K step: +32 bytes inside a K-major 128-byte row (+2 in the 16-byte address field),
+    // or two 8-row groups of an MN-major tile
+    constexpr uint64_t a_step = A_MN ? (kMnKStepBytes >> 4) : 2;
+#pragma unroll
+    for (int i = 0; i < FT; ++i) {
+      const uint32_t sai = sa + i * (kBM * kBK * 2);
+      const uint64_t adesc = A_MN ? smem_desc_sw128_mn(sai) : smem_desc_sw128(sai);
+#pragma unroll
+      for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
+        tc_mma_bf16(d_tmem + (uint32_t)(i * BN), adesc + a_step * (uint64_t)kk,
+                    bdesc + (uint64_t)(2 * kk), idesc, (kb | kk) != 0 ? 1u : 0u);
+      }
+    }
+    tc_commit(B.empty(ring.stage));
+    ring.next(B.S);
+  }
+  return true;
+}
+
+// Epilogue role (one of warps 2..9), one tile: reads the FT accumulators at acc_tmem (this warp's
+// TMEM lane quarter, alternate 16-column chunks by `half`) and writes the tile's outputs.
+template <int BN, int FT, int EPI>
+__device__ __forceinline__ void epilogue_tile(const Tile& tl, const Params& p, uint32_t acc_tmem,
+                                              int quarter, int half, int lane, uint8_t* st) {
+#pragma unroll 1
+  for (int fi = 0; fi < FT; ++fi) {
+    const int fw = tl.f0 + fi * kBM + quarter * 32;  // first feature of this warp
+    const int f = fw + lane;
+    const bool f_ok = f < p.n_out;
+    const float bv = (p.bias != nullptr && f_ok)
+                         ? bf16_to_f32(reinterpret_cast<const uint16_t*>(p.bias)[(int64_t)tl.e * p.n_out + f])
+                         : 0.0f;
+    const uint32_t taddr = acc_tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(fi * BN);
+    for (int c0 = half * 16; c0 < tl.n_valid; c0 += 32) {
+      uint32_t r[16];
+      tmem_ld_32x32b_x16(taddr + (uint32_t)c0, r);
+      tmem_ld_wait();
+      const int nc = min(16, tl.n_valid - c0);
+      if constexpr (EPI == kEpiGeluGradBf16) {
+        // dZ = dH * GeLU'(z): stage dH [16 tokens][32 features] fp32, then each lane takes 8
+        // features of one token: 16-byte loads of GeLU'(z) and 16-byte stores of dZ
+        float* s32 = reinterpret_cast<float*>(st);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) s32[c * 32 + lane] = __uint_as_float(r[c]);
+        __syncwarp();
+#pragma unroll
+        for (int id = lane; id < 64; id += 32) {
+          const int row = id >> 2, q = id & 3;
+          const int ff = fw + 8 * q;
+          if (row < nc && ff < p.n_out) {
+            const int64_t o = (int64_t)(tl.row0 + c0 + row) * p.n_out + ff;
+            const uint4 gv = *reinterpret_cast<const uint4*>(p.g_in + o);
+            const float4 h0 = *reinterpret_cast<const float4*>(s32 + row * 32 + 8 * q);
+            const float4 h1 = *reinterpret_cast<const float4*>(s32 + row * 32 + 8 * q + 4);
+            uint4 ov;
+            ov.x = (uint32_t)f32_to_bf16_rn(h0.x * __uint_as_float(gv.x << 16)) |
+                   ((uint32_t)f32_to_bf16_rn(h0.y * __uint_as_float(gv.x & 0xffff0000u)) << 16);
+            ov.y = (uint32_t)f32_to_bf16_rn(h0.z * __uint_as_float(gv.y << 16)) |
+                   ((uint32_t)f32_to_bf16_rn(h0.w * __uint_as_float(gv.y & 0xffff0000u)) << 16);
+            ov.z = (uint32_t)f32_to_bf16_rn(h1.x * __uint_as_float(gv.z << 16)) |
+                   ((uint32_t)f32_to_bf16_rn(h1.y * __uint_as_float(gv.z & 0xffff0000u)) << 16);
+            ov.w = (uint32_t)f32_to_bf16_rn(h1.z * __uint_as_float(gv.w << 16)) |
+                   ((uint32_t)f32_to_bf16_rn(h1.w * __uint_as_float(gv.w & 0xffff0000u)) << 16);
+            *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.out) + o) = ov;
+          }
+        }
+        __syncwarp();
+      } else if constexpr (EPI == kEpiGeluBf16 || EPI == kEpiGeluBf16Train) {
+        // stage [16 tokens][32 features] bf16, then 16-byte stores of 8 features of one token
+        // (the training variant stages GeLU'(z) the same way, after GeLU(z))
+        uint16_t* s16 = reinterpret_cast<uint16_t*>(st);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) s16[c * 32 + lane] = f32_to_bf16_rn(gelu_erf(__uint_as_float(r[c]) + bv));
+        __syncwarp();
+        if constexpr (EPI == kEpiGeluBf16Train) {
+          uint16_t* g16 = s16 + 16 * 32;
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            g16[c * 32 + lane] = f32_to_bf16_rn(gelu_erf_grad(__uint_as_float(r[c]) + bv));
+          __syncwarp();
+#pragma unroll
+          for (int id = lane; id < 64; id += 32) {
+            const int row = id >> 2, q = id & 3;
+            const int ff = fw + 8 * q;
+            if (row < nc && ff < p.n_out)
+              *reinterpret_cast<uint4*>(p.g_out + (int64_t)(tl.row0 + c0 + row) * p.n_out + ff) =
+                  *reinterpret_cast<const uint4*>(st + 1024 + row * 64 + q * 16);
+          }
+        }
+#pragma unroll
+        for (int id = lane; id < 64; id += 32) {
+          const int row = id >> 2, q = id & 3;
+          const int ff = fw + 8 * q;
+          if (row < nc && ff < p.n_out)
+            *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.out) +
+                                      (int64_t)(tl.row0 + c0 + row) * p.n_out + ff) =
+                *reinterpret_cast<const uint4*>(st + row * 64 + q * 16);
+        }
+        __syncwarp();
+      } else if constexpr (EPI == kEpiF32) {
+        // stage [16 tokens][32 features] fp32, then 16-byte stores of 4 features of one token
+        float* s32 = reinterpret_cast<float*>(st);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) s32[c * 32 + lane] = __uint_as_float(r[c]) + bv;
+        __syncwarp();
+#pragma unroll
+        for (int id = lane; id < 128; id += 32) {
+          const int row = id >> 3, q = id & 7;
+          const int ff = fw + 4 * q;
+          if (row < nc && ff < p.n_out)
+            *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) +
+                                       (int64_t)(tl.row0 + c0 + row) * p.n_out + ff) =
+                *reinterpret_cast<const float4*>(st + row * 128 + q * 16);
+        }
+        __syncwarp();
+      } else {
+        // fused combine: y (or the dense MLP output) = acc + bias staged as fp32 [16][32]; each
+        // lane then finishes 4 features of one token row of the layer output
+        const CombineArgs& cb = p.cmb;
+        float* s32 = reinterpret_cast<float*>(st);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) s32[c * 32 + lane] = __uint_as_float(r[c]) + bv;
+        __syncwarp();
+#pragma unroll
+        for (int id = lane; id < 128; id += 32) {
+          const int row = id >> 3, q = id & 7;
+          const int ff = fw + 4 * q;
+          if (row < nc && ff < p.n_out) {
+            const int64_t pr = (int64_t)(tl.row0 + c0 + row);  // packed row (dense: token)
+            const float4 v = *reinterpret_cast<const float4*>(st + row * 128 + q * 16);
+            int64_t t;
+            float a[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            if constexpr (EPI == kEpiCombineExpert) {
+              t = cb.row_token[pr];
+            } else {
+              t = pr;
+            }
+            if (cb.residual) {
+              const uint2 rb = *reinterpret_cast<const uint2*>(cb.residual + t * p.n_out + ff);
+              a[0] = __uint_as_float(rb.x << 16);
+              a[1] = __uint_as_float(rb.x & 0xffff0000u);
+              a[2] = __uint_as_float(rb.y << 16);
+              a[3] = __uint_as_float(rb.y & 0xffff0000u);
+            }
+            if constexpr (EPI == kEpiCombineExpert) {
+              const float g = cb.gates[t];
+              a[0] = fmaf(g, v.x, a[0]);
+              a[1] = fmaf(g, v.y, a[1]);
+              a[2] = fmaf(g, v.z, a[2]);
+              a[3] = fmaf(g, v.w, a[3]);
+            } else {
+              a[0] += v.x;
+              a[1] += v.y;
+              a[2] += v.z;
+              a[3] += v.w;
+              for (int j = 0; j < cb.k; ++j) {
+                const int sl = cb.slot[t * cb.k + j];
+                if (sl < 0) continue;
+                const int e = cb.ids[t * cb.k + j];
+                if (e < 0 || e >= cb.E_experts) continue;
+                const int64_t yr = (int64_t)cb.offsets[e] + sl;
+                if (yr >= cb.rows_y) {
+                  set_device_error(p.status, MOE_DEVERR_BAD_ROW);
+                  continue;
+                }
+                const float g = cb.gates[t * cb.k + j];
+                const float4 y = *reinterpret_cast<const float4*>(cb.y + yr * p.n_out + ff);
+                a[0] = fmaf(g, y.x, a[0]);
+                a[1] = fmaf(g, y.y, a[1]);
+                a[2] = fmaf(g, y.z, a[2]);
+                a[3] = fmaf(g, y.w, a[3]);
+              }
+            }
+            if (cb.out_bf16) {
+              uint2 o;
+              o.x = (uint32_t)f32_to_bf16_rn(a[0]) | ((uint32_t)f32_to_bf16_rn(a[1]) << 16);
+              o.y = (uint32_t)f32_to_bf16_rn(a[2]) | ((uint32_t)f32_to_bf16_rn(a[3]) << 16);
+              *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(cb.out) + t * p.n_out + ff) = o;
+            } else {
+              *reinterpret_cast<float4*>(reinterpret_cast<float*>(cb.out) + t * p.n_out + ff) =
+                  make_float4(a[0], a[1], a[2], a[3]);
+            }
+          }
+        }
+        __syncwarp();
+      }
+    }
+  }
+}
+
+// Builds the tile list of a grouped problem in shared memory (one warp): seg[e] = first packed
+// row of expert e, prefix[e] = first tile of expert e, prefix[E] = the tile count (0 and a device
+// error if the offsets are not non-decreasing within [0, rows_max]).
+template <int BN>
+__device__ __forceinline__ void build_tile_list(const Params& p, int n_ftiles, int* prefix,
+                                                int* seg, int lane) {
+  const int E = p.E;
+  const int chunk = (E + 31) / 32;
+  const int e0 = min(E, lane * chunk), e1 = min(E, e0 + chunk);
+  bool bad = false;
+  int local = 0;
+  // offsets == nullptr: one segment covering all rows_max rows (dense MLP, E == 1)
+  auto off = [&](int e) -> int {
+    return p.offsets ? p.offsets[e] : (e == 0 ? 0 : (int)p.rows_max);
+  };
+  for (int e = e0; e < e1; ++e) {
+    const int a = off(e), b = off(e + 1);
+    seg[e] = a;
+    if (a < 0 || b < a || (int64_t)b > p.rows_max) bad = true;
+    else local += n_ftiles * ((b - a + BN - 1) / BN);
+  }
+  if (lane == 0) seg[E] = off(E);
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  int run = incl - local;
+  for (int e = e0; e < e1; ++e) {
+    prefix[e] = run;
+    const int a = seg[e], b = off(e + 1);
+    if (!(a < 0 || b < a || (int64_t)b > p.rows_max)) run += n_ftiles * ((b - a + BN - 1) / BN);
+  }
+  const int total = __shfl_sync(0xffffffffu, incl, 31);
+  bad = __any_sync(0xffffffffu, bad);
+  __syncwarp();
+  if (lane == 0) {
+    prefix[E] = bad ? 0 : total;
+    if (bad && blockIdx.x == 0) set_device_error(p.status, MOE_DEVERR_BAD_OFFSETS);
   }
 }
 
@@ -176,23 +514,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int S = C::kStages;
-  auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
-  auto empty_bar = [&](int s) { return smem_u32(&bars[S + s]); };
-  auto tfull_bar = [&](int a) { return smem_u32(&bars[2 * S + a]); };
-  auto tempty_bar = [&](int a) { return smem_u32(&bars[2 * S + 2 + a]); };
-  const uint32_t drain_bar = smem_u32(&bars[2 * S + 4]);
+  const Bars B{smem_u32(bars), S};
 
   // ------------------------------------------------------------ prologue
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 1);
+      mbar_init(B.full(s), 1);
+      mbar_init(B.empty(s), 1);
     }
     for (int a = 0; a < 2; ++a) {
-      mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), kEpiWarps * 32);
+      mbar_init(B.tfull(a), 1);
+      mbar_init(B.tempty(a), kEpiWarps * 32);
     }
-    mbar_init(drain_bar, 1);
+    mbar_init(B.drain(), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -208,146 +542,56 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   const int n_ftiles = (p.n_out + kBM * FT - 1) / (kBM * FT);
-  if (warp == 2) {
-    // Tile list: prefix[e] = first tile of expert e; validates the device offsets.
-    const int E = p.E;
-    const int chunk = (E + 31) / 32;
-    const int e0 = min(E, lane * chunk), e1 = min(E, e0 + chunk);
-    bool bad = false;
-    int local = 0;
-    // offsets == nullptr: one segment covering all rows_max rows (dense MLP, E == 1)
-    auto off = [&](int e) -> int {
-      return p.offsets ? p.offsets[e] : (e == 0 ? 0 : (int)p.rows_max);
-    };
-    for (int e = e0; e < e1; ++e) {
-      const int a = off(e), b = off(e + 1);
-      seg[e] = a;
-      if (a < 0 || b < a || (int64_t)b > p.rows_max) bad = true;
-      else local += n_ftiles * ((b - a + BN - 1) / BN);
-    }
-    if (lane == 0) seg[E] = off(E);
-    int incl = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
-    }
-    int run = incl - local;
-    for (int e = e0; e < e1; ++e) {
-      prefix[e] = run;
-      const int a = seg[e], b = off(e + 1);
-      if (!(a < 0 || b < a || (int64_t)b > p.rows_max)) run += n_ftiles * ((b - a + BN - 1) / BN);
-    }
-    const int total = __shfl_sync(0xffffffffu, incl, 31);
-    bad = __any_sync(0xffffffffu, bad);
-    __syncwarp();
-    if (lane == 0) {
-      prefix[E] = bad ? 0 : total;
-      if (bad && blockIdx.x == 0) set_device_error(p.status, MOE_DEVERR_BAD_OFFSETS);
-    }
-  }
+  if (warp == 2) build_tile_list<BN>(p, n_ftiles, prefix, seg, lane);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const int total_tiles = prefix[p.E];
   const int n_kb = (p.K + kBK - 1) / kBK;
+  const bool one_seg = p.offsets == nullptr;
+  auto tile_at = [&](int t) {
+    return one_seg ? decode_dense_tile<BN, FT>(t, p.rows_max, n_ftiles)
+                   : decode_tile<BN, FT>(t, prefix, seg, p.E, n_ftiles);
+  };
 
   if (warp == 0) {
     // ---------------------------------------------------------- TMA producer
     if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
+      Ring ring;
       int issued = 0;
-      for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
-        const Tile tl = decode_tile<BN, FT>(t, prefix, seg, p.E, n_ftiles);
-        const int w_row = tl.e * p.n_out + tl.f0;
-        bool ok = true;
-        for (int kb = 0; kb < n_kb; ++kb) {
-          if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, p.status)) {
-            ok = false;
-            break;
-          }
-          const uint32_t sa = base_addr + stage * C::kStageBytes;
-          mbar_arrive_expect_tx(full_bar(stage), C::kStageBytes);
-#pragma unroll
-          for (int i = 0; i < FT; ++i) {
-            const uint32_t sai = sa + i * (kBM * kBK * 2);
-            if constexpr (A_MN) {
-              const int k_row = tl.e * p.K + kb * kBK;
-              tma_load_2d(sai, &tmW, tl.f0 + i * kBM, k_row, full_bar(stage));
-              tma_load_2d(sai + kBM * kBK, &tmW, tl.f0 + i * kBM + 64, k_row, full_bar(stage));
-            } else {
-              // rows past this expert's n_out (odd tile count) belong to the next expert or are
-              // out of range; the epilogue masks those features
-              tma_load_2d(sai, &tmW, kb * kBK, w_row + i * kBM, full_bar(stage));
-            }
-          }
-          tma_load_2d(sa + C::kABytes, &tmX, kb * kBK, tl.row0, full_bar(stage));
-          ++issued;
-          if (++stage == S) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-        if (!ok) break;
+      for (int t = blockIdx.x; t < total_tiles && !p.selftest_no_copies; t += gridDim.x) {
+        if (!produce_tile<BN, FT, A_MN>(tile_at(t), &tmW, &tmX, p, n_kb, base_addr, C::kStageBytes,
+                                        C::kABytes, B, ring, issued, abort_flag))
+          break;
       }
       // drain: the last min(issued, S) loads may still be landing
       for (int i = max(0, issued - S); i < issued; ++i)
-        mbar_wait_drain(full_bar(i % S), (uint32_t)((i / S) & 1), p.status);
+        mbar_wait_drain(B.full(i % S), (uint32_t)((i / S) & 1), p.status);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
+      Ring ring;
       int acc = 0;
       uint32_t acc_phase = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-        const Tile tl = decode_tile<BN, FT>(t, prefix, seg, p.E, n_ftiles);
-        if (!mbar_wait_bounded(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.status)) break;
+      for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+        if (!mbar_wait_bounded(B.tempty(acc), acc_phase ^ 1u, abort_flag, p.status,
+                               p.wait_limit_ns))
+          break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * FT * BN);
-        const int n_mma = max(16, (tl.n_valid + 15) & ~15);
-        const uint32_t idesc = idesc_bf16_f32_major(kBM, n_mma, A_MN, false);
-        for (int kb = 0; kb < n_kb; ++kb) {
-          if (!mbar_wait_bounded(full_bar(stage), phase, abort_flag, p.status)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t sa = base_addr + stage * C::kStageBytes;
-          const uint64_t bdesc = smem_desc_sw128(sa + C::kABytes);
-          // K step: +32 bytes inside a K-major 128-byte row (+2 in the 16-byte address field),
-          // or two 8-row groups of an MN-major tile
-          constexpr uint64_t a_step = A_MN ? (kMnKStepBytes >> 4) : 2;
-#pragma unroll
-          for (int i = 0; i < FT; ++i) {
-            const uint32_t sai = sa + i * (kBM * kBK * 2);
-            const uint64_t adesc = A_MN ? smem_desc_sw128_mn(sai) : smem_desc_sw128(sai);
-#pragma unroll
-            for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
-              tc_mma_bf16(d_tmem + (uint32_t)(i * BN), adesc + a_step * (uint64_t)kk,
-                          bdesc + (uint64_t)(2 * kk), idesc, (kb | kk) != 0 ? 1u : 0u);
-            }
-          }
-          tc_commit(empty_bar(stage));
-          if (++stage == S) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-        if (!ok) break;
-        tc_commit(tfull_bar(acc));
+        if (!mma_tile<BN, FT, A_MN>(tile_at(t), tmem_base + (uint32_t)(acc * FT * BN), p, n_kb,
+                                    base_addr, C::kStageBytes, C::kABytes, B, ring, abort_flag))
+          break;
+        tc_commit(B.tfull(acc));
         if (++acc == 2) {
           acc = 0;
           acc_phase ^= 1u;
         }
       }
       // drain every MMA this thread issued before TMEM is released
-      tc_commit(drain_bar);
-      mbar_wait_drain(drain_bar, 0, p.status);
+      tc_commit(B.drain());
+      mbar_wait_drain(B.drain(), 0, p.status);
     }
   } else {
     // ---------------------------------------------------------- epilogue (warps 2..9)
@@ -358,176 +602,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
-      const Tile tl = decode_tile<BN, FT>(t, prefix, seg, p.E, n_ftiles);
-      if (!mbar_wait_bounded_warp(tfull_bar(acc), acc_phase, abort_flag, p.status)) break;
+      if (!mbar_wait_bounded_warp(B.tfull(acc), acc_phase, abort_flag, p.status,
+                                  p.wait_limit_ns))
+        break;
       tc_fence_after();
-#pragma unroll 1
-      for (int fi = 0; fi < FT; ++fi) {
-      const int fw = tl.f0 + fi * kBM + quarter * 32;  // first feature of this warp
-      const int f = fw + lane;
-      const bool f_ok = f < p.n_out;
-      const float bv = (p.bias != nullptr && f_ok)
-                           ? bf16_to_f32(reinterpret_cast<const uint16_t*>(p.bias)[(int64_t)tl.e * p.n_out + f])
-                           : 0.0f;
-      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) +
-                             (uint32_t)(acc * FT * BN + fi * BN);
-      for (int c0 = half * 16; c0 < tl.n_valid; c0 += 32) {
-        uint32_t r[16];
-        tmem_ld_32x32b_x16(taddr + (uint32_t)c0, r);
-        tmem_ld_wait();
-        const int nc = min(16, tl.n_valid - c0);
-        if constexpr (EPI == kEpiGeluGradBf16) {
-          // dZ = dH * GeLU'(z): stage dH [16 tokens][32 features] fp32, then each lane takes 8
-          // features of one token: 16-byte loads of GeLU'(z) and 16-byte stores of dZ
-          float* s32 = reinterpret_cast<float*>(st);
-#pragma unroll
-          for (int c = 0; c < 16; ++c) s32[c * 32 + lane] = __uint_as_float(r[c]);
-          __syncwarp();
-#pragma unroll
-          for (int id = lane; id < 64; id += 32) {
-            const int row = id >> 2, q = id & 3;
-            const int ff = fw + 8 * q;
-            if (row < nc && ff < p.n_out) {
-              const int64_t o = (int64_t)(tl.row0 + c0 + row) * p.n_out + ff;
-              const uint4 gv = *reinterpret_cast<const uint4*>(p.g_in + o);
-              const float4 h0 = *reinterpret_cast<const float4*>(s32 + row * 32 + 8 * q);
-              const float4 h1 = *reinterpret_cast<const float4*>(s32 + row * 32 + 8 * q + 4);
-              uint4 ov;
-              ov.x = (uint32_t)f32_to_bf16_rn(h0.x * __uint_as_float(gv.x << 16)) |
-                     ((uint32_t)f32_to_bf16_rn(h0.y * __uint_as_float(gv.x & 0xffff0000u)) << 16);
-              ov.y = (uint32_t)f32_to_bf16_rn(h0.z * __uint_as_float(gv.y << 16)) |
-                     ((uint32_t)f32_to_bf16_rn(h0.w * __uint_as_float(gv.y & 0xffff0000u)) << 16);
-              ov.z = (uint32_t)f32_to_bf16_rn(h1.x * __uint_as_float(gv.z << 16)) |
-                     ((uint32_t)f32_to_bf16_rn(h1.y * __uint_as_float(gv.z & 0xffff0000u)) << 16);
-              ov.w = (uint32_t)f32_to_bf16_rn(h1.z * __uint_as_float(gv.w << 16)) |
-                     ((uint32_t)f32_to_bf16_rn(h1.w * __uint_as_float(gv.w & 0xffff0000u)) << 16);
-              *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.out) + o) = ov;
-            }
-          }
-          __syncwarp();
-        } else if constexpr (EPI == kEpiGeluBf16 || EPI == kEpiGeluBf16Train) {
-          // stage [16 tokens][32 features] bf16, then 16-byte stores of 8 features of one token
-          // (the training variant stages GeLU'(z) the same way, after GeLU(z))
-          uint16_t* s16 = reinterpret_cast<uint16_t*>(st);
-#pragma unroll
-          for (int c = 0; c < 16; ++c) s16[c * 32 + lane] = f32_to_bf16_rn(gelu_erf(__uint_as_float(r[c]) + bv));
-          __syncwarp();
-          if constexpr (EPI == kEpiGeluBf16Train) {
-            uint16_t* g16 = s16 + 16 * 32;
-#pragma unroll
-            for (int c = 0; c < 16; ++c)
-              g16[c * 32 + lane] = f32_to_bf16_rn(gelu_erf_grad(__uint_as_float(r[c]) + bv));
-            __syncwarp();
-#pragma unroll
-            for (int id = lane; id < 64; id += 32) {
-              const int row = id >> 2, q = id & 3;
-              const int ff = fw + 8 * q;
-              if (row < nc && ff < p.n_out)
-                *reinterpret_cast<uint4*>(p.g_out + (int64_t)(tl.row0 + c0 + row) * p.n_out + ff) =
-                    *reinterpret_cast<const uint4*>(st + 1024 + row * 64 + q * 16);
-            }
-          }
-#pragma unroll
-          for (int id = lane; id < 64; id += 32) {
-            const int row = id >> 2, q = id & 3;
-            const int ff = fw + 8 * q;
-            if (row < nc && ff < p.n_out)
-              *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.out) +
-                                        (int64_t)(tl.row0 + c0 + row) * p.n_out + ff) =
-                  *reinterpret_cast<const uint4*>(st + row * 64 + q * 16);
-          }
-          __syncwarp();
-        } else if constexpr (EPI == kEpiF32) {
-          // stage [16 tokens][32 features] fp32, then 16-byte stores of 4 features of one token
-          float* s32 = reinterpret_cast<float*>(st);
-#pragma unroll
-          for (int c = 0; c < 16; ++c) s32[c * 32 + lane] = __uint_as_float(r[c]) + bv;
-          __syncwarp();
-#pragma unroll
-          for (int id = lane; id < 128; id += 32) {
-            const int row = id >> 3, q = id & 7;
-            const int ff = fw + 4 * q;
-            if (row < nc && ff < p.n_out)
-              *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) +
-                                         (int64_t)(tl.row0 + c0 + row) * p.n_out + ff) =
-                  *reinterpret_cast<const float4*>(st + row * 128 + q * 16);
-          }
-          __syncwarp();
-        } else {
-          // fused combine: y (or the dense MLP output) = acc + bias staged as fp32 [16][32]; each
-          // lane then finishes 4 features of one token row of the layer output
-          const CombineArgs& cb = p.cmb;
-          float* s32 = reinterpret_cast<float*>(st);
-#pragma unroll
-          for (int c = 0; c < 16; ++c) s32[c * 32 + lane] = __uint_as_float(r[c]) + bv;
-          __syncwarp();
-#pragma unroll
-          for (int id = lane; id < 128; id += 32) {
-            const int row = id >> 3, q = id & 7;
-            const int ff = fw + 4 * q;
-            if (row < nc && ff < p.n_out) {
-              const int64_t pr = (int64_t)(tl.row0 + c0 + row);  // packed row (dense: token)
-              const float4 v = *reinterpret_cast<const float4*>(st + row * 128 + q * 16);
-              int64_t t;
-              float a[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-              if constexpr (EPI == kEpiCombineExpert) {
-                t = cb.row_token[pr];
-              } else {
-                t = pr;
-              }
-              if (cb.residual) {
-                const uint2 rb = *reinterpret_cast<const uint2*>(cb.residual + t * p.n_out + ff);
-                a[0] = __uint_as_float(rb.x << 16);
-                a[1] = __uint_as_float(rb.x & 0xffff0000u);
-                a[2] = __uint_as_float(rb.y << 16);
-                a[3] = __uint_as_float(rb.y & 0xffff0000u);
-              }
-              if constexpr (EPI == kEpiCombineExpert) {
-                const float g = cb.gates[t];
-                a[0] = fmaf(g, v.x, a[0]);
-                a[1] = fmaf(g, v.y, a[1]);
-                a[2] = fmaf(g, v.z, a[2]);
-                a[3] = fmaf(g, v.w, a[3]);
-              } else {
-                a[0] += v.x;
-                a[1] += v.y;
-                a[2] += v.z;
-                a[3] += v.w;
-                for (int j = 0; j < cb.k; ++j) {
-                  const int sl = cb.slot[t * cb.k + j];
-                  if (sl < 0) continue;
-                  const int e = cb.ids[t * cb.k + j];
-                  if (e < 0 || e >= cb.E_experts) continue;
-                  const int64_t yr = (int64_t)cb.offsets[e] + sl;
-                  if (yr >= cb.rows_y) {
-                    set_device_error(p.status, MOE_DEVERR_BAD_ROW);
-                    continue;
-                  }
-                  const float g = cb.gates[t * cb.k + j];
-                  const float4 y = *reinterpret_cast<const float4*>(cb.y + yr * p.n_out + ff);
-                  a[0] = fmaf(g, y.x, a[0]);
-                  a[1] = fmaf(g, y.y, a[1]);
-                  a[2] = fmaf(g, y.z, a[2]);
-                  a[3] = fmaf(g, y.w, a[3]);
-                }
-              }
-              if (cb.out_bf16) {
-                uint2 o;
-                o.x = (uint32_t)f32_to_bf16_rn(a[0]) | ((uint32_t)f32_to_bf16_rn(a[1]) << 16);
-                o.y = (uint32_t)f32_to_bf16_rn(a[2]) | ((uint32_t)f32_to_bf16_rn(a[3]) << 16);
-                *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(cb.out) + t * p.n_out + ff) = o;
-              } else {
-                *reinterpret_cast<float4*>(reinterpret_cast<float*>(cb.out) + t * p.n_out + ff) =
-                    make_float4(a[0], a[1], a[2], a[3]);
-              }
-            }
-          }
-          __syncwarp();
-        }
-      }
-      }  // feature tiles
+      epilogue_tile<BN, FT, EPI>(tile_at(t), p, tmem_base + (uint32_t)(acc * FT * BN), quarter,
+                                 half, lane, st);
       tc_fence_before();
-      mbar_arrive(tempty_bar(acc));
+      mbar_arrive(B.tempty(acc));
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1u;
@@ -542,6 +624,185 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+// Two GEMM problems of one layer co-scheduled in one persistent launch: problem 0 is the grouped
+// expert layer (BN0 tokens per tile, two 128-feature tiles per CTA tile), problem 1 the PR-MoE
+// dense MLP layer (one segment of all tokens, 256 tokens x 128 features per tile), with the same
+// epilogue kind. The expert layers stream their weights from HBM with the tensor pipe mostly idle,
+// the dense layers keep it busy with little HBM traffic: interleaving their tiles on every SM lets
+// the two overlap instead of taking turns. The combined tile sequence takes problem-0 tile number
+// floor(t n0 / N) when floor((t + 1) n0 / N) > floor(t n0 / N), else problem-1 tile
+// t - floor(t n0 / N) (N = n0 + n1), so any window of consecutive tiles holds both in proportion;
+// CTA b takes tiles b, b + gridDim.x, ... as in the single-problem kernel. Stages are 48 KB (the
+// larger of the two problems' stage sizes) and each accumulator is 256 TMEM columns.
+constexpr int kCoBN1 = 256;
+constexpr int kCoStageBytes = 48 * 1024;
+constexpr int kCoStages = (200 * 1024) / kCoStageBytes;
+constexpr int kCoAccCols = 256;
+constexpr int kCoSmemBytes = 1024 + kCoStages * kCoStageBytes + kEpiWarps * kStageTileBytes +
+                             Cfg<kCoBN1, 1>::kAuxBytes;
+static_assert(Cfg<kCoBN1, 1>::kStageBytes == kCoStageBytes, "dense stage size");
+static_assert(Cfg<128, 2>::kStageBytes <= kCoStageBytes, "expert stage size");
+static_assert(2 * kCoStages + 5 <= 64, "barrier area too small");
+static_assert(kCoSmemBytes <= 227 * 1024, "shared memory budget");
+
+template <int BN0, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    co_gemm_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__ CUtensorMap tmX0,
+                   const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmX1,
+                   const Params p0, const Params p1) {
+  static_assert(2 * BN0 <= kCoAccCols, "two expert accumulators per buffer");
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t base_addr = (raw_addr + 1023u) & ~1023u;
+  uint8_t* base = smem_raw + (base_addr - raw_addr);
+
+  uint8_t* stage_tiles = base + kCoStages * kCoStageBytes;
+  uint8_t* aux = stage_tiles + kEpiWarps * kStageTileBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(aux);
+  constexpr int kBarBytes = Cfg<kCoBN1, 1>::kBarBytes;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(aux + kBarBytes);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(aux + kBarBytes + 4);
+  int* prefix = reinterpret_cast<int*>(aux + kBarBytes + 16);
+  int* seg = prefix + (MOE_MAX_EXPERTS + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int S = kCoStages;
+  const Bars B{smem_u32(bars), S};
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(B.full(s), 1);
+      mbar_init(B.empty(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(B.tfull(a), 1);
+      mbar_init(B.tempty(a), kEpiWarps * 32);
+    }
+    mbar_init(B.drain(), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  pdl_wait();
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&tmW0);
+    tma_prefetch_desc(&tmX0);
+    tma_prefetch_desc(&tmW1);
+    tma_prefetch_desc(&tmX1);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), 2 * kCoAccCols);
+    tmem_relinquish();
+  }
+  const int nft0 = (p0.n_out + 2 * kBM - 1) / (2 * kBM);
+  const int nft1 = (p1.n_out + kBM - 1) / kBM;
+  if (warp == 2) build_tile_list<BN0>(p0, nft0, prefix, seg, lane);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const int n0 = prefix[p0.E];
+  const int n1 = nft1 * (int)((p1.rows_max + kCoBN1 - 1) / kCoBN1);
+  const int total = n0 + n1;
+  const int nkb0 = (p0.K + kBK - 1) / kBK;
+  const int nkb1 = (p1.K + kBK - 1) / kBK;
+  // problem and tile of combined tile t
+  auto which = [&](int t, int& local) -> int {
+    const int c = (int)(((int64_t)t * n0) / total);
+    const int c1 = (int)(((int64_t)(t + 1) * n0) / total);
+    if (c1 > c) {
+      local = c;
+      return 0;
+    }
+    local = t - c;
+    return 1;
+  };
+  constexpr uint32_t kA0 = 2 * kBM * kBK * 2;  // two weight boxes
+  constexpr uint32_t kA1 = kBM * kBK * 2;      // one weight box
+
+  if (warp == 0) {
+    if (lane == 0) {
+      Ring ring;
+      int issued = 0;
+      for (int t = blockIdx.x; t < total; t += gridDim.x) {
+        int u;
+        const bool ok = which(t, u) == 0
+                            ? produce_tile<BN0, 2, false>(decode_tile<BN0, 2>(u, prefix, seg, p0.E, nft0),
+                                                          &tmW0, &tmX0, p0, nkb0, base_addr,
+                                                          kCoStageBytes, kA0, B, ring, issued,
+                                                          abort_flag)
+                            : produce_tile<kCoBN1, 1, false>(
+                                  decode_dense_tile<kCoBN1, 1>(u, p1.rows_max, nft1), &tmW1, &tmX1,
+                                  p1, nkb1, base_addr, kCoStageBytes, kA1, B, ring, issued,
+                                  abort_flag);
+        if (!ok) break;
+      }
+      for (int i = max(0, issued - S); i < issued; ++i)
+        mbar_wait_drain(B.full(i % S), (uint32_t)((i / S) & 1), p0.status);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      Ring ring;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      for (int t = blockIdx.x; t < total; t += gridDim.x) {
+        if (!mbar_wait_bounded(B.tempty(acc), acc_phase ^ 1u, abort_flag, p0.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kCoAccCols);
+        int u;
+        const bool ok = which(t, u) == 0
+                            ? mma_tile<BN0, 2, false>(decode_tile<BN0, 2>(u, prefix, seg, p0.E, nft0),
+                                                      d_tmem, p0, nkb0, base_addr, kCoStageBytes,
+                                                      kA0, B, ring, abort_flag)
+                            : mma_tile<kCoBN1, 1, false>(
+                                  decode_dense_tile<kCoBN1, 1>(u, p1.rows_max, nft1), d_tmem, p1,
+                                  nkb1, base_addr, kCoStageBytes, kA1, B, ring, abort_flag);
+        if (!ok) break;
+        tc_commit(B.tfull(acc));
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      tc_commit(B.drain());
+      mbar_wait_drain(B.drain(), 0, p0.status);
+    }
+  } else {
+    const int ew = warp - 2;
+    const int quarter = warp & 3;
+    const int half = ew >> 2;
+    uint8_t* st = stage_tiles + ew * kStageTileBytes;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      if (!mbar_wait_bounded_warp(B.tfull(acc), acc_phase, abort_flag, p0.status)) break;
+      tc_fence_after();
+      const uint32_t acc_tmem = tmem_base + (uint32_t)(acc * kCoAccCols);
+      int u;
+      if (which(t, u) == 0)
+        epilogue_tile<BN0, 2, EPI>(decode_tile<BN0, 2>(u, prefix, seg, p0.E, nft0), p0, acc_tmem,
+                                   quarter, half, lane, st);
+      else
+        epilogue_tile<kCoBN1, 1, EPI>(decode_dense_tile<kCoBN1, 1>(u, p1.rows_max, nft1), p1,
+                                      acc_tmem, quarter, half, lane, st);
+      tc_fence_before();
+      mbar_arrive(B.tempty(acc));
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  pdl_trigger();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 2 * kCoAccCols);
   }
 }
 
@@ -600,6 +861,18 @@ cudaError_t launch_one(const CUtensorMap& tmW, const CUtensorMap& tmX, const Par
   cudaError_t e = ensure_dynamic_smem(kern, smem, attr_done);
   if (e != cudaSuccess) return e;
   return launch_kernel(kern, dim3(num_sms()), dim3(kThreads), smem, stream, tmW, tmX, p);
+}
+
+template <int BN0, int EPI>
+cudaError_t launch_co(const CUtensorMap& tmW0, const CUtensorMap& tmX0, const CUtensorMap& tmW1,
+                      const CUtensorMap& tmX1, const Params& p0, const Params& p1,
+                      cudaStream_t stream) {
+  auto kern = co_gemm_kernel<BN0, EPI>;
+  static int attr_done[64] = {0};  // per instantiation and device
+  cudaError_t e = ensure_dynamic_smem(kern, kCoSmemBytes, attr_done);
+  if (e != cudaSuccess) return e;
+  return launch_kernel(kern, dim3(num_sms()), dim3(kThreads), kCoSmemBytes, stream, tmW0, tmX0,
+                       tmW1, tmX1, p0, p1);
 }
 
 }  // namespace
@@ -722,6 +995,56 @@ cudaError_t enqueue_gemm2_combine(const void* h, const int32_t* offsets, int E, 
   Params p{offsets, E, N, K, rows_max, bias, nullptr, status, c, nullptr, nullptr};
   return fc.dense ? launch_bn<kEpiCombineDense>(BN, tmW, tmX, p, stream, capacity_hint)
                   : launch_bn<kEpiCombineExpert>(BN, tmW, tmX, p, stream, capacity_hint);
+}
+
+bool co_gemm_supported(int64_t capacity_hint) {
+  return pick_token_tile(capacity_hint) <= 128;  // two expert accumulators fit one 256-column buffer
+}
+
+cudaError_t enqueue_co_gemm_bf16(const void* xp, const int32_t* offsets, int E, int64_t rows_max,
+                                 const void* w, const void* bias, void* out, int64_t capacity_hint,
+                                 const void* x_dense, int64_t T, const void* w_dense,
+                                 const void* bias_dense, void* out_dense, int K, int N, bool gelu,
+                                 int* status, cudaStream_t stream) {
+  if (T == 0 && rows_max == 0) return cudaSuccess;
+  const int BN0 = pick_token_tile(capacity_hint);
+  if (BN0 > 128) return cudaErrorInvalidValue;
+  CUtensorMap tmW0, tmX0, tmW1, tmX1;
+  // an empty expert problem still needs valid maps: point them at the dense operands (no tile
+  // of problem 0 exists, so nothing is loaded through them)
+  const bool no_rows = rows_max == 0;
+  if (!make_kmajor_map(&tmW0, w, (int64_t)E * N, K, kBM) ||
+      !make_kmajor_map(&tmX0, no_rows ? x_dense : xp, no_rows ? T : rows_max, K, BN0) ||
+      !make_kmajor_map(&tmW1, w_dense, N, K, kBM) ||
+      !make_kmajor_map(&tmX1, x_dense, T, K, kCoBN1))
+    return cudaErrorInvalidValue;
+  Params p0{offsets, E, N, K, rows_max, bias, out, status, CombineArgs{}, nullptr, nullptr};
+  Params p1{nullptr, 1, N, K, T, bias_dense, out_dense, status, CombineArgs{}, nullptr, nullptr};
+  auto go = [&](auto tag) -> cudaError_t {
+    constexpr int EPI = decltype(tag)::value;
+    switch (BN0) {
+      case 16: return launch_co<16, EPI>(tmW0, tmX0, tmW1, tmX1, p0, p1, stream);
+      case 32: return launch_co<32, EPI>(tmW0, tmX0, tmW1, tmX1, p0, p1, stream);
+      case 64: return launch_co<64, EPI>(tmW0, tmX0, tmW1, tmX1, p0, p1, stream);
+      default: return launch_co<128, EPI>(tmW0, tmX0, tmW1, tmX1, p0, p1, stream);
+    }
+  };
+  return gelu ? go(std::integral_constant<int, kEpiGeluBf16>{})
+              : go(std::integral_constant<int, kEpiF32>{});
+}
+
+cudaError_t enqueue_selftest_bounded_wait(void* scratch, uint64_t wait_limit_ns, int* status,
+                                         cudaStream_t stream) {
+  // one expert of 128 features x 64 K and one 16-row token tile, maps over the scratch (nothing
+  // is copied: the TMA role is told to issue no copy)
+  uint8_t* b = static_cast<uint8_t*>(scratch);
+  CUtensorMap tmW, tmX;
+  if (!make_kmajor_map(&tmW, b, kBM, kBK, kBM) || !make_kmajor_map(&tmX, b, 16, kBK, 16))
+    return cudaErrorInvalidValue;
+  Params p{nullptr, 1, kBM, kBK, 16, nullptr, b, status, CombineArgs{}, nullptr, nullptr};
+  p.selftest_no_copies = 1;
+  p.wait_limit_ns = wait_limit_ns;
+  return launch_one<16, kEpiF32, false, 1>(tmW, tmX, p, stream);
 }
 
 cudaError_t enqueue_expert_ffn_bf16(const void* x_packed, const int32_t* offsets, int E,

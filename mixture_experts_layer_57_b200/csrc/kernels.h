@@ -18,6 +18,8 @@ int num_sms();
 
 // Whether launches carry the programmatic-dependent-launch attribute (MOE_PDL=0 disables it).
 bool pdl_enabled();
+// Whether bf16 PR-MoE layers co-schedule expert and dense GEMM layers (MOE_COSCHEDULE=0: no).
+bool coschedule_enabled();
 
 // Launches kern<<<grid, block, smem, stream>>>(args...) as a programmatic dependent launch and
 // counts it.
@@ -74,7 +76,8 @@ struct RouterDispatchCount {
 // int64 (the accumulators' fixed-point values); sums over shards give the whole batch's.
 inline int64_t router_partials_count(int E) { return 4 * (int64_t)E + 1; }
 // logits may be nullptr (not returned).
-// renormalize: gates of the k choices divided by their sum. losses (optional): [z-loss,
+// renormalize: gates of the k choices divided by their sum; probs (optional, [T, k]): the chosen
+// experts' probabilities before that division (the priority ranking key). losses (optional): [z-loss,
 // CoV^2 of Importance, CoV^2 of Load]. export_partials (optional): instead of finalising, the
 // last block writes the integer partials there (lb_stats and losses must then be nullptr).
 cudaError_t enqueue_router(const void* x, bool x_bf16, int64_t T, int d, const float* w_router,
@@ -83,7 +86,13 @@ cudaError_t enqueue_router(const void* x, bool x_bf16, int64_t T, int d, const f
                            const RouterScratch& scratch, int* status, cudaStream_t stream,
                            RouterDispatchCount dcount = RouterDispatchCount{},
                            bool renormalize = false, float* losses = nullptr,
-                           int64_t* export_partials = nullptr, int64_t T_kernel_choice = -1);
+                           int64_t* export_partials = nullptr, int64_t T_kernel_choice = -1,
+                           float* probs = nullptr, const uint16_t* w_prepared = nullptr);
+// w_prepared (optional): W_r already split (enqueue_router_prepare); the tensor-core path then
+// skips the split, and the logits kernel zeroes the statistics accumulators instead.
+// Splits W_r [E, d] into the three bf16 parts [E, 3 * router_split_dpad(d)].
+cudaError_t enqueue_router_prepare(const float* w_router, int E, int d, uint16_t* out,
+                                   cudaStream_t stream);
 // T_kernel_choice (>= T): the batch size that selects the logits kernel (a token shard takes the
 // whole batch's, so every token's logits come from the same arithmetic).
 // f, Q, aux (lb_stats, optional) and the router losses (optional) from summed partials of T
@@ -91,9 +100,11 @@ cudaError_t enqueue_router(const void* x, bool x_bf16, int64_t T, int d, const f
 cudaError_t enqueue_router_finalize(const int64_t* totals, int64_t T, int E, float aux_alpha,
                                     float* lb_stats, float* losses, cudaStream_t stream);
 // logits = x W_r^T + b_r on tcgen05 from the exact split W_r = hi + mid + lo (bf16 each).
+// zero_acc (optional): accumulators the kernel zeroes before its dependents start.
 cudaError_t enqueue_router_logits_tc(const void* x, int64_t T, int d, const uint16_t* w_split,
                                      int dpad, const float* router_bias, int E, float* logits,
-                                     int* status, cudaStream_t stream);
+                                     int* status, cudaStream_t stream,
+                                     const RouterAccum* zero_acc = nullptr);
 
 // Raises a kernel's dynamic shared-memory limit to `bytes` on the current device, once per
 // device (done_per_device: a zero-initialised [64] array owned by the launching function).
@@ -109,6 +120,26 @@ cudaError_t ensure_dynamic_smem(Kern kern, int bytes, int* done_per_device) {
   return e;
 }
 
+// One layer of the experts and one layer of the PR-MoE dense MLP co-scheduled in one persistent
+// launch (the expert tiles stream weights from HBM, the dense tiles keep the tensor pipe busy):
+//   experts: out[r] = act(W[e] xp[r] + bias[e]) for the packed rows of every expert (offsets),
+//   dense:   out_dense[t] = act(W_dense x_dense[t] + bias_dense) for t < T,
+// both with K inputs and N outputs; gelu: bf16 GeLU outputs (layer 1), else fp32 (layer 2).
+// co_gemm_supported: whether the expert token tile (from capacity_hint) allows it (<= 128 rows).
+bool co_gemm_supported(int64_t capacity_hint);
+cudaError_t enqueue_co_gemm_bf16(const void* xp, const int32_t* offsets, int E, int64_t rows_max,
+                                 const void* w, const void* bias, void* out, int64_t capacity_hint,
+                                 const void* x_dense, int64_t T, const void* w_dense,
+                                 const void* bias_dense, void* out_dense, int K, int N, bool gelu,
+                                 int* status, cudaStream_t stream);
+
+// Failure-detection self-test: one grouped-GEMM launch whose TMA role issues no copy, so its MMA
+// role waits on a barrier nobody arrives at; every wait gives up after wait_limit_ns, records
+// MOE_DEVERR_TIMEOUT in *status and the kernel returns. scratch: >= 32 KB of device memory (the
+// tensor maps' base; never read or written).
+cudaError_t enqueue_selftest_bounded_wait(void* scratch, uint64_t wait_limit_ns, int* status,
+                                         cudaStream_t stream);
+
 // ---------------------------------------------------------------- dispatch
 constexpr int kDispatchSeg = 256;  // (token, choice) pairs per counting segment (one warp)
 inline int64_t dispatch_num_segments(int64_t pairs) {
@@ -121,11 +152,12 @@ struct DroppedRows {
   bool out_bf16 = true;
   bool add_x = true;
 };
-// Overflow by priority (optional): each expert keeps its C pairs of largest gate (ties -> lower
-// pair index) and packs them in that order. prio_list [T k] and demand_offsets [E + 1] are scratch.
+// Overflow by priority (optional): each expert keeps its C pairs of largest router probability
+// (ties -> lower pair index) and packs them in that order. keys [2 T k] (two ping-pong halves of
+// 64-bit sort keys) and demand_offsets [E + 1] are scratch.
 struct PriorityDispatch {
-  const float* gates = nullptr;  // [T, k]; nullptr = first-come
-  int32_t* list = nullptr;
+  const float* probs = nullptr;  // [T, k] probabilities before renormalisation; nullptr = first-come
+  uint64_t* keys = nullptr;
   int32_t* demand_offsets = nullptr;
 };
 // Token shards (optional): this shard is `rank` of G consecutive token blocks; demand_all [G, E]

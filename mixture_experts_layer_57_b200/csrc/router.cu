@@ -157,7 +157,7 @@ __global__ void __launch_bounds__(256) router_prep_kernel(const float* __restric
                                                           int d, int dpad, uint16_t* __restrict__ out,
                                                           RouterAccum acc) {
   pdl_wait();
-  if (blockIdx.x == 0) {
+  if (blockIdx.x == 0 && acc.q != nullptr) {
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
       acc.q[e] = 0ull;
       acc.c[e] = 0u;
@@ -266,7 +266,8 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
                                                           float* __restrict__ lb,
                                                           RouterDispatchCount dc, int renorm,
                                                           float* __restrict__ losses,
-                                                          int64_t* __restrict__ exported) {
+                                                          int64_t* __restrict__ exported,
+                                                          float* __restrict__ probs) {
   __shared__ float qs[8][MOE_MAX_EXPERTS];
   // per expert: first-choice count << 16 | choice count (each at most kRouterTokensPerBlock)
   __shared__ unsigned cs[MOE_MAX_EXPERTS];
@@ -373,6 +374,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
       if (lane == owner) taken |= 1u << slot_i;
       if (lane == 0) {
         ids[t * k + j] = bi;
+        if (probs != nullptr) probs[t * k + j] = pv;  // before any renormalisation
         if (!renorm) {
           gates[t * k + j] = pv;
           count_choice(bi, j, pv);
@@ -481,12 +483,13 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
 template <int EPL>
 cudaError_t launch_topk(const float* logits, int64_t T, int E, int k, int32_t* ids, float* gates,
                         const RouterAccum& acc, float alpha, float* lb, RouterDispatchCount dc,
-                        int renorm, float* losses, int64_t* exported, cudaStream_t stream) {
+                        int renorm, float* losses, int64_t* exported, float* probs,
+                        cudaStream_t stream) {
   const dim3 grid((unsigned)router_num_blocks(T));
   const bool extra = losses != nullptr || exported != nullptr;
   auto go = [&](auto kern) {
     return launch_kernel(kern, grid, dim3(256), 0, stream, (const float*)logits, T, E, k, ids,
-                         gates, acc, alpha, lb, dc, renorm, losses, exported);
+                         gates, acc, alpha, lb, dc, renorm, losses, exported, probs);
   };
   if (dc.local_rank != nullptr)
     return extra ? go(router_topk_kernel<EPL, true, true>)
@@ -502,26 +505,29 @@ cudaError_t enqueue_router(const void* x, bool x_bf16, int64_t T, int d, const f
                            float* gates, float* lb_stats, float aux_alpha,
                            const RouterScratch& scr, int* status, cudaStream_t stream,
                            RouterDispatchCount dc, bool renormalize, float* losses,
-                           int64_t* exported, int64_t T_kernel_choice) {
+                           int64_t* exported, int64_t T_kernel_choice, float* probs,
+                           const uint16_t* w_prepared) {
   if (T == 0) return cudaSuccess;
   if (!logits) logits = scr.logits_scratch;
   const bool gemv = (T_kernel_choice > T ? T_kernel_choice : T) <= kRouterGemvMaxT;
   const bool tc = !gemv && router_uses_tensor_cores(x_bf16, d);
+  const bool prepared = tc && w_prepared != nullptr;
   const int dpad = router_split_dpad(d);
   const int64_t n = tc ? (int64_t)E * dpad : 0;
   const unsigned blocks = (unsigned)(n == 0 ? 1 : ((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096));
-  cudaError_t err;
+  cudaError_t err = cudaSuccess;
   if (gemv) {
     err = launch_kernel(x_bf16 ? router_gemv_kernel<true> : router_gemv_kernel<false>, dim3(E),
                         dim3(256), 0, stream, x, w_router, router_bias, T, d, E, logits, scr.acc);
-  } else {
+  } else if (!prepared) {
     err = launch_kernel(router_prep_kernel, dim3(blocks), dim3(256), 0, stream, w_router, E, d, dpad,
                         tc ? scr.w_split : nullptr, scr.acc);
   }
   if (err != cudaSuccess) return err;
   if (tc) {
-    cudaError_t e = enqueue_router_logits_tc(x, T, d, scr.w_split, dpad, router_bias, E, logits,
-                                             status, stream);
+    cudaError_t e = enqueue_router_logits_tc(x, T, d, prepared ? w_prepared : scr.w_split, dpad,
+                                             router_bias, E, logits, status, stream,
+                                             prepared ? &scr.acc : nullptr);
     if (e != cudaSuccess) return e;
   } else if (!gemv) {
     dim3 grid((unsigned)((T + kLBM - 1) / kLBM), (E + kLBN - 1) / kLBN);
@@ -533,21 +539,31 @@ cudaError_t enqueue_router(const void* x, bool x_bf16, int64_t T, int d, const f
   const int rn = renormalize ? 1 : 0;
   if (E <= 32)
     return launch_topk<1>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, rn,
-                          losses, exported, stream);
+                          losses, exported, probs, stream);
   if (E <= 64)
     return launch_topk<2>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, rn,
-                          losses, exported, stream);
+                          losses, exported, probs, stream);
   if (E <= 128)
     return launch_topk<4>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, rn,
-                          losses, exported, stream);
+                          losses, exported, probs, stream);
   if (E <= 256)
     return launch_topk<8>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, rn,
-                          losses, exported, stream);
+                          losses, exported, probs, stream);
   if (E <= 512)
     return launch_topk<16>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, rn,
-                           losses, exported, stream);
+                           losses, exported, probs, stream);
   return launch_topk<32>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, rn,
-                         losses, exported, stream);
+                         losses, exported, probs, stream);
+}
+
+cudaError_t enqueue_router_prepare(const float* w_router, int E, int d, uint16_t* out,
+                                   cudaStream_t stream) {
+  const int dpad = router_split_dpad(d);
+  const int64_t n = (int64_t)E * dpad;
+  const unsigned blocks = (unsigned)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+  // no statistics here: an accumulator set whose pointers are all null is skipped by block 0
+  return launch_kernel(router_prep_kernel, dim3(blocks), dim3(256), 0, stream, w_router, E, d,
+                       dpad, out, RouterAccum{});
 }
 
 cudaError_t enqueue_router_finalize(const int64_t* totals, int64_t T, int E, float aux_alpha,

@@ -49,6 +49,8 @@ struct RParams {
   const float* bias;  // [E] fp32 or nullptr
   float* logits;      // [T, E]
   int* status;
+  RouterAccum acc;    // zeroed by block 0 when zero_acc (no split kernel ran before this one)
+  int zero_acc;
 };
 
 __device__ __forceinline__ void mbar_wait_drain_r(uint32_t bar, uint32_t parity, int* status) {
@@ -101,6 +103,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     tma_prefetch_desc(&tmX);
     tma_prefetch_desc(&tmW);
+  }
+  if (p.zero_acc && blockIdx.x == 0) {
+    for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
+      p.acc.q[e] = 0ull;
+      p.acc.c[e] = 0u;
+      p.acc.imp[e] = 0ull;
+      p.acc.load[e] = 0u;
+    }
+    if (threadIdx.x == 0) {
+      *p.acc.z = 0ull;
+      *p.acc.ticket = 0u;
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_holder), C::kTmemCols);
@@ -279,7 +293,7 @@ cudaError_t launch_tc(const CUtensorMap& tmX, const CUtensorMap& tmW, const RPar
 
 cudaError_t enqueue_router_logits_tc(const void* x, int64_t T, int d, const uint16_t* w_split,
                                      int dpad, const float* router_bias, int E, float* logits,
-                                     int* status, cudaStream_t stream) {
+                                     int* status, cudaStream_t stream, const RouterAccum* zero_acc) {
   if (T == 0) return cudaSuccess;
   const int slice = E < kSlice ? E : kSlice;
   int NE = 16;
@@ -288,7 +302,8 @@ cudaError_t enqueue_router_logits_tc(const void* x, int64_t T, int d, const uint
   CUtensorMap tmX, tmW;
   if (!make_map(&tmX, x, T, d, kTM) || !make_map(&tmW, w_split, E, 3 * dpad, NE))
     return cudaErrorInvalidValue;
-  const RParams p{T, E, dpad, n_slices, router_bias, logits, status};
+  const RParams p{T, E, dpad, n_slices, router_bias, logits, status,
+                  zero_acc ? *zero_acc : RouterAccum{}, zero_acc ? 1 : 0};
   const int ntiles = (int)((T + kTM - 1) / kTM) * n_slices;
   switch (NE) {
     case 16: return launch_tc<16>(tmX, tmW, p, ntiles, stream);

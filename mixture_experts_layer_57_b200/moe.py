@@ -45,14 +45,15 @@ class LayerArgs(ctypes.Structure):
                 ("dense_b1", ctypes.c_void_p), ("dense_w2", ctypes.c_void_p),
                 ("dense_b2", ctypes.c_void_p), ("add_input_residual", ctypes.c_int),
                 ("aux_alpha", ctypes.c_float), ("overflow_policy", ctypes.c_int),
-                ("renormalize_gates", ctypes.c_int)]
+                ("renormalize_gates", ctypes.c_int), ("w_router_prepared", ctypes.c_void_p)]
 
 
 class LayerAux(ctypes.Structure):
     _fields_ = [("logits", ctypes.c_void_p), ("expert_ids", ctypes.c_void_p),
                 ("gates", ctypes.c_void_p), ("slot", ctypes.c_void_p),
                 ("expert_counts", ctypes.c_void_p), ("expert_offsets", ctypes.c_void_p),
-                ("lb_stats", ctypes.c_void_p), ("router_losses", ctypes.c_void_p)]
+                ("lb_stats", ctypes.c_void_p), ("router_losses", ctypes.c_void_p),
+                ("topk_probs", ctypes.c_void_p)]
 
 
 class LayerGrads(ctypes.Structure):
@@ -82,9 +83,11 @@ def lib() -> ctypes.CDLL:
             "moe_capacity": ([i64, i32, i32, f64, P(i64)], i32),
             "moe_packed_rows_max": ([i64, i32, i32, i64, P(i64)], i32),
             "moe_router_workspace_bytes": ([i64, i32, i32, P(sz)], i32),
+            "moe_router_prepare_bytes": ([i32, i32, P(sz)], i32),
+            "moe_router_prepare": ([vp, i32, i32, vp, sz, vp], i32),
             "moe_router_topk": ([vp, i32, i64, i32, vp, vp, i32, i32, vp, vp, vp, vp, f32, vp, sz, vp], i32),
             "moe_router_topk_ex": ([vp, i32, i64, i32, vp, vp, i32, i32, vp, vp, vp, vp, f32, i32, vp,
-                                    vp, sz, vp], i32),
+                                    vp, vp, sz, vp], i32),
             "moe_dispatch_workspace_bytes": ([i64, i32, i32, P(sz)], i32),
             "moe_dispatch": ([vp, i32, i64, i32, vp, i32, i32, i64, vp, vp, vp, vp, vp, i64, vp, sz, vp], i32),
             "moe_dispatch_priority": ([vp, i32, i64, i32, vp, vp, i32, i32, i64, vp, vp, vp, vp, vp, i64,
@@ -109,6 +112,7 @@ def lib() -> ctypes.CDLL:
             "moe_layer_backward": ([P(LayerArgs), vp, f32, f32, P(LayerGrads), vp, sz, vp], i32),
             "moe_workspace_reset": ([vp, sz, vp], i32),
             "moe_get_device_error": ([vp, P(i32), vp], i32),
+            "moe_selftest_bounded_wait": ([vp, sz, ctypes.c_uint64, vp], i32),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -181,6 +185,20 @@ def _ws_bytes(fn: str, *args) -> int:
     return out.value
 
 
+def moe_router_prepare(w_router: torch.Tensor, out: Optional[torch.Tensor] = None,
+                       stream=None) -> torch.Tensor:
+    """The router weight split for the tensor-core logits kernel (pass it to layer_args as
+    w_router_prepared; prepare again whenever w_router changes)."""
+    E, d = w_router.shape
+    n = ctypes.c_size_t()
+    _check("moe_router_prepare_bytes", lib().moe_router_prepare_bytes(E, d, ctypes.byref(n)))
+    if out is None:
+        out = torch.empty(n.value, dtype=torch.uint8, device=w_router.device)
+    _check("moe_router_prepare", lib().moe_router_prepare(_ptr(w_router), E, d, _ptr(out),
+                                                          out.numel(), _stream(stream)))
+    return out
+
+
 def moe_router_workspace_bytes(T, E, d_model):
     return _ws_bytes("moe_router_workspace_bytes", T, E, d_model)
 
@@ -203,9 +221,10 @@ def moe_router_topk(x: torch.Tensor, w_router: torch.Tensor, k: int,
                     router_bias: Optional[torch.Tensor] = None, logits=None, expert_ids=None,
                     gates=None, lb_stats=None, aux_alpha: float = 0.01, want_stats: bool = True,
                     ws: Optional[torch.Tensor] = None, stream=None, renormalize: bool = False,
-                    router_losses=None) -> dict:
+                    router_losses=None, probs=None) -> dict:
     """moe_router_topk, or moe_router_topk_ex when ``renormalize`` is set or ``router_losses``
-    (a [3] fp32 tensor, or True to allocate one) is given."""
+    (a [3] fp32 tensor, or True to allocate one) or ``probs`` (a [T, k] fp32 tensor, or True:
+    the probabilities before renormalisation) is given."""
     T, d = x.shape
     E = w_router.shape[0]
     dev = x.device
@@ -221,24 +240,27 @@ def moe_router_topk(x: torch.Tensor, w_router: torch.Tensor, k: int,
         ws = workspace(moe_router_workspace_bytes(T, E, d), dev)
     if router_losses is True:
         router_losses = torch.empty(3, dtype=torch.float32, device=dev)
-    if renormalize or router_losses is not None:
+    if probs is True:
+        probs = torch.empty(T, k, dtype=torch.float32, device=dev)
+    if renormalize or router_losses is not None or probs is not None:
         _check("moe_router_topk_ex", lib().moe_router_topk_ex(
             _ptr(x), _dt(x), T, d, _ptr(w_router), _ptr(router_bias), E, k, _ptr(logits),
             _ptr(expert_ids), _ptr(gates), _ptr(lb_stats), aux_alpha, int(bool(renormalize)),
-            _ptr(router_losses), _ptr(ws), ws.numel(), _stream(stream)))
+            _ptr(router_losses), _ptr(probs), _ptr(ws), ws.numel(), _stream(stream)))
     else:
         _check("moe_router_topk", lib().moe_router_topk(
             _ptr(x), _dt(x), T, d, _ptr(w_router), _ptr(router_bias), E, k, _ptr(logits),
             _ptr(expert_ids), _ptr(gates), _ptr(lb_stats), aux_alpha, _ptr(ws), ws.numel(),
             _stream(stream)))
     return dict(logits=logits, expert_ids=expert_ids, gates=gates, lb_stats=lb_stats, ws=ws,
-                router_losses=router_losses)
+                router_losses=router_losses, probs=probs)
 
 
 def moe_dispatch(x: torch.Tensor, expert_ids: torch.Tensor, E: int, C: int, rows_max=None,
                  slot=None, expert_counts=None, expert_offsets=None, row_token=None, x_packed=None,
-                 ws=None, stream=None, priority_gates: Optional[torch.Tensor] = None) -> dict:
-    """moe_dispatch, or moe_dispatch_priority when ``priority_gates`` ([T, k] fp32) is given."""
+                 ws=None, stream=None, priority_probs: Optional[torch.Tensor] = None) -> dict:
+    """moe_dispatch, or moe_dispatch_priority when ``priority_probs`` ([T, k] fp32 router
+    probabilities before any renormalisation) is given."""
     T, d = x.shape
     k = expert_ids.shape[1]
     dev = x.device
@@ -256,9 +278,9 @@ def moe_dispatch(x: torch.Tensor, expert_ids: torch.Tensor, E: int, C: int, rows
         x_packed = torch.empty(max(rows_max, 1), d, dtype=x.dtype, device=dev)
     if ws is None:
         ws = workspace(moe_dispatch_workspace_bytes(T, E, k), dev)
-    if priority_gates is not None:
+    if priority_probs is not None:
         _check("moe_dispatch_priority", lib().moe_dispatch_priority(
-            _ptr(x), _dt(x), T, d, _ptr(expert_ids), _ptr(priority_gates), E, k, C, _ptr(slot),
+            _ptr(x), _dt(x), T, d, _ptr(expert_ids), _ptr(priority_probs), E, k, C, _ptr(slot),
             _ptr(expert_counts), _ptr(expert_offsets), _ptr(row_token), _ptr(x_packed), rows_max,
             _ptr(ws), ws.numel(), _stream(stream)))
     else:
@@ -365,7 +387,7 @@ def moe_combine(y_packed: torch.Tensor, expert_offsets, expert_ids, slot, gates,
 def layer_args(x, w_router, w1, b1, w2, b2, k: int, capacity_factor: float, router_bias=None,
                dense=None, add_input_residual: bool = True, aux_alpha: float = 0.01,
                out_dtype=None, overflow_priority: bool = False,
-               renormalize_gates: bool = False) -> LayerArgs:
+               renormalize_gates: bool = False, w_router_prepared=None) -> LayerArgs:
     """Fill a ``moe_layer_args`` struct from tensors (dense = (w1, b1, w2, b2) or None)."""
     T, d = x.shape
     E, d_ff, _ = w1.shape
@@ -380,7 +402,8 @@ def layer_args(x, w_router, w1, b1, w2, b2, k: int, capacity_factor: float, rout
                      aux_alpha=aux_alpha,
                      overflow_policy=MOE_OVERFLOW_PRIORITY if overflow_priority else
                      MOE_OVERFLOW_FIRST_COME,
-                     renormalize_gates=int(bool(renormalize_gates)))
+                     renormalize_gates=int(bool(renormalize_gates)),
+                     w_router_prepared=_ptr(w_router_prepared))
 
 
 def moe_layer_workspace_bytes(args: LayerArgs) -> int:
@@ -549,3 +572,18 @@ def moe_get_device_error(ws: torch.Tensor, stream=None) -> int:
 
 def moe_last_launch_count() -> int:
     return lib().moe_last_launch_count()
+
+
+MOE_SELFTEST_WS_BYTES = 256 + 32768
+
+
+def moe_selftest_bounded_wait(wait_limit_ns: int, ws: Optional[torch.Tensor] = None,
+                              device=None, stream=None) -> torch.Tensor:
+    """Enqueue the failure-detection self-test (a grouped-GEMM launch whose wait can never
+    complete and must give up after ``wait_limit_ns``); returns the workspace whose status
+    block then holds MOE_DEVERR_TIMEOUT (read it with moe_get_device_error)."""
+    if ws is None:
+        ws = workspace(MOE_SELFTEST_WS_BYTES, device if device is not None else "cuda")
+    _check("moe_selftest_bounded_wait", lib().moe_selftest_bounded_wait(
+        _ptr(ws), ws.numel(), int(wait_limit_ns), _stream(stream)))
+    return ws

@@ -68,26 +68,39 @@ void synth_uniform_f64(uint64_t seed, uint64_t stream, uint64_t offset, int64_t 
   for (int64_t i = 0; i < n; ++i) out[i] = uniform01(key, offset + (uint64_t)i);
 }
 
+/* Normal draws of elements [offset, offset + n): each Box-Muller pair (2m, 2m + 1) is formed once
+ * and gives both of its elements (the same values as normal01 element by element). */
+#define SYNTH_NORMAL_LOOP(STORE)                                                          \
+  const uint64_t key = synth_key(seed, stream);                                           \
+  if (n <= 0) return;                                                                     \
+  const int64_t m0 = (int64_t)(offset >> 1), m1 = (int64_t)((offset + (uint64_t)n - 1) >> 1); \
+  _Pragma("omp parallel for schedule(static)")                                            \
+  for (int64_t m = m0; m <= m1; ++m) {                                                    \
+    const double u1 = uniform01(key, 2 * (uint64_t)m);                                    \
+    const double u2 = uniform01(key, 2 * (uint64_t)m + 1);                                \
+    const double r = sqrt(-2.0 * log(u1));                                                \
+    const double a = 6.283185307179586476925286766559 * u2;                               \
+    for (int b = 0; b < 2; ++b) {                                                         \
+      const uint64_t i = 2 * (uint64_t)m + (uint64_t)b;                                   \
+      if (i < offset || i >= offset + (uint64_t)n) continue;                              \
+      const double v = mean + std * (b ? r * sin(a) : r * cos(a));                        \
+      STORE;                                                                              \
+    }                                                                                     \
+  }
+
 void synth_normal_f64(uint64_t seed, uint64_t stream, uint64_t offset, int64_t n, double mean,
                       double std, double* out) {
-  const uint64_t key = synth_key(seed, stream);
-#pragma omp parallel for schedule(static)
-  for (int64_t i = 0; i < n; ++i) out[i] = mean + std * normal01(key, offset + (uint64_t)i);
+  SYNTH_NORMAL_LOOP(out[i - offset] = v)
 }
 
 void synth_normal_f32(uint64_t seed, uint64_t stream, uint64_t offset, int64_t n, double mean,
                       double std, float* out) {
-  const uint64_t key = synth_key(seed, stream);
-#pragma omp parallel for schedule(static)
-  for (int64_t i = 0; i < n; ++i) out[i] = (float)(mean + std * normal01(key, offset + (uint64_t)i));
+  SYNTH_NORMAL_LOOP(out[i - offset] = (float)v)
 }
 
 void synth_normal_bf16(uint64_t seed, uint64_t stream, uint64_t offset, int64_t n, double mean,
                        double std, uint16_t* out) {
-  const uint64_t key = synth_key(seed, stream);
-#pragma omp parallel for schedule(static)
-  for (int64_t i = 0; i < n; ++i)
-    out[i] = f32_to_bf16_bits((float)(mean + std * normal01(key, offset + (uint64_t)i)));
+  SYNTH_NORMAL_LOOP(out[i - offset] = f32_to_bf16_bits((float)v))
 }
 
 /* A seeded permutation of 1..n (Fisher-Yates, swap index from draw % (i + 1)). */

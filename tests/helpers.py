@@ -48,7 +48,7 @@ def dev_inputs(inp: dict, device="cuda") -> dict:
 
 def run_layer(w: synth.Workload, d_inp: dict, out_dtype=None, add_input_residual=None,
               ws: torch.Tensor = None, overflow_priority: bool = False, renormalize: bool = False,
-              want_losses: bool = False) -> dict:
+              want_losses: bool = False, w_router_prepared=None) -> dict:
     """One moe_layer_forward on device inputs; returns host copies of every output."""
     T, E, k = w.T, w.E, w.k
     x = d_inp["x"]
@@ -60,7 +60,7 @@ def run_layer(w: synth.Workload, d_inp: dict, out_dtype=None, add_input_residual
                           k=k, capacity_factor=w.capacity_factor, router_bias=d_inp.get("router_bias"),
                           dense=dense, add_input_residual=res, aux_alpha=w.aux_alpha,
                           out_dtype=out_dtype, overflow_priority=overflow_priority,
-                          renormalize_gates=renormalize)
+                          renormalize_gates=renormalize, w_router_prepared=w_router_prepared)
     dev = x.device
     aux = dict(logits=torch.empty(T, E, dtype=torch.float32, device=dev),
                expert_ids=torch.empty(T, k, dtype=torch.int32, device=dev),
@@ -68,7 +68,8 @@ def run_layer(w: synth.Workload, d_inp: dict, out_dtype=None, add_input_residual
                slot=torch.empty(T, k, dtype=torch.int32, device=dev),
                expert_counts=torch.empty(E, dtype=torch.int32, device=dev),
                expert_offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
-               lb_stats=torch.empty(2 * E + 1, dtype=torch.float32, device=dev))
+               lb_stats=torch.empty(2 * E + 1, dtype=torch.float32, device=dev),
+               topk_probs=torch.empty(T, k, dtype=torch.float32, device=dev))
     if want_losses:
         aux["router_losses"] = torch.empty(3, dtype=torch.float32, device=dev)
     odt = x.dtype if out_dtype is None else out_dtype
@@ -108,3 +109,62 @@ def check_out(got: np.ndarray, ref: np.ndarray, layer_bf16: bool, out_bf16: bool
         assert not bad.any(), f"{what}: {bad.sum()} elements beyond 2e-2 + half ulp (max {max_abs})"
         assert rel <= BF16_REL_L2, f"{what}: rel-L2 {rel}"
     return max_abs, rel
+
+
+def oracle_layer(inp: dict, w: synth.Workload, tokens=None, threads: int = 0, **kw) -> dict:
+    """oracle.layer_forward of the workload, the output rows of `tokens` (None = all) computed by
+    several independent oracle calls on chunks of the tokens in parallel threads (the oracle's C
+    code runs outside the interpreter lock; each call routes the whole batch itself, so every
+    chunk sees the same routing). Returns layer_forward's dict for the requested tokens."""
+    import concurrent.futures as cf
+    import os
+
+    import oracle
+    tok = np.arange(w.T, dtype=np.int64) if tokens is None else np.asarray(tokens, dtype=np.int64)
+    n_thr = threads or max(1, min(16, (os.cpu_count() or 1), len(tok)))
+    common = dict(add_input_residual=w.add_input_residual, aux_alpha=w.aux_alpha)
+    common.update(kw)
+    if n_thr == 1 or len(tok) < 2:
+        return oracle.layer_forward(inp, w.T, w.d_model, w.d_ff, w.E, w.k, w.capacity_factor,
+                                    tokens=tok, **common)
+    chunks = [c for c in np.array_split(tok, n_thr) if len(c)]
+    with cf.ThreadPoolExecutor(len(chunks)) as ex:
+        parts = list(ex.map(lambda c: oracle.layer_forward(
+            inp, w.T, w.d_model, w.d_ff, w.E, w.k, w.capacity_factor, tokens=c, **common), chunks))
+    r = dict(parts[0])
+    r["out_exact"] = np.concatenate([p["out_exact"] for p in parts])
+    r["out"] = np.concatenate([p["out"] for p in parts])
+    r["tokens"] = tok
+    return r
+
+
+def spread_tokens(w: synth.Workload, ids: np.ndarray, slot: np.ndarray, n_min: int,
+                  rng: np.random.Generator, tile: int = 128) -> np.ndarray:
+    """Output rows to compare on a full-size workload: a kept token of every expert that keeps
+    one, the first and last kept tokens of the largest segments and those on each side of a
+    token-tile boundary inside them, dropped tokens and (k > 1) partially dropped ones, the first
+    and last token, then random kept tokens up to n_min."""
+    T, k = ids.shape
+    pick = {0, T - 1}
+    kept_pair = slot >= 0
+    for e in np.unique(ids[kept_pair]):
+        t_e = np.nonzero((ids == e) & kept_pair)[0]
+        pick.add(int(rng.choice(t_e)))
+    sizes = [(int(((ids == e) & kept_pair).sum()), e) for e in np.unique(ids)]
+    for _, e in sorted(sizes, reverse=True)[:4]:
+        # kept tokens of e in packed-row order (slot order)
+        t_e, j_e = np.nonzero((ids == e) & kept_pair)
+        order = t_e[np.argsort(slot[t_e, j_e], kind="stable")]
+        pick.update(int(order[i]) for i in (0, len(order) - 1))
+        for b in range(tile, len(order), tile):
+            pick.update(int(order[i]) for i in (b - 1, b))
+    dropped = np.nonzero((~kept_pair).all(1))[0]
+    partial = np.nonzero((~kept_pair).any(1) & kept_pair.any(1))[0]
+    for group in (dropped, partial):
+        if len(group):
+            pick.update(int(t) for t in rng.choice(group, min(len(group), 16), replace=False))
+    kept = np.nonzero(kept_pair.all(1))[0]
+    need = n_min - len(pick)
+    if need > 0 and len(kept):
+        pick.update(int(t) for t in rng.choice(kept, min(len(kept), need), replace=False))
+    return np.array(sorted(pick), dtype=np.int64)

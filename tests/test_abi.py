@@ -28,7 +28,7 @@ def test_exports_every_declared_symbol(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.moe_abi_version() == 2
+    assert L.moe_abi_version() == 3
     for code, name in moe.STATUS_NAMES.items():
         assert L.moe_status_string(code).decode() == name
 
@@ -47,6 +47,14 @@ def test_capacity_and_rows(L):
     for args in [(-1, 4, 1, 1.0), (4, 0, 1, 1.0), (4, 4, 0, 1.0), (4, 4, 1, -1.0),
                  (4, 4, 1, float("nan")), (4, 4, 1, float("inf"))]:
         assert L.moe_capacity(*args, ctypes.byref(c)) == 1
+
+
+def test_capacity_of_decimal_factor(L):
+    # ceil(k T / E x cf) of the decimal factor: 100 tokens / 10 experts x 1.1 = 11, not 12
+    assert moe.moe_capacity(100, 10, 1, 1.1) == 11
+    assert moe.moe_capacity(1000, 100, 1, 1.1) == 11
+    assert moe.moe_capacity(700, 10, 1, 0.7) == 49
+    assert moe.moe_capacity(30, 10, 1, 1.1) == 4
 
 
 def test_capacity_matches_oracle_formula(L):
@@ -92,17 +100,33 @@ def test_router_validation(L):
 def test_router_ex_validation(L, monkeypatch):
     def call(**kw):
         a = dict(x=FAKE, xdt=1, T=16, d=64, w=FAKE, b=None, E=8, k=2, logits=None, ids=FAKE,
-                 gates=FAKE, lb=None, alpha=0.01, rn=1, losses=FAKE, ws=FAKE, wsb=1 << 30)
+                 gates=FAKE, lb=None, alpha=0.01, rn=1, losses=FAKE, probs=None, ws=FAKE,
+                 wsb=1 << 30)
         a.update(kw)
         return L.moe_router_topk_ex(a["x"], a["xdt"], a["T"], a["d"], a["w"], a["b"], a["E"],
                                     a["k"], a["logits"], a["ids"], a["gates"], a["lb"], a["alpha"],
-                                    a["rn"], a["losses"], a["ws"], a["wsb"], None)
+                                    a["rn"], a["losses"], a["probs"], a["ws"], a["wsb"], None)
     assert call(k=3, E=2) == 1
     assert call(losses=FAKE + 4) == 6           # misaligned router_losses
+    assert call(probs=FAKE + 4) == 6            # misaligned probabilities output
     assert call(wsb=100) == 3
     monkeypatch.setenv("MOE_FAULT_INJECT", "moe_router_topk_ex")
     assert call() == 4
     assert _router(L, wsb=100) == 3             # the plain entry is a different name
+
+
+def test_router_prepare_validation(L, monkeypatch):
+    n = ctypes.c_size_t()
+    assert L.moe_router_prepare_bytes(128, 1000, ctypes.byref(n)) == 0
+    assert n.value == 128 * 3 * 1024 * 2                 # three bf16 parts, K padded to 64
+    assert L.moe_router_prepare_bytes(0, 64, ctypes.byref(n)) == 1
+    assert L.moe_router_prepare_bytes(2048, 64, ctypes.byref(n)) == 2
+    big = 1 << 30
+    assert L.moe_router_prepare(None, 8, 64, FAKE, big, None) == 1
+    assert L.moe_router_prepare(FAKE, 8, 64, FAKE + 8, big, None) == 6
+    assert L.moe_router_prepare(FAKE, 8, 64, FAKE, 100, None) == 3
+    monkeypatch.setenv("MOE_FAULT_INJECT", "moe_router_prepare")
+    assert L.moe_router_prepare(FAKE, 8, 64, FAKE, big, None) == 4
 
 
 def test_dispatch_priority_validation(L):
@@ -113,7 +137,7 @@ def test_dispatch_priority_validation(L):
         return L.moe_dispatch_priority(a["x"], a["dt"], a["T"], a["d"], a["ids"], a["g"], a["E"],
                                        a["k"], a["C"], a["slot"], a["cnt"], a["off"], a["rt"],
                                        a["xp"], a["rows"], a["ws"], a["wsb"], None)
-    assert call(g=None) == 1                    # gates are required
+    assert call(g=None) == 1                    # the probabilities are required
     assert call(g=FAKE + 4) == 6
     assert call(C=-1) == 1
     assert call(rows=15) == 1

@@ -1,8 +1,8 @@
 """GPU parity of the layer's backward pass (moe_layer_forward_train + moe_layer_backward) against
 the oracle's chain rule (oracle.layer_backward, pinned by finite differences).
 
-The oracle differentiates the same routing: it takes the GPU's fp32 logits and gates, so top-k,
-slots and the priority order are the GPU's. Tolerances (gradient g against the oracle's r, over
+The oracle differentiates the same routing: it takes the GPU's fp32 logits and the chosen
+experts' fp32 probabilities, so top-k, slots and the priority order are the GPU's. Tolerances (gradient g against the oracle's r, over
 each tensor): fp32 layers, relative L2 <= 1e-5 and max |g - r| <= 1e-4 max |r|; bf16 layers (the
 backward GEMM operands dY, dZ and GeLU'(z) are rounded to bf16, fp32 accumulation, dx returned
 in bf16), relative L2 <= 1e-2 and max |g - r| <= 5e-2 max |r|.
@@ -35,7 +35,8 @@ def run_train(w: synth.Workload, d_inp: dict, dout_dev, aux_weight=0.0, z_weight
     aux = dict(logits=torch.empty(T, E, dtype=torch.float32, device=dev),
                expert_ids=torch.empty(T, k, dtype=torch.int32, device=dev),
                gates=torch.empty(T, k, dtype=torch.float32, device=dev),
-               slot=torch.empty(T, k, dtype=torch.int32, device=dev))
+               slot=torch.empty(T, k, dtype=torch.int32, device=dev),
+               topk_probs=torch.empty(T, k, dtype=torch.float32, device=dev))
     out = torch.empty(T, d, dtype=x.dtype, device=dev)
     ws = moe.moe_layer_forward_train(args, out, aux=aux)
     f32 = dict(dtype=torch.float32, device=dev)
@@ -85,7 +86,7 @@ def backward_parity(w: synth.Workload, aux_weight=0.3, z_weight=0.1, renormalize
     ref = oracle.layer_backward(inp, w.T, w.d_model, w.d_ff, w.E, w.k, w.capacity_factor,
                                 as_f64(dout_h), add_input_residual=w.add_input_residual,
                                 aux_alpha=w.aux_alpha, aux_weight=aux_weight, z_weight=z_weight,
-                                logits_in=got["logits"], gates_in=got["gates"],
+                                logits_in=got["logits"], probs_in=got["topk_probs"],
                                 overflow_priority=overflow_priority, renormalize=renormalize)
     res = {}
     pairs = [("dx", "dx"), ("dw_router", "dw_router"), ("db_router", "db_router"),
@@ -124,6 +125,15 @@ def test_backward_bf16_workloads_reduced(cuda_ok, cfg, T, shape, kw):
     backward_parity(w, **kw)
 
 
+def test_backward_bf16_full_k(cuda_ok):
+    # the headline workload's layer widths (K = 1024 into layer 1, K = 4096 into layer 2, and
+    # d_ff = 4096 output features of the weight gradients) on a few hundred tokens; 8 experts keep
+    # the oracle's float64 weight gradients small
+    w = synth.WORKLOADS[2].with_(T=320, E=8, capacity_factor=1.0)
+    got, _, _ = backward_parity(w, renormalize=True, overflow_priority=True)
+    assert (got["slot"] < 0).any()
+
+
 def test_backward_bf16_ragged_dims(cuda_ok):
     # d and d_ff not multiples of 64 (MN-major tails), top-2, drops
     w = synth.Workload("ragged", T=300, d_model=264, d_ff=200, E=5, k=2, capacity_factor=0.8,
@@ -148,7 +158,7 @@ def test_backward_bf16_one_hot_expert(cuda_ok):
     assert np.abs(others).max() == 0.0
     ref = oracle.layer_backward(inp, w.T, w.d_model, w.d_ff, w.E, w.k, w.capacity_factor,
                                 as_f64(dout), aux_alpha=w.aux_alpha, logits_in=got["logits"],
-                                gates_in=got["gates"])
+                                probs_in=got["topk_probs"])
     for n in ("dw1", "dw2", "dx", "dw_router"):
         compare(n, got[n], ref[n], True)
 

@@ -2,9 +2,10 @@
 
 Routing and dispatch (ids, slots, demand counts, offsets) are bit-exact given the GPU's fp32
 logits; the oracle runs the whole layer on those logits and its outputs are compared within the
-tolerances of tests/helpers.py. Full-size workloads compare every token's routing and a sample of
-output rows (all kinds: kept, dropped, top-2 partially dropped); reduced versions of each workload
-compare every output row.
+tolerances of tests/helpers.py. Full-size workloads compare every token's routing and at least
+128 output rows spread over the path's cases (a kept token of every touched expert, the first and
+last rows and the token-tile boundaries of the largest segments, dropped and partially dropped
+tokens); reduced versions of each workload compare every output row.
 """
 import numpy as np
 import pytest
@@ -12,7 +13,7 @@ import torch
 
 import oracle
 import synth
-from tests.helpers import check_out, dev_inputs, run_layer, to_dev
+from tests.helpers import check_out, dev_inputs, oracle_layer, run_layer, spread_tokens, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -29,19 +30,14 @@ def layer_parity(w: synth.Workload, inp=None, d_inp=None, n_sample=None, out_dty
     if n_sample is None or n_sample >= w.T:
         tokens = np.arange(w.T)
     else:
-        slot_probe, _ = oracle.assign_slots(
-            oracle.route(got["logits"], w.k)[0], w.E, oracle.capacity(w.T, w.E, w.k, w.capacity_factor))
-        dropped = np.where((slot_probe < 0).any(1))[0]
-        kept = np.where((slot_probe >= 0).all(1))[0]
-        pick = [rng.choice(dropped, min(len(dropped), n_sample // 4), replace=False)] if len(dropped) else []
-        pick.append(rng.choice(kept, min(len(kept), n_sample - sum(len(p) for p in pick)), replace=False))
-        tokens = np.sort(np.concatenate(pick + [[0, w.T - 1]]).astype(np.int64))
-        tokens = np.unique(tokens)
+        ids_probe = oracle.route(got["logits"], w.k)[0]
+        slot_probe, _ = oracle.assign_slots(ids_probe, w.E,
+                                            oracle.capacity(w.T, w.E, w.k, w.capacity_factor))
+        tokens = spread_tokens(w, ids_probe, slot_probe, n_sample, rng)
     bf16 = w.dtype == "bf16"
     out_bf16 = bf16 if out_dtype is None else out_dtype == torch.bfloat16
-    ref = oracle.layer_forward(inp, w.T, w.d_model, w.d_ff, w.E, w.k, w.capacity_factor,
-                               add_input_residual=res, aux_alpha=w.aux_alpha,
-                               logits_in=got["logits"], tokens=tokens, out_bf16=out_bf16)
+    ref = oracle_layer(inp, w, tokens, add_input_residual=res, logits_in=got["logits"],
+                       out_bf16=out_bf16)
     assert np.array_equal(got["expert_ids"], ref["ids"])
     np.testing.assert_allclose(got["gates"], ref["gates"], rtol=2e-6, atol=1e-12)
     assert np.array_equal(got["slot"], ref["slot"])
@@ -75,15 +71,38 @@ def test_reduced_workloads_all_rows(cuda_ok, cfg, T):
     layer_parity(w, out_dtype=torch.float32)
 
 
-@pytest.mark.parametrize("cfg,n", [(2, 256), (3, 24), (4, 20), (5, 32)])
+@pytest.mark.parametrize("cfg,n", [(2, 256), (3, 160), (4, 128), (5, 32)])
 def test_full_workloads_sampled(cuda_ok, cfg, n):
     w = synth.WORKLOADS[cfg]
     inp = synth.make_inputs(w)
     d_inp = dev_inputs(inp)
     r = layer_parity(w, inp, d_inp, n_sample=n, seed=cfg)
+    assert len(r["tokens"]) >= min(n, w.T)
     r32 = layer_parity(w, inp, d_inp, n_sample=n // 2, out_dtype=torch.float32, seed=cfg + 10)
     print(f"workload {cfg}: bf16-out max-abs {r['max_abs']:.3e} rel-L2 {r['rel']:.3e}; "
           f"fp32-out max-abs {r32['max_abs']:.3e} rel-L2 {r32['rel']:.3e}")
+
+
+@pytest.mark.parametrize("shape", [
+    dict(T=2048, d_model=1024, d_ff=2048, E=16),    # capacity 128: 128-token expert tiles
+    dict(T=1000, d_model=512, d_ff=1024, E=128),    # capacity 8: 16-token expert tiles, ragged T
+    dict(T=300, d_model=256, d_ff=128, E=4),        # one 128-feature tile per expert
+])
+def test_prmoe_coscheduled_equals_sequential(cuda_ok, monkeypatch, shape):
+    # the expert and dense GEMM layers co-scheduled in one launch each (default) give the same
+    # bits as the sequential launches with the combine fused into the dense layer 2 epilogue;
+    # both match the oracle
+    w = synth.WORKLOADS[3].with_(**shape)
+    inp = synth.make_inputs(w)
+    d_inp = dev_inputs(inp)
+    co = layer_parity(w, inp, d_inp)["got"]
+    monkeypatch.setenv("MOE_COSCHEDULE", "0")
+    seq = layer_parity(w, inp, d_inp)["got"]
+    # co-scheduled: two GEMM launches and the combine; sequential: four GEMM launches
+    assert co["launches"] == seq["launches"] - 1
+    assert np.array_equal(co["out"], seq["out"])
+    for name in ("expert_ids", "gates", "slot", "expert_offsets", "lb_stats"):
+        assert np.array_equal(co[name], seq[name]), name
 
 
 def test_prmoe_both_residual_conventions(cuda_ok):

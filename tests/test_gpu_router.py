@@ -113,3 +113,28 @@ def test_router_zero_tokens(cuda_ok):
     r = moe.moe_router_topk(x, torch.randn(8, 64, device="cuda"), 2)
     assert moe.moe_last_launch_count() == 0
     assert r["expert_ids"].shape == (0, 2)
+
+
+@pytest.mark.parametrize("cfg,T", [(2, 4096), (3, 1000), (4, 2048), (2, 64)])
+def test_prepared_router_weight_gives_identical_layer(cuda_ok, cfg, T):
+    # the router weight split once (moe_router_prepare) and passed to the layer gives the same
+    # bits as the split done inside every call; at T <= 64 (fp32 GEMV router) it is ignored
+    from tests.helpers import dev_inputs, run_layer
+    w = synth.WORKLOADS[cfg].with_(T=T)
+    if cfg in (3, 4):
+        w = w.with_(d_model=1024, d_ff=2048)
+    inp = synth.make_inputs(w)
+    d_inp = dev_inputs(inp)
+    plain = run_layer(w, d_inp, want_losses=True)
+    prep = moe.moe_router_prepare(d_inp["w_router"])
+    ready = run_layer(w, d_inp, want_losses=True, w_router_prepared=prep)
+    assert plain["device_error"] == 0 and ready["device_error"] == 0
+    for name in plain:
+        if isinstance(plain[name], np.ndarray):
+            assert np.array_equal(plain[name].view(np.uint8), ready[name].view(np.uint8)), name
+    # the prepared weight is the exact split: hi + mid + lo == W_r
+    E, d = inp["w_router"].shape
+    dpad = (d + 63) // 64 * 64
+    parts = to_host(prep).view(np.uint16).reshape(E, 3, dpad)[:, :, :d]
+    widened = synth.bf16_bits_to_f32(parts).astype(np.float64)
+    np.testing.assert_array_equal(widened.sum(1), inp["w_router"].astype(np.float64))

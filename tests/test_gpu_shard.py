@@ -1,12 +1,14 @@
-"""GPU check of the token-sharded layer (moe_layer_forward_shard_begin / _end) against the
-whole-batch layer on one GPU, which the other tests hold to the oracle.
+"""GPU check of the token-sharded layer (moe_layer_forward_shard_begin / _end) against the oracle
+on the whole batch, and against the whole-batch layer on one GPU.
 
 The G shards run one after another on the one GPU: every shard's begin, then the exchange done by
 hand (the demands stacked in shard order, the statistics partials summed), then every shard's end.
-No kernel waits on another shard. Expected: ids, gates and output rows bit for bit; a token keeps
-a choice exactly when the whole batch keeps it, at local slot = global slot - the earlier shards'
-demand; lb_stats and router losses bit for bit when the shards before the last hold multiples of 64
-tokens.
+No kernel waits on another shard. Against the oracle (run on the whole batch from the shards' own
+fp32 logits and probabilities): ids exact, gates to 2e-6, every token's global slot exact (local
+slot + the earlier shards' demand), demand per expert exact, f exact and Q, aux, z-loss and CoV^2
+within the single-GPU tolerances, every output row within the output tolerances. Against the
+whole-batch layer: ids, gates and output rows bit for bit; lb_stats and router losses bit for bit
+when the shards before the last hold multiples of 64 tokens.
 """
 import numpy as np
 import pytest
@@ -14,7 +16,7 @@ import torch
 
 import synth
 from mixture_experts_layer_57_b200 import moe
-from tests.helpers import dev_inputs, run_layer, to_host
+from tests.helpers import check_out, dev_inputs, oracle_layer, run_layer, to_host
 
 pytestmark = pytest.mark.gpu
 
@@ -36,7 +38,9 @@ def run_shards(w: synth.Workload, d_inp: dict, sizes, renormalize=False):
                               add_input_residual=w.add_input_residual, aux_alpha=w.aux_alpha,
                               renormalize_gates=renormalize)
         dev = x.device
-        aux = dict(expert_ids=torch.empty(n, k, dtype=torch.int32, device=dev),
+        aux = dict(logits=torch.empty(n, E, dtype=torch.float32, device=dev),
+                   topk_probs=torch.empty(n, k, dtype=torch.float32, device=dev),
+                   expert_ids=torch.empty(n, k, dtype=torch.int32, device=dev),
                    gates=torch.empty(n, k, dtype=torch.float32, device=dev),
                    slot=torch.empty(n, k, dtype=torch.int32, device=dev),
                    expert_counts=torch.empty(E, dtype=torch.int32, device=dev),
@@ -62,11 +66,44 @@ def run_shards(w: synth.Workload, d_inp: dict, sizes, renormalize=False):
                demand_all=to_host(demand_all),
                lb=[to_host(s["aux"]["lb_stats"]) for s in shards],
                losses=[to_host(s["aux"]["router_losses"]) for s in shards])
-    for name in ("expert_ids", "gates", "slot"):
+    for name in ("expert_ids", "gates", "slot", "logits", "topk_probs"):
         res[name] = np.concatenate([to_host(s["aux"][name]) for s in shards])
     res["counts"] = [to_host(s["aux"]["expert_counts"]) for s in shards]
     res["offsets"] = [to_host(s["aux"]["expert_offsets"]) for s in shards]
     return res
+
+
+def check_against_oracle(w, inp, sizes, sh, renormalize):
+    """The shards' results against the oracle's layer over the whole batch."""
+    ref = oracle_layer(inp, w, logits_in=sh["logits"], probs_in=sh["topk_probs"],
+                       renormalize=renormalize)
+    assert np.array_equal(sh["expert_ids"], ref["ids"])
+    np.testing.assert_allclose(sh["gates"], ref["gates"], rtol=2e-6, atol=1e-12)
+    assert np.array_equal(sh["demand_all"].sum(0), ref["counts"])
+    base = np.concatenate([np.zeros((1, w.E), np.int64),
+                           np.cumsum(sh["demand_all"], axis=0)[:-1]]).astype(np.int64)
+    t0 = 0
+    for r, n in enumerate(sizes):
+        ids = sh["expert_ids"][t0:t0 + n]
+        ls = sh["slot"][t0:t0 + n]
+        rs = ref["slot"][t0:t0 + n]
+        assert np.array_equal(ls < 0, rs < 0), r
+        kept = ls >= 0
+        assert np.array_equal(ls[kept] + base[r][ids[kept]], rs[kept]), r
+        t0 += n
+    E = w.E
+    for r in range(len(sizes)):
+        lb = sh["lb"][r]
+        np.testing.assert_array_equal(lb[:E], ref["f"].astype(np.float32))
+        np.testing.assert_allclose(lb[E:2 * E], ref["Q"], rtol=1e-5, atol=1e-9)
+        assert abs(lb[2 * E] - ref["aux"]) <= 1e-5 * abs(ref["aux"]) + 1e-9
+        z, ci, cl = sh["losses"][r]
+        assert abs(z - ref["z_loss"]) <= 1e-5 * abs(ref["z_loss"]) + 1e-6
+        assert abs(ci - ref["cov2_importance"]) <= 1e-5 * abs(ref["cov2_importance"]) + 1e-7
+        assert abs(cl - ref["cov2_load"]) <= 1e-6 * abs(ref["cov2_load"]) + 1e-9
+    bf16 = w.dtype == "bf16"
+    check_out(sh["out"], ref["out_exact"], bf16, bf16, what=f"{w.name} shards {sizes}")
+    return ref
 
 
 def compare(w, sizes, renormalize=False, exact_stats=True):
@@ -74,6 +111,7 @@ def compare(w, sizes, renormalize=False, exact_stats=True):
     d_inp = dev_inputs(inp)
     whole = run_layer(w, d_inp, renormalize=renormalize, want_losses=True)
     sh = run_shards(w, d_inp, sizes, renormalize=renormalize)
+    check_against_oracle(w, inp, sizes, sh, renormalize)
     assert np.array_equal(sh["expert_ids"], whole["expert_ids"])
     assert np.array_equal(sh["gates"], whole["gates"])
     # kept exactly where the whole batch keeps; local slot = global slot - earlier demand

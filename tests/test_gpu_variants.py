@@ -3,7 +3,8 @@ z-loss and the CoV^2 of Importance and Load (moe_router_topk_ex), overflow by pr
 (moe_dispatch_priority), and both inside moe_layer_forward.
 
 Ids, slots, counts and offsets are bit-exact (the oracle decides on the GPU's fp32 logits and, for
-the priority order, on the GPU's fp32 gates); renormalised gates match to 2e-6 relative; z-loss
+the priority order, on the GPU's fp32 router probabilities, which rank the pairs before and
+after any renormalisation of the gates); renormalised gates match to 2e-6 relative; z-loss
 and CoV^2 of Importance to 1e-5 relative (fp32 per-token terms, fixed-point sums); CoV^2 of Load
 to 1e-6 (integer counts).
 """
@@ -30,9 +31,10 @@ def check_losses(got, ref, what=""):
 def router_ex(w: synth.Workload, inp: dict, renormalize: bool):
     r = moe.moe_router_topk(to_dev(inp["x"]), to_dev(inp["w_router"]), w.k,
                             router_bias=to_dev(inp.get("router_bias")), aux_alpha=w.aux_alpha,
-                            renormalize=renormalize, router_losses=True)
+                            renormalize=renormalize, router_losses=True, probs=True)
     assert moe.moe_get_device_error(r["ws"]) == 0
-    return {n: to_host(r[n]) for n in ("logits", "expert_ids", "gates", "lb_stats", "router_losses")}
+    return {n: to_host(r[n]) for n in ("logits", "expert_ids", "gates", "lb_stats", "router_losses",
+                                       "probs")}
 
 
 def router_only(w):
@@ -48,9 +50,13 @@ def test_router_variants_workloads(cuda_ok, cfg, renormalize):
     got = router_ex(w, inp, renormalize)
     ids, gates = oracle.route(got["logits"], w.k)
     assert np.array_equal(got["expert_ids"], ids)
+    # the probabilities output is the softmax p of each choice, renormalised or not
+    np.testing.assert_allclose(got["probs"], gates, rtol=2e-6, atol=1e-12)
     if renormalize:
         gates = oracle.renormalize_gates(gates)
         np.testing.assert_allclose(got["gates"].sum(1), 1.0, rtol=1e-5)
+    else:
+        assert np.array_equal(got["probs"], got["gates"])
     np.testing.assert_allclose(got["gates"], gates, rtol=2e-6, atol=1e-12)
     # the losses from the GPU's own logits and gates
     check_losses(got["router_losses"], oracle.router_losses(got["logits"], got["expert_ids"],
@@ -90,11 +96,11 @@ def test_router_z_loss_closed_form(cuda_ok):
     assert abs(z - (0.75 + np.log(E)) ** 2) <= 1e-5 * z
 
 
-def check_priority_dispatch(x_host, ids, gates, E, C):
+def check_priority_dispatch(x_host, ids, probs, E, C):
     T, k = ids.shape
-    r = moe.moe_dispatch(to_dev(x_host), to_dev(ids), E, C, priority_gates=to_dev(gates))
+    r = moe.moe_dispatch(to_dev(x_host), to_dev(ids), E, C, priority_probs=to_dev(probs))
     assert moe.moe_get_device_error(r["ws"]) == 0
-    slot, counts = oracle.assign_slots_priority(ids, gates, E, C)
+    slot, counts = oracle.assign_slots_priority(ids, probs, E, C)
     assert np.array_equal(to_host(r["slot"]), slot)
     assert np.array_equal(to_host(r["expert_counts"]), counts)
     off = np.concatenate([[0], np.cumsum(np.minimum(counts, C))]).astype(np.int32)
@@ -152,6 +158,22 @@ def test_priority_matches_capacity_example(cuda_ok):
     assert [tk for tk in range(4) if slot[tk, 0] < 0] == g["page_priority_order_dropped"]
 
 
+def assert_priority_active(got, E, C):
+    """Every expert keeps the pairs of its C largest router probabilities (before any
+    renormalisation), and at least one expert keeps a different set than first-come would."""
+    ids, slot, p = got["expert_ids"], got["slot"], got["topk_probs"]
+    fc, _ = oracle.assign_slots(ids, E, C)
+    differs = False
+    for e in np.unique(ids):
+        t_e, j_e = np.nonzero(ids == e)
+        kept = slot[t_e, j_e] >= 0
+        if kept.all() or not kept.any():
+            continue
+        assert p[t_e, j_e][kept].min() >= p[t_e, j_e][~kept].max(), e
+        differs |= not np.array_equal(kept, fc[t_e, j_e] >= 0)
+    assert differs, "priority kept the same pairs as first-come"
+
+
 def layer_variant_parity(w: synth.Workload, overflow_priority=True, renormalize=True):
     inp = synth.make_inputs(w)
     d_inp = dev_inputs(inp)
@@ -163,9 +185,10 @@ def layer_variant_parity(w: synth.Workload, overflow_priority=True, renormalize=
                                add_input_residual=w.add_input_residual, aux_alpha=w.aux_alpha,
                                logits_in=got["logits"], out_bf16=bf16,
                                overflow_priority=overflow_priority, renormalize=renormalize,
-                               gates_in=got["gates"])
+                               probs_in=got["topk_probs"])
     assert np.array_equal(got["expert_ids"], ref["ids"])
     ids, gates = oracle.route(got["logits"], w.k)
+    np.testing.assert_allclose(got["topk_probs"], gates, rtol=2e-6, atol=1e-12)
     if renormalize:
         gates = oracle.renormalize_gates(gates)
     np.testing.assert_allclose(got["gates"], gates, rtol=2e-6, atol=1e-12)
@@ -180,8 +203,42 @@ def layer_variant_parity(w: synth.Workload, overflow_priority=True, renormalize=
 
 
 def test_layer_priority_renorm_tiny_fp32(cuda_ok):
-    got, ref = layer_variant_parity(synth.WORKLOADS[1])
+    w = synth.WORKLOADS[1]
+    got, ref = layer_variant_parity(w)
     assert (got["slot"] < 0).any()
+    assert (got["gates"] == 1.0).all()  # top-1 gates renormalise to 1, the ranking does not
+    assert_priority_active(got, w.E, ref["C"])
+
+
+def test_layer_priority_renorm_page_example(cuda_ok):
+    # comparison article, "Expert Capacity Overflow": capacity 2 for expert 0's three tokens; by
+    # router probability t3 (0.859) and t0 (0.817) keep it and t1 (0.669) overflows. The layer
+    # routes the printed logits (x = logits, W_r = identity) with renormalised top-1 gates, which
+    # are all 1.0; the ranking still follows the probabilities, unlike first-come (drops t3).
+    from tests.conftest import golden
+    g = golden("capacity_overflow.json")
+    t = golden("top1_four_tokens.json")
+    w = synth.Workload("page", T=4, d_model=2, d_ff=8, E=2, k=1, capacity_factor=1.0, dtype="f32",
+                       w_router_std=1.0, w_std=0.3, b_std=0.1, seed=3)
+    inp = synth.make_inputs(w)
+    inp["x"] = np.array(t["logits"], dtype=np.float32)
+    inp["w_router"] = np.eye(2, dtype=np.float32)
+    for renorm in (True, False):
+        got = run_layer(w, dev_inputs(inp), overflow_priority=True, renormalize=renorm)
+        assert got["device_error"] == 0
+        slot = got["slot"][:, 0]
+        assert [tk for tk in (3, 0, 1) if slot[tk] >= 0] == g["page_priority_order_kept_E0"]
+        assert [tk for tk in range(4) if slot[tk] < 0] == g["page_priority_order_dropped"]
+        fc = run_layer(w, dev_inputs(inp), overflow_priority=False, renormalize=renorm)
+        assert [tk for tk in range(4) if fc["slot"][tk, 0] < 0] == g["first_come_reading_dropped"]
+        assert not np.array_equal(got["slot"], fc["slot"])
+        if renorm:
+            assert (got["gates"] == 1.0).all()
+        ref = oracle.layer_forward(inp, 4, 2, 8, 2, 1, 1.0, logits_in=got["logits"],
+                                   overflow_priority=True, renormalize=renorm,
+                                   probs_in=got["topk_probs"])
+        assert np.array_equal(got["slot"], ref["slot"])
+        check_out(got["out"], ref["out_exact"], False, False, what="page example")
 
 
 @pytest.mark.parametrize("cfg,T,policy", [
@@ -196,11 +253,12 @@ def test_layer_variants_reduced(cuda_ok, cfg, T, policy):
     if cfg == 4:
         shrink.update(d_model=1024, d_ff=2048)
     w = w.with_(**shrink)
-    got, _ = layer_variant_parity(w, *policy)
+    got, ref = layer_variant_parity(w, *policy)
     if policy[0]:
         # the priority path changes which pairs are kept, not how many
-        slot_fc, _ = oracle.assign_slots(got["expert_ids"], w.E, moe.moe_capacity(w.T, w.E, w.k, w.capacity_factor))
+        slot_fc, _ = oracle.assign_slots(got["expert_ids"], w.E, ref["C"])
         assert (slot_fc >= 0).sum() == (got["slot"] >= 0).sum()
+        assert_priority_active(got, w.E, ref["C"])
 
 
 def test_layer_priority_all_tokens_to_one_expert(cuda_ok):
