@@ -303,9 +303,10 @@ def stage_work(w: synth.Workload, R: int, E_t: int, E: int):
     stage_bytes["experts_dense_gemm2"] = stage_bytes["expert_gemm2"] + dense_gemm2
     for n in ("experts_dense_gemm1", "experts_dense_gemm2"):
         stage_flops[n] = 2.0 * (R + T) * dm * df
-    # the routing stages: the router's logits are 2 T d E FLOP over x (read once), W_r and the
-    # logits/ids/gates; dispatch moves the kept rows (read + write)
-    stage_bytes["router"] = T * dm * es + E * dm * 4 + 2 * T * E * 4 + T * k * 8
+    # the routing stages: the router's logits are 2 T d E FLOP over x (read once) and W_r, with
+    # ids, gates and the dispatch ranks written (the logits are an intermediate that stays on
+    # chip); dispatch moves the kept rows (read + write)
+    stage_bytes["router"] = T * dm * es + E * dm * 4 + T * k * 12
     stage_flops["router"] = 2.0 * T * dm * E
     stage_bytes["dispatch"] = 2 * R * dm * es + T * k * 12 + 2 * (E + 1) * 4
     stage_flops["dispatch"] = 0.0
@@ -494,6 +495,12 @@ def main():
     stage_bytes, stage_flops = stage_work(w, R, E_t, E)
     peaks, peak_src = load_peaks()
     stages = stage_rates(bd, stage_bytes, stage_flops, peaks)
+    if "router" in stages and bf16:
+        # the tensor-core router multiplies three bf16 parts of W_r: 3x the algorithmic FLOPs
+        r = stages["router"]
+        r["tensor_frac_of_three_part_work"] = 3 * r["tensor_frac"]
+        r["roofline_ms"] = 1e3 * max(stage_bytes["router"] / (peaks["hbm_gbs"] * 1e9),
+                                     3 * stage_flops["router"] / (peaks["bf16_tflops"] * 1e12))
     gemm_stages = [n for n in bd if n in stage_bytes and n.startswith(("expert", "dense"))]
     dom = max(gemm_stages, key=lambda n: bd[n])
     t_dom = bd[dom] / 1e3

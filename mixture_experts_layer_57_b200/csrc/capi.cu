@@ -26,6 +26,14 @@ bool pdl_enabled() {
   return on;
 }
 
+// Whether the tensor-core router runs softmax, top-k and the statistics in its own epilogue
+// (MOE_FUSED_ROUTER=0: a separate top-k kernel reads the logits back; both give the same bits).
+// Read at every call.
+bool router_fusion_enabled() {
+  const char* v = std::getenv("MOE_FUSED_ROUTER");
+  return !(v != nullptr && v[0] == '0');
+}
+
 // Whether bf16 PR-MoE layers co-schedule each expert GEMM layer with the dense MLP's layer in one
 // launch (MOE_COSCHEDULE=0 runs them one after another, the dense layer 2 with the combine fused;
 // both give the same bits). Read at every call.

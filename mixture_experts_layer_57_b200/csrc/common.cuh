@@ -136,6 +136,21 @@ __device__ __forceinline__ bool mbar_wait_bounded_warp(uint32_t bar, uint32_t pa
   }
 }
 
+// Named barrier `id` of `nthreads` threads that also ORs a predicate over them: every
+// participating thread gets the same answer (used to leave a loop together).
+__device__ __forceinline__ bool named_barrier_any(int id, int nthreads, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+
 // ---------------------------------------------------------------- TMA (loads into this CTA only)
 
 __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {

@@ -106,6 +106,19 @@ cudaError_t enqueue_router_logits_tc(const void* x, int64_t T, int d, const uint
                                      int* status, cudaStream_t stream,
                                      const RouterAccum* zero_acc = nullptr);
 
+// The tensor-core router with softmax, top-k, the statistics (and the dispatch ranks) fused into
+// its epilogue (router_fused_supported: E <= 128). The statistics accumulators must be zero when it
+// starts. logits may be nullptr (not written).
+bool router_fused_supported(int E);
+// Whether the router uses the fused kernel where it can (MOE_FUSED_ROUTER=0: the two kernels).
+bool router_fusion_enabled();
+cudaError_t enqueue_router_fused(const void* x, int64_t T, int d, const uint16_t* w_split,
+                                 int dpad, const float* router_bias, int E, int k, float* logits,
+                                 int32_t* ids, float* gates, float* probs, const RouterAccum& acc,
+                                 float aux_alpha, float* lb_stats, RouterDispatchCount dc,
+                                 bool renormalize, float* losses, int64_t* exported, int* status,
+                                 cudaStream_t stream);
+
 // Raises a kernel's dynamic shared-memory limit to `bytes` on the current device, once per
 // device (done_per_device: a zero-initialised [64] array owned by the launching function).
 template <class Kern>

@@ -25,6 +25,7 @@
 //                         Importance and Load (survey notes §1.1.4.1)
 #include "common.cuh"
 #include "kernels.h"
+#include "router_topk.cuh"
 
 namespace moe {
 namespace {
@@ -191,56 +192,6 @@ __global__ void __launch_bounds__(256) router_prep_kernel(const float* __restric
   pdl_trigger();
 }
 
-constexpr double kQScale = 4294967296.0;  // 2^32: fixed-point scale of the p sums
-constexpr double kZScale = 16777216.0;    // 2^24: fixed-point scale of the (log Z)^2 sums
-constexpr double kIScale = 16777216.0;    // 2^24: fixed-point scale of the gate sums
-
-// f, Q, aux and the router losses from the integer totals of T tokens; called by every thread
-// of one 256-thread block (prod: E floats of shared memory). Totals are read through accessors so
-// that the top-k kernel's last block and the shard finalisation run the same arithmetic.
-template <class Q, class Cn, class I, class L>
-__device__ void router_finalize_block(int E, int64_t T, float alpha, Q q_at, Cn c_at, I imp_at,
-                                      L load_at, unsigned long long zsum, float* lb, float* losses,
-                                      float* prod) {
-  if (lb != nullptr) {
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-      const float Qe = (float)((double)q_at(e) / kQScale / (double)T);
-      const float f = (float)c_at(e) / (float)T;
-      lb[e] = f;
-      lb[E + e] = Qe;
-      prod[e] = f * Qe;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      float s = 0.0f;
-      for (int e = 0; e < E; ++e) s += prod[e];
-      lb[2 * E] = alpha * (float)E * s;
-    }
-  }
-  if (losses != nullptr && threadIdx.x == 0) {
-    // z-loss = mean over tokens of (log Z)^2; CoV^2 = population variance / mean^2 over experts
-    losses[0] = (float)((double)zsum / kZScale / (double)T);
-    double mi = 0.0, ml = 0.0;
-    for (int e = 0; e < E; ++e) {
-      mi += (double)imp_at(e) / kIScale;
-      ml += (double)load_at(e);
-    }
-    mi /= E;
-    ml /= E;
-    double vi = 0.0, vl = 0.0;
-    for (int e = 0; e < E; ++e) {
-      const double a = (double)imp_at(e) / kIScale - mi;
-      const double b = (double)load_at(e) - ml;
-      vi += a * a;
-      vl += b * b;
-    }
-    vi /= E;
-    vl /= E;
-    losses[1] = mi > 0.0 ? (float)(vi / (mi * mi)) : 0.0f;
-    losses[2] = ml > 0.0 ? (float)(vl / (ml * ml)) : 0.0f;
-  }
-}
-
 __global__ void __launch_bounds__(256)
     router_finalize_kernel(const int64_t* __restrict__ tot, int64_t T, int E, float alpha,
                            float* __restrict__ lb, float* __restrict__ losses) {
@@ -251,233 +202,22 @@ __global__ void __launch_bounds__(256)
       [&](int e) { return (unsigned long long)tot[E + e]; },
       [&](int e) { return (unsigned long long)tot[2 * E + e]; },
       [&](int e) { return (unsigned long long)tot[3 * E + e]; }, (unsigned long long)tot[4 * E],
-      lb, losses, prod);
+      lb, losses, prod, threadIdx.x, blockDim.x, BlockSync{});
   pdl_trigger();
 }
 
-// EPL = experts per lane (E <= 32 * EPL); expert e lives in lane e % 32, slot e / 32.
-// COUNT: also rank this block's (token, choice) pairs per expert in pair order for dispatch.
 template <int EPL, bool COUNT, bool EXTRA>
 __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restrict__ logits,
-                                                          int64_t T, int E, int k,
-                                                          int32_t* __restrict__ ids,
-                                                          float* __restrict__ gates,
-                                                          RouterAccum acc, float alpha,
-                                                          float* __restrict__ lb,
-                                                          RouterDispatchCount dc, int renorm,
-                                                          float* __restrict__ losses,
-                                                          int64_t* __restrict__ exported,
-                                                          float* __restrict__ probs) {
-  __shared__ float qs[8][MOE_MAX_EXPERTS];
-  // per expert: first-choice count << 16 | choice count (each at most kRouterTokensPerBlock)
-  __shared__ unsigned cs[MOE_MAX_EXPERTS];
-  // gate sums, 2^-24 fixed point (< 2^31 per block); only with the extra statistics
-  __shared__ unsigned imp_s[EXTRA ? MOE_MAX_EXPERTS : 1];
-  __shared__ float zs[8];
-  __shared__ float prod[MOE_MAX_EXPERTS];
-  __shared__ int is_last;
-  __shared__ int blk_ids[COUNT ? kRouterTokensPerBlock * MOE_MAX_TOPK : 1];
+                                                          const TopkOut ko) {
+  __shared__ TopkShared<MOE_MAX_EXPERTS, COUNT, EXTRA> sh;
   pdl_wait();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int e = threadIdx.x; e < E; e += 256) {
-    cs[e] = 0u;
-    if constexpr (EXTRA) imp_s[e] = 0u;
-  }
-  __syncthreads();
-  float zw = 0.0f;  // this warp's sum of (log Z)^2 over its tokens, in token order
-  float q[EPL];
-#pragma unroll
-  for (int i = 0; i < EPL; ++i) q[i] = 0.0f;
   const int64_t tb = (int64_t)blockIdx.x * kRouterTokensPerBlock;
-  for (int r = warp; r < kRouterTokensPerBlock; r += 8) {
-    const int64_t t = tb + r;
-    if (t >= T) break;
-    float l[EPL];
-    float m = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-      const int e = lane + 32 * i;
-      l[i] = e < E ? logits[t * E + e] : -INFINITY;
-      m = fmaxf(m, l[i]);
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float ex[EPL];
-    float s = 0.0f;
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-      ex[i] = (lane + 32 * i) < E ? expf(l[i] - m) : 0.0f;
-      s += ex[i];
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if constexpr (EXTRA) {
-      const float lz = m + logf(s);  // log sum_e exp(l_e)
-      zw += lz * lz;
-    }
-    float p[EPL];
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-      p[i] = ex[i] / s;
-      q[i] += p[i];
-    }
-    // first choice: the lowest expert index holding the maximum logit (ballot per slot)
-    int bi = 0x7fffffff;
-#pragma unroll
-    for (int i = EPL - 1; i >= 0; --i) {
-      const unsigned b = __ballot_sync(0xffffffffu, (lane + 32 * i) < E && l[i] == m);
-      if (b) bi = 32 * i + __ffs(b) - 1;
-    }
-    // per-block integer counts (order-independent): first choices, and with the extra
-    // statistics every choice and its gate
-    auto count_choice = [&](int e, int j, float g) {
-      if constexpr (EXTRA) {
-        atomicAdd(&cs[e], j == 0 ? 0x10001u : 1u);
-        atomicAdd(&imp_s[e], __float2uint_rn(g * (float)kIScale));
-      } else if (j == 0) {
-        atomicAdd(&cs[e], 0x10000u);
-      }
-    };
-    uint32_t taken = 0;
-    float gv[MOE_MAX_TOPK];
-    int gi[MOE_MAX_TOPK];
-    float gsum = 0.0f;
-    for (int j = 0; j < k; ++j) {
-      if (j > 0) {
-        // later choices: (value desc, index asc) warp argmax over the experts not yet taken
-        float bv = -INFINITY;
-        bi = 0x7fffffff;
-#pragma unroll
-        for (int i = 0; i < EPL; ++i) {
-          const int e = lane + 32 * i;
-          if (e < E && !(taken >> i & 1u) && (l[i] > bv || bi == 0x7fffffff)) {
-            bv = l[i];
-            bi = e;
-          }
-        }
-#pragma unroll
-        for (int o = 16; o; o >>= 1) {
-          const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-          const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-          if (ov > bv || (ov == bv && oi < bi)) {
-            bv = ov;
-            bi = oi;
-          }
-        }
-      }
-      const int owner = bi & 31, slot_i = bi >> 5;
-      float pv = 0.0f;
-#pragma unroll
-      for (int i = 0; i < EPL; ++i)
-        if (i == slot_i) pv = p[i];
-      pv = __shfl_sync(0xffffffffu, pv, owner);
-      if (lane == owner) taken |= 1u << slot_i;
-      if (lane == 0) {
-        ids[t * k + j] = bi;
-        if (probs != nullptr) probs[t * k + j] = pv;  // before any renormalisation
-        if (!renorm) {
-          gates[t * k + j] = pv;
-          count_choice(bi, j, pv);
-        }
-        if constexpr (COUNT) blk_ids[r * k + j] = bi;
-      }
-      if (renorm) {
-#pragma unroll
-        for (int jj = 0; jj < MOE_MAX_TOPK; ++jj)
-          if (jj == j) {
-            gv[jj] = pv;
-            gi[jj] = bi;
-          }
-        gsum += pv;
-      }
-    }
-    if (renorm && lane == 0) {
-#pragma unroll
-      for (int j = 0; j < MOE_MAX_TOPK; ++j) {
-        if (j >= k) break;
-        const float g = gv[j] / gsum;
-        gates[t * k + j] = g;
-        count_choice(gi[j], j, g);
-      }
-    }
-  }
-  if (lane == 0) zs[warp] = zw;
-  if constexpr (COUNT) {
-    // rank the block's pairs per expert in pair order (warp 0), write ranks and segment counts
-    __syncthreads();
-    int* run = reinterpret_cast<int*>(prod);  // reused as running counts until the finalize
-    for (int e = threadIdx.x; e < E; e += 256) run[e] = 0;
-    __syncthreads();
-    const int64_t ntok = min((int64_t)kRouterTokensPerBlock, T - tb);
-    const int npairs = (int)ntok * k;
-    if (warp == 0) {
-      const unsigned lt = (1u << lane) - 1u;
-      for (int c = 0; c < npairs; c += 32) {
-        const int pl = c + lane;
-        const int e = pl < npairs ? blk_ids[pl] : -1;
-        const unsigned same = __match_any_sync(0xffffffffu, e);
-        const int rank = __popc(same & lt);
-        const int base = e >= 0 ? run[e] : 0;
-        __syncwarp();
-        if (e >= 0 && rank == 0) run[e] = base + __popc(same);
-        __syncwarp();
-        if (pl < npairs) dc.local_rank[tb * k + pl] = base + rank;
-      }
-    }
-    __syncthreads();
-    for (int e = threadIdx.x; e < E; e += 256) dc.seg_counts[(int64_t)blockIdx.x * E + e] = run[e];
-    __syncthreads();
-  }
-  // block sums of p in a fixed order (warps ascending), then integer accumulation
-#pragma unroll
-  for (int i = 0; i < EPL; ++i) {
-    const int e = lane + 32 * i;
-    if (e < E) qs[warp][e] = q[i];
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += 256) {
-    float sum = 0.0f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) sum += qs[w][e];
-    const unsigned long long fx = (unsigned long long)llrint((double)sum * kQScale);
-    if (fx) atomicAdd(&acc.q[e], fx);
-    if (cs[e] >> 16) atomicAdd(&acc.c[e], cs[e] >> 16);
-    if constexpr (EXTRA) {
-      if (cs[e] & 0xffffu) atomicAdd(&acc.load[e], cs[e] & 0xffffu);
-      if (imp_s[e]) atomicAdd(&acc.imp[e], (unsigned long long)imp_s[e]);
-    }
-  }
-  if (EXTRA && threadIdx.x == 0) {
-    float zb = 0.0f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) zb += zs[w];
-    atomicAdd(acc.z, (unsigned long long)llrint((double)zb * kZScale));
-  }
+  const int E = ko.E;
+  topk_block<EPL, COUNT, EXTRA>(
+      ko, (int64_t)blockIdx.x, [&](int r, int e) { return logits[(tb + r) * E + e]; },
+      BlockSync{}, (int)threadIdx.x, sh);
   pdl_trigger();
-  if (lb == nullptr && losses == nullptr && exported == nullptr) return;
-  // the last block to finish turns the totals into f, Q, aux (and the losses), or exports them
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) is_last = atomicAdd(acc.ticket, 1u) == gridDim.x - 1;
-  __syncthreads();
-  if (!is_last) return;
-  __threadfence();
-  if (exported != nullptr) {
-    for (int e = threadIdx.x; e < E; e += 256) {
-      exported[e] = (int64_t)atomicAdd(&acc.q[e], 0ull);
-      exported[E + e] = (int64_t)atomicAdd(&acc.c[e], 0u);
-      exported[2 * E + e] = (int64_t)atomicAdd(&acc.imp[e], 0ull);
-      exported[3 * E + e] = (int64_t)atomicAdd(&acc.load[e], 0u);
-    }
-    if (threadIdx.x == 0) exported[4 * E] = (int64_t)atomicAdd(acc.z, 0ull);
-    return;
-  }
-  router_finalize_block(
-      E, T, alpha, [&](int e) { return atomicAdd(&acc.q[e], 0ull); },
-      [&](int e) { return (unsigned long long)atomicAdd(&acc.c[e], 0u); },
-      [&](int e) { return atomicAdd(&acc.imp[e], 0ull); },
-      [&](int e) { return (unsigned long long)atomicAdd(&acc.load[e], 0u); },
-      atomicAdd(acc.z, 0ull), lb, losses, prod);
+  topk_block_last(ko, gridDim.x, BlockSync{}, (int)threadIdx.x, sh);
 }
 
 template <int EPL>
@@ -487,9 +227,9 @@ cudaError_t launch_topk(const float* logits, int64_t T, int E, int k, int32_t* i
                         cudaStream_t stream) {
   const dim3 grid((unsigned)router_num_blocks(T));
   const bool extra = losses != nullptr || exported != nullptr;
+  const TopkOut ko{T, E, k, ids, gates, probs, acc, alpha, lb, dc, renorm, losses, exported};
   auto go = [&](auto kern) {
-    return launch_kernel(kern, grid, dim3(256), 0, stream, (const float*)logits, T, E, k, ids,
-                         gates, acc, alpha, lb, dc, renorm, losses, exported, probs);
+    return launch_kernel(kern, grid, dim3(256), 0, stream, (const float*)logits, ko);
   };
   if (dc.local_rank != nullptr)
     return extra ? go(router_topk_kernel<EPL, true, true>)
@@ -508,10 +248,12 @@ cudaError_t enqueue_router(const void* x, bool x_bf16, int64_t T, int d, const f
                            int64_t* exported, int64_t T_kernel_choice, float* probs,
                            const uint16_t* w_prepared) {
   if (T == 0) return cudaSuccess;
+  float* const logits_out = logits;  // the caller's (may be nullptr)
   if (!logits) logits = scr.logits_scratch;
   const bool gemv = (T_kernel_choice > T ? T_kernel_choice : T) <= kRouterGemvMaxT;
   const bool tc = !gemv && router_uses_tensor_cores(x_bf16, d);
   const bool prepared = tc && w_prepared != nullptr;
+  const bool fused = tc && router_fused_supported(E) && router_fusion_enabled();
   const int dpad = router_split_dpad(d);
   const int64_t n = tc ? (int64_t)E * dpad : 0;
   const unsigned blocks = (unsigned)(n == 0 ? 1 : ((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096));
@@ -524,6 +266,17 @@ cudaError_t enqueue_router(const void* x, bool x_bf16, int64_t T, int d, const f
                         tc ? scr.w_split : nullptr, scr.acc);
   }
   if (err != cudaSuccess) return err;
+  if (fused) {
+    if (prepared) {
+      // no split kernel ran to zero the statistics accumulators (contiguous in the workspace)
+      const size_t n = (size_t)((const char*)(scr.acc.ticket + 1) - (const char*)scr.acc.q);
+      err = cudaMemsetAsync(scr.acc.q, 0, n, stream);
+      if (err != cudaSuccess) return err;
+    }
+    return enqueue_router_fused(x, T, d, prepared ? w_prepared : scr.w_split, dpad, router_bias, E,
+                                k, logits_out, ids, gates, probs, scr.acc, aux_alpha, lb_stats, dc,
+                                renormalize, losses, exported, status, stream);
+  }
   if (tc) {
     cudaError_t e = enqueue_router_logits_tc(x, T, d, prepared ? w_prepared : scr.w_split, dpad,
                                              router_bias, E, logits, status, stream,

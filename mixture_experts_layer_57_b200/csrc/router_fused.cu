@@ -18,6 +18,7 @@
 // Bounded waits as in the grouped GEMM (MOE_DEVERR_TIMEOUT, drain, free TMEM).
 #include "common.cuh"
 #include "kernels.h"
+#include "router_topk.cuh"
 
 namespace moe {
 namespace {
@@ -253,6 +254,226 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// The router with softmax, top-k and the statistics fused into the tensor-core kernel's epilogue
+// (E <= 128, one expert slice): after a tile's MMAs, the 8 epilogue warps copy the 128 x NE fp32
+// logits (+ bias) from TMEM into shared memory, reusing pipeline stage 0 (the tile's MMAs have
+// read it; the TMA role loads the next tile into stage 0 only after the epilogue is done with it),
+// with the column index XOR-ed by the token (row) index so that both the column-wise copy and the
+// row-wise reads below are free of bank conflicts. They then run the standalone top-k kernel's
+// code (router_topk.cuh) on the tile's two 64-token statistics blocks, one warp per token, so ids,
+// gates, statistics and dispatch ranks are those of the two-kernel path bit for bit, and the
+// logits reach global memory only when the caller asks for them.
+constexpr int kFusedThreads = 320;  // TMA, MMA, 8 epilogue warps
+
+template <int NE>
+__device__ __forceinline__ int lswz(int row, int col) {
+  return row * NE + (col ^ (row & (NE >= 32 ? 31 : NE - 1)));
+}
+
+template <int NE, int EPL, bool COUNT, bool EXTRA>
+__global__ void __launch_bounds__(kFusedThreads, 1)
+    router_fused_kernel(const __grid_constant__ CUtensorMap tmX,
+                        const __grid_constant__ CUtensorMap tmW, const RParams p,
+                        const TopkOut ko) {
+  using C = RCfg<NE>;
+  static_assert(kTM * NE * 4 <= C::kStageBytes, "the logits tile must fit one stage");
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t base_addr = (raw_addr + 1023u) & ~1023u;
+  uint8_t* base = smem_raw + (base_addr - raw_addr);
+  float* L = reinterpret_cast<float*>(base);  // stage 0, reused for the tile's logits
+  using Sh = TopkShared<kSlice, COUNT, EXTRA>;
+  Sh& sh = *reinterpret_cast<Sh*>(base + C::kStages * C::kStageBytes);
+  uint8_t* aux = base + C::kStages * C::kStageBytes + ((sizeof(Sh) + 15) / 16) * 16;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(aux);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(aux + C::kBarBytes);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(aux + C::kBarBytes + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = C::kStages;
+  auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
+  auto empty_bar = [&](int s) { return smem_u32(&bars[S + s]); };
+  auto tfull_bar = [&](int a) { return smem_u32(&bars[2 * S + a]); };
+  auto tempty_bar = [&](int a) { return smem_u32(&bars[2 * S + 2 + a]); };
+  const uint32_t drain_bar = smem_u32(&bars[2 * S + 4]);
+  const uint32_t lfree_bar = smem_u32(&bars[2 * S + 5]);  // the epilogue is done with stage 0
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 8 * 32);
+    }
+    mbar_init(drain_bar, 1);
+    mbar_init(lfree_bar, 8 * 32);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  pdl_wait();
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmW);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const int ntiles = (int)((p.T + kTM - 1) / kTM);
+  const int n_kb = p.dpad / kBK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0, issued = 0, n_local = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++n_local) {
+        bool waited = n_local == 0;  // this CTA's first tile: stage 0 holds no logits yet
+        for (int kb = 0; kb < n_kb; ++kb) {
+          if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          if (stage == 0 && !waited) {
+            // the previous tile's epilogue reads its logits from stage 0
+            if (!mbar_wait_bounded(lfree_bar, (uint32_t)((n_local - 1) & 1), abort_flag, p.status)) {
+              ok = false;
+              break;
+            }
+            waited = true;
+          }
+          const uint32_t sa = base_addr + stage * C::kStageBytes;
+          mbar_arrive_expect_tx(full_bar(stage), C::kStageBytes);
+          tma_load_2d(sa, &tmX, kb * kBK, t * kTM, full_bar(stage));
+#pragma unroll
+          for (int part = 0; part < 3; ++part)
+            tma_load_2d(sa + C::kABytes + part * C::kBPartBytes, &tmW, part * p.dpad + kb * kBK, 0,
+                        full_bar(stage));
+          ++issued;
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      for (int i = max(0, issued - S); i < issued; ++i)
+        mbar_wait_drain_r(full_bar(i % S), (uint32_t)((i / S) & 1), p.status);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      constexpr uint32_t idesc = idesc_bf16_f32(kTM, NE);
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        if (!mbar_wait_bounded(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * NE);
+        for (int kb = 0; kb < n_kb; ++kb) {
+          if (!mbar_wait_bounded(full_bar(stage), phase, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = base_addr + stage * C::kStageBytes;
+          const uint64_t adesc = smem_desc_sw128(sa);
+#pragma unroll
+          for (int part = 0; part < 3; ++part) {
+            const uint64_t bdesc = smem_desc_sw128(sa + C::kABytes + part * C::kBPartBytes);
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk)
+              tc_mma_bf16(d_tmem, adesc + (uint64_t)(2 * kk), bdesc + (uint64_t)(2 * kk), idesc,
+                          (kb | part | kk) != 0 ? 1u : 0u);
+          }
+          tc_commit(empty_bar(stage));
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(tfull_bar(acc));
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      tc_commit(drain_bar);
+      mbar_wait_drain_r(drain_bar, 0, p.status);
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue: top-k of the tile
+    const int tid = threadIdx.x - 64;  // 0..255
+    const int ew = warp - 2;
+    const int quarter = warp & 3;      // TMEM lanes (tokens) [32*quarter, 32*quarter + 32)
+    const int half = ew >> 2;          // 16-expert chunks half, half + 2, ...
+    const NamedSync sync{1, 256};
+    const unsigned n_blocks = (unsigned)((p.T + kRouterTokensPerBlock - 1) / kRouterTokensPerBlock);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+      // the 8 warps meet at named barriers below: they leave together if any wait gave up
+      const bool ok = mbar_wait_bounded_warp(tfull_bar(acc), acc_phase, abort_flag, p.status);
+      if (named_barrier_any(1, 256, !ok)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * NE);
+      const int row = quarter * 32 + lane;  // token within the tile
+      for (int c0 = half * 16; c0 < NE; c0 += 32) {
+        uint32_t r[16];
+        tmem_ld_32x32b_x16(taddr + (uint32_t)c0, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const int e = c0 + c;
+          const float b = (p.bias && e < p.E) ? p.bias[e] : 0.0f;
+          L[lswz<NE>(row, e)] = __uint_as_float(r[c]) + b;
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(tempty_bar(acc));  // the accumulator is free for the tile after next
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+      sync();
+      const int64_t t0 = (int64_t)t * kTM;
+      if (p.logits != nullptr) {
+        // whole rows: thread i writes experts i, i + 256, ... of the tile, row-major
+        const int ne = p.E;
+        for (int i = tid; i < kTM * ne; i += 256) {
+          const int rr = i / ne, e = i - rr * ne;
+          if (t0 + rr < p.T) p.logits[(t0 + rr) * ne + e] = L[lswz<NE>(rr, e)];
+        }
+      }
+#pragma unroll 1
+      for (int b = 0; b < kTM / kRouterTokensPerBlock; ++b) {
+        const int64_t blk = t0 / kRouterTokensPerBlock + b;
+        if (blk * kRouterTokensPerBlock >= p.T) break;
+        const int rb = b * kRouterTokensPerBlock;
+        topk_block<EPL, COUNT, EXTRA>(
+            ko, blk, [&](int r, int e) { return L[lswz<NE>(rb + r, e)]; }, sync, tid, sh);
+        topk_block_last(ko, n_blocks, sync, tid, sh);
+        sync();  // the statistics scratch is reused by the next block
+      }
+      mbar_arrive(lfree_bar);  // stage 0 may take the next tile's data
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  pdl_trigger();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -289,7 +510,63 @@ cudaError_t launch_tc(const CUtensorMap& tmX, const CUtensorMap& tmW, const RPar
   return launch_kernel(kern, dim3(grid), dim3(kThreads), RCfg<NE>::kSmemBytes, stream, tmX, tmW, p);
 }
 
+template <int NE, bool COUNT, bool EXTRA>
+cudaError_t launch_fused(const CUtensorMap& tmX, const CUtensorMap& tmW, const RParams& p,
+                         const TopkOut& ko, int ntiles, cudaStream_t stream) {
+  constexpr int EPL = NE >= 32 ? NE / 32 : 1;
+  auto kern = router_fused_kernel<NE, EPL, COUNT, EXTRA>;
+  constexpr int smem = 1024 + RCfg<NE>::kStages * RCfg<NE>::kStageBytes +
+                       (int)((sizeof(TopkShared<kSlice, COUNT, EXTRA>) + 15) / 16 * 16) +
+                       RCfg<NE>::kBarBytes + 16;
+  static_assert(smem <= 227 * 1024, "shared memory budget");
+  static_assert(2 * RCfg<NE>::kStages + 6 <= RCfg<NE>::kBarBytes / 8, "barrier area too small");
+  static int attr_done[64] = {0};  // per device
+  cudaError_t e = ensure_dynamic_smem(kern, smem, attr_done);
+  if (e != cudaSuccess) return e;
+  const int grid = ntiles < num_sms() ? ntiles : num_sms();
+  return launch_kernel(kern, dim3(grid), dim3(kFusedThreads), smem, stream, tmX, tmW, p, ko);
+}
+
+template <int NE>
+cudaError_t launch_fused_ne(const CUtensorMap& tmX, const CUtensorMap& tmW, const RParams& p,
+                            const TopkOut& ko, int ntiles, cudaStream_t stream) {
+  const bool count = ko.dc.local_rank != nullptr;
+  const bool extra = ko.losses != nullptr || ko.exported != nullptr;
+  if (count)
+    return extra ? launch_fused<NE, true, true>(tmX, tmW, p, ko, ntiles, stream)
+                 : launch_fused<NE, true, false>(tmX, tmW, p, ko, ntiles, stream);
+  return extra ? launch_fused<NE, false, true>(tmX, tmW, p, ko, ntiles, stream)
+               : launch_fused<NE, false, false>(tmX, tmW, p, ko, ntiles, stream);
+}
+
 }  // namespace
+
+bool router_fused_supported(int E) { return E <= kSlice; }
+
+cudaError_t enqueue_router_fused(const void* x, int64_t T, int d, const uint16_t* w_split,
+                                 int dpad, const float* router_bias, int E, int k, float* logits,
+                                 int32_t* ids, float* gates, float* probs, const RouterAccum& acc,
+                                 float aux_alpha, float* lb_stats, RouterDispatchCount dc,
+                                 bool renormalize, float* losses, int64_t* exported, int* status,
+                                 cudaStream_t stream) {
+  if (T == 0) return cudaSuccess;
+  if (E > kSlice) return cudaErrorInvalidValue;
+  int NE = 16;
+  while (NE < E) NE <<= 1;
+  CUtensorMap tmX, tmW;
+  if (!make_map(&tmX, x, T, d, kTM) || !make_map(&tmW, w_split, E, 3 * dpad, NE))
+    return cudaErrorInvalidValue;
+  const RParams p{T, E, dpad, 1, router_bias, logits, status, RouterAccum{}, 0};
+  const TopkOut ko{T, E, k, ids, gates, probs, acc, aux_alpha, lb_stats, dc,
+                   renormalize ? 1 : 0, losses, exported};
+  const int ntiles = (int)((T + kTM - 1) / kTM);
+  switch (NE) {
+    case 16: return launch_fused_ne<16>(tmX, tmW, p, ko, ntiles, stream);
+    case 32: return launch_fused_ne<32>(tmX, tmW, p, ko, ntiles, stream);
+    case 64: return launch_fused_ne<64>(tmX, tmW, p, ko, ntiles, stream);
+    default: return launch_fused_ne<128>(tmX, tmW, p, ko, ntiles, stream);
+  }
+}
 
 cudaError_t enqueue_router_logits_tc(const void* x, int64_t T, int d, const uint16_t* w_split,
                                      int dpad, const float* router_bias, int E, float* logits,

@@ -138,3 +138,62 @@ def test_prepared_router_weight_gives_identical_layer(cuda_ok, cfg, T):
     parts = to_host(prep).view(np.uint16).reshape(E, 3, dpad)[:, :, :d]
     widened = synth.bf16_bits_to_f32(parts).astype(np.float64)
     np.testing.assert_array_equal(widened.sum(1), inp["w_router"].astype(np.float64))
+
+
+def _router_all(inp, k, renormalize, want_losses):
+    r = moe.moe_router_topk(to_dev(inp["x"]), to_dev(inp["w_router"]), k,
+                            router_bias=to_dev(inp.get("router_bias")), renormalize=renormalize,
+                            router_losses=True if want_losses else None, probs=True)
+    assert moe.moe_get_device_error(r["ws"]) == 0
+    return {n: to_host(v) for n, v in r.items() if isinstance(v, torch.Tensor) and n != "ws"}
+
+
+@pytest.mark.parametrize("T,d,E,k,renorm,extra", [
+    (16384, 1024, 128, 1, False, False),   # the headline router: one tile per CTA
+    (40000, 64, 128, 2, True, True),       # several tiles per CTA: stage 0 handed back and forth
+    (20000, 256, 37, 3, False, True),      # E not a power of two, 64-expert tile
+    (300, 128, 8, 2, True, True),          # 16-expert tile, ragged last tile
+    (1000, 512, 32, 1, False, False),
+])
+def test_fused_router_equals_two_kernels(cuda_ok, monkeypatch, T, d, E, k, renorm, extra):
+    # softmax, top-k and the statistics in the tensor-core kernel's epilogue give the bits of the
+    # separate top-k kernel reading the logits back
+    w = synth.Workload("fused", T=T, d_model=d, d_ff=8, E=E, k=k, capacity_factor=1.0,
+                       dtype="bf16", w_router_std=0.05, router_bias="normal", router_bias_std=0.3,
+                       seed=T + E)
+    inp = synth.make_inputs(w)
+    fused = _router_all(inp, k, renorm, extra)
+    monkeypatch.setenv("MOE_FUSED_ROUTER", "0")
+    two = _router_all(inp, k, renorm, extra)
+    for name in two:
+        assert np.array_equal(fused[name].view(np.uint8), two[name].view(np.uint8)), name
+    check_router(w, inp, fused, sample=np.arange(0, T, max(1, T // 512)), k=k)
+
+
+def test_fused_router_layer_without_logits_output(cuda_ok, monkeypatch):
+    # the layer with no logits requested (nothing of them reaches global memory) gives the same
+    # routing, dispatch and output as with them, and as the two-kernel router
+    from tests.helpers import dev_inputs
+    w = synth.WORKLOADS[2].with_(T=4096, d_model=512, d_ff=1024)
+    d_inp = dev_inputs(synth.make_inputs(w))
+    args = moe.layer_args(d_inp["x"], d_inp["w_router"], d_inp["w1"], d_inp["b1"], d_inp["w2"],
+                          d_inp["b2"], k=w.k, capacity_factor=w.capacity_factor)
+
+    def run(with_logits):
+        aux = dict(expert_ids=torch.empty(w.T, 1, dtype=torch.int32, device="cuda"),
+                   slot=torch.empty(w.T, 1, dtype=torch.int32, device="cuda"),
+                   lb_stats=torch.empty(2 * w.E + 1, dtype=torch.float32, device="cuda"))
+        if with_logits:
+            aux["logits"] = torch.empty(w.T, w.E, dtype=torch.float32, device="cuda")
+        out = torch.empty(w.T, w.d_model, dtype=torch.bfloat16, device="cuda")
+        ws = moe.workspace(moe.moe_layer_workspace_bytes(args), "cuda")
+        moe.moe_layer_forward(args, out, aux=aux, ws=ws)
+        assert moe.moe_get_device_error(ws) == 0
+        return {n: to_host(t) for n, t in aux.items() if n != "logits"} | {"out": to_host(out)}
+
+    a, b = run(False), run(True)
+    monkeypatch.setenv("MOE_FUSED_ROUTER", "0")
+    c = run(False)
+    for n in a:
+        assert np.array_equal(a[n], b[n]), n
+        assert np.array_equal(a[n], c[n]), n
