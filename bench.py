@@ -234,6 +234,8 @@ def run_reference(args, dist: Dist):
     w = synth.WORKLOADS[args.workload]
     if args.tokens:
         w = w.with_(T=args.tokens, name=f"{w.name}-T{args.tokens}")
+    if args.experts:
+        w = w.with_(E=args.experts, name=f"{w.name}-E{args.experts}")
     inp = synth.make_inputs(w)
     # the GPU path's routing is not used here: the logits of all T tokens come from the oracle,
     # computed once (outside the steps); each step then pays the router for its own tokens
@@ -434,6 +436,9 @@ def main():
                     help="skip the other workloads' per-workload entries")
     ap.add_argument("--tokens", type=int, default=None,
                     help="run the workload with T tokens instead of its own (profiling captures)")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="run the workload with E experts instead of its own (profiling captures "
+                         "that must stay small: T / E tokens per expert keeps the capacity)")
     args = ap.parse_args()
     dist = Dist()
     if args.gpus != dist.world and dist.world > 1:
@@ -452,6 +457,8 @@ def main():
     w = synth.WORKLOADS[args.workload]
     if args.tokens:
         w = w.with_(T=args.tokens, name=f"{w.name}-T{args.tokens}")
+    if args.experts:
+        w = w.with_(E=args.experts, name=f"{w.name}-E{args.experts}")
     run = LayerRun(moe, w, device)
     inp, d = run.inp, run.d
     T, E, k, dm, df = w.T, w.E, w.k, w.d_model, w.d_ff
@@ -554,7 +561,7 @@ def main():
         own["sequential"] = {"stages": seq, "ms_per_step_sum": float(sum(bd_seq.values()))}
         own["experts"] = group_rate(seq, ["expert_gemm1", "expert_gemm2"], peaks)
         own["dense_mlp"] = group_rate(seq, ["dense_gemm1", "dense_gemm2_combine"], peaks)
-    if not args.skip_others and not args.tokens and dist.world == 1:
+    if not args.skip_others and not args.tokens and not args.experts and dist.world == 1:
         for wid in (4, 5, 2):
             if wid == args.workload:
                 continue
@@ -575,6 +582,11 @@ def main():
     for name in ("gpt350m-moe128", "gpt1.3b-prmoe128"):
         if name in entries and entries[name]["experts"]:
             bars[f"{name} experts hbm_frac (weight-bound, >= 0.70)"] = entries[name]["experts"]["hbm_frac"]
+
+    # ---------------------------------------------------------- priority overflow, worst case
+    prio_collapse = None
+    if not args.skip_others and dist.world == 1:
+        prio_collapse = priority_collapse(moe, device, stream)
 
     # ---------------------------------------------------------- end to end through the API
     e2e = None
@@ -611,7 +623,8 @@ def main():
             "gpu_launches": launches_per_step * args.steps,
             "breakdown_ms": bd, "routing": routing, "north_star_bars": bars,
             "headline_groups": own,
-            "per_workload": per_workload, "train_step": train,
+            "per_workload": per_workload, "priority_dispatch_collapse": prio_collapse,
+            "train_step": train,
             "step_ms": {"min": float(min(step_ms)), "p10": float(np.percentile(step_ms, 10)),
                         "median": float(np.median(step_ms)),
                         "p90": float(np.percentile(step_ms, 90)), "max": float(max(step_ms))}}
@@ -619,6 +632,38 @@ def main():
         print(json.dumps(line), flush=True)
     dist.close()
     return 0
+
+
+def priority_collapse(moe, device, stream) -> dict:
+    """moe_dispatch_priority when every token picks one expert (the ranking's worst case: one
+    list of T pairs), event-timed at two batch sizes to show how the time grows with T."""
+    out = {}
+    gen = torch.Generator(device=device).manual_seed(3)
+    for T in (16384, 65536):
+        E, d = 128, 1024
+        x = torch.randn(T, d, generator=gen, device=device).to(torch.bfloat16)
+        ids = torch.full((T, 1), 3, dtype=torch.int32, device=device)
+        probs = torch.rand(T, 1, generator=gen, device=device)
+        C = moe.moe_capacity(T, E, 1, 1.0)
+        r = moe.moe_dispatch(x, ids, E, C, priority_probs=probs)
+        for _ in range(3):
+            moe.moe_dispatch(x, ids, E, C, priority_probs=probs, **{k: r[k] for k in (
+                "slot", "expert_counts", "expert_offsets", "row_token", "x_packed", "ws")})
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(10)]
+        for a, b in evs:
+            a.record(stream)
+            moe.moe_dispatch(x, ids, E, C, priority_probs=probs, stream=stream, **{k: r[k] for k in (
+                "slot", "expert_counts", "expert_offsets", "row_token", "x_packed", "ws")})
+            b.record(stream)
+        torch.cuda.synchronize()
+        assert moe.moe_get_device_error(r["ws"]) == 0
+        kept = int((r["slot"] >= 0).sum())
+        out[str(T)] = {"ms": float(np.median([a.elapsed_time(b) for a, b in evs])),
+                       "kept": kept, "capacity": C,
+                       "launches": moe.moe_last_launch_count()}
+    return out
 
 
 def host_cpu() -> dict:
@@ -721,37 +766,97 @@ def train_step(moe, args_c, d, w, stream, flush_buf, args, dist, device, E_t, R)
 
 
 def end_to_end(moe, args_c, d, w, ws, stream, args, dist, device) -> dict:
-    """Same metric through the public call with host buffers: per step H2D of x from pinned
-    memory, moe_layer_forward, D2H of the output into pinned memory, all inside the events."""
+    """Same metric through the public call with host buffers, as a serving loop runs it: every
+    step copies its x from pinned host memory to the device (copy-in stream), runs
+    moe_layer_forward (compute stream) and copies the output back to pinned host memory
+    (copy-out stream), all inside the timed region; two device buffers let step i's copies
+    overlap steps i - 1 and i + 1 (events order each buffer's reuse). Also reported: the same
+    with the three operations serialised on one stream."""
+    from mixture_experts_layer_57_b200 import moe as _moe
     T, dm = w.T, w.d_model
-    x_dev = d["x"]
-    x_pin = torch.empty(x_dev.shape, dtype=x_dev.dtype, pin_memory=True)
-    x_pin.copy_(x_dev.cpu())
-    out_dev = torch.empty(T, dm, dtype=x_dev.dtype, device=device)
-    out_pin = torch.empty(T, dm, dtype=x_dev.dtype, pin_memory=True)
+    x_dev0 = d["x"]
+    x_pin = torch.empty(x_dev0.shape, dtype=x_dev0.dtype, pin_memory=True)
+    x_pin.copy_(x_dev0.cpu())
+    xs = [torch.empty_like(x_dev0) for _ in range(2)]
+    outs = [torch.empty(T, dm, dtype=x_dev0.dtype, device=device) for _ in range(2)]
+    out_pins = [torch.empty(T, dm, dtype=x_dev0.dtype, pin_memory=True) for _ in range(2)]
+    step_args = []
+    for b in range(2):
+        a = _moe.LayerArgs()
+        ctypes_copy(a, args_c)
+        a.x = xs[b].data_ptr()
+        step_args.append(a)
+    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    ev = lambda: torch.cuda.Event()
+    in_done = [ev(), ev()]
+    fwd_done = [ev(), ev()]
+    out_done = [ev(), ev()]
+    started = [False, False]
 
-    def step():
-        x_dev.copy_(x_pin, non_blocking=True)
-        moe.moe_layer_forward(args_c, out_dev, ws=ws, stream=stream)
-        out_pin.copy_(out_dev, non_blocking=True)
+    def step(i):
+        b = i % 2
+        with torch.cuda.stream(s_in):
+            if started[b]:
+                s_in.wait_event(fwd_done[b])      # the forward of step i - 2 has read xs[b]
+            xs[b].copy_(x_pin, non_blocking=True)
+            in_done[b].record(s_in)
+        stream.wait_event(in_done[b])
+        if started[b]:
+            stream.wait_event(out_done[b])        # step i - 2's output has been copied out
+        moe.moe_layer_forward(step_args[b], outs[b], ws=ws, stream=stream)
+        fwd_done[b].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(fwd_done[b])
+            out_pins[b].copy_(outs[b], non_blocking=True)
+            out_done[b].record(s_out)
+        started[b] = True
 
-    for _ in range(max(3, args.warmup)):
-        step()
+    for i in range(max(3, args.warmup)):
+        step(i)
     torch.cuda.synchronize()
     n = max(3, min(args.steps, 50))
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     dist.barrier()
     torch.cuda.synchronize()
+    t0.record(stream)
+    s_in.wait_event(t0)
+    s_out.wait_event(t0)
     for i in range(n):
-        evs[i][0].record(stream)
-        step()
-        evs[i][1].record(stream)
+        step(i)
+    stream.wait_event(out_done[(n - 1) % 2])
+    t1.record(stream)
     torch.cuda.synchronize()
     dist.barrier()
-    ms = dist.max(float(np.mean([a.elapsed_time(b) for a, b in evs])), device)
-    es = x_dev.element_size()
+    ms = dist.max(t0.elapsed_time(t1) / n, device)
+    assert torch.equal(out_pins[(n - 1) % 2], outs[(n - 1) % 2].cpu())
+
+    # the serial form: copy in, forward, copy out on one stream, each step waiting for the last
+    def serial():
+        xs[0].copy_(x_pin, non_blocking=True)
+        moe.moe_layer_forward(step_args[0], outs[0], ws=ws, stream=stream)
+        out_pins[0].copy_(outs[0], non_blocking=True)
+
+    for _ in range(3):
+        serial()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for a, b in evs:
+        a.record(stream)
+        serial()
+        b.record(stream)
+    torch.cuda.synchronize()
+    ms_serial = dist.max(float(np.mean([a.elapsed_time(b) for a, b in evs])), device)
+    es = x_dev0.element_size()
     return {"value": args.gpus * T / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms, "steps": n,
-            "h2d_bytes_per_step": T * dm * es, "d2h_bytes_per_step": T * dm * out_pin.element_size()}
+            "h2d_bytes_per_step": T * dm * es, "d2h_bytes_per_step": T * dm * out_pins[0].element_size(),
+            "pipeline": "copy-in, compute and copy-out streams, two device buffers",
+            "serial": {"value": args.gpus * T / (ms_serial / 1e3), "ms_per_step": ms_serial}}
+
+
+def ctypes_copy(dst, src):
+    """Field-by-field copy of a ctypes structure."""
+    for name, _ in src._fields_:
+        setattr(dst, name, getattr(src, name))
 
 
 if __name__ == "__main__":

@@ -47,12 +47,29 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
     for (int v = 0; v < VEC; ++v) acc[v] = 0.0f;
     if (residual) {
+      if constexpr (VEC == 4 && RES_BF16) {
+        const uint2 rb = *reinterpret_cast<const uint2*>(
+            reinterpret_cast<const uint16_t*>(residual) + t * d + c);
+        acc[0] = __uint_as_float(rb.x << 16);
+        acc[1] = __uint_as_float(rb.x & 0xffff0000u);
+        acc[2] = __uint_as_float(rb.y << 16);
+        acc[3] = __uint_as_float(rb.y & 0xffff0000u);
+      } else {
 #pragma unroll
-      for (int v = 0; v < VEC; ++v) acc[v] = load_elem<RES_BF16>(residual, t * d + c + v);
+        for (int v = 0; v < VEC; ++v) acc[v] = load_elem<RES_BF16>(residual, t * d + c + v);
+      }
     }
     if (dense) {
+      if constexpr (VEC == 4) {
+        const float4 q = *reinterpret_cast<const float4*>(dense + t * d + c);
+        acc[0] += q.x;
+        acc[1] += q.y;
+        acc[2] += q.z;
+        acc[3] += q.w;
+      } else {
 #pragma unroll
-      for (int v = 0; v < VEC; ++v) acc[v] += dense[t * d + c + v];
+        for (int v = 0; v < VEC; ++v) acc[v] += dense[t * d + c + v];
+      }
     }
     for (int j = 0; j < nk; ++j) {
       const float* src = y + row[j] * d + c;
@@ -67,10 +84,19 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
       for (int v = 0; v < VEC; ++v) acc[v] = fmaf(g[j], yv[v], acc[v]);
     }
-    if constexpr (OUT_BF16) {
+    if constexpr (OUT_BF16 && VEC == 4) {
+      // one 8-byte store of the 4 rounded values (d % 4 == 0, so t * d + c is a multiple of 4)
+      uint2 o;
+      o.x = (uint32_t)f32_to_bf16_rn(acc[0]) | ((uint32_t)f32_to_bf16_rn(acc[1]) << 16);
+      o.y = (uint32_t)f32_to_bf16_rn(acc[2]) | ((uint32_t)f32_to_bf16_rn(acc[3]) << 16);
+      *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(out) + t * d + c) = o;
+    } else if constexpr (OUT_BF16) {
       uint16_t* o = reinterpret_cast<uint16_t*>(out) + t * d + c;
 #pragma unroll
       for (int v = 0; v < VEC; ++v) o[v] = f32_to_bf16_rn(acc[v]);
+    } else if constexpr (VEC == 4) {
+      *reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + t * d + c) =
+          make_float4(acc[0], acc[1], acc[2], acc[3]);
     } else {
       float* o = reinterpret_cast<float*>(out) + t * d + c;
 #pragma unroll

@@ -163,7 +163,7 @@ def spread_tokens(w: synth.Workload, ids: np.ndarray, slot: np.ndarray, n_min: i
     for group in (dropped, partial):
         if len(group):
             pick.update(int(t) for t in rng.choice(group, min(len(group), 16), replace=False))
-    kept = np.nonzero(kept_pair.all(1))[0]
+    kept = np.setdiff1d(np.nonzero(kept_pair.all(1))[0], np.array(sorted(pick), dtype=np.int64))
     need = n_min - len(pick)
     if need > 0 and len(kept):
         pick.update(int(t) for t in rng.choice(kept, min(len(kept), need), replace=False))

@@ -87,6 +87,7 @@ def test_full_workloads_sampled(cuda_ok, cfg, n):
     dict(T=2048, d_model=1024, d_ff=2048, E=16),    # capacity 128: 128-token expert tiles
     dict(T=1000, d_model=512, d_ff=1024, E=128),    # capacity 8: 16-token expert tiles, ragged T
     dict(T=300, d_model=256, d_ff=128, E=4),        # one 128-feature tile per expert
+    dict(T=600, d_model=256, d_ff=512, E=8, capacity_factor=0.0),  # no expert rows at all
 ])
 def test_prmoe_coscheduled_equals_sequential(cuda_ok, monkeypatch, shape):
     # the expert and dense GEMM layers co-scheduled in one launch each (default) give the same
@@ -172,16 +173,16 @@ def test_determinism_bitwise(cuda_ok):
 def test_launch_count(cuda_ok):
     w = synth.WORKLOADS[3].with_(T=256, d_model=128, d_ff=256)
     got = run_layer(w, dev_inputs(synth.make_inputs(w)))
-    # router 3 (prep: weight split + zeroed accumulators, tensor-core logits, top-k with the
-    # statistics and the dispatch ranks), dispatch 2 (scan, scatter), experts 2, dense MLP 2 (its
-    # layer 2 carries the combine)
-    assert got["launches"] == 9
+    # router 2 (prep: weight split + zeroed accumulators; tensor-core logits with softmax, top-k,
+    # the statistics and the dispatch ranks in the epilogue), dispatch 2 (scan, scatter), the
+    # expert and dense layers co-scheduled 2, the combine 1
+    assert got["launches"] == 7
     w1 = synth.WORKLOADS[2].with_(T=256, d_model=128, d_ff=256)
     got = run_layer(w1, dev_inputs(synth.make_inputs(w1)))
-    assert got["launches"] == 7      # top-1: the combine is fused into the experts' layer 2
+    assert got["launches"] == 6      # top-1: the combine is fused into the experts' layer 2
     w2 = synth.WORKLOADS[4].with_(T=256, d_model=128, d_ff=256)
     got = run_layer(w2, dev_inputs(synth.make_inputs(w2)))
-    assert got["launches"] == 8      # top-2: gather combine kernel
+    assert got["launches"] == 7      # top-2: gather combine kernel
 
 
 @pytest.mark.parametrize("cfg", [2, 3, 4])
@@ -200,8 +201,8 @@ def test_profiled_forward_matches_and_labels_stages(cuda_ok, cfg):
     names = moe.moe_layer_forward_profiled(args, out, evs)
     torch.cuda.synchronize()
     want = {2: ["start", "router", "dispatch", "expert_gemm1", "expert_gemm2_combine"],
-            3: ["start", "router", "dispatch", "expert_gemm1", "expert_gemm2", "dense_gemm1",
-                "dense_gemm2_combine"],
+            3: ["start", "router", "dispatch", "experts_dense_gemm1", "experts_dense_gemm2",
+                "combine"],
             4: ["start", "router", "dispatch", "expert_gemm1", "expert_gemm2", "combine"]}[cfg]
     assert names == want
     assert all(evs[i].elapsed_time(evs[i + 1]) >= 0 for i in range(len(names) - 1))

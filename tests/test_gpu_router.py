@@ -167,7 +167,11 @@ def test_fused_router_equals_two_kernels(cuda_ok, monkeypatch, T, d, E, k, renor
     two = _router_all(inp, k, renorm, extra)
     for name in two:
         assert np.array_equal(fused[name].view(np.uint8), two[name].view(np.uint8)), name
-    check_router(w, inp, fused, sample=np.arange(0, T, max(1, T // 512)), k=k)
+    # against the oracle: the probabilities output carries the unrenormalised gates
+    check_router(w, inp, {**fused, "gates": fused["probs"]},
+                 sample=np.arange(0, T, max(1, T // 512)), k=k)
+    if renorm:
+        np.testing.assert_allclose(fused["gates"].sum(1), 1.0, rtol=1e-5)
 
 
 def test_fused_router_layer_without_logits_output(cuda_ok, monkeypatch):
