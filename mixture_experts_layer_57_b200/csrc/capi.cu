@@ -34,16 +34,6 @@ bool router_fusion_enabled() {
   return !(v != nullptr && v[0] == '0');
 }
 
-// K blocks of weights the grouped GEMM prefetches into L2 ahead of its loads when an expert's
-// rows fit one token tile, so its weights stream from HBM exactly once (MOE_L2_PREFETCH=<n>,
-// default 8; 0 turns it off). Read at every call.
-int l2_prefetch_kblocks() {
-  const char* v = std::getenv("MOE_L2_PREFETCH");
-  if (v == nullptr || v[0] == '\0') return 8;
-  const int n = std::atoi(v);
-  return n < 0 ? 0 : (n > 64 ? 64 : n);
-}
-
 // Whether bf16 PR-MoE layers co-schedule each expert GEMM layer with the dense MLP's layer in one
 // launch (MOE_COSCHEDULE=0 runs them one after another, the dense layer 2 with the combine fused;
 // both give the same bits). Read at every call.

@@ -120,10 +120,6 @@ struct Params {
   // wait_limit_ns. Normal launches: selftest_no_copies = 0, wait_limit_ns = kWaitLimitNs.
   int selftest_no_copies = 0;
   uint64_t wait_limit_ns = kWaitLimitNs;
-  // Weight boxes the TMA role prefetches into L2 ahead of its loads, in K blocks (0 = none): a
-  // tile that streams its weights from HBM once keeps more bytes in flight than its shared-memory
-  // stages hold, so fewer SMs can keep HBM busy.
-  int l2_prefetch_kb = 0;
 };
 
 struct Tile {
@@ -221,14 +217,7 @@ __device__ __forceinline__ bool produce_tile(const Tile& tl, const CUtensorMap* 
                                              int& issued, volatile int* abort_flag) {
   constexpr uint32_t kTx = FT * kBM * kBK * 2 + BN * kBK * 2;
   const int w_row = tl.e * p.n_out + tl.f0;
-  const int pf = A_MN ? 0 : p.l2_prefetch_kb;
-  auto prefetch = [&](int kb) {
-#pragma unroll
-    for (int i = 0; i < FT; ++i) tma_prefetch_l2_2d(tmW, kb * kBK, w_row + i * kBM);
-  };
-  for (int kb = 0; kb < min(pf, n_kb); ++kb) prefetch(kb);
   for (int kb = 0; kb < n_kb; ++kb) {
-    if (pf > 0 && kb + pf < n_kb) prefetch(kb + pf);
     if (!mbar_wait_bounded(B.empty(ring.stage), ring.phase ^ 1u, abort_flag, p.status,
                            p.wait_limit_ns))
       return false;
@@ -913,12 +902,6 @@ static int pick_token_tile(int64_t capacity_hint) {
 #define MOE_GG_FT 2
 #endif
 
-// L2 prefetch distance for a layer: grouped layers whose experts fit one token tile stream each
-// weight tile from HBM once; compute-bound and one-segment layers reuse theirs from L2.
-static int prefetch_kb_for(const int32_t* offsets, int64_t capacity_hint) {
-  return (offsets != nullptr && capacity_hint <= 128) ? l2_prefetch_kblocks() : 0;
-}
-
 // Fraction of the last wave's CTA slots that hold a tile (tiles over persistent CTAs).
 static double wave_efficiency(int64_t tiles) {
   const int64_t s = num_sms();
@@ -963,7 +946,6 @@ cudaError_t enqueue_grouped_gemm_bf16(const void* x, const int32_t* offsets, int
   if (!make_kmajor_map(&tmW, w, (int64_t)E * N, K, kBM) || !make_kmajor_map(&tmX, x, rows_max, K, BN))
     return cudaErrorInvalidValue;
   Params p{offsets, E, N, K, rows_max, bias, out, status, CombineArgs{}, nullptr, nullptr};
-  p.l2_prefetch_kb = prefetch_kb_for(offsets, capacity_hint);
   return gelu ? launch_bn<kEpiGeluBf16>(BN, tmW, tmX, p, stream, capacity_hint)
               : launch_bn<kEpiF32>(BN, tmW, tmX, p, stream, capacity_hint);
 }
@@ -980,7 +962,6 @@ cudaError_t enqueue_grouped_gemm_bf16_train(const void* x, const int32_t* offset
     return cudaErrorInvalidValue;
   Params p{offsets, E, N, K, rows_max, bias, h_out, status, CombineArgs{}, nullptr,
            (uint16_t*)g_out};
-  p.l2_prefetch_kb = prefetch_kb_for(offsets, capacity_hint);
   return launch_bn<kEpiGeluBf16Train>(BN, tmW, tmX, p, stream, capacity_hint);
 }
 
@@ -1012,7 +993,6 @@ cudaError_t enqueue_gemm2_combine(const void* h, const int32_t* offsets, int E, 
                 (const uint16_t*)fc.residual, fc.out, fc.out_bf16 ? 1 : 0, fc.k, fc.E_experts,
                 fc.rows_y};
   Params p{offsets, E, N, K, rows_max, bias, nullptr, status, c, nullptr, nullptr};
-  p.l2_prefetch_kb = prefetch_kb_for(offsets, capacity_hint);
   return fc.dense ? launch_bn<kEpiCombineDense>(BN, tmW, tmX, p, stream, capacity_hint)
                   : launch_bn<kEpiCombineExpert>(BN, tmW, tmX, p, stream, capacity_hint);
 }
@@ -1040,7 +1020,6 @@ cudaError_t enqueue_co_gemm_bf16(const void* xp, const int32_t* offsets, int E, 
     return cudaErrorInvalidValue;
   Params p0{offsets, E, N, K, rows_max, bias, out, status, CombineArgs{}, nullptr, nullptr};
   Params p1{nullptr, 1, N, K, T, bias_dense, out_dense, status, CombineArgs{}, nullptr, nullptr};
-  p0.l2_prefetch_kb = prefetch_kb_for(offsets, capacity_hint);
   auto go = [&](auto tag) -> cudaError_t {
     constexpr int EPI = decltype(tag)::value;
     switch (BN0) {

@@ -18,8 +18,6 @@ int num_sms();
 
 // Whether launches carry the programmatic-dependent-launch attribute (MOE_PDL=0 disables it).
 bool pdl_enabled();
-// L2 prefetch distance of weight-streaming expert GEMM tiles in K blocks (MOE_L2_PREFETCH).
-int l2_prefetch_kblocks();
 // Whether bf16 PR-MoE layers co-schedule expert and dense GEMM layers (MOE_COSCHEDULE=0: no).
 bool coschedule_enabled();
 

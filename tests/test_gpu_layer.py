@@ -99,8 +99,10 @@ def test_prmoe_coscheduled_equals_sequential(cuda_ok, monkeypatch, shape):
     co = layer_parity(w, inp, d_inp)["got"]
     monkeypatch.setenv("MOE_COSCHEDULE", "0")
     seq = layer_parity(w, inp, d_inp)["got"]
-    # co-scheduled: two GEMM launches and the combine; sequential: four GEMM launches
-    assert co["launches"] == seq["launches"] - 1
+    # co-scheduled: two GEMM launches and the combine; sequential: four GEMM launches, or only
+    # the dense MLP's two when no expert keeps a row
+    no_rows = int(co["expert_offsets"][-1]) == 0
+    assert co["launches"] == seq["launches"] + (1 if no_rows else -1)
     assert np.array_equal(co["out"], seq["out"])
     for name in ("expert_ids", "gates", "slot", "expert_offsets", "lb_stats"):
         assert np.array_equal(co[name], seq[name]), name
