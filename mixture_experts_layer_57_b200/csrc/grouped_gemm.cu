@@ -35,6 +35,7 @@
 // Every wait is bounded (about 2 s): on expiry the kernel records MOE_DEVERR_TIMEOUT in the
 // status word, the other roles stop, in-flight TMA copies and MMAs are drained, TMEM is freed.
 #include <algorithm>
+#include <cstdlib>
 #include <type_traits>
 
 #include "common.cuh"
@@ -76,8 +77,9 @@ struct Cfg {
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kStagesFit = (200 * 1024) / kStageBytes;
   static constexpr int kStages = kStagesFit > MOE_GG_MAX_STAGES ? MOE_GG_MAX_STAGES : kStagesFit;
-  static constexpr int kTmemCols = (2 * FT * BN) < 32 ? 32 : (2 * FT * BN);
-  static_assert(2 * FT * BN <= 512, "two buffers of FT accumulators must fit TMEM");
+  static constexpr int kNumAcc = 2;  // the epilogue of tile i overlaps the MMAs of tile i + 1
+  static constexpr int kTmemCols = (kNumAcc * FT * BN) < 32 ? 32 : (kNumAcc * FT * BN);
+  static_assert(kNumAcc * FT * BN <= 512, "two buffers of FT accumulators must fit TMEM");
   // barriers: full[S], empty[S], tmem_full[2], tmem_empty[2], drain  (8 bytes each, <= 64 of them)
   static constexpr int kBarBytes = 8 * 64;
   static constexpr int kAuxBytes = kBarBytes + 16 + 2 * 4 * (MOE_MAX_EXPERTS + 1);
@@ -584,7 +586,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     base_addr, C::kStageBytes, C::kABytes, B, ring, abort_flag))
           break;
         tc_commit(B.tfull(acc));
-        if (++acc == 2) {
+        if (++acc == C::kNumAcc) {
           acc = 0;
           acc_phase ^= 1u;
         }
@@ -610,7 +612,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                  half, lane, st);
       tc_fence_before();
       mbar_arrive(B.tempty(acc));
-      if (++acc == 2) {
+      if (++acc == C::kNumAcc) {
         acc = 0;
         acc_phase ^= 1u;
       }
