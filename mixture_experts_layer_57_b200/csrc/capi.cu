@@ -639,11 +639,12 @@ moe_status layer_forward_impl(const moe_layer_args* a, void* out, moe_layer_aux*
     dcount.local_rank = w.dispatch.local_rank;
     dcount.seg_counts = w.dispatch.seg_counts;
     const bool begin = sh.mode == kShardBegin;
+    // the statistics are left as integer accumulators: the dispatch scan finalises them below,
+    // off the router's critical path (a shard exports them instead)
     e = enqueue_router(a->x, bf16, T, d, a->w_router, a->router_bias, E, k, logits, ids, gates,
-                       begin ? nullptr : lb, a->aux_alpha, w.router.scr, status, stream, dcount,
-                       a->renormalize_gates != 0, begin ? nullptr : losses,
-                       begin ? sh.partials_out : nullptr, sh.T_global, probs,
-                       (const uint16_t*)a->w_router_prepared);
+                       nullptr, a->aux_alpha, w.router.scr, status, stream, dcount,
+                       a->renormalize_gates != 0, nullptr, begin ? sh.partials_out : nullptr,
+                       sh.T_global, probs, (const uint16_t*)a->w_router_prepared);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     rec.mark("router");
   }
@@ -687,10 +688,18 @@ moe_status layer_forward_impl(const moe_layer_args* a, void* out, moe_layer_aux*
     prio.keys = w.dispatch.prio_keys;
     prio.demand_offsets = w.dispatch.demand_offsets;
   }
+  StatsFinalize fin;
+  if (sh.mode == kWhole) {
+    fin.acc = w.router.scr.acc;
+    fin.T = T;
+    fin.alpha = a->aux_alpha;
+    fin.lb = lb;
+    fin.losses = losses;
+  }
   e = enqueue_dispatch(a->x, bf16, T, d, ids, E, k, w.C, slot, counts, offsets, w.row_token,
                        w.x_packed, w.rows_max, w.dispatch.local_rank, w.dispatch.seg_counts,
                        w.dispatch.seg_base, status, stream, dropped,
-                       (int)kRouterTokensPerBlock * k, prio, shard);
+                       (int)kRouterTokensPerBlock * k, prio, shard, false, fin);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   rec.mark("dispatch");
 

@@ -36,6 +36,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "router_topk.cuh"
 
 namespace moe {
 namespace {
@@ -112,8 +113,9 @@ __global__ void __launch_bounds__(1024)
     dispatch_scan_kernel(const int32_t* __restrict__ seg_counts, int64_t nseg, int E, int64_t C,
                          int32_t* __restrict__ seg_base, int32_t* __restrict__ counts,
                          int32_t* __restrict__ offsets, int32_t* __restrict__ demand_offsets,
-                         ShardBase shard) {
+                         ShardBase shard, StatsFinalize fin) {
   __shared__ int run_sum[1024];
+  __shared__ float prod[MOE_MAX_EXPERTS];
   __shared__ int kept[MOE_MAX_EXPERTS];
   __shared__ int warp_sums[32];
   pdl_wait();
@@ -182,6 +184,15 @@ __global__ void __launch_bounds__(1024)
     block_exclusive_scan_experts(tid < E ? counts[tid] : 0, E, warp_sums, demand_offsets);
   }
   pdl_trigger();
+  if (fin.lb != nullptr || fin.losses != nullptr) {
+    // the router's statistics from its integer accumulators (complete: the router kernel ended)
+    const RouterAccum& a = fin.acc;
+    router_finalize_block(
+        E, fin.T, fin.alpha, [&](int e) { return a.q[e]; },
+        [&](int e) { return (unsigned long long)a.c[e]; }, [&](int e) { return a.imp[e]; },
+        [&](int e) { return (unsigned long long)a.load[e]; }, *a.z, fin.lb, fin.losses, prod, tid,
+        1024, BlockSync{});
+  }
 }
 
 // Sort key of a pair for the priority order: ascending keys = probability descending, then pair
@@ -386,7 +397,7 @@ cudaError_t enqueue_dispatch(const void* x, bool bf16, int64_t T, int d, const i
                              int32_t* local_rank, int32_t* seg_counts, int32_t* seg_base,
                              int* status, cudaStream_t stream, DroppedRows dropped,
                              int counted_seg_len, PriorityDispatch prio, ShardBase shard,
-                             bool scan_only) {
+                             bool scan_only, StatsFinalize fin) {
   const int64_t pairs = T * k;
   const int seg_len = counted_seg_len > 0 ? counted_seg_len : kDispatchSeg;
   const int64_t nseg = (pairs + seg_len - 1) / seg_len;
@@ -400,7 +411,7 @@ cudaError_t enqueue_dispatch(const void* x, bool bf16, int64_t T, int d, const i
   {
     cudaError_t e = launch_kernel(dispatch_scan_kernel, dim3(1), dim3(1024), 0, stream,
                                   (const int32_t*)seg_counts, nseg, E, C, seg_base, counts, offsets,
-                                  prio.probs != nullptr ? prio.demand_offsets : nullptr, shard);
+                                  prio.probs != nullptr ? prio.demand_offsets : nullptr, shard, fin);
     if (e != cudaSuccess) return e;
   }
   if (scan_only) return cudaGetLastError();

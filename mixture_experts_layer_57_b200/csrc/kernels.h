@@ -183,13 +183,24 @@ struct ShardBase {
   int rank = 0;
   int32_t* cap_local = nullptr;
 };
+// Optional: the router's load-balance statistics finalised by the dispatch scan kernel (the
+// router then leaves them as integer accumulators): f, Q, aux into lb and the router losses into
+// losses (either may be nullptr), from the accumulators of T tokens.
+struct StatsFinalize {
+  RouterAccum acc{};
+  int64_t T = 0;
+  float alpha = 0.0f;
+  float* lb = nullptr;
+  float* losses = nullptr;
+};
 cudaError_t enqueue_dispatch(const void* x, bool bf16, int64_t T, int d, const int32_t* ids, int E,
                              int k, int64_t C, int32_t* slot, int32_t* counts, int32_t* offsets,
                              int32_t* row_token, void* x_packed, int64_t rows_max,
                              int32_t* local_rank, int32_t* seg_counts, int32_t* seg_base,
                              int* status, cudaStream_t stream, DroppedRows dropped = DroppedRows{},
                              int counted_seg_len = 0, PriorityDispatch prio = PriorityDispatch{},
-                             ShardBase shard = ShardBase{}, bool scan_only = false);
+                             ShardBase shard = ShardBase{}, bool scan_only = false,
+                             StatsFinalize fin = StatsFinalize{});
 // counted_seg_len > 0: local_rank and seg_counts were already written (segments of that many
 // pairs) by the router's top-k kernel; the counting kernel is skipped.
 

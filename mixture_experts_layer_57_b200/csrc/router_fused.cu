@@ -135,6 +135,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
         const int tok_tile = t / p.n_slices, slice = t % p.n_slices;
+        if (slice == 0)  // the tile's x rows into L2 at once (see the fused kernel)
+          for (int kb = 0; kb < n_kb; ++kb) tma_prefetch_l2_2d(&tmX, kb * kBK, tok_tile * kTM);
         for (int kb = 0; kb < n_kb; ++kb) {
           if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, p.status)) {
             ok = false;
@@ -335,6 +337,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++n_local) {
         bool waited = n_local == 0;  // this CTA's first tile: stage 0 holds no logits yet
+        // the tile's x rows, read from HBM once, requested into L2 at once: the stage ring alone
+        // keeps too few bytes in flight to hide DRAM latency (the weight parts are L2 hits)
+        for (int kb = 0; kb < n_kb; ++kb) tma_prefetch_l2_2d(&tmX, kb * kBK, t * kTM);
         for (int kb = 0; kb < n_kb; ++kb) {
           if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, p.status)) {
             ok = false;

@@ -146,115 +146,142 @@ __device__ __forceinline__ void topk_block(const TopkOut& ko, int64_t blk, Logit
 #pragma unroll
   for (int i = 0; i < EPL; ++i) q[i] = 0.0f;
   const int64_t tb = blk * kRouterTokensPerBlock;
-  for (int r = warp; r < kRouterTokensPerBlock; r += 8) {
-    const int64_t t = tb + r;
-    if (t >= T) break;
-    float l[EPL];
-    float m = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-      const int e = lane + 32 * i;
-      l[i] = e < E ? logit_at(r, e) : -INFINITY;
-      m = fmaxf(m, l[i]);
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float ex[EPL];
-    float s = 0.0f;
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-      ex[i] = (lane + 32 * i) < E ? expf(l[i] - m) : 0.0f;
-      s += ex[i];
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  // per-block integer counts (order-independent): first choices, and with the extra
+  // statistics every choice and its gate
+  auto count_choice = [&](int e, int j, float g) {
     if constexpr (EXTRA) {
-      const float lz = m + logf(s);  // log sum_e exp(l_e)
-      zw += lz * lz;
+      atomicAdd(&cs[e], j == 0 ? 0x10001u : 1u);
+      atomicAdd(&imp_s[e], __float2uint_rn(g * (float)kIScale));
+    } else if (j == 0) {
+      atomicAdd(&cs[e], 0x10000u);
     }
-    float p[EPL];
+  };
+  // A warp takes its tokens r = warp, warp + 8, ... TPI at a time (r, r + 8, ...): their softmaxes
+  // are computed with the shuffle reductions interleaved (independent dependency chains), and each
+  // token's p is added to this warp's sums in token order, as one at a time would. Two tokens for
+  // up to 128 experts; one beyond (the registers would not hold two).
+  constexpr int TPI = EPL <= 4 ? 2 : 1;
+  for (int r0 = warp; r0 < kRouterTokensPerBlock; r0 += 8 * TPI) {
+    int rr[TPI];
+    bool ok[TPI];
+    float l[TPI][EPL], m[TPI], s[TPI], p[TPI][EPL];
 #pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-      p[i] = ex[i] / s;
-      q[i] += p[i];
-    }
-    // first choice: the lowest expert index holding the maximum logit (ballot per slot)
-    int bi = 0x7fffffff;
+    for (int u = 0; u < TPI; ++u) {
+      rr[u] = r0 + 8 * u;
+      ok[u] = rr[u] < kRouterTokensPerBlock && tb + rr[u] < T;
+      m[u] = -INFINITY;
 #pragma unroll
-    for (int i = EPL - 1; i >= 0; --i) {
-      const unsigned b = __ballot_sync(0xffffffffu, (lane + 32 * i) < E && l[i] == m);
-      if (b) bi = 32 * i + __ffs(b) - 1;
+      for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        l[u][i] = (ok[u] && e < E) ? logit_at(rr[u], e) : -INFINITY;
+        m[u] = fmaxf(m[u], l[u][i]);
+      }
     }
-    // per-block integer counts (order-independent): first choices, and with the extra
-    // statistics every choice and its gate
-    auto count_choice = [&](int e, int j, float g) {
+    if (!ok[0]) break;
+#pragma unroll
+    for (int o = 16; o; o >>= 1)
+#pragma unroll
+      for (int u = 0; u < TPI; ++u) m[u] = fmaxf(m[u], __shfl_xor_sync(0xffffffffu, m[u], o));
+    float ex[TPI][EPL];
+#pragma unroll
+    for (int u = 0; u < TPI; ++u) {
+      s[u] = 0.0f;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        ex[u][i] = (ok[u] && (lane + 32 * i) < E) ? expf(l[u][i] - m[u]) : 0.0f;
+        s[u] += ex[u][i];
+      }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1)
+#pragma unroll
+      for (int u = 0; u < TPI; ++u) s[u] += __shfl_xor_sync(0xffffffffu, s[u], o);
+#pragma unroll
+    for (int u = 0; u < TPI; ++u) {
+      if (!ok[u]) continue;
       if constexpr (EXTRA) {
-        atomicAdd(&cs[e], j == 0 ? 0x10001u : 1u);
-        atomicAdd(&imp_s[e], __float2uint_rn(g * (float)kIScale));
-      } else if (j == 0) {
-        atomicAdd(&cs[e], 0x10000u);
+        const float lz = m[u] + logf(s[u]);  // log sum_e exp(l_e)
+        zw += lz * lz;
       }
-    };
-    uint32_t taken = 0;
-    float gv[MOE_MAX_TOPK];
-    int gi[MOE_MAX_TOPK];
-    float gsum = 0.0f;
-    for (int j = 0; j < k; ++j) {
-      if (j > 0) {
-        // later choices: (value desc, index asc) warp argmax over the experts not yet taken
-        float bv = -INFINITY;
-        bi = 0x7fffffff;
 #pragma unroll
-        for (int i = 0; i < EPL; ++i) {
-          const int e = lane + 32 * i;
-          if (e < E && !(taken >> i & 1u) && (l[i] > bv || bi == 0x7fffffff)) {
-            bv = l[i];
-            bi = e;
-          }
-        }
-#pragma unroll
-        for (int o = 16; o; o >>= 1) {
-          const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-          const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-          if (ov > bv || (ov == bv && oi < bi)) {
-            bv = ov;
-            bi = oi;
-          }
-        }
-      }
-      const int owner = bi & 31, slot_i = bi >> 5;
-      float pv = 0.0f;
-#pragma unroll
-      for (int i = 0; i < EPL; ++i)
-        if (i == slot_i) pv = p[i];
-      pv = __shfl_sync(0xffffffffu, pv, owner);
-      if (lane == owner) taken |= 1u << slot_i;
-      if (lane == 0) {
-        ids[t * k + j] = bi;
-        if (probs != nullptr) probs[t * k + j] = pv;  // before any renormalisation
-        if (!renorm) {
-          gates[t * k + j] = pv;
-          count_choice(bi, j, pv);
-        }
-        if constexpr (COUNT) blk_ids[r * k + j] = bi;
-      }
-      if (renorm) {
-#pragma unroll
-        for (int jj = 0; jj < MOE_MAX_TOPK; ++jj)
-          if (jj == j) {
-            gv[jj] = pv;
-            gi[jj] = bi;
-          }
-        gsum += pv;
+      for (int i = 0; i < EPL; ++i) {
+        p[u][i] = ex[u][i] / s[u];
+        q[i] += p[u][i];
       }
     }
-    if (renorm && lane == 0) {
 #pragma unroll
-      for (int j = 0; j < MOE_MAX_TOPK; ++j) {
-        if (j >= k) break;
-        const float g = gv[j] / gsum;
-        gates[t * k + j] = g;
-        count_choice(gi[j], j, g);
+    for (int u = 0; u < TPI; ++u) {
+      if (!ok[u]) break;
+      const int r = rr[u];
+      const int64_t t = tb + r;
+      // first choice: the lowest expert index holding the maximum logit (ballot per slot)
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int i = EPL - 1; i >= 0; --i) {
+        const unsigned b = __ballot_sync(0xffffffffu, (lane + 32 * i) < E && l[u][i] == m[u]);
+        if (b) bi = 32 * i + __ffs(b) - 1;
+      }
+      uint32_t taken = 0;
+      float gv[MOE_MAX_TOPK];
+      int gi[MOE_MAX_TOPK];
+      float gsum = 0.0f;
+      for (int j = 0; j < k; ++j) {
+        if (j > 0) {
+          // later choices: (value desc, index asc) warp argmax over the experts not yet taken
+          float bv = -INFINITY;
+          bi = 0x7fffffff;
+#pragma unroll
+          for (int i = 0; i < EPL; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E && !(taken >> i & 1u) && (l[u][i] > bv || bi == 0x7fffffff)) {
+              bv = l[u][i];
+              bi = e;
+            }
+          }
+#pragma unroll
+          for (int o = 16; o; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (ov > bv || (ov == bv && oi < bi)) {
+              bv = ov;
+              bi = oi;
+            }
+          }
+        }
+        const int owner = bi & 31, slot_i = bi >> 5;
+        float pv = 0.0f;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i)
+          if (i == slot_i) pv = p[u][i];
+        pv = __shfl_sync(0xffffffffu, pv, owner);
+        if (lane == owner) taken |= 1u << slot_i;
+        if (lane == 0) {
+          ids[t * k + j] = bi;
+          if (probs != nullptr) probs[t * k + j] = pv;  // before any renormalisation
+          if (!renorm) {
+            gates[t * k + j] = pv;
+            count_choice(bi, j, pv);
+          }
+          if constexpr (COUNT) blk_ids[r * k + j] = bi;
+        }
+        if (renorm) {
+#pragma unroll
+          for (int jj = 0; jj < MOE_MAX_TOPK; ++jj)
+            if (jj == j) {
+              gv[jj] = pv;
+              gi[jj] = bi;
+            }
+          gsum += pv;
+        }
+      }
+      if (renorm && lane == 0) {
+#pragma unroll
+        for (int j = 0; j < MOE_MAX_TOPK; ++j) {
+          if (j >= k) break;
+          const float g = gv[j] / gsum;
+          gates[t * k + j] = g;
+          count_choice(gi[j], j, g);
+        }
       }
     }
   }
