@@ -644,7 +644,8 @@ moe_status layer_forward_impl(const moe_layer_args* a, void* out, moe_layer_aux*
     e = enqueue_router(a->x, bf16, T, d, a->w_router, a->router_bias, E, k, logits, ids, gates,
                        nullptr, a->aux_alpha, w.router.scr, status, stream, dcount,
                        a->renormalize_gates != 0, nullptr, begin ? sh.partials_out : nullptr,
-                       sh.T_global, probs, (const uint16_t*)a->w_router_prepared);
+                       sh.T_global, probs, (const uint16_t*)a->w_router_prepared,
+                       losses != nullptr);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     rec.mark("router");
   }

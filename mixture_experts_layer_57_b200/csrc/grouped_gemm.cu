@@ -150,21 +150,27 @@ __device__ __forceinline__ Tile decode_tile(int t, const int* prefix, const int*
   return tl;
 }
 
-// Tile order of a one-segment problem (the dense MLP: rows = tokens): groups of kDenseGroup token
-// tiles; inside a group, every token tile of the group for feature tile 0, then for feature tile
-// 1, and so on. The tiles in flight at one time then share a few weight tiles and a few token
-// tiles (a working set that stays in L2), where a feature-tile-major order would sweep all the
-// tokens once per feature tile.
-constexpr int kDenseGroup = 16;
+// Tile order of a one-segment problem (the dense MLP: rows = tokens): groups of token tiles;
+// inside a group, every token tile of the group for feature tile 0, then for feature tile 1, and
+// so on. The tiles in flight at one time then share a few weight tiles and a few token tiles (a
+// working set that stays in L2), where a feature-tile-major order would sweep all the tokens once
+// per feature tile. A group holds about 24 MB of token rows (16 tiles at K = 2048, 6 at K = 8192)
+// and at most 16 tiles.
+__host__ __device__ __forceinline__ int dense_group_tiles(int BN, int K) {
+  const int64_t per_tile = (int64_t)BN * K * 2;
+  const int64_t g = (int64_t)(24 << 20) / (per_tile > 0 ? per_tile : 1);
+  return g < 1 ? 1 : (g > 16 ? 16 : (int)g);
+}
 template <int BN, int FT>
-__device__ __forceinline__ Tile decode_dense_tile(int u, int64_t rows, int n_ftiles) {
+__device__ __forceinline__ Tile decode_dense_tile(int u, int64_t rows, int n_ftiles, int K) {
+  const int group = dense_group_tiles(BN, K);
   const int n_tt = (int)((rows + BN - 1) / BN);
-  const int per_group = n_ftiles * kDenseGroup;
+  const int per_group = n_ftiles * group;
   const int g = u / per_group;
   const int in = u - g * per_group;
-  const int gt = min(kDenseGroup, n_tt - g * kDenseGroup);
+  const int gt = min(group, n_tt - g * group);
   const int ft = in / gt;
-  const int jt = g * kDenseGroup + (in - ft * gt);
+  const int jt = g * group + (in - ft * gt);
   Tile tl;
   tl.e = 0;
   tl.f0 = ft * kBM * FT;
@@ -553,7 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_kb = (p.K + kBK - 1) / kBK;
   const bool one_seg = p.offsets == nullptr;
   auto tile_at = [&](int t) {
-    return one_seg ? decode_dense_tile<BN, FT>(t, p.rows_max, n_ftiles)
+    return one_seg ? decode_dense_tile<BN, FT>(t, p.rows_max, n_ftiles, p.K)
                    : decode_tile<BN, FT>(t, prefix, seg, p.E, n_ftiles);
   };
 
@@ -737,7 +743,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                           kCoStageBytes, kA0, B, ring, issued,
                                                           abort_flag)
                             : produce_tile<kCoBN1, 1, false>(
-                                  decode_dense_tile<kCoBN1, 1>(u, p1.rows_max, nft1), &tmW1, &tmX1,
+                                  decode_dense_tile<kCoBN1, 1>(u, p1.rows_max, nft1, p1.K), &tmW1, &tmX1,
                                   p1, nkb1, base_addr, kCoStageBytes, kA1, B, ring, issued,
                                   abort_flag);
         if (!ok) break;
@@ -760,7 +766,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                       d_tmem, p0, nkb0, base_addr, kCoStageBytes,
                                                       kA0, B, ring, abort_flag)
                             : mma_tile<kCoBN1, 1, false>(
-                                  decode_dense_tile<kCoBN1, 1>(u, p1.rows_max, nft1), d_tmem, p1,
+                                  decode_dense_tile<kCoBN1, 1>(u, p1.rows_max, nft1, p1.K), d_tmem, p1,
                                   nkb1, base_addr, kCoStageBytes, kA1, B, ring, abort_flag);
         if (!ok) break;
         tc_commit(B.tfull(acc));
@@ -788,7 +794,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         epilogue_tile<BN0, 2, EPI>(decode_tile<BN0, 2>(u, prefix, seg, p0.E, nft0), p0, acc_tmem,
                                    quarter, half, lane, st);
       else
-        epilogue_tile<kCoBN1, 1, EPI>(decode_dense_tile<kCoBN1, 1>(u, p1.rows_max, nft1), p1,
+        epilogue_tile<kCoBN1, 1, EPI>(decode_dense_tile<kCoBN1, 1>(u, p1.rows_max, nft1, p1.K), p1,
                                       acc_tmem, quarter, half, lane, st);
       tc_fence_before();
       mbar_arrive(B.tempty(acc));

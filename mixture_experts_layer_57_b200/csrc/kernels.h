@@ -87,7 +87,10 @@ cudaError_t enqueue_router(const void* x, bool x_bf16, int64_t T, int d, const f
                            RouterDispatchCount dcount = RouterDispatchCount{},
                            bool renormalize = false, float* losses = nullptr,
                            int64_t* export_partials = nullptr, int64_t T_kernel_choice = -1,
-                           float* probs = nullptr, const uint16_t* w_prepared = nullptr);
+                           float* probs = nullptr, const uint16_t* w_prepared = nullptr,
+                           bool extra_stats = false);
+// extra_stats: accumulate the z-loss, Importance and Load sums although losses == nullptr (a
+// later kernel finalises them from the accumulators).
 // w_prepared (optional): W_r already split (enqueue_router_prepare); the tensor-core path then
 // skips the split, and the logits kernel zeroes the statistics accumulators instead.
 // Splits W_r [E, d] into the three bf16 parts [E, 3 * router_split_dpad(d)].
@@ -116,8 +119,8 @@ cudaError_t enqueue_router_fused(const void* x, int64_t T, int d, const uint16_t
                                  int dpad, const float* router_bias, int E, int k, float* logits,
                                  int32_t* ids, float* gates, float* probs, const RouterAccum& acc,
                                  float aux_alpha, float* lb_stats, RouterDispatchCount dc,
-                                 bool renormalize, float* losses, int64_t* exported, int* status,
-                                 cudaStream_t stream);
+                                 bool renormalize, float* losses, int64_t* exported,
+                                 bool extra_stats, int* status, cudaStream_t stream);
 
 // Raises a kernel's dynamic shared-memory limit to `bytes` on the current device, once per
 // device (done_per_device: a zero-initialised [64] array owned by the launching function).

@@ -224,10 +224,11 @@ template <int EPL>
 cudaError_t launch_topk(const float* logits, int64_t T, int E, int k, int32_t* ids, float* gates,
                         const RouterAccum& acc, float alpha, float* lb, RouterDispatchCount dc,
                         int renorm, float* losses, int64_t* exported, float* probs,
-                        cudaStream_t stream) {
+                        bool extra_stats, cudaStream_t stream) {
   const dim3 grid((unsigned)router_num_blocks(T));
-  const bool extra = losses != nullptr || exported != nullptr;
-  const TopkOut ko{T, E, k, ids, gates, probs, acc, alpha, lb, dc, renorm, losses, exported};
+  const bool extra = losses != nullptr || exported != nullptr || extra_stats;
+  const TopkOut ko{T, E, k,     ids,    gates,    probs,   acc,
+                   alpha, lb, dc, renorm, losses, exported, extra_stats ? 1 : 0};
   auto go = [&](auto kern) {
     return launch_kernel(kern, grid, dim3(256), 0, stream, (const float*)logits, ko);
   };
@@ -246,7 +247,7 @@ cudaError_t enqueue_router(const void* x, bool x_bf16, int64_t T, int d, const f
                            const RouterScratch& scr, int* status, cudaStream_t stream,
                            RouterDispatchCount dc, bool renormalize, float* losses,
                            int64_t* exported, int64_t T_kernel_choice, float* probs,
-                           const uint16_t* w_prepared) {
+                           const uint16_t* w_prepared, bool extra_stats) {
   if (T == 0) return cudaSuccess;
   float* const logits_out = logits;  // the caller's (may be nullptr)
   if (!logits) logits = scr.logits_scratch;
@@ -275,7 +276,7 @@ cudaError_t enqueue_router(const void* x, bool x_bf16, int64_t T, int d, const f
     }
     return enqueue_router_fused(x, T, d, prepared ? w_prepared : scr.w_split, dpad, router_bias, E,
                                 k, logits_out, ids, gates, probs, scr.acc, aux_alpha, lb_stats, dc,
-                                renormalize, losses, exported, status, stream);
+                                renormalize, losses, exported, extra_stats, status, stream);
   }
   if (tc) {
     cudaError_t e = enqueue_router_logits_tc(x, T, d, prepared ? w_prepared : scr.w_split, dpad,
@@ -292,21 +293,21 @@ cudaError_t enqueue_router(const void* x, bool x_bf16, int64_t T, int d, const f
   const int rn = renormalize ? 1 : 0;
   if (E <= 32)
     return launch_topk<1>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, rn,
-                          losses, exported, probs, stream);
+                          losses, exported, probs, extra_stats, stream);
   if (E <= 64)
     return launch_topk<2>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, rn,
-                          losses, exported, probs, stream);
+                          losses, exported, probs, extra_stats, stream);
   if (E <= 128)
     return launch_topk<4>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, rn,
-                          losses, exported, probs, stream);
+                          losses, exported, probs, extra_stats, stream);
   if (E <= 256)
     return launch_topk<8>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, rn,
-                          losses, exported, probs, stream);
+                          losses, exported, probs, extra_stats, stream);
   if (E <= 512)
     return launch_topk<16>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, rn,
-                           losses, exported, probs, stream);
+                           losses, exported, probs, extra_stats, stream);
   return launch_topk<32>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, rn,
-                         losses, exported, probs, stream);
+                         losses, exported, probs, extra_stats, stream);
 }
 
 cudaError_t enqueue_router_prepare(const float* w_router, int E, int d, uint16_t* out,

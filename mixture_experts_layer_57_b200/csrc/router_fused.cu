@@ -133,6 +133,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0, issued = 0;
       uint32_t phase = 0;
       bool ok = true;
+      // the weight parts into L2 first, a share per CTA (see the fused kernel)
+      for (int b = blockIdx.x; b < 3 * n_kb * p.n_slices; b += gridDim.x) {
+        const int sl = b / (3 * n_kb), rem = b % (3 * n_kb);
+        tma_prefetch_l2_2d(&tmW, (rem / n_kb) * p.dpad + (rem % n_kb) * kBK, sl * kSlice);
+      }
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
         const int tok_tile = t / p.n_slices, slice = t % p.n_slices;
         if (slice == 0)  // the tile's x rows into L2 at once (see the fused kernel)
@@ -335,6 +340,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       int stage = 0, issued = 0, n_local = 0;
       uint32_t phase = 0;
       bool ok = true;
+      // every CTA runs the K blocks in the same order at about the same time, so each weight box
+      // would be requested by all of them before its first copy reached L2: the CTAs first pull
+      // the split weight (3 * dpad / 64 boxes) into L2 between them, a share each
+      for (int b = blockIdx.x; b < 3 * n_kb; b += gridDim.x)
+        tma_prefetch_l2_2d(&tmW, (b / n_kb) * p.dpad + (b % n_kb) * kBK, 0);
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++n_local) {
         bool waited = n_local == 0;  // this CTA's first tile: stage 0 holds no logits yet
         // the tile's x rows, read from HBM once, requested into L2 at once: the stage ring alone
@@ -536,7 +546,7 @@ template <int NE>
 cudaError_t launch_fused_ne(const CUtensorMap& tmX, const CUtensorMap& tmW, const RParams& p,
                             const TopkOut& ko, int ntiles, cudaStream_t stream) {
   const bool count = ko.dc.local_rank != nullptr;
-  const bool extra = ko.losses != nullptr || ko.exported != nullptr;
+  const bool extra = ko.losses != nullptr || ko.exported != nullptr || ko.extra_stats != 0;
   if (count)
     return extra ? launch_fused<NE, true, true>(tmX, tmW, p, ko, ntiles, stream)
                  : launch_fused<NE, true, false>(tmX, tmW, p, ko, ntiles, stream);
@@ -552,8 +562,8 @@ cudaError_t enqueue_router_fused(const void* x, int64_t T, int d, const uint16_t
                                  int dpad, const float* router_bias, int E, int k, float* logits,
                                  int32_t* ids, float* gates, float* probs, const RouterAccum& acc,
                                  float aux_alpha, float* lb_stats, RouterDispatchCount dc,
-                                 bool renormalize, float* losses, int64_t* exported, int* status,
-                                 cudaStream_t stream) {
+                                 bool renormalize, float* losses, int64_t* exported,
+                                 bool extra_stats, int* status, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
   if (E > kSlice) return cudaErrorInvalidValue;
   int NE = 16;
@@ -562,8 +572,8 @@ cudaError_t enqueue_router_fused(const void* x, int64_t T, int d, const uint16_t
   if (!make_map(&tmX, x, T, d, kTM) || !make_map(&tmW, w_split, E, 3 * dpad, NE))
     return cudaErrorInvalidValue;
   const RParams p{T, E, dpad, 1, router_bias, logits, status, RouterAccum{}, 0};
-  const TopkOut ko{T, E, k, ids, gates, probs, acc, aux_alpha, lb_stats, dc,
-                   renormalize ? 1 : 0, losses, exported};
+  const TopkOut ko{T,  E,  k,  ids, gates, probs, acc, aux_alpha, lb_stats, dc, renormalize ? 1 : 0,
+                   losses, exported, extra_stats ? 1 : 0};
   const int ntiles = (int)((T + kTM - 1) / kTM);
   switch (NE) {
     case 16: return launch_fused_ne<16>(tmX, tmW, p, ko, ntiles, stream);

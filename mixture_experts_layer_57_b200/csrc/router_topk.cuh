@@ -105,6 +105,9 @@ struct TopkOut {
   int renorm;
   float* losses;
   int64_t* exported;
+  // accumulate the z-loss, Importance and Load sums although this launch writes no losses (the
+  // dispatch scan finalises them)
+  int extra_stats;
 };
 
 // Softmax, top-k and the statistics of the 64-token block `blk` (tokens [64 blk, 64 blk + 64)),
