@@ -25,10 +25,15 @@ __global__ void __launch_bounds__(256)
   const int lane = threadIdx.x & 31;
   const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (t >= T) return;
+  // the kept choices in order, held in registers (fully unrolled over the largest k): row -1 and
+  // gate 0 for a choice that is dropped or out of range
   int64_t row[MOE_MAX_TOPK];
   float g[MOE_MAX_TOPK];
-  int nk = 0;
-  for (int j = 0; j < k; ++j) {
+#pragma unroll
+  for (int j = 0; j < MOE_MAX_TOPK; ++j) {
+    row[j] = -1;
+    g[j] = 0.0f;
+    if (j >= k) continue;
     const int s = slot[t * k + j];
     if (s < 0) continue;
     const int e = ids[t * k + j];
@@ -38,10 +43,11 @@ __global__ void __launch_bounds__(256)
       if (lane == 0) set_device_error(status, MOE_DEVERR_BAD_ROW);
       continue;
     }
-    row[nk] = r;
-    g[nk] = gates[t * k + j];
-    ++nk;
+    row[j] = r;
+    g[j] = gates[t * k + j];
   }
+  // (VEC == 4: the loop is unrolled so that each lane has several rows' loads in flight)
+#pragma unroll 4
   for (int c = lane * VEC; c < d; c += 32 * VEC) {
     float acc[VEC];
 #pragma unroll
@@ -71,7 +77,9 @@ __global__ void __launch_bounds__(256)
         for (int v = 0; v < VEC; ++v) acc[v] += dense[t * d + c + v];
       }
     }
-    for (int j = 0; j < nk; ++j) {
+#pragma unroll
+    for (int j = 0; j < MOE_MAX_TOPK; ++j) {
+      if (row[j] < 0) continue;
       const float* src = y + row[j] * d + c;
       float yv[VEC];
       if constexpr (VEC == 4) {
