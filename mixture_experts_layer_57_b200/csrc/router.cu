@@ -14,8 +14,11 @@
 //   logits                router_logits_tc_kernel (router_fused.cu, tcgen05: x * W_r =
 //                         x*hi + x*mid + x*lo from exact products, fp32 accumulation) for bf16 x,
 //                         or router_logits_kernel below (fp32 FMA) for fp32 x
-//   router_topk_kernel    one warp per token: max, sum of exp, p = exp(l - max) / sum,
-//                         k rounds of warp argmax on the logits (ties -> lower index), gates
+//   router_topk_tile_kernel (E <= 128) 128 tokens per block, two threads per token, the code
+//                         the tensor-core router runs in its epilogue (router_topk.cuh);
+//   router_topk_kernel    (E > 128) one warp per token. Both: max, sum of exp,
+//                         p = exp(l - max) / sum,
+//                         k rounds of argmax on the logits (ties -> lower index), gates
 //                         (optionally renormalised over the k choices: survey notes §1.1.1.1);
 //                         per-block sums of p (fixed order), first-choice counts, gate sums
 //                         (Importance), choice counts (Load) and (log Z)^2 (comparison article,
@@ -220,6 +223,51 @@ __global__ void __launch_bounds__(256) router_topk_kernel(const float* __restric
   topk_block_last(ko, gridDim.x, BlockSync{}, (int)threadIdx.x, sh);
 }
 
+// E <= 128: one 128-token tile per block, its logits staged in shared memory in the layout of
+// the tensor-core router's epilogue, then the tile top-k that epilogue runs.
+template <int NE, bool COUNT, bool EXTRA>
+__global__ void __launch_bounds__(256) router_topk_tile_kernel(const float* __restrict__ logits,
+                                                               const TopkOut ko) {
+  extern __shared__ __align__(16) uint8_t tile_smem[];
+  float* L = reinterpret_cast<float*>(tile_smem);
+  auto& sh = *reinterpret_cast<TileShared<COUNT, EXTRA>*>(tile_smem + tile_logits_bytes<NE>());
+  pdl_wait();
+  const int64_t tile = blockIdx.x;
+  const int64_t t0 = tile * kTileTokens;
+  const int E = ko.E;
+  const int n = (int)min((int64_t)kTileTokens, ko.T - t0) * E;
+  for (int i = threadIdx.x; i < n; i += 256) {
+    const int r = i / E, e = i - r * E;
+    L[lpos<NE>(r, e)] = logits[t0 * E + i];
+  }
+  __syncthreads();
+  topk_tile<NE, COUNT, EXTRA>(ko, tile, L, BlockSync{}, (int)threadIdx.x, sh);
+  pdl_trigger();
+  const unsigned n_blocks = (unsigned)((ko.T + kRouterTokensPerBlock - 1) / kRouterTokensPerBlock);
+  topk_tile_last(ko, tile, n_blocks, BlockSync{}, (int)threadIdx.x, sh);
+}
+
+template <int NE, bool COUNT, bool EXTRA>
+cudaError_t launch_topk_tile(const float* logits, const TopkOut& ko, cudaStream_t stream) {
+  auto kern = router_topk_tile_kernel<NE, COUNT, EXTRA>;
+  constexpr int smem = tile_logits_bytes<NE>() + (int)sizeof(TileShared<COUNT, EXTRA>);
+  static int attr_done[64] = {0};  // per device
+  cudaError_t e = ensure_dynamic_smem(kern, smem, attr_done);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((unsigned)((ko.T + kTileTokens - 1) / kTileTokens));
+  return launch_kernel(kern, grid, dim3(256), smem, stream, logits, ko);
+}
+
+template <int NE>
+cudaError_t launch_topk_tile_ne(const float* logits, const TopkOut& ko, bool count, bool extra,
+                                cudaStream_t stream) {
+  if (count)
+    return extra ? launch_topk_tile<NE, true, true>(logits, ko, stream)
+                 : launch_topk_tile<NE, true, false>(logits, ko, stream);
+  return extra ? launch_topk_tile<NE, false, true>(logits, ko, stream)
+               : launch_topk_tile<NE, false, false>(logits, ko, stream);
+}
+
 template <int EPL>
 cudaError_t launch_topk(const float* logits, int64_t T, int E, int k, int32_t* ids, float* gates,
                         const RouterAccum& acc, float alpha, float* lb, RouterDispatchCount dc,
@@ -229,14 +277,23 @@ cudaError_t launch_topk(const float* logits, int64_t T, int E, int k, int32_t* i
   const bool extra = losses != nullptr || exported != nullptr || extra_stats;
   const TopkOut ko{T, E, k,     ids,    gates,    probs,   acc,
                    alpha, lb, dc, renorm, losses, exported, extra_stats ? 1 : 0};
-  auto go = [&](auto kern) {
-    return launch_kernel(kern, grid, dim3(256), 0, stream, (const float*)logits, ko);
-  };
-  if (dc.local_rank != nullptr)
-    return extra ? go(router_topk_kernel<EPL, true, true>)
-                 : go(router_topk_kernel<EPL, true, false>);
-  return extra ? go(router_topk_kernel<EPL, false, true>)
-               : go(router_topk_kernel<EPL, false, false>);
+  if constexpr (EPL * 32 <= kTileExperts) {
+    (void)grid;
+    const bool count = dc.local_rank != nullptr;
+    if (E <= 16) return launch_topk_tile_ne<16>(logits, ko, count, extra, stream);
+    if (E <= 32) return launch_topk_tile_ne<32>(logits, ko, count, extra, stream);
+    if (E <= 64) return launch_topk_tile_ne<64>(logits, ko, count, extra, stream);
+    return launch_topk_tile_ne<128>(logits, ko, count, extra, stream);
+  } else {
+    auto go = [&](auto kern) {
+      return launch_kernel(kern, grid, dim3(256), 0, stream, (const float*)logits, ko);
+    };
+    if (dc.local_rank != nullptr)
+      return extra ? go(router_topk_kernel<EPL, true, true>)
+                   : go(router_topk_kernel<EPL, true, false>);
+    return extra ? go(router_topk_kernel<EPL, false, true>)
+                 : go(router_topk_kernel<EPL, false, false>);
+  }
 }
 
 }  // namespace
@@ -291,13 +348,7 @@ cudaError_t enqueue_router(const void* x, bool x_bf16, int64_t T, int d, const f
   }
   const RouterAccum& a = scr.acc;
   const int rn = renormalize ? 1 : 0;
-  if (E <= 32)
-    return launch_topk<1>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, rn,
-                          losses, exported, probs, extra_stats, stream);
-  if (E <= 64)
-    return launch_topk<2>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, rn,
-                          losses, exported, probs, extra_stats, stream);
-  if (E <= 128)
+  if (E <= 128)  // the tile top-k (launch_topk's E <= 128 branch)
     return launch_topk<4>(logits, T, E, k, ids, gates, a, aux_alpha, lb_stats, dc, rn,
                           losses, exported, probs, extra_stats, stream);
   if (E <= 256)

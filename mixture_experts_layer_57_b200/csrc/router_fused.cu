@@ -266,32 +266,40 @@ __global__ void __launch_bounds__(kThreads, 1)
 // logits (+ bias) from TMEM into shared memory, reusing pipeline stage 0 (the tile's MMAs have
 // read it; the TMA role loads the next tile into stage 0 only after the epilogue is done with it),
 // with the column index XOR-ed by the token (row) index so that both the column-wise copy and the
-// row-wise reads below are free of bank conflicts. They then run the standalone top-k kernel's
-// code (router_topk.cuh) on the tile's two 64-token statistics blocks, one warp per token, so ids,
-// gates, statistics and dispatch ranks are those of the two-kernel path bit for bit, and the
-// logits reach global memory only when the caller asks for them.
+// reads of the top-k are free of bank conflicts. They then run the tile top-k (router_topk.cuh:
+// two threads per token, all 128 tokens at once) that the standalone top-k kernel also runs for
+// E <= 128, so ids, gates, statistics and dispatch ranks are those of the two-kernel path bit for
+// bit, and the logits reach global memory only when the caller asks for them.
 constexpr int kFusedThreads = 320;  // TMA, MMA, 8 epilogue warps
 
+// The tile's logits (128 rows of NE + 1 floats) take stage 0 and, where they are longer, a gap of
+// whole KB between stage 0 and stage 1 (stages stay 1024-byte aligned for the 128-byte swizzle).
 template <int NE>
-__device__ __forceinline__ int lswz(int row, int col) {
-  return row * NE + (col ^ (row & (NE >= 32 ? 31 : NE - 1)));
+constexpr int fused_stage_gap() {
+  constexpr int over = tile_logits_bytes<NE>() - RCfg<NE>::kStageBytes;
+  return over <= 0 ? 0 : (over + 1023) / 1024 * 1024;
 }
 
-template <int NE, int EPL, bool COUNT, bool EXTRA>
+template <int NE, bool COUNT, bool EXTRA>
 __global__ void __launch_bounds__(kFusedThreads, 1)
     router_fused_kernel(const __grid_constant__ CUtensorMap tmX,
                         const __grid_constant__ CUtensorMap tmW, const RParams p,
                         const TopkOut ko) {
   using C = RCfg<NE>;
-  static_assert(kTM * NE * 4 <= C::kStageBytes, "the logits tile must fit one stage");
+  constexpr int kGap = fused_stage_gap<NE>();
+  static_assert(tile_logits_bytes<NE>() <= C::kStageBytes + kGap, "the logits tile must fit");
+  static_assert(kTM == kTileTokens, "one top-k tile per MMA tile");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t base_addr = (raw_addr + 1023u) & ~1023u;
   uint8_t* base = smem_raw + (base_addr - raw_addr);
-  float* L = reinterpret_cast<float*>(base);  // stage 0, reused for the tile's logits
-  using Sh = TopkShared<kSlice, COUNT, EXTRA>;
-  Sh& sh = *reinterpret_cast<Sh*>(base + C::kStages * C::kStageBytes);
-  uint8_t* aux = base + C::kStages * C::kStageBytes + ((sizeof(Sh) + 15) / 16) * 16;
+  float* L = reinterpret_cast<float*>(base);  // stage 0 (and the gap after it): the tile's logits
+  using Sh = TileShared<COUNT, EXTRA>;
+  Sh& sh = *reinterpret_cast<Sh*>(base + C::kStages * C::kStageBytes + kGap);
+  uint8_t* aux = base + C::kStages * C::kStageBytes + kGap + ((sizeof(Sh) + 15) / 16) * 16;
+  auto stage_addr = [&](int s) {
+    return base_addr + (uint32_t)(s * C::kStageBytes + (s > 0 ? kGap : 0));
+  };
   uint64_t* bars = reinterpret_cast<uint64_t*>(aux);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(aux + C::kBarBytes);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(aux + C::kBarBytes + 4);
@@ -363,7 +371,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             }
             waited = true;
           }
-          const uint32_t sa = base_addr + stage * C::kStageBytes;
+          const uint32_t sa = stage_addr(stage);
           mbar_arrive_expect_tx(full_bar(stage), C::kStageBytes);
           tma_load_2d(sa, &tmX, kb * kBK, t * kTM, full_bar(stage));
 #pragma unroll
@@ -396,7 +404,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t sa = base_addr + stage * C::kStageBytes;
+          const uint32_t sa = stage_addr(stage);
           const uint64_t adesc = smem_desc_sw128(sa);
 #pragma unroll
           for (int part = 0; part < 3; ++part) {
@@ -443,11 +451,16 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         uint32_t r[16];
         tmem_ld_32x32b_x16(taddr + (uint32_t)c0, r);
         tmem_ld_wait();
+        float4* dst = reinterpret_cast<float4*>(L + lpos<NE>(row, c0));
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const int e = c0 + c;
-          const float b = (p.bias && e < p.E) ? p.bias[e] : 0.0f;
-          L[lswz<NE>(row, e)] = __uint_as_float(r[c]) + b;
+        for (int c = 0; c < 16; c += 4) {
+          float f[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int e = c0 + c + u;
+            f[u] = __uint_as_float(r[c + u]) + ((p.bias && e < p.E) ? p.bias[e] : 0.0f);
+          }
+          dst[c / 4] = make_float4(f[0], f[1], f[2], f[3]);
         }
       }
       tc_fence_before();
@@ -463,19 +476,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         const int ne = p.E;
         for (int i = tid; i < kTM * ne; i += 256) {
           const int rr = i / ne, e = i - rr * ne;
-          if (t0 + rr < p.T) p.logits[(t0 + rr) * ne + e] = L[lswz<NE>(rr, e)];
+          if (t0 + rr < p.T) p.logits[(t0 + rr) * ne + e] = L[lpos<NE>(rr, e)];
         }
       }
-#pragma unroll 1
-      for (int b = 0; b < kTM / kRouterTokensPerBlock; ++b) {
-        const int64_t blk = t0 / kRouterTokensPerBlock + b;
-        if (blk * kRouterTokensPerBlock >= p.T) break;
-        const int rb = b * kRouterTokensPerBlock;
-        topk_block<EPL, COUNT, EXTRA>(
-            ko, blk, [&](int r, int e) { return L[lswz<NE>(rb + r, e)]; }, sync, tid, sh);
-        topk_block_last(ko, n_blocks, sync, tid, sh);
-        sync();  // the statistics scratch is reused by the next block
-      }
+      topk_tile<NE, COUNT, EXTRA>(ko, t, L, sync, tid, sh);
+      topk_tile_last(ko, t, n_blocks, sync, tid, sh);
       mbar_arrive(lfree_bar);  // stage 0 may take the next tile's data
     }
   }
@@ -528,10 +533,9 @@ cudaError_t launch_tc(const CUtensorMap& tmX, const CUtensorMap& tmW, const RPar
 template <int NE, bool COUNT, bool EXTRA>
 cudaError_t launch_fused(const CUtensorMap& tmX, const CUtensorMap& tmW, const RParams& p,
                          const TopkOut& ko, int ntiles, cudaStream_t stream) {
-  constexpr int EPL = NE >= 32 ? NE / 32 : 1;
-  auto kern = router_fused_kernel<NE, EPL, COUNT, EXTRA>;
-  constexpr int smem = 1024 + RCfg<NE>::kStages * RCfg<NE>::kStageBytes +
-                       (int)((sizeof(TopkShared<kSlice, COUNT, EXTRA>) + 15) / 16 * 16) +
+  auto kern = router_fused_kernel<NE, COUNT, EXTRA>;
+  constexpr int smem = 1024 + RCfg<NE>::kStages * RCfg<NE>::kStageBytes + fused_stage_gap<NE>() +
+                       (int)((sizeof(TileShared<COUNT, EXTRA>) + 15) / 16 * 16) +
                        RCfg<NE>::kBarBytes + 16;
   static_assert(smem <= 227 * 1024, "shared memory budget");
   static_assert(2 * RCfg<NE>::kStages + 6 <= RCfg<NE>::kBarBytes / 8, "barrier area too small");

@@ -342,25 +342,20 @@ __device__ __forceinline__ void topk_block(const TopkOut& ko, int64_t blk, Logit
   }
 }
 
-// After topk_block: the last of the n_blocks statistics blocks to finish turns the totals into
-// f, Q, aux (and the losses), or exports them (token shards).
-template <int E_MAX, bool COUNT, bool EXTRA, class Sync>
-__device__ __forceinline__ void topk_block_last(const TopkOut& ko, unsigned n_blocks, Sync sync,
-                                                int tid, TopkShared<E_MAX, COUNT, EXTRA>& sh) {
+// The last of the n_blocks statistics blocks to finish turns the totals into f, Q, aux (and the
+// losses), or exports them (token shards). The calling group has just completed `nb` blocks; it
+// finds out whether they were the last through a ticket counter.
+template <class Sync>
+__device__ __forceinline__ void topk_finish(const TopkOut& ko, unsigned nb, unsigned n_blocks,
+                                            Sync sync, int tid, int& is_last, float* prod) {
   if (ko.lb == nullptr && ko.losses == nullptr && ko.exported == nullptr) return;
   const int64_t T = ko.T;
   const int E = ko.E;
   const RouterAccum& acc = ko.acc;
-  const float alpha = ko.alpha;
-  float* lb = ko.lb;
-  float* losses = ko.losses;
   int64_t* exported = ko.exported;
-  int& is_last = sh.is_last;
-  auto& prod = sh.prod;
-    // the last block to finish turns the totals into f, Q, aux (and the losses), or exports them
   __threadfence();
   sync();
-  if (tid == 0) is_last = atomicAdd(acc.ticket, 1u) == n_blocks - 1;
+  if (tid == 0) is_last = atomicAdd(acc.ticket, nb) + nb == n_blocks;
   sync();
   if (!is_last) return;
   __threadfence();
@@ -375,11 +370,308 @@ __device__ __forceinline__ void topk_block_last(const TopkOut& ko, unsigned n_bl
     return;
   }
   router_finalize_block(
-      E, T, alpha, [&](int e) { return atomicAdd(&acc.q[e], 0ull); },
+      E, T, ko.alpha, [&](int e) { return atomicAdd(&acc.q[e], 0ull); },
       [&](int e) { return (unsigned long long)atomicAdd(&acc.c[e], 0u); },
       [&](int e) { return atomicAdd(&acc.imp[e], 0ull); },
       [&](int e) { return (unsigned long long)atomicAdd(&acc.load[e], 0u); },
-      atomicAdd(acc.z, 0ull), lb, losses, prod, tid, 256, sync);
+      atomicAdd(acc.z, 0ull), ko.lb, ko.losses, prod, tid, 256, sync);
+}
+
+// After topk_block (one statistics block).
+template <int E_MAX, bool COUNT, bool EXTRA, class Sync>
+__device__ __forceinline__ void topk_block_last(const TopkOut& ko, unsigned n_blocks, Sync sync,
+                                                int tid, TopkShared<E_MAX, COUNT, EXTRA>& sh) {
+  topk_finish(ko, 1u, n_blocks, sync, tid, sh.is_last, sh.prod);
+}
+
+// ------------------------------------------------------------------------------------------------
+// Up to 128 experts: the tile variant. A tile is 128 tokens (two statistics blocks) whose logits
+// sit in shared memory as fp32 rows of NE columns (NE = E rounded up to a power of two >= 16) with
+// a row stride of NE + 4 floats: rows stay 16-byte aligned, and a warp moving 16 bytes per lane
+// along 32 consecutive rows, or along one row, touches every bank equally often (no conflicts).
+// Token r of the tile belongs to lane r % 32 of warps r / 32 (experts [0, NE/2)) and r / 32 + 4
+// (experts [NE/2, NE)); each thread loads its half of the row into registers with 16-byte loads,
+// works on it in expert order with independent partial results, and the two halves meet through
+// shared memory. All 128 tokens of a tile are thus in flight at once.
+
+constexpr int kTileTokens = 2 * kRouterTokensPerBlock;
+constexpr int kTileExperts = 128;
+
+template <int NE>
+__device__ __forceinline__ int lpos(int row, int col) {
+  return row * (NE + 4) + col;
+}
+// Bytes of a tile's logits in shared memory.
+template <int NE>
+constexpr int tile_logits_bytes() {
+  return kTileTokens * (NE + 4) * 4;
+}
+
+// Shared memory of one tile's top-k besides the logits.
+template <bool COUNT, bool EXTRA>
+struct TileShared {
+  float part_v[2][kTileTokens];  // per half of a row: max, then the best candidate's logit
+  int part_i[2][kTileTokens];    // per half: the best candidate's expert
+  float part_s[2][kTileTokens];  // per half: the sum of exp(l - max)
+  float rs[kTileTokens];         // per token: 1 / sum of exp(l - max)
+  float qpart[2][4][kTileExperts];  // per block, row quarter and expert: partial sums of p
+  // per block and expert: first-choice count << 16 | choice count
+  unsigned cs[2][kTileExperts];
+  // gate sums per block and expert, 2^-24 fixed point (extra statistics only)
+  unsigned imp_s[EXTRA ? 2 : 1][kTileExperts];
+  float z2[EXTRA ? kTileTokens : 1];  // (log Z)^2 per token
+  int choice[kTileTokens][MOE_MAX_TOPK];  // per token: the chosen experts in choice order
+  int run[COUNT ? 2 : 1][kTileExperts];
+  int blk_ids[COUNT ? 2 : 1][COUNT ? kRouterTokensPerBlock * MOE_MAX_TOPK : 1];
+  float prod[kTileExperts];
+  int is_last;
+};
+
+// (value desc, index asc): is (v, i) ahead of (bv, bi)?
+__device__ __forceinline__ bool topk_ahead(float v, int i, float bv, int bi) {
+  return v > bv || (v == bv && i < bi);
+}
+
+// Softmax, top-k and the statistics of tile `tile` (tokens [128 tile, 128 tile + 128), statistics
+// blocks 2 tile and 2 tile + 1) by 256 threads synchronised by `sync`. L holds the tile's fp32
+// logits (rows = tokens, lpos<NE> layout); the exponentials below overwrite them. Per token: the
+// largest logit m and k rounds of (logit desc, index asc) argmax over the experts not yet taken
+// (the first round is the max pass itself); then x_e = exp(l_e - m), s = the sum of x_e (each
+// thread adds its half in expert order as four interleaved partial sums, then s = s_lo + s_hi),
+// p_e = x_e * (1 / s), gates = the chosen p (optionally renormalised over the k choices in choice
+// order: survey notes §1.1.1.1). Per block: the sums of p per expert (token order within
+// quarters of 16 tokens, then the quarters in order), the first-choice counts, and with the extra statistics the gate sums (Importance), the choice
+// counts (Load) and the sum of (log Z)^2 in token order (comparison article, "Router Z-loss");
+// all are added to the global accumulators as integers (fixed point), so the totals do not
+// depend on the order of the tiles. COUNT: also rank each block's (token, choice) pairs per
+// expert in pair order for dispatch.
+template <int NE, bool COUNT, bool EXTRA, class Sync>
+__device__ __forceinline__ void topk_tile(const TopkOut& ko, int64_t tile, float* L, Sync sync,
+                                          int tid, TileShared<COUNT, EXTRA>& sh) {
+  static_assert(NE >= 16 && NE <= kTileExperts && (NE & (NE - 1)) == 0, "expert tile");
+  constexpr int NPT = NE / 2;  // experts per thread
+  static_assert(NPT <= 64 && NPT % 4 == 0, "taken mask, 16-byte loads");
+  const int64_t T = ko.T;
+  const int E = ko.E, k = ko.k;
+  const int renorm = ko.renorm;
+  const RouterAccum& acc = ko.acc;
+  const RouterDispatchCount& dc = ko.dc;
+  const int64_t t0 = tile * kTileTokens;
+  const int ntok = (int)min((int64_t)kTileTokens, T - t0);
+  for (int i = tid; i < 2 * kTileExperts; i += 256) {
+    (&sh.cs[0][0])[i] = 0u;
+    if constexpr (EXTRA) (&sh.imp_s[0][0])[i] = 0u;
+    if constexpr (COUNT) (&sh.run[0][0])[i] = 0;
+  }
+  const int warp = tid >> 5, lane = tid & 31;
+  const int h = warp >> 2;                // half of the row
+  const int r = (warp & 3) * 32 + lane;   // token row in the tile
+  const int b = r / kRouterTokensPerBlock;
+  const bool ok = r < ntok;
+  const int e0 = h * NPT;
+  const int ne = ok ? max(0, min(NPT, E - e0)) : 0;  // experts of this half
+  float4* rowv = reinterpret_cast<float4*>(L + lpos<NE>(r, e0));
+  float v[NPT];  // this half's logits, then -inf past the last expert
+#pragma unroll
+  for (int q = 0; q < NPT / 4; ++q) {
+    const float4 f = rowv[q];
+    v[4 * q] = f.x;
+    v[4 * q + 1] = f.y;
+    v[4 * q + 2] = f.z;
+    v[4 * q + 3] = f.w;
+  }
+#pragma unroll
+  for (int i = 0; i < NPT; ++i)
+    if (i >= ne) v[i] = -INFINITY;
+  // the best (logit desc, index asc) among this half's experts not yet taken: four chains in
+  // expert order (a later equal logit never wins within a chain), merged
+  unsigned long long taken = 0ull;  // bit i: expert e0 + i already chosen
+  auto best_of_half = [&](float& bv, int& bi) {
+    float cv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+    int ci[4] = {0x7fffffff, 0x7fffffff, 0x7fffffff, 0x7fffffff};
+#pragma unroll
+    for (int i = 0; i < NPT; ++i) {
+      if (!((taken >> i) & 1ull) && v[i] > cv[i & 3]) {
+        cv[i & 3] = v[i];
+        ci[i & 3] = e0 + i;
+      }
+    }
+    bv = cv[0];
+    bi = ci[0];
+#pragma unroll
+    for (int c = 1; c < 4; ++c)
+      if (topk_ahead(cv[c], ci[c], bv, bi)) {
+        bv = cv[c];
+        bi = ci[c];
+      }
+  };
+  // one round: both halves offer their best; the winner is the same for both threads
+  auto choose = [&](int j, float& wv) {
+    float bv;
+    int bi;
+    best_of_half(bv, bi);
+    sync();  // the previous round's reads of part_v / part_i are done
+    sh.part_v[h][r] = bv;
+    sh.part_i[h][r] = bi;
+    sync();
+    const float ov = sh.part_v[h ^ 1][r];
+    const int oi = sh.part_i[h ^ 1][r];
+    const bool mine = !topk_ahead(ov, oi, bv, bi);
+    const int wi = mine ? bi : oi;
+    wv = mine ? bv : ov;
+    if (mine && bi >= e0 && bi < e0 + ne) taken |= 1ull << (bi - e0);
+    if (h == 0) sh.choice[r][j] = wi;
+  };
+  float m;  // the largest logit: the first round's winner
+  choose(0, m);
+  for (int j = 1; j < k; ++j) {
+    float wv;
+    choose(j, wv);
+  }
+  // x_e = exp(l_e - m) in place of the logits, and their sum
+  float a[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+  for (int q = 0; q < NPT / 4; ++q) {
+    float x[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int i = 4 * q + c;
+      x[c] = i < ne ? expf(v[i] - m) : 0.0f;
+      a[c] += x[c];
+    }
+    rowv[q] = make_float4(x[0], x[1], x[2], x[3]);
+  }
+  sh.part_s[h][r] = (a[0] + a[1]) + (a[2] + a[3]);
+  sync();  // the halves' sums and exponentials are in shared memory
+  const int64_t t = t0 + r;
+  if (ok && h == 0) {
+    const float s = sh.part_s[0][r] + sh.part_s[1][r];
+    const float rs = 1.0f / s;
+    sh.rs[r] = rs;
+    if constexpr (EXTRA) {
+      const float lz = m + logf(s);  // log sum_e exp(l_e)
+      sh.z2[r] = lz * lz;
+    }
+    const float* xr = L + lpos<NE>(r, 0);
+    // per-block integer counts (order-independent): first choices, and with the extra
+    // statistics every choice and its gate
+    auto count_choice = [&](int e, int j, float g) {
+      if (e < 0 || e >= E) return;
+      if constexpr (EXTRA) {
+        atomicAdd(&sh.cs[b][e], j == 0 ? 0x10001u : 1u);
+        atomicAdd(&sh.imp_s[b][e], __float2uint_rn(g * (float)kIScale));
+      } else if (j == 0) {
+        atomicAdd(&sh.cs[b][e], 0x10000u);
+      }
+    };
+    auto p_of = [&](int e) { return (e >= 0 && e < E) ? xr[e] * rs : 0.0f; };
+    float gsum = 0.0f;
+    for (int j = 0; j < k; ++j) {
+      const int e = sh.choice[r][j];
+      const float pv = p_of(e);
+      ko.ids[t * k + j] = e;
+      if (ko.probs != nullptr) ko.probs[t * k + j] = pv;  // before any renormalisation
+      if (!renorm) {
+        ko.gates[t * k + j] = pv;
+        count_choice(e, j, pv);
+      }
+      if constexpr (COUNT)
+        sh.blk_ids[b][(r - b * kRouterTokensPerBlock) * k + j] = (e >= 0 && e < E) ? e : -1;
+      gsum += pv;
+    }
+    if (renorm) {
+      for (int j = 0; j < k; ++j) {
+        const int e = sh.choice[r][j];
+        const float g = p_of(e) / gsum;
+        ko.gates[t * k + j] = g;
+        count_choice(e, j, g);
+      }
+    }
+  }
+  sync();
+  // tokens of each block present in this tile
+  const int nb0 = min(ntok, kRouterTokensPerBlock);
+  const int nb1 = max(0, ntok - kRouterTokensPerBlock);
+  if constexpr (COUNT) {
+    // rank each block's pairs per expert in pair order (warp 0: block 0, warp 4: block 1)
+    if ((warp & 3) == 0) {
+      const int bb = warp >> 2;
+      const int npairs = (bb == 0 ? nb0 : nb1) * k;
+      const int64_t pair0 = (t0 + bb * kRouterTokensPerBlock) * k;
+      const unsigned lt = (1u << lane) - 1u;
+      for (int c = 0; c < npairs; c += 32) {
+        const int pl = c + lane;
+        const int e = pl < npairs ? sh.blk_ids[bb][pl] : -1;
+        const unsigned same = __match_any_sync(0xffffffffu, e);
+        const int rank = __popc(same & lt);
+        const int base = e >= 0 ? sh.run[bb][e] : 0;
+        __syncwarp();
+        if (e >= 0 && rank == 0) sh.run[bb][e] = base + __popc(same);
+        __syncwarp();
+        if (pl < npairs) dc.local_rank[pair0 + pl] = e >= 0 ? base + rank : -1;
+      }
+    }
+  }
+  // per block and expert: the sum of p over the block's tokens. Thread (block, quarter, quad)
+  // adds rows [16 quarter, 16 quarter + 16) of its block in token order for experts
+  // [4 quad, 4 quad + 4); the quarters' sums are then added in quarter order.
+  {
+    const int bb = tid >> 7, quarter = (tid >> 5) & 3, quad = tid & 31;
+    const int n = bb == 0 ? nb0 : nb1;
+    const int row0 = bb * kRouterTokensPerBlock + quarter * 16;
+    const int nr = min(16, max(0, n - quarter * 16));
+    if (4 * quad < NE) {
+      float q[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      for (int u = 0; u < nr; ++u) {
+        const float4 f = *reinterpret_cast<const float4*>(L + lpos<NE>(row0 + u, 4 * quad));
+        const float rs = sh.rs[row0 + u];
+        q[0] += f.x * rs;
+        q[1] += f.y * rs;
+        q[2] += f.z * rs;
+        q[3] += f.w * rs;
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) sh.qpart[bb][quarter][4 * quad + c] = q[c];
+    }
+  }
+  sync();
+  {
+    const int bb = tid >> 7, e = tid & (kTileExperts - 1);
+    const int n = bb == 0 ? nb0 : nb1;
+    if (n > 0 && e < E) {
+      const float sum = ((sh.qpart[bb][0][e] + sh.qpart[bb][1][e]) + sh.qpart[bb][2][e]) +
+                        sh.qpart[bb][3][e];
+      const unsigned long long fx = (unsigned long long)llrint((double)sum * kQScale);
+      if (fx) atomicAdd(&acc.q[e], fx);
+      const unsigned cs = sh.cs[bb][e];
+      if (cs >> 16) atomicAdd(&acc.c[e], cs >> 16);
+      if constexpr (EXTRA) {
+        if (cs & 0xffffu) atomicAdd(&acc.load[e], cs & 0xffffu);
+        if (sh.imp_s[bb][e]) atomicAdd(&acc.imp[e], (unsigned long long)sh.imp_s[bb][e]);
+      }
+    }
+    if (EXTRA && n > 0 && e == 0) {
+      float zb = 0.0f;
+      for (int u = 0; u < n; ++u) zb += sh.z2[bb * kRouterTokensPerBlock + u];
+      atomicAdd(acc.z, (unsigned long long)llrint((double)zb * kZScale));
+    }
+  }
+  if constexpr (COUNT) {
+    const int64_t blk0 = tile * 2;
+    for (int i = tid; i < 2 * E; i += 256) {
+      const int bb = i / E, e = i - bb * E;
+      if ((bb == 0 ? nb0 : nb1) > 0) dc.seg_counts[(blk0 + bb) * E + e] = sh.run[bb][e];
+    }
+  }
+}
+
+// After topk_tile: the tile completed one or two statistics blocks.
+template <bool COUNT, bool EXTRA, class Sync>
+__device__ __forceinline__ void topk_tile_last(const TopkOut& ko, int64_t tile, unsigned n_blocks,
+                                               Sync sync, int tid, TileShared<COUNT, EXTRA>& sh) {
+  const int64_t t0 = tile * kTileTokens;
+  const unsigned nb = ko.T - t0 > kRouterTokensPerBlock ? 2u : 1u;
+  topk_finish(ko, nb, n_blocks, sync, tid, sh.is_last, sh.prod);
 }
 
 }  // namespace
