@@ -355,9 +355,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         tma_prefetch_l2_2d(&tmW, (b / n_kb) * p.dpad + (b % n_kb) * kBK, 0);
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++n_local) {
         bool waited = n_local == 0;  // this CTA's first tile: stage 0 holds no logits yet
-        // the tile's x rows, read from HBM once, requested into L2 at once: the stage ring alone
-        // keeps too few bytes in flight to hide DRAM latency (the weight parts are L2 hits)
-        for (int kb = 0; kb < n_kb; ++kb) tma_prefetch_l2_2d(&tmX, kb * kBK, t * kTM);
         for (int kb = 0; kb < n_kb; ++kb) {
           if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, p.status)) {
             ok = false;
@@ -378,6 +375,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
           for (int part = 0; part < 3; ++part)
             tma_load_2d(sa + C::kABytes + part * C::kBPartBytes, &tmW, part * p.dpad + kb * kBK, 0,
                         full_bar(stage));
+          // once the ring is full, the rest of the tile's x rows (read from HBM once) are asked
+          // into L2 at once: the ring alone keeps too few bytes in flight to hide DRAM latency
+          // (the weight parts are L2 hits); asking first would delay the ring's first loads
+          if (kb == min(S, n_kb) - 1)
+            for (int kq = kb + 1; kq < n_kb; ++kq) tma_prefetch_l2_2d(&tmX, kq * kBK, t * kTM);
           ++issued;
           if (++stage == S) {
             stage = 0;

@@ -528,15 +528,15 @@ __device__ __forceinline__ void topk_tile(const TopkOut& ko, int64_t tile, float
     float wv;
     choose(j, wv);
   }
-  // x_e = exp(l_e - m) in place of the logits, and their sum
+  // x_e = exp(l_e - m) in place of the logits, and their sum (past the last expert v = -inf, so
+  // x = 0 there without a branch; rows past the tile's tokens are never read back)
   float a[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
   for (int q = 0; q < NPT / 4; ++q) {
     float x[4];
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-      const int i = 4 * q + c;
-      x[c] = i < ne ? expf(v[i] - m) : 0.0f;
+      x[c] = expf(v[4 * q + c] - m);
       a[c] += x[c];
     }
     rowv[q] = make_float4(x[0], x[1], x[2], x[3]);
