@@ -42,6 +42,11 @@ bool coschedule_enabled() {
   return !(v != nullptr && v[0] == '0');
 }
 
+bool pair_mma_enabled() {
+  const char* v = std::getenv("MOE_PAIR_MMA");
+  return !(v != nullptr && v[0] == '0');
+}
+
 int num_sms() {
   static int cache[64] = {0};
   int dev = 0;

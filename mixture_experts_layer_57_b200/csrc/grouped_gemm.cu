@@ -814,6 +814,247 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+
+// Tiles on CTA pairs (cta_group::2). A cluster of two CTAs takes each tile together with MMAs of
+// M = 256: each CTA holds 128 of the 256 output features of an MMA (its A half) and half of the
+// tile's tokens (its B half), so each SM loads half of the token operand instead of all of it:
+// for a tile of 256 features x 256 tokens a CTA loads 32 KB per K step (one 128-row weight box
+// and 128 token rows), against 48 KB for the same tensor work per SM with one CTA per tile. This
+// pays where the tensor pipe is the bound (wide expert tiles of a compute-bound layer, the PR-MoE
+// dense MLP); where the expert weights stream from HBM the two SMs in lockstep wait for the
+// slower copy of every stage, and one CTA per tile is faster (measured). Problem 0 is the expert
+// GEMM (tiles of NB0 x 256 features x BN0 tokens: NB0 MMAs of M = 256 per K step, NB0 weight
+// boxes and BN0 / 2 token rows per CTA and stage), problem 1 an optional dense GEMM (256 x 256
+// tiles), interleaved as in co_gemm_kernel. Protocol per stage: both CTAs' producers wait their
+// own empty barrier and load their halves; the loads count on the leader's full barrier, whose
+// expected bytes the leader's producer sets for both; the leader's MMA warp waits it, issues the
+// MMAs (K = 16 each) and commits to the empty barrier of both CTAs. Per tile: the leader commits
+// to both CTAs' accumulator-full barriers; both CTAs' epilogues read their 128 TMEM lanes and
+// arrive on the leader's accumulator-empty barrier (2 x 256 arrivals). Waits stay bounded; both
+// CTAs meet at a cluster barrier after set-up and before freeing TMEM and exiting.
+constexpr int kPairBN1 = 256;  // dense tile tokens (128 per CTA)
+constexpr int kPairAccCols = 256;
+template <int BN0, int NB0, int STAGE_BYTES, int STAGES>
+struct PairCfg {
+  static constexpr int kSmemBytes =
+      1024 + STAGES * STAGE_BYTES + kEpiWarps * kStageTileBytes + Cfg<128, 1>::kAuxBytes;
+  static_assert(kBM * kBK * 2 + (kPairBN1 / 2) * kBK * 2 <= STAGE_BYTES, "dense pair stage");
+  static_assert(NB0 * kBM * kBK * 2 + (BN0 / 2) * kBK * 2 <= STAGE_BYTES, "expert pair stage");
+  static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+  static_assert(NB0 * BN0 <= kPairAccCols, "expert accumulators per buffer");
+  static_assert(2 * STAGES + 5 <= 64, "barrier area too small");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+};
+
+template <int EPI, int BN0, int NB0, int STAGE_BYTES, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+    co_pair_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__ CUtensorMap tmX0,
+                   const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmX1,
+                   const Params p0, const Params p1) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t base_addr = (raw_addr + 1023u) & ~1023u;
+  uint8_t* base = smem_raw + (base_addr - raw_addr);
+  uint8_t* stage_tiles = base + STAGES * STAGE_BYTES;
+  uint8_t* aux = stage_tiles + kEpiWarps * kStageTileBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(aux);
+  constexpr int kBarBytes = Cfg<128, 1>::kBarBytes;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(aux + kBarBytes);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(aux + kBarBytes + 4);
+  int* prefix = reinterpret_cast<int*>(aux + kBarBytes + 16);
+  int* seg = prefix + (MOE_MAX_EXPERTS + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int S = STAGES;
+  const Bars B{smem_u32(bars), S};
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = (int)(blockIdx.x >> 1), n_pairs = (int)(gridDim.x >> 1);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(B.full(s), 1);
+      mbar_init(B.empty(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(B.tfull(a), 1);
+      mbar_init(B.tempty(a), 2 * kEpiWarps * 32);
+    }
+    mbar_init(B.drain(), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  pdl_wait();
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&tmW0);
+    tma_prefetch_desc(&tmX0);
+    tma_prefetch_desc(&tmW1);
+    tma_prefetch_desc(&tmX1);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_holder), 2 * kPairAccCols);
+    tmem_relinquish_pair();
+  }
+  const int nft0 = (p0.n_out + NB0 * 2 * kBM - 1) / (NB0 * 2 * kBM);  // expert tiles
+  const int nft1 = (p1.n_out + 2 * kBM - 1) / (2 * kBM);  // dense tiles of 256 features
+  if (warp == 2) build_tile_list<BN0>(p0, nft0, prefix, seg, lane);
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync();  // barriers initialised and TMEM allocated in both CTAs
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const int n0 = prefix[p0.E];
+  const int n1 = nft1 * (int)((p1.rows_max + kPairBN1 - 1) / kPairBN1);
+  const int total = n0 + n1;
+  const int nkb0 = (p0.K + kBK - 1) / kBK;
+  const int nkb1 = (p1.K + kBK - 1) / kBK;
+  auto which = [&](int t, int& local) -> int {
+    const int c = (int)(((int64_t)t * n0) / total);
+    const int c1 = (int)(((int64_t)(t + 1) * n0) / total);
+    if (c1 > c) {
+      local = c;
+      return 0;
+    }
+    local = t - c;
+    return 1;
+  };
+  constexpr uint32_t kBox = kBM * kBK * 2;  // one 128-row weight box
+  // stage layout per CTA: weight boxes at 0 (and kBox), this CTA's token rows after them
+
+  if (warp == 0) {
+    if (lane == 0) {
+      Ring ring;
+      int issued = 0;
+      bool ok = true;
+      for (int t = pair; t < total && ok; t += n_pairs) {
+        int u;
+        const int prob = which(t, u);
+        const Tile tl = prob == 0 ? decode_tile<BN0, 2 * NB0>(u, prefix, seg, p0.E, nft0)
+                                  : decode_dense_tile<kPairBN1, 2>(u, p1.rows_max, nft1, p1.K);
+        const Params& p = prob == 0 ? p0 : p1;
+        const CUtensorMap* tmW = prob == 0 ? &tmW0 : &tmW1;
+        const CUtensorMap* tmX = prob == 0 ? &tmX0 : &tmX1;
+        const int n_box = prob == 0 ? NB0 : 1;  // weight boxes per CTA and stage
+        const int half_rows = (prob == 0 ? BN0 : kPairBN1) / 2;
+        const uint32_t x_off = (uint32_t)n_box * kBox;
+        const uint32_t tx = 2u * (x_off + (uint32_t)half_rows * kBK * 2);
+        // MMA i of the tile covers features [f0 + 256 i, f0 + 256 i + 256); this CTA holds its
+        // rows 128 rank ..
+        const int w_row = tl.e * p.n_out + tl.f0 + (int)rank * kBM;
+        const int x_row = tl.row0 + (int)rank * half_rows;
+        const int nkb = prob == 0 ? nkb0 : nkb1;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait_bounded(B.empty(ring.stage), ring.phase ^ 1u, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sa = base_addr + ring.stage * STAGE_BYTES;
+          const uint32_t full_leader = cluster_addr(B.full(ring.stage), 0);
+          if (leader) mbar_arrive_expect_tx(B.full(ring.stage), tx);
+          for (int i = 0; i < n_box; ++i)
+            tma_load_2d_pair(sa + i * kBox, tmW, kb * kBK, w_row + i * 2 * kBM, full_leader);
+          tma_load_2d_pair(sa + x_off, tmX, kb * kBK, x_row, full_leader);
+          ++issued;
+          ring.next(S);
+        }
+      }
+      // the leader's full barriers count both CTAs' copies: it waits for the last ones; the
+      // other CTA stays resident until then (cluster barrier below)
+      if (leader)
+        for (int i = max(0, issued - S); i < issued; ++i)
+          mbar_wait_drain(B.full(i % S), (uint32_t)((i / S) & 1), p0.status);
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      Ring ring;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int t = pair; t < total && ok; t += n_pairs) {
+        if (!mbar_wait_bounded(B.tempty(acc), acc_phase ^ 1u, abort_flag, p0.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kPairAccCols);
+        int u;
+        const int prob = which(t, u);
+        const int nkb = prob == 0 ? nkb0 : nkb1;
+        const int n_box = prob == 0 ? NB0 : 1;
+        const int n_tok = prob == 0 ? BN0 : kPairBN1;
+        const uint32_t idesc = idesc_bf16_f32(2 * kBM, n_tok);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait_bounded(B.full(ring.stage), ring.phase, abort_flag, p0.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = base_addr + ring.stage * STAGE_BYTES;
+          const uint64_t bdesc = smem_desc_sw128(sa + (uint32_t)n_box * kBox);
+          for (int i = 0; i < n_box; ++i) {
+            const uint64_t adesc = smem_desc_sw128(sa + i * kBox);
+#pragma unroll
+            for (int kk = 0; kk < kBK / kUmmaK; ++kk)
+              tc_mma_bf16_pair(d_tmem + (uint32_t)(i * n_tok), adesc + (uint64_t)(2 * kk),
+                               bdesc + (uint64_t)(2 * kk), idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          tc_commit_pair_both(B.empty(ring.stage));
+          ring.next(S);
+        }
+        if (!ok) break;
+        tc_commit_pair_both(B.tfull(acc));
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      tc_commit_pair_local(B.drain());
+      mbar_wait_drain(B.drain(), 0, p0.status);
+    }
+  } else {
+    const int ew = warp - 2;
+    const int quarter = warp & 3;
+    const int half = ew >> 2;
+    uint8_t* st = stage_tiles + ew * kStageTileBytes;
+    const uint32_t tempty0 = cluster_addr(B.tempty(0), 0), tempty1 = cluster_addr(B.tempty(1), 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = pair; t < total; t += n_pairs) {
+      if (!mbar_wait_bounded_warp(B.tfull(acc), acc_phase, abort_flag, p0.status)) break;
+      tc_fence_after();
+      const uint32_t acc_tmem = tmem_base + (uint32_t)(acc * kPairAccCols);
+      int u;
+      if (which(t, u) == 0) {
+        const Tile t4 = decode_tile<BN0, 2 * NB0>(u, prefix, seg, p0.E, nft0);
+#pragma unroll 1
+        for (int i = 0; i < NB0; ++i) {
+          Tile tl = t4;
+          tl.f0 += i * 2 * kBM + (int)rank * kBM;
+          epilogue_tile<BN0, 1, EPI>(tl, p0, acc_tmem + (uint32_t)(i * BN0), quarter,
+                                          half, lane, st);
+        }
+      } else {
+        Tile tl = decode_dense_tile<kPairBN1, 2>(u, p1.rows_max, nft1, p1.K);
+        tl.f0 += (int)rank * kBM;
+        epilogue_tile<kPairBN1, 1, EPI>(tl, p1, acc_tmem, quarter, half, lane, st);
+      }
+      tc_fence_before();
+      mbar_arrive_cluster(acc == 0 ? tempty0 : tempty1);  // the leader's barrier
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync();  // no copy, commit or arrive targets either CTA after this
+  pdl_trigger();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, 2 * kPairAccCols);
+  }
+}
+
 // ---------------------------------------------------------------- host side
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -881,6 +1122,43 @@ cudaError_t launch_co(const CUtensorMap& tmW0, const CUtensorMap& tmX0, const CU
   if (e != cudaSuccess) return e;
   return launch_kernel(kern, dim3(num_sms()), dim3(kThreads), kCoSmemBytes, stream, tmW0, tmX0,
                        tmW1, tmX1, p0, p1);
+}
+
+// Launch as clusters of two CTAs (co_pair_kernel), with programmatic dependent launch.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pair(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                        cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
+  count_launch();
+  return e;
+}
+
+template <int EPI, int BN0, int NB0, int STAGE_BYTES, int STAGES>
+cudaError_t launch_co_pair(const CUtensorMap& tmW0, const CUtensorMap& tmX0,
+                           const CUtensorMap& tmW1, const CUtensorMap& tmX1, const Params& p0,
+                           const Params& p1, cudaStream_t stream) {
+  auto kern = co_pair_kernel<EPI, BN0, NB0, STAGE_BYTES, STAGES>;
+  constexpr int smem = PairCfg<BN0, NB0, STAGE_BYTES, STAGES>::kSmemBytes;
+  static int attr_done[64] = {0};  // per instantiation and device
+  cudaError_t e = ensure_dynamic_smem(kern, smem, attr_done);
+  if (e != cudaSuccess) return e;
+  const int grid = num_sms() & ~1;
+  return launch_pair(kern, dim3(grid), dim3(kThreads), smem, stream, tmW0, tmX0, tmW1, tmX1, p0,
+                     p1);
 }
 
 }  // namespace
@@ -954,6 +1232,17 @@ cudaError_t enqueue_grouped_gemm_bf16(const void* x, const int32_t* offsets, int
   if (!make_kmajor_map(&tmW, w, (int64_t)E * N, K, kBM) || !make_kmajor_map(&tmX, x, rows_max, K, BN))
     return cudaErrorInvalidValue;
   Params p{offsets, E, N, K, rows_max, bias, out, status, CombineArgs{}, nullptr, nullptr};
+  if (BN == 256 && pair_mma_enabled() && num_sms() >= 2) {
+    // wide (compute-bound) expert tiles on CTA pairs: 256 features x 256 tokens, 128 token rows
+    // per CTA; no second problem (its maps point at this one's operands and it has no tiles)
+    CUtensorMap tmXh;
+    if (!make_kmajor_map(&tmXh, x, rows_max, K, 128)) return cudaErrorInvalidValue;
+    Params none{nullptr, 1, N, K, 0, nullptr, nullptr, status, CombineArgs{}, nullptr, nullptr};
+    return gelu ? launch_co_pair<kEpiGeluBf16, 256, 1, 32 * 1024, 6>(tmW, tmXh, tmW, tmXh, p, none,
+                                                                     stream)
+                : launch_co_pair<kEpiF32, 256, 1, 32 * 1024, 6>(tmW, tmXh, tmW, tmXh, p, none,
+                                                                stream);
+  }
   return gelu ? launch_bn<kEpiGeluBf16>(BN, tmW, tmX, p, stream, capacity_hint)
               : launch_bn<kEpiF32>(BN, tmW, tmX, p, stream, capacity_hint);
 }

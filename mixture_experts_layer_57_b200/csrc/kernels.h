@@ -20,6 +20,9 @@ int num_sms();
 bool pdl_enabled();
 // Whether bf16 PR-MoE layers co-schedule expert and dense GEMM layers (MOE_COSCHEDULE=0: no).
 bool coschedule_enabled();
+// Wide (256-token) expert GEMM tiles on CTA pairs (cta_group::2 MMAs); MOE_PAIR_MMA=0 keeps one
+// CTA per tile. Read at every call.
+bool pair_mma_enabled();
 
 // Launches kern<<<grid, block, smem, stream>>>(args...) as a programmatic dependent launch and
 // counts it.
