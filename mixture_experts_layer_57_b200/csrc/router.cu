@@ -114,6 +114,66 @@ __global__ void __launch_bounds__(256) router_gemv_kernel(const void* __restrict
     }
   }
   const float* wr = w + (int64_t)e * d;
+  if constexpr (XBF16) {
+    if ((d & 7) == 0) {
+      // Each lane owns elements lane*8 + 256 j (j = 0, 1, ...) of the weight row; a warp takes
+      // tokens warp, warp + 8, ... four at a time. Per chunk of four j, the lane's weights and the
+      // four tokens' x values are all requested before the first FMA (24 independent 16/32-byte
+      // loads in flight instead of one round trip per j). Every sum adds its products in the
+      // same order as one token at a time would (j ascending, 8 elements each), then the same
+      // warp reduction.
+      const uint16_t* xb = reinterpret_cast<const uint16_t*>(x);
+      for (int64_t t0 = warp; t0 < T; t0 += 32) {
+        float s[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        for (int j0 = 0; j0 < d; j0 += 1024) {
+          float4 wv[8];
+          uint4 xv[4][4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int i = j0 + 256 * q + lane * 8;
+            const bool in = i < d;
+            wv[2 * q] = in ? *reinterpret_cast<const float4*>(wr + i) : make_float4(0, 0, 0, 0);
+            wv[2 * q + 1] = in ? *reinterpret_cast<const float4*>(wr + i + 4) : make_float4(0, 0, 0, 0);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int64_t t = t0 + 8 * u;
+              xv[u][q] = (in && t < T) ? *reinterpret_cast<const uint4*>(xb + t * d + i)
+                                       : make_uint4(0, 0, 0, 0);
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              if (j0 + 256 * q + lane * 8 >= d) continue;
+              const uint4 xq = xv[u][q];
+              const float4 w0 = wv[2 * q], w1 = wv[2 * q + 1];
+              float a = s[u];
+              a = fmaf(__uint_as_float(xq.x << 16), w0.x, a);
+              a = fmaf(__uint_as_float(xq.x & 0xffff0000u), w0.y, a);
+              a = fmaf(__uint_as_float(xq.y << 16), w0.z, a);
+              a = fmaf(__uint_as_float(xq.y & 0xffff0000u), w0.w, a);
+              a = fmaf(__uint_as_float(xq.z << 16), w1.x, a);
+              a = fmaf(__uint_as_float(xq.z & 0xffff0000u), w1.y, a);
+              a = fmaf(__uint_as_float(xq.w << 16), w1.z, a);
+              a = fmaf(__uint_as_float(xq.w & 0xffff0000u), w1.w, a);
+              s[u] = a;
+            }
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          float v = s[u];
+#pragma unroll
+          for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+          const int64_t t = t0 + 8 * u;
+          if (lane == 0 && t < T) logits[t * E + e] = v + (bias ? bias[e] : 0.0f);
+        }
+      }
+      pdl_trigger();
+      return;
+    }
+  }
   for (int64_t t = warp; t < T; t += 8) {
     float s = 0.0f;
     if constexpr (XBF16) {
