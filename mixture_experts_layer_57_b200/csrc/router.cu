@@ -88,9 +88,9 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const void* __restri
   pdl_trigger();
 }
 
-// Decode-sized batches (T <= kRouterGemvMaxT): one block per expert, warp per token, lanes over
-// K with 16-byte loads, fp32 FMA, fixed-order warp reduction; block 0 also zeroes the statistics
-// accumulators (this kernel then replaces the prep kernel).
+// Decode-sized batches (T <= kRouterGemvMaxT): one block per expert, a warp per token (four at a
+// time), lanes over K with 16-byte loads, fp32 FMA, fixed-order warp reduction; block 0 also
+// zeroes the statistics accumulators (this kernel then replaces the prep kernel).
 template <bool XBF16>
 __global__ void __launch_bounds__(256) router_gemv_kernel(const void* __restrict__ x,
                                                           const float* __restrict__ w,
