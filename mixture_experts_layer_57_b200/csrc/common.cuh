@@ -310,7 +310,7 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
                : "memory");
 }
 // 2D tiled load into this CTA's shared memory whose completion counts on `cluster_bar`, an
-// mbarrier of either CTA of the pair (no multicast: the box lands in this CTA only).
+// mbarrier of either CTA of the pair (the box lands in this CTA's shared memory only).
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void* tmap, int32_t x,
                                                  int32_t y, uint32_t cluster_bar) {
   asm volatile(
@@ -342,20 +342,18 @@ __device__ __forceinline__ void tc_mma_bf16_pair(uint32_t d_tmem, uint64_t a_des
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-// Arrive once on the mbarrier at offset `bar` in both CTAs of the pair when the leader's earlier
-// MMAs have completed (a completion signal, not a data copy).
-__device__ __forceinline__ void tc_commit_pair_both(uint32_t bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
-      " [%0], %1;" ::"r"(bar),
-      "h"((unsigned short)0x3)
-      : "memory");
-}
-// The same, on this CTA's mbarrier only.
+// Arrive once on the mbarrier `bar` (a shared::cluster address: this CTA's or the peer's) when
+// the leader's earlier MMAs have completed.
 __device__ __forceinline__ void tc_commit_pair_local(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                    bar)
                : "memory");
+}
+// The same on the mbarrier at offset `bar` in both CTAs of the pair: one commit to this CTA's
+// barrier and one to the peer's (its cluster address).
+__device__ __forceinline__ void tc_commit_pair_both(uint32_t bar, uint32_t peer_bar) {
+  tc_commit_pair_local(bar);
+  tc_commit_pair_local(peer_bar);
 }
 
 // ---------------------------------------------------------------- programmatic dependent launch

@@ -1003,11 +1003,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               tc_mma_bf16_pair(d_tmem + (uint32_t)(i * n_tok), adesc + (uint64_t)(2 * kk),
                                bdesc + (uint64_t)(2 * kk), idesc, (kb | kk) != 0 ? 1u : 0u);
           }
-          tc_commit_pair_both(B.empty(ring.stage));
+          tc_commit_pair_both(B.empty(ring.stage), cluster_addr(B.empty(ring.stage), 1));
           ring.next(S);
         }
         if (!ok) break;
-        tc_commit_pair_both(B.tfull(acc));
+        tc_commit_pair_both(B.tfull(acc), cluster_addr(B.tfull(acc), 1));
         if (++acc == 2) {
           acc = 0;
           acc_phase ^= 1u;
