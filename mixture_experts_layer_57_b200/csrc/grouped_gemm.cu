@@ -916,6 +916,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int total = n0 + n1;
   const int nkb0 = (p0.K + kBK - 1) / kBK;
   const int nkb1 = (p1.K + kBK - 1) / kBK;
+  // problem 0's tile u: (expert, feature tile, token tile) order, or for one segment (the dense
+  // MLP run alone) the grouped order of decode_dense_tile
+  auto tile0 = [&](int u) -> Tile {
+    return p0.offsets != nullptr ? decode_tile<BN0, 2 * NB0>(u, prefix, seg, p0.E, nft0)
+                                 : decode_dense_tile<BN0, 2 * NB0>(u, p0.rows_max, nft0, p0.K);
+  };
   auto which = [&](int t, int& local) -> int {
     const int c = (int)(((int64_t)t * n0) / total);
     const int c1 = (int)(((int64_t)(t + 1) * n0) / total);
@@ -937,7 +943,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = pair; t < total && ok; t += n_pairs) {
         int u;
         const int prob = which(t, u);
-        const Tile tl = prob == 0 ? decode_tile<BN0, 2 * NB0>(u, prefix, seg, p0.E, nft0)
+        const Tile tl = prob == 0 ? tile0(u)
                                   : decode_dense_tile<kPairBN1, 2>(u, p1.rows_max, nft1, p1.K);
         const Params& p = prob == 0 ? p0 : p1;
         const CUtensorMap* tmW = prob == 0 ? &tmW0 : &tmW1;
@@ -1030,7 +1036,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t acc_tmem = tmem_base + (uint32_t)(acc * kPairAccCols);
       int u;
       if (which(t, u) == 0) {
-        const Tile t4 = decode_tile<BN0, 2 * NB0>(u, prefix, seg, p0.E, nft0);
+        const Tile t4 = tile0(u);
 #pragma unroll 1
         for (int i = 0; i < NB0; ++i) {
           Tile tl = t4;
