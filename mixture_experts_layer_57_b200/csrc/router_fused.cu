@@ -280,6 +280,48 @@ constexpr int fused_stage_gap() {
   return over <= 0 ? 0 : (over + 1023) / 1024 * 1024;
 }
 
+// Epilogue helpers of the fused kernels. One warp copies its 32 TMEM lanes (tokens `row`) of the
+// accumulator at taddr, 16-expert chunks half, half + 2, ..., plus the bias, into the tile's
+// logits rows in shared memory (16-byte stores).
+template <int NE>
+__device__ __forceinline__ void router_acc_to_smem(uint32_t taddr, int row, int half,
+                                                   const RParams& p, float* L) {
+  for (int c0 = half * 16; c0 < NE; c0 += 32) {
+    uint32_t r[16];
+    tmem_ld_32x32b_x16(taddr + (uint32_t)c0, r);
+    tmem_ld_wait();
+    float4* dst = reinterpret_cast<float4*>(L + lpos<NE>(row, c0));
+#pragma unroll
+    for (int c = 0; c < 16; c += 4) {
+      float f[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = c0 + c + u;
+        f[u] = __uint_as_float(r[c + u]) + ((p.bias && e < p.E) ? p.bias[e] : 0.0f);
+      }
+      dst[c / 4] = make_float4(f[0], f[1], f[2], f[3]);
+    }
+  }
+}
+// The tile's logits output (when asked for) and its top-k, by the 256 epilogue threads.
+template <int NE, bool COUNT, bool EXTRA>
+__device__ __forceinline__ void router_tile_outputs(const RParams& p, const TopkOut& ko,
+                                                    int64_t tile, float* L, NamedSync sync,
+                                                    int tid, TileShared<COUNT, EXTRA>& sh,
+                                                    unsigned n_blocks) {
+  const int64_t t0 = tile * kTM;
+  if (p.logits != nullptr) {
+    // whole rows: thread i writes experts i, i + 256, ... of the tile, row-major
+    const int ne = p.E;
+    for (int i = tid; i < kTM * ne; i += 256) {
+      const int rr = i / ne, e = i - rr * ne;
+      if (t0 + rr < p.T) p.logits[(t0 + rr) * ne + e] = L[lpos<NE>(rr, e)];
+    }
+  }
+  topk_tile<NE, COUNT, EXTRA>(ko, tile, L, sync, tid, sh);
+  topk_tile_last(ko, tile, n_blocks, sync, tid, sh);
+}
+
 template <int NE, bool COUNT, bool EXTRA>
 __global__ void __launch_bounds__(kFusedThreads, 1)
     router_fused_kernel(const __grid_constant__ CUtensorMap tmX,
@@ -448,23 +490,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
       if (named_barrier_any(1, 256, !ok)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * NE);
-      const int row = quarter * 32 + lane;  // token within the tile
-      for (int c0 = half * 16; c0 < NE; c0 += 32) {
-        uint32_t r[16];
-        tmem_ld_32x32b_x16(taddr + (uint32_t)c0, r);
-        tmem_ld_wait();
-        float4* dst = reinterpret_cast<float4*>(L + lpos<NE>(row, c0));
-#pragma unroll
-        for (int c = 0; c < 16; c += 4) {
-          float f[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int e = c0 + c + u;
-            f[u] = __uint_as_float(r[c + u]) + ((p.bias && e < p.E) ? p.bias[e] : 0.0f);
-          }
-          dst[c / 4] = make_float4(f[0], f[1], f[2], f[3]);
-        }
-      }
+      router_acc_to_smem<NE>(taddr, quarter * 32 + lane, half, p, L);
       tc_fence_before();
       mbar_arrive(tempty_bar(acc));  // the accumulator is free for the tile after next
       if (++acc == 2) {
@@ -472,17 +498,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         acc_phase ^= 1u;
       }
       sync();
-      const int64_t t0 = (int64_t)t * kTM;
-      if (p.logits != nullptr) {
-        // whole rows: thread i writes experts i, i + 256, ... of the tile, row-major
-        const int ne = p.E;
-        for (int i = tid; i < kTM * ne; i += 256) {
-          const int rr = i / ne, e = i - rr * ne;
-          if (t0 + rr < p.T) p.logits[(t0 + rr) * ne + e] = L[lpos<NE>(rr, e)];
-        }
-      }
-      topk_tile<NE, COUNT, EXTRA>(ko, t, L, sync, tid, sh);
-      topk_tile_last(ko, t, n_blocks, sync, tid, sh);
+      router_tile_outputs<NE, COUNT, EXTRA>(p, ko, t, L, sync, tid, sh, n_blocks);
       mbar_arrive(lfree_bar);  // stage 0 may take the next tile's data
     }
   }
@@ -495,6 +511,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     tmem_dealloc(tmem_base, C::kTmemCols);
   }
 }
+
+
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
