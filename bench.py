@@ -7,7 +7,7 @@ the workload's T tokens of seeded synthetic input already resident in HBM. The d
 is the largest one that the metric's configurations list: the GPT-1.3B+MoE-128 PR-MoE layer
 (T=16384, d=2048, d_ff=8192, E=128, top-1, fixed dense MLP). The other workloads (top-2 E=8,
 decode, GPT-350M+MoE-128) are measured in the same process as `per_workload` entries, each stage
-against its roofline, and `north_star_bars` collects the target fractions. L2 is flushed (256 MiB write) between
+against its roofline, and `target_bars` collects the target fractions. L2 is flushed (256 MiB write) between
 timed steps; each step is timed with CUDA events on the launching stream; the K-step region is
 bracketed by a barrier and device synchronisation on both sides; the max over ranks is taken.
 N > 1 (under torchrun) runs N independent replicas, one per GPU: the layer has no exchange step
@@ -571,8 +571,8 @@ def main():
                                                    warmup=max(3, min(args.warmup, 5)))
     entries = dict(per_workload)
     entries[w.name] = own
-    # the benchmark spec's bars: >= 60% of dense bf16 tensor peak on the prefill GEMMs that are
-    # compute-bound (top-2 experts, PR-MoE dense MLP), >= 70% of HBM bandwidth on decode
+    # the layer's performance targets: >= 60% of dense bf16 tensor peak on the prefill GEMMs that
+    # are compute-bound (top-2 experts, PR-MoE dense MLP), >= 70% of HBM bandwidth on decode
     if "top2-e8-zipf" in entries and entries["top2-e8-zipf"]["experts"]:
         bars["top2-e8-zipf experts tensor_frac (>= 0.60)"] = entries["top2-e8-zipf"]["experts"]["tensor_frac"]
     if "gpt1.3b-prmoe128" in entries and entries["gpt1.3b-prmoe128"]["dense_mlp"]:
@@ -621,7 +621,7 @@ def main():
             "config": workload_config(w, args.gpus), "roofline": roof, "cpu_baseline": cpu,
             "clocks": clocks.summary(), "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps,
-            "breakdown_ms": bd, "routing": routing, "north_star_bars": bars,
+            "breakdown_ms": bd, "routing": routing, "target_bars": bars,
             "headline_groups": own,
             "per_workload": per_workload, "priority_dispatch_collapse": prio_collapse,
             "train_step": train,
