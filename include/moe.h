@@ -35,6 +35,14 @@
  *   - Environment variable MOE_FAULT_INJECT=<entry point name> makes that entry point
  *     return MOE_ERR_CUDA without enqueueing anything (host-side fault injection for
  *     callers' error paths).
+ *   - Performance switches, all on by default and all bit-identical in their results
+ *     (set to 0 to turn one off, for A/B timing): MOE_PDL (programmatic dependent launch
+ *     between the layer's kernels; read once per process), MOE_FUSED_ROUTER (softmax,
+ *     top-k and the statistics in the tensor-core router's epilogue), MOE_COSCHEDULE (a
+ *     PR-MoE layer's expert and dense GEMM layers share one launch), MOE_PAIR_MMA (expert
+ *     GEMMs with 256-column tiles run as two-SM CTA pairs), MOE_W_EVICT_FIRST (the L2
+ *     evict-first hint on expert weights read once per layer). All but MOE_PDL are read at
+ *     every call.
  */
 #ifndef MOE_H_
 #define MOE_H_

@@ -42,6 +42,8 @@ bool coschedule_enabled() {
   return !(v != nullptr && v[0] == '0');
 }
 
+// Whether expert GEMMs with 256-column tiles run as two-SM CTA pairs that share each B tile
+// (MOE_PAIR_MMA=0: one CTA per tile; both give the same bits). Read at every call.
 bool pair_mma_enabled() {
   const char* v = std::getenv("MOE_PAIR_MMA");
   return !(v != nullptr && v[0] == '0');
