@@ -225,8 +225,10 @@ __device__ __forceinline__ bool produce_tile(const Tile& tl, const CUtensorMap* 
                                              const CUtensorMap* tmX, const Params& p, int n_kb,
                                              uint32_t base_addr, uint32_t stage_stride,
                                              uint32_t a_bytes, const Bars& B, Ring& ring,
-                                             int& issued, volatile int* abort_flag) {
-  constexpr uint32_t kTx = FT * kBM * kBK * 2 + BN * kBK * 2;
+                                             int& issued, volatile int* abort_flag,
+                                             int x_rows = BN) {
+  // x_rows: the token box height of tmX (at least the tile's MMA N; rows past it are not read)
+  const uint32_t kTx = FT * kBM * kBK * 2 + (uint32_t)x_rows * kBK * 2;
   const int w_row = tl.e * p.n_out + tl.f0;
   const uint64_t w_policy = p.w_read_once ? l2_policy_evict_first() : 0ull;
   for (int kb = 0; kb < n_kb; ++kb) {
@@ -667,7 +669,8 @@ template <int BN0, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     co_gemm_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__ CUtensorMap tmX0,
                    const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmX1,
-                   const Params p0, const Params p1) {
+                   const __grid_constant__ CUtensorMap tmX0_32,
+                   const __grid_constant__ CUtensorMap tmX0_64, const Params p0, const Params p1) {
   static_assert(2 * BN0 <= kCoAccCols, "two expert accumulators per buffer");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -707,6 +710,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmX0);
     tma_prefetch_desc(&tmW1);
     tma_prefetch_desc(&tmX1);
+    if (BN0 > 32) tma_prefetch_desc(&tmX0_32);
+    if (BN0 > 64) tma_prefetch_desc(&tmX0_64);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_holder), 2 * kCoAccCols);
@@ -744,15 +749,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       int issued = 0;
       for (int t = blockIdx.x; t < total; t += gridDim.x) {
         int u;
-        const bool ok = which(t, u) == 0
-                            ? produce_tile<BN0, 2, false>(decode_tile<BN0, 2>(u, prefix, seg, p0.E, nft0),
-                                                          &tmW0, &tmX0, p0, nkb0, base_addr,
-                                                          kCoStageBytes, kA0, B, ring, issued,
-                                                          abort_flag)
-                            : produce_tile<kCoBN1, 1, false>(
+        bool ok;
+        if (which(t, u) == 0) {
+          // an expert tile loads only the token rows its MMAs read (the tile's rows rounded up to
+          // 16, then to a box of 32, 64 or BN0 rows): the stage fill that short segments leave
+          // for the weight stream, which is what bounds these tiles
+          const Tile tl = decode_tile<BN0, 2>(u, prefix, seg, p0.E, nft0);
+          const int n_mma = max(16, (tl.n_valid + 15) & ~15);
+          const bool r32 = BN0 > 32 && n_mma <= 32, r64 = !r32 && BN0 > 64 && n_mma <= 64;
+          ok = produce_tile<BN0, 2, false>(tl, &tmW0, r32 ? &tmX0_32 : (r64 ? &tmX0_64 : &tmX0), p0,
+                                           nkb0, base_addr, kCoStageBytes, kA0, B, ring, issued,
+                                           abort_flag, r32 ? 32 : (r64 ? 64 : BN0));
+        } else {
+          ok = produce_tile<kCoBN1, 1, false>(
                                   decode_dense_tile<kCoBN1, 1>(u, p1.rows_max, nft1, p1.K), &tmW1, &tmX1,
                                   p1, nkb1, base_addr, kCoStageBytes, kA1, B, ring, issued,
                                   abort_flag);
+        }
         if (!ok) break;
       }
       for (int i = max(0, issued - S); i < issued; ++i)
@@ -1127,14 +1140,15 @@ cudaError_t launch_one(const CUtensorMap& tmW, const CUtensorMap& tmX, const Par
 
 template <int BN0, int EPI>
 cudaError_t launch_co(const CUtensorMap& tmW0, const CUtensorMap& tmX0, const CUtensorMap& tmW1,
-                      const CUtensorMap& tmX1, const Params& p0, const Params& p1,
+                      const CUtensorMap& tmX1, const CUtensorMap& tmX0_32,
+                      const CUtensorMap& tmX0_64, const Params& p0, const Params& p1,
                       cudaStream_t stream) {
   auto kern = co_gemm_kernel<BN0, EPI>;
   static int attr_done[64] = {0};  // per instantiation and device
   cudaError_t e = ensure_dynamic_smem(kern, kCoSmemBytes, attr_done);
   if (e != cudaSuccess) return e;
   return launch_kernel(kern, dim3(num_sms()), dim3(kThreads), kCoSmemBytes, stream, tmW0, tmX0,
-                       tmW1, tmX1, p0, p1);
+                       tmW1, tmX1, tmX0_32, tmX0_64, p0, p1);
 }
 
 // Launch as clusters of two CTAs (co_pair_kernel), with programmatic dependent launch.
@@ -1334,8 +1348,13 @@ cudaError_t enqueue_co_gemm_bf16(const void* xp, const int32_t* offsets, int E, 
   // an empty expert problem still needs valid maps: point them at the dense operands (no tile
   // of problem 0 exists, so nothing is loaded through them)
   const bool no_rows = rows_max == 0;
+  CUtensorMap tmX0_32, tmX0_64;  // shorter token boxes for expert tiles of few rows
+  const void* x0 = no_rows ? x_dense : xp;
+  const int64_t rows0 = no_rows ? T : rows_max;
   if (!make_kmajor_map(&tmW0, w, (int64_t)E * N, K, kBM) ||
-      !make_kmajor_map(&tmX0, no_rows ? x_dense : xp, no_rows ? T : rows_max, K, BN0) ||
+      !make_kmajor_map(&tmX0, x0, rows0, K, BN0) ||
+      !make_kmajor_map(&tmX0_32, x0, rows0, K, BN0 < 32 ? BN0 : 32) ||
+      !make_kmajor_map(&tmX0_64, x0, rows0, K, BN0 < 64 ? BN0 : 64) ||
       !make_kmajor_map(&tmW1, w_dense, N, K, kBM) ||
       !make_kmajor_map(&tmX1, x_dense, T, K, kCoBN1))
     return cudaErrorInvalidValue;
@@ -1345,10 +1364,10 @@ cudaError_t enqueue_co_gemm_bf16(const void* xp, const int32_t* offsets, int E, 
   auto go = [&](auto tag) -> cudaError_t {
     constexpr int EPI = decltype(tag)::value;
     switch (BN0) {
-      case 16: return launch_co<16, EPI>(tmW0, tmX0, tmW1, tmX1, p0, p1, stream);
-      case 32: return launch_co<32, EPI>(tmW0, tmX0, tmW1, tmX1, p0, p1, stream);
-      case 64: return launch_co<64, EPI>(tmW0, tmX0, tmW1, tmX1, p0, p1, stream);
-      default: return launch_co<128, EPI>(tmW0, tmX0, tmW1, tmX1, p0, p1, stream);
+      case 16: return launch_co<16, EPI>(tmW0, tmX0, tmW1, tmX1, tmX0_32, tmX0_64, p0, p1, stream);
+      case 32: return launch_co<32, EPI>(tmW0, tmX0, tmW1, tmX1, tmX0_32, tmX0_64, p0, p1, stream);
+      case 64: return launch_co<64, EPI>(tmW0, tmX0, tmW1, tmX1, tmX0_32, tmX0_64, p0, p1, stream);
+      default: return launch_co<128, EPI>(tmW0, tmX0, tmW1, tmX1, tmX0_32, tmX0_64, p0, p1, stream);
     }
   };
   return gelu ? go(std::integral_constant<int, kEpiGeluBf16>{})
