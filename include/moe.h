@@ -65,7 +65,7 @@ typedef struct CUstream_st* moe_stream_t; /* the same handle as cudaStream_t */
 typedef enum {
   MOE_OK = 0,
   MOE_ERR_INVALID_ARGUMENT = 1,    /* NULL pointer, negative size, k > E, ... */
-  MOE_ERR_UNSUPPORTED = 2,         /* valid but outside what this build implements */
+  MOE_ERR_UNSUPPORTED = 2,         /* valid but outside what the library implements */
   MOE_ERR_WORKSPACE_TOO_SMALL = 3, /* ws_bytes below the *_workspace_bytes answer */
   MOE_ERR_CUDA = 4,                /* a CUDA runtime call failed (or fault injection) */
   MOE_ERR_DEVICE_FLAG = 5,         /* moe_get_device_error found a device-side error */
